@@ -1,0 +1,202 @@
+"""CPU oracle for additive-quantised matrix products (numpy-facing wrapper).
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline / reference arm of ``bench.py`` may import this package.  The
+CUDA library never imports, links or calls it, and it imports nothing from
+the CUDA library.
+
+The arithmetic lives in ``aq_oracle.c`` (plain C, fp64, no blocking); this
+module compiles it with gcc on first use and marshals numpy arrays.  What it
+computes, after "Extreme Compression of Large Language Models via Additive
+Quantization" (AQLM wiki entry, "Niveau intermédiaire"; devtrends.ru summary,
+"Как это работает технически?"):
+
+* ``decode``:  W[o][8g+j] = RN16(sum_k C_k[codes[o][g][k]][j]) (optionally
+  RN16(s[o] * W[o][i]));
+* ``matmul``:  y[o][b] = s[o] * sum_i W[o][i] * x[i][b] in fp64, plus the
+  per-element magnitude sum_i |s||W||x| used to scale the tolerance;
+* ``pack`` / ``unpack``: the library's documented packed code layout;
+* ``bits_per_weight`` and ``layer_bytes``: the bit-rate closed form and the
+  storage it implies.
+
+Binary16 values cross this interface as ``np.uint16`` bit patterns or
+``np.float16`` arrays (viewed as uint16).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "aq_oracle.c")
+_BUILD = os.path.join(_HERE, "_build")
+_LIB_PATH = os.path.join(_BUILD, "libaqoracle.so")
+_lock = threading.Lock()
+_lib = None
+
+_c_i64 = ctypes.c_int64
+_c_int = ctypes.c_int
+_vp = ctypes.c_void_p
+
+
+def build(force: bool = False) -> str:
+    """Compile ``aq_oracle.c`` into ``_build/libaqoracle.so`` (gcc, fp64,
+    no fast-math, no FMA contraction)."""
+    os.makedirs(_BUILD, exist_ok=True)
+    stale = (not os.path.exists(_LIB_PATH)
+             or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC))
+    if force or stale:
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fopenmp",
+               "-fPIC", "-shared", "-o", tmp, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            lib.aqo_half_to_double.argtypes = [ctypes.c_uint16]
+            lib.aqo_half_to_double.restype = ctypes.c_double
+            lib.aqo_double_to_half.argtypes = [ctypes.c_double]
+            lib.aqo_double_to_half.restype = ctypes.c_uint16
+            lib.aqo_bits_per_weight.argtypes = [_c_int, _c_int, _c_int]
+            lib.aqo_bits_per_weight.restype = ctypes.c_double
+            lib.aqo_layer_bytes.argtypes = [_c_i64, _c_i64, _c_int, _c_int]
+            lib.aqo_layer_bytes.restype = ctypes.c_double
+            lib.aqo_decode.argtypes = [_c_i64, _c_i64, _c_int, _c_int, _vp, _vp, _vp, _vp]
+            lib.aqo_decode.restype = _c_int
+            lib.aqo_matmul.argtypes = [_c_i64, _c_i64, _c_int, _c_int, _vp, _vp, _vp,
+                                       _vp, _c_i64, _vp, _c_i64, _vp, _vp, _c_int]
+            lib.aqo_matmul.restype = _c_int
+            lib.aqo_packed_bytes.argtypes = [_c_i64, _c_i64, _c_int, _c_int]
+            lib.aqo_packed_bytes.restype = _c_i64
+            lib.aqo_pack.argtypes = [_c_i64, _c_i64, _c_int, _c_int, _vp, _vp]
+            lib.aqo_pack.restype = _c_int
+            lib.aqo_unpack.argtypes = [_c_i64, _c_i64, _c_int, _c_int, _vp, _vp]
+            lib.aqo_unpack.restype = _c_int
+            lib.aqo_max_threads.argtypes = []
+            lib.aqo_max_threads.restype = _c_int
+            _lib = lib
+    return _lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data
+
+
+def _bits(a) -> np.ndarray:
+    """binary16 array (float16 or uint16) -> contiguous uint16 bit patterns."""
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.float16:
+        return a.view(np.uint16)
+    if a.dtype != np.uint16:
+        raise TypeError(f"expected float16/uint16, got {a.dtype}")
+    return a
+
+
+def _codes(codes, K, B) -> np.ndarray:
+    want = np.uint8 if B <= 8 else np.uint16
+    codes = np.ascontiguousarray(codes)
+    if codes.dtype != want:
+        raise TypeError(f"codes must be {np.dtype(want).name} for B={B}")
+    if codes.ndim != 3 or codes.shape[2] != K:
+        raise ValueError("codes must be [out][in/8][K]")
+    return codes
+
+
+# -- scalar helpers ---------------------------------------------------------
+
+def half_to_double(h: int) -> float:
+    return _load().aqo_half_to_double(int(h) & 0xFFFF)
+
+
+def double_to_half(v: float) -> int:
+    return int(_load().aqo_double_to_half(float(v)))
+
+
+def bits_per_weight(K: int, B: int, g: int = 8) -> float:
+    return _load().aqo_bits_per_weight(K, B, g)
+
+
+def layer_bytes(out: int, inp: int, K: int, B: int) -> float:
+    return _load().aqo_layer_bytes(out, inp, K, B)
+
+
+def max_threads() -> int:
+    return _load().aqo_max_threads()
+
+
+# -- array functions --------------------------------------------------------
+
+def decode(codes, codebooks, scales=None) -> np.ndarray:
+    """Dequantised W ``[out][in]`` as float16 (exact sum, one RN-even)."""
+    cb = _bits(codebooks)
+    K, ncw, g = cb.shape
+    B = int(ncw).bit_length() - 1
+    if g != 8 or (1 << B) != ncw:
+        raise ValueError("codebooks must be [K][2**B][8]")
+    codes = _codes(codes, K, B)
+    out, G, _ = codes.shape
+    s = None if scales is None else _bits(scales)
+    w = np.empty((out, G * 8), dtype=np.uint16)
+    rc = _load().aqo_decode(out, G * 8, K, B, _ptr(codes), _ptr(cb), _ptr(s), _ptr(w))
+    if rc:
+        raise RuntimeError(f"aqo_decode failed ({rc})")
+    return w.view(np.float16)
+
+
+def matmul(codes, codebooks, scales, x, rows=None, threads: int = 1):
+    """``(y, bound)`` in float64; y = diag(s) W x for all rows or ``rows``."""
+    cb = _bits(codebooks)
+    K, ncw, _ = cb.shape
+    B = int(ncw).bit_length() - 1
+    codes = _codes(codes, K, B)
+    out, G, _ = codes.shape
+    xb = _bits(x)
+    if xb.ndim != 2 or xb.shape[0] != G * 8:
+        raise ValueError("x must be [in][n]")
+    n = xb.shape[1]
+    s = None if scales is None else _bits(scales)
+    r = None if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    nrows = out if r is None else len(r)
+    y = np.empty((nrows, n), dtype=np.float64)
+    bound = np.empty((nrows, n), dtype=np.float64)
+    rc = _load().aqo_matmul(out, G * 8, K, B, _ptr(codes), _ptr(cb), _ptr(s), _ptr(xb),
+                            n, _ptr(r), nrows, _ptr(y), _ptr(bound), int(threads))
+    if rc:
+        raise RuntimeError(f"aqo_matmul failed ({rc})")
+    return y, bound
+
+
+def packed_bytes(out: int, inp: int, K: int, B: int) -> int:
+    n = _load().aqo_packed_bytes(out, inp, K, B)
+    if n < 0:
+        raise ValueError("unsupported layer for the packed layout")
+    return int(n)
+
+
+def pack(codes, K: int, B: int) -> np.ndarray:
+    codes = _codes(codes, K, B)
+    out, G, _ = codes.shape
+    buf = np.empty(packed_bytes(out, G * 8, K, B), dtype=np.uint8)
+    if _load().aqo_pack(out, G * 8, K, B, _ptr(codes), _ptr(buf)):
+        raise RuntimeError("aqo_pack failed")
+    return buf
+
+
+def unpack(packed, out: int, inp: int, K: int, B: int) -> np.ndarray:
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    if packed.size != packed_bytes(out, inp, K, B):
+        raise ValueError("packed buffer has the wrong size")
+    codes = np.empty((out, inp // 8, K), dtype=np.uint8 if B <= 8 else np.uint16)
+    if _load().aqo_unpack(out, inp, K, B, _ptr(packed), _ptr(codes)):
+        raise RuntimeError("aqo_unpack failed")
+    return codes

@@ -1,0 +1,314 @@
+/*
+ * CPU oracle for additive-quantised matrix products.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may include, link or
+ * call this file: only tests/, __graft_entry__.smoke() and the CPU-baseline /
+ * reference arm of bench.py use it.  It shares no code, header, table or
+ * constant with the CUDA library; it is written from the method's definition
+ * and is deliberately plain and slow (no blocking, no reordering).
+ *
+ * Sources (web pages on "Extreme Compression of Large Language Models via
+ * Additive Quantization", Egiazarian et al., ICML 2024):
+ *   - AQLM wiki entry (brain.gartu.xyz), section "Niveau intermédiaire":
+ *     each group of weights is approximated by the sum of one vector from each
+ *     of K codebooks, w ~ C_1[i_1] + ... + C_K[i_K]; bit rate per weight is
+ *     K * log2(codebook size) / group size.
+ *   - devtrends.ru summary ("AQLM — Сжимаем языковые модели без потерь"), section "Как это работает технически?":
+ *     groups are 8 consecutive weights (in_group_size = 8).
+ *   - arXiv 2401.06118 abstract: the GPU/CPU kernels compute the product of
+ *     the quantised matrix with activations for token generation.
+ * The per-row scale s and the packed code layout are this library's interface
+ * (the pages mention neither); the oracle follows their written definitions:
+ *   y[o][b] = s[o] * sum_i W[o][i] * x[i][b],
+ *   W[o][8g+j] = RN16( sum_k C_k[codes[o][g][k]][j] ).
+ *
+ * Readings of points the pages leave open:
+ *   - the sum over k is formed exactly (fp64 holds any sum of <= 8 binary16
+ *     values exactly) and rounded once to binary16, ties to even;
+ *   - the product with x and the scale are taken in fp64 from the binary16
+ *     values, no intermediate rounding;
+ *   - codes are unsigned, code k selects a row of codebook k.
+ *
+ * Pins (tests/test_oracle_pins.py): conversions against numpy's binary16,
+ * exhaustive single-group decode, one-hot codebooks, additivity, permutation
+ * invariance, integer-exact products, pure-Python brute force on tiny inputs,
+ * the pages' bit-rate examples and model sizes, pack round trip and
+ * hand-worked layout offsets.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define AQO_GROUP 8
+
+/* ------------------------------------------------------------------------ */
+/* IEEE 754 binary16, written from the format definition:                   */
+/* 1 sign bit, 5 exponent bits (bias 15), 10 fraction bits.                 */
+/* ------------------------------------------------------------------------ */
+
+double aqo_half_to_double(uint16_t h)
+{
+    int sign = (h >> 15) & 1;
+    int e = (h >> 10) & 0x1f;
+    int f = h & 0x3ff;
+    double v;
+    if (e == 0) {
+        v = ldexp((double)f, -24); /* zero or subnormal: f * 2^-24 */
+    } else if (e == 31) {
+        v = f ? NAN : INFINITY;
+    } else {
+        v = ldexp((double)(1024 + f), e - 25); /* 1.f * 2^(e-15) */
+    }
+    return sign ? -v : v;
+}
+
+/* q >= 0 holds an exact value; return it rounded to an integer, ties to even. */
+static double round_half_even(double q)
+{
+    double fl = floor(q);
+    double d = q - fl; /* exact: q and fl share the exponent range */
+    if (d > 0.5) return fl + 1.0;
+    if (d < 0.5) return fl;
+    return (fmod(fl, 2.0) == 0.0) ? fl : fl + 1.0;
+}
+
+uint16_t aqo_double_to_half(double v)
+{
+    uint16_t sign = signbit(v) ? 0x8000 : 0;
+    double a = fabs(v);
+    if (isnan(v)) return (uint16_t)(sign | 0x7e00);
+    /* 65504 is the largest finite value; the midpoint to 2^16 is 65520,
+     * which rounds to even (upwards, to infinity). */
+    if (a >= 65520.0) return (uint16_t)(sign | 0x7c00);
+    if (a < ldexp(1.0, -14)) {
+        /* subnormal range: value = m * 2^-24, m in [0, 1024]; m == 1024 is
+         * the smallest normal number and encodes correctly as 0x0400. */
+        double m = round_half_even(ldexp(a, 24));
+        return (uint16_t)(sign | (uint16_t)m);
+    }
+    int ex;
+    frexp(a, &ex); /* a = f * 2^ex, f in [0.5, 1) -> a in [2^(ex-1), 2^ex) */
+    int e = ex - 1;                             /* unbiased exponent */
+    double m = round_half_even(ldexp(a, 10 - e)); /* in [1024, 2048] */
+    if (m == 2048.0) {
+        m = 1024.0;
+        e += 1;
+    }
+    if (e + 15 >= 31) return (uint16_t)(sign | 0x7c00);
+    return (uint16_t)(sign | (uint16_t)((e + 15) << 10) | (uint16_t)(m - 1024.0));
+}
+
+/* ------------------------------------------------------------------------ */
+/* Bit rate and storage (wiki entry, "Niveau intermédiaire").               */
+/* ------------------------------------------------------------------------ */
+
+/* bits per weight = K * log2(codebook size) / group size; codebook size 2^B */
+double aqo_bits_per_weight(int K, int B, int g)
+{
+    return (double)K * (double)B / (double)g;
+}
+
+/* Bytes one quantised layer occupies: codes at K*B bits per group of 8,
+ * K codebooks of 2^B binary16 8-vectors, one binary16 scale per row. */
+double aqo_layer_bytes(int64_t out, int64_t in, int K, int B)
+{
+    double code_bits = (double)out * (double)(in / AQO_GROUP) * K * B;
+    double codebook_bytes = (double)K * ldexp(1.0, B) * AQO_GROUP * 2.0;
+    return code_bits / 8.0 + codebook_bytes + 2.0 * (double)out;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Decode (additive reconstruction of one group).                           */
+/* ------------------------------------------------------------------------ */
+
+static uint32_t code_at(const void *codes, int B, int64_t idx)
+{
+    if (B <= 8) return ((const uint8_t *)codes)[idx];
+    return ((const uint16_t *)codes)[idx];
+}
+
+static int check_scheme(int64_t out, int64_t in, int K, int B)
+{
+    if (out < 0 || in < 0 || in % AQO_GROUP) return -1;
+    if (K < 1 || K > 8 || B < 1 || B > 16) return -1;
+    return 0;
+}
+
+/* Row o of W as doubles (each value already rounded to binary16). */
+static void decode_row(int64_t o, int64_t in, int K, int B, const void *codes,
+                       const uint16_t *codebooks, double *row)
+{
+    int64_t G = in / AQO_GROUP;
+    int64_t ncw = (int64_t)1 << B;
+    for (int64_t g = 0; g < G; ++g) {
+        for (int j = 0; j < AQO_GROUP; ++j) {
+            /* The sum starts from the first term (not from +0), so a lone
+             * -0 codeword entry stays -0; it is exact: <= 8 binary16 terms. */
+            double sum = 0.0;
+            for (int k = 0; k < K; ++k) {
+                uint32_t c = code_at(codes, B, (o * G + g) * K + k);
+                double term = aqo_half_to_double(codebooks[((int64_t)k * ncw + c) * AQO_GROUP + j]);
+                sum = (k == 0) ? term : sum + term;
+            }
+            row[g * AQO_GROUP + j] = aqo_half_to_double(aqo_double_to_half(sum));
+        }
+    }
+}
+
+/* W[o][i] as binary16 bits; with scales != NULL, RN16(s[o] * W[o][i]). */
+int aqo_decode(int64_t out, int64_t in, int K, int B, const void *codes,
+               const uint16_t *codebooks, const uint16_t *scales, uint16_t *w)
+{
+    if (check_scheme(out, in, K, B)) return -1;
+    double *row = (double *)malloc(sizeof(double) * (size_t)(in > 0 ? in : 1));
+    if (!row) return -2;
+    for (int64_t o = 0; o < out; ++o) {
+        decode_row(o, in, K, B, codes, codebooks, row);
+        double s = scales ? aqo_half_to_double(scales[o]) : 1.0;
+        for (int64_t i = 0; i < in; ++i)
+            w[o * in + i] = scales ? aqo_double_to_half(s * row[i])
+                                   : aqo_double_to_half(row[i]);
+    }
+    free(row);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Product y = diag(s) * W * x in fp64 (x is [in][n]).                      */
+/* rows == NULL: all rows, y is [out][n]; else y is [nrows][n] for the      */
+/* listed rows.  bound (optional) receives sum_i |s||W||x| per element, the */
+/* scale of the tolerance the GPU results are checked against.             */
+/* ------------------------------------------------------------------------ */
+
+int aqo_matmul(int64_t out, int64_t in, int K, int B, const void *codes,
+               const uint16_t *codebooks, const uint16_t *scales,
+               const uint16_t *x, int64_t n, const int64_t *rows, int64_t nrows,
+               double *y, double *bound, int threads)
+{
+    if (check_scheme(out, in, K, B) || n < 0) return -1;
+    if (!rows) nrows = out;
+    for (int64_t r = 0; rows && r < nrows; ++r)
+        if (rows[r] < 0 || rows[r] >= out) return -1;
+    double *xd = (double *)malloc(sizeof(double) * (size_t)(in * n > 0 ? in * n : 1));
+    if (!xd) return -2;
+    for (int64_t t = 0; t < in * n; ++t) xd[t] = aqo_half_to_double(x[t]);
+    int err = 0;
+#ifdef _OPENMP
+    if (threads < 1) threads = 1;
+#pragma omp parallel num_threads(threads)
+#endif
+    {
+        double *row = (double *)malloc(sizeof(double) * (size_t)(in > 0 ? in : 1));
+        if (!row) {
+            err = -2;
+        } else {
+#ifdef _OPENMP
+#pragma omp for schedule(dynamic, 8)
+#endif
+            for (int64_t r = 0; r < nrows; ++r) {
+                int64_t o = rows ? rows[r] : r;
+                decode_row(o, in, K, B, codes, codebooks, row);
+                double s = scales ? aqo_half_to_double(scales[o]) : 1.0;
+                for (int64_t b = 0; b < n; ++b) {
+                    double acc = 0.0, mag = 0.0;
+                    for (int64_t i = 0; i < in; ++i) {
+                        acc += row[i] * xd[i * n + b];
+                        mag += fabs(row[i] * xd[i * n + b]);
+                    }
+                    y[r * n + b] = s * acc;
+                    if (bound) bound[r * n + b] = fabs(s) * mag;
+                }
+            }
+            free(row);
+        }
+    }
+    free(xd);
+    return err;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Packed code layout (the library's documented interface).                 */
+/*                                                                          */
+/* Each group (o, g) has one 16-bit word: for one 16-bit codebook the code  */
+/* itself, for two 8-bit codebooks code[k=0] | code[k=1] << 8.  Rows are    */
+/* padded to a multiple of 8 and groups to a multiple of 32 with zero words.*/
+/* Word (o, g) is stored little-endian at byte                              */
+/*   ((o / 8) * (Gp / 32) + g / 32) * 512 + (g % 32) * 16 + (o % 8) * 2     */
+/* where Gp is the padded group count: a 512-byte tile holds 8 rows x 32    */
+/* groups, each 16-byte chunk holds one group for 8 consecutive rows.       */
+/* ------------------------------------------------------------------------ */
+
+static int packed_scheme_ok(int K, int B)
+{
+    return (K == 1 && B == 16) || (K == 2 && B == 8);
+}
+
+int64_t aqo_packed_bytes(int64_t out, int64_t in, int K, int B)
+{
+    if (check_scheme(out, in, K, B) || !packed_scheme_ok(K, B)) return -1;
+    int64_t rows = (out + 7) / 8 * 8;
+    int64_t gp = (in / AQO_GROUP + 31) / 32 * 32;
+    return rows * gp * 2;
+}
+
+static int64_t packed_offset(int64_t o, int64_t g, int64_t gp)
+{
+    return ((o / 8) * (gp / 32) + g / 32) * 512 + (g % 32) * 16 + (o % 8) * 2;
+}
+
+int aqo_pack(int64_t out, int64_t in, int K, int B, const void *codes, uint8_t *packed)
+{
+    int64_t nbytes = aqo_packed_bytes(out, in, K, B);
+    if (nbytes < 0) return -1;
+    int64_t G = in / AQO_GROUP;
+    int64_t gp = (G + 31) / 32 * 32;
+    memset(packed, 0, (size_t)nbytes);
+    for (int64_t o = 0; o < out; ++o) {
+        for (int64_t g = 0; g < G; ++g) {
+            uint32_t word;
+            if (K == 1) {
+                word = code_at(codes, B, o * G + g);
+            } else {
+                word = code_at(codes, B, (o * G + g) * 2 + 0) |
+                       (code_at(codes, B, (o * G + g) * 2 + 1) << 8);
+            }
+            int64_t at = packed_offset(o, g, gp);
+            packed[at] = (uint8_t)(word & 0xff);
+            packed[at + 1] = (uint8_t)(word >> 8);
+        }
+    }
+    return 0;
+}
+
+int aqo_unpack(int64_t out, int64_t in, int K, int B, const uint8_t *packed, void *codes)
+{
+    if (aqo_packed_bytes(out, in, K, B) < 0) return -1;
+    int64_t G = in / AQO_GROUP;
+    int64_t gp = (G + 31) / 32 * 32;
+    for (int64_t o = 0; o < out; ++o) {
+        for (int64_t g = 0; g < G; ++g) {
+            int64_t at = packed_offset(o, g, gp);
+            uint32_t word = (uint32_t)packed[at] | ((uint32_t)packed[at + 1] << 8);
+            if (K == 1) {
+                ((uint16_t *)codes)[o * G + g] = (uint16_t)word;
+            } else {
+                ((uint8_t *)codes)[(o * G + g) * 2 + 0] = (uint8_t)(word & 0xff);
+                ((uint8_t *)codes)[(o * G + g) * 2 + 1] = (uint8_t)(word >> 8);
+            }
+        }
+    }
+    return 0;
+}
+
+int aqo_max_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
