@@ -1,0 +1,169 @@
+// C ABI of libaq_b200.so: argument validation and dispatch (see include/aq.h).
+//
+// Every entry point validates its arguments on the host before touching the
+// GPU; on error nothing is launched.  No exception crosses the interface.
+#include <stdint.h>
+
+#include "aq_common.cuh"
+
+namespace {
+
+using aqk::Geom;
+
+constexpr int kVersion = 10000;  // 1.0.0
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Descriptor checks shared by all entry points.
+aq_status check_desc(const aq_layer_desc *d)
+{
+    if (!d) return AQ_ERR_INVALID_ARG;
+    if (d->out_features < 1 || d->in_features < 8 || d->in_features % 8) return AQ_ERR_INVALID_ARG;
+    if (d->group_size != 8) return AQ_ERR_UNSUPPORTED;
+    const bool ok = (d->num_codebooks == 1 && d->nbits == 16) || (d->num_codebooks == 2 && d->nbits == 8);
+    if (!ok) return AQ_ERR_UNSUPPORTED;
+    // keep every byte offset and element count within 64-bit range and the
+    // per-row chunk count within 32-bit kernel indices
+    if ((int64_t)d->out_features * d->in_features > (int64_t)1 << 40) return AQ_ERR_INVALID_ARG;
+    // grid.y of the split-K launches is bounded by 65535 group blocks
+    if (d->in_features > (1 << 24) || d->out_features > (1 << 28)) return AQ_ERR_INVALID_ARG;
+    return AQ_OK;
+}
+
+aq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? AQ_OK : AQ_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+const char *aq_status_string(aq_status status)
+{
+    switch (status) {
+    case AQ_OK: return "success";
+    case AQ_ERR_INVALID_ARG: return "invalid argument";
+    case AQ_ERR_UNSUPPORTED: return "unsupported layer (scheme or group size)";
+    case AQ_ERR_MISALIGNED: return "array pointer not 16-byte aligned";
+    case AQ_ERR_WORKSPACE: return "workspace missing or too small";
+    case AQ_ERR_CUDA: return "CUDA runtime error";
+    case AQ_ERR_TIMEOUT: return "a bounded device-side wait gave up";
+    }
+    return "unknown status";
+}
+
+int aq_version(void) { return kVersion; }
+
+size_t aq_packed_codes_bytes(const aq_layer_desc *desc)
+{
+    if (check_desc(desc) != AQ_OK) return 0;
+    const Geom g = aqk::make_geom(*desc);
+    return (size_t)g.rows8 * g.gp * 2;
+}
+
+size_t aq_gemv_workspace_bytes(const aq_layer_desc *desc, int batch)
+{
+    if (check_desc(desc) != AQ_OK || batch < 1 || batch > 16) return 0;
+    return aqh::gemv_workspace_bytes(aqk::make_geom(*desc), batch);
+}
+
+size_t aq_gemm_workspace_bytes(const aq_layer_desc *desc, int T)
+{
+    if (check_desc(desc) != AQ_OK || T < 1) return 0;
+    return aqh::gemm_workspace_bytes(aqk::make_geom(*desc), T);
+}
+
+aq_status aq_workspace_status(void *workspace, aq_stream_t stream)
+{
+    if (!workspace) return AQ_ERR_INVALID_ARG;
+    if (!aligned16(workspace)) return AQ_ERR_MISALIGNED;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint32_t word = 0;
+    cudaError_t e = cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return AQ_ERR_CUDA;
+    if (word == 0) return AQ_OK;
+    e = cudaMemsetAsync(workspace, 0, sizeof(word), s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return AQ_ERR_CUDA;
+    return word == AQ_ERR_TIMEOUT ? AQ_ERR_TIMEOUT : AQ_ERR_CUDA;
+}
+
+aq_status aq_selftest_bounded_wait(void *workspace, int spin_limit, aq_stream_t stream)
+{
+    if (!workspace || spin_limit < 1 || spin_limit > (1 << 20)) return AQ_ERR_INVALID_ARG;
+    if (!aligned16(workspace)) return AQ_ERR_MISALIGNED;
+    return from_cuda(aqh::launch_selftest_wait(workspace, spin_limit, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+aq_status aq_pack_codes(const aq_layer_desc *desc, const void *codes, void *packed, aq_stream_t stream)
+{
+    aq_status st = check_desc(desc);
+    if (st != AQ_OK) return st;
+    if (!codes || !packed) return AQ_ERR_INVALID_ARG;
+    if (!aligned16(packed)) return AQ_ERR_MISALIGNED;
+    if (desc->nbits == 16 && (reinterpret_cast<uintptr_t>(codes) & 1u)) return AQ_ERR_MISALIGNED;
+    return from_cuda(aqh::launch_pack(aqk::make_geom(*desc), codes, packed,
+                                      reinterpret_cast<cudaStream_t>(stream)));
+}
+
+aq_status aq_unpack_codes(const aq_layer_desc *desc, const void *packed, void *codes, aq_stream_t stream)
+{
+    aq_status st = check_desc(desc);
+    if (st != AQ_OK) return st;
+    if (!codes || !packed) return AQ_ERR_INVALID_ARG;
+    if (!aligned16(packed)) return AQ_ERR_MISALIGNED;
+    if (desc->nbits == 16 && (reinterpret_cast<uintptr_t>(codes) & 1u)) return AQ_ERR_MISALIGNED;
+    return from_cuda(aqh::launch_unpack(aqk::make_geom(*desc), packed, codes,
+                                        reinterpret_cast<cudaStream_t>(stream)));
+}
+
+aq_status aq_dequant(const aq_layer_desc *desc, const void *packed, const uint16_t *codebooks,
+                     const uint16_t *scales, uint16_t *w, aq_stream_t stream)
+{
+    aq_status st = check_desc(desc);
+    if (st != AQ_OK) return st;
+    if (!packed || !codebooks || !w) return AQ_ERR_INVALID_ARG;
+    if (!aligned16(packed) || !aligned16(codebooks) || !aligned16(w)) return AQ_ERR_MISALIGNED;
+    if (scales && (reinterpret_cast<uintptr_t>(scales) & 1u)) return AQ_ERR_MISALIGNED;
+    return from_cuda(aqh::launch_dequant(aqk::make_geom(*desc), packed, codebooks, scales, w,
+                                         reinterpret_cast<cudaStream_t>(stream)));
+}
+
+aq_status aq_gemv(const aq_layer_desc *desc, const void *packed, const uint16_t *codebooks,
+                  const uint16_t *scales, const uint16_t *x, int batch, uint16_t *y,
+                  void *workspace, size_t workspace_bytes, aq_stream_t stream)
+{
+    aq_status st = check_desc(desc);
+    if (st != AQ_OK) return st;
+    if (batch < 1 || batch > 16) return AQ_ERR_INVALID_ARG;
+    if (!packed || !codebooks || !x || !y) return AQ_ERR_INVALID_ARG;
+    if (!aligned16(packed) || !aligned16(codebooks) || !aligned16(x) || !aligned16(y))
+        return AQ_ERR_MISALIGNED;
+    if (scales && (reinterpret_cast<uintptr_t>(scales) & 1u)) return AQ_ERR_MISALIGNED;
+    const Geom g = aqk::make_geom(*desc);
+    const size_t need = aqh::gemv_workspace_bytes(g, batch);
+    if (!workspace || workspace_bytes < need) return AQ_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return AQ_ERR_MISALIGNED;
+    return from_cuda(aqh::launch_gemv(g, packed, codebooks, scales, x, batch, y, workspace,
+                                      reinterpret_cast<cudaStream_t>(stream)));
+}
+
+aq_status aq_gemm(const aq_layer_desc *desc, const void *packed, const uint16_t *codebooks,
+                  const uint16_t *scales, const uint16_t *x, int T, uint16_t *y,
+                  void *workspace, size_t workspace_bytes, aq_stream_t stream)
+{
+    aq_status st = check_desc(desc);
+    if (st != AQ_OK) return st;
+    if (T < 1 || T > (1 << 22)) return AQ_ERR_INVALID_ARG;  // grid.y = T/128 <= 32768
+    if (!packed || !codebooks || !x || !y) return AQ_ERR_INVALID_ARG;
+    if (!aligned16(packed) || !aligned16(codebooks) || !aligned16(x) || !aligned16(y))
+        return AQ_ERR_MISALIGNED;
+    if (scales && (reinterpret_cast<uintptr_t>(scales) & 1u)) return AQ_ERR_MISALIGNED;
+    const Geom g = aqk::make_geom(*desc);
+    const size_t need = aqh::gemm_workspace_bytes(g, T);
+    if (!workspace || workspace_bytes < need) return AQ_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return AQ_ERR_MISALIGNED;
+    return from_cuda(aqh::launch_gemm(g, packed, codebooks, scales, x, T, y, workspace,
+                                      reinterpret_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,188 @@
+/*
+ * aq.h -- C ABI of the B200 (sm_100a) additive-quantised matrix product
+ * library (libaq_b200.so).
+ *
+ * What it computes.  The additive quantisation of "Extreme Compression of
+ * Large Language Models via Additive Quantization" (Egiazarian et al., ICML
+ * 2024) stores each group of 8 consecutive input weights of one output row
+ * as K codes; the group is rebuilt as the sum of one 8-vector from each of K
+ * codebooks (AQLM wiki entry, brain.gartu.xyz, section "Niveau
+ * intermédiaire": w ~ C_1[i_1] + ... + C_K[i_K]; devtrends.ru summary
+ * "AQLM — Сжимаем языковые модели без потерь", section "Как это работает
+ * технически?": groups of 8, in_group_size).  With K codebooks of 2^B
+ * entries the bit rate is K*B/8 bits per weight ("Niveau intermédiaire",
+ * bit-rate formula).  The library multiplies the decoded matrix by
+ * activations, the operation the paper's abstract (arXiv 2401.06118) names
+ * for token generation, with one scale per output row:
+ *
+ *     W[o][8g+j] = RN16( sum_k C_k[codes[o][g][k]][j] )          (decode)
+ *     y[o][b]    = RN16( s[o] * sum_i W[o][i] * x[i][b] )        (product)
+ *
+ * Supported schemes (devtrends.ru, section "Схемы квантования"): "1x16"
+ * (K = 1, B = 16) and "2x8" (K = 2, B = 8); both are 2 bits per weight.
+ *
+ * Conventions shared by every entry point:
+ *  - binary16 values are passed as uint16_t bit patterns (IEEE 754 half);
+ *  - every array pointer is a DEVICE pointer on the current CUDA device,
+ *    owned by the caller; the library allocates no memory and keeps no
+ *    state between calls (thread-safe; calls on one stream are ordered);
+ *  - work is enqueued on `stream` (NULL = legacy default stream) and the
+ *    call returns after the launch; the caller synchronises;
+ *  - all arguments are validated on the host before anything is launched;
+ *    on any error status nothing is launched and no output byte is written;
+ *  - array pointers must be 16-byte aligned (AQ_ERR_MISALIGNED otherwise);
+ *  - no C++ exception crosses this interface.
+ *
+ * Packed code layout (produced by aq_pack_codes, consumed by every kernel).
+ * Each group (o, g) owns one 16-bit word: for 1x16 the code itself, for 2x8
+ * codes[o][g][0] | codes[o][g][1] << 8.  Rows are padded to a multiple of 8
+ * and groups to a multiple of 32 (Gp = padded group count); padding words
+ * are zero.  Word (o, g) is stored little-endian at byte
+ *
+ *     ((o / 8) * (Gp / 32) + g / 32) * 512  +  (g % 32) * 16  +  (o % 8) * 2
+ *
+ * i.e. 512-byte tiles of 8 rows x 32 groups, tile-rows in row order; inside
+ * a tile the 16-byte chunk c holds group 32*(g/32)+c for the tile's 8 rows,
+ * so one warp-wide 128-bit load fetches a whole tile.
+ */
+#ifndef AQ_B200_H
+#define AQ_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t (a pointer to the runtime's opaque stream). */
+struct CUstream_st;
+typedef struct CUstream_st *aq_stream_t;
+
+typedef enum {
+    AQ_OK = 0,
+    AQ_ERR_INVALID_ARG = 1, /* null pointer, bad size, in % 8 != 0, ...     */
+    AQ_ERR_UNSUPPORTED = 2, /* (K, B) or group size this build cannot run  */
+    AQ_ERR_MISALIGNED = 3,  /* an array pointer not 16-byte aligned         */
+    AQ_ERR_WORKSPACE = 4,   /* workspace missing or smaller than required   */
+    AQ_ERR_CUDA = 5,        /* the CUDA runtime reported an error           */
+    AQ_ERR_TIMEOUT = 6      /* a bounded device-side wait gave up           */
+} aq_status;
+
+/* One quantised linear layer: y[out] = diag(s) W[out][in] x[in]. */
+typedef struct {
+    int32_t out_features;  /* rows of W, 1 .. 2^28                         */
+    int32_t in_features;   /* columns of W, 8 .. 2^24, multiple of 8       */
+    int32_t group_size;    /* weights per code group; must be 8            */
+    int32_t num_codebooks; /* K: 1 (with nbits 16) or 2 (with nbits 8)     */
+    int32_t nbits;         /* B: bits per code, codebook has 2^B entries   */
+} aq_layer_desc;
+
+/* Static, NUL-terminated description of a status; never NULL. */
+const char *aq_status_string(aq_status status);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int aq_version(void);
+
+/*
+ * Bytes of the packed code buffer for `desc` (layout above): padded rows x
+ * padded groups x 2.  Returns 0 for an invalid or unsupported descriptor.
+ * Host-only; needs no GPU.
+ */
+size_t aq_packed_codes_bytes(const aq_layer_desc *desc);
+
+/*
+ * Workspace.  aq_gemv and aq_gemm take a caller-owned device workspace.  Its
+ * first 16 bytes hold a status word that a kernel sets when a bounded wait
+ * gives up (read it with aq_workspace_status); the rest holds split-K
+ * partial sums and arrival counters.  A workspace must be zero-filled once
+ * before its first use; every completed call leaves it ready for the next
+ * (counters back at zero).  Calls that may overlap in time (different
+ * streams) must not share a workspace.
+ *
+ * The sizes below are host-only (no GPU needed) and depend on the
+ * descriptor and batch / token count alone.  They return 0 for invalid
+ * arguments, never less than 16 otherwise.
+ */
+size_t aq_gemv_workspace_bytes(const aq_layer_desc *desc, int batch);
+size_t aq_gemm_workspace_bytes(const aq_layer_desc *desc, int T);
+
+/*
+ * Read and clear the status word of `workspace` after all work queued on
+ * `stream` has finished (this call synchronises `stream`).  Returns AQ_OK,
+ * AQ_ERR_TIMEOUT if a kernel's bounded wait gave up since the last read, or
+ * AQ_ERR_CUDA.
+ */
+aq_status aq_workspace_status(void *workspace, aq_stream_t stream);
+
+/*
+ * Test aid for failure detection: launches one CTA that waits on a barrier
+ * nothing will ever complete, gives up after `spin_limit` polls, records
+ * AQ_ERR_TIMEOUT in the workspace status word and returns.  The context
+ * stays usable.  spin_limit in 1..1<<20.
+ */
+aq_status aq_selftest_bounded_wait(void *workspace, int spin_limit, aq_stream_t stream);
+
+/*
+ * Interleave codes into the packed layout (offline, once per layer).
+ *   codes  [out][in/8][K]: uint8 for 2x8, uint16 for 1x16 (row-major).
+ *   packed aq_packed_codes_bytes(desc) bytes; every byte is written,
+ *          padding included.
+ * `codes` needs only the alignment of its element type; `packed` 16 bytes.
+ */
+aq_status aq_pack_codes(const aq_layer_desc *desc, const void *codes, void *packed,
+                        aq_stream_t stream);
+
+/* Inverse of aq_pack_codes (a test aid): packed -> codes[out][in/8][K]. */
+aq_status aq_unpack_codes(const aq_layer_desc *desc, const void *packed, void *codes,
+                          aq_stream_t stream);
+
+/*
+ * Dequantise: w[o][i] = RN16(sum_k C_k[codes[o][g][k]][i - 8g]) with
+ * g = i / 8, or, when `scales` is not NULL, RN16(s[o] * that value).  The sum
+ * is rounded once (round to nearest, ties to even) and matches the exact sum
+ * bit for bit.
+ *   packed    aq_packed_codes_bytes(desc) bytes (from aq_pack_codes)
+ *   codebooks [K][2^B][8] binary16
+ *   scales    [out] binary16 or NULL
+ *   w         [out][in] binary16, row-major (written in full)
+ */
+aq_status aq_dequant(const aq_layer_desc *desc, const void *packed, const uint16_t *codebooks,
+                     const uint16_t *scales, uint16_t *w, aq_stream_t stream);
+
+/*
+ * Decode-time product for batch 1..16:
+ *   y[o][b] = RN16(s[o] * sum_i W[o][i] x[i][b]), fp32 accumulation.
+ *   packed    from aq_pack_codes
+ *   codebooks [K][2^B][8] binary16
+ *   scales    [out] binary16, or NULL for s = 1
+ *   x         [in][batch] binary16, row-major
+ *   y         [out][batch] binary16, row-major (written in full)
+ *   workspace >= aq_gemv_workspace_bytes(desc, batch) bytes (see above)
+ * Results are deterministic: the same inputs give the same bits.
+ * AQ_ERR_INVALID_ARG for batch outside 1..16.
+ */
+aq_status aq_gemv(const aq_layer_desc *desc, const void *packed, const uint16_t *codebooks,
+                  const uint16_t *scales, const uint16_t *x, int batch, uint16_t *y,
+                  void *workspace, size_t workspace_bytes, aq_stream_t stream);
+
+/*
+ * Prefill product for 1 <= T <= 2^22 tokens on the tensor cores (tcgen05.mma with
+ * binary16 operands and fp32 accumulation in tensor memory):
+ *   y[o][t] = RN16(s[o] * sum_i W[o][i] x[i][t]).
+ *   x [in][T] binary16 row-major; y [out][T] binary16 row-major; other
+ *   arguments as for aq_gemv; workspace >= aq_gemm_workspace_bytes(desc, T).
+ * Every wait inside the kernel is bounded: if one gives up, the kernel
+ * records AQ_ERR_TIMEOUT in the workspace status word (see
+ * aq_workspace_status), frees its tensor memory and returns; the output is
+ * then incomplete but the context stays usable.
+ */
+aq_status aq_gemm(const aq_layer_desc *desc, const void *packed, const uint16_t *codebooks,
+                  const uint16_t *scales, const uint16_t *x, int T, uint16_t *y,
+                  void *workspace, size_t workspace_bytes, aq_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* AQ_B200_H */

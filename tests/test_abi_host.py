@@ -1,0 +1,149 @@
+"""Host-side checks of the C ABI (no GPU needed, no kernel launched).
+
+The library must load, export every function include/aq.h declares, size
+buffers like the documented layout (checked against the oracle's
+independent implementation), and reject bad arguments before any launch.
+Every call below either touches no device memory or carries an argument
+the host validation rejects, so nothing here can reach a kernel.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import additive_quantized_matmul_b200 as aq
+import oracle
+from conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "aq.h")
+FAKE = 0x10000  # 16-byte aligned, never dereferenced: every call using it is rejected first
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(aq_[a-z_]+)\s*\(", text)))
+
+
+def test_header_and_binding_agree():
+    assert declared_functions() == sorted(aq.EXPORTED_SYMBOLS)
+
+
+def test_library_exports_every_declared_symbol():
+    out = subprocess.run(["nm", "-D", "--defined-only", aq.library_path],
+                         capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (aq_\w+)", out))
+    missing = set(declared_functions()) - exported
+    assert not missing, missing
+    for name in declared_functions():
+        assert hasattr(aq.lib, name)
+
+
+def test_library_has_no_oracle_or_torch_dependency():
+    out = subprocess.run(["nm", "-D", aq.library_path], capture_output=True, text=True).stdout
+    assert "aqo_" not in out
+    ldd = subprocess.run(["ldd", aq.library_path], capture_output=True, text=True).stdout
+    assert "torch" not in ldd and "aqoracle" not in ldd
+
+
+def test_version_and_status_strings():
+    assert aq.aq_version() == 10000
+    for s in range(7):
+        assert aq.aq_status_string(s)
+    assert aq.aq_status_string(99) == "unknown status"
+
+
+@pytest.mark.parametrize("out,inp,K,B", [(1, 8, 1, 16), (20, 520, 1, 16), (20, 520, 2, 8),
+                                         (4096, 4096, 1, 16), (11008, 4096, 2, 8),
+                                         (4096, 11008, 2, 8), (28672, 8192, 1, 16), (37, 360, 2, 8)])
+def test_packed_bytes_matches_oracle(out, inp, K, B):
+    d = aq.LayerDesc.make(out, inp, K, B)
+    assert aq.aq_packed_codes_bytes(d) == oracle.packed_bytes(out, inp, K, B)
+
+
+@pytest.mark.parametrize("desc,why", [
+    ((0, 64, 8, 1, 16), "no rows"), ((16, 0, 8, 1, 16), "no columns"), ((16, 12, 8, 1, 16), "in % 8"),
+    ((16, 64, 4, 1, 16), "group size"), ((16, 64, 8, 2, 16), "2x16"), ((16, 64, 8, 8, 8), "8x8"),
+    ((16, 64, 8, 1, 8), "1x8"), ((-1, 64, 8, 1, 16), "negative"),
+])
+def test_invalid_descriptors(desc, why):
+    d = aq.LayerDesc(*desc)
+    assert aq.aq_packed_codes_bytes(d) == 0, why
+    assert aq.aq_gemv_workspace_bytes(d, 1) == 0, why
+    want = 2 if desc[2] != 8 or (desc[3], desc[4]) not in ((1, 16), (2, 8)) else 1
+    if desc[0] < 1 or desc[1] < 8 or desc[1] % 8:
+        want = 1
+    st = aq.lib.aq_gemv(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, 1, FAKE, FAKE, 1 << 20, None)
+    assert st == want, why
+    st = aq.lib.aq_dequant(ctypes.byref(d), FAKE, FAKE, None, FAKE, None)
+    assert st == want, why
+
+
+def test_workspace_sizes_host_only():
+    d = aq.LayerDesc.make(4096, 4096, 1, 16)
+    for b in range(1, 17):
+        assert aq.aq_gemv_workspace_bytes(d, b) >= 16
+    assert aq.aq_gemv_workspace_bytes(d, 0) == 0
+    assert aq.aq_gemv_workspace_bytes(d, 17) == 0
+    assert aq.aq_gemm_workspace_bytes(d, 2048) >= 16
+    assert aq.aq_gemm_workspace_bytes(d, 0) == 0
+
+
+def _gemv(d, packed=FAKE, cb=FAKE, s=FAKE, x=FAKE, batch=1, y=FAKE, ws=FAKE, wsb=1 << 30):
+    return aq.lib.aq_gemv(ctypes.byref(d), packed, cb, s, x, batch, y, ws, wsb, None)
+
+
+def _gemm(d, packed=FAKE, cb=FAKE, s=FAKE, x=FAKE, T=64, y=FAKE, ws=FAKE, wsb=1 << 30):
+    return aq.lib.aq_gemm(ctypes.byref(d), packed, cb, s, x, T, y, ws, wsb, None)
+
+
+def test_gemv_argument_errors():
+    d = aq.LayerDesc.make(64, 256, 2, 8)
+    assert _gemv(None if False else d, batch=0) == 1
+    assert _gemv(d, batch=17) == 1
+    assert _gemv(d, packed=None) == 1
+    assert _gemv(d, cb=None) == 1
+    assert _gemv(d, x=None) == 1
+    assert _gemv(d, y=None) == 1
+    assert _gemv(d, packed=FAKE + 8) == 3
+    assert _gemv(d, x=FAKE + 2) == 3
+    assert _gemv(d, y=FAKE + 4) == 3
+    assert _gemv(d, cb=FAKE + 1) == 3
+    assert _gemv(d, s=FAKE + 1) == 3
+    assert _gemv(d, ws=None) == 4
+    assert _gemv(d, wsb=8) == 4
+    assert _gemv(d, ws=FAKE + 8) == 3
+    assert aq.lib.aq_gemv(None, FAKE, FAKE, FAKE, FAKE, 1, FAKE, FAKE, 1 << 20, None) == 1
+
+
+def test_gemm_argument_errors():
+    d = aq.LayerDesc.make(64, 256, 1, 16)
+    assert _gemm(d, T=0) == 1
+    assert _gemm(d, T=-5) == 1
+    assert _gemm(d, x=None) == 1
+    assert _gemm(d, y=FAKE + 2) == 3
+    assert _gemm(d, ws=None) == 4
+    assert _gemm(d, wsb=0) == 4
+
+
+def test_pack_and_misc_argument_errors():
+    d = aq.LayerDesc.make(64, 256, 1, 16)
+    assert aq.lib.aq_pack_codes(ctypes.byref(d), None, FAKE, None) == 1
+    assert aq.lib.aq_pack_codes(ctypes.byref(d), FAKE, FAKE + 4, None) == 3
+    assert aq.lib.aq_pack_codes(ctypes.byref(d), FAKE + 1, FAKE, None) == 3  # u16 codes odd address
+    assert aq.lib.aq_unpack_codes(ctypes.byref(d), FAKE + 8, FAKE, None) == 3
+    assert aq.lib.aq_dequant(ctypes.byref(d), FAKE, FAKE, FAKE + 1, FAKE, None) == 3
+    assert aq.lib.aq_workspace_status(None, None) == 1
+    assert aq.lib.aq_workspace_status(FAKE + 4, None) == 3
+    assert aq.lib.aq_selftest_bounded_wait(FAKE, 0, None) == 1
+    assert aq.lib.aq_selftest_bounded_wait(FAKE, (1 << 20) + 1, None) == 1
+    assert aq.lib.aq_selftest_bounded_wait(None, 10, None) == 1
+
+
+def test_binding_raises_on_error():
+    d = aq.LayerDesc.make(64, 256, 1, 16)
+    with pytest.raises(aq.AQError) as e:
+        aq.aq_gemv(d, FAKE, FAKE, FAKE, FAKE, 0, FAKE, FAKE, 1 << 20, stream=0)
+    assert e.value.name == "AQ_ERR_INVALID_ARG"

@@ -1,0 +1,240 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Codes, packed bytes and dequantised weights must match bit for bit; products
+must satisfy |y_gpu - y_ref| <= 1e-2 * sum_i |s||W||x| + 1e-3 per element,
+y_ref being the fp64 oracle.  Small layers are compared in full (several
+tiles plus ragged tails); the full-size workloads are compared on sampled
+rows, in the launch configuration the benchmark uses.
+"""
+import numpy as np
+import pytest
+import torch
+
+import additive_quantized_matmul_b200 as aq
+import oracle
+from aq_inputs import LayerSpec, make_activations, make_layer, workload
+from aqtest import (DevLayer, assert_close, dev, guarded, guards_intact, run_gemm, run_gemv,
+                    to_f16, workspace)
+
+pytestmark = pytest.mark.gpu
+
+SCHEMES = [(1, 16), (2, 8)]
+SMALL_SHAPES = [(8, 8), (37, 360), (256, 512), (1000, 1032), (64, 4096), (4100, 264)]
+
+
+def _layer(out, inp, K, B, seed, **kw):
+    return make_layer(LayerSpec(out, inp, K, B, codebook_sigma=kw.pop("sigma", 0.05), **kw), seed)
+
+
+# ---------------------------------------------------------------------------
+# pack / unpack / dequant: bit-exact
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("K,B", SCHEMES)
+@pytest.mark.parametrize("out,inp", SMALL_SHAPES)
+def test_pack_matches_oracle_bytes(K, B, out, inp):
+    layer = _layer(out, inp, K, B, out * 7 + inp)
+    dl = DevLayer(layer)
+    want = oracle.pack(layer.codes, K, B)
+    got = dl.packed.cpu().numpy()
+    assert np.array_equal(got, want)
+    back = torch.empty_like(dl.codes)
+    aq.aq_unpack_codes(dl.desc, dl.packed, back)
+    torch.cuda.synchronize()
+    assert torch.equal(back, dl.codes)
+
+
+@pytest.mark.parametrize("K,B", SCHEMES)
+@pytest.mark.parametrize("out,inp", SMALL_SHAPES)
+@pytest.mark.parametrize("scaled", [False, True])
+def test_dequant_bit_exact(K, B, out, inp, scaled):
+    layer = _layer(out, inp, K, B, out + inp + K)
+    dl = DevLayer(layer)
+    full, w = guarded(out * inp)
+    aq.aq_dequant(dl.desc, dl.packed, dl.codebooks, dl.scales if scaled else None, w)
+    torch.cuda.synchronize()
+    assert guards_intact(full)
+    want = oracle.decode(layer.codes, layer.codebooks, layer.scales if scaled else None)
+    assert np.array_equal(w.cpu().numpy().view(np.uint16).reshape(out, inp), want.view(np.uint16))
+
+
+def test_dequant_signed_zero_and_extremes():
+    layer = _layer(64, 256, 2, 8, 5)
+    cb = layer.codebooks.copy()
+    cb[0, :16] = -0.0
+    cb[1, :16] = -0.0
+    cb[0, 16:32] = 65504.0          # sums overflow to inf, as RN16 says
+    cb[1, 16:32] = 32.0
+    cb[0, 32:48] = np.float16(2.0 ** -24)  # subnormal sums
+    cb[1, 32:48] = np.float16(2.0 ** -24)
+    layer.codebooks = cb
+    layer.codes[:, :, :] = np.random.default_rng(1).integers(0, 48, size=layer.codes.shape)
+    dl = DevLayer(layer)
+    w = torch.empty(64 * 256, dtype=torch.int16, device="cuda")
+    aq.aq_dequant(dl.desc, dl.packed, dl.codebooks, None, w)
+    torch.cuda.synchronize()
+    want = oracle.decode(layer.codes, layer.codebooks)
+    assert np.array_equal(w.cpu().numpy().view(np.uint16).reshape(64, 256), want.view(np.uint16))
+
+
+# ---------------------------------------------------------------------------
+# decode-time product (batch 1..16)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("K,B", SCHEMES)
+@pytest.mark.parametrize("out,inp", SMALL_SHAPES)
+@pytest.mark.parametrize("batch", [1, 4, 16])
+def test_gemv_matches_oracle(K, B, out, inp, batch):
+    layer = _layer(out, inp, K, B, out * 3 + inp + batch)
+    x = make_activations(inp, batch, 77 + batch)
+    dl = DevLayer(layer)
+    y = run_gemv(dl, x)
+    ref, bound = oracle.matmul(layer.codes, layer.codebooks, layer.scales, x)
+    assert_close(y, ref, bound, f"gemv {K}x{B} {out}x{inp} b{batch}")
+
+
+@pytest.mark.parametrize("K,B", SCHEMES)
+@pytest.mark.parametrize("batch", range(1, 17))
+def test_gemv_every_batch(K, B, batch):
+    layer = _layer(300, 1032, K, B, 1234)
+    x = make_activations(1032, batch, batch)
+    dl = DevLayer(layer)
+    y = run_gemv(dl, x)
+    ref, bound = oracle.matmul(layer.codes, layer.codebooks, layer.scales, x)
+    assert_close(y, ref, bound, f"gemv {K}x{B} b{batch}")
+
+
+@pytest.mark.parametrize("K,B", SCHEMES)
+def test_gemv_deterministic_and_workspace_reusable(K, B):
+    layer = _layer(1024, 8192, K, B, 99)
+    dl = DevLayer(layer)
+    for batch in (1, 3, 16):
+        x = make_activations(8192, batch, batch)
+        ws = workspace(aq.aq_gemv_workspace_bytes(dl.desc, batch))
+        y1 = run_gemv(dl, x, ws)
+        y2 = run_gemv(dl, x, ws)  # counters must be back at zero
+        assert np.array_equal(y1, y2)
+        assert int(ws[16:].view(torch.int32)[: 1024 // 8].abs().sum().item()) == 0
+        ref, bound = oracle.matmul(layer.codes, layer.codebooks, layer.scales, x)
+        assert_close(y1, ref, bound, f"gemv {K}x{B} b{batch}")
+
+
+def test_gemv_without_scales_and_zipf_codes():
+    layer = _layer(512, 2048, 2, 8, 3, code_dist="zipf")
+    dl = DevLayer(layer)
+    x = make_activations(2048, 1, 4)
+    xd = dev(x.view(np.uint16))
+    y = torch.empty(512, dtype=torch.int16, device="cuda")
+    ws = workspace(aq.aq_gemv_workspace_bytes(dl.desc, 1))
+    aq.aq_gemv(dl.desc, dl.packed, dl.codebooks, None, xd, 1, y, ws)
+    torch.cuda.synchronize()
+    ref, bound = oracle.matmul(layer.codes, layer.codebooks, None, x)
+    assert_close(to_f16(y).astype(np.float64)[:, None], ref, bound, "gemv no scales")
+
+
+def test_gemv_rejects_small_workspace_without_writing():
+    layer = _layer(256, 512, 2, 8, 4)
+    dl = DevLayer(layer)
+    xd = dev(make_activations(512, 1, 1).view(np.uint16))
+    full, y = guarded(256)
+    ws = workspace(16)
+    need = aq.aq_gemv_workspace_bytes(dl.desc, 1)
+    with pytest.raises(aq.AQError) as e:
+        aq.aq_gemv(dl.desc, dl.packed, dl.codebooks, dl.scales, xd, 1, y, ws, need - 1)
+    assert e.value.name == "AQ_ERR_WORKSPACE"
+    torch.cuda.synchronize()
+    assert guards_intact(full) and bool((y == 0x7E5A).all())
+
+
+# ---------------------------------------------------------------------------
+# prefill product on the tensor cores
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("K,B", SCHEMES)
+@pytest.mark.parametrize("out,inp", [(128, 64), (256, 512), (129, 136), (1000, 1032), (8, 8)])
+@pytest.mark.parametrize("T", [1, 5, 8, 64, 136, 300])
+def test_gemm_matches_oracle(K, B, out, inp, T):
+    layer = _layer(out, inp, K, B, out + inp * 5 + T)
+    x = make_activations(inp, T, T)
+    dl = DevLayer(layer)
+    y = run_gemm(dl, x)
+    ref, bound = oracle.matmul(layer.codes, layer.codebooks, layer.scales, x)
+    assert_close(y, ref, bound, f"gemm {K}x{B} {out}x{inp} T{T}")
+
+
+def test_gemm_deterministic():
+    layer = _layer(512, 1024, 1, 16, 8)
+    dl = DevLayer(layer)
+    x = make_activations(1024, 256, 9)
+    assert np.array_equal(run_gemm(dl, x), run_gemm(dl, x))
+
+
+# ---------------------------------------------------------------------------
+# bounded waits report instead of hanging
+# ---------------------------------------------------------------------------
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    ws = workspace(16)
+    aq.aq_selftest_bounded_wait(ws, 1000)
+    assert aq.aq_workspace_status(ws) == 6  # AQ_ERR_TIMEOUT
+    assert aq.aq_workspace_status(ws) == 0  # cleared by the read
+    layer = _layer(64, 256, 1, 16, 2)
+    dl = DevLayer(layer)
+    x = make_activations(256, 2, 3)
+    ref, bound = oracle.matmul(layer.codes, layer.codebooks, layer.scales, x)
+    assert_close(run_gemv(dl, x), ref, bound, "after timeout")
+
+
+# ---------------------------------------------------------------------------
+# full-size workloads, sampled rows (same launch configuration as bench.py)
+# ---------------------------------------------------------------------------
+
+def _sample_rows(out, n=48, seed=0):
+    rng = np.random.default_rng(seed)
+    rows = set(rng.choice(out, size=min(n, out), replace=False).tolist())
+    rows.update({0, out - 1, min(out - 1, 127), min(out - 1, 128)})
+    return np.array(sorted(rows))
+
+
+@pytest.mark.parametrize("name", ["tiny-2x8", "llama2-7b-1x16", "llama2-7b-mlp-2x8", "llama2-70b-1x16"])
+def test_gemv_full_size_sampled(name):
+    wl = workload(name)
+    for i, (tag, spec) in enumerate(wl["layers"]):
+        layer = make_layer(spec, (wl["seed"], i))
+        dl = DevLayer(layer)
+        for batch in wl["n"]:
+            x = make_activations(spec.in_features, batch, (wl["seed"], i, batch))
+            y = run_gemv(dl, x)
+            rows = _sample_rows(spec.out_features, seed=i)
+            ref, bound = oracle.matmul(layer.codes, layer.codebooks, layer.scales, x, rows=rows, threads=8)
+            assert_close(y[rows], ref, bound, f"{name}/{tag} b{batch}")
+        del dl
+        torch.cuda.empty_cache()
+
+
+def test_gemm_full_size_sampled():
+    wl = workload("llama2-7b-prefill")
+    for i, (tag, spec) in enumerate(wl["layers"]):
+        layer = make_layer(spec, (wl["seed"], i))
+        dl = DevLayer(layer)
+        for T in wl["n"]:
+            x = make_activations(spec.in_features, T, (wl["seed"], i, T))
+            y = run_gemm(dl, x)
+            rows = _sample_rows(spec.out_features, n=12, seed=i)
+            ref, bound = oracle.matmul(layer.codes, layer.codebooks, layer.scales, x, rows=rows, threads=8)
+            assert_close(y[rows], ref, bound, f"prefill/{tag} T{T}")
+        del dl
+        torch.cuda.empty_cache()
+
+
+def test_dequant_full_size_sampled():
+    spec = LayerSpec(28672, 8192, 1, 16)
+    layer = make_layer(spec, 5)
+    dl = DevLayer(layer)
+    w = torch.empty(spec.out_features * spec.in_features, dtype=torch.int16, device="cuda")
+    aq.aq_dequant(dl.desc, dl.packed, dl.codebooks, dl.scales, w)
+    torch.cuda.synchronize()
+    rows = _sample_rows(spec.out_features, n=64)
+    got = w.view(spec.out_features, spec.in_features)[torch.from_numpy(rows).cuda()].cpu().numpy()
+    want = oracle.decode(layer.codes[rows], layer.codebooks, layer.scales[rows])
+    assert np.array_equal(got.view(np.uint16), want.view(np.uint16))
