@@ -67,18 +67,19 @@ __device__ __forceinline__ uint32_t f2h2(float a, float b)
     return *reinterpret_cast<uint32_t *>(&h);
 }
 
-// Sum of two binary16 8-vectors rounded once to binary16.  The fp32 sum of
-// two binary16 values, rounded to binary16, equals the correctly rounded
-// exact sum (24 >= 2*11 + 2 bits, so the double rounding is innocuous).
+// Sum of two binary16 8-vectors rounded once to binary16 (IEEE binary16
+// addition, round to nearest even: the correctly rounded exact sum, signed
+// zeros and overflow to infinity included).
+__device__ __forceinline__ uint32_t hadd2_u32(uint32_t a, uint32_t b)
+{
+    __half2 r = __hadd2(*reinterpret_cast<__half2 *>(&a), *reinterpret_cast<__half2 *>(&b));
+    return *reinterpret_cast<uint32_t *>(&r);
+}
+
 __device__ __forceinline__ uint4 add_round_h8(uint4 a, uint4 b)
 {
-    uint4 r;
-    float2 x, y;
-    x = h2f2(a.x); y = h2f2(b.x); r.x = f2h2(x.x + y.x, x.y + y.y);
-    x = h2f2(a.y); y = h2f2(b.y); r.y = f2h2(x.x + y.x, x.y + y.y);
-    x = h2f2(a.z); y = h2f2(b.z); r.z = f2h2(x.x + y.x, x.y + y.y);
-    x = h2f2(a.w); y = h2f2(b.w); r.w = f2h2(x.x + y.x, x.y + y.y);
-    return r;
+    return make_uint4(hadd2_u32(a.x, b.x), hadd2_u32(a.y, b.y), hadd2_u32(a.z, b.z),
+                      hadd2_u32(a.w, b.w));
 }
 
 // s * w for eight binary16 w, rounded once (the fp32 product is exact).
@@ -105,22 +106,20 @@ __device__ __forceinline__ float dot8(uint4 w, uint4 x, float acc)
     return acc;
 }
 
+// Read-only loads.  Not volatile: the compiler may hoist them, so that all
+// independent gathers of a thread are in flight before the first use.
 __device__ __forceinline__ uint4 ldg_nc_v4(const void *p)
 {
-    uint4 r;
-    asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-                 : "l"(p));
-    return r;
+    return __ldg(reinterpret_cast<const uint4 *>(p));
 }
 
 // Streaming load: read once, do not keep in L1.
 __device__ __forceinline__ uint4 ldg_stream_v4(const void *p)
 {
     uint4 r;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-                 : "l"(p));
+    asm("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+        : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+        : "l"(p));
     return r;
 }
 

@@ -13,7 +13,10 @@
 // Every wait is bounded (wall-clock limit via %globaltimer): on give-up the
 // kernel records AQ_ERR_TIMEOUT in the workspace status word, drains what
 // it issued (again bounded), frees its tensor memory and returns.
-#include "aq_common.cuh"
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "tc_common.cuh"
 
 namespace aqk {
 
@@ -24,115 +27,6 @@ constexpr int kStages = 2;
 constexpr int kGemmThreads = 128;  // 4 warps: decode, stage X, epilogue
 constexpr int kTileABytes = kBM * kBK * 2;  // 16 KiB
 constexpr int kTileBBytes = kBK * kBN * 2;  // 16 KiB
-constexpr uint64_t kWaitNs = 1000000000ull; // 1 s per wait
-
-// ---- PTX wrappers -----------------------------------------------------------
-
-__device__ __forceinline__ uint64_t globaltimer()
-{
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-
-// Wait for a phase of an mbarrier for at most `ns` nanoseconds.
-__device__ __forceinline__ bool mbar_wait_ns(uint64_t *bar, uint32_t parity, uint64_t ns)
-{
-    if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = globaltimer();
-    for (uint32_t i = 0; i < (1u << 30); ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if (globaltimer() - t0 > ns) return false;
-    }
-    return false;
-}
-
-__device__ __forceinline__ void fence_proxy_async_smem()
-{
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-__device__ __forceinline__ void tmem_alloc(uint32_t *dst_smem, uint32_t ncols)
-{
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
-                 ::"r"(smem_u32(dst_smem)), "r"(ncols));
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::);
-}
-
-__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols)
-{
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols));
-}
-
-// D[tmem] (+)= A[smem desc] * B[smem desc]; accumulate selects D += vs D =.
-__device__ __forceinline__ void mma_f16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                           uint32_t idesc, uint32_t accumulate)
-{
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
-}
-
-// Arrive (once) on `bar` when every tcgen05.mma issued so far by this thread
-// has completed.
-__device__ __forceinline__ void mma_commit(uint64_t *bar)
-{
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
-                 ::"r"(smem_u32(bar)) : "memory");
-}
-
-// 32 lanes x 16 consecutive fp32 columns of tensor memory -> 16 registers.
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float v[16])
-{
-    uint32_t r[16];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
-}
-
-// Shared-memory matrix descriptor (sm_100 layout): start address >> 4 in
-// bits 0-13, leading byte offset >> 4 in 16-29, stride byte offset >> 4 in
-// 32-45, descriptor version 1 in bits 46-47, swizzle mode in 61-63
-// (2 = 128-byte swizzle).
-__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr, uint32_t lbo, uint32_t sbo)
-{
-    uint64_t d = 0;
-    d |= (uint64_t)((addr >> 4) & 0x3fff);
-    d |= (uint64_t)((lbo >> 4) & 0x3fff) << 16;
-    d |= (uint64_t)((sbo >> 4) & 0x3fff) << 32;
-    d |= (uint64_t)1 << 46;
-    d |= (uint64_t)2 << 61;
-    return d;
-}
-
-// Instruction descriptor for kind::f16: fp32 accumulator (bits 4-5 = 1),
-// binary16 A and B (formats 0), A K-major (bit 15 = 0), B MN-major
-// (bit 16 = 1), N >> 3 in bits 17-22, M >> 4 in bits 24-28.
-__host__ __device__ constexpr uint32_t make_idesc(int M, int N)
-{
-    return (1u << 4) | (0u << 7) | (0u << 10) | (0u << 15) | (1u << 16) |
-           ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
-}
-
-// Byte offset of 16-byte chunk c (0..7) of row r in a 128-byte-swizzled
-// tile of 128-byte rows (rows 8-aligned into 1024-byte atoms).
-__device__ __forceinline__ uint32_t sw128(uint32_t row, uint32_t c)
-{
-    return row * 128u + ((c ^ (row & 7u)) << 4);
-}
-
 // ---- kernel -----------------------------------------------------------------
 
 template <int K>
@@ -292,6 +186,237 @@ gemm_tc_kernel(Geom L, const uint4 *__restrict__ packed, const uint4 *__restrict
     if (warp == 0) tmem_dealloc(tmem, kBN);
 }
 
+
+// ---- warp-specialised kernel (T a multiple of 8) ---------------------------
+//
+// Tile M = 128 rows x N = 256 tokens, K = 64 per stage, 4-stage ring.
+//   warp 0     X producer: one lane issues four 2-D TMA loads per stage (64
+//              tokens x 64 features each, 128-byte swizzle, MN-major) that
+//              complete on full_b[stage];
+//   warp 1     MMA issuer: one lane waits for full_a/full_b, issues four
+//              tcgen05.mma (M 128, N 256, K 16) into a 256-column fp32 TMEM
+//              accumulator and commits to empty[stage] (buffer free) and,
+//              after the last stage, to acc_full;
+//   warps 2-5  decoders, then epilogue: thread t owns code chunk (row tile
+//              t/8, group t%8) of each stage.  1x16: the 8 codewords go from
+//              the L2-resident codebook straight into the swizzled A tile by
+//              16-byte cp.async, a few stages ahead; 2x8: codewords come from
+//              the codebooks in shared memory, summed with binary16 adds.
+//              Each thread fences its writes to the async proxy and arrives
+//              on full_a[stage] (128 arrivals).  The epilogue reads TMEM lanes
+//              32*(warp%4).. with tcgen05.ld, scales, rounds and stores.
+constexpr int kWsBN = 256;
+constexpr int kWsStages = 4;
+constexpr int kWsThreads = 192;               // 6 warps
+constexpr int kWsTileB = kBK * kWsBN * 2;     // 32 KiB
+constexpr int kWsLag = 2;                     // cp.async stages in flight per decoder (< ring depth)
+
+template <int K>
+__global__ void __launch_bounds__(kWsThreads, 1)
+gemm_ws_kernel(const __grid_constant__ CUtensorMap xmap, Geom L, const uint4 *__restrict__ packed,
+               const uint4 *__restrict__ cb, const uint16_t *__restrict__ scales, int T,
+               uint16_t *__restrict__ y, void *ws)
+{
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    uint8_t *smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+    uint8_t *tileA = smem;                                   // [4][16 KiB]
+    uint8_t *tileB = smem + kWsStages * kTileABytes;         // [4][32 KiB]
+    uint4 *scb = reinterpret_cast<uint4 *>(tileB + kWsStages * kWsTileB);
+    uint64_t *full_a = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(scb) + (K == 2 ? 512 * 16 : 0));
+    uint64_t *full_b = full_a + kWsStages;
+    uint64_t *empty = full_b + kWsStages;
+    uint64_t *acc_full = empty + kWsStages;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 1);
+    uint32_t *abort_flag = tmem_slot + 1;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int m0 = blockIdx.x * kBM;
+    const int n0 = blockIdx.y * kWsBN;
+    const int nk = (L.in + kBK - 1) / kBK;
+
+    if (K == 1 && tid == 0) prefetch_table_share(cb, 65536u * 16u);
+    if (K == 2)
+        for (int i = tid; i < 512; i += kWsThreads) scb[i] = cb[i];
+    if (tid == 0) {
+        for (int s = 0; s < kWsStages; ++s) {
+            mbar_init(&full_a[s], 128);
+            mbar_init(&full_b[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(acc_full, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) tmem_alloc(tmem_slot, kWsBN);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    volatile uint32_t *abort_v = abort_flag;
+
+    if (warp == 0) {
+        // ---------------- X producer ----------------
+        if (lane == 0) {
+            for (int s = 0; s < nk; ++s) {
+                const int buf = s % kWsStages;
+                if (s >= kWsStages && !mbar_wait_ns(&empty[buf], ((s / kWsStages) - 1) & 1, kWaitNs)) {
+                    *abort_v = 1;
+                    break;
+                }
+                if (*abort_v) break;
+                mbar_arrive_expect_tx(&full_b[buf], kWsTileB);
+                const uint32_t dst = smem_u32(tileB + buf * kWsTileB);
+#pragma unroll
+                for (int q = 0; q < kWsBN / 64; ++q)
+                    tma_load_2d(dst + q * (kBK * 128), &xmap, n0 + 64 * q, s * kBK, &full_b[buf]);
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            const uint32_t idesc = make_idesc(kBM, kWsBN, true);
+            int s = 0;
+            for (; s < nk; ++s) {
+                const int buf = s % kWsStages;
+                const uint32_t par = (s / kWsStages) & 1;
+                if (!mbar_wait_ns(&full_a[buf], par, kWaitNs) || !mbar_wait_ns(&full_b[buf], par, kWaitNs)) {
+                    *abort_v = 1;
+                    break;
+                }
+                if (*abort_v) break;
+                tc_fence_after();
+                const uint32_t a0 = smem_u32(tileA + buf * kTileABytes);
+                const uint32_t b0 = smem_u32(tileB + buf * kWsTileB);
+#pragma unroll
+                for (int ks = 0; ks < kBK / 16; ++ks) {
+                    const uint64_t ad = smem_desc_sw128(a0 + ks * 32, 16, 1024);
+                    const uint64_t bd = smem_desc_sw128(b0 + ks * 2048, kBK * 128, 1024);
+                    mma_f16_ss(tmem, ad, bd, idesc, (s > 0 || ks > 0) ? 1u : 0u);
+                }
+                mma_commit(&empty[buf]);
+            }
+            mma_commit(acc_full);  // completes when every MMA issued above has
+        }
+    } else {
+        // ---------------- decoders ----------------
+        const int t = tid - 64;  // 0..127
+        const int rt_l = t >> 3, gi = t & 7;
+        const int rt = (m0 >> 3) + rt_l;
+        const bool rows_live = rt < L.rtiles;
+        // code chunks kCodeAhead stages ahead (register ring): a stage's
+        // gathers never wait on an HBM round trip
+        constexpr int kCodeAhead = 4;
+        uint4 code_ring[kCodeAhead];
+#pragma unroll
+        for (int q = 0; q < kCodeAhead; ++q)
+            code_ring[q] = (q < nk && rows_live && q * 8 + gi < L.G) ? ldg_stream_v4(packed + (size_t)rt * L.gp + q * 8 + gi)
+                                                                    : make_uint4(0, 0, 0, 0);
+        const int lag = (K == 1) ? kWsLag : 0;
+        for (int s = 0; s < nk + lag; ++s) {
+            if (s < nk) {
+                const int buf = s % kWsStages;
+                if (s >= kWsStages && !mbar_wait_ns(&empty[buf], ((s / kWsStages) - 1) & 1, kWaitNs)) {
+                    *abort_v = 1;
+                }
+                if (*abort_v) break;
+                uint4 code = code_ring[0];
+#pragma unroll
+                for (int q = 1; q < kCodeAhead; ++q)
+                    if ((s & (kCodeAhead - 1)) == q) code = code_ring[q];
+                const bool live = rows_live && s * 8 + gi < L.G;
+                {
+                    const int g = (s + kCodeAhead) * 8 + gi;
+                    const uint4 nxt = (s + kCodeAhead < nk && rows_live && g < L.G)
+                                          ? ldg_stream_v4(packed + (size_t)rt * L.gp + g)
+                                          : make_uint4(0, 0, 0, 0);
+#pragma unroll
+                    for (int q = 0; q < kCodeAhead; ++q)
+                        if ((s & (kCodeAhead - 1)) == q) code_ring[q] = nxt;
+                }
+                uint32_t wd[8];
+                wd[0] = code.x & 0xffff; wd[1] = code.x >> 16; wd[2] = code.y & 0xffff; wd[3] = code.y >> 16;
+                wd[4] = code.z & 0xffff; wd[5] = code.z >> 16; wd[6] = code.w & 0xffff; wd[7] = code.w >> 16;
+                uint8_t *A = tileA + buf * kTileABytes;
+                if (K == 1) {
+                    const uint32_t a0 = smem_u32(A);
+#pragma unroll
+                    for (int r = 0; r < 8; ++r)
+                        cp_async16(a0 + sw128(rt_l * 8 + r, gi), live ? (const void *)(cb + wd[r]) : (const void *)cb,
+                                   live ? 16u : 0u);
+                } else {
+#pragma unroll
+                    for (int r = 0; r < 8; ++r) {
+                        const uint4 v = live ? add_round_h8(scb[wd[r] & 0xff], scb[256 + (wd[r] >> 8)])
+                                             : make_uint4(0, 0, 0, 0);
+                        *reinterpret_cast<uint4 *>(A + sw128(rt_l * 8 + r, gi)) = v;
+                    }
+                }
+            }
+            if (K == 1) {
+                cp_async_commit();
+                const int j = s - lag;
+                if (j >= 0) {
+                    cp_async_wait<kWsLag>();
+                    fence_proxy_async_smem();
+                    mbar_arrive(&full_a[j % kWsStages]);
+                }
+            } else {
+                fence_proxy_async_smem();
+                mbar_arrive(&full_a[s % kWsStages]);
+            }
+        }
+        cp_async_wait<0>();
+        // ---------------- epilogue ----------------
+        const bool got = (*abort_v == 0) && mbar_wait_ns(acc_full, 0, kWaitNs);
+        if (!got) *abort_v = 1;
+        tc_fence_after();
+        // every decoder warp takes the same branch: abort is only set before
+        // this point by a role that gave up, or just above by a lane whose
+        // wait failed (then its warp-mates see it through the ballot)
+        const bool warp_ok = __all_sync(0xffffffffu, got);
+        if (warp_ok) {
+            const int q = warp & 3;  // TMEM lane quarter of this warp
+            const int row = m0 + q * 32 + lane;
+            const float sc = (row < L.out && scales) ? __half2float(__ushort_as_half(scales[row])) : 1.f;
+            const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16);
+#pragma unroll 1
+            for (int c0 = 0; c0 < kWsBN; c0 += 16) {
+                float v[16];
+                tmem_ld16(tbase + c0, v);
+                const int gn = n0 + c0;
+                if (row < L.out && gn < T) {
+                    uint16_t *dst = y + (size_t)row * T + gn;
+                    if (gn + 16 <= T) {
+                        const uint4 o0 = make_uint4(f2h2(sc * v[0], sc * v[1]), f2h2(sc * v[2], sc * v[3]),
+                                                    f2h2(sc * v[4], sc * v[5]), f2h2(sc * v[6], sc * v[7]));
+                        const uint4 o1 = make_uint4(f2h2(sc * v[8], sc * v[9]), f2h2(sc * v[10], sc * v[11]),
+                                                    f2h2(sc * v[12], sc * v[13]), f2h2(sc * v[14], sc * v[15]));
+                        reinterpret_cast<uint4 *>(dst)[0] = o0;
+                        reinterpret_cast<uint4 *>(dst)[1] = o1;
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j)
+                            if (gn + j < T) dst[j] = __half_as_ushort(__float2half_rn(sc * v[j]));
+                    }
+                }
+            }
+        }
+    }
+    __syncthreads();
+    if (*abort_v) {
+        // something gave up: record it and drain what was issued (bounded)
+        if (tid == 0) record_status(ws, AQ_ERR_TIMEOUT);
+        if (tid == 32) mbar_wait_ns(acc_full, 0, kWaitNs);
+        if (tid == 0)
+            for (int s = max(0, nk - kWsStages); s < nk; ++s)
+                mbar_wait_ns(&full_b[s % kWsStages], (s / kWsStages) & 1, kWaitNs);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, kWsBN);
+}
+
 // ---- self-test of the bounded wait -----------------------------------------
 
 __global__ void selftest_wait_kernel(void *ws, int spin_limit)
@@ -320,15 +445,61 @@ static constexpr int gemm_smem_bytes()
            kStages * 8 + 16;
 }
 
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+static constexpr int gemm_ws_smem_bytes(int K)
+{
+    return 1024 + kWsStages * (kTileABytes + kWsTileB) + (K == 2 ? 512 * 16 : 0) +
+           (3 * kWsStages + 1) * 8 + 16;
+}
+
 cudaError_t launch_gemm(const Geom &g, const void *packed, const uint16_t *cb,
                         const uint16_t *scales, const uint16_t *x, int T, uint16_t *y, void *ws,
                         cudaStream_t s)
 {
-    const int smem = gemm_smem_bytes();
-    dim3 grid((g.out + kBM - 1) / kBM, (T + kBN - 1) / kBN);
     const uint4 *pk = reinterpret_cast<const uint4 *>(packed);
     const uint4 *c = reinterpret_cast<const uint4 *>(cb);
     cudaError_t e;
+    PFN_cuTensorMapEncodeTiled_v12000 encode = (T % 8 == 0) ? tensor_map_encoder() : nullptr;
+    if (encode) {
+        // X [in][T] binary16: innermost dimension tokens, box 64 tokens x 64 features
+        CUtensorMap map;
+        cuuint64_t dims[2] = {(cuuint64_t)T, (cuuint64_t)g.in};
+        cuuint64_t strides[1] = {(cuuint64_t)T * 2};
+        cuuint32_t box[2] = {64, (cuuint32_t)kBK};
+        cuuint32_t estr[2] = {1, 1};
+        CUresult r = encode(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<uint16_t *>(x), dims, strides,
+                            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+        const dim3 grid((g.out + kBM - 1) / kBM, (T + kWsBN - 1) / kWsBN);
+        const int smem = gemm_ws_smem_bytes(g.K);
+        if (g.K == 1) {
+            e = cudaFuncSetAttribute(gemm_ws_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+            if (e != cudaSuccess) return e;
+            gemm_ws_kernel<1><<<grid, kWsThreads, smem, s>>>(map, g, pk, c, scales, T, y, ws);
+        } else {
+            e = cudaFuncSetAttribute(gemm_ws_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+            if (e != cudaSuccess) return e;
+            gemm_ws_kernel<2><<<grid, kWsThreads, smem, s>>>(map, g, pk, c, scales, T, y, ws);
+        }
+        return cudaGetLastError();
+    }
+    // T not a multiple of 8: rows of X are not 16-byte aligned for TMA; the
+    // two-stage kernel stages X with ordinary loads.
+    const int smem = gemm_smem_bytes();
+    const dim3 grid((g.out + kBM - 1) / kBM, (T + kBN - 1) / kBN);
     if (g.K == 1) {
         e = cudaFuncSetAttribute(gemm_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;

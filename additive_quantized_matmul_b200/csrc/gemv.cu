@@ -1,25 +1,27 @@
-// Decode-time product y = diag(s) W x for batch 1..16 on CUDA cores (sm_100a).
+// Decode-time product y = diag(s) W x for batch 1..16 (sm_100a).
 //
-// W is never materialised: each 8-weight group is rebuilt from its codes on
-// the fly (AQLM wiki entry, "Niveau intermédiaire": w ~ sum_k C_k[i_k];
-// devtrends.ru summary, "Как это работает технически?": groups of 8) and
-// multiplied with the matching 8 activations; the products the paper's
-// abstract names for token generation.
+// W is never materialised in HBM: each 8-weight group is rebuilt from its
+// codes on the fly (AQLM wiki entry, "Niveau intermédiaire": w ~ sum_k
+// C_k[i_k]; devtrends.ru summary, "Как это работает технически?": groups of
+// 8) and multiplied with the matching 8 activations, the product the
+// paper's abstract names for token generation.
 //
-// Work decomposition shared by the kernels: a warp owns one 8-row tile and
-// a set of 32-group blocks; lane l takes group 32*gb + l and loads the
-// 16-byte packed chunk holding that group's code word for all 8 rows, so
-// one warp load streams 512 contiguous bytes of codes.  Each lane keeps
-// eight row accumulators; a 9-shuffle reduce-scatter sums them over lanes.
+// Two kernels, chosen by scheme and batch:
+//  * 2x8, batch 1 -- `gemv_2x8_lut_kernel`: per-group codebook x activation
+//    tables in shared memory, lane-private so random codes never conflict;
+//    two 4-byte table reads per group.
+//  * 1x16 any batch, 2x8 batch 2..16 -- `gemv_tc_kernel`: codes are decoded
+//    into a 128x64 binary16 tile in shared memory (128-byte-swizzled,
+//    K-major) and multiplied by the activations on the tensor cores
+//    (tcgen05.mma, M = 128, N = 16, fp32 accumulator in tensor memory), so
+//    the cost per group does not grow with the batch.  For 1x16 the bound is
+//    the rate of random 16-byte codeword reads from the L2-resident 1 MiB
+//    codebook (about one request per SM clock), not HBM.
 // Split-K partial sums go to the workspace and the last CTA to arrive for a
-// row range adds them in a fixed order (no float atomics: results are
-// bit-reproducible).
-#include "aq_common.cuh"
+// row range adds them in split order (no float atomics: bit-reproducible).
+#include "tc_common.cuh"
 
 namespace aqk {
-
-constexpr int kWarps = 8;
-constexpr int kThreads = kWarps * 32;
 
 struct SplitK {
     float *partials;      // [ks][rows8][batch]
@@ -27,12 +29,13 @@ struct SplitK {
 };
 
 // Called by every thread of a CTA after it stored its partial sums for rows
-// [row0, row0 + nrows), columns [col0, col0 + ncols) of split blockIdx.y.
-// The last CTA of the row range to arrive reduces the splits in split order
-// and writes y.
+// [row0, row0 + nrows), columns [0, batch) of split blockIdx.y (nrows is a
+// multiple of 8, so the block is a whole number of float4).  The last CTA of
+// the row range to arrive reduces the splits in split order, writes y and
+// resets the counter for the next call.  All loads of a float4 are issued
+// before the (ordered) sum, so the finish costs about one L2 round trip.
 __device__ __forceinline__ void splitk_finish(const Geom &L, SplitK sk, int row0, int nrows,
-                                              int batch, int col0, int ncols,
-                                              const uint16_t *__restrict__ scales,
+                                              int batch, const uint16_t *__restrict__ scales,
                                               uint16_t *__restrict__ y)
 {
     __shared__ unsigned s_last;
@@ -46,117 +49,41 @@ __device__ __forceinline__ void splitk_finish(const Geom &L, SplitK sk, int row0
     if (!s_last) return;
     __threadfence();
     const int ks = gridDim.y;
-    const size_t stride = (size_t)L.rows8 * batch;
-    for (int e = threadIdx.x; e < nrows * ncols; e += blockDim.x) {
-        int row = row0 + e / ncols;
-        int b = col0 + e % ncols;
-        if (row >= L.out) continue;
-        const float *p = sk.partials + (size_t)row * batch + b;
-        float v = 0.f;
-        for (int s = 0; s < ks; ++s) v += __ldcg(p + s * stride);
-        float sc = scales ? __half2float(__ushort_as_half(scales[row])) : 1.f;
-        y[(size_t)row * batch + b] = __half_as_ushort(__float2half_rn(sc * v));
+    const size_t vstride = (size_t)L.rows8 * batch / 4;
+    const float4 *base = reinterpret_cast<const float4 *>(sk.partials + (size_t)row0 * batch);
+    const int nvec = nrows * batch / 4;
+    for (int e = threadIdx.x; e < nvec; e += blockDim.x) {
+        float4 acc = __ldcg(base + e);
+        for (int s0 = 1; s0 < ks; s0 += 8) {
+            float4 t[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                if (s0 + j < ks) t[j] = __ldcg(base + (size_t)(s0 + j) * vstride + e);
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                if (s0 + j < ks) {
+                    acc.x += t[j].x; acc.y += t[j].y; acc.z += t[j].z; acc.w += t[j].w;
+                }
+        }
+        const float v[4] = {acc.x, acc.y, acc.z, acc.w};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const int idx = e * 4 + c;
+            const int row = row0 + idx / batch;
+            const int b = idx % batch;
+            if (row < L.out) {
+                const float sc = scales ? __half2float(__ushort_as_half(scales[row])) : 1.f;
+                y[(size_t)row * batch + b] = __half_as_ushort(__float2half_rn(sc * v[c]));
+            }
+        }
     }
-    if (threadIdx.x == 0) sk.counters[blockIdx.x] = 0u;  // ready for the next call
+    if (threadIdx.x == 0) sk.counters[blockIdx.x] = 0u;
 }
 
-// ---------------------------------------------------------------------------
-// Row-warp kernel: any scheme, NB batch columns per pass (NB in {1, 2, 4}).
-// grid = (row tiles, splits); block = 8 warps, warp w of split s takes group
-// blocks gb0 + w, gb0 + w + 8, ... of the split's range.
-// ---------------------------------------------------------------------------
-template <int K, int NB>
-__global__ void __launch_bounds__(kThreads)
-gemv_rowwarp_kernel(Geom L, const uint4 *__restrict__ packed, const uint4 *__restrict__ cb,
-                    const uint16_t *__restrict__ scales, const uint16_t *__restrict__ x,
-                    int batch, int col0, uint16_t *__restrict__ y, SplitK sk, int gbs_per_split)
+__device__ __forceinline__ void unpack8(uint4 c, uint32_t w[8])
 {
-    __shared__ uint4 scb[K == 2 ? 512 : 1];
-    __shared__ float red[kWarps][8][NB];
-    if (K == 2) {
-        for (int i = threadIdx.x; i < 512; i += kThreads) scb[i] = cb[i];
-        __syncthreads();
-    }
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int rt = blockIdx.x;
-    const int gb0 = blockIdx.y * gbs_per_split;
-    const int gb1 = min(L.gblocks, gb0 + gbs_per_split);
-    const int ncols = min(NB, batch - col0);
-
-    float acc[8][NB];
-#pragma unroll
-    for (int r = 0; r < 8; ++r)
-#pragma unroll
-        for (int b = 0; b < NB; ++b) acc[r][b] = 0.f;
-
-    for (int gb = gb0 + warp; gb < gb1; gb += kWarps) {
-        const int g = gb * 32 + lane;
-        if (g >= L.G) continue;  // padded group: no activations
-        const uint4 chunk = ldg_stream_v4(packed + (size_t)rt * L.gp + g);
-        uint4 xg[NB];
-        if (NB == 1 && batch == 1) {
-            xg[0] = ldg_nc_v4(x + (size_t)g * 8);
-        } else {
-#pragma unroll
-            for (int b = 0; b < NB; ++b) {
-                uint16_t h[8];
-#pragma unroll
-                for (int j = 0; j < 8; ++j)
-                    h[j] = (b < ncols) ? x[((size_t)g * 8 + j) * batch + col0 + b] : (uint16_t)0;
-                xg[b] = make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16),
-                                   h[4] | (h[5] << 16), h[6] | (h[7] << 16));
-            }
-        }
-        const uint32_t wd[8] = {chunk.x & 0xffff, chunk.x >> 16, chunk.y & 0xffff, chunk.y >> 16,
-                                chunk.z & 0xffff, chunk.z >> 16, chunk.w & 0xffff, chunk.w >> 16};
-#pragma unroll
-        for (int r = 0; r < 8; ++r) {
-            uint4 wv;
-            if (K == 1)
-                wv = ldg_nc_v4(cb + wd[r]);
-            else
-                wv = add_round_h8(scb[wd[r] & 0xff], scb[256 + (wd[r] >> 8)]);
-#pragma unroll
-            for (int b = 0; b < NB; ++b) acc[r][b] = dot8(wv, xg[b], acc[r][b]);
-        }
-    }
-#pragma unroll
-    for (int b = 0; b < NB; ++b) {
-        float col[8];
-#pragma unroll
-        for (int r = 0; r < 8; ++r) col[r] = acc[r][b];
-        float v = warp_reduce8(col, lane);
-        if ((lane & 3) == 0) red[warp][reduced_row_of_lane(lane)][b] = v;
-    }
-    __syncthreads();
-    // Fixed-order sum over warps: thread t < 8*ncols owns (row, column).
-    const int row0 = rt * 8;
-    if (gridDim.y == 1) {
-        if (threadIdx.x < 8 * NB) {
-            int r = threadIdx.x / NB, b = threadIdx.x % NB;
-            int row = row0 + r;
-            if (b < ncols && row < L.out) {
-                float v = 0.f;
-#pragma unroll
-                for (int w = 0; w < kWarps; ++w) v += red[w][r][b];
-                float sc = scales ? __half2float(__ushort_as_half(scales[row])) : 1.f;
-                y[(size_t)row * batch + col0 + b] = __half_as_ushort(__float2half_rn(sc * v));
-            }
-        }
-        return;
-    }
-    if (threadIdx.x < 8 * NB) {
-        int r = threadIdx.x / NB, b = threadIdx.x % NB;
-        if (b < ncols) {
-            float v = 0.f;
-#pragma unroll
-            for (int w = 0; w < kWarps; ++w) v += red[w][r][b];
-            sk.partials[(size_t)blockIdx.y * L.rows8 * batch + (size_t)(row0 + r) * batch + col0 + b] = v;
-        }
-    }
-    // Column chunks of a batch > 4 are separate stream-ordered launches; the
-    // last CTA of each resets the counter before the next launch starts.
-    splitk_finish(L, sk, row0, 8, batch, col0, ncols, scales, y);
+    w[0] = c.x & 0xffff; w[1] = c.x >> 16; w[2] = c.y & 0xffff; w[3] = c.y >> 16;
+    w[4] = c.z & 0xffff; w[5] = c.z >> 16; w[6] = c.w & 0xffff; w[7] = c.w >> 16;
 }
 
 // ---------------------------------------------------------------------------
@@ -169,7 +96,10 @@ gemv_rowwarp_kernel(Geom L, const uint4 *__restrict__ packed, const uint4 *__res
 // A row's contribution from the block is then two table reads per group.
 // grid = (row ranges, group blocks); each CTA is one split of the K sum.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kThreads)
+constexpr int kLutWarps = 8;
+constexpr int kLutMaxTilesPerWarp = 12;  // row tiles per CTA <= 8 warps x 12
+
+__global__ void __launch_bounds__(kLutWarps * 32)
 gemv_2x8_lut_kernel(Geom L, const uint4 *__restrict__ packed, const uint4 *__restrict__ cb,
                     const uint16_t *__restrict__ scales, const uint16_t *__restrict__ x,
                     uint16_t *__restrict__ y, SplitK sk, int rt_per_cta)
@@ -178,37 +108,49 @@ gemv_2x8_lut_kernel(Geom L, const uint4 *__restrict__ packed, const uint4 *__res
     __shared__ uint4 xs[32];        // activations of the block's 32 groups
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gb = blockIdx.y;
+    const int rt0 = blockIdx.x * rt_per_cta;
+    const int rt1 = min(L.rtiles, rt0 + rt_per_cta);
+    // This warp's code chunks (row tiles rt0 + warp + 8j) are requested before
+    // the tables are built, so their HBM latency hides behind the build.
+    uint4 chunk[kLutMaxTilesPerWarp];
+#pragma unroll
+    for (int j = 0; j < kLutMaxTilesPerWarp; ++j) {
+        const int rt = rt0 + warp + j * kLutWarps;
+        chunk[j] = (rt < rt1) ? ldg_stream_v4(packed + (size_t)rt * L.gp + gb * 32 + lane) : make_uint4(0, 0, 0, 0);
+    }
+    grid_dependency_wait();  // x, y and the workspace follow the previous launch
+    grid_launch_dependents();
     if (threadIdx.x < 32) {
-        int g = gb * 32 + threadIdx.x;
+        const int g = gb * 32 + threadIdx.x;
         xs[threadIdx.x] = (g < L.G) ? ldg_nc_v4(x + (size_t)g * 8) : make_uint4(0, 0, 0, 0);
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < 2 * 256 * 32; e += kThreads) {
+    for (int e = threadIdx.x; e < 2 * 256 * 32; e += kLutWarps * 32) {
         const int l = e & 31;
         const int kc = e >> 5;  // k*256 + c
         lut[e] = dot8(ldg_nc_v4(cb + kc), xs[l], 0.f);
     }
     __syncthreads();
-    const int rt0 = blockIdx.x * rt_per_cta;
-    const int rt1 = min(L.rtiles, rt0 + rt_per_cta);
     const float *lut0 = lut + lane;
     const float *lut1 = lut + 256 * 32 + lane;
     float *part = sk.partials + (size_t)gb * L.rows8;
-    for (int rt = rt0 + warp; rt < rt1; rt += kWarps) {
-        const uint4 chunk = ldg_stream_v4(packed + (size_t)rt * L.gp + gb * 32 + lane);
-        const uint32_t v[4] = {chunk.x, chunk.y, chunk.z, chunk.w};
+#pragma unroll
+    for (int j = 0; j < kLutMaxTilesPerWarp; ++j) {
+        const int rt = rt0 + warp + j * kLutWarps;
+        if (rt >= rt1) break;
+        const uint32_t v[4] = {chunk[j].x, chunk[j].y, chunk[j].z, chunk[j].w};
         float acc[8];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             acc[2 * i] = lut0[(v[i] & 0xff) * 32] + lut1[((v[i] >> 8) & 0xff) * 32];
             acc[2 * i + 1] = lut0[((v[i] >> 16) & 0xff) * 32] + lut1[(v[i] >> 24) * 32];
         }
-        float r = warp_reduce8(acc, lane);
+        const float r = warp_reduce8(acc, lane);
         if ((lane & 3) == 0) {
-            int row = rt * 8 + reduced_row_of_lane(lane);
+            const int row = rt * 8 + reduced_row_of_lane(lane);
             if (gridDim.y == 1) {
                 if (row < L.out) {
-                    float sc = scales ? __half2float(__ushort_as_half(scales[row])) : 1.f;
+                    const float sc = scales ? __half2float(__ushort_as_half(scales[row])) : 1.f;
                     y[row] = __half_as_ushort(__float2half_rn(sc * r));
                 }
             } else {
@@ -217,7 +159,236 @@ gemv_2x8_lut_kernel(Geom L, const uint4 *__restrict__ packed, const uint4 *__res
         }
     }
     if (gridDim.y == 1) return;
-    splitk_finish(L, sk, rt0 * 8, (rt1 - rt0) * 8, 1, 0, 1, scales, y);
+    splitk_finish(L, sk, rt0 * 8, (rt1 - rt0) * 8, 1, scales, y);
+}
+
+// ---------------------------------------------------------------------------
+// Small-batch product on the tensor cores (any batch for 1x16, batch 2..16
+// for 2x8).
+//
+// CTA = 128 rows x one split of the K range, 128 threads.  Per stage of 64
+// input features (8 groups) thread t owns code chunk (row tile t/8, group
+// t%8) of the 128 x 64 A tile (128-byte swizzle, K-major):
+//  * 1x16: the chunk's 8 codewords are the weights; they are copied straight
+//    from the L2-resident codebook into the A tile with 16-byte cp.async, so
+//    gathers of several stages are in flight without holding registers;
+//  * 2x8: the two codewords per weight group are read from the codebooks in
+//    shared memory and summed with binary16 adds (one rounding), then stored.
+// x rows of the stage go to the B tile (MN-major, 32-byte swizzle: 64 rows
+// of 16 batch columns, zero-padded).  A ring of kTcRing stage buffers; the
+// MMAs of stage i are issued kTcLag stages after its copies, by thread 0:
+// four tcgen05.mma (M = 128, N = 16, K = 16) into an fp32 accumulator in
+// tensor memory, committed to the buffer's mbarrier, which the producer
+// waits on (bounded) before refilling that buffer.
+// ---------------------------------------------------------------------------
+constexpr int kTcThreads = 128;
+constexpr int kTcBM = 128;
+constexpr int kTcN = 16;
+// ring depth and copy-to-MMA lag: deep for the asynchronous 1x16 gathers,
+// short for the synchronous 2x8 decode
+template <int K> struct TcRing;
+template <> struct TcRing<1> { static constexpr int depth = 5, lag = 3; };
+template <> struct TcRing<2> { static constexpr int depth = 3, lag = 1; };
+constexpr int kTcTileA = kTcBM * 64 * 2;  // 16 KiB
+constexpr int kTcTileB = 64 * 32;         // 2 KiB: 64 rows x 16 columns
+constexpr int kTcXSlot = 64 * 16 * 2;     // raw x rows of one stage, batch <= 16
+constexpr int kTcTmemCols = 32;
+
+template <int K>
+__global__ void __launch_bounds__(kTcThreads)
+gemv_tc_kernel(Geom L, const uint4 *__restrict__ packed, const uint4 *__restrict__ cb,
+               const uint16_t *__restrict__ scales, const uint16_t *__restrict__ x, int batch,
+               uint16_t *__restrict__ y, SplitK sk, void *ws, int stages_per_split)
+{
+    constexpr int kTcRing = TcRing<K>::depth, kTcLag = TcRing<K>::lag;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    uint8_t *smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+    uint8_t *tileA = smem;                                  // [ring][16 KiB]
+    uint8_t *tileB = smem + kTcRing * kTcTileA;             // [ring][2 KiB]
+    uint8_t *xring = tileB + kTcRing * kTcTileB;            // [ring][2 KiB] raw x rows
+    uint4 *scb = reinterpret_cast<uint4 *>(xring + kTcRing * kTcXSlot);  // 2x8 codebooks
+    uint64_t *bars = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(scb) + (K == 2 ? 512 * 16 : 0));
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + kTcRing);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int m0 = blockIdx.x * kTcBM;
+    const int nst = (L.G + 7) / 8;  // 64-feature stages
+    const int s0 = blockIdx.y * stages_per_split;
+    const int s1 = min(nst, s0 + stages_per_split);
+    const int nloc = max(0, s1 - s0);
+
+    if (K == 1 && tid == 0) prefetch_table_share(cb, 65536u * 16u);
+    if (K == 2)
+        for (int i = tid; i < 512; i += kTcThreads) scb[i] = cb[i];
+    if (tid == 0) {
+        for (int s = 0; s < kTcRing; ++s) mbar_init(&bars[s], 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) tmem_alloc(tmem_slot, kTcTmemCols);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t idesc = make_idesc(kTcBM, kTcN, true);
+
+    const int rt_l = tid >> 3, gi = tid & 7;     // A role
+    const int rt = (m0 >> 3) + rt_l;
+    const int kr = tid >> 1, hb = tid & 1;        // B role: feature row, 8-column half
+    const bool rows_live = rt < L.rtiles;
+
+    // code chunks are loaded kCodeAhead stages ahead (a register ring), so
+    // that a stage's codeword gathers never wait on an HBM round trip
+    constexpr int kCodeAhead = 4;
+    uint4 code_ring[kCodeAhead];
+#pragma unroll
+    for (int q = 0; q < kCodeAhead; ++q) {
+        const int g = (s0 + q) * 8 + gi;
+        code_ring[q] = (q < nloc && rows_live && g < L.G) ? ldg_stream_v4(packed + (size_t)rt * L.gp + g)
+                                                          : make_uint4(0, 0, 0, 0);
+    }
+
+    const bool x_direct = (batch == 16 || batch == 8);
+    // everything above touched weights only; x, y and the workspace may be
+    // written by the previous launch on the stream
+    grid_dependency_wait();
+    grid_launch_dependents();
+    bool ok = true;
+    // stage loop unrolled by the code-ring depth so every ring index is static
+    for (int i0 = 0; ok && i0 < nloc + kTcLag; i0 += kCodeAhead) {
+#pragma unroll
+        for (int u = 0; u < kCodeAhead; ++u) {
+            const int i = i0 + u;
+            if (!ok || i >= nloc + kTcLag) break;
+            // ---- produce stage i ------------------------------------------------
+            if (i < nloc) {
+                const int s = s0 + i, buf = i % kTcRing;
+                if (i >= kTcRing) {  // buffer is free once the MMAs of stage i - ring completed
+                    const bool got = mbar_wait_ns(&bars[buf], ((i - kTcRing) / kTcRing) & 1, kWaitNs);
+                    if (!__syncthreads_and(got)) ok = false;
+                }
+                if (!ok) break;
+                const uint4 code = code_ring[u];
+                const bool live = rows_live && s * 8 + gi < L.G;
+                {
+                    const int g = (s + kCodeAhead) * 8 + gi;
+                    code_ring[u] = (i + kCodeAhead < nloc && rows_live && g < L.G)
+                                       ? ldg_stream_v4(packed + (size_t)rt * L.gp + g)
+                                       : make_uint4(0, 0, 0, 0);
+                }
+                uint8_t *A = tileA + buf * kTcTileA;
+                uint32_t wd[8];
+                unpack8(code, wd);
+                if (K == 1) {
+                    const uint32_t a0 = smem_u32(A);
+#pragma unroll
+                    for (int r = 0; r < 8; ++r)
+                        cp_async16(a0 + sw128(rt_l * 8 + r, gi), live ? (const void *)(cb + wd[r]) : (const void *)cb,
+                                   live ? 16u : 0u);
+                } else {
+#pragma unroll
+                    for (int r = 0; r < 8; ++r) {
+                        const uint4 v = live ? add_round_h8(scb[wd[r] & 0xff], scb[256 + (wd[r] >> 8)])
+                                             : make_uint4(0, 0, 0, 0);
+                        *reinterpret_cast<uint4 *>(A + sw128(rt_l * 8 + r, gi)) = v;
+                    }
+                }
+                // x rows k of this stage: columns 8*hb .. 8*hb+7 straight into
+                // the B tile when a row is 16 or 32 bytes, else the raw rows
+                // (64*batch*2 contiguous bytes) into the stage's x slot
+                if (x_direct) {
+                    uint8_t *Bt = tileB + buf * kTcTileB;
+                    const int k = s * 64 + kr, n0 = hb * 8;
+                    const uint32_t bdst = smem_u32(Bt) + sw32(kr, hb);
+                    const bool in = k < L.in && n0 < batch;
+                    cp_async16(bdst, in ? (const void *)(x + (size_t)k * batch + n0) : (const void *)x, in ? 16u : 0u);
+                } else if (tid < 8 * batch) {
+                    const int valid = max(0, min(64, L.in - s * 64)) * batch * 2;
+                    const int nb = max(0, min(16, valid - tid * 16));
+                    const uint8_t *src = reinterpret_cast<const uint8_t *>(x + (size_t)s * 64 * batch) + tid * 16;
+                    cp_async16(smem_u32(xring + buf * kTcXSlot) + tid * 16, nb > 0 ? (const void *)src : (const void *)x,
+                               (uint32_t)nb);
+                }
+            }
+            cp_async_commit();  // one group per iteration (empty in the drain)
+            // ---- consume stage j = i - lag: its copies are complete ----------------
+            const int j = i - kTcLag;
+            if (j >= 0) {
+                cp_async_wait<TcRing<K>::lag>();
+                if (!x_direct) {
+                    // every thread's copies of stage j are complete: build the
+                    // B tile rows from the stage's raw x slot
+                    __syncthreads();
+                    const uint16_t *xs = reinterpret_cast<const uint16_t *>(xring + (j % kTcRing) * kTcXSlot);
+                    const int n0 = hb * 8;
+                    uint16_t h[8];
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) h[q] = (n0 + q < batch) ? xs[kr * batch + n0 + q] : (uint16_t)0;
+                    *reinterpret_cast<uint4 *>(tileB + (j % kTcRing) * kTcTileB + sw32(kr, hb)) =
+                        make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16), h[4] | (h[5] << 16), h[6] | (h[7] << 16));
+                }
+                fence_proxy_async_smem();
+                __syncthreads();
+                if (tid == 0) {
+                    tc_fence_after();
+                    const int buf = j % kTcRing;
+                    const uint32_t a0 = smem_u32(tileA + buf * kTcTileA);
+                    const uint32_t b0 = smem_u32(tileB + buf * kTcTileB);
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks) {
+                        const uint64_t ad = smem_desc_sw128(a0 + ks * 32, 16, 1024);
+                        const uint64_t bd = smem_desc(b0 + ks * 512, kTcTileB, 256, kSwizzle32B);
+                        mma_f16_ss(tmem, ad, bd, idesc, (j > 0 || ks > 0) ? 1u : 0u);
+                    }
+                    mma_commit(&bars[buf]);
+                }
+            }
+        }
+    }
+    cp_async_wait<0>();
+    if (ok && nloc > 0) {
+        const int last = nloc - 1;
+        ok = __syncthreads_and(mbar_wait_ns(&bars[last % kTcRing], (last / kTcRing) & 1, kWaitNs));
+    } else {
+        ok = __syncthreads_and(ok);
+    }
+    if (!ok) {
+        if (tid == 0) record_status(ws, AQ_ERR_TIMEOUT);
+        // drain whatever MMAs were issued (bounded), so tensor memory is idle
+        for (int q = max(0, nloc - kTcRing); q < nloc; ++q)
+            mbar_wait_ns(&bars[q % kTcRing], (q / kTcRing) & 1, kWaitNs);
+    }
+    tc_fence_after();
+    const int row = m0 + warp * 32 + lane;
+    if (ok) {
+        float v[16];
+        if (nloc > 0) {
+            tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16), v);
+        } else {
+#pragma unroll
+            for (int n = 0; n < 16; ++n) v[n] = 0.f;
+        }
+        if (row < L.out) {
+            if (gridDim.y == 1) {
+                const float sc = scales ? __half2float(__ushort_as_half(scales[row])) : 1.f;
+#pragma unroll
+                for (int n = 0; n < 16; ++n)
+                    if (n < batch)
+                        y[(size_t)row * batch + n] = __half_as_ushort(__float2half_rn(sc * v[n]));
+            } else {
+                float *p = sk.partials + (size_t)blockIdx.y * L.rows8 * batch + (size_t)row * batch;
+#pragma unroll
+                for (int n = 0; n < 16; ++n)
+                    if (n < batch) p[n] = v[n];
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, kTcTmemCols);
+    // arrive even after a timeout so the counters stay consistent (the
+    // status word already tells the caller the output is incomplete)
+    if (gridDim.y > 1) splitk_finish(L, sk, m0, kTcBM, batch, scales, y);
 }
 
 }  // namespace aqk
@@ -227,13 +398,13 @@ using namespace aqk;
 
 namespace {
 
-enum Path { kRowWarp = 0, kLut2x8 = 1 };
+enum Path { kLut2x8 = 1, kTensor = 2 };
 
 struct GemvPlan {
     Path path;
-    int ks;             // splits of the group sum (grid.y)
-    int gbs_per_split;  // group blocks per split (row-warp path)
-    int rt_per_cta;     // row tiles per CTA
+    int ks;          // splits of the group sum (grid.y)
+    int per_split;   // group blocks (LUT: 1) or 64-feature stages (tensor) per split
+    int rt_per_cta;  // row tiles per CTA (LUT path)
     int grid_x;
     size_t ws_bytes;
 };
@@ -248,26 +419,64 @@ GemvPlan plan_gemv(const Geom &g, int batch)
     if (batch == 1 && g.K == 2) {
         p.path = kLut2x8;
         p.ks = g.gblocks;
-        // enough rows per CTA to amortise the 16K-entry table, ~300 CTAs
-        long pairs = (long)g.rtiles * g.gblocks;
-        int rt = (int)((pairs + 299) / 300);
+        const long pairs = (long)g.rtiles * g.gblocks;
+        int rt = (int)((pairs + 299) / 300);  // ~300 CTAs, enough rows to amortise the table
         rt = max(rt, 8);
+        rt = min(rt, kLutWarps * kLutMaxTilesPerWarp);
         rt = min(rt, g.rtiles);
         p.rt_per_cta = rt;
         p.grid_x = (g.rtiles + rt - 1) / rt;
-        p.gbs_per_split = 1;
+        p.per_split = 1;
     } else {
-        p.path = kRowWarp;
-        p.rt_per_cta = 1;
-        p.grid_x = g.rtiles;
-        int ks = (512 + g.rtiles - 1) / g.rtiles;
-        ks = max(1, min(ks, min(8, g.gblocks)));
-        p.gbs_per_split = (g.gblocks + ks - 1) / ks;
-        p.ks = (g.gblocks + p.gbs_per_split - 1) / p.gbs_per_split;
+        p.path = kTensor;
+        const int mtiles = (g.out + kTcBM - 1) / kTcBM;
+        const int nst = (g.G + 7) / 8;
+        // ~1024 CTAs at batch 1 (short tail, many gathers in flight), fewer
+        // splits as the batch grows (split-K partials scale with the batch)
+        const int target = 1024 / max(1, batch / 2);
+        int ks = (target + mtiles - 1) / mtiles;
+        ks = max(1, min(ks, (nst + 7) / 8));  // at least 8 stages per CTA: the ring fills
+        p.per_split = (nst + ks - 1) / ks;
+        p.ks = (nst + p.per_split - 1) / p.per_split;
+        p.grid_x = mtiles;
+        p.rt_per_cta = kTcBM / 8;
     }
     p.ws_bytes = kWsHeader + align16(sizeof(unsigned) * (size_t)p.grid_x);
     if (p.ks > 1) p.ws_bytes += (size_t)p.ks * g.rows8 * batch * sizeof(float);
     return p;
+}
+
+// ring of (A tile, B tile, x slot) + codebooks + barriers and TMEM slot
+template <int K>
+constexpr int tc_smem_bytes()
+{
+    return 1024 + TcRing<K>::depth * (kTcTileA + kTcTileB + kTcXSlot) + (K == 2 ? 512 * 16 : 0) + 128;
+}
+
+template <class Kern>
+cudaError_t set_smem(Kern k, int bytes)
+{
+    return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+// Launch with programmatic stream serialisation: the kernel's weight-only
+// prologue may overlap the tail of the previous kernel on the stream; the
+// kernel itself waits (griddepcontrol.wait) before touching x, y or the
+// workspace.
+template <class... KArgs, class... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, int smem, cudaStream_t s, Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
 }
 
 }  // namespace
@@ -286,43 +495,37 @@ cudaError_t launch_gemv(const Geom &g, const void *packed, const uint16_t *cb,
                                             align16(sizeof(unsigned) * (size_t)p.grid_x));
     const uint4 *pk = reinterpret_cast<const uint4 *>(packed);
     const uint4 *c = reinterpret_cast<const uint4 *>(cb);
-    dim3 grid(p.grid_x, p.ks);
-    if (p.path == kLut2x8) {
+    const dim3 grid(p.grid_x, p.ks);
+    cudaError_t e = cudaSuccess;
+    switch (p.path) {
+    case kLut2x8: {
         const int smem = 2 * 256 * 32 * sizeof(float);
-        static bool attr_set = false;  // idempotent, benign race
-        if (!attr_set) {
-            cudaError_t e = cudaFuncSetAttribute(gemv_2x8_lut_kernel,
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-            if (e != cudaSuccess) return e;
-            attr_set = true;
-        }
-        gemv_2x8_lut_kernel<<<grid, kThreads, smem, s>>>(g, pk, c, scales, x, y, sk, p.rt_per_cta);
-        return cudaGetLastError();
-    }
-    if (batch == 1) {
-        if (g.K == 1)
-            gemv_rowwarp_kernel<1, 1><<<grid, kThreads, 0, s>>>(g, pk, c, scales, x, 1, 0, y, sk, p.gbs_per_split);
-        else
-            gemv_rowwarp_kernel<2, 1><<<grid, kThreads, 0, s>>>(g, pk, c, scales, x, 1, 0, y, sk, p.gbs_per_split);
-        return cudaGetLastError();
-    }
-    const int nb = batch == 2 ? 2 : 4;
-    for (int col0 = 0; col0 < batch; col0 += nb) {
-        if (g.K == 1) {
-            if (nb == 2)
-                gemv_rowwarp_kernel<1, 2><<<grid, kThreads, 0, s>>>(g, pk, c, scales, x, batch, col0, y, sk, p.gbs_per_split);
-            else
-                gemv_rowwarp_kernel<1, 4><<<grid, kThreads, 0, s>>>(g, pk, c, scales, x, batch, col0, y, sk, p.gbs_per_split);
-        } else {
-            if (nb == 2)
-                gemv_rowwarp_kernel<2, 2><<<grid, kThreads, 0, s>>>(g, pk, c, scales, x, batch, col0, y, sk, p.gbs_per_split);
-            else
-                gemv_rowwarp_kernel<2, 4><<<grid, kThreads, 0, s>>>(g, pk, c, scales, x, batch, col0, y, sk, p.gbs_per_split);
-        }
-        cudaError_t e = cudaGetLastError();
+        e = set_smem(gemv_2x8_lut_kernel, smem);
         if (e != cudaSuccess) return e;
+        e = launch_pdl(gemv_2x8_lut_kernel, grid, dim3(kLutWarps * 32), smem, s, g, pk, c, scales, x, y, sk,
+                       p.rt_per_cta);
+        if (e != cudaSuccess) return e;
+        break;
     }
-    return cudaSuccess;
+    case kTensor:
+        if (g.K == 1) {
+            const int smem = tc_smem_bytes<1>();
+            e = set_smem(gemv_tc_kernel<1>, smem);
+            if (e != cudaSuccess) return e;
+            e = launch_pdl(gemv_tc_kernel<1>, grid, dim3(kTcThreads), smem, s, g, pk, c, scales, x, batch, y, sk, ws,
+                           p.per_split);
+            if (e != cudaSuccess) return e;
+        } else {
+            const int smem = tc_smem_bytes<2>();
+            e = set_smem(gemv_tc_kernel<2>, smem);
+            if (e != cudaSuccess) return e;
+            e = launch_pdl(gemv_tc_kernel<2>, grid, dim3(kTcThreads), smem, s, g, pk, c, scales, x, batch, y, sk, ws,
+                           p.per_split);
+            if (e != cudaSuccess) return e;
+        }
+        break;
+    }
+    return cudaGetLastError();
 }
 
 }  // namespace aqh

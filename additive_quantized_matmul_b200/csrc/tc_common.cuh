@@ -1,0 +1,187 @@
+// tcgen05 / TMEM / shared-memory-descriptor helpers (sm_100a inline PTX).
+//
+// Descriptor and instruction formats follow the PTX ISA for tcgen05.mma
+// (shared-memory matrix descriptor: start >> 4 in bits 0-13, leading byte
+// offset >> 4 in 16-29, stride byte offset >> 4 in 32-45, version 1 in
+// 46-47, swizzle mode in 61-63; instruction descriptor for kind::f16: D
+// format bits 4-5, A/B formats 7-9/10-12, A/B major bits 15/16, N >> 3 in
+// 17-22, M >> 4 in 24-28).
+#pragma once
+
+#include "aq_common.cuh"
+
+namespace aqk {
+
+constexpr uint64_t kWaitNs = 1000000000ull; // 1 s per wait
+
+// ---- PTX wrappers -----------------------------------------------------------
+
+__device__ __forceinline__ uint64_t globaltimer()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Wait for a phase of an mbarrier for at most `ns` nanoseconds.
+__device__ __forceinline__ bool mbar_wait_ns(uint64_t *bar, uint32_t parity, uint64_t ns)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer();
+    for (uint32_t i = 0; i < (1u << 30); ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (globaltimer() - t0 > ns) return false;
+    }
+    return false;
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_alloc(uint32_t *dst_smem, uint32_t ncols)
+{
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                 ::"r"(smem_u32(dst_smem)), "r"(ncols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::);
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols));
+}
+
+// D[tmem] (+)= A[smem desc] * B[smem desc]; accumulate selects D += vs D =.
+__device__ __forceinline__ void mma_f16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                           uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
+}
+
+// Arrive (once) on `bar` when every tcgen05.mma issued so far by this thread
+// has completed.
+__device__ __forceinline__ void mma_commit(uint64_t *bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 ::"r"(smem_u32(bar)) : "memory");
+}
+
+// 32 lanes x 16 consecutive fp32 columns of tensor memory -> 16 registers.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float v[16])
+{
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Shared-memory matrix descriptor (sm_100 layout): start address >> 4 in
+// bits 0-13, leading byte offset >> 4 in 16-29, stride byte offset >> 4 in
+// 32-45, descriptor version 1 in bits 46-47, swizzle mode in 61-63
+// (2 = 128-byte swizzle, 6 = 32-byte swizzle).
+constexpr uint32_t kSwizzle128B = 2;
+constexpr uint32_t kSwizzle32B = 6;
+
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo, uint32_t mode)
+{
+    uint64_t d = 0;
+    d |= (uint64_t)((addr >> 4) & 0x3fff);
+    d |= (uint64_t)((lbo >> 4) & 0x3fff) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3fff) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)(mode & 7) << 61;
+    return d;
+}
+
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr, uint32_t lbo, uint32_t sbo)
+{
+    return smem_desc(addr, lbo, sbo, kSwizzle128B);
+}
+
+// Instruction descriptor for kind::f16: fp32 accumulator (bits 4-5 = 1),
+// binary16 A and B (formats 0), A K-major (bit 15 = 0), B MN-major
+// (bit 16 = 1) unless b_mn_major is false, N >> 3 in bits 17-22, M >> 4 in
+// bits 24-28.
+__host__ __device__ constexpr uint32_t make_idesc(int M, int N, bool b_mn_major = true)
+{
+    return (1u << 4) | (0u << 7) | (0u << 10) | (0u << 15) | ((b_mn_major ? 1u : 0u) << 16) |
+           ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// Byte offset of 16-byte chunk c (0..7) of row r in a 128-byte-swizzled
+// tile of 128-byte rows (rows 8-aligned into 1024-byte atoms).
+__device__ __forceinline__ uint32_t sw128(uint32_t row, uint32_t c)
+{
+    return row * 128u + ((c ^ (row & 7u)) << 4);
+}
+
+// Byte offset of 16-byte chunk c (0..1) of row r in a 32-byte-swizzled tile
+// of 32-byte rows (8-row, 256-byte atoms): address bit 4 ^= address bit 7.
+__device__ __forceinline__ uint32_t sw32(uint32_t row, uint32_t c)
+{
+    return row * 32u + ((c ^ ((row >> 2) & 1u)) << 4);
+}
+
+// 16-byte asynchronous global -> shared copy (L2 only, no L1 allocation).
+// src_bytes = 0 writes 16 zero bytes without reading the source.
+__device__ __forceinline__ void cp_async16(uint32_t dst_smem, const void *src, uint32_t src_bytes)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst_smem), "l"(src), "r"(src_bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// Programmatic dependent launch: wait until the grids this launch depends
+// on have completed and their writes are visible (returns at once for an
+// ordinary launch), and allow the next dependent launch to start its
+// prologue.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Bulk prefetch of [p, p + bytes) into L2 (p and bytes multiples of 16).
+__device__ __forceinline__ void prefetch_l2_bulk(const void *p, uint32_t bytes)
+{
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+// Each CTA of the grid prefetches its share of a table into L2, so that the
+// table's first random reads hit L2 instead of queueing on DRAM sector misses.
+__device__ __forceinline__ void prefetch_table_share(const void *table, uint32_t bytes)
+{
+    const uint32_t ncta = gridDim.x * gridDim.y;
+    const uint32_t id = blockIdx.y * gridDim.x + blockIdx.x;
+    const uint32_t share = ((bytes + ncta - 1) / ncta + 255u) & ~255u;
+    const uint32_t off = id * share;
+    if (off < bytes) prefetch_l2_bulk(reinterpret_cast<const uint8_t *>(table) + off, min(share, bytes - off));
+}
+
+// 2-D tiled TMA load (no multicast) of box {c0.., c1..} into shared memory,
+// completing `bytes` on the mbarrier.  c0 is the innermost coordinate.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst_smem, const void *tmap, int c0, int c1, uint64_t *bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(dst_smem), "l"(tmap), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+        : "memory");
+}
+
+}  // namespace aqk

@@ -58,8 +58,10 @@ def measured_peaks() -> dict:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         d = json.load(open(p))
-        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"], "source": "measured"}
-    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
 # ---------------------------------------------------------------------------
@@ -230,85 +232,108 @@ def run_reference(args) -> None:
 # GPU arm
 # ---------------------------------------------------------------------------
 
-def count_graph_kernels(graph) -> int | None:
-    try:
-        from cuda.bindings import runtime as rt
-        g = graph.raw_cuda_graph()
-        err, _, n = rt.cudaGraphGetNodes(g, 0)
-        if int(err) != 0:
-            return None
-        err, nodes, n = rt.cudaGraphGetNodes(g, n)
-        kinds = [rt.cudaGraphNodeGetType(nd)[1] for nd in nodes]
-        return sum(1 for k in kinds if k == rt.cudaGraphNodeType.cudaGraphNodeTypeKernel)
-    except Exception:
-        return None
+def count_graph_kernels(graph) -> int:
+    """Kernel nodes in a captured graph (needs ``keep_graph=True``)."""
+    from cuda.bindings import runtime as rt
+    raw = graph.raw_cuda_graph()
+    g = raw if isinstance(raw, rt.cudaGraph_t) else rt.cudaGraph_t(init_value=int(raw))
+    err, _, n = rt.cudaGraphGetNodes(g, 0)
+    if int(err) != 0:
+        raise RuntimeError(f"cudaGraphGetNodes: {err}")
+    err, nodes, n = rt.cudaGraphGetNodes(g, n)
+    if int(err) != 0:
+        raise RuntimeError(f"cudaGraphGetNodes: {err}")
+    kernel = rt.cudaGraphNodeType.cudaGraphNodeTypeKernel
+    count = 0
+    for nd in nodes[:n]:
+        err, t = rt.cudaGraphNodeGetType(nd)
+        if int(err) == 0 and t == kernel:
+            count += 1
+    return count
+
+
+def flops(spec: LayerSpec, n: int) -> int:
+    return 2 * spec.out_features * spec.in_features * n
 
 
 def run_gpu(args) -> None:
     import torch
 
     import additive_quantized_matmul_b200 as aq
+    from aq_inputs import workload
 
     world, rank, local = dist_env()
     torch.cuda.set_device(local)
     dist = init_dist(world, "nccl")
     dev = torch.device("cuda", local)
-    desc = aq.LayerDesc.make(SPEC.out_features, SPEC.in_features, SPEC.num_codebooks, SPEC.nbits)
+    wl = workload(args.workload)
+    op = "gemm" if args.workload == "llama2-7b-prefill" else "gemv"
+    peaks = measured_peaks()
 
-    layer_bytes = alg_bytes(SPEC, 0)
-    nlayers = args.layers or max(8, int(3 * L2_BYTES / layer_bytes) + 1)
-    # ---- build the rotation set of distinct layers (seeded per rank) --------
-    layers = []
-    for i in range(nlayers):
-        L = make_layer(SPEC, (SEED, rank, i))  # seeded per rank and layer
-        codes = torch.from_numpy(L.codes.view(np.int16)).to(dev)
-        packed = torch.empty(aq.aq_packed_codes_bytes(desc), dtype=torch.uint8, device=dev)
-        aq.aq_pack_codes(desc, codes, packed)
-        cb = torch.from_numpy(L.codebooks.view(np.int16)).to(dev)
-        sc = torch.from_numpy(L.scales.view(np.int16)).to(dev)
-        layers.append((packed, cb, sc))
+    # ---- units: one (layer shape, batch) product kind each, over a rotation
+    #      set of copies at distinct addresses (> 3x L2 per shape) -----------
+    units = []
+    for si, (tag, spec) in enumerate(wl["layers"]):
+        desc = aq.LayerDesc.make(spec.out_features, spec.in_features, spec.num_codebooks, spec.nbits)
+        L = make_layer(spec, (wl["seed"], rank, si))  # seeded per rank and shape
+        codes = torch.from_numpy(L.codes.view(np.int16) if spec.nbits > 8 else L.codes).to(dev)
+        packed0 = torch.empty(aq.aq_packed_codes_bytes(desc), dtype=torch.uint8, device=dev)
+        aq.aq_pack_codes(desc, codes, packed0)
+        cb0 = torch.from_numpy(L.codebooks.view(np.int16)).to(dev)
+        sc0 = torch.from_numpy(L.scales.view(np.int16)).to(dev)
         del codes, L
-    xs = {b: torch.from_numpy(make_activations(SPEC.in_features, b, (SEED, rank, b)).view(np.int16)).to(dev)
-          for b in BATCHES}
-    ys = {b: [torch.empty(SPEC.out_features * b, dtype=torch.int16, device=dev) for _ in range(nlayers)]
-          for b in BATCHES}
-    ws = {b: torch.zeros(aq.aq_gemv_workspace_bytes(desc, b), dtype=torch.uint8, device=dev)
-          for b in BATCHES}
+        lb = alg_bytes(spec, 0)
+        ncopies = args.layers or max(3 if op == "gemm" else 4, int(3 * L2_BYTES / lb) + 1)
+        copies = [(packed0.clone(), cb0.clone(), sc0.clone()) for _ in range(ncopies)]
+        del packed0, cb0, sc0
+        for n in wl["n"]:
+            x = torch.from_numpy(make_activations(spec.in_features, n, (wl["seed"], rank, si, n)).view(np.int16)).to(dev)
+            nbytes = (aq.aq_gemm_workspace_bytes(desc, n) if op == "gemm" else aq.aq_gemv_workspace_bytes(desc, n))
+            units.append({
+                "tag": tag, "spec": spec, "n": n, "desc": desc, "copies": copies, "x": x,
+                "ys": [torch.empty(spec.out_features * n, dtype=torch.int16, device=dev) for _ in range(ncopies)],
+                "ws": torch.zeros(max(nbytes, 16), dtype=torch.uint8, device=dev),
+                # two events per group of same-shape launches (event nodes between
+                # every launch would add their own cost to each measurement)
+                "evs": [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)],
+            })
     torch.cuda.synchronize()
-
     stream = torch.cuda.Stream(device=dev)
-    # events around every product inside the graph (external record nodes)
-    evs = {b: [torch.cuda.Event(enable_timing=True, external=True) for _ in range(nlayers + 1)]
-           for b in BATCHES}
+
+    def call(u, i, s):
+        packed, cb, sc = u["copies"][i]
+        if op == "gemm":
+            aq.aq_gemm(u["desc"], packed, cb, sc, u["x"], u["n"], u["ys"][i], u["ws"], stream=s)
+        else:
+            aq.aq_gemv(u["desc"], packed, cb, sc, u["x"], u["n"], u["ys"][i], u["ws"], stream=s)
 
     def one_step(record: bool):
         s = torch.cuda.current_stream()
-        for b in BATCHES:
+        for u in units:
             if record:
-                evs[b][0].record(s)
-            for i, (packed, cb, sc) in enumerate(layers):
-                aq.aq_gemv(desc, packed, cb, sc, xs[b], b, ys[b][i], ws[b], stream=s)
-                if record:
-                    evs[b][i + 1].record(s)
+                u["evs"][0].record(s)
+            for i in range(len(u["copies"])):
+                call(u, i, s)
+            if record:
+                u["evs"][1].record(s)
 
-    # eager warm-up (also JIT-free: the library is AOT compiled)
     with torch.cuda.stream(stream):
-        one_step(False)
+        one_step(False)  # eager warm-up (the library is compiled ahead of time)
     torch.cuda.synchronize()
-    graph = torch.cuda.CUDAGraph()
+    graph = torch.cuda.CUDAGraph(keep_graph=True)
     with torch.cuda.graph(graph, stream=stream):
         one_step(True)
     launches_per_step = count_graph_kernels(graph)
+    graph.instantiate()
     torch.cuda.synchronize()
-
     for _ in range(max(args.warmup, 0)):
         graph.replay()
     torch.cuda.synchronize()
 
     t_start = torch.cuda.Event(enable_timing=True)
     t_stop = torch.cuda.Event(enable_timing=True)
-    gpu_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local]) \
-        if os.environ.get("CUDA_VISIBLE_DEVICES", "").replace(",", "").isdigit() else local
+    cvd = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    gpu_index = int(cvd.split(",")[local]) if cvd.replace(",", "").isdigit() else local
     os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
     sampler = ClockSampler(gpu_index, os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv"))
     if dist is not None:
@@ -323,51 +348,66 @@ def run_gpu(args) -> None:
         torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
-    elapsed_ms = t_start.elapsed_time(t_stop)
-    elapsed_ms = max_over_ranks(elapsed_ms, dist, dev)
+    elapsed_ms = max_over_ranks(t_start.elapsed_time(t_stop), dist, dev)
+    status_ok = all(aq.aq_workspace_status(u["ws"]) == 0 for u in units)
 
-    # per-product durations from the last replay inside the timed region
-    per_b = {}
-    for b in BATCHES:
-        t = [evs[b][i].elapsed_time(evs[b][i + 1]) for i in range(nlayers)]
-        per_b[b] = {"us_per_call": 1e3 * float(np.mean(t)), "us_median": 1e3 * float(np.median(t))}
-    step_bytes = nlayers * sum(alg_bytes(SPEC, b) for b in BATCHES)
-    value = world * step_bytes * args.steps / (elapsed_ms * 1e-3) / 1e9
-    peaks = measured_peaks()
+    # average duration per launch of each group, from the last replay inside
+    # the timed region (events on the launching stream)
     kernels = []
-    for b in BATCHES:
-        us = per_b[b]["us_per_call"]
-        gbs = alg_bytes(SPEC, b) / (us * 1e-6) / 1e9
-        kernels.append({"batch": b, "us_per_layer": round(us, 3), "gbs": round(gbs, 1),
-                        "frac_hbm": round(gbs / peaks["hbm_gbs"], 4),
-                        "bytes_per_call": alg_bytes(SPEC, b)})
-    dom = max(kernels, key=lambda k: k["us_per_layer"])
-    roofline = {"bound": "hbm", "achieved": dom["gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": round(dom["gbs"] / peaks["hbm_gbs"], 4), "traffic": None,
-                "kernel": f"aq_gemv batch {dom['batch']} (4096x4096 1x16)",
-                "peak_source": f"{peaks['source']} hbm_gbs (MEASURED_PEAKS.json copy bandwidth)"}
+    step_bytes = step_flops = 0
+    for u in units:
+        us = 1e3 * u["evs"][0].elapsed_time(u["evs"][1]) / len(u["copies"])
+        nb, nf = alg_bytes(u["spec"], u["n"]), flops(u["spec"], u["n"])
+        step_bytes += nb * len(u["copies"])
+        step_flops += nf * len(u["copies"])
+        k = {"layer": u["tag"], "n": u["n"], "us_per_layer": round(us, 3),
+             "gbs": round(nb / (us * 1e-6) / 1e9, 1), "tflops": round(nf / (us * 1e-6) / 1e12, 2),
+             "bytes_per_call": nb, "copies": len(u["copies"]), "total_us": us * len(u["copies"])}
+        k["frac_hbm"] = round(k["gbs"] / peaks["hbm_gbs"], 4)
+        k["frac_tensor"] = round(k["tflops"] / peaks["bf16_tflops_sustained"], 4)
+        kernels.append(k)
+    dom = max(kernels, key=lambda k: k["total_us"])
+    if op == "gemm":
+        value = world * step_flops * args.steps / (elapsed_ms * 1e-3) / 1e12
+        unit = "TFLOP/s"
+        roofline = {"bound": "tensor", "achieved": dom["tflops"], "peak": peaks["bf16_tflops_sustained"],
+                    "unit": "TFLOP/s", "frac": dom["frac_tensor"], "traffic": None,
+                    "kernel": f"aq_gemm {dom['layer']} T={dom['n']}",
+                    "peak_source": f"{peaks['source']} bf16_tflops_sustained (cuBLAS bf16; fp16 tcgen05 has the same rate)"}
+    else:
+        value = world * step_bytes * args.steps / (elapsed_ms * 1e-3) / 1e9
+        unit = "GB/s"
+        roofline = {"bound": "hbm", "achieved": dom["gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": dom["frac_hbm"], "traffic": None,
+                    "kernel": f"aq_gemv {dom['layer']} batch {dom['n']}",
+                    "peak_source": f"{peaks['source']} hbm_gbs (STREAM-style copy)"}
+    for k in kernels:
+        del k["total_us"]
 
     # ---- end-to-end through the public API with host buffers ----------------
     e2e = None
     if not args.skip_e2e:
-        hx = {b: torch.empty((nlayers, SPEC.in_features * b), dtype=torch.int16).pin_memory() for b in BATCHES}
-        hy = {b: torch.empty((nlayers, SPEC.out_features * b), dtype=torch.int16).pin_memory() for b in BATCHES}
-        for b in BATCHES:
-            hx[b].copy_(xs[b].cpu().reshape(1, -1).expand(nlayers, -1))
-        dx = {b: torch.empty((nlayers, SPEC.in_features * b), dtype=torch.int16, device=dev) for b in BATCHES}
-        dy = {b: torch.empty((nlayers, SPEC.out_features * b), dtype=torch.int16, device=dev) for b in BATCHES}
-        h2d = sum(hx[b].numel() * 2 for b in BATCHES)
-        d2h = sum(hy[b].numel() * 2 for b in BATCHES)
+        hx = [torch.empty((len(u["copies"]), u["x"].numel()), dtype=torch.int16).pin_memory() for u in units]
+        hy = [torch.empty((len(u["copies"]), u["ys"][0].numel()), dtype=torch.int16).pin_memory() for u in units]
+        dx = [torch.empty(h.shape, dtype=torch.int16, device=dev) for h in hx]
+        dy = [torch.empty(h.shape, dtype=torch.int16, device=dev) for h in hy]
+        for h, u in zip(hx, units):
+            h.copy_(u["x"].cpu().reshape(1, -1).expand(h.shape[0], -1))
+        h2d = sum(h.numel() * 2 for h in hx)
+        d2h = sum(h.numel() * 2 for h in hy)
         e_steps = max(1, min(args.steps, args.e2e_steps))
 
         def e2e_step():
-            for b in BATCHES:
-                dx[b].copy_(hx[b], non_blocking=True)
-            for b in BATCHES:
-                for i, (packed, cb, sc) in enumerate(layers):
-                    aq.aq_gemv(desc, packed, cb, sc, dx[b][i], b, dy[b][i], ws[b])
-            for b in BATCHES:
-                hy[b].copy_(dy[b], non_blocking=True)
+            for d, h in zip(dx, hx):
+                d.copy_(h, non_blocking=True)
+            for ui, u in enumerate(units):
+                for i, (packed, cb, sc) in enumerate(u["copies"]):
+                    if op == "gemm":
+                        aq.aq_gemm(u["desc"], packed, cb, sc, dx[ui][i], u["n"], dy[ui][i], u["ws"])
+                    else:
+                        aq.aq_gemv(u["desc"], packed, cb, sc, dx[ui][i], u["n"], dy[ui][i], u["ws"])
+            for h, d in zip(hy, dy):
+                h.copy_(d, non_blocking=True)
 
         e2e_step()
         torch.cuda.synchronize()
@@ -380,32 +420,36 @@ def run_gpu(args) -> None:
         e1.record()
         torch.cuda.synchronize()
         e_ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
-        e2e = {"value": round(world * step_bytes * e_steps / (e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+        tot = (step_flops / 1e12) if op == "gemm" else (step_bytes / 1e9)
+        e2e = {"value": round(world * tot * e_steps / (e_ms * 1e-3), 2), "unit": unit,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e_steps,
-               "api": "additive_quantized_matmul_b200.aq_gemv (C ABI via ctypes), eager"}
+               "api": "additive_quantized_matmul_b200 (C ABI via ctypes), eager, pinned host buffers"}
 
     cpu = None
-    if rank == 0 and world == 1 and not args.skip_cpu:
+    if rank == 0 and world == 1 and not args.skip_cpu and op == "gemv":
         cpu = cpu_baseline()
 
     if rank == 0:
+        spec0 = wl["layers"][0][1]
         line = {
-            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+            "metric": METRIC, "value": round(value, 2), "unit": unit, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(elapsed_ms / args.steps, 4), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f16", "accumulate": "f32",
             "data": "synthetic",
-            "config": {"workload": WORKLOAD, "layer": "4096x4096 1x16 g8 (2 bits/weight)",
-                       "batches": list(BATCHES), "layers_per_step": nlayers,
-                       "l2": f"inputs larger than L2: {nlayers} distinct layers, "
-                             f"{nlayers * layer_bytes / 1e6:.0f} MB of codes+codebooks per pass, "
-                             f"batch-major order (> 3x the 126 MB L2)",
+            "config": {"workload": args.workload,
+                       "layers": [f"{t} {s.scheme} g8" for t, s in wl["layers"]],
+                       "n": list(wl["n"]),
+                       "copies_per_shape": [len(u["copies"]) for u in units[::len(wl["n"])]],
+                       "l2": "inputs larger than L2: per shape, copies at distinct addresses whose "
+                             "bytes exceed 3x the 126 MB L2, visited in turn before any is re-read",
                        "parallelism": f"replicas x{world} (independent layers per rank)"},
-            "us_per_layer": {str(k["batch"]): k["us_per_layer"] for k in kernels},
             "kernels": kernels, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-            "clocks": sampler.summary(),
-            "gpu_launches": None if launches_per_step is None else launches_per_step * args.steps,
+            "clocks": sampler.summary(), "status_ok": status_ok,
+            "gpu_launches": launches_per_step * args.steps,
         }
+        if op == "gemv" and args.workload == WORKLOAD:
+            line["us_per_layer"] = {str(k["n"]): k["us_per_layer"] for k in kernels}
         print(json.dumps(line), flush=True)
     del graph
     if dist is not None:
@@ -418,7 +462,10 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--layers", type=int, default=0, help="rotation set size (0: > 3x L2)")
+    ap.add_argument("--workload", default=WORKLOAD,
+                    help="llama2-7b-1x16 (default), llama2-7b-mlp-2x8, llama2-70b-1x16, "
+                         "llama2-7b-prefill, tiny-2x8")
+    ap.add_argument("--layers", type=int, default=0, help="copies per shape (0: > 3x L2)")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--skip-cpu", action="store_true")
