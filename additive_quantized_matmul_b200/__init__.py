@@ -20,7 +20,8 @@ __all__ = [
     "AQError", "LayerDesc", "lib", "library_path", "aq_version", "aq_status_string",
     "aq_packed_codes_bytes", "aq_gemv_workspace_bytes", "aq_gemm_workspace_bytes",
     "aq_workspace_status", "aq_selftest_bounded_wait", "aq_pack_codes", "aq_unpack_codes",
-    "aq_dequant", "aq_gemv", "aq_gemm", "EXPORTED_SYMBOLS",
+    "aq_dequant", "aq_gemv", "aq_gemv_noalloc", "aq_gemm", "EXPORTED_SYMBOLS",
+    "GEMV_NOALLOC_SCRATCH_BYTES",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -35,8 +36,12 @@ STATUS_NAMES = {0: "AQ_OK", 1: "AQ_ERR_INVALID_ARG", 2: "AQ_ERR_UNSUPPORTED",
 EXPORTED_SYMBOLS = (
     "aq_status_string", "aq_version", "aq_packed_codes_bytes", "aq_gemv_workspace_bytes",
     "aq_gemm_workspace_bytes", "aq_workspace_status", "aq_selftest_bounded_wait",
-    "aq_pack_codes", "aq_unpack_codes", "aq_dequant", "aq_gemv", "aq_gemm",
+    "aq_pack_codes", "aq_unpack_codes", "aq_dequant", "aq_gemv", "aq_gemv_noalloc", "aq_gemm",
 )
+
+# AQ_GEMV_NOALLOC_SCRATCH_BYTES of include/aq.h: the fixed scratch behind
+# aq_gemv_noalloc.
+GEMV_NOALLOC_SCRATCH_BYTES = 4 << 20
 
 
 class AQError(RuntimeError):
@@ -63,7 +68,7 @@ def _load() -> ctypes.CDLL:
     if not os.path.exists(library_path):
         raise ImportError(
             f"{library_path} is missing: build it with "
-            "`python -m additive_quantized_matmul_b200.build` (nvcc, sm_100a)")
+            "`python additive_quantized_matmul_b200/build.py` (nvcc, sm_100a)")
     L = ctypes.CDLL(library_path)
     vp, sz, i32 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
     dp = ctypes.POINTER(LayerDesc)
@@ -80,6 +85,7 @@ def _load() -> ctypes.CDLL:
         "aq_dequant": ([dp, vp, vp, vp, vp, vp], i32),
         "aq_gemv": ([dp, vp, vp, vp, vp, i32, vp, vp, sz, vp], i32),
         "aq_gemm": ([dp, vp, vp, vp, vp, i32, vp, vp, sz, vp], i32),
+        "aq_gemv_noalloc": ([dp, vp, vp, vp, vp, i32, vp, vp], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -165,6 +171,14 @@ def aq_gemv(desc: LayerDesc, packed, codebooks, scales, x, batch: int, y, worksp
     _check("aq_gemv", lib.aq_gemv(ctypes.byref(desc), _ptr(packed), _ptr(codebooks), _ptr(scales),
                                   _ptr(x), batch, _ptr(y), _ptr(workspace), workspace_bytes,
                                   _stream(stream)))
+
+
+def aq_gemv_noalloc(desc: LayerDesc, packed, codebooks, scales, x, batch: int, y, stream=None) -> None:
+    """aq_gemv for callers that cannot allocate device memory: the split-K
+    scratch is a fixed array inside the library (see include/aq.h); calls
+    that overlap on the GPU must not be issued."""
+    _check("aq_gemv_noalloc", lib.aq_gemv_noalloc(ctypes.byref(desc), _ptr(packed), _ptr(codebooks),
+                                                  _ptr(scales), _ptr(x), batch, _ptr(y), _stream(stream)))
 
 
 def aq_gemm(desc: LayerDesc, packed, codebooks, scales, x, T: int, y, workspace,

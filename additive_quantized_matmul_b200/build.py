@@ -1,6 +1,7 @@
 """Build libaq_b200.so from csrc/*.cu for sm_100a (nvcc, in-tree).
 
-Usage: ``python -m additive_quantized_matmul_b200.build`` or ``build()``.
+Usage: ``python additive_quantized_matmul_b200/build.py [--force]`` (run by
+path: importing the package loads the library this script builds).
 Rebuilds only when a source or header is newer than the library.
 """
 from __future__ import annotations

@@ -147,6 +147,26 @@ aq_status aq_gemv(const aq_layer_desc *desc, const void *packed, const uint16_t 
                                       reinterpret_cast<cudaStream_t>(stream)));
 }
 
+aq_status aq_gemv_noalloc(const aq_layer_desc *desc, const void *packed, const uint16_t *codebooks,
+                          const uint16_t *scales, const uint16_t *x, int batch, uint16_t *y,
+                          aq_stream_t stream)
+{
+    aq_status st = check_desc(desc);
+    if (st != AQ_OK) return st;
+    if (batch < 1 || batch > 16) return AQ_ERR_INVALID_ARG;
+    if (!packed || !codebooks || !x || !y) return AQ_ERR_INVALID_ARG;
+    if (!aligned16(packed) || !aligned16(codebooks) || !aligned16(x) || !aligned16(y))
+        return AQ_ERR_MISALIGNED;
+    if (scales && (reinterpret_cast<uintptr_t>(scales) & 1u)) return AQ_ERR_MISALIGNED;
+    const Geom g = aqk::make_geom(*desc);
+    if (aqh::gemv_workspace_bytes(g, batch) > AQ_GEMV_NOALLOC_SCRATCH_BYTES) return AQ_ERR_WORKSPACE;
+    bool too_large = false;
+    const cudaError_t e = aqh::launch_gemv_noalloc(g, packed, codebooks, scales, x, batch, y,
+                                                   reinterpret_cast<cudaStream_t>(stream), &too_large);
+    if (too_large) return AQ_ERR_WORKSPACE;
+    return from_cuda(e);
+}
+
 aq_status aq_gemm(const aq_layer_desc *desc, const void *packed, const uint16_t *codebooks,
                   const uint16_t *scales, const uint16_t *x, int T, uint16_t *y,
                   void *workspace, size_t workspace_bytes, aq_stream_t stream)

@@ -220,6 +220,9 @@ size_t gemv_workspace_bytes(const aqk::Geom &g, int batch);
 cudaError_t launch_gemv(const aqk::Geom &g, const void *packed, const uint16_t *cb,
                         const uint16_t *scales, const uint16_t *x, int batch, uint16_t *y,
                         void *ws, cudaStream_t s);
+cudaError_t launch_gemv_noalloc(const aqk::Geom &g, const void *packed, const uint16_t *cb,
+                                const uint16_t *scales, const uint16_t *x, int batch, uint16_t *y,
+                                cudaStream_t s, bool *too_large);
 size_t gemm_workspace_bytes(const aqk::Geom &g, int T);
 cudaError_t launch_gemm(const aqk::Geom &g, const void *packed, const uint16_t *cb,
                         const uint16_t *scales, const uint16_t *x, int T, uint16_t *y,

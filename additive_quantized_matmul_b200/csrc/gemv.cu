@@ -19,6 +19,8 @@
 //    codebook (about one request per SM clock), not HBM.
 // Split-K partial sums go to the workspace and the last CTA to arrive for a
 // row range adds them in split order (no float atomics: bit-reproducible).
+#include <mutex>
+
 #include "tc_common.cuh"
 
 namespace aqk {
@@ -526,6 +528,63 @@ cudaError_t launch_gemv(const Geom &g, const void *packed, const uint16_t *cb,
         break;
     }
     return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Decode-time product without caller-provided workspace.
+//
+// The split-K partial sums, arrival counters and status word live in one
+// file-scope device array (every GPU that loads this library holds it until
+// the process exits).  Host code must not hand the array's name to a kernel:
+// on the host it is only a stand-in, so its device address is looked up once
+// per device, with that device current, through cudaGetSymbolAddress.  All
+// calls share the array, so calls that overlap on the GPU race; each call
+// clears the status word and counters (cudaMemsetAsync on its stream) before
+// its kernel starts.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_gemv_scratch[AQ_GEMV_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mutex;
+void *g_scratch_ptr[kMaxDevices] = {};
+
+cudaError_t scratch_for_current_device(void **out)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_scratch_mutex);
+    if (!g_scratch_ptr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_gemv_scratch);
+        if (e != cudaSuccess) return e;
+        g_scratch_ptr[dev] = p;
+    }
+    *out = g_scratch_ptr[dev];
+    return cudaSuccess;
+}
+
+}  // namespace
+
+cudaError_t launch_gemv_noalloc(const Geom &g, const void *packed, const uint16_t *cb,
+                                const uint16_t *scales, const uint16_t *x, int batch, uint16_t *y,
+                                cudaStream_t s, bool *too_large)
+{
+    const GemvPlan p = plan_gemv(g, batch);
+    *too_large = p.ws_bytes > AQ_GEMV_NOALLOC_SCRATCH_BYTES;
+    if (*too_large) return cudaSuccess;
+    void *scratch = nullptr;
+    cudaError_t e = scratch_for_current_device(&scratch);
+    if (e != cudaSuccess) return e;
+    // status word and arrival counters must start at zero; the partials are
+    // fully written before they are read
+    const size_t clear = kWsHeader + align16(sizeof(unsigned) * (size_t)p.grid_x);
+    e = cudaMemsetAsync(scratch, 0, clear, s);
+    if (e != cudaSuccess) return e;
+    return launch_gemv(g, packed, cb, scales, x, batch, y, scratch, s);
 }
 
 }  // namespace aqh

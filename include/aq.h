@@ -167,6 +167,37 @@ aq_status aq_gemv(const aq_layer_desc *desc, const void *packed, const uint16_t 
                   void *workspace, size_t workspace_bytes, aq_stream_t stream);
 
 /*
+ * aq_gemv without a workspace argument, for callers that cannot allocate
+ * device memory: code that runs where the host framework owns every device
+ * allocation, real-time loops that forbid allocation after start-up, or
+ * plugins handed only input and output buffers.  The paper has no
+ * counterpart; this is an interface convenience.
+ *
+ * Same arguments, results and bits as aq_gemv, minus the workspace.  The
+ * split-K scratch is a fixed device array inside the library of
+ * AQ_GEMV_NOALLOC_SCRATCH_BYTES bytes, which every GPU that loads the
+ * library holds until the process exits.  The call allocates nothing (no
+ * cudaMalloc/cudaFree, no allocating library routine); it clears the part
+ * of the array that must start at zero with cudaMemsetAsync on `stream`.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress, with that device current); make that first call
+ *    before any stream capture on that device.
+ *  - Every call shares the one array and it keeps the last call's contents:
+ *    calls whose kernels may overlap on the GPU (different streams) race and
+ *    give wrong results.  Serialise them, or use aq_gemv with a workspace
+ *    per stream.
+ *  - AQ_ERR_WORKSPACE if the layer and batch need more scratch than the
+ *    array holds (aq_gemv_workspace_bytes(desc, batch) greater than
+ *    AQ_GEMV_NOALLOC_SCRATCH_BYTES); nothing is launched then.
+ *  - A bounded wait that gives up inside the kernel cannot be reported (the
+ *    status word is internal): use aq_gemv when that report is needed.
+ */
+#define AQ_GEMV_NOALLOC_SCRATCH_BYTES (4u << 20)
+aq_status aq_gemv_noalloc(const aq_layer_desc *desc, const void *packed, const uint16_t *codebooks,
+                          const uint16_t *scales, const uint16_t *x, int batch, uint16_t *y,
+                          aq_stream_t stream);
+
+/*
  * Prefill product for 1 <= T <= 2^22 tokens on the tensor cores (tcgen05.mma with
  * binary16 operands and fp32 accumulation in tensor memory):
  *   y[o][t] = RN16(s[o] * sum_i W[o][i] x[i][t]).

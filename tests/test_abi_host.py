@@ -147,3 +147,22 @@ def test_binding_raises_on_error():
     with pytest.raises(aq.AQError) as e:
         aq.aq_gemv(d, FAKE, FAKE, FAKE, FAKE, 0, FAKE, FAKE, 1 << 20, stream=0)
     assert e.value.name == "AQ_ERR_INVALID_ARG"
+
+
+def test_gemv_noalloc_argument_errors():
+    d = aq.LayerDesc.make(64, 256, 1, 16)
+    f = aq.lib.aq_gemv_noalloc
+    assert f(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, 0, FAKE, None) == 1
+    assert f(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, 17, FAKE, None) == 1
+    assert f(ctypes.byref(d), None, FAKE, FAKE, FAKE, 1, FAKE, None) == 1
+    assert f(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE + 8, 1, FAKE, None) == 3
+    assert f(None, FAKE, FAKE, FAKE, FAKE, 1, FAKE, None) == 1
+    big = aq.LayerDesc.make(32768, 65536, 2, 8)  # needs more scratch than the fixed array
+    assert aq.aq_gemv_workspace_bytes(big, 1) > aq.GEMV_NOALLOC_SCRATCH_BYTES
+    assert f(ctypes.byref(big), FAKE, FAKE, FAKE, FAKE, 1, FAKE, None) == 4
+
+
+def test_noalloc_scratch_size_matches_header():
+    text = open(HEADER).read()
+    m = re.search(r"#define AQ_GEMV_NOALLOC_SCRATCH_BYTES \((\d+)u << (\d+)\)", text)
+    assert m and int(m.group(1)) << int(m.group(2)) == aq.GEMV_NOALLOC_SCRATCH_BYTES
