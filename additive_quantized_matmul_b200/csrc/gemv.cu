@@ -166,27 +166,32 @@ gemv_2x8_lut_kernel(Geom L, const uint4 *__restrict__ packed, const uint4 *__res
 
 // ---------------------------------------------------------------------------
 // Small-batch product on the tensor cores (any batch for 1x16, batch 2..16
-// for 2x8).
+// for 2x8), warp-specialised.
 //
-// CTA = 128 rows x one split of the K range, 128 threads.  Per stage of 64
-// input features (8 groups) thread t owns code chunk (row tile t/8, group
-// t%8) of the 128 x 64 A tile (128-byte swizzle, K-major):
-//  * 1x16: the chunk's 8 codewords are the weights; they are copied straight
-//    from the L2-resident codebook into the A tile with 16-byte cp.async, so
-//    gathers of several stages are in flight without holding registers;
+// CTA = 128 rows x one split of the K range; 4 decoder warps + 1 MMA warp.
+// Per stage of 64 input features (8 groups), decoder thread t owns code chunk
+// (row tile t/8, group t%8) of the 128 x 64 A tile (128-byte swizzle,
+// K-major):
+//  * 1x16: the chunk's 8 codewords are the weights; they go straight from
+//    the L2-resident codebook into the A tile with 16-byte cp.async, several
+//    stages ahead, without holding registers;
 //  * 2x8: the two codewords per weight group are read from the codebooks in
 //    shared memory and summed with binary16 adds (one rounding), then stored.
-// x rows of the stage go to the B tile (MN-major, 32-byte swizzle: 64 rows
-// of 16 batch columns, zero-padded).  A ring of kTcRing stage buffers; the
-// MMAs of stage i are issued kTcLag stages after its copies, by thread 0:
-// four tcgen05.mma (M = 128, N = 16, K = 16) into an fp32 accumulator in
-// tensor memory, committed to the buffer's mbarrier, which the producer
-// waits on (bounded) before refilling that buffer.
+// x rows of the stage go straight into the B tile when a row is 16 or 32
+// bytes (MN-major, 32-byte swizzle, 16 columns zero-padded), else as raw rows
+// into the stage's x slot.  A decoder never waits for another: once its own
+// copies of stage j have landed it fences them to the async proxy and arrives
+// on full[j].  The MMA warp waits on full[j], builds the B tile from the x
+// slot if needed, and one lane issues four tcgen05.mma (M 128, N 16, K 16)
+// into the fp32 TMEM accumulator and commits to empty[j] (the decoders'
+// signal that the buffer may be refilled) and, after the last stage, to
+// acc_full.  Every wait is bounded.
 // ---------------------------------------------------------------------------
-constexpr int kTcThreads = 128;
+constexpr int kTcDecoders = 128;
+constexpr int kTcThreads = kTcDecoders + 32;
 constexpr int kTcBM = 128;
 constexpr int kTcN = 16;
-// ring depth and copy-to-MMA lag: deep for the asynchronous 1x16 gathers,
+// ring depth and copy-to-signal lag: deep for the asynchronous 1x16 gathers,
 // short for the synchronous 2x8 decode
 template <int K> struct TcRing;
 template <> struct TcRing<1> { static constexpr int depth = 5, lag = 3; };
@@ -195,6 +200,7 @@ constexpr int kTcTileA = kTcBM * 64 * 2;  // 16 KiB
 constexpr int kTcTileB = 64 * 32;         // 2 KiB: 64 rows x 16 columns
 constexpr int kTcXSlot = 64 * 16 * 2;     // raw x rows of one stage, batch <= 16
 constexpr int kTcTmemCols = 32;
+constexpr int kCodeAhead = 4;             // code chunks requested this many stages ahead
 
 template <int K>
 __global__ void __launch_bounds__(kTcThreads)
@@ -202,16 +208,19 @@ gemv_tc_kernel(Geom L, const uint4 *__restrict__ packed, const uint4 *__restrict
                const uint16_t *__restrict__ scales, const uint16_t *__restrict__ x, int batch,
                uint16_t *__restrict__ y, SplitK sk, void *ws, int stages_per_split)
 {
-    constexpr int kTcRing = TcRing<K>::depth, kTcLag = TcRing<K>::lag;
+    constexpr int R = TcRing<K>::depth, LAG = TcRing<K>::lag;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t *smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-    uint8_t *tileA = smem;                                  // [ring][16 KiB]
-    uint8_t *tileB = smem + kTcRing * kTcTileA;             // [ring][2 KiB]
-    uint8_t *xring = tileB + kTcRing * kTcTileB;            // [ring][2 KiB] raw x rows
-    uint4 *scb = reinterpret_cast<uint4 *>(xring + kTcRing * kTcXSlot);  // 2x8 codebooks
-    uint64_t *bars = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(scb) + (K == 2 ? 512 * 16 : 0));
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + kTcRing);
+    uint8_t *tileA = smem;                    // [R][16 KiB]
+    uint8_t *tileB = tileA + R * kTcTileA;    // [R][2 KiB]
+    uint8_t *xring = tileB + R * kTcTileB;    // [R][2 KiB] raw x rows
+    uint4 *scb = reinterpret_cast<uint4 *>(xring + R * kTcXSlot);  // 2x8 codebooks
+    uint64_t *full = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(scb) + (K == 2 ? 512 * 16 : 0));
+    uint64_t *empty = full + R;
+    uint64_t *acc_full = empty + R;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 1);
+    uint32_t *abort_flag = tmem_slot + 1;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int m0 = blockIdx.x * kTcBM;
@@ -219,12 +228,18 @@ gemv_tc_kernel(Geom L, const uint4 *__restrict__ packed, const uint4 *__restrict
     const int s0 = blockIdx.y * stages_per_split;
     const int s1 = min(nst, s0 + stages_per_split);
     const int nloc = max(0, s1 - s0);
+    const bool x_direct = (batch == 16 || batch == 8);
 
     if (K == 1 && tid == 0) prefetch_table_share(cb, 65536u * 16u);
     if (K == 2)
         for (int i = tid; i < 512; i += kTcThreads) scb[i] = cb[i];
     if (tid == 0) {
-        for (int s = 0; s < kTcRing; ++s) mbar_init(&bars[s], 1);
+        for (int s = 0; s < R; ++s) {
+            mbar_init(&full[s], kTcDecoders);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(acc_full, 1);
+        *abort_flag = 0;
         fence_mbar_init();
     }
     if (warp == 0) tmem_alloc(tmem_slot, kTcTmemCols);
@@ -232,157 +247,166 @@ gemv_tc_kernel(Geom L, const uint4 *__restrict__ packed, const uint4 *__restrict
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t idesc = make_idesc(kTcBM, kTcN, true);
+    volatile uint32_t *abort_v = abort_flag;
 
-    const int rt_l = tid >> 3, gi = tid & 7;     // A role
-    const int rt = (m0 >> 3) + rt_l;
-    const int kr = tid >> 1, hb = tid & 1;        // B role: feature row, 8-column half
-    const bool rows_live = rt < L.rtiles;
-
-    // code chunks are loaded kCodeAhead stages ahead (a register ring), so
-    // that a stage's codeword gathers never wait on an HBM round trip
-    constexpr int kCodeAhead = 4;
-    uint4 code_ring[kCodeAhead];
+    if (warp < kTcDecoders / 32) {
+        // ------------------------------ decoders ------------------------------
+        const int rt_l = tid >> 3, gi = tid & 7;  // A role: row tile, group
+        const int rt = (m0 >> 3) + rt_l;
+        const bool rows_live = rt < L.rtiles;
+        const int kr = tid >> 1, hb = tid & 1;    // B role: feature row, 8-column half
+        uint4 code_ring[kCodeAhead];
 #pragma unroll
-    for (int q = 0; q < kCodeAhead; ++q) {
-        const int g = (s0 + q) * 8 + gi;
-        code_ring[q] = (q < nloc && rows_live && g < L.G) ? ldg_stream_v4(packed + (size_t)rt * L.gp + g)
-                                                          : make_uint4(0, 0, 0, 0);
-    }
-
-    const bool x_direct = (batch == 16 || batch == 8);
-    // everything above touched weights only; x, y and the workspace may be
-    // written by the previous launch on the stream
-    grid_dependency_wait();
-    grid_launch_dependents();
-    bool ok = true;
-    // stage loop unrolled by the code-ring depth so every ring index is static
-    for (int i0 = 0; ok && i0 < nloc + kTcLag; i0 += kCodeAhead) {
+        for (int q = 0; q < kCodeAhead; ++q) {
+            const int g = (s0 + q) * 8 + gi;
+            code_ring[q] = (q < nloc && rows_live && g < L.G) ? ldg_stream_v4(packed + (size_t)rt * L.gp + g)
+                                                              : make_uint4(0, 0, 0, 0);
+        }
+        // everything above touched weights only; x, y and the workspace may
+        // be written by the previous launch on the stream
+        grid_dependency_wait();
+        grid_launch_dependents();
+        bool ok = true;
+        // stage loop unrolled by the code-ring depth so every ring index is static
+        for (int i0 = 0; ok && i0 < nloc + LAG; i0 += kCodeAhead) {
 #pragma unroll
-        for (int u = 0; u < kCodeAhead; ++u) {
-            const int i = i0 + u;
-            if (!ok || i >= nloc + kTcLag) break;
-            // ---- produce stage i ------------------------------------------------
-            if (i < nloc) {
-                const int s = s0 + i, buf = i % kTcRing;
-                if (i >= kTcRing) {  // buffer is free once the MMAs of stage i - ring completed
-                    const bool got = mbar_wait_ns(&bars[buf], ((i - kTcRing) / kTcRing) & 1, kWaitNs);
-                    if (!__syncthreads_and(got)) ok = false;
-                }
-                if (!ok) break;
-                const uint4 code = code_ring[u];
-                const bool live = rows_live && s * 8 + gi < L.G;
-                {
-                    const int g = (s + kCodeAhead) * 8 + gi;
-                    code_ring[u] = (i + kCodeAhead < nloc && rows_live && g < L.G)
-                                       ? ldg_stream_v4(packed + (size_t)rt * L.gp + g)
-                                       : make_uint4(0, 0, 0, 0);
-                }
-                uint8_t *A = tileA + buf * kTcTileA;
-                uint32_t wd[8];
-                unpack8(code, wd);
-                if (K == 1) {
-                    const uint32_t a0 = smem_u32(A);
+            for (int u = 0; u < kCodeAhead; ++u) {
+                const int i = i0 + u;
+                if (i >= nloc + LAG) break;
+                if (i < nloc) {
+                    const int s = s0 + i, buf = i % R;
+                    // the buffer is free once the MMAs of stage i - R completed
+                    if (i >= R && !mbar_wait_ns(&empty[buf], ((i / R) - 1) & 1, kWaitNs)) *abort_v = 1;
+                    if (*abort_v) {
+                        ok = false;
+                        break;
+                    }
+                    const uint4 code = code_ring[u];
+                    {
+                        const int g = (s + kCodeAhead) * 8 + gi;
+                        code_ring[u] = (i + kCodeAhead < nloc && rows_live && g < L.G)
+                                           ? ldg_stream_v4(packed + (size_t)rt * L.gp + g)
+                                           : make_uint4(0, 0, 0, 0);
+                    }
+                    const bool live = rows_live && s * 8 + gi < L.G;
+                    uint8_t *A = tileA + buf * kTcTileA;
+                    uint32_t wd[8];
+                    unpack8(code, wd);
+                    if (K == 1) {
+                        const uint32_t a0 = smem_u32(A);
 #pragma unroll
-                    for (int r = 0; r < 8; ++r)
-                        cp_async16(a0 + sw128(rt_l * 8 + r, gi), live ? (const void *)(cb + wd[r]) : (const void *)cb,
-                                   live ? 16u : 0u);
-                } else {
+                        for (int r = 0; r < 8; ++r)
+                            cp_async16(a0 + sw128(rt_l * 8 + r, gi), live ? (const void *)(cb + wd[r]) : (const void *)cb,
+                                       live ? 16u : 0u);
+                    } else {
 #pragma unroll
-                    for (int r = 0; r < 8; ++r) {
-                        const uint4 v = live ? add_round_h8(scb[wd[r] & 0xff], scb[256 + (wd[r] >> 8)])
-                                             : make_uint4(0, 0, 0, 0);
-                        *reinterpret_cast<uint4 *>(A + sw128(rt_l * 8 + r, gi)) = v;
+                        for (int r = 0; r < 8; ++r) {
+                            const uint4 v = live ? add_round_h8(scb[wd[r] & 0xff], scb[256 + (wd[r] >> 8)])
+                                                 : make_uint4(0, 0, 0, 0);
+                            *reinterpret_cast<uint4 *>(A + sw128(rt_l * 8 + r, gi)) = v;
+                        }
+                    }
+                    // x rows of this stage: straight into the B tile when a row is
+                    // 16 or 32 bytes, else the raw rows into the stage's x slot
+                    if (x_direct) {
+                        const int k = s * 64 + kr, n0 = hb * 8;
+                        const bool in = k < L.in && n0 < batch;
+                        cp_async16(smem_u32(tileB + buf * kTcTileB) + sw32(kr, hb),
+                                   in ? (const void *)(x + (size_t)k * batch + n0) : (const void *)x, in ? 16u : 0u);
+                    } else if (tid < 8 * batch) {
+                        const int valid = max(0, min(64, L.in - s * 64)) * batch * 2;
+                        const int nb = max(0, min(16, valid - tid * 16));
+                        const uint8_t *src = reinterpret_cast<const uint8_t *>(x + (size_t)s * 64 * batch) + tid * 16;
+                        cp_async16(smem_u32(xring + buf * kTcXSlot) + tid * 16, nb > 0 ? (const void *)src : (const void *)x,
+                                   (uint32_t)nb);
                     }
                 }
-                // x rows k of this stage: columns 8*hb .. 8*hb+7 straight into
-                // the B tile when a row is 16 or 32 bytes, else the raw rows
-                // (64*batch*2 contiguous bytes) into the stage's x slot
-                if (x_direct) {
-                    uint8_t *Bt = tileB + buf * kTcTileB;
-                    const int k = s * 64 + kr, n0 = hb * 8;
-                    const uint32_t bdst = smem_u32(Bt) + sw32(kr, hb);
-                    const bool in = k < L.in && n0 < batch;
-                    cp_async16(bdst, in ? (const void *)(x + (size_t)k * batch + n0) : (const void *)x, in ? 16u : 0u);
-                } else if (tid < 8 * batch) {
-                    const int valid = max(0, min(64, L.in - s * 64)) * batch * 2;
-                    const int nb = max(0, min(16, valid - tid * 16));
-                    const uint8_t *src = reinterpret_cast<const uint8_t *>(x + (size_t)s * 64 * batch) + tid * 16;
-                    cp_async16(smem_u32(xring + buf * kTcXSlot) + tid * 16, nb > 0 ? (const void *)src : (const void *)x,
-                               (uint32_t)nb);
+                cp_async_commit();  // one group per iteration (empty in the drain)
+                const int j = i - LAG;
+                if (j >= 0) {
+                    // this thread's copies of stage j have landed: publish them
+                    cp_async_wait<LAG>();
+                    fence_proxy_async_smem();
+                    mbar_arrive(&full[j % R]);
                 }
             }
-            cp_async_commit();  // one group per iteration (empty in the drain)
-            // ---- consume stage j = i - lag: its copies are complete ----------------
-            const int j = i - kTcLag;
-            if (j >= 0) {
-                cp_async_wait<TcRing<K>::lag>();
-                if (!x_direct) {
-                    // every thread's copies of stage j are complete: build the
-                    // B tile rows from the stage's raw x slot
-                    __syncthreads();
-                    const uint16_t *xs = reinterpret_cast<const uint16_t *>(xring + (j % kTcRing) * kTcXSlot);
-                    const int n0 = hb * 8;
+        }
+        cp_async_wait<0>();
+        // ------------------------------ epilogue ------------------------------
+        const bool got = (*abort_v == 0) && mbar_wait_ns(acc_full, 0, kWaitNs);
+        if (!got) *abort_v = 1;
+        tc_fence_after();
+        if (__all_sync(0xffffffffu, got)) {
+            const int row = m0 + warp * 32 + lane;  // TMEM lane quarter = warp
+            float v[16];
+            if (nloc > 0) {
+                tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16), v);
+            } else {
+#pragma unroll
+                for (int n = 0; n < 16; ++n) v[n] = 0.f;
+            }
+            if (row < L.out) {
+                if (gridDim.y == 1) {
+                    const float sc = scales ? __half2float(__ushort_as_half(scales[row])) : 1.f;
+#pragma unroll
+                    for (int n = 0; n < 16; ++n)
+                        if (n < batch)
+                            y[(size_t)row * batch + n] = __half_as_ushort(__float2half_rn(sc * v[n]));
+                } else {
+                    float *p = sk.partials + (size_t)blockIdx.y * L.rows8 * batch + (size_t)row * batch;
+#pragma unroll
+                    for (int n = 0; n < 16; ++n)
+                        if (n < batch) p[n] = v[n];
+                }
+            }
+        }
+    } else {
+        // ------------------------------ MMA warp ------------------------------
+        const uint32_t idesc = make_idesc(kTcBM, kTcN, true);
+        for (int j = 0; j < nloc; ++j) {
+            const int buf = j % R;
+            const bool got = mbar_wait_ns(&full[buf], (j / R) & 1, kWaitNs);
+            if (!__all_sync(0xffffffffu, got)) {
+                *abort_v = 1;
+                break;
+            }
+            if (__any_sync(0xffffffffu, *abort_v != 0)) break;
+            if (!x_direct) {
+                // B tile rows from the stage's raw x slot: 64 rows x 2 halves
+                const uint16_t *xs = reinterpret_cast<const uint16_t *>(xring + buf * kTcXSlot);
+#pragma unroll
+                for (int c = lane; c < 128; c += 32) {
+                    const int krow = c >> 1, n0 = (c & 1) * 8;
                     uint16_t h[8];
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) h[q] = (n0 + q < batch) ? xs[kr * batch + n0 + q] : (uint16_t)0;
-                    *reinterpret_cast<uint4 *>(tileB + (j % kTcRing) * kTcTileB + sw32(kr, hb)) =
+                    for (int q = 0; q < 8; ++q) h[q] = (n0 + q < batch) ? xs[krow * batch + n0 + q] : (uint16_t)0;
+                    *reinterpret_cast<uint4 *>(tileB + buf * kTcTileB + sw32(krow, c & 1)) =
                         make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16), h[4] | (h[5] << 16), h[6] | (h[7] << 16));
                 }
                 fence_proxy_async_smem();
-                __syncthreads();
-                if (tid == 0) {
-                    tc_fence_after();
-                    const int buf = j % kTcRing;
-                    const uint32_t a0 = smem_u32(tileA + buf * kTcTileA);
-                    const uint32_t b0 = smem_u32(tileB + buf * kTcTileB);
+            }
+            __syncwarp();
+            if (lane == 0) {
+                tc_fence_after();
+                const uint32_t a0 = smem_u32(tileA + buf * kTcTileA);
+                const uint32_t b0 = smem_u32(tileB + buf * kTcTileB);
 #pragma unroll
-                    for (int ks = 0; ks < 4; ++ks) {
-                        const uint64_t ad = smem_desc_sw128(a0 + ks * 32, 16, 1024);
-                        const uint64_t bd = smem_desc(b0 + ks * 512, kTcTileB, 256, kSwizzle32B);
-                        mma_f16_ss(tmem, ad, bd, idesc, (j > 0 || ks > 0) ? 1u : 0u);
-                    }
-                    mma_commit(&bars[buf]);
+                for (int ks = 0; ks < 4; ++ks) {
+                    const uint64_t ad = smem_desc_sw128(a0 + ks * 32, 16, 1024);
+                    const uint64_t bd = smem_desc(b0 + ks * 512, kTcTileB, 256, kSwizzle32B);
+                    mma_f16_ss(tmem, ad, bd, idesc, (j > 0 || ks > 0) ? 1u : 0u);
                 }
+                mma_commit(&empty[buf]);
             }
+            __syncwarp();
         }
+        if (lane == 0) mma_commit(acc_full);  // completes when every MMA issued above has
     }
-    cp_async_wait<0>();
-    if (ok && nloc > 0) {
-        const int last = nloc - 1;
-        ok = __syncthreads_and(mbar_wait_ns(&bars[last % kTcRing], (last / kTcRing) & 1, kWaitNs));
-    } else {
-        ok = __syncthreads_and(ok);
-    }
-    if (!ok) {
-        if (tid == 0) record_status(ws, AQ_ERR_TIMEOUT);
-        // drain whatever MMAs were issued (bounded), so tensor memory is idle
-        for (int q = max(0, nloc - kTcRing); q < nloc; ++q)
-            mbar_wait_ns(&bars[q % kTcRing], (q / kTcRing) & 1, kWaitNs);
-    }
-    tc_fence_after();
-    const int row = m0 + warp * 32 + lane;
-    if (ok) {
-        float v[16];
-        if (nloc > 0) {
-            tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16), v);
-        } else {
-#pragma unroll
-            for (int n = 0; n < 16; ++n) v[n] = 0.f;
-        }
-        if (row < L.out) {
-            if (gridDim.y == 1) {
-                const float sc = scales ? __half2float(__ushort_as_half(scales[row])) : 1.f;
-#pragma unroll
-                for (int n = 0; n < 16; ++n)
-                    if (n < batch)
-                        y[(size_t)row * batch + n] = __half_as_ushort(__float2half_rn(sc * v[n]));
-            } else {
-                float *p = sk.partials + (size_t)blockIdx.y * L.rows8 * batch + (size_t)row * batch;
-#pragma unroll
-                for (int n = 0; n < 16; ++n)
-                    if (n < batch) p[n] = v[n];
-            }
+    __syncthreads();
+    if (*abort_v) {
+        if (tid == 0) {
+            record_status(ws, AQ_ERR_TIMEOUT);
+            mbar_wait_ns(acc_full, 0, kWaitNs);  // drain the issued MMAs (bounded)
         }
     }
     tc_fence_before();
@@ -448,11 +472,12 @@ GemvPlan plan_gemv(const Geom &g, int batch)
     return p;
 }
 
-// ring of (A tile, B tile, x slot) + codebooks + barriers and TMEM slot
+// ring of (A tile, B tile, x slot) + codebooks + barriers, TMEM slot, flag
 template <int K>
 constexpr int tc_smem_bytes()
 {
-    return 1024 + TcRing<K>::depth * (kTcTileA + kTcTileB + kTcXSlot) + (K == 2 ? 512 * 16 : 0) + 128;
+    return 1024 + TcRing<K>::depth * (kTcTileA + kTcTileB + kTcXSlot) + (K == 2 ? 512 * 16 : 0) +
+           (2 * TcRing<K>::depth + 1) * 8 + 16;
 }
 
 template <class Kern>
