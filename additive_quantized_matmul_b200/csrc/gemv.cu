@@ -106,8 +106,9 @@ gemv_2x8_lut_kernel(Geom L, const uint4 *__restrict__ packed, const uint4 *__res
                     const uint16_t *__restrict__ scales, const uint16_t *__restrict__ x,
                     uint16_t *__restrict__ y, SplitK sk, int rt_per_cta)
 {
-    extern __shared__ float lut[];  // [2][256][32]
-    __shared__ uint4 xs[32];        // activations of the block's 32 groups
+    extern __shared__ float lut[];  // [2][256][32] tables, then one codebook as fp32 [256][8]
+    float *cbf = lut + 2 * 256 * 32;
+    __shared__ float4 xf[32][2];    // activations of the block's 32 groups, fp32
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gb = blockIdx.y;
     const int rt0 = blockIdx.x * rt_per_cta;
@@ -124,13 +125,37 @@ gemv_2x8_lut_kernel(Geom L, const uint4 *__restrict__ packed, const uint4 *__res
     grid_launch_dependents();
     if (threadIdx.x < 32) {
         const int g = gb * 32 + threadIdx.x;
-        xs[threadIdx.x] = (g < L.G) ? ldg_nc_v4(x + (size_t)g * 8) : make_uint4(0, 0, 0, 0);
+        const uint4 v = (g < L.G) ? ldg_nc_v4(x + (size_t)g * 8) : make_uint4(0, 0, 0, 0);
+        const float2 a = h2f2(v.x), b = h2f2(v.y), c = h2f2(v.z), d = h2f2(v.w);
+        xf[threadIdx.x][0] = make_float4(a.x, a.y, b.x, b.y);
+        xf[threadIdx.x][1] = make_float4(c.x, c.y, d.x, d.y);
     }
-    __syncthreads();
-    for (int e = threadIdx.x; e < 2 * 256 * 32; e += kLutWarps * 32) {
-        const int l = e & 31;
-        const int kc = e >> 5;  // k*256 + c
-        lut[e] = dot8(ldg_nc_v4(cb + kc), xs[l], 0.f);
+    // Tables, one codebook at a time: stage it as fp32, then entry e of the
+    // table (codeword e >> 5, group e & 31) is an 8-term dot product read
+    // entirely from shared memory (codeword broadcast, x conflict-free).
+    for (int k = 0; k < 2; ++k) {
+        __syncthreads();  // xf ready / previous codebook no longer read
+        {
+            const int c = threadIdx.x;  // 256 threads, one codeword each
+            const uint4 v = ldg_nc_v4(cb + k * 256 + c);
+            const float2 a = h2f2(v.x), b = h2f2(v.y), cc = h2f2(v.z), d = h2f2(v.w);
+            reinterpret_cast<float4 *>(cbf)[2 * c] = make_float4(a.x, a.y, b.x, b.y);
+            reinterpret_cast<float4 *>(cbf)[2 * c + 1] = make_float4(cc.x, cc.y, d.x, d.y);
+        }
+        __syncthreads();
+        float *tab = lut + k * 256 * 32;
+#pragma unroll 4
+        for (int e = threadIdx.x; e < 256 * 32; e += kLutWarps * 32) {
+            const int l = e & 31, c = e >> 5;
+            const float4 c0 = reinterpret_cast<const float4 *>(cbf)[2 * c];
+            const float4 c1 = reinterpret_cast<const float4 *>(cbf)[2 * c + 1];
+            const float4 x0 = xf[l][0], x1 = xf[l][1];
+            float acc = c0.x * x0.x;
+            acc = fmaf(c0.y, x0.y, acc); acc = fmaf(c0.z, x0.z, acc); acc = fmaf(c0.w, x0.w, acc);
+            acc = fmaf(c1.x, x1.x, acc); acc = fmaf(c1.y, x1.y, acc); acc = fmaf(c1.z, x1.z, acc);
+            acc = fmaf(c1.w, x1.w, acc);
+            tab[e] = acc;
+        }
     }
     __syncthreads();
     const float *lut0 = lut + lane;
@@ -526,7 +551,7 @@ cudaError_t launch_gemv(const Geom &g, const void *packed, const uint16_t *cb,
     cudaError_t e = cudaSuccess;
     switch (p.path) {
     case kLut2x8: {
-        const int smem = 2 * 256 * 32 * sizeof(float);
+        const int smem = (2 * 256 * 32 + 256 * 8) * sizeof(float);  // tables + one fp32 codebook
         e = set_smem(gemv_2x8_lut_kernel, smem);
         if (e != cudaSuccess) return e;
         e = launch_pdl(gemv_2x8_lut_kernel, grid, dim3(kLutWarps * 32), smem, s, g, pk, c, scales, x, y, sk,

@@ -252,6 +252,22 @@ def count_graph_kernels(graph) -> int:
     return count
 
 
+def recorded_traffic(workload_name: str, batch: int):
+    """DRAM bytes per launch from the committed ncu record, or None when the
+    kernel sources changed since the counters were taken."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "traffic_gemv_tc.json")
+    if workload_name != WORKLOAD or not os.path.exists(p):
+        return None
+    rec = json.load(open(p))
+    h = hashlib.sha256()
+    for f in rec["sources"]:
+        h.update(open(os.path.join(ROOT, f), "rb").read())
+    if h.hexdigest() != rec["sources_sha256"]:
+        return None
+    return rec["per_launch_bytes"].get(str(batch))
+
+
 def flops(spec: LayerSpec, n: int) -> int:
     return 2 * spec.out_features * spec.in_features * n
 
@@ -378,7 +394,7 @@ def run_gpu(args) -> None:
         value = world * step_bytes * args.steps / (elapsed_ms * 1e-3) / 1e9
         unit = "GB/s"
         roofline = {"bound": "hbm", "achieved": dom["gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                    "frac": dom["frac_hbm"], "traffic": None,
+                    "frac": dom["frac_hbm"], "traffic": recorded_traffic(args.workload, dom["n"]),
                     "kernel": f"aq_gemv {dom['layer']} batch {dom['n']}",
                     "peak_source": f"{peaks['source']} hbm_gbs (STREAM-style copy)"}
     for k in kernels:
