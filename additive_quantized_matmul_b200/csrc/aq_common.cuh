@@ -113,13 +113,15 @@ __device__ __forceinline__ uint4 ldg_nc_v4(const void *p)
     return __ldg(reinterpret_cast<const uint4 *>(p));
 }
 
-// Streaming load: read once, do not keep in L1.
+// Streaming load: read once, do not keep in L1.  Volatile, so a load
+// written as a prefetch is issued where it is written rather than sunk by
+// the compiler to its first use.
 __device__ __forceinline__ uint4 ldg_stream_v4(const void *p)
 {
     uint4 r;
-    asm("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-        : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-        : "l"(p));
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
     return r;
 }
 

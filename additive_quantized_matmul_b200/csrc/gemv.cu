@@ -106,55 +106,53 @@ gemv_2x8_lut_kernel(Geom L, const uint4 *__restrict__ packed, const uint4 *__res
                     const uint16_t *__restrict__ scales, const uint16_t *__restrict__ x,
                     uint16_t *__restrict__ y, SplitK sk, int rt_per_cta)
 {
-    extern __shared__ float lut[];  // [2][256][32] tables, then one codebook as fp32 [256][8]
-    float *cbf = lut + 2 * 256 * 32;
-    __shared__ float4 xf[32][2];    // activations of the block's 32 groups, fp32
+    extern __shared__ float lut[];  // [2][256][32] tables
+    __shared__ uint4 scb[512];      // both codebooks, binary16
+    __shared__ uint4 xs[32];        // activations of the block's 32 groups
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gb = blockIdx.y;
     const int rt0 = blockIdx.x * rt_per_cta;
     const int rt1 = min(L.rtiles, rt0 + rt_per_cta);
-    // This warp's code chunks (row tiles rt0 + warp + 8j) are requested before
-    // the tables are built, so their HBM latency hides behind the build.
+    // Weights first: this warp's code chunks (row tiles rt0 + warp + 8j) and
+    // the codebooks are requested before anything waits, so their latency
+    // hides behind the table build.
     uint4 chunk[kLutMaxTilesPerWarp];
 #pragma unroll
     for (int j = 0; j < kLutMaxTilesPerWarp; ++j) {
         const int rt = rt0 + warp + j * kLutWarps;
         chunk[j] = (rt < rt1) ? ldg_stream_v4(packed + (size_t)rt * L.gp + gb * 32 + lane) : make_uint4(0, 0, 0, 0);
     }
+    const uint4 cw0 = ldg_stream_v4(cb + threadIdx.x), cw1 = ldg_stream_v4(cb + 256 + threadIdx.x);
     grid_dependency_wait();  // x, y and the workspace follow the previous launch
     grid_launch_dependents();
     if (threadIdx.x < 32) {
         const int g = gb * 32 + threadIdx.x;
-        const uint4 v = (g < L.G) ? ldg_nc_v4(x + (size_t)g * 8) : make_uint4(0, 0, 0, 0);
-        const float2 a = h2f2(v.x), b = h2f2(v.y), c = h2f2(v.z), d = h2f2(v.w);
-        xf[threadIdx.x][0] = make_float4(a.x, a.y, b.x, b.y);
-        xf[threadIdx.x][1] = make_float4(c.x, c.y, d.x, d.y);
+        xs[threadIdx.x] = (g < L.G) ? ldg_nc_v4(x + (size_t)g * 8) : make_uint4(0, 0, 0, 0);
     }
-    // Tables, one codebook at a time: stage it as fp32, then entry e of the
-    // table (codeword e >> 5, group e & 31) is an 8-term dot product read
-    // entirely from shared memory (codeword broadcast, x conflict-free).
-    for (int k = 0; k < 2; ++k) {
-        __syncthreads();  // xf ready / previous codebook no longer read
+    scb[threadIdx.x] = cw0;
+    scb[256 + threadIdx.x] = cw1;
+    __syncthreads();
+    // Both tables in one pass.  Thread t always computes group l = t % 32
+    // (its 8 activations stay in registers); entry e = t + 256 i is codeword
+    // kc = t / 32 + 8 i of codebook kc / 256, read as a broadcast.
+    {
+        const int l = threadIdx.x & 31;
+        float xv[8];
         {
-            const int c = threadIdx.x;  // 256 threads, one codeword each
-            const uint4 v = ldg_nc_v4(cb + k * 256 + c);
-            const float2 a = h2f2(v.x), b = h2f2(v.y), cc = h2f2(v.z), d = h2f2(v.w);
-            reinterpret_cast<float4 *>(cbf)[2 * c] = make_float4(a.x, a.y, b.x, b.y);
-            reinterpret_cast<float4 *>(cbf)[2 * c + 1] = make_float4(cc.x, cc.y, d.x, d.y);
+            const uint4 v = xs[l];
+            const float2 a = h2f2(v.x), b = h2f2(v.y), c = h2f2(v.z), d = h2f2(v.w);
+            xv[0] = a.x; xv[1] = a.y; xv[2] = b.x; xv[3] = b.y; xv[4] = c.x; xv[5] = c.y; xv[6] = d.x; xv[7] = d.y;
         }
-        __syncthreads();
-        float *tab = lut + k * 256 * 32;
-#pragma unroll 4
-        for (int e = threadIdx.x; e < 256 * 32; e += kLutWarps * 32) {
-            const int l = e & 31, c = e >> 5;
-            const float4 c0 = reinterpret_cast<const float4 *>(cbf)[2 * c];
-            const float4 c1 = reinterpret_cast<const float4 *>(cbf)[2 * c + 1];
-            const float4 x0 = xf[l][0], x1 = xf[l][1];
-            float acc = c0.x * x0.x;
-            acc = fmaf(c0.y, x0.y, acc); acc = fmaf(c0.z, x0.z, acc); acc = fmaf(c0.w, x0.w, acc);
-            acc = fmaf(c1.x, x1.x, acc); acc = fmaf(c1.y, x1.y, acc); acc = fmaf(c1.z, x1.z, acc);
-            acc = fmaf(c1.w, x1.w, acc);
-            tab[e] = acc;
+#pragma unroll 8
+        for (int i = 0; i < 2 * 256 * 32 / (kLutWarps * 32); ++i) {
+            const int kc = (threadIdx.x >> 5) + kLutWarps * i;
+            const uint4 w = scb[kc];
+            const float2 a = h2f2(w.x), b = h2f2(w.y), c = h2f2(w.z), d = h2f2(w.w);
+            float acc = a.x * xv[0];
+            acc = fmaf(a.y, xv[1], acc); acc = fmaf(b.x, xv[2], acc); acc = fmaf(b.y, xv[3], acc);
+            acc = fmaf(c.x, xv[4], acc); acc = fmaf(c.y, xv[5], acc); acc = fmaf(d.x, xv[6], acc);
+            acc = fmaf(d.y, xv[7], acc);
+            lut[kc * 32 + l] = acc;
         }
     }
     __syncthreads();
@@ -551,7 +549,7 @@ cudaError_t launch_gemv(const Geom &g, const void *packed, const uint16_t *cb,
     cudaError_t e = cudaSuccess;
     switch (p.path) {
     case kLut2x8: {
-        const int smem = (2 * 256 * 32 + 256 * 8) * sizeof(float);  // tables + one fp32 codebook
+        const int smem = 2 * 256 * 32 * sizeof(float);  // the two tables
         e = set_smem(gemv_2x8_lut_kernel, smem);
         if (e != cudaSuccess) return e;
         e = launch_pdl(gemv_2x8_lut_kernel, grid, dim3(kLutWarps * 32), smem, s, g, pk, c, scales, x, y, sk,
