@@ -20,6 +20,10 @@ constexpr int kGroup = 8;        // weights per code group (in_group_size)
 constexpr int kTileRows = 8;     // rows per packed chunk
 constexpr int kGroupBlock = 32;  // groups per warp-wide load
 
+// Streaming multiprocessors of a B200 (two dies of 74); launch plans size
+// their grids in multiples of it.
+constexpr int kNumSMs = 148;
+
 struct Geom {
     int out, in, G;   // rows, columns, groups (in / 8)
     int K, B;         // codebooks, bits per code
@@ -111,6 +115,13 @@ __device__ __forceinline__ float dot8(uint4 w, uint4 x, float acc)
 __device__ __forceinline__ uint4 ldg_nc_v4(const void *p)
 {
     return __ldg(reinterpret_cast<const uint4 *>(p));
+}
+
+// Release + acquire fence at GPU scope (orders this thread's, and by
+// cumulativity its CTA's barrier-ordered, memory accesses against the next).
+__device__ __forceinline__ void fence_acq_rel_gpu()
+{
+    asm volatile("fence.acq_rel.gpu;" ::: "memory");
 }
 
 // Streaming load: read once, do not keep in L1.  Volatile, so a load

@@ -41,15 +41,18 @@ __device__ __forceinline__ void splitk_finish(const Geom &L, SplitK sk, int row0
                                               uint16_t *__restrict__ y)
 {
     __shared__ unsigned s_last;
-    __threadfence();
     __syncthreads();
     if (threadIdx.x == 0) {
-        unsigned prev = atomicAdd(&sk.counters[blockIdx.x], 1u);
+        // the barrier orders the CTA's partial stores before this thread's
+        // release fence, which publishes them with the counter increment;
+        // the last CTA's acquire fence orders its reads after all of them
+        fence_acq_rel_gpu();
+        const unsigned prev = atomicAdd(&sk.counters[blockIdx.x], 1u);
         s_last = (prev == gridDim.y - 1) ? 1u : 0u;
+        if (s_last) fence_acq_rel_gpu();
     }
     __syncthreads();
     if (!s_last) return;
-    __threadfence();
     const int ks = gridDim.y;
     const size_t vstride = (size_t)L.rows8 * batch / 4;
     const float4 *base = reinterpret_cast<const float4 *>(sk.partials + (size_t)row0 * batch);
@@ -93,36 +96,91 @@ __device__ __forceinline__ void unpack8(uint4 c, uint32_t w[8])
 //
 // For one block of 32 groups the CTA tabulates L_k[g][c] = <C_k[c], x_g> for
 // both codebooks (2 x 256 x 32 fp32 = 64 KiB of shared memory), laid out
-// lane-private: entry (k, c, lane) at word (k*256 + c)*32 + lane, so lane l
+// lane-private: entry (k, c, g) at word (k*256 + c)*32 + g, so lane l
 // (group 32*gb + l) always reads bank l and random codes never conflict.
 // A row's contribution from the block is then two table reads per group.
+//
+// The tables are one small matrix product, T[g][k*256 + c] =
+// sum_j x_g[j] C_k[c][j] (32 x 512, inner size 8), computed with
+// mma.sync m16n8k8 (binary16 operands, fp32 accumulation; each product of
+// two binary16 values is exact in fp32).  For each codeword it holds, the
+// accumulator fragment gives a lane groups gid, gid+8, gid+16, gid+24 (gid =
+// lane / 4), while the four lanes of a quad hold four different codewords.
+// Lanes rotate their four group slots by their index within the quad before
+// storing, so every store instruction covers 32 distinct groups, i.e. 32
+// distinct banks.  (A 16-byte store of a lane's four groups cannot be made
+// conflict-free: the eight lanes of a store phase would write eight groups
+// four times over, in four rows.)
 // grid = (row ranges, group blocks); each CTA is one split of the K sum.
+// Code chunks stream through a per-warp register ring, issued before the
+// CTA waits on the previous launch.
 // ---------------------------------------------------------------------------
 constexpr int kLutWarps = 8;
-constexpr int kLutMaxTilesPerWarp = 12;  // row tiles per CTA <= 8 warps x 12
+constexpr int kLutRing = 2;  // quads of code chunks (4 row tiles) in flight per warp
 
-__global__ void __launch_bounds__(kLutWarps * 32)
+// Reduce-scatter of 32 values per lane over the warp: lane l returns the
+// sum over all lanes of a[l].  Five butterfly levels; at each, a lane keeps
+// the half of its values selected by its own lane bit and adds the partner's
+// copy of that half.  16 + 8 + 4 + 2 + 1 shuffles, all of a level independent.
+__device__ __forceinline__ float warp_reduce32(float a[32], int lane)
+{
+    float b[16], c[8], d[4], e[2];
+    bool h = lane & 16;
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+        b[i] = (h ? a[i + 16] : a[i]) + __shfl_xor_sync(0xffffffffu, h ? a[i] : a[i + 16], 16);
+    h = lane & 8;
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+        c[i] = (h ? b[i + 8] : b[i]) + __shfl_xor_sync(0xffffffffu, h ? b[i] : b[i + 8], 8);
+    h = lane & 4;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        d[i] = (h ? c[i + 4] : c[i]) + __shfl_xor_sync(0xffffffffu, h ? c[i] : c[i + 4], 4);
+    h = lane & 2;
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+        e[i] = (h ? d[i + 2] : d[i]) + __shfl_xor_sync(0xffffffffu, h ? d[i] : d[i + 2], 2);
+    h = lane & 1;
+    return (h ? e[1] : e[0]) + __shfl_xor_sync(0xffffffffu, h ? e[0] : e[1], 1);
+}
+
+// D = A(16x8, row) * B(8x8, col), binary16 in, fp32 out (no addend).
+__device__ __forceinline__ void mma_m16n8k8(float d[4], uint32_t a0, uint32_t a1, uint32_t b0)
+{
+    asm("mma.sync.aligned.m16n8k8.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5}, {%6}, {%7,%7,%7,%7};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a0), "r"(a1), "r"(b0), "f"(0.f));
+}
+
+__global__ void __launch_bounds__(kLutWarps * 32, 2)
 gemv_2x8_lut_kernel(Geom L, const uint4 *__restrict__ packed, const uint4 *__restrict__ cb,
                     const uint16_t *__restrict__ scales, const uint16_t *__restrict__ x,
                     uint16_t *__restrict__ y, SplitK sk, int rt_per_cta)
 {
-    extern __shared__ float lut[];  // [2][256][32] tables
-    __shared__ uint4 scb[512];      // both codebooks, binary16
-    __shared__ uint4 xs[32];        // activations of the block's 32 groups
+    extern __shared__ float lut[];       // [2][256][32] tables
+    __shared__ uint4 scb[512];           // both codebooks, binary16, row k*256 + c
+    __shared__ uint4 xs[32];             // activations of the block's 32 groups
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gb = blockIdx.y;
     const int rt0 = blockIdx.x * rt_per_cta;
     const int rt1 = min(L.rtiles, rt0 + rt_per_cta);
-    // Weights first: this warp's code chunks (row tiles rt0 + warp + 8j) and
-    // the codebooks are requested before anything waits, so their latency
-    // hides behind the table build.
-    uint4 chunk[kLutMaxTilesPerWarp];
-#pragma unroll
-    for (int j = 0; j < kLutMaxTilesPerWarp; ++j) {
-        const int rt = rt0 + warp + j * kLutWarps;
-        chunk[j] = (rt < rt1) ? ldg_stream_v4(packed + (size_t)rt * L.gp + gb * 32 + lane) : make_uint4(0, 0, 0, 0);
-    }
+    // this warp's row quads (4 row tiles, 32 rows) start at row tile
+    // rt0 + 4 (warp + kLutWarps j), j < nq; tiles at or past rt1 read as zero
+    const int nq = ((rt1 - rt0 + 3) / 4 - warp + kLutWarps - 1) / kLutWarps;
+    const uint4 *src = packed + (size_t)(rt0 + 4 * warp) * L.gp + gb * 32 + lane;
+    const size_t qstep = (size_t)4 * kLutWarps * L.gp;
+    const int tile_lim = rt1 - rt0 - 4 * warp;  // tile 4 kLutWarps j + t exists iff below this
+    // codebooks first: the table build needs them, the lookups come later
     const uint4 cw0 = ldg_stream_v4(cb + threadIdx.x), cw1 = ldg_stream_v4(cb + 256 + threadIdx.x);
+    uint4 ring[kLutRing][4];
+#pragma unroll
+    for (int i = 0; i < kLutRing; ++i)
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+            ring[i][t] = (i < nq && 4 * kLutWarps * i + t < tile_lim)
+                             ? ldg_stream_v4(src + i * qstep + (size_t)t * L.gp)
+                             : make_uint4(0, 0, 0, 0);
     grid_dependency_wait();  // x, y and the workspace follow the previous launch
     grid_launch_dependents();
     if (threadIdx.x < 32) {
@@ -132,54 +190,79 @@ gemv_2x8_lut_kernel(Geom L, const uint4 *__restrict__ packed, const uint4 *__res
     scb[threadIdx.x] = cw0;
     scb[256 + threadIdx.x] = cw1;
     __syncthreads();
-    // Both tables in one pass.  Thread t always computes group l = t % 32
-    // (its 8 activations stay in registers); entry e = t + 256 i is codeword
-    // kc = t / 32 + 8 i of codebook kc / 256, read as a broadcast.
     {
-        const int l = threadIdx.x & 31;
-        float xv[8];
-        {
-            const uint4 v = xs[l];
-            const float2 a = h2f2(v.x), b = h2f2(v.y), c = h2f2(v.z), d = h2f2(v.w);
-            xv[0] = a.x; xv[1] = a.y; xv[2] = b.x; xv[3] = b.y; xv[4] = c.x; xv[5] = c.y; xv[6] = d.x; xv[7] = d.y;
+        // warp w fills codewords kc in [64w, 64w + 64) for all 32 groups
+        const int gid = lane >> 2, t4 = lane & 3;
+        const uint32_t *xw = reinterpret_cast<const uint32_t *>(xs);
+        const uint32_t *cbw = reinterpret_cast<const uint32_t *>(scb);
+        uint32_t a[2][2];
+#pragma unroll
+        for (int m = 0; m < 2; ++m) {
+            a[m][0] = xw[(16 * m + gid) * 4 + t4];
+            a[m][1] = xw[(16 * m + gid + 8) * 4 + t4];
         }
-#pragma unroll 8
-        for (int i = 0; i < 2 * 256 * 32 / (kLutWarps * 32); ++i) {
-            const int kc = (threadIdx.x >> 5) + kLutWarps * i;
-            const uint4 w = scb[kc];
-            const float2 a = h2f2(w.x), b = h2f2(w.y), c = h2f2(w.z), d = h2f2(w.w);
-            float acc = a.x * xv[0];
-            acc = fmaf(a.y, xv[1], acc); acc = fmaf(b.x, xv[2], acc); acc = fmaf(b.y, xv[3], acc);
-            acc = fmaf(c.x, xv[4], acc); acc = fmaf(c.y, xv[5], acc); acc = fmaf(d.x, xv[6], acc);
-            acc = fmaf(d.y, xv[7], acc);
-            lut[kc * 32 + l] = acc;
+        const int kc0 = warp * 64;
+        float *dst = lut + (kc0 + 2 * t4) * 32 + gid;
+        int off[4];
+#pragma unroll
+        for (int s = 0; s < 4; ++s) off[s] = 8 * ((t4 + s) & 3);
+#pragma unroll
+        for (int n = 0; n < 8; ++n) {
+            const uint32_t b0 = cbw[(kc0 + 8 * n + gid) * 4 + t4];
+            float d0[4], d1[4];
+            mma_m16n8k8(d0, a[0][0], a[0][1], b0);  // groups gid, gid + 8
+            mma_m16n8k8(d1, a[1][0], a[1][1], b0);  // groups gid + 16, gid + 24
+#pragma unroll
+            for (int b = 0; b < 2; ++b) {
+                // v[q] belongs to group gid + 8q, codeword kc0 + 8n + 2 t4 + b
+                const float v[4] = {d0[b], d0[2 + b], d1[b], d1[2 + b]};
+                float r[4], w[4];
+#pragma unroll
+                for (int s = 0; s < 4; ++s) r[s] = (t4 & 1) ? v[(s + 1) & 3] : v[s];
+#pragma unroll
+                for (int s = 0; s < 4; ++s) w[s] = (t4 & 2) ? r[(s + 2) & 3] : r[s];
+                // w[s] = v[(t4 + s) & 3]: slot s writes group gid + off[s]
+#pragma unroll
+                for (int s = 0; s < 4; ++s) dst[n * 256 + b * 32 + off[s]] = w[s];
+            }
         }
     }
     __syncthreads();
     const float *lut0 = lut + lane;
     const float *lut1 = lut + 256 * 32 + lane;
     float *part = sk.partials + (size_t)gb * L.rows8;
+    for (int j0 = 0; j0 < nq; j0 += kLutRing) {
 #pragma unroll
-    for (int j = 0; j < kLutMaxTilesPerWarp; ++j) {
-        const int rt = rt0 + warp + j * kLutWarps;
-        if (rt >= rt1) break;
-        const uint32_t v[4] = {chunk[j].x, chunk[j].y, chunk[j].z, chunk[j].w};
-        float acc[8];
+        for (int i = 0; i < kLutRing; ++i) {
+            const int j = j0 + i;
+            if (j >= nq) break;
+            float acc[32];  // acc[8 t + r]: row r of tile t of the quad, this lane's group
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            acc[2 * i] = lut0[(v[i] & 0xff) * 32] + lut1[((v[i] >> 8) & 0xff) * 32];
-            acc[2 * i + 1] = lut0[((v[i] >> 16) & 0xff) * 32] + lut1[(v[i] >> 24) * 32];
-        }
-        const float r = warp_reduce8(acc, lane);
-        if ((lane & 3) == 0) {
-            const int row = rt * 8 + reduced_row_of_lane(lane);
-            if (gridDim.y == 1) {
-                if (row < L.out) {
-                    const float sc = scales ? __half2float(__ushort_as_half(scales[row])) : 1.f;
-                    y[row] = __half_as_ushort(__float2half_rn(sc * r));
+            for (int t = 0; t < 4; ++t) {
+                const uint32_t v[4] = {ring[i][t].x, ring[i][t].y, ring[i][t].z, ring[i][t].w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    acc[8 * t + 2 * q] = lut0[(v[q] & 0xff) * 32] + lut1[((v[q] >> 8) & 0xff) * 32];
+                    acc[8 * t + 2 * q + 1] = lut0[((v[q] >> 16) & 0xff) * 32] + lut1[(v[q] >> 24) * 32];
                 }
-            } else {
-                part[row] = r;
+            }
+            const int jn = j + kLutRing;
+#pragma unroll
+            for (int t = 0; t < 4; ++t)
+                ring[i][t] = (jn < nq && 4 * kLutWarps * jn + t < tile_lim)
+                                 ? ldg_stream_v4(src + jn * qstep + (size_t)t * L.gp)
+                                 : make_uint4(0, 0, 0, 0);
+            const float r = warp_reduce32(acc, lane);
+            const int row = (rt0 + 4 * (warp + kLutWarps * j)) * 8 + lane;
+            if (row < rt1 * 8) {
+                if (gridDim.y == 1) {
+                    if (row < L.out) {
+                        const float sc = scales ? __half2float(__ushort_as_half(scales[row])) : 1.f;
+                        y[row] = __half_as_ushort(__float2half_rn(sc * r));
+                    }
+                } else {
+                    part[row] = r;
+                }
             }
         }
     }
@@ -468,13 +551,11 @@ GemvPlan plan_gemv(const Geom &g, int batch)
     if (batch == 1 && g.K == 2) {
         p.path = kLut2x8;
         p.ks = g.gblocks;
-        const long pairs = (long)g.rtiles * g.gblocks;
-        int rt = (int)((pairs + 299) / 300);  // ~300 CTAs, enough rows to amortise the table
-        rt = max(rt, 8);
-        rt = min(rt, kLutWarps * kLutMaxTilesPerWarp);
-        rt = min(rt, g.rtiles);
-        p.rt_per_cta = rt;
-        p.grid_x = (g.rtiles + rt - 1) / rt;
+        // two CTAs per SM in one wave: every CTA builds its tables once, and
+        // a third CTA per SM fits, so the next launch can start early
+        const int ranges = max(1, min(g.rtiles, 2 * kNumSMs / g.gblocks));
+        p.rt_per_cta = ((g.rtiles + ranges - 1) / ranges + 3) & ~3;  // whole quads of tiles
+        p.grid_x = (g.rtiles + p.rt_per_cta - 1) / p.rt_per_cta;
         p.per_split = 1;
     } else {
         p.path = kTensor;
