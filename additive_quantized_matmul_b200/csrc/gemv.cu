@@ -405,12 +405,20 @@ gemv_tc_kernel(Geom L, const uint4 *__restrict__ packed, const uint4 *__restrict
                             cp_async16(a0 + sw128(rt_l * 8 + r, gi), live ? (const void *)(cb + wd[r]) : (const void *)cb,
                                        live ? 16u : 0u);
                     } else {
+                        // every codeword read is issued before the first tile
+                        // store: the codebooks and the tile share one shared
+                        // array, so a store would otherwise hold back the
+                        // next row's reads and serialise the eight rows
+                        uint4 c0[8], c1[8];
 #pragma unroll
                         for (int r = 0; r < 8; ++r) {
-                            const uint4 v = live ? add_round_h8(scb[wd[r] & 0xff], scb[256 + (wd[r] >> 8)])
-                                                 : make_uint4(0, 0, 0, 0);
-                            *reinterpret_cast<uint4 *>(A + sw128(rt_l * 8 + r, gi)) = v;
+                            c0[r] = scb[wd[r] & 0xff];
+                            c1[r] = scb[256 + (wd[r] >> 8)];
                         }
+#pragma unroll
+                        for (int r = 0; r < 8; ++r)
+                            *reinterpret_cast<uint4 *>(A + sw128(rt_l * 8 + r, gi)) =
+                                live ? add_round_h8(c0[r], c1[r]) : make_uint4(0, 0, 0, 0);
                     }
                     // x rows of this stage: straight into the B tile when a row is
                     // 16 or 32 bytes, else the raw rows into the stage's x slot
@@ -561,9 +569,10 @@ GemvPlan plan_gemv(const Geom &g, int batch)
         p.path = kTensor;
         const int mtiles = (g.out + kTcBM - 1) / kTcBM;
         const int nst = (g.G + 7) / 8;
-        // ~1024 CTAs at batch 1 (short tail, many gathers in flight), fewer
-        // splits as the batch grows (split-K partials scale with the batch)
-        const int target = 1024 / max(1, batch / 2);
+        // ~1024 CTAs at batch 1 (short tail, many gathers in flight), ~4 per
+        // SM above it: the decoders of one CTA wait on shared-memory and L2
+        // latency, so several CTAs per SM keep the pipes busy
+        const int target = batch == 1 ? 1024 : 4 * kNumSMs;
         int ks = (target + mtiles - 1) / mtiles;
         ks = max(1, min(ks, (nst + 7) / 8));  // at least 8 stages per CTA: the ring fills
         p.per_split = (nst + ks - 1) / ks;
