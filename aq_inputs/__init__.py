@@ -142,8 +142,20 @@ def workload(name: str) -> dict:
             for tag, (o, i) in LLAMA2_7B_BLOCK.items():
                 layers.append((f"{tag}-{K}x{B}", LayerSpec(o, i, K, B)))
         return {"layers": layers, "n": [512, 2048], "seed": 1004}
+    if name == "llama2-7b-block":
+        # the seven linears of one decoder block per scheme, run as a chain:
+        # each entry is (tag, spec, input) with input None for the block's
+        # input vector, else the tag of the layer whose output it consumes
+        # (q, k, v read the block input; o reads v; gate and up read o;
+        # down reads up)
+        src = {"q": None, "k": None, "v": None, "o": "v", "gate": "o", "up": "o", "down": "up"}
+        chains = []
+        for K, B in ((1, 16), (2, 8)):
+            chains.append((f"block-{K}x{B}",
+                           [(tag, LayerSpec(o, i, K, B), src[tag]) for tag, (o, i) in LLAMA2_7B_BLOCK.items()]))
+        return {"layers": [], "chains": chains, "n": [1], "seed": 1005}
     raise KeyError(name)
 
 
 WORKLOADS = ("tiny-2x8", "llama2-7b-1x16", "llama2-7b-mlp-2x8",
-             "llama2-70b-1x16", "llama2-7b-prefill")
+             "llama2-70b-1x16", "llama2-7b-prefill", "llama2-7b-block")

@@ -288,16 +288,19 @@ def run_gpu(args) -> None:
 
     # ---- units: one (layer shape, batch) product kind each, over a rotation
     #      set of copies at distinct addresses (> 3x L2 per shape) -----------
+    def device_layer(spec, seed):
+        desc = aq.LayerDesc.make(spec.out_features, spec.in_features, spec.num_codebooks, spec.nbits)
+        L = make_layer(spec, seed)
+        codes = torch.from_numpy(L.codes.view(np.int16) if spec.nbits > 8 else L.codes).to(dev)
+        packed = torch.empty(aq.aq_packed_codes_bytes(desc), dtype=torch.uint8, device=dev)
+        aq.aq_pack_codes(desc, codes, packed)
+        cb = torch.from_numpy(L.codebooks.view(np.int16)).to(dev)
+        sc = torch.from_numpy(L.scales.view(np.int16)).to(dev)
+        return desc, packed, cb, sc
+
     units = []
     for si, (tag, spec) in enumerate(wl["layers"]):
-        desc = aq.LayerDesc.make(spec.out_features, spec.in_features, spec.num_codebooks, spec.nbits)
-        L = make_layer(spec, (wl["seed"], rank, si))  # seeded per rank and shape
-        codes = torch.from_numpy(L.codes.view(np.int16) if spec.nbits > 8 else L.codes).to(dev)
-        packed0 = torch.empty(aq.aq_packed_codes_bytes(desc), dtype=torch.uint8, device=dev)
-        aq.aq_pack_codes(desc, codes, packed0)
-        cb0 = torch.from_numpy(L.codebooks.view(np.int16)).to(dev)
-        sc0 = torch.from_numpy(L.scales.view(np.int16)).to(dev)
-        del codes, L
+        desc, packed0, cb0, sc0 = device_layer(spec, (wl["seed"], rank, si))  # seeded per rank and shape
         lb = alg_bytes(spec, 0)
         ncopies = args.layers or max(3 if op == "gemm" else 4, int(3 * L2_BYTES / lb) + 1)
         copies = [(packed0.clone(), cb0.clone(), sc0.clone()) for _ in range(ncopies)]
@@ -307,21 +310,58 @@ def run_gpu(args) -> None:
             nbytes = (aq.aq_gemm_workspace_bytes(desc, n) if op == "gemm" else aq.aq_gemv_workspace_bytes(desc, n))
             units.append({
                 "tag": tag, "spec": spec, "n": n, "desc": desc, "copies": copies, "x": x,
+                "bytes": alg_bytes(spec, n), "flops": flops(spec, n),
                 "ys": [torch.empty(spec.out_features * n, dtype=torch.int16, device=dev) for _ in range(ncopies)],
                 "ws": torch.zeros(max(nbytes, 16), dtype=torch.uint8, device=dev),
                 # two events per group of same-shape launches (event nodes between
                 # every launch would add their own cost to each measurement)
                 "evs": [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)],
             })
+    # chained decoder blocks: one unit per scheme, each copy a whole block of
+    # layers whose inputs are the block input or an earlier layer's output
+    for ci, (tag, chain) in enumerate(wl.get("chains", [])):
+        layers = [device_layer(spec, (wl["seed"], rank, ci, li)) for li, (_, spec, _) in enumerate(chain)]
+        block_bytes = sum(alg_bytes(spec, 1) for _, spec, _ in chain)
+        ncopies = args.layers or max(4, int(3 * L2_BYTES / block_bytes) + 1)
+        copies = [[(p.clone(), c.clone(), q.clone()) for _, p, c, q in layers] for _ in range(ncopies)]
+        tags = [t for t, _, _ in chain]
+        wsb = max(aq.aq_gemv_workspace_bytes(d, 1) for d, _, _, _ in layers)
+        units.append({
+            "tag": tag, "n": 1, "copies": copies,
+            "chain": [(d, spec, None if s_ is None else tags.index(s_)) for (d, _, _, _), (_, spec, s_) in zip(layers, chain)],
+            "x": torch.from_numpy(make_activations(chain[0][1].in_features, 1, (wl["seed"], rank, ci)).view(np.int16)).to(dev),
+            "ys": [[torch.empty(spec.out_features, dtype=torch.int16, device=dev) for _, spec, _ in chain]
+                   for _ in range(ncopies)],
+            "bytes": block_bytes, "flops": sum(flops(spec, 1) for _, spec, _ in chain),
+            "ws": torch.zeros(max(wsb, 16), dtype=torch.uint8, device=dev),
+            "evs": [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)],
+        })
+        del layers
     torch.cuda.synchronize()
     stream = torch.cuda.Stream(device=dev)
 
-    def call(u, i, s):
+    def run(u, i, x_in, y_out, s):
+        """Copy i of unit u on stream s: one product, or a whole chained block
+        (whose last layer writes y_out, the others their own buffers)."""
+        if "chain" in u:
+            ys = u["ys"][i]
+            for li, (desc, spec, src) in enumerate(u["chain"]):
+                packed, cb, sc = u["copies"][i][li]
+                inp = x_in if src is None else ys[src]
+                out = y_out if li == len(u["chain"]) - 1 else ys[li]
+                aq.aq_gemv(desc, packed, cb, sc, inp, 1, out, u["ws"], stream=s)
+            return
         packed, cb, sc = u["copies"][i]
         if op == "gemm":
-            aq.aq_gemm(u["desc"], packed, cb, sc, u["x"], u["n"], u["ys"][i], u["ws"], stream=s)
+            aq.aq_gemm(u["desc"], packed, cb, sc, x_in, u["n"], y_out, u["ws"], stream=s)
         else:
-            aq.aq_gemv(u["desc"], packed, cb, sc, u["x"], u["n"], u["ys"][i], u["ws"], stream=s)
+            aq.aq_gemv(u["desc"], packed, cb, sc, x_in, u["n"], y_out, u["ws"], stream=s)
+
+    def out_buf(u, i):
+        return u["ys"][i][-1] if "chain" in u else u["ys"][i]
+
+    def call(u, i, s):
+        run(u, i, u["x"], out_buf(u, i), s)
 
     def one_step(record: bool):
         s = torch.cuda.current_stream()
@@ -373,12 +413,15 @@ def run_gpu(args) -> None:
     step_bytes = step_flops = 0
     for u in units:
         us = 1e3 * u["evs"][0].elapsed_time(u["evs"][1]) / len(u["copies"])
-        nb, nf = alg_bytes(u["spec"], u["n"]), flops(u["spec"], u["n"])
+        nb, nf = u["bytes"], u["flops"]
         step_bytes += nb * len(u["copies"])
         step_flops += nf * len(u["copies"])
         k = {"layer": u["tag"], "n": u["n"], "us_per_layer": round(us, 3),
              "gbs": round(nb / (us * 1e-6) / 1e9, 1), "tflops": round(nf / (us * 1e-6) / 1e12, 2),
              "bytes_per_call": nb, "copies": len(u["copies"]), "total_us": us * len(u["copies"])}
+        if "chain" in u:  # one call is a whole block of layers
+            k["layers_per_call"] = len(u["chain"])
+            k["us_per_block"] = k.pop("us_per_layer")
         k["frac_hbm"] = round(k["gbs"] / peaks["hbm_gbs"], 4)
         k["frac_tensor"] = round(k["tflops"] / peaks["bf16_tflops_sustained"], 4)
         kernels.append(k)
@@ -404,7 +447,7 @@ def run_gpu(args) -> None:
     e2e = None
     if not args.skip_e2e:
         hx = [torch.empty((len(u["copies"]), u["x"].numel()), dtype=torch.int16).pin_memory() for u in units]
-        hy = [torch.empty((len(u["copies"]), u["ys"][0].numel()), dtype=torch.int16).pin_memory() for u in units]
+        hy = [torch.empty((len(u["copies"]), out_buf(u, 0).numel()), dtype=torch.int16).pin_memory() for u in units]
         dx = [torch.empty(h.shape, dtype=torch.int16, device=dev) for h in hx]
         dy = [torch.empty(h.shape, dtype=torch.int16, device=dev) for h in hy]
         for h, u in zip(hx, units):
@@ -416,12 +459,10 @@ def run_gpu(args) -> None:
         def e2e_step():
             for d, h in zip(dx, hx):
                 d.copy_(h, non_blocking=True)
+            s = torch.cuda.current_stream()
             for ui, u in enumerate(units):
-                for i, (packed, cb, sc) in enumerate(u["copies"]):
-                    if op == "gemm":
-                        aq.aq_gemm(u["desc"], packed, cb, sc, dx[ui][i], u["n"], dy[ui][i], u["ws"])
-                    else:
-                        aq.aq_gemv(u["desc"], packed, cb, sc, dx[ui][i], u["n"], dy[ui][i], u["ws"])
+                for i in range(len(u["copies"])):
+                    run(u, i, dx[ui][i], dy[ui][i], s)
             for h, d in zip(hy, dy):
                 h.copy_(d, non_blocking=True)
 
@@ -442,11 +483,13 @@ def run_gpu(args) -> None:
                "api": "additive_quantized_matmul_b200 (C ABI via ctypes), eager, pinned host buffers"}
 
     cpu = None
-    if rank == 0 and world == 1 and not args.skip_cpu and op == "gemv":
+    if rank == 0 and world == 1 and not args.skip_cpu and args.workload == WORKLOAD:
         cpu = cpu_baseline()
 
     if rank == 0:
-        spec0 = wl["layers"][0][1]
+        shapes = [f"{t} {sp.scheme} g8" for t, sp in wl["layers"]]
+        shapes += [f"{t}: " + ", ".join(f"{lt} {sp.out_features}x{sp.in_features} {sp.scheme}" for lt, sp, _ in ch)
+                   for t, ch in wl.get("chains", [])]
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": unit, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
@@ -454,9 +497,12 @@ def run_gpu(args) -> None:
             "scaling": "weak", "vs_baseline": None, "dtype": "f16", "accumulate": "f32",
             "data": "synthetic",
             "config": {"workload": args.workload,
-                       "layers": [f"{t} {s.scheme} g8" for t, s in wl["layers"]],
+                       "layers": shapes,
                        "n": list(wl["n"]),
                        "copies_per_shape": [len(u["copies"]) for u in units[::len(wl["n"])]],
+                       **({"chain": "per block: q, k, v read the block input; o reads v; gate and up "
+                                    "read o; down reads up (one stream, each launch waits on the previous)"}
+                          if wl.get("chains") else {}),
                        "l2": "inputs larger than L2: per shape, copies at distinct addresses whose "
                              "bytes exceed 3x the 126 MB L2, visited in turn before any is re-read",
                        "parallelism": f"replicas x{world} (independent layers per rank)"},
@@ -480,7 +526,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=WORKLOAD,
                     help="llama2-7b-1x16 (default), llama2-7b-mlp-2x8, llama2-70b-1x16, "
-                         "llama2-7b-prefill, tiny-2x8")
+                         "llama2-7b-prefill, llama2-7b-block, tiny-2x8")
     ap.add_argument("--layers", type=int, default=0, help="copies per shape (0: > 3x L2)")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--skip-e2e", action="store_true")
