@@ -233,18 +233,20 @@ int aqo_matmul(int64_t out, int64_t in, int K, int B, const void *codes,
 /* ------------------------------------------------------------------------ */
 /* Packed code layout (the library's documented interface).                 */
 /*                                                                          */
-/* Each group (o, g) has one 16-bit word: for one 16-bit codebook the code  */
-/* itself, for two 8-bit codebooks code[k=0] | code[k=1] << 8.  Rows are    */
+/* Each group (o, g) has one word of W = K*B/8 bytes holding its K codes,   */
+/* code k in bits [k*B, (k+1)*B) (1x16: the code; 2x8: c0 | c1 << 8; 1x8:   */
+/* one byte; 2x16: c0 | c1 << 16; 8x8: eight bytes, c0 first).  Rows are    */
 /* padded to a multiple of 8 and groups to a multiple of 32 with zero words.*/
 /* Word (o, g) is stored little-endian at byte                              */
-/*   ((o / 8) * (Gp / 32) + g / 32) * 512 + (g % 32) * 16 + (o % 8) * 2     */
-/* where Gp is the padded group count: a 512-byte tile holds 8 rows x 32    */
-/* groups, each 16-byte chunk holds one group for 8 consecutive rows.       */
+/*   ((o / 8) * (Gp / 32) + g / 32) * 256 W + (g % 32) * 8 W + (o % 8) * W  */
+/* where Gp is the padded group count: a 256 W-byte tile holds 8 rows x 32  */
+/* groups, each 8 W-byte chunk holds one group for 8 consecutive rows.      */
 /* ------------------------------------------------------------------------ */
 
 static int packed_scheme_ok(int K, int B)
 {
-    return (K == 1 && B == 16) || (K == 2 && B == 8);
+    return (K == 1 && B == 16) || (K == 2 && B == 8) || (K == 1 && B == 8) ||
+           (K == 2 && B == 16) || (K == 8 && B == 8);
 }
 
 int64_t aqo_packed_bytes(int64_t out, int64_t in, int K, int B)
@@ -252,12 +254,12 @@ int64_t aqo_packed_bytes(int64_t out, int64_t in, int K, int B)
     if (check_scheme(out, in, K, B) || !packed_scheme_ok(K, B)) return -1;
     int64_t rows = (out + 7) / 8 * 8;
     int64_t gp = (in / AQO_GROUP + 31) / 32 * 32;
-    return rows * gp * 2;
+    return rows * gp * (K * B / 8);
 }
 
-static int64_t packed_offset(int64_t o, int64_t g, int64_t gp)
+static int64_t packed_offset(int64_t o, int64_t g, int64_t gp, int64_t W)
 {
-    return ((o / 8) * (gp / 32) + g / 32) * 512 + (g % 32) * 16 + (o % 8) * 2;
+    return ((o / 8) * (gp / 32) + g / 32) * 256 * W + (g % 32) * 8 * W + (o % 8) * W;
 }
 
 int aqo_pack(int64_t out, int64_t in, int K, int B, const void *codes, uint8_t *packed)
@@ -266,19 +268,15 @@ int aqo_pack(int64_t out, int64_t in, int K, int B, const void *codes, uint8_t *
     if (nbytes < 0) return -1;
     int64_t G = in / AQO_GROUP;
     int64_t gp = (G + 31) / 32 * 32;
+    int64_t W = K * B / 8;
     memset(packed, 0, (size_t)nbytes);
     for (int64_t o = 0; o < out; ++o) {
         for (int64_t g = 0; g < G; ++g) {
-            uint32_t word;
-            if (K == 1) {
-                word = code_at(codes, B, o * G + g);
-            } else {
-                word = code_at(codes, B, (o * G + g) * 2 + 0) |
-                       (code_at(codes, B, (o * G + g) * 2 + 1) << 8);
-            }
-            int64_t at = packed_offset(o, g, gp);
-            packed[at] = (uint8_t)(word & 0xff);
-            packed[at + 1] = (uint8_t)(word >> 8);
+            uint64_t word = 0;
+            for (int k = 0; k < K; ++k)
+                word |= (uint64_t)code_at(codes, B, (o * G + g) * K + k) << (k * B);
+            int64_t at = packed_offset(o, g, gp, W);
+            for (int64_t b = 0; b < W; ++b) packed[at + b] = (uint8_t)(word >> (8 * b));
         }
     }
     return 0;
@@ -289,15 +287,19 @@ int aqo_unpack(int64_t out, int64_t in, int K, int B, const uint8_t *packed, voi
     if (aqo_packed_bytes(out, in, K, B) < 0) return -1;
     int64_t G = in / AQO_GROUP;
     int64_t gp = (G + 31) / 32 * 32;
+    int64_t W = K * B / 8;
+    uint64_t mask = (B == 16) ? 0xffffu : 0xffu;
     for (int64_t o = 0; o < out; ++o) {
         for (int64_t g = 0; g < G; ++g) {
-            int64_t at = packed_offset(o, g, gp);
-            uint32_t word = (uint32_t)packed[at] | ((uint32_t)packed[at + 1] << 8);
-            if (K == 1) {
-                ((uint16_t *)codes)[o * G + g] = (uint16_t)word;
-            } else {
-                ((uint8_t *)codes)[(o * G + g) * 2 + 0] = (uint8_t)(word & 0xff);
-                ((uint8_t *)codes)[(o * G + g) * 2 + 1] = (uint8_t)(word >> 8);
+            int64_t at = packed_offset(o, g, gp, W);
+            uint64_t word = 0;
+            for (int64_t b = 0; b < W; ++b) word |= (uint64_t)packed[at + b] << (8 * b);
+            for (int k = 0; k < K; ++k) {
+                uint64_t c = (word >> (k * B)) & mask;
+                if (B <= 8)
+                    ((uint8_t *)codes)[(o * G + g) * K + k] = (uint8_t)c;
+                else
+                    ((uint16_t *)codes)[(o * G + g) * K + k] = (uint16_t)c;
             }
         }
     }

@@ -93,7 +93,7 @@ def test_bitrate_page_examples(golden_dir):
         assert oracle.bits_per_weight(case["K"], case["B"], 8) == case["bits_per_weight"]
 
 
-@pytest.mark.parametrize("K,B", [(1, 16), (2, 8)])
+@pytest.mark.parametrize("K,B", [(1, 16), (2, 8), (1, 8), (2, 16), (8, 8)])
 @pytest.mark.parametrize("out,inp", [(4096, 4096), (11008, 4096), (8, 256)])
 def test_packed_size_matches_bitrate(K, B, out, inp):
     # aligned shapes carry no padding: bytes * 8 / weights == K * B / 8
@@ -238,7 +238,8 @@ def _dyadic_layer(out, inp, K, B, seed):
 
 
 @pytest.mark.parametrize("out,inp,K,B,n", [(1, 8, 1, 2, 1), (3, 16, 2, 2, 2), (4, 16, 2, 8, 3),
-                                           (2, 8, 1, 8, 1), (4, 8, 2, 2, 4)])
+                                           (2, 8, 1, 8, 1), (4, 8, 2, 2, 4), (2, 16, 8, 8, 2),
+                                           (3, 8, 2, 16, 1), (2, 16, 4, 3, 2)])
 def test_matmul_brute_force_exact(out, inp, K, B, n):
     """Triple loop over (g, j, k) in exact rationals, without forming W."""
     codes, cb, s = _dyadic_layer(out, inp, K, B, out * 100 + inp + K + B)
@@ -253,6 +254,38 @@ def test_matmul_brute_force_exact(out, inp, K, B, n):
                     for k in range(K):
                         acc += Fraction(float(cb[k, codes[o, g, k], j])) * Fraction(float(x[8 * g + j, b]))
             assert y[o, b] == float(Fraction(float(s[o])) * acc)
+
+
+def test_decode_eight_codebooks_one_rounding_of_exact_sum():
+    """K = 8: each weight is the exact sum of eight binary16 terms of widely
+    different magnitudes, rounded once (checked against numpy's binary16
+    conversion of the exact rational sum, which is exact in a double)."""
+    rng = np.random.default_rng(21)
+    K, B = 8, 8
+    mant = rng.integers(1024, 2048, size=(K, 1 << B, 8))
+    expo = rng.integers(-24, 6, size=(K, 1 << B, 8))
+    sign = rng.choice([-1.0, 1.0], size=(K, 1 << B, 8))
+    cb = (sign * mant * np.exp2(expo - 10.0)).astype(np.float16)
+    assert np.all(np.isfinite(cb))
+    out, G = 6, 5
+    codes = rng.integers(0, 1 << B, size=(out, G, K)).astype(np.uint8)
+    w = oracle.decode(codes, cb)
+    for o in range(out):
+        for g in range(G):
+            for j in range(8):
+                exact = sum(Fraction(float(cb[k, codes[o, g, k], j])) for k in range(K))
+                assert w[o, 8 * g + j].view(np.uint16) == np.float16(float(exact)).view(np.uint16)
+
+
+def test_decode_eight_codebooks_rounds_the_sum_not_the_terms():
+    # 1 + 7 * 2^-12 = 1 + 1.75 ulp: one rounding gives 1 + 2 ulp, while
+    # rounding after every addition would stay at 1
+    cb = np.zeros((8, 256, 8), dtype=np.float16)
+    cb[0, 1, 0] = 1.0
+    cb[1:, 1, 0] = 2.0 ** -12
+    codes = np.ones((1, 1, 8), dtype=np.uint8)
+    w = oracle.decode(codes, cb)
+    assert float(w[0, 0]) == 1.0 + 2.0 ** -9
 
 
 def test_matmul_uses_rounded_weights():
@@ -335,8 +368,38 @@ def test_pack_hand_worked_offsets(golden_dir):
     assert int(p2.astype(np.int64).sum()) == 0xAB + 0xCD
 
 
+def test_pack_hand_worked_offsets_wide_words(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "pack_offsets_wide.json")))
+    L = g["layer"]
+    G = L["in"] // 8
+    for sch in g["schemes"]:
+        K, B, W = sch["K"], sch["B"], sch["W"]
+        assert oracle.packed_bytes(L["out"], L["in"], K, B) == sch["packed_bytes"]
+        dt = np.uint8 if B <= 8 else np.uint16
+        # one nonzero code at a time: its bytes must sit at the worked offset
+        for key, byte in g["offsets_bytes"][str(W)].items():
+            o, gg = map(int, key.split(","))
+            codes = np.zeros((L["out"], G, K), dtype=dt)
+            codes[o, gg, 0] = 0x5A
+            p = oracle.pack(codes, K, B)
+            assert p[byte] == 0x5A and int(p.astype(np.int64).sum()) == 0x5A, (K, B, key)
+        for e in g["offsets_in_words"]:
+            codes = np.zeros((L["out"], G, K), dtype=dt)
+            codes[e["o"], e["g"], 0] = 0x33
+            p = oracle.pack(codes, K, B)
+            assert p[e["word"] * W] == 0x33, (K, B, e)
+    # byte order inside a word
+    c = np.zeros((L["out"], G, 2), dtype=np.uint16)
+    c[0, 0] = (0x1234, 0xABCD)
+    assert list(oracle.pack(c, 2, 16)[:4]) == [0x34, 0x12, 0xCD, 0xAB]
+    c8 = np.zeros((L["out"], G, 8), dtype=np.uint8)
+    c8[0, 0] = np.arange(1, 9)
+    assert list(oracle.pack(c8, 8, 8)[:8]) == list(range(1, 9))
+
+
 @pytest.mark.parametrize("out,inp,K,B", [(1, 8, 1, 16), (20, 520, 1, 16), (20, 520, 2, 8),
-                                         (37, 8 * 45, 2, 8), (256, 512, 2, 8)])
+                                         (37, 8 * 45, 2, 8), (256, 512, 2, 8), (20, 520, 1, 8),
+                                         (37, 8 * 45, 2, 16), (20, 520, 8, 8), (1, 8, 8, 8)])
 def test_pack_roundtrip_and_padding(out, inp, K, B):
     spec = LayerSpec(out, inp, K, B)
     layer = make_layer(spec, out + inp)
@@ -344,6 +407,6 @@ def test_pack_roundtrip_and_padding(out, inp, K, B):
     assert np.array_equal(oracle.unpack(packed, out, inp, K, B), layer.codes)
     rows = -(-out // 8) * 8
     gp = -(-(inp // 8) // 32) * 32
-    assert packed.size == rows * gp * 2
+    assert packed.size == rows * gp * K * B // 8
     # zero padding: the byte sum equals the code-byte sum
     assert int(packed.astype(np.int64).sum()) == int(layer.codes.view(np.uint8).astype(np.int64).sum())
