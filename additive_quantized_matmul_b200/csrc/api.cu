@@ -4,7 +4,7 @@
 // GPU; on error nothing is launched.  No exception crosses the interface.
 #include <stdint.h>
 
-#include "aq_common.cuh"
+#include "scheme.cuh"
 
 namespace {
 
@@ -20,8 +20,7 @@ aq_status check_desc(const aq_layer_desc *d)
     if (!d) return AQ_ERR_INVALID_ARG;
     if (d->out_features < 1 || d->in_features < 8 || d->in_features % 8) return AQ_ERR_INVALID_ARG;
     if (d->group_size != 8) return AQ_ERR_UNSUPPORTED;
-    const bool ok = (d->num_codebooks == 1 && d->nbits == 16) || (d->num_codebooks == 2 && d->nbits == 8);
-    if (!ok) return AQ_ERR_UNSUPPORTED;
+    if (!aqk::scheme_supported(d->num_codebooks, d->nbits)) return AQ_ERR_UNSUPPORTED;
     // keep every byte offset and element count within 64-bit range and the
     // per-row chunk count within 32-bit kernel indices
     if ((int64_t)d->out_features * d->in_features > (int64_t)1 << 40) return AQ_ERR_INVALID_ARG;
@@ -56,7 +55,7 @@ size_t aq_packed_codes_bytes(const aq_layer_desc *desc)
 {
     if (check_desc(desc) != AQ_OK) return 0;
     const Geom g = aqk::make_geom(*desc);
-    return (size_t)g.rows8 * g.gp * 2;
+    return (size_t)g.rows8 * g.gp * (g.K * g.B / 8);
 }
 
 size_t aq_gemv_workspace_bytes(const aq_layer_desc *desc, int batch)

@@ -1,11 +1,11 @@
 // Shared device/host helpers of the sm_100a additive-quantised product library.
 //
 // Packed code layout (documented in include/aq.h): for each 8-row tile rt and
-// each padded group g there is one 16-byte chunk holding the 16-bit words of
-// rows 8rt..8rt+7 for group g.  Chunk (rt, g) sits at chunk index rt*Gp + g
-// (equivalently byte ((o/8)*(Gp/32) + g/32)*512 + (g%32)*16 + (o%8)*2 for
-// word (o, g)), so 32 consecutive groups of one row tile are 512 contiguous
-// bytes: one warp-wide 128-bit load.
+// each padded group g there is one chunk of 8 W bytes (W = K*B/8 bytes per
+// word) holding the words of rows 8rt..8rt+7 for group g.  Chunk (rt, g)
+// sits at chunk index rt*Gp + g, so 32 consecutive groups of one row tile
+// are contiguous (512 bytes for the 2-bit schemes: one warp-wide 128-bit
+// load).
 #pragma once
 
 #include <cuda_fp16.h>

@@ -16,6 +16,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include "scheme.cuh"
 #include "tc_common.cuh"
 
 namespace aqk {
@@ -29,9 +30,9 @@ constexpr int kTileABytes = kBM * kBK * 2;  // 16 KiB
 constexpr int kTileBBytes = kBK * kBN * 2;  // 16 KiB
 // ---- kernel -----------------------------------------------------------------
 
-template <int K>
+template <class S>
 __global__ void __launch_bounds__(kGemmThreads, 1)
-gemm_tc_kernel(Geom L, const uint4 *__restrict__ packed, const uint4 *__restrict__ cb,
+gemm_tc_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restrict__ cb,
                const uint16_t *__restrict__ scales, const uint16_t *__restrict__ x, int T,
                uint16_t *__restrict__ y, void *ws)
 {
@@ -41,16 +42,16 @@ gemm_tc_kernel(Geom L, const uint4 *__restrict__ packed, const uint4 *__restrict
     uint8_t *smem = smem_raw + pad;
     uint8_t *tileA = smem;                                // [2][16 KiB]
     uint8_t *tileB = smem + kStages * kTileABytes;        // [2][16 KiB]
-    uint4 *scb = reinterpret_cast<uint4 *>(tileB + kStages * kTileBBytes);  // 2x8 codebooks
-    uint64_t *bars = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(scb) + 512 * 16);
+    uint4 *scb = reinterpret_cast<uint4 *>(tileB + kStages * kTileBBytes);  // B = 8 codebooks
+    uint64_t *bars = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(scb) + S::kSmemBookBytes);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + kStages);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int m0 = blockIdx.x * kBM;
     const int n0 = blockIdx.y * kBN;
 
-    if (K == 2)
-        for (int i = tid; i < 512; i += kGemmThreads) scb[i] = cb[i];
+    if constexpr (S::kBooksInSmem)
+        for (int i = tid; i < S::K * 256; i += kGemmThreads) scb[i] = cb[i];
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) mbar_init(&bars[s], 1);
         fence_mbar_init();
@@ -82,21 +83,15 @@ gemm_tc_kernel(Geom L, const uint4 *__restrict__ packed, const uint4 *__restrict
             const int rt_l = tid >> 3, gi = tid & 7;
             const int rt = (m0 >> 3) + rt_l;
             const int g = kt * 8 + gi;
-            uint32_t wd[8];
             const bool live = (rt < L.rtiles) && (g < L.G);
-            if (live) {
-                uint4 c = ldg_nc_v4(packed + (size_t)rt * L.gp + g);
-                wd[0] = c.x & 0xffff; wd[1] = c.x >> 16; wd[2] = c.y & 0xffff; wd[3] = c.y >> 16;
-                wd[4] = c.z & 0xffff; wd[5] = c.z >> 16; wd[6] = c.w & 0xffff; wd[7] = c.w >> 16;
-            }
+            const Chunk<S> code = load_chunk<S>(packed, (size_t)rt * L.gp + g, live);
 #pragma unroll
             for (int r = 0; r < 8; ++r) {
                 uint4 v = make_uint4(0, 0, 0, 0);
                 if (live) {
-                    if (K == 1)
-                        v = ldg_nc_v4(cb + wd[r]);
-                    else
-                        v = add_round_h8(scb[wd[r] & 0xff], scb[256 + (wd[r] >> 8)]);
+                    uint4 t[S::K];
+                    gather_terms<S>(code, r, scb, cb, t);
+                    v = sum_round_fast_h8<S::K>(t);
                 }
                 const uint32_t row = rt_l * 8 + r;
                 *reinterpret_cast<uint4 *>(A + sw128(row, gi)) = v;
@@ -206,24 +201,28 @@ gemm_tc_kernel(Geom L, const uint4 *__restrict__ packed, const uint4 *__restrict
 //              on full_a[stage] (128 arrivals).  The epilogue reads TMEM lanes
 //              32*(warp%4).. with tcgen05.ld, scales, rounds and stores.
 constexpr int kWsBN = 256;
-constexpr int kWsStages = 4;
+// ring depth: 4 stages, 3 when the 32 KiB of 8x8 codebooks share the
+// shared memory (4 x 48 KiB + 32 KiB would not fit)
+template <class S>
+constexpr int kWsStagesOf = (S::kSmemBookBytes > 8192) ? 3 : 4;
 constexpr int kWsThreads = 192;               // 6 warps
 constexpr int kWsTileB = kBK * kWsBN * 2;     // 32 KiB
 constexpr int kWsLag = 2;                     // cp.async stages in flight per decoder (< ring depth)
 
-template <int K>
+template <class S>
 __global__ void __launch_bounds__(kWsThreads, 1)
-gemm_ws_kernel(const __grid_constant__ CUtensorMap xmap, Geom L, const uint4 *__restrict__ packed,
+gemm_ws_kernel(const __grid_constant__ CUtensorMap xmap, Geom L, const uint8_t *__restrict__ packed,
                const uint4 *__restrict__ cb, const uint16_t *__restrict__ scales, int T,
                uint16_t *__restrict__ y, void *ws)
 {
+    constexpr int kWsStages = kWsStagesOf<S>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t *smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-    uint8_t *tileA = smem;                                   // [4][16 KiB]
-    uint8_t *tileB = smem + kWsStages * kTileABytes;         // [4][32 KiB]
+    uint8_t *tileA = smem;                                   // [stages][16 KiB]
+    uint8_t *tileB = smem + kWsStages * kTileABytes;         // [stages][32 KiB]
     uint4 *scb = reinterpret_cast<uint4 *>(tileB + kWsStages * kWsTileB);
-    uint64_t *full_a = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(scb) + (K == 2 ? 512 * 16 : 0));
+    uint64_t *full_a = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(scb) + S::kSmemBookBytes);
     uint64_t *full_b = full_a + kWsStages;
     uint64_t *empty = full_b + kWsStages;
     uint64_t *acc_full = empty + kWsStages;
@@ -235,9 +234,12 @@ gemm_ws_kernel(const __grid_constant__ CUtensorMap xmap, Geom L, const uint4 *__
     const int n0 = blockIdx.y * kWsBN;
     const int nk = (L.in + kBK - 1) / kBK;
 
-    if (K == 1 && tid == 0) prefetch_table_share(cb, 65536u * 16u);
-    if (K == 2)
-        for (int i = tid; i < 512; i += kWsThreads) scb[i] = cb[i];
+    // 1x16: codewords go from L2 into the tile by cp.async, copies of kWsLag
+    // stages in flight; other schemes decode in registers
+    constexpr bool kAsyncWeights = (S::K == 1 && S::B == 16);
+    if (S::B == 16 && tid == 0) prefetch_table_share(cb, (uint32_t)S::K * 65536u * 16u);
+    if constexpr (S::kBooksInSmem)
+        for (int i = tid; i < S::K * 256; i += kWsThreads) scb[i] = cb[i];
     if (tid == 0) {
         for (int s = 0; s < kWsStages; ++s) {
             mbar_init(&full_a[s], 128);
@@ -307,12 +309,11 @@ gemm_ws_kernel(const __grid_constant__ CUtensorMap xmap, Geom L, const uint4 *__
         // code chunks kCodeAhead stages ahead (register ring): a stage's
         // gathers never wait on an HBM round trip
         constexpr int kCodeAhead = 4;
-        uint4 code_ring[kCodeAhead];
+        Chunk<S> code_ring[kCodeAhead];
 #pragma unroll
         for (int q = 0; q < kCodeAhead; ++q)
-            code_ring[q] = (q < nk && rows_live && q * 8 + gi < L.G) ? ldg_stream_v4(packed + (size_t)rt * L.gp + q * 8 + gi)
-                                                                    : make_uint4(0, 0, 0, 0);
-        const int lag = (K == 1) ? kWsLag : 0;
+            code_ring[q] = load_chunk<S>(packed, (size_t)rt * L.gp + q * 8 + gi, q < nk && rows_live && q * 8 + gi < L.G);
+        const int lag = kAsyncWeights ? kWsLag : 0;
         for (int s = 0; s < nk + lag; ++s) {
             if (s < nk) {
                 const int buf = s % kWsStages;
@@ -320,40 +321,47 @@ gemm_ws_kernel(const __grid_constant__ CUtensorMap xmap, Geom L, const uint4 *__
                     *abort_v = 1;
                 }
                 if (*abort_v) break;
-                uint4 code = code_ring[0];
+                Chunk<S> code = code_ring[0];
 #pragma unroll
                 for (int q = 1; q < kCodeAhead; ++q)
                     if ((s & (kCodeAhead - 1)) == q) code = code_ring[q];
                 const bool live = rows_live && s * 8 + gi < L.G;
                 {
                     const int g = (s + kCodeAhead) * 8 + gi;
-                    const uint4 nxt = (s + kCodeAhead < nk && rows_live && g < L.G)
-                                          ? ldg_stream_v4(packed + (size_t)rt * L.gp + g)
-                                          : make_uint4(0, 0, 0, 0);
+                    const Chunk<S> nxt = load_chunk<S>(packed, (size_t)rt * L.gp + g,
+                                                       s + kCodeAhead < nk && rows_live && g < L.G);
 #pragma unroll
                     for (int q = 0; q < kCodeAhead; ++q)
                         if ((s & (kCodeAhead - 1)) == q) code_ring[q] = nxt;
                 }
-                uint32_t wd[8];
-                wd[0] = code.x & 0xffff; wd[1] = code.x >> 16; wd[2] = code.y & 0xffff; wd[3] = code.y >> 16;
-                wd[4] = code.z & 0xffff; wd[5] = code.z >> 16; wd[6] = code.w & 0xffff; wd[7] = code.w >> 16;
                 uint8_t *A = tileA + buf * kTileABytes;
-                if (K == 1) {
+                if constexpr (kAsyncWeights) {
                     const uint32_t a0 = smem_u32(A);
 #pragma unroll
                     for (int r = 0; r < 8; ++r)
-                        cp_async16(a0 + sw128(rt_l * 8 + r, gi), live ? (const void *)(cb + wd[r]) : (const void *)cb,
-                                   live ? 16u : 0u);
+                        cp_async16(a0 + sw128(rt_l * 8 + r, gi),
+                                   live ? (const void *)(cb + code.code(r, 0)) : (const void *)cb, live ? 16u : 0u);
+                } else if constexpr (S::K <= 2) {
+                    // all codeword reads before the first tile store (the
+                    // books and the tile share one shared array)
+                    uint4 t[8][S::K];
+#pragma unroll
+                    for (int r = 0; r < 8; ++r) gather_terms<S>(code, r, scb, cb, t[r]);
+#pragma unroll
+                    for (int r = 0; r < 8; ++r)
+                        *reinterpret_cast<uint4 *>(A + sw128(rt_l * 8 + r, gi)) =
+                            live ? sum_round_fast_h8<S::K>(t[r]) : make_uint4(0, 0, 0, 0);
                 } else {
 #pragma unroll
                     for (int r = 0; r < 8; ++r) {
-                        const uint4 v = live ? add_round_h8(scb[wd[r] & 0xff], scb[256 + (wd[r] >> 8)])
-                                             : make_uint4(0, 0, 0, 0);
-                        *reinterpret_cast<uint4 *>(A + sw128(rt_l * 8 + r, gi)) = v;
+                        uint4 t[S::K];
+                        gather_terms<S>(code, r, scb, cb, t);
+                        *reinterpret_cast<uint4 *>(A + sw128(rt_l * 8 + r, gi)) =
+                            live ? sum_round_fast_h8<S::K>(t) : make_uint4(0, 0, 0, 0);
                     }
                 }
             }
-            if (K == 1) {
+            if constexpr (kAsyncWeights) {
                 cp_async_commit();
                 const int j = s - lag;
                 if (j >= 0) {
@@ -439,9 +447,10 @@ using namespace aqk;
 
 size_t gemm_workspace_bytes(const Geom &, int) { return kWsHeader; }
 
+template <class S>
 static constexpr int gemm_smem_bytes()
 {
-    return 1024 /* alignment slack */ + kStages * (kTileABytes + kTileBBytes) + 512 * 16 +
+    return 1024 /* alignment slack */ + kStages * (kTileABytes + kTileBBytes) + S::kSmemBookBytes +
            kStages * 8 + 16;
 }
 
@@ -458,19 +467,18 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
     return fn;
 }
 
-static constexpr int gemm_ws_smem_bytes(int K)
+template <class S>
+static constexpr int gemm_ws_smem_bytes()
 {
-    return 1024 + kWsStages * (kTileABytes + kWsTileB) + (K == 2 ? 512 * 16 : 0) +
-           (3 * kWsStages + 1) * 8 + 16;
+    return 1024 + kWsStagesOf<S> * (kTileABytes + kWsTileB) + S::kSmemBookBytes + (3 * kWsStagesOf<S> + 1) * 8 + 16;
 }
 
 cudaError_t launch_gemm(const Geom &g, const void *packed, const uint16_t *cb,
                         const uint16_t *scales, const uint16_t *x, int T, uint16_t *y, void *ws,
                         cudaStream_t s)
 {
-    const uint4 *pk = reinterpret_cast<const uint4 *>(packed);
+    const uint8_t *pk = reinterpret_cast<const uint8_t *>(packed);
     const uint4 *c = reinterpret_cast<const uint4 *>(cb);
-    cudaError_t e;
     PFN_cuTensorMapEncodeTiled_v12000 encode = (T % 8 == 0) ? tensor_map_encoder() : nullptr;
     if (encode) {
         // X [in][T] binary16: innermost dimension tokens, box 64 tokens x 64 features
@@ -484,32 +492,27 @@ cudaError_t launch_gemm(const Geom &g, const void *packed, const uint16_t *cb,
                             CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
         const dim3 grid((g.out + kBM - 1) / kBM, (T + kWsBN - 1) / kWsBN);
-        const int smem = gemm_ws_smem_bytes(g.K);
-        if (g.K == 1) {
-            e = cudaFuncSetAttribute(gemm_ws_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        return with_scheme(g, [&](auto sch) {
+            using S = decltype(sch);
+            constexpr int smem = gemm_ws_smem_bytes<S>();
+            static_assert(smem <= 227 * 1024, "shared memory of the warp-specialised GEMM");
+            cudaError_t e = cudaFuncSetAttribute(gemm_ws_kernel<S>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
             if (e != cudaSuccess) return e;
-            gemm_ws_kernel<1><<<grid, kWsThreads, smem, s>>>(map, g, pk, c, scales, T, y, ws);
-        } else {
-            e = cudaFuncSetAttribute(gemm_ws_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-            if (e != cudaSuccess) return e;
-            gemm_ws_kernel<2><<<grid, kWsThreads, smem, s>>>(map, g, pk, c, scales, T, y, ws);
-        }
-        return cudaGetLastError();
+            gemm_ws_kernel<S><<<grid, kWsThreads, smem, s>>>(map, g, pk, c, scales, T, y, ws);
+            return cudaGetLastError();
+        });
     }
     // T not a multiple of 8: rows of X are not 16-byte aligned for TMA; the
     // two-stage kernel stages X with ordinary loads.
-    const int smem = gemm_smem_bytes();
     const dim3 grid((g.out + kBM - 1) / kBM, (T + kBN - 1) / kBN);
-    if (g.K == 1) {
-        e = cudaFuncSetAttribute(gemm_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    return with_scheme(g, [&](auto sch) {
+        using S = decltype(sch);
+        constexpr int smem = gemm_smem_bytes<S>();
+        cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<S>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
-        gemm_tc_kernel<1><<<grid, kGemmThreads, smem, s>>>(g, pk, c, scales, x, T, y, ws);
-    } else {
-        e = cudaFuncSetAttribute(gemm_tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-        gemm_tc_kernel<2><<<grid, kGemmThreads, smem, s>>>(g, pk, c, scales, x, T, y, ws);
-    }
-    return cudaGetLastError();
+        gemm_tc_kernel<S><<<grid, kGemmThreads, smem, s>>>(g, pk, c, scales, x, T, y, ws);
+        return cudaGetLastError();
+    });
 }
 
 cudaError_t launch_selftest_wait(void *ws, int spin_limit, cudaStream_t s)

@@ -7,20 +7,23 @@
 // paper's abstract names for token generation.
 //
 // Two kernels, chosen by scheme and batch:
-//  * 2x8, batch 1 -- `gemv_2x8_lut_kernel`: per-group codebook x activation
-//    tables in shared memory, lane-private so random codes never conflict;
-//    two 4-byte table reads per group.
-//  * 1x16 any batch, 2x8 batch 2..16 -- `gemv_tc_kernel`: codes are decoded
-//    into a 128x64 binary16 tile in shared memory (128-byte-swizzled,
-//    K-major) and multiplied by the activations on the tensor cores
-//    (tcgen05.mma, M = 128, N = 16, fp32 accumulator in tensor memory), so
-//    the cost per group does not grow with the batch.  For 1x16 the bound is
-//    the rate of random 16-byte codeword reads from the L2-resident 1 MiB
-//    codebook (about one request per SM clock), not HBM.
+//  * 8-bit codes with one or two codebooks (1x8, 2x8), batch 1 --
+//    `gemv_lut_kernel`: per-group codebook x activation tables in shared
+//    memory, lane-private so random codes never conflict; K 4-byte table
+//    reads per group.
+//  * every other case (1x16, 2x16, 8x8 at any batch; 1x8, 2x8 at batch
+//    2..16) -- `gemv_tc_kernel`: codes are decoded into a 128x64 binary16
+//    tile in shared memory (128-byte-swizzled, K-major) and multiplied by the
+//    activations on the tensor cores (tcgen05.mma, M = 128, N = 16, fp32
+//    accumulator in tensor memory), so the cost per group does not grow with
+//    the batch.  For 1x16 the bound is the rate of random 16-byte codeword
+//    reads from the L2-resident 1 MiB codebook (about one request per SM
+//    clock), not HBM.
 // Split-K partial sums go to the workspace and the last CTA to arrive for a
 // row range adds them in split order (no float atomics: bit-reproducible).
 #include <mutex>
 
+#include "scheme.cuh"
 #include "tc_common.cuh"
 
 namespace aqk {
@@ -85,12 +88,6 @@ __device__ __forceinline__ void splitk_finish(const Geom &L, SplitK sk, int row0
     if (threadIdx.x == 0) sk.counters[blockIdx.x] = 0u;
 }
 
-__device__ __forceinline__ void unpack8(uint4 c, uint32_t w[8])
-{
-    w[0] = c.x & 0xffff; w[1] = c.x >> 16; w[2] = c.y & 0xffff; w[3] = c.y >> 16;
-    w[4] = c.z & 0xffff; w[5] = c.z >> 16; w[6] = c.w & 0xffff; w[7] = c.w >> 16;
-}
-
 // ---------------------------------------------------------------------------
 // 2x8, batch 1: per-group codebook x activation lookup tables.
 //
@@ -153,13 +150,16 @@ __device__ __forceinline__ void mma_m16n8k8(float d[4], uint32_t a0, uint32_t a1
         : "r"(a0), "r"(a1), "r"(b0), "f"(0.f));
 }
 
+template <class S>
 __global__ void __launch_bounds__(kLutWarps * 32, 2)
-gemv_2x8_lut_kernel(Geom L, const uint4 *__restrict__ packed, const uint4 *__restrict__ cb,
-                    const uint16_t *__restrict__ scales, const uint16_t *__restrict__ x,
-                    uint16_t *__restrict__ y, SplitK sk, int rt_per_cta)
+gemv_lut_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restrict__ cb,
+                const uint16_t *__restrict__ scales, const uint16_t *__restrict__ x,
+                uint16_t *__restrict__ y, SplitK sk, int rt_per_cta)
 {
-    extern __shared__ float lut[];       // [2][256][32] tables
-    __shared__ uint4 scb[512];           // both codebooks, binary16, row k*256 + c
+    static_assert(S::B == 8 && S::K <= 2, "tables for one or two 8-bit codebooks");
+    constexpr int K = S::K;
+    extern __shared__ float lut[];       // [K][256][32] tables
+    __shared__ uint4 scb[K * 256];       // the codebooks, binary16, row k*256 + c
     __shared__ uint4 xs[32];             // activations of the block's 32 groups
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gb = blockIdx.y;
@@ -168,30 +168,31 @@ gemv_2x8_lut_kernel(Geom L, const uint4 *__restrict__ packed, const uint4 *__res
     // this warp's row quads (4 row tiles, 32 rows) start at row tile
     // rt0 + 4 (warp + kLutWarps j), j < nq; tiles at or past rt1 read as zero
     const int nq = ((rt1 - rt0 + 3) / 4 - warp + kLutWarps - 1) / kLutWarps;
-    const uint4 *src = packed + (size_t)(rt0 + 4 * warp) * L.gp + gb * 32 + lane;
+    const size_t src = (size_t)(rt0 + 4 * warp) * L.gp + gb * 32 + lane;  // chunk index of tile 0
     const size_t qstep = (size_t)4 * kLutWarps * L.gp;
     const int tile_lim = rt1 - rt0 - 4 * warp;  // tile 4 kLutWarps j + t exists iff below this
     // codebooks first: the table build needs them, the lookups come later
-    const uint4 cw0 = ldg_stream_v4(cb + threadIdx.x), cw1 = ldg_stream_v4(cb + 256 + threadIdx.x);
-    uint4 ring[kLutRing][4];
+    uint4 cw[K];
+#pragma unroll
+    for (int k = 0; k < K; ++k) cw[k] = ldg_stream_v4(cb + k * 256 + threadIdx.x);
+    Chunk<S> ring[kLutRing][4];
 #pragma unroll
     for (int i = 0; i < kLutRing; ++i)
 #pragma unroll
         for (int t = 0; t < 4; ++t)
-            ring[i][t] = (i < nq && 4 * kLutWarps * i + t < tile_lim)
-                             ? ldg_stream_v4(src + i * qstep + (size_t)t * L.gp)
-                             : make_uint4(0, 0, 0, 0);
+            ring[i][t] = load_chunk<S>(packed, src + i * qstep + (size_t)t * L.gp,
+                                       i < nq && 4 * kLutWarps * i + t < tile_lim);
     grid_dependency_wait();  // x, y and the workspace follow the previous launch
     grid_launch_dependents();
     if (threadIdx.x < 32) {
         const int g = gb * 32 + threadIdx.x;
         xs[threadIdx.x] = (g < L.G) ? ldg_nc_v4(x + (size_t)g * 8) : make_uint4(0, 0, 0, 0);
     }
-    scb[threadIdx.x] = cw0;
-    scb[256 + threadIdx.x] = cw1;
+#pragma unroll
+    for (int k = 0; k < K; ++k) scb[k * 256 + threadIdx.x] = cw[k];
     __syncthreads();
     {
-        // warp w fills codewords kc in [64w, 64w + 64) for all 32 groups
+        // warp w fills codewords kc in [32 K w, 32 K (w + 1)) for all 32 groups
         const int gid = lane >> 2, t4 = lane & 3;
         const uint32_t *xw = reinterpret_cast<const uint32_t *>(xs);
         const uint32_t *cbw = reinterpret_cast<const uint32_t *>(scb);
@@ -201,13 +202,13 @@ gemv_2x8_lut_kernel(Geom L, const uint4 *__restrict__ packed, const uint4 *__res
             a[m][0] = xw[(16 * m + gid) * 4 + t4];
             a[m][1] = xw[(16 * m + gid + 8) * 4 + t4];
         }
-        const int kc0 = warp * 64;
+        const int kc0 = warp * 32 * K;
         float *dst = lut + (kc0 + 2 * t4) * 32 + gid;
         int off[4];
 #pragma unroll
         for (int s = 0; s < 4; ++s) off[s] = 8 * ((t4 + s) & 3);
 #pragma unroll
-        for (int n = 0; n < 8; ++n) {
+        for (int n = 0; n < 4 * K; ++n) {
             const uint32_t b0 = cbw[(kc0 + 8 * n + gid) * 4 + t4];
             float d0[4], d1[4];
             mma_m16n8k8(d0, a[0][0], a[0][1], b0);  // groups gid, gid + 8
@@ -228,8 +229,7 @@ gemv_2x8_lut_kernel(Geom L, const uint4 *__restrict__ packed, const uint4 *__res
         }
     }
     __syncthreads();
-    const float *lut0 = lut + lane;
-    const float *lut1 = lut + 256 * 32 + lane;
+    const float *lutl = lut + lane;  // table k at lutl + k * 256 * 32
     float *part = sk.partials + (size_t)gb * L.rows8;
     for (int j0 = 0; j0 < nq; j0 += kLutRing) {
 #pragma unroll
@@ -238,20 +238,19 @@ gemv_2x8_lut_kernel(Geom L, const uint4 *__restrict__ packed, const uint4 *__res
             if (j >= nq) break;
             float acc[32];  // acc[8 t + r]: row r of tile t of the quad, this lane's group
 #pragma unroll
-            for (int t = 0; t < 4; ++t) {
-                const uint32_t v[4] = {ring[i][t].x, ring[i][t].y, ring[i][t].z, ring[i][t].w};
+            for (int t = 0; t < 4; ++t)
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    acc[8 * t + 2 * q] = lut0[(v[q] & 0xff) * 32] + lut1[((v[q] >> 8) & 0xff) * 32];
-                    acc[8 * t + 2 * q + 1] = lut0[((v[q] >> 16) & 0xff) * 32] + lut1[(v[q] >> 24) * 32];
+                for (int r = 0; r < 8; ++r) {
+                    float a = lutl[ring[i][t].code(r, 0) * 32];
+#pragma unroll
+                    for (int k = 1; k < K; ++k) a += lutl[(k * 256 + ring[i][t].code(r, k)) * 32];
+                    acc[8 * t + r] = a;
                 }
-            }
             const int jn = j + kLutRing;
 #pragma unroll
             for (int t = 0; t < 4; ++t)
-                ring[i][t] = (jn < nq && 4 * kLutWarps * jn + t < tile_lim)
-                                 ? ldg_stream_v4(src + jn * qstep + (size_t)t * L.gp)
-                                 : make_uint4(0, 0, 0, 0);
+                ring[i][t] = load_chunk<S>(packed, src + jn * qstep + (size_t)t * L.gp,
+                                           jn < nq && 4 * kLutWarps * jn + t < tile_lim);
             const float r = warp_reduce32(acc, lane);
             const int row = (rt0 + 4 * (warp + kLutWarps * j)) * 8 + lane;
             if (row < rt1 * 8) {
@@ -299,30 +298,34 @@ constexpr int kTcBM = 128;
 constexpr int kTcN = 16;
 // ring depth and copy-to-signal lag: deep for the asynchronous 1x16 gathers,
 // short for the synchronous 2x8 decode
-template <int K> struct TcRing;
-template <> struct TcRing<1> { static constexpr int depth = 5, lag = 3; };
-template <> struct TcRing<2> { static constexpr int depth = 3, lag = 1; };
+// Ring depth and copy lag: 1x16 codewords arrive by cp.async from L2 (deep
+// ring, copies of three stages in flight); the other schemes decode in
+// registers, so only the x copies are asynchronous.
+template <class S> struct TcRing {
+    static constexpr bool kAsyncWeights = (S::K == 1 && S::B == 16);
+    static constexpr int depth = kAsyncWeights ? 5 : 3, lag = kAsyncWeights ? 3 : 1;
+};
 constexpr int kTcTileA = kTcBM * 64 * 2;  // 16 KiB
 constexpr int kTcTileB = 64 * 32;         // 2 KiB: 64 rows x 16 columns
 constexpr int kTcXSlot = 64 * 16 * 2;     // raw x rows of one stage, batch <= 16
 constexpr int kTcTmemCols = 32;
 constexpr int kCodeAhead = 4;             // code chunks requested this many stages ahead
 
-template <int K>
+template <class S>
 __global__ void __launch_bounds__(kTcThreads)
-gemv_tc_kernel(Geom L, const uint4 *__restrict__ packed, const uint4 *__restrict__ cb,
+gemv_tc_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restrict__ cb,
                const uint16_t *__restrict__ scales, const uint16_t *__restrict__ x, int batch,
                uint16_t *__restrict__ y, SplitK sk, void *ws, int stages_per_split)
 {
-    constexpr int R = TcRing<K>::depth, LAG = TcRing<K>::lag;
+    constexpr int R = TcRing<S>::depth, LAG = TcRing<S>::lag;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t *smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
     uint8_t *tileA = smem;                    // [R][16 KiB]
     uint8_t *tileB = tileA + R * kTcTileA;    // [R][2 KiB]
     uint8_t *xring = tileB + R * kTcTileB;    // [R][2 KiB] raw x rows
-    uint4 *scb = reinterpret_cast<uint4 *>(xring + R * kTcXSlot);  // 2x8 codebooks
-    uint64_t *full = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(scb) + (K == 2 ? 512 * 16 : 0));
+    uint4 *scb = reinterpret_cast<uint4 *>(xring + R * kTcXSlot);  // B = 8 codebooks
+    uint64_t *full = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(scb) + S::kSmemBookBytes);
     uint64_t *empty = full + R;
     uint64_t *acc_full = empty + R;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 1);
@@ -336,9 +339,9 @@ gemv_tc_kernel(Geom L, const uint4 *__restrict__ packed, const uint4 *__restrict
     const int nloc = max(0, s1 - s0);
     const bool x_direct = (batch == 16 || batch == 8);
 
-    if (K == 1 && tid == 0) prefetch_table_share(cb, 65536u * 16u);
-    if (K == 2)
-        for (int i = tid; i < 512; i += kTcThreads) scb[i] = cb[i];
+    if (S::B == 16 && tid == 0) prefetch_table_share(cb, (uint32_t)S::K * 65536u * 16u);
+    if constexpr (S::kBooksInSmem)
+        for (int i = tid; i < S::K * 256; i += kTcThreads) scb[i] = cb[i];
     if (tid == 0) {
         for (int s = 0; s < R; ++s) {
             mbar_init(&full[s], kTcDecoders);
@@ -361,12 +364,11 @@ gemv_tc_kernel(Geom L, const uint4 *__restrict__ packed, const uint4 *__restrict
         const int rt = (m0 >> 3) + rt_l;
         const bool rows_live = rt < L.rtiles;
         const int kr = tid >> 1, hb = tid & 1;    // B role: feature row, 8-column half
-        uint4 code_ring[kCodeAhead];
+        Chunk<S> code_ring[kCodeAhead];
 #pragma unroll
         for (int q = 0; q < kCodeAhead; ++q) {
             const int g = (s0 + q) * 8 + gi;
-            code_ring[q] = (q < nloc && rows_live && g < L.G) ? ldg_stream_v4(packed + (size_t)rt * L.gp + g)
-                                                              : make_uint4(0, 0, 0, 0);
+            code_ring[q] = load_chunk<S>(packed, (size_t)rt * L.gp + g, q < nloc && rows_live && g < L.G);
         }
         // everything above touched weights only; x, y and the workspace may
         // be written by the previous launch on the stream
@@ -387,38 +389,40 @@ gemv_tc_kernel(Geom L, const uint4 *__restrict__ packed, const uint4 *__restrict
                         ok = false;
                         break;
                     }
-                    const uint4 code = code_ring[u];
+                    const Chunk<S> code = code_ring[u];
                     {
                         const int g = (s + kCodeAhead) * 8 + gi;
-                        code_ring[u] = (i + kCodeAhead < nloc && rows_live && g < L.G)
-                                           ? ldg_stream_v4(packed + (size_t)rt * L.gp + g)
-                                           : make_uint4(0, 0, 0, 0);
+                        code_ring[u] = load_chunk<S>(packed, (size_t)rt * L.gp + g,
+                                                     i + kCodeAhead < nloc && rows_live && g < L.G);
                     }
                     const bool live = rows_live && s * 8 + gi < L.G;
                     uint8_t *A = tileA + buf * kTcTileA;
-                    uint32_t wd[8];
-                    unpack8(code, wd);
-                    if (K == 1) {
+                    if constexpr (TcRing<S>::kAsyncWeights) {
                         const uint32_t a0 = smem_u32(A);
 #pragma unroll
                         for (int r = 0; r < 8; ++r)
-                            cp_async16(a0 + sw128(rt_l * 8 + r, gi), live ? (const void *)(cb + wd[r]) : (const void *)cb,
-                                       live ? 16u : 0u);
-                    } else {
+                            cp_async16(a0 + sw128(rt_l * 8 + r, gi),
+                                       live ? (const void *)(cb + code.code(r, 0)) : (const void *)cb, live ? 16u : 0u);
+                    } else if constexpr (S::K <= 2) {
                         // every codeword read is issued before the first tile
                         // store: the codebooks and the tile share one shared
                         // array, so a store would otherwise hold back the
                         // next row's reads and serialise the eight rows
-                        uint4 c0[8], c1[8];
+                        uint4 t[8][S::K];
 #pragma unroll
-                        for (int r = 0; r < 8; ++r) {
-                            c0[r] = scb[wd[r] & 0xff];
-                            c1[r] = scb[256 + (wd[r] >> 8)];
-                        }
+                        for (int r = 0; r < 8; ++r) gather_terms<S>(code, r, scb, cb, t[r]);
 #pragma unroll
                         for (int r = 0; r < 8; ++r)
                             *reinterpret_cast<uint4 *>(A + sw128(rt_l * 8 + r, gi)) =
-                                live ? add_round_h8(c0[r], c1[r]) : make_uint4(0, 0, 0, 0);
+                                live ? sum_round_fast_h8<S::K>(t[r]) : make_uint4(0, 0, 0, 0);
+                    } else {
+#pragma unroll
+                        for (int r = 0; r < 8; ++r) {
+                            uint4 t[S::K];
+                            gather_terms<S>(code, r, scb, cb, t);
+                            *reinterpret_cast<uint4 *>(A + sw128(rt_l * 8 + r, gi)) =
+                                live ? sum_round_fast_h8<S::K>(t) : make_uint4(0, 0, 0, 0);
+                        }
                     }
                     // x rows of this stage: straight into the B tile when a row is
                     // 16 or 32 bytes, else the raw rows into the stage's x slot
@@ -538,7 +542,7 @@ using namespace aqk;
 
 namespace {
 
-enum Path { kLut2x8 = 1, kTensor = 2 };
+enum Path { kLut = 1, kTensor = 2 };
 
 struct GemvPlan {
     Path path;
@@ -556,8 +560,8 @@ inline size_t align16(size_t v) { return (v + 15) / 16 * 16; }
 GemvPlan plan_gemv(const Geom &g, int batch)
 {
     GemvPlan p{};
-    if (batch == 1 && g.K == 2) {
-        p.path = kLut2x8;
+    if (batch == 1 && g.B == 8 && g.K <= 2) {
+        p.path = kLut;
         p.ks = g.gblocks;
         // two CTAs per SM in one wave: every CTA builds its tables once, and
         // a third CTA per SM fits, so the next launch can start early
@@ -586,11 +590,11 @@ GemvPlan plan_gemv(const Geom &g, int batch)
 }
 
 // ring of (A tile, B tile, x slot) + codebooks + barriers, TMEM slot, flag
-template <int K>
+template <class S>
 constexpr int tc_smem_bytes()
 {
-    return 1024 + TcRing<K>::depth * (kTcTileA + kTcTileB + kTcXSlot) + (K == 2 ? 512 * 16 : 0) +
-           (2 * TcRing<K>::depth + 1) * 8 + 16;
+    return 1024 + TcRing<S>::depth * (kTcTileA + kTcTileB + kTcXSlot) + S::kSmemBookBytes +
+           (2 * TcRing<S>::depth + 1) * 8 + 16;
 }
 
 template <class Kern>
@@ -633,38 +637,35 @@ cudaError_t launch_gemv(const Geom &g, const void *packed, const uint16_t *cb,
     sk.counters = reinterpret_cast<unsigned *>(base + kWsHeader);
     sk.partials = reinterpret_cast<float *>(base + kWsHeader +
                                             align16(sizeof(unsigned) * (size_t)p.grid_x));
-    const uint4 *pk = reinterpret_cast<const uint4 *>(packed);
+    const uint8_t *pk = reinterpret_cast<const uint8_t *>(packed);
     const uint4 *c = reinterpret_cast<const uint4 *>(cb);
     const dim3 grid(p.grid_x, p.ks);
     cudaError_t e = cudaSuccess;
-    switch (p.path) {
-    case kLut2x8: {
-        const int smem = 2 * 256 * 32 * sizeof(float);  // the two tables
-        e = set_smem(gemv_2x8_lut_kernel, smem);
-        if (e != cudaSuccess) return e;
-        e = launch_pdl(gemv_2x8_lut_kernel, grid, dim3(kLutWarps * 32), smem, s, g, pk, c, scales, x, y, sk,
-                       p.rt_per_cta);
-        if (e != cudaSuccess) return e;
-        break;
+    if (p.path == kLut) {
+        const int smem = g.K * 256 * 32 * (int)sizeof(float);  // the tables
+        auto lut = [&](auto sch) {
+            using S = decltype(sch);
+            if constexpr (S::B == 8 && S::K <= 2) {
+                cudaError_t r = set_smem(gemv_lut_kernel<S>, smem);
+                if (r != cudaSuccess) return r;
+                return launch_pdl(gemv_lut_kernel<S>, grid, dim3(kLutWarps * 32), smem, s, g, pk, c, scales, x, y,
+                                  sk, p.rt_per_cta);
+            } else {
+                return cudaErrorInvalidValue;
+            }
+        };
+        e = with_scheme(g, lut);
+    } else {
+        e = with_scheme(g, [&](auto sch) {
+            using S = decltype(sch);
+            const int smem = tc_smem_bytes<S>();
+            cudaError_t r = set_smem(gemv_tc_kernel<S>, smem);
+            if (r != cudaSuccess) return r;
+            return launch_pdl(gemv_tc_kernel<S>, grid, dim3(kTcThreads), smem, s, g, pk, c, scales, x, batch, y, sk,
+                              ws, p.per_split);
+        });
     }
-    case kTensor:
-        if (g.K == 1) {
-            const int smem = tc_smem_bytes<1>();
-            e = set_smem(gemv_tc_kernel<1>, smem);
-            if (e != cudaSuccess) return e;
-            e = launch_pdl(gemv_tc_kernel<1>, grid, dim3(kTcThreads), smem, s, g, pk, c, scales, x, batch, y, sk, ws,
-                           p.per_split);
-            if (e != cudaSuccess) return e;
-        } else {
-            const int smem = tc_smem_bytes<2>();
-            e = set_smem(gemv_tc_kernel<2>, smem);
-            if (e != cudaSuccess) return e;
-            e = launch_pdl(gemv_tc_kernel<2>, grid, dim3(kTcThreads), smem, s, g, pk, c, scales, x, batch, y, sk, ws,
-                           p.per_split);
-            if (e != cudaSuccess) return e;
-        }
-        break;
-    }
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

@@ -18,8 +18,11 @@
  *     W[o][8g+j] = RN16( sum_k C_k[codes[o][g][k]][j] )          (decode)
  *     y[o][b]    = RN16( s[o] * sum_i W[o][i] * x[i][b] )        (product)
  *
- * Supported schemes (devtrends.ru, section "Схемы квантования"): "1x16"
- * (K = 1, B = 16) and "2x8" (K = 2, B = 8); both are 2 bits per weight.
+ * Supported schemes (K x B): "1x16" and "2x8" (2 bits per weight) and
+ * "8x8" (8 bits per weight), named in devtrends.ru, section "Схемы
+ * квантования"; "2x16" (4 bits per weight), the AQLM wiki entry's example in
+ * "Niveau intermédiaire"; "1x8" (1 bit per weight), devtrends.ru's notes on
+ * 1-bit models.  Codes are uint8 for B = 8 and uint16 for B = 16.
  *
  * Conventions shared by every entry point:
  *  - binary16 values are passed as uint16_t bit patterns (IEEE 754 half);
@@ -34,16 +37,19 @@
  *  - no C++ exception crosses this interface.
  *
  * Packed code layout (produced by aq_pack_codes, consumed by every kernel).
- * Each group (o, g) owns one 16-bit word: for 1x16 the code itself, for 2x8
- * codes[o][g][0] | codes[o][g][1] << 8.  Rows are padded to a multiple of 8
- * and groups to a multiple of 32 (Gp = padded group count); padding words
- * are zero.  Word (o, g) is stored little-endian at byte
+ * Each group (o, g) owns one word of W = K*B/8 bytes holding its K codes,
+ * code k in bits [k*B, (k+1)*B) (1x16: the code; 2x8: c0 | c1 << 8; 1x8:
+ * one byte; 2x16: c0 | c1 << 16; 8x8: eight bytes, c0 first).  Rows are
+ * padded to a multiple of 8 and groups to a multiple of 32 (Gp = padded
+ * group count); padding words are zero.  Word (o, g) is stored
+ * little-endian at byte
  *
- *     ((o / 8) * (Gp / 32) + g / 32) * 512  +  (g % 32) * 16  +  (o % 8) * 2
+ *     ((o / 8) * (Gp / 32) + g / 32) * 256 W  +  (g % 32) * 8 W  +  (o % 8) * W
  *
- * i.e. 512-byte tiles of 8 rows x 32 groups, tile-rows in row order; inside
- * a tile the 16-byte chunk c holds group 32*(g/32)+c for the tile's 8 rows,
- * so one warp-wide 128-bit load fetches a whole tile.
+ * i.e. 256 W-byte tiles of 8 rows x 32 groups, tile-rows in row order;
+ * inside a tile the 8 W-byte chunk c holds group 32*(g/32)+c for the
+ * tile's 8 rows (for the 2-bit schemes a 16-byte chunk, so one warp-wide
+ * 128-bit load fetches a whole tile).
  */
 #ifndef AQ_B200_H
 #define AQ_B200_H
@@ -74,7 +80,7 @@ typedef struct {
     int32_t out_features;  /* rows of W, 1 .. 2^28                         */
     int32_t in_features;   /* columns of W, 8 .. 2^24, multiple of 8       */
     int32_t group_size;    /* weights per code group; must be 8            */
-    int32_t num_codebooks; /* K: 1 (with nbits 16) or 2 (with nbits 8)     */
+    int32_t num_codebooks; /* K: 1x16, 2x8, 1x8, 2x16 or 8x8 with nbits    */
     int32_t nbits;         /* B: bits per code, codebook has 2^B entries   */
 } aq_layer_desc;
 
@@ -125,7 +131,7 @@ aq_status aq_selftest_bounded_wait(void *workspace, int spin_limit, aq_stream_t 
 
 /*
  * Interleave codes into the packed layout (offline, once per layer).
- *   codes  [out][in/8][K]: uint8 for 2x8, uint16 for 1x16 (row-major).
+ *   codes  [out][in/8][K]: uint8 for B = 8, uint16 for B = 16 (row-major).
  *   packed aq_packed_codes_bytes(desc) bytes; every byte is written,
  *          padding included.
  * `codes` needs only the alignment of its element type; `packed` 16 bytes.

@@ -55,9 +55,14 @@ def test_version_and_status_strings():
     assert aq.aq_status_string(99) == "unknown status"
 
 
+SCHEMES = ((1, 16), (2, 8), (1, 8), (2, 16), (8, 8))
+
+
 @pytest.mark.parametrize("out,inp,K,B", [(1, 8, 1, 16), (20, 520, 1, 16), (20, 520, 2, 8),
                                          (4096, 4096, 1, 16), (11008, 4096, 2, 8),
-                                         (4096, 11008, 2, 8), (28672, 8192, 1, 16), (37, 360, 2, 8)])
+                                         (4096, 11008, 2, 8), (28672, 8192, 1, 16), (37, 360, 2, 8),
+                                         (20, 520, 1, 8), (37, 360, 2, 16), (20, 520, 8, 8),
+                                         (4096, 4096, 8, 8), (11008, 4096, 2, 16)])
 def test_packed_bytes_matches_oracle(out, inp, K, B):
     d = aq.LayerDesc.make(out, inp, K, B)
     assert aq.aq_packed_codes_bytes(d) == oracle.packed_bytes(out, inp, K, B)
@@ -65,14 +70,15 @@ def test_packed_bytes_matches_oracle(out, inp, K, B):
 
 @pytest.mark.parametrize("desc,why", [
     ((0, 64, 8, 1, 16), "no rows"), ((16, 0, 8, 1, 16), "no columns"), ((16, 12, 8, 1, 16), "in % 8"),
-    ((16, 64, 4, 1, 16), "group size"), ((16, 64, 8, 2, 16), "2x16"), ((16, 64, 8, 8, 8), "8x8"),
-    ((16, 64, 8, 1, 8), "1x8"), ((-1, 64, 8, 1, 16), "negative"),
+    ((16, 64, 4, 1, 16), "group size"), ((16, 64, 8, 4, 8), "4x8"), ((16, 64, 8, 2, 4), "2x4"),
+    ((16, 64, 8, 1, 12), "1x12"), ((16, 64, 8, 3, 8), "3x8"), ((16, 64, 8, 8, 16), "8x16"),
+    ((-1, 64, 8, 1, 16), "negative"),
 ])
 def test_invalid_descriptors(desc, why):
     d = aq.LayerDesc(*desc)
     assert aq.aq_packed_codes_bytes(d) == 0, why
     assert aq.aq_gemv_workspace_bytes(d, 1) == 0, why
-    want = 2 if desc[2] != 8 or (desc[3], desc[4]) not in ((1, 16), (2, 8)) else 1
+    want = 2 if desc[2] != 8 or (desc[3], desc[4]) not in SCHEMES else 1
     if desc[0] < 1 or desc[1] < 8 or desc[1] % 8:
         want = 1
     st = aq.lib.aq_gemv(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, 1, FAKE, FAKE, 1 << 20, None)

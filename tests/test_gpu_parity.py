@@ -18,7 +18,8 @@ from aqtest import (DevLayer, assert_close, dev, guarded, guards_intact, run_gem
 
 pytestmark = pytest.mark.gpu
 
-SCHEMES = [(1, 16), (2, 8)]
+SCHEMES = [(1, 16), (2, 8), (1, 8), (2, 16), (8, 8)]
+NEW_SCHEMES = [(1, 8), (2, 16), (8, 8)]
 SMALL_SHAPES = [(8, 8), (37, 360), (256, 512), (1000, 1032), (64, 4096), (4100, 264)]
 
 
@@ -55,6 +56,26 @@ def test_dequant_bit_exact(K, B, out, inp, scaled):
     torch.cuda.synchronize()
     assert guards_intact(full)
     want = oracle.decode(layer.codes, layer.codebooks, layer.scales if scaled else None)
+    assert np.array_equal(w.cpu().numpy().view(np.uint16).reshape(out, inp), want.view(np.uint16))
+
+
+def test_dequant_eight_codebooks_exact_sum_of_mixed_magnitudes():
+    """8x8: the eight terms span many binades, so a sum rounded at every
+    step (or in fp32) would differ from the exact sum rounded once."""
+    rng = np.random.default_rng(5)
+    K, B, out, inp = 8, 8, 64, 512
+    mant = rng.integers(1024, 2048, size=(K, 256, 8))
+    expo = rng.integers(-24, 6, size=(K, 256, 8))
+    sign = rng.choice([-1.0, 1.0], size=(K, 256, 8))
+    cb = (sign * mant * np.exp2(expo - 10.0)).astype(np.float16)
+    layer = _layer(out, inp, K, B, 3)
+    layer.codebooks[...] = cb
+    dl = DevLayer(layer)
+    full, w = guarded(out * inp)
+    aq.aq_dequant(dl.desc, dl.packed, dl.codebooks, None, w)
+    torch.cuda.synchronize()
+    assert guards_intact(full)
+    want = oracle.decode(layer.codes, layer.codebooks)
     assert np.array_equal(w.cpu().numpy().view(np.uint16).reshape(out, inp), want.view(np.uint16))
 
 
@@ -243,3 +264,30 @@ def test_dequant_full_size_sampled():
     got = w.view(spec.out_features, spec.in_features)[torch.from_numpy(rows).cuda()].cpu().numpy()
     want = oracle.decode(layer.codes[rows], layer.codebooks, layer.scales[rows])
     assert np.array_equal(got.view(np.uint16), want.view(np.uint16))
+
+
+@pytest.mark.parametrize("K,B", NEW_SCHEMES)
+def test_other_schemes_llama_shape_sampled(K, B):
+    """1x8, 2x16 and 8x8 at a Llama-2-7B MLP shape: products at batch 1, 8
+    and 16, a prefill product and the dequantised matrix, on sampled rows."""
+    spec = LayerSpec(11008, 4096, K, B)
+    layer = make_layer(spec, (K, B))
+    dl = DevLayer(layer)
+    rows = _sample_rows(spec.out_features, n=24, seed=K + B)
+    for batch in (1, 8, 16):
+        x = make_activations(spec.in_features, batch, (K, B, batch))
+        y = run_gemv(dl, x)
+        ref, bound = oracle.matmul(layer.codes, layer.codebooks, layer.scales, x, rows=rows, threads=8)
+        assert_close(y[rows], ref, bound, f"{K}x{B} b{batch}")
+    x = make_activations(spec.in_features, 512, (K, B, 512))
+    y = run_gemm(dl, x)
+    ref, bound = oracle.matmul(layer.codes, layer.codebooks, layer.scales, x, rows=rows[:8], threads=8)
+    assert_close(y[rows[:8]], ref, bound, f"{K}x{B} T512")
+    w = torch.empty(spec.out_features * spec.in_features, dtype=torch.int16, device="cuda")
+    aq.aq_dequant(dl.desc, dl.packed, dl.codebooks, dl.scales, w)
+    torch.cuda.synchronize()
+    got = w.view(spec.out_features, spec.in_features)[torch.from_numpy(rows).cuda()].cpu().numpy()
+    want = oracle.decode(layer.codes[rows], layer.codebooks, layer.scales[rows])
+    assert np.array_equal(got.view(np.uint16), want.view(np.uint16))
+    del dl
+    torch.cuda.empty_cache()
