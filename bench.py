@@ -526,7 +526,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=WORKLOAD,
                     help="llama2-7b-1x16 (default), llama2-7b-mlp-2x8, llama2-70b-1x16, "
-                         "llama2-7b-prefill, llama2-7b-block, tiny-2x8")
+                         "llama2-7b-prefill, llama2-7b-block, llama2-7b-schemes, tiny-2x8")
     ap.add_argument("--layers", type=int, default=0, help="copies per shape (0: > 3x L2)")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--skip-e2e", action="store_true")
