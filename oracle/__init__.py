@@ -15,6 +15,9 @@ Quantization" (AQLM wiki entry, "Niveau intermédiaire"; devtrends.ru summary,
   RN16(s[o] * W[o][i]));
 * ``matmul``:  y[o][b] = s[o] * sum_i W[o][i] * x[i][b] in fp64, plus the
   per-element magnitude sum_i |s||W||x| used to scale the tolerance;
+* ``backward``: gradients of sum(gy * y) with respect to the row scales and
+  the codebook entries (the decode's rounding taken as the identity), with
+  magnitude bounds;
 * ``pack`` / ``unpack``: the library's documented packed code layout;
 * ``bits_per_weight`` and ``layer_bytes``: the bit-rate closed form and the
   storage it implies.
@@ -76,6 +79,9 @@ def _load():
             lib.aqo_matmul.argtypes = [_c_i64, _c_i64, _c_int, _c_int, _vp, _vp, _vp,
                                        _vp, _c_i64, _vp, _c_i64, _vp, _vp, _c_int]
             lib.aqo_matmul.restype = _c_int
+            lib.aqo_backward.argtypes = [_c_i64, _c_i64, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp,
+                                         _c_i64, _vp, _vp, _vp, _vp]
+            lib.aqo_backward.restype = _c_int
             lib.aqo_packed_bytes.argtypes = [_c_i64, _c_i64, _c_int, _c_int]
             lib.aqo_packed_bytes.restype = _c_i64
             lib.aqo_pack.argtypes = [_c_i64, _c_i64, _c_int, _c_int, _vp, _vp]
@@ -174,6 +180,33 @@ def matmul(codes, codebooks, scales, x, rows=None, threads: int = 1):
     if rc:
         raise RuntimeError(f"aqo_matmul failed ({rc})")
     return y, bound
+
+
+def backward(codes, codebooks, scales, x, gy):
+    """Gradients of sum(gy * y), y = diag(s) W x, with respect to the row
+    scales and the codebooks (rounding of the decode taken as the identity).
+
+    Returns ``(grad_s [out], grad_s_bound, grad_cb [K][2^B][8], grad_cb_bound)``
+    in float64; the bounds are the same sums of absolute terms."""
+    cb = _bits(codebooks)
+    K, ncw, _ = cb.shape
+    B = int(ncw).bit_length() - 1
+    codes = _codes(codes, K, B)
+    out, G, _ = codes.shape
+    xb, gyb = _bits(x), _bits(gy)
+    if xb.ndim != 2 or xb.shape[0] != G * 8 or gyb.shape != (out, xb.shape[1]):
+        raise ValueError("x must be [in][n] and gy [out][n]")
+    n = xb.shape[1]
+    s = None if scales is None else _bits(scales)
+    gs = np.empty(out, dtype=np.float64)
+    gsb = np.empty(out, dtype=np.float64)
+    gc = np.empty((K, ncw, 8), dtype=np.float64)
+    gcb = np.empty((K, ncw, 8), dtype=np.float64)
+    rc = _load().aqo_backward(out, G * 8, K, B, _ptr(codes), _ptr(cb), _ptr(s), _ptr(xb), _ptr(gyb), n,
+                              _ptr(gs), _ptr(gsb), _ptr(gc), _ptr(gcb))
+    if rc:
+        raise RuntimeError(f"aqo_backward failed ({rc})")
+    return gs, gsb, gc, gcb
 
 
 def packed_bytes(out: int, inp: int, K: int, B: int) -> int:

@@ -27,7 +27,10 @@
  *     values exactly) and rounded once to binary16, ties to even;
  *   - the product with x and the scale are taken in fp64 from the binary16
  *     values, no intermediate rounding;
- *   - codes are unsigned, code k selects a row of codebook k.
+ *   - codes are unsigned, code k selects a row of codebook k;
+ *   - for the gradient with respect to the codebooks and scales (the fine-
+ *     tuning step the wiki entry describes: codebooks are learned jointly
+ *     with the codes), the decode's rounding is taken as the identity.
  *
  * Pins (tests/test_oracle_pins.py): conversions against numpy's binary16,
  * exhaustive single-group decode, one-hot codebooks, additivity, permutation
@@ -228,6 +231,78 @@ int aqo_matmul(int64_t out, int64_t in, int K, int B, const void *codes,
     }
     free(xd);
     return err;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Gradient with respect to the row scales and the codebooks.               */
+/*                                                                          */
+/* For L = sum_{o,b} gy[o][b] y[o][b] with y = diag(s) W x and              */
+/* W[o][8g+j] = RN16(sum_k C_k[i_k][j]) (AQLM wiki entry, "Niveau            */
+/* intermédiaire": the additive decode), the rounding is taken as the       */
+/* identity (its derivative wherever it is differentiable), so each weight  */
+/* depends on codeword entry C_k[c][j] with derivative 1 when i_k = c:       */
+/*   M[o][i]         = sum_b gy[o][b] x[i][b]                               */
+/*   grad_s[o]       = sum_i W[o][i] M[o][i]                                */
+/*   grad_C[k][c][j] = sum of s[o] M[o][8g+j] over every (o, g) whose code   */
+/*                     k is c                                               */
+/* with the magnitudes of the same sums (absolute value of every term) as   */
+/* error bounds.  All in double from the binary16 inputs.                   */
+/* ------------------------------------------------------------------------ */
+
+int aqo_backward(int64_t out, int64_t in, int K, int B, const void *codes,
+                 const uint16_t *codebooks, const uint16_t *scales, const uint16_t *x,
+                 const uint16_t *gy, int64_t n, double *grad_s, double *grad_s_bound,
+                 double *grad_cb, double *grad_cb_bound)
+{
+    if (check_scheme(out, in, K, B) || n < 0) return -1;
+    int64_t G = in / AQO_GROUP;
+    int64_t ncb = (int64_t)K << B;
+    double *xd = (double *)malloc(sizeof(double) * (size_t)(in * n > 0 ? in * n : 1));
+    double *row = (double *)malloc(sizeof(double) * (size_t)(in > 0 ? in : 1));
+    double *m = (double *)malloc(sizeof(double) * (size_t)(in > 0 ? in : 1));
+    double *mabs = (double *)malloc(sizeof(double) * (size_t)(in > 0 ? in : 1));
+    if (!xd || !row || !m || !mabs) {
+        free(xd); free(row); free(m); free(mabs);
+        return -2;
+    }
+    for (int64_t t = 0; t < in * n; ++t) xd[t] = aqo_half_to_double(x[t]);
+    for (int64_t e = 0; e < ncb * AQO_GROUP; ++e) {
+        if (grad_cb) grad_cb[e] = 0.0;
+        if (grad_cb_bound) grad_cb_bound[e] = 0.0;
+    }
+    for (int64_t o = 0; o < out; ++o) {
+        decode_row(o, in, K, B, codes, codebooks, row);
+        double s = scales ? aqo_half_to_double(scales[o]) : 1.0;
+        for (int64_t i = 0; i < in; ++i) {
+            double acc = 0.0, mag = 0.0;
+            for (int64_t b = 0; b < n; ++b) {
+                double t = aqo_half_to_double(gy[o * n + b]) * xd[i * n + b];
+                acc += t;
+                mag += fabs(t);
+            }
+            m[i] = acc;
+            mabs[i] = mag;
+        }
+        double gs = 0.0, gsb = 0.0;
+        for (int64_t i = 0; i < in; ++i) {
+            gs += row[i] * m[i];
+            gsb += fabs(row[i]) * mabs[i];
+        }
+        if (grad_s) grad_s[o] = gs;
+        if (grad_s_bound) grad_s_bound[o] = gsb;
+        for (int64_t g = 0; g < G; ++g) {
+            for (int k = 0; k < K; ++k) {
+                uint32_t c = code_at(codes, B, (o * G + g) * K + k);
+                int64_t base = (((int64_t)k << B) + c) * AQO_GROUP;
+                for (int j = 0; j < AQO_GROUP; ++j) {
+                    if (grad_cb) grad_cb[base + j] += s * m[g * AQO_GROUP + j];
+                    if (grad_cb_bound) grad_cb_bound[base + j] += fabs(s) * mabs[g * AQO_GROUP + j];
+                }
+            }
+        }
+    }
+    free(xd); free(row); free(m); free(mabs);
+    return 0;
 }
 
 /* ------------------------------------------------------------------------ */

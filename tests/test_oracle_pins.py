@@ -410,3 +410,63 @@ def test_pack_roundtrip_and_padding(out, inp, K, B):
     assert packed.size == rows * gp * K * B // 8
     # zero padding: the byte sum equals the code-byte sum
     assert int(packed.astype(np.int64).sum()) == int(layer.codes.view(np.uint8).astype(np.int64).sum())
+
+
+# ---------------------------------------------------------------------------
+# Gradient with respect to scales and codebooks
+# ---------------------------------------------------------------------------
+
+def _loss(codes, cb, s, x, gy):
+    """L = sum(gy * y) from the forward product, in exact rationals."""
+    y, _ = oracle.matmul(codes, cb, s, x)
+    return sum(Fraction(float(gy[o, b])) * Fraction(float(y[o, b]))
+               for o in range(y.shape[0]) for b in range(y.shape[1]))
+
+
+@pytest.mark.parametrize("out,inp,K,B,n", [(3, 16, 2, 3, 2), (2, 24, 1, 4, 3), (4, 8, 8, 2, 1),
+                                           (2, 16, 2, 8, 2), (3, 8, 1, 16, 2)])
+def test_backward_matches_finite_differences_exactly(out, inp, K, B, n):
+    """Dyadic inputs keep every decode exact, so L is linear in each codebook
+    entry and each scale and a unit finite difference of the forward product
+    is the exact partial derivative."""
+    codes, cb, s = _dyadic_layer(out, inp, K, B, out + inp + K + B + n)
+    rng = np.random.default_rng(out * 31 + n)
+    x = (rng.integers(-8, 9, size=(inp, n)) / 4.0).astype(np.float16)
+    gy = (rng.integers(-8, 9, size=(out, n)) / 4.0).astype(np.float16)
+    gs, _, gc, _ = oracle.backward(codes, cb, s, x, gy)
+    base = _loss(codes, cb, s, x, gy)
+    # every scale
+    for o in range(out):
+        s2 = s.copy()
+        s2[o] = s2[o] + np.float16(0.25)
+        assert (_loss(codes, cb, s2, x, gy) - base) * 4 == Fraction(float(gs[o])), o
+    # codebook entries that are used, and one that is not (gradient 0)
+    used = {(k, int(codes[o, g, k])) for o in range(out) for g in range(inp // 8) for k in range(K)}
+    probe = sorted(used)[:6] + [(k, c) for k in range(K) for c in range(1 << B) if (k, c) not in used][:1]
+    for k, c in probe:
+        for j in (0, 3, 7):
+            cb2 = cb.copy()
+            cb2[k, c, j] = cb2[k, c, j] + np.float16(0.125)
+            assert (_loss(codes, cb2, s, x, gy) - base) * 8 == Fraction(float(gc[k, c, j])), (k, c, j)
+
+
+def test_backward_euler_identity():
+    """L is linear in the codebooks (exact decode) and in s, so
+    sum(C * dL/dC) = L = sum_o s_o dL/ds_o."""
+    codes, cb, s = _dyadic_layer(5, 64, 2, 4, 9)
+    rng = np.random.default_rng(3)
+    x = (rng.integers(-8, 9, size=(64, 4)) / 4.0).astype(np.float16)
+    gy = (rng.integers(-8, 9, size=(5, 4)) / 4.0).astype(np.float16)
+    gs, _, gc, _ = oracle.backward(codes, cb, s, x, gy)
+    L = _loss(codes, cb, s, x, gy)
+    assert sum(Fraction(float(a)) * Fraction(float(b)) for a, b in zip(cb.ravel(), gc.ravel())) == L
+    assert sum(Fraction(float(a)) * Fraction(float(b)) for a, b in zip(s, gs)) == L
+
+
+def test_backward_bounds_dominate():
+    layer = make_layer(LayerSpec(40, 264, 2, 8, codebook_sigma=0.05), 8)
+    x = make_activations(264, 6, 1)
+    gy = make_activations(40, 6, 2)
+    gs, gsb, gc, gcb = oracle.backward(layer.codes, layer.codebooks, layer.scales, x, gy)
+    assert np.all(np.abs(gs) <= gsb) and np.all(np.abs(gc) <= gcb)
+    assert np.all(gcb >= 0) and gsb.min() > 0
