@@ -20,7 +20,8 @@ __all__ = [
     "AQError", "LayerDesc", "lib", "library_path", "aq_version", "aq_status_string",
     "aq_packed_codes_bytes", "aq_gemv_workspace_bytes", "aq_gemm_workspace_bytes",
     "aq_workspace_status", "aq_selftest_bounded_wait", "aq_pack_codes", "aq_unpack_codes",
-    "aq_dequant", "aq_gemv", "aq_gemv_noalloc", "aq_gemm", "EXPORTED_SYMBOLS",
+    "aq_dequant", "aq_gemv", "aq_gemv_noalloc", "aq_gemm", "aq_param_grad_workspace_bytes",
+    "aq_param_grad", "EXPORTED_SYMBOLS",
     "GEMV_NOALLOC_SCRATCH_BYTES",
 ]
 
@@ -37,6 +38,7 @@ EXPORTED_SYMBOLS = (
     "aq_status_string", "aq_version", "aq_packed_codes_bytes", "aq_gemv_workspace_bytes",
     "aq_gemm_workspace_bytes", "aq_workspace_status", "aq_selftest_bounded_wait",
     "aq_pack_codes", "aq_unpack_codes", "aq_dequant", "aq_gemv", "aq_gemv_noalloc", "aq_gemm",
+    "aq_param_grad_workspace_bytes", "aq_param_grad",
 )
 
 # AQ_GEMV_NOALLOC_SCRATCH_BYTES of include/aq.h: the fixed scratch behind
@@ -86,6 +88,8 @@ def _load() -> ctypes.CDLL:
         "aq_gemv": ([dp, vp, vp, vp, vp, i32, vp, vp, sz, vp], i32),
         "aq_gemm": ([dp, vp, vp, vp, vp, i32, vp, vp, sz, vp], i32),
         "aq_gemv_noalloc": ([dp, vp, vp, vp, vp, i32, vp, vp], i32),
+        "aq_param_grad_workspace_bytes": ([dp, i32], sz),
+        "aq_param_grad": ([dp, vp, vp, vp, vp, vp, i32, vp, vp, vp, sz, vp], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -188,3 +192,18 @@ def aq_gemm(desc: LayerDesc, packed, codebooks, scales, x, T: int, y, workspace,
     _check("aq_gemm", lib.aq_gemm(ctypes.byref(desc), _ptr(packed), _ptr(codebooks), _ptr(scales),
                                   _ptr(x), T, _ptr(y), _ptr(workspace), workspace_bytes,
                                   _stream(stream)))
+
+
+def aq_param_grad_workspace_bytes(desc: LayerDesc, T: int) -> int:
+    return lib.aq_param_grad_workspace_bytes(ctypes.byref(desc), T)
+
+
+def aq_param_grad(desc: LayerDesc, packed, codebooks, scales, x, gy, T: int, grad_scales, grad_codebooks,
+                  workspace, workspace_bytes: int | None = None, stream=None) -> None:
+    """dL/ds [out] and dL/dC [K][2^B][8] (fp32, overwritten; either may be
+    None) for L = sum(gy * y), y = diag(s) W x; x [in][T], gy [out][T]."""
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    _check("aq_param_grad", lib.aq_param_grad(ctypes.byref(desc), _ptr(packed), _ptr(codebooks), _ptr(scales),
+                                              _ptr(x), _ptr(gy), T, _ptr(grad_scales), _ptr(grad_codebooks),
+                                              _ptr(workspace), workspace_bytes, _stream(stream)))

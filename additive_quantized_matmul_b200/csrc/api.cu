@@ -185,4 +185,31 @@ aq_status aq_gemm(const aq_layer_desc *desc, const void *packed, const uint16_t 
                                       reinterpret_cast<cudaStream_t>(stream)));
 }
 
+size_t aq_param_grad_workspace_bytes(const aq_layer_desc *desc, int T)
+{
+    if (check_desc(desc) != AQ_OK || T < 8 || T > (1 << 22) || T % 8) return 0;
+    return aqh::param_grad_workspace_bytes(aqk::make_geom(*desc), T);
+}
+
+aq_status aq_param_grad(const aq_layer_desc *desc, const void *packed, const uint16_t *codebooks,
+                        const uint16_t *scales, const uint16_t *x, const uint16_t *gy, int T,
+                        float *grad_scales, float *grad_codebooks, void *workspace,
+                        size_t workspace_bytes, aq_stream_t stream)
+{
+    aq_status st = check_desc(desc);
+    if (st != AQ_OK) return st;
+    if (T < 8 || T > (1 << 22) || T % 8) return AQ_ERR_INVALID_ARG;
+    if (!packed || !codebooks || !x || !gy) return AQ_ERR_INVALID_ARG;
+    if (!aligned16(packed) || !aligned16(codebooks) || !aligned16(x) || !aligned16(gy) ||
+        (grad_scales && !aligned16(grad_scales)) || (grad_codebooks && !aligned16(grad_codebooks)))
+        return AQ_ERR_MISALIGNED;
+    if (scales && (reinterpret_cast<uintptr_t>(scales) & 1u)) return AQ_ERR_MISALIGNED;
+    const Geom g = aqk::make_geom(*desc);
+    const size_t need = aqh::param_grad_workspace_bytes(g, T);
+    if (!workspace || workspace_bytes < need) return AQ_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return AQ_ERR_MISALIGNED;
+    return from_cuda(aqh::launch_param_grad(g, packed, codebooks, scales, x, gy, T, grad_scales, grad_codebooks,
+                                            workspace, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

@@ -218,6 +218,37 @@ aq_status aq_gemm(const aq_layer_desc *desc, const void *packed, const uint16_t 
                   const uint16_t *scales, const uint16_t *x, int T, uint16_t *y,
                   void *workspace, size_t workspace_bytes, aq_stream_t stream);
 
+/*
+ * Parameter gradient of a quantised layer: for the loss L = sum(gy * y) with
+ * y = diag(s) W x (the product of aq_gemm), the gradients with respect to
+ * the row scales and the codebook entries, which the step that fine-tunes
+ * the codebooks after the codes are fixed needs (AQLM wiki entry, "Niveau
+ * tech avancé": codebooks learned jointly with the codes by minimising the
+ * layer's output error).  The decode's binary16 rounding is taken as the
+ * identity, so with M[o][i] = sum_b gy[o][b] x[i][b]:
+ *
+ *     grad_scales[o]          = sum_i W[o][i] M[o][i]
+ *     grad_codebooks[k][c][j] = sum of s[o] M[o][8g+j] over the groups (o, g)
+ *                               whose code k is c          (s = 1 if NULL)
+ *
+ *   x              [in][T]  binary16 (the layer input),
+ *   gy             [out][T] binary16 (dL/dy),
+ *   T              tokens, 8..1<<22 and a multiple of 8 (the rows of x and
+ *                  gy are read by TMA, whose row pitch must be a multiple of
+ *                  16 bytes; pad with zero tokens otherwise),
+ *   grad_scales    [out] fp32, overwritten; NULL to skip,
+ *   grad_codebooks [K][2^B][8] fp32, overwritten; NULL to skip,
+ *   workspace      >= aq_param_grad_workspace_bytes(desc, T) bytes (status
+ *                  word; AQ_ERR_TIMEOUT there if a bounded wait gave up).
+ * The sums are accumulated with fp32 atomic adds: their order, and so the
+ * last bits of the result, may change from run to run.
+ */
+size_t aq_param_grad_workspace_bytes(const aq_layer_desc *desc, int T);
+aq_status aq_param_grad(const aq_layer_desc *desc, const void *packed, const uint16_t *codebooks,
+                        const uint16_t *scales, const uint16_t *x, const uint16_t *gy, int T,
+                        float *grad_scales, float *grad_codebooks, void *workspace,
+                        size_t workspace_bytes, aq_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

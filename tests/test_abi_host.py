@@ -172,3 +172,21 @@ def test_noalloc_scratch_size_matches_header():
     text = open(HEADER).read()
     m = re.search(r"#define AQ_GEMV_NOALLOC_SCRATCH_BYTES \((\d+)u << (\d+)\)", text)
     assert m and int(m.group(1)) << int(m.group(2)) == aq.GEMV_NOALLOC_SCRATCH_BYTES
+
+
+def test_param_grad_argument_errors():
+    d = aq.LayerDesc.make(64, 256, 2, 8)
+    f = aq.lib.aq_param_grad
+
+    def call(T=64, x=FAKE, gy=FAKE, gs=FAKE, gc=FAKE, ws=FAKE, wsb=1 << 20, packed=FAKE, s=FAKE):
+        return f(ctypes.byref(d), packed, FAKE, s, x, gy, T, gs, gc, ws, wsb, None)
+
+    assert aq.aq_param_grad_workspace_bytes(d, 64) >= 16
+    assert aq.aq_param_grad_workspace_bytes(d, 12) == 0  # T % 8
+    assert call(T=0) == 1 and call(T=12) == 1 and call(T=4) == 1
+    assert call(x=None) == 1 and call(gy=None) == 1 and call(packed=None) == 1
+    assert call(x=FAKE + 8) == 3 and call(gy=FAKE + 2) == 3
+    assert call(gs=FAKE + 4) == 3 and call(gc=FAKE + 8) == 3 and call(s=FAKE + 1) == 3
+    assert call(ws=None) == 4 and call(wsb=4) == 4
+    bad = aq.LayerDesc.make(64, 256, 4, 8)
+    assert f(ctypes.byref(bad), FAKE, FAKE, FAKE, FAKE, FAKE, 64, FAKE, FAKE, FAKE, 1 << 20, None) == 2
