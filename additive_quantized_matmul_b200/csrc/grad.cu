@@ -14,10 +14,14 @@
 // both operands K-major, 128-byte swizzle, loaded by TMA without multicast,
 // fp32 accumulator in tensor memory).  The epilogue reads M from TMEM, one
 // row per thread: it decodes the row's 16 weight groups for grad_s, and
-// scatters s[o] M into grad_C -- through shared-memory fp32 accumulators for
-// 8-bit codebooks (flushed once per CTA), by global vector atomics for the
-// 65536-entry 16-bit codebooks.  Atomic adds make the summation order of
-// grad_C and grad_s vary from run to run (fp32 rounding only).
+// scatters s[o] M into grad_C.  8-bit codebooks: fp32 accumulators in shared
+// memory, one private copy per epilogue warp, updated without atomics (lanes
+// holding the same codeword take turns, found with __match_any_sync; shared
+// float atomics cost 2.5x the whole kernel here), summed and flushed to
+// global memory once per CTA; 8x8, whose four copies would not fit, keeps
+// one copy with shared atomics.  16-bit codebooks (65536 entries): global
+// float4 atomics.  Global atomics make the summation order of grad_C and
+// grad_s vary from run to run (fp32 rounding only).
 //
 // Roles: warp 0 TMA producer, warp 1 MMA issuer, warps 2-5 epilogue.  Every
 // wait is bounded; on give-up the kernel records AQ_ERR_TIMEOUT, drains what
@@ -42,10 +46,16 @@ constexpr int kGradTileB = kGradBN * kGradBK * 2;  // 16 KiB of x
 template <class S>
 constexpr int kGradStagesOf = (S::kSmemBookBytes > 8192) ? 3 : 4;
 
+// 8-bit codebook gradients accumulate in shared memory: one private copy
+// per epilogue warp (race-free adds, no atomics) when four copies fit, else
+// (8x8) one copy updated with shared-memory atomics.
+template <class S>
+constexpr bool kGradPrivateAcc = S::kBooksInSmem && S::K <= 2;
+
 template <class S>
 constexpr int grad_acc_floats()
 {
-    return S::kBooksInSmem ? S::K * 256 * 8 : 0;
+    return S::kBooksInSmem ? S::K * 256 * 8 * (kGradPrivateAcc<S> ? 4 : 1) : 0;
 }
 
 template <class S>
@@ -165,6 +175,7 @@ param_grad_kernel(const __grid_constant__ CUtensorMap gymap, const __grid_consta
             const float so = (row_ok && scales) ? __half2float(__ushort_as_half(scales[o])) : 1.f;
             const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16);
             float gs = 0.f;
+            float *wacc = sacc + (kGradPrivateAcc<S> ? (warp - 2) * S::K * 256 * 8 : 0);
 #pragma unroll 1
             for (int c0 = 0; c0 < kGradBN; c0 += 16) {
                 float v[16];
@@ -172,13 +183,18 @@ param_grad_kernel(const __grid_constant__ CUtensorMap gymap, const __grid_consta
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     const int g = (n0 + c0) / 8 + h;
-                    if (!row_ok || g >= L.G) continue;
-                    const uint64_t word = load_word<S>(L, packed, o, g);
+                    if (g >= L.G) continue;  // the same for the whole warp
                     uint32_t code[S::K];
+                    if (row_ok) {
+                        const uint64_t word = load_word<S>(L, packed, o, g);
 #pragma unroll
-                    for (int k = 0; k < S::K; ++k) code[k] = (uint32_t)(word >> (k * S::B)) & S::kMask;
+                        for (int k = 0; k < S::K; ++k) code[k] = (uint32_t)(word >> (k * S::B)) & S::kMask;
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < S::K; ++k) code[k] = 0u;
+                    }
                     const float *m = v + 8 * h;
-                    if (grad_s) {
+                    if (grad_s && row_ok) {
                         uint4 t[S::K];
 #pragma unroll
                         for (int k = 0; k < S::K; ++k) {
@@ -197,14 +213,36 @@ param_grad_kernel(const __grid_constant__ CUtensorMap gymap, const __grid_consta
                     if (grad_cb) {
 #pragma unroll
                         for (int k = 0; k < S::K; ++k) {
-                            if constexpr (S::kBooksInSmem) {
-                                float *a = sacc + (k * 256 + code[k]) * 8;
+                            const float4 a0 = make_float4(so * m[0], so * m[1], so * m[2], so * m[3]);
+                            const float4 a1 = make_float4(so * m[4], so * m[5], so * m[6], so * m[7]);
+                            if constexpr (kGradPrivateAcc<S>) {
+                                // lanes with the same codeword take turns (rank among
+                                // their peers); other lanes' rows go in the same round
+                                const uint32_t key = row_ok ? (uint32_t)code[k] : 0x10000u + lane;
+                                const uint32_t peers = __match_any_sync(0xffffffffu, key);
+                                const int rank = __popc(peers & ((1u << lane) - 1u));
+                                const int rounds = (int)__reduce_max_sync(0xffffffffu, (uint32_t)__popc(peers));
+                                float4 *dst = reinterpret_cast<float4 *>(wacc + (k * 256 + code[k]) * 8);
+                                for (int r = 0; r < rounds; ++r) {
+                                    if (row_ok && rank == r) {
+                                        float4 b0 = dst[0], b1 = dst[1];
+                                        b0.x += a0.x; b0.y += a0.y; b0.z += a0.z; b0.w += a0.w;
+                                        b1.x += a1.x; b1.y += a1.y; b1.z += a1.z; b1.w += a1.w;
+                                        dst[0] = b0;
+                                        dst[1] = b1;
+                                    }
+                                    __syncwarp();
+                                }
+                            } else if constexpr (S::kBooksInSmem) {
+                                if (row_ok) {
+                                    float *a = wacc + (k * 256 + code[k]) * 8;
 #pragma unroll
-                                for (int j = 0; j < 8; ++j) atomicAdd(a + j, so * m[j]);
-                            } else {
+                                    for (int j = 0; j < 8; ++j) atomicAdd(a + j, so * m[j]);
+                                }
+                            } else if (row_ok) {
                                 float4 *a = reinterpret_cast<float4 *>(grad_cb + (((size_t)k << S::B) + code[k]) * 8);
-                                atomicAdd(a, make_float4(so * m[0], so * m[1], so * m[2], so * m[3]));
-                                atomicAdd(a + 1, make_float4(so * m[4], so * m[5], so * m[6], so * m[7]));
+                                atomicAdd(a, a0);
+                                atomicAdd(a + 1, a1);
                             }
                         }
                     }
@@ -222,11 +260,21 @@ param_grad_kernel(const __grid_constant__ CUtensorMap gymap, const __grid_consta
             for (int s = max(0, nk - ST); s < nk; ++s) mbar_wait_ns(&full[s % ST], (s / ST) & 1, kWaitNs);
     } else if constexpr (S::kBooksInSmem) {
         // this CTA's share of the 8-bit codebook gradient, once
-        if (grad_cb)
-            for (int i = tid; i < grad_acc_floats<S>(); i += kGradThreads) {
-                const float a = sacc[i];
-                if (a != 0.f) atomicAdd(grad_cb + i, a);
+        if (grad_cb) {
+            constexpr int n4 = S::K * 256 * 8 / 4;  // float4 per copy
+            constexpr int copies = kGradPrivateAcc<S> ? 4 : 1;
+            const float4 *acc4 = reinterpret_cast<const float4 *>(sacc);
+            for (int i = tid; i < n4; i += kGradThreads) {
+                float4 a = acc4[i];
+#pragma unroll
+                for (int w = 1; w < copies; ++w) {
+                    const float4 b = acc4[w * n4 + i];
+                    a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
+                }
+                if (a.x != 0.f || a.y != 0.f || a.z != 0.f || a.w != 0.f)
+                    atomicAdd(reinterpret_cast<float4 *>(grad_cb) + i, a);
             }
+        }
     }
     tc_fence_before();
     __syncthreads();

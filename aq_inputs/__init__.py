@@ -142,6 +142,11 @@ def workload(name: str) -> dict:
             for tag, (o, i) in LLAMA2_7B_BLOCK.items():
                 layers.append((f"{tag}-{K}x{B}", LayerSpec(o, i, K, B)))
         return {"layers": layers, "n": [512, 2048], "seed": 1004}
+    if name == "llama2-7b-grad":
+        # parameter gradient (codebooks, scales) of block shapes over 2048 tokens
+        layers = [(f"{tag}-{K}x{B}", LayerSpec(o, i, K, B)) for K, B in ((1, 16), (2, 8))
+                  for tag, (o, i) in (("q", LLAMA2_7B_BLOCK["q"]), ("gate", LLAMA2_7B_BLOCK["gate"]))]
+        return {"layers": layers, "n": [2048], "seed": 1007}
     if name == "llama2-7b-schemes":
         # the other schemes the pages name, at the Llama-2-7B MLP up shape
         layers = [(f"11008x4096-{K}x{B}", LayerSpec(11008, 4096, K, B)) for K, B in ((1, 8), (2, 16), (8, 8))]
@@ -162,4 +167,4 @@ def workload(name: str) -> dict:
 
 
 WORKLOADS = ("tiny-2x8", "llama2-7b-1x16", "llama2-7b-mlp-2x8",
-             "llama2-70b-1x16", "llama2-7b-prefill", "llama2-7b-block", "llama2-7b-schemes")
+             "llama2-70b-1x16", "llama2-7b-prefill", "llama2-7b-block", "llama2-7b-schemes", "llama2-7b-grad")

@@ -283,7 +283,8 @@ def run_gpu(args) -> None:
     dist = init_dist(world, "nccl")
     dev = torch.device("cuda", local)
     wl = workload(args.workload)
-    op = "gemm" if args.workload == "llama2-7b-prefill" else "gemv"
+    op = {"llama2-7b-prefill": "gemm", "llama2-7b-grad": "grad"}.get(args.workload, "gemv")
+    tensor_op = op in ("gemm", "grad")  # reported in TFLOP/s against the tensor peak
     peaks = measured_peaks()
 
     # ---- units: one (layer shape, batch) product kind each, over a rotation
@@ -302,15 +303,21 @@ def run_gpu(args) -> None:
     for si, (tag, spec) in enumerate(wl["layers"]):
         desc, packed0, cb0, sc0 = device_layer(spec, (wl["seed"], rank, si))  # seeded per rank and shape
         lb = alg_bytes(spec, 0)
-        ncopies = args.layers or max(3 if op == "gemm" else 4, int(3 * L2_BYTES / lb) + 1)
+        ncopies = args.layers or (3 if tensor_op else max(4, int(3 * L2_BYTES / lb) + 1))
         copies = [(packed0.clone(), cb0.clone(), sc0.clone()) for _ in range(ncopies)]
         del packed0, cb0, sc0
         for n in wl["n"]:
             x = torch.from_numpy(make_activations(spec.in_features, n, (wl["seed"], rank, si, n)).view(np.int16)).to(dev)
-            nbytes = (aq.aq_gemm_workspace_bytes(desc, n) if op == "gemm" else aq.aq_gemv_workspace_bytes(desc, n))
+            nbytes = {"gemm": aq.aq_gemm_workspace_bytes, "grad": aq.aq_param_grad_workspace_bytes,
+                      "gemv": aq.aq_gemv_workspace_bytes}[op](desc, n)
             units.append({
                 "tag": tag, "spec": spec, "n": n, "desc": desc, "copies": copies, "x": x,
                 "bytes": alg_bytes(spec, n), "flops": flops(spec, n),
+                **({"gy": torch.from_numpy(make_activations(spec.out_features, n, (wl["seed"], rank, si, n, 1))
+                                           .view(np.int16)).to(dev),
+                    "grad_s": torch.empty(spec.out_features, dtype=torch.float32, device=dev),
+                    "grad_cb": torch.empty((spec.num_codebooks << spec.nbits) * 8, dtype=torch.float32, device=dev)}
+                   if op == "grad" else {}),
                 "ys": [torch.empty(spec.out_features * n, dtype=torch.int16, device=dev) for _ in range(ncopies)],
                 "ws": torch.zeros(max(nbytes, 16), dtype=torch.uint8, device=dev),
                 # two events per group of same-shape launches (event nodes between
@@ -352,7 +359,10 @@ def run_gpu(args) -> None:
                 aq.aq_gemv(desc, packed, cb, sc, inp, 1, out, u["ws"], stream=s)
             return
         packed, cb, sc = u["copies"][i]
-        if op == "gemm":
+        if op == "grad":
+            aq.aq_param_grad(u["desc"], packed, cb, sc, x_in, u["gy"], u["n"], u["grad_s"], u["grad_cb"], u["ws"],
+                             stream=s)
+        elif op == "gemm":
             aq.aq_gemm(u["desc"], packed, cb, sc, x_in, u["n"], y_out, u["ws"], stream=s)
         else:
             aq.aq_gemv(u["desc"], packed, cb, sc, x_in, u["n"], y_out, u["ws"], stream=s)
@@ -426,12 +436,12 @@ def run_gpu(args) -> None:
         k["frac_tensor"] = round(k["tflops"] / peaks["bf16_tflops_sustained"], 4)
         kernels.append(k)
     dom = max(kernels, key=lambda k: k["total_us"])
-    if op == "gemm":
+    if tensor_op:
         value = world * step_flops * args.steps / (elapsed_ms * 1e-3) / 1e12
         unit = "TFLOP/s"
         roofline = {"bound": "tensor", "achieved": dom["tflops"], "peak": peaks["bf16_tflops_sustained"],
                     "unit": "TFLOP/s", "frac": dom["frac_tensor"], "traffic": None,
-                    "kernel": f"aq_gemm {dom['layer']} T={dom['n']}",
+                    "kernel": f"aq_{'param_grad' if op == 'grad' else 'gemm'} {dom['layer']} T={dom['n']}",
                     "peak_source": f"{peaks['source']} bf16_tflops_sustained (cuBLAS bf16; fp16 tcgen05 has the same rate)"}
     else:
         value = world * step_bytes * args.steps / (elapsed_ms * 1e-3) / 1e9
@@ -445,7 +455,7 @@ def run_gpu(args) -> None:
 
     # ---- end-to-end through the public API with host buffers ----------------
     e2e = None
-    if not args.skip_e2e:
+    if not args.skip_e2e and op != "grad":  # the gradient's outputs are parameters, not a per-step result
         hx = [torch.empty((len(u["copies"]), u["x"].numel()), dtype=torch.int16).pin_memory() for u in units]
         hy = [torch.empty((len(u["copies"]), out_buf(u, 0).numel()), dtype=torch.int16).pin_memory() for u in units]
         dx = [torch.empty(h.shape, dtype=torch.int16, device=dev) for h in hx]
@@ -477,7 +487,7 @@ def run_gpu(args) -> None:
         e1.record()
         torch.cuda.synchronize()
         e_ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
-        tot = (step_flops / 1e12) if op == "gemm" else (step_bytes / 1e9)
+        tot = (step_flops / 1e12) if tensor_op else (step_bytes / 1e9)
         e2e = {"value": round(world * tot * e_steps / (e_ms * 1e-3), 2), "unit": unit,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e_steps,
                "api": "additive_quantized_matmul_b200 (C ABI via ctypes), eager, pinned host buffers"}
@@ -526,7 +536,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=WORKLOAD,
                     help="llama2-7b-1x16 (default), llama2-7b-mlp-2x8, llama2-70b-1x16, "
-                         "llama2-7b-prefill, llama2-7b-block, llama2-7b-schemes, tiny-2x8")
+                         "llama2-7b-prefill, llama2-7b-block, llama2-7b-schemes, llama2-7b-grad, tiny-2x8")
     ap.add_argument("--layers", type=int, default=0, help="copies per shape (0: > 3x L2)")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--skip-e2e", action="store_true")
