@@ -9,7 +9,9 @@
 //     grad_s[o]       = sum_i W[o][i] M[o][i]
 //     grad_C[k][c][j] = sum of s[o] M[o][8g+j] over the (o, g) whose code k is c.
 //
-// One kernel: CTA tile 128 rows x 128 input features (16 groups); the
+// One persistent kernel (a CTA per SM walks 128-row x 128-feature tiles,
+// 16 groups each, with two accumulator buffers in tensor memory so the
+// epilogue of one tile overlaps the MMAs of the next); the
 // contraction over tokens runs on the tensor cores (tcgen05.mma kind::f16,
 // both operands K-major, 128-byte swizzle, loaded by TMA without multicast,
 // fp32 accumulator in tensor memory).  The epilogue reads M from TMEM, one
@@ -29,6 +31,8 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
+
 #include "scheme.cuh"
 #include "tc_common.cuh"
 
@@ -38,6 +42,7 @@ constexpr int kGradBM = 128;                      // rows of W per CTA (MMA M)
 constexpr int kGradBN = 128;                      // input features per CTA (MMA N)
 constexpr int kGradBK = 64;                       // tokens per stage
 constexpr int kGradThreads = 192;                 // 6 warps
+constexpr int kGradEpilogueThreads = 128;         // warps 2-5
 constexpr int kGradTileA = kGradBM * kGradBK * 2;  // 16 KiB of gy
 constexpr int kGradTileB = kGradBN * kGradBK * 2;  // 16 KiB of x
 
@@ -62,7 +67,7 @@ template <class S>
 constexpr int grad_smem_bytes()
 {
     return 1024 + kGradStagesOf<S> * (kGradTileA + kGradTileB) + S::kSmemBookBytes + grad_acc_floats<S>() * 4 +
-           (2 * kGradStagesOf<S> + 1) * 8 + 16;
+           (2 * kGradStagesOf<S> + 4) * 8 + 16;
 }
 
 // The packed word of (row o, group g): K*B/8 bytes.
@@ -93,13 +98,14 @@ param_grad_kernel(const __grid_constant__ CUtensorMap gymap, const __grid_consta
     float *sacc = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(scb) + S::kSmemBookBytes);
     uint64_t *full = reinterpret_cast<uint64_t *>(sacc + grad_acc_floats<S>());
     uint64_t *empty = full + ST;
-    uint64_t *acc_full = empty + ST;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 1);
+    uint64_t *acc_full = empty + ST;   // [2] accumulator buffer ready for the epilogue
+    uint64_t *acc_empty = acc_full + 2;  // [2] accumulator buffer drained by the epilogue
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 2);
     uint32_t *abort_flag = tmem_slot + 1;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int m0 = blockIdx.x * kGradBM;
-    const int n0 = blockIdx.y * kGradBN;
+    const int ntn = (L.in + kGradBN - 1) / kGradBN;
+    const int ntiles = ((L.out + kGradBM - 1) / kGradBM) * ntn;
     const int nk = (T + kGradBK - 1) / kGradBK;
 
     if constexpr (S::kBooksInSmem) {
@@ -111,71 +117,100 @@ param_grad_kernel(const __grid_constant__ CUtensorMap gymap, const __grid_consta
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(acc_full, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], kGradEpilogueThreads);
+        }
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 0) tmem_alloc(tmem_slot, kGradBN);
+    if (warp == 0) tmem_alloc(tmem_slot, 2 * kGradBN);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     volatile uint32_t *abort_v = abort_flag;
 
+    // This CTA's tiles: t = blockIdx.x + gridDim.x * lt, row block t / ntn,
+    // feature block t % ntn.  Stage counter q runs across tiles.
     if (warp == 0) {
         // ---------------- TMA producer: gy and x tiles ----------------
         if (lane == 0) {
-            for (int s = 0; s < nk; ++s) {
-                const int buf = s % ST;
-                if (s >= ST && !mbar_wait_ns(&empty[buf], ((s / ST) - 1) & 1, kWaitNs)) {
-                    *abort_v = 1;
-                    break;
+            int q = 0;
+            for (int t = blockIdx.x; t < ntiles && !*abort_v; t += gridDim.x) {
+                const int m0 = (t / ntn) * kGradBM, n0 = (t % ntn) * kGradBN;
+                for (int s = 0; s < nk; ++s, ++q) {
+                    const int buf = q % ST;
+                    if (q >= ST && !mbar_wait_ns(&empty[buf], ((q / ST) - 1) & 1, kWaitNs)) {
+                        *abort_v = 1;
+                        break;
+                    }
+                    if (*abort_v) break;
+                    mbar_arrive_expect_tx(&full[buf], kGradTileA + kGradTileB);
+                    tma_load_2d(smem_u32(tileA + buf * kGradTileA), &gymap, s * kGradBK, m0, &full[buf]);
+                    tma_load_2d(smem_u32(tileB + buf * kGradTileB), &xmap, s * kGradBK, n0, &full[buf]);
                 }
-                if (*abort_v) break;
-                mbar_arrive_expect_tx(&full[buf], kGradTileA + kGradTileB);
-                tma_load_2d(smem_u32(tileA + buf * kGradTileA), &gymap, s * kGradBK, m0, &full[buf]);
-                tma_load_2d(smem_u32(tileB + buf * kGradTileB), &xmap, s * kGradBK, n0, &full[buf]);
             }
+            // copies of the last ring's worth of stages may still be landing
+            // (only after an abort): wait for them, bounded
+            for (int qq = max(0, q - ST); qq < q; ++qq) mbar_wait_ns(&full[qq % ST], (qq / ST) & 1, kWaitNs);
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
         if (lane == 0) {
             const uint32_t idesc = make_idesc(kGradBM, kGradBN, false);  // both operands K-major
-            for (int s = 0; s < nk; ++s) {
-                const int buf = s % ST;
-                if (!mbar_wait_ns(&full[buf], (s / ST) & 1, kWaitNs)) {
+            int q = 0, lt = 0;
+            for (int t = blockIdx.x; t < ntiles && !*abort_v; t += gridDim.x, ++lt) {
+                const int ab = lt & 1;
+                // the epilogue has drained this accumulator buffer (tile lt - 2)
+                if (lt >= 2 && !mbar_wait_ns(&acc_empty[ab], ((lt >> 1) - 1) & 1, kWaitNs)) {
                     *abort_v = 1;
                     break;
                 }
-                if (*abort_v) break;
                 tc_fence_after();
-                const uint32_t a0 = smem_u32(tileA + buf * kGradTileA);
-                const uint32_t b0 = smem_u32(tileB + buf * kGradTileB);
+                const uint32_t acc = tmem + (uint32_t)(ab * kGradBN);
+                for (int s = 0; s < nk; ++s, ++q) {
+                    const int buf = q % ST;
+                    if (!mbar_wait_ns(&full[buf], (q / ST) & 1, kWaitNs)) {
+                        *abort_v = 1;
+                        break;
+                    }
+                    if (*abort_v) break;
+                    tc_fence_after();
+                    const uint32_t a0 = smem_u32(tileA + buf * kGradTileA);
+                    const uint32_t b0 = smem_u32(tileB + buf * kGradTileB);
 #pragma unroll
-                for (int ks = 0; ks < kGradBK / 16; ++ks) {
-                    const uint64_t ad = smem_desc_sw128(a0 + ks * 32, 16, 1024);
-                    const uint64_t bd = smem_desc_sw128(b0 + ks * 32, 16, 1024);
-                    mma_f16_ss(tmem, ad, bd, idesc, (s > 0 || ks > 0) ? 1u : 0u);
+                    for (int ks = 0; ks < kGradBK / 16; ++ks) {
+                        const uint64_t ad = smem_desc_sw128(a0 + ks * 32, 16, 1024);
+                        const uint64_t bd = smem_desc_sw128(b0 + ks * 32, 16, 1024);
+                        mma_f16_ss(acc, ad, bd, idesc, (s > 0 || ks > 0) ? 1u : 0u);
+                    }
+                    mma_commit(&empty[buf]);
                 }
-                mma_commit(&empty[buf]);
+                mma_commit(&acc_full[ab]);  // completes when this tile's MMAs have
             }
-            mma_commit(acc_full);  // completes when every MMA issued above has
+            // the last stage's commit completes once every MMA issued here has:
+            // none may still write tensor memory when it is freed
+            if (q > 0) mbar_wait_ns(&empty[(q - 1) % ST], ((q - 1) / ST) & 1, kWaitNs);
         }
     } else {
-        // ---------------- epilogue: one row per thread ----------------
-        const bool got = (*abort_v == 0) && mbar_wait_ns(acc_full, 0, kWaitNs);
-        if (!got) *abort_v = 1;
-        tc_fence_after();
-        // every lane of the warp takes the same branch (tcgen05.ld is
-        // warp-collective): a failed wait in any lane skips the whole warp
-        if (__all_sync(0xffffffffu, got)) {
-            const int q = warp & 3;  // TMEM lane quarter of this warp
-            const int o = m0 + q * 32 + lane;
+        // ---------------- epilogue: one row per thread, tile after tile ----------------
+        const int qd = warp & 3;  // TMEM lane quarter of this warp
+        float *wacc = sacc + (kGradPrivateAcc<S> ? (warp - 2) * S::K * 256 * 8 : 0);
+        int lt = 0;
+        for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++lt) {
+            const int ab = lt & 1;
+            const bool got = (*abort_v == 0) && mbar_wait_ns(&acc_full[ab], (lt >> 1) & 1, kWaitNs);
+            if (!got) *abort_v = 1;
+            // tcgen05.ld is warp-collective: a failed wait in any lane ends the warp
+            if (!__all_sync(0xffffffffu, got)) break;
+            tc_fence_after();
+            const int m0 = (t / ntn) * kGradBM, n0 = (t % ntn) * kGradBN;
+            const int o = m0 + qd * 32 + lane;
             const bool row_ok = o < L.out;
             const float so = (row_ok && scales) ? __half2float(__ushort_as_half(scales[o])) : 1.f;
-            const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16);
+            const uint32_t tbase = tmem + (uint32_t)(ab * kGradBN) + ((uint32_t)(qd * 32) << 16);
             float gs = 0.f;
-            float *wacc = sacc + (kGradPrivateAcc<S> ? (warp - 2) * S::K * 256 * 8 : 0);
 #pragma unroll 1
             for (int c0 = 0; c0 < kGradBN; c0 += 16) {
                 float v[16];
@@ -249,15 +284,13 @@ param_grad_kernel(const __grid_constant__ CUtensorMap gymap, const __grid_consta
                 }
             }
             if (row_ok && grad_s) atomicAdd(grad_s + o, gs);
+            tc_fence_before();
+            mbar_arrive(&acc_empty[ab]);  // this thread is done with the buffer
         }
     }
     __syncthreads();
     if (*abort_v) {
-        // something gave up: record it and drain what was issued (bounded)
         if (tid == 0) record_status(ws, AQ_ERR_TIMEOUT);
-        if (tid == 32) mbar_wait_ns(acc_full, 0, kWaitNs);
-        if (tid == 0)
-            for (int s = max(0, nk - ST); s < nk; ++s) mbar_wait_ns(&full[s % ST], (s / ST) & 1, kWaitNs);
     } else if constexpr (S::kBooksInSmem) {
         // this CTA's share of the 8-bit codebook gradient, once
         if (grad_cb) {
@@ -278,7 +311,7 @@ param_grad_kernel(const __grid_constant__ CUtensorMap gymap, const __grid_consta
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, kGradBN);
+    if (warp == 0) tmem_dealloc(tmem, 2 * kGradBN);
 }
 
 }  // namespace aqk
@@ -333,7 +366,10 @@ cudaError_t launch_param_grad(const Geom &g, const void *packed, const uint16_t 
     CUtensorMap gymap, xmap;
     if (!token_major_map(encode, &gymap, gy, g.out, T) || !token_major_map(encode, &xmap, x, g.in, T))
         return cudaErrorInvalidValue;
-    const dim3 grid((g.out + kGradBM - 1) / kGradBM, (g.in + kGradBN - 1) / kGradBN);
+    // persistent: one CTA per SM (its shared memory allows no second), each
+    // walking tiles blockIdx.x, blockIdx.x + gridDim.x, ...
+    const long ntiles = (long)((g.out + kGradBM - 1) / kGradBM) * ((g.in + kGradBN - 1) / kGradBN);
+    const dim3 grid((unsigned)std::min<long>(ntiles, kNumSMs));
     const uint8_t *pk = reinterpret_cast<const uint8_t *>(packed);
     const uint4 *c = reinterpret_cast<const uint4 *>(cb);
     return with_scheme(g, [&](auto sch) {
