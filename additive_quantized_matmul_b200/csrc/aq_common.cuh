@@ -48,6 +48,8 @@ inline Geom make_geom(const aq_layer_desc &d)
     return g;
 }
 
+inline size_t align16(size_t v) { return (v + 15) / 16 * 16; }
+
 // Workspace header: status word at byte 0 (AQ_ERR_TIMEOUT when a bounded
 // wait gave up), arrival counters from byte 16.
 constexpr size_t kWsHeader = 16;

@@ -16,6 +16,9 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
+#include <type_traits>
+
 #include "scheme.cuh"
 #include "tc_common.cuh"
 
@@ -184,14 +187,19 @@ gemm_tc_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restri
 
 // ---- warp-specialised kernel (T a multiple of 8) ---------------------------
 //
-// Tile M = 128 rows x N = 256 tokens, K = 64 per stage, 4-stage ring.
-//   warp 0     X producer: one lane issues four 2-D TMA loads per stage (64
+// Tile M = 128 rows x N = BN tokens (256 or 512), K = 64 per stage; the
+// decoded W tile feeds BN tokens, so BN = 512 halves the decode work per
+// MMA (the 1x16 decode, ~1024 random L2 gathers per stage, is slower than
+// the four N = 256 MMAs of a stage).  Split-K over the input features
+// (blockIdx.z) fills the SMs when the tile grid is small.
+//   warp 0     X producer: one lane issues BN/64 2-D TMA loads per stage (64
 //              tokens x 64 features each, 128-byte swizzle, MN-major) that
 //              complete on full_b[stage];
-//   warp 1     MMA issuer: one lane waits for full_a/full_b, issues four
-//              tcgen05.mma (M 128, N 256, K 16) into a 256-column fp32 TMEM
-//              accumulator and commits to empty[stage] (buffer free) and,
-//              after the last stage, to acc_full;
+//   warp 1     MMA issuer: one lane waits for full_a/full_b, issues
+//              tcgen05.mma (M 128, N 256, K 16; two per K step for BN = 512)
+//              into a BN-column fp32 TMEM accumulator and commits to
+//              empty[stage] (buffer free) and, after the last stage, to
+//              acc_full;
 //   warps 2-5  decoders, then epilogue: thread t owns code chunk (row tile
 //              t/8, group t%8) of each stage.  1x16: the 8 codewords go from
 //              the L2-resident codebook straight into the swizzled A tile by
@@ -199,23 +207,98 @@ gemm_tc_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restri
 //              the codebooks in shared memory, summed with binary16 adds.
 //              Each thread fences its writes to the async proxy and arrives
 //              on full_a[stage] (128 arrivals).  The epilogue reads TMEM lanes
-//              32*(warp%4).. with tcgen05.ld, scales, rounds and stores.
-constexpr int kWsBN = 256;
-// ring depth: 4 stages, 3 when the 32 KiB of 8x8 codebooks share the
-// shared memory (4 x 48 KiB + 32 KiB would not fit)
-template <class S>
-constexpr int kWsStagesOf = (S::kSmemBookBytes > 8192) ? 3 : 4;
+//              32*(warp%4).. with tcgen05.ld, scales, rounds and stores (one
+//              split), or stores fp32 partial sums that the last CTA of the
+//              tile adds in split order (several splits).
+// Ring depth: 4 stages of (16 KiB A + 32 KiB B) for BN = 256, 3 when the
+// 32 KiB of 8x8 codebooks share the shared memory; 2 stages of (16 + 64 KiB)
+// for BN = 512.
+template <class S, int BN>
+constexpr int kWsStagesOf = (BN == 512) ? 2 : (S::kSmemBookBytes > 8192) ? 3 : 4;
 constexpr int kWsThreads = 192;               // 6 warps
-constexpr int kWsTileB = kBK * kWsBN * 2;     // 32 KiB
 constexpr int kWsLag = 2;                     // cp.async stages in flight per decoder (< ring depth)
 
-template <class S>
+struct GemmSplit {
+    float *partials;     // [splits][out][T] fp32, or null with one split
+    unsigned *counters;  // [grid.x * grid.y] arrivals per output tile
+};
+
+// Called by every thread after the CTA stored its partial sums for output
+// tile (m0, n0) of split blockIdx.z.  The last CTA of the tile to arrive adds
+// the splits in split order (bit-reproducible), scales, rounds to binary16,
+// writes y and resets the tile's counter for the next call.
+__device__ __forceinline__ void gemm_split_finish(const Geom &L, GemmSplit sp, int m0, int n0, int bn, int T,
+                                                  const uint16_t *__restrict__ scales, uint16_t *__restrict__ y)
+{
+    __shared__ unsigned s_last;
+    __syncthreads();
+    const unsigned tile = blockIdx.y * gridDim.x + blockIdx.x;
+    if (threadIdx.x == 0) {
+        // the barrier orders the CTA's partial stores before this thread's
+        // release fence; the last CTA's acquire fence orders its reads
+        fence_acq_rel_gpu();
+        const unsigned prev = atomicAdd(&sp.counters[tile], 1u);
+        s_last = (prev == gridDim.z - 1) ? 1u : 0u;
+        if (s_last) fence_acq_rel_gpu();
+    }
+    __syncthreads();
+    if (!s_last) return;
+    const int cols4 = bn / 4;
+    const int ks = (int)gridDim.z;
+    const size_t zstride = (size_t)L.out * T / 4;  // float4 per split
+    // four float4 per thread per pass and four splits per batch of loads:
+    // sixteen independent L2 reads in flight; each element still adds its
+    // splits in split order
+    constexpr int kE = 4;
+    for (int e0 = threadIdx.x; e0 < kBM * cols4; e0 += kE * blockDim.x) {
+        const float4 *p[kE];
+        bool ok[kE];
+        float4 acc[kE];
+#pragma unroll
+        for (int i = 0; i < kE; ++i) {
+            const int e = e0 + i * blockDim.x;
+            const int row = m0 + e / cols4, gn = n0 + 4 * (e % cols4);
+            ok[i] = e < kBM * cols4 && row < L.out && gn < T;
+            p[i] = reinterpret_cast<const float4 *>(sp.partials + (size_t)(ok[i] ? row : 0) * T + (ok[i] ? gn : 0));
+            acc[i] = ok[i] ? __ldcg(p[i]) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        for (int z0 = 1; z0 < ks; z0 += 4) {
+            float4 t[4][kE];
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+#pragma unroll
+                for (int i = 0; i < kE; ++i)
+                    if (z0 + j < ks && ok[i]) t[j][i] = __ldcg(p[i] + (size_t)(z0 + j) * zstride);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+#pragma unroll
+                for (int i = 0; i < kE; ++i)
+                    if (z0 + j < ks && ok[i]) {
+                        acc[i].x += t[j][i].x; acc[i].y += t[j][i].y; acc[i].z += t[j][i].z; acc[i].w += t[j][i].w;
+                    }
+        }
+#pragma unroll
+        for (int i = 0; i < kE; ++i) {
+            if (!ok[i]) continue;
+            const int e = e0 + i * blockDim.x;
+            const int row = m0 + e / cols4, gn = n0 + 4 * (e % cols4);
+            const float sc = scales ? __half2float(__ushort_as_half(scales[row])) : 1.f;
+            *reinterpret_cast<uint2 *>(y + (size_t)row * T + gn) =
+                make_uint2(f2h2(sc * acc[i].x, sc * acc[i].y), f2h2(sc * acc[i].z, sc * acc[i].w));
+        }
+    }
+    if (threadIdx.x == 0) sp.counters[tile] = 0u;
+}
+
+template <class S, int BN>
 __global__ void __launch_bounds__(kWsThreads, 1)
 gemm_ws_kernel(const __grid_constant__ CUtensorMap xmap, Geom L, const uint8_t *__restrict__ packed,
                const uint4 *__restrict__ cb, const uint16_t *__restrict__ scales, int T,
-               uint16_t *__restrict__ y, void *ws)
+               uint16_t *__restrict__ y, void *ws, GemmSplit sp, int stages_per_split)
 {
-    constexpr int kWsStages = kWsStagesOf<S>;
+    constexpr int kWsStages = kWsStagesOf<S, BN>;
+    constexpr int kWsTileB = kBK * BN * 2;   // 32 or 64 KiB
+    constexpr int kN = BN < 256 ? BN : 256;  // N of one MMA instruction
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t *smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -231,8 +314,11 @@ gemm_ws_kernel(const __grid_constant__ CUtensorMap xmap, Geom L, const uint8_t *
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int m0 = blockIdx.x * kBM;
-    const int n0 = blockIdx.y * kWsBN;
-    const int nk = (L.in + kBK - 1) / kBK;
+    const int n0 = blockIdx.y * BN;
+    // this split's stages: global stages s0 .. s0 + nk - 1 (64 features each)
+    const int s0 = blockIdx.z * stages_per_split;
+    const int nk = max(0, min((L.in + kBK - 1) / kBK, s0 + stages_per_split) - s0);
+    const int g0 = s0 * 8;  // first code group of the split
 
     // 1x16: codewords go from L2 into the tile by cp.async, copies of kWsLag
     // stages in flight; other schemes decode in registers
@@ -250,7 +336,7 @@ gemm_ws_kernel(const __grid_constant__ CUtensorMap xmap, Geom L, const uint8_t *
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 0) tmem_alloc(tmem_slot, kWsBN);
+    if (warp == 0) tmem_alloc(tmem_slot, BN);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -270,14 +356,14 @@ gemm_ws_kernel(const __grid_constant__ CUtensorMap xmap, Geom L, const uint8_t *
                 mbar_arrive_expect_tx(&full_b[buf], kWsTileB);
                 const uint32_t dst = smem_u32(tileB + buf * kWsTileB);
 #pragma unroll
-                for (int q = 0; q < kWsBN / 64; ++q)
-                    tma_load_2d(dst + q * (kBK * 128), &xmap, n0 + 64 * q, s * kBK, &full_b[buf]);
+                for (int q = 0; q < BN / 64; ++q)
+                    tma_load_2d(dst + q * (kBK * 128), &xmap, n0 + 64 * q, (s0 + s) * kBK, &full_b[buf]);
             }
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
         if (lane == 0) {
-            const uint32_t idesc = make_idesc(kBM, kWsBN, true);
+            const uint32_t idesc = make_idesc(kBM, kN, true);
             int s = 0;
             for (; s < nk; ++s) {
                 const int buf = s % kWsStages;
@@ -293,8 +379,12 @@ gemm_ws_kernel(const __grid_constant__ CUtensorMap xmap, Geom L, const uint8_t *
 #pragma unroll
                 for (int ks = 0; ks < kBK / 16; ++ks) {
                     const uint64_t ad = smem_desc_sw128(a0 + ks * 32, 16, 1024);
-                    const uint64_t bd = smem_desc_sw128(b0 + ks * 2048, kBK * 128, 1024);
-                    mma_f16_ss(tmem, ad, bd, idesc, (s > 0 || ks > 0) ? 1u : 0u);
+#pragma unroll
+                    for (int h = 0; h < BN / kN; ++h) {
+                        // tokens 256 h .. : four 64-token boxes further on
+                        const uint64_t bd = smem_desc_sw128(b0 + h * (kN / 64) * (kBK * 128) + ks * 2048, kBK * 128, 1024);
+                        mma_f16_ss(tmem + h * kN, ad, bd, idesc, (s > 0 || ks > 0) ? 1u : 0u);
+                    }
                 }
                 mma_commit(&empty[buf]);
             }
@@ -312,66 +402,75 @@ gemm_ws_kernel(const __grid_constant__ CUtensorMap xmap, Geom L, const uint8_t *
         Chunk<S> code_ring[kCodeAhead];
 #pragma unroll
         for (int q = 0; q < kCodeAhead; ++q)
-            code_ring[q] = load_chunk<S>(packed, (size_t)rt * L.gp + q * 8 + gi, q < nk && rows_live && q * 8 + gi < L.G);
-        const int lag = kAsyncWeights ? kWsLag : 0;
-        for (int s = 0; s < nk + lag; ++s) {
-            if (s < nk) {
-                const int buf = s % kWsStages;
-                if (s >= kWsStages && !mbar_wait_ns(&empty[buf], ((s / kWsStages) - 1) & 1, kWaitNs)) {
-                    *abort_v = 1;
-                }
-                if (*abort_v) break;
-                Chunk<S> code = code_ring[0];
+            code_ring[q] = load_chunk<S>(packed, (size_t)rt * L.gp + g0 + q * 8 + gi,
+                                         q < nk && rows_live && g0 + q * 8 + gi < L.G);
+        // copies of kLag stages stay in flight; a stage is published kLag
+        // iterations after it is issued, so kLag must stay below the ring
+        // depth (the decoder waits for the MMAs of stage s - depth first)
+        constexpr int kLag = kAsyncWeights ? (kWsLag < kWsStages - 1 ? kWsLag : kWsStages - 1) : 0;
+        static_assert(kLag < kWsStages, "copy lag must be below the ring depth");
+        bool ok = true;
+        // unrolled by the ring depth so every ring index is static
+        for (int s0i = 0; ok && s0i < nk + kLag; s0i += kCodeAhead) {
 #pragma unroll
-                for (int q = 1; q < kCodeAhead; ++q)
-                    if ((s & (kCodeAhead - 1)) == q) code = code_ring[q];
-                const bool live = rows_live && s * 8 + gi < L.G;
-                {
-                    const int g = (s + kCodeAhead) * 8 + gi;
-                    const Chunk<S> nxt = load_chunk<S>(packed, (size_t)rt * L.gp + g,
-                                                       s + kCodeAhead < nk && rows_live && g < L.G);
+            for (int u = 0; u < kCodeAhead; ++u) {
+                const int s = s0i + u;
+                if (s >= nk + kLag) break;
+                if (s < nk) {
+                    const int buf = s % kWsStages;
+                    if (s >= kWsStages && !mbar_wait_ns(&empty[buf], ((s / kWsStages) - 1) & 1, kWaitNs)) {
+                        *abort_v = 1;
+                    }
+                    if (*abort_v) {
+                        ok = false;
+                        break;
+                    }
+                    const Chunk<S> code = code_ring[u];
+                    const bool live = rows_live && g0 + s * 8 + gi < L.G;
+                    {
+                        const int g = g0 + (s + kCodeAhead) * 8 + gi;
+                        code_ring[u] = load_chunk<S>(packed, (size_t)rt * L.gp + g,
+                                                     s + kCodeAhead < nk && rows_live && g < L.G);
+                    }
+                    uint8_t *A = tileA + buf * kTileABytes;
+                    if constexpr (kAsyncWeights) {
+                        const uint32_t a0 = smem_u32(A);
 #pragma unroll
-                    for (int q = 0; q < kCodeAhead; ++q)
-                        if ((s & (kCodeAhead - 1)) == q) code_ring[q] = nxt;
-                }
-                uint8_t *A = tileA + buf * kTileABytes;
-                if constexpr (kAsyncWeights) {
-                    const uint32_t a0 = smem_u32(A);
+                        for (int r = 0; r < 8; ++r)
+                            cp_async16(a0 + sw128(rt_l * 8 + r, gi),
+                                       live ? (const void *)(cb + code.code(r, 0)) : (const void *)cb, live ? 16u : 0u);
+                    } else if constexpr (S::K <= 2) {
+                        // all codeword reads before the first tile store (the
+                        // books and the tile share one shared array)
+                        uint4 t[8][S::K];
 #pragma unroll
-                    for (int r = 0; r < 8; ++r)
-                        cp_async16(a0 + sw128(rt_l * 8 + r, gi),
-                                   live ? (const void *)(cb + code.code(r, 0)) : (const void *)cb, live ? 16u : 0u);
-                } else if constexpr (S::K <= 2) {
-                    // all codeword reads before the first tile store (the
-                    // books and the tile share one shared array)
-                    uint4 t[8][S::K];
+                        for (int r = 0; r < 8; ++r) gather_terms<S>(code, r, scb, cb, t[r]);
 #pragma unroll
-                    for (int r = 0; r < 8; ++r) gather_terms<S>(code, r, scb, cb, t[r]);
+                        for (int r = 0; r < 8; ++r)
+                            *reinterpret_cast<uint4 *>(A + sw128(rt_l * 8 + r, gi)) =
+                                live ? sum_round_fast_h8<S::K>(t[r]) : make_uint4(0, 0, 0, 0);
+                    } else {
 #pragma unroll
-                    for (int r = 0; r < 8; ++r)
-                        *reinterpret_cast<uint4 *>(A + sw128(rt_l * 8 + r, gi)) =
-                            live ? sum_round_fast_h8<S::K>(t[r]) : make_uint4(0, 0, 0, 0);
-                } else {
-#pragma unroll
-                    for (int r = 0; r < 8; ++r) {
-                        uint4 t[S::K];
-                        gather_terms<S>(code, r, scb, cb, t);
-                        *reinterpret_cast<uint4 *>(A + sw128(rt_l * 8 + r, gi)) =
-                            live ? sum_round_fast_h8<S::K>(t) : make_uint4(0, 0, 0, 0);
+                        for (int r = 0; r < 8; ++r) {
+                            uint4 t[S::K];
+                            gather_terms<S>(code, r, scb, cb, t);
+                            *reinterpret_cast<uint4 *>(A + sw128(rt_l * 8 + r, gi)) =
+                                live ? sum_round_fast_h8<S::K>(t) : make_uint4(0, 0, 0, 0);
+                        }
                     }
                 }
-            }
-            if constexpr (kAsyncWeights) {
-                cp_async_commit();
-                const int j = s - lag;
-                if (j >= 0) {
-                    cp_async_wait<kWsLag>();
+                if constexpr (kAsyncWeights) {
+                    cp_async_commit();
+                    const int j = s - kLag;
+                    if (j >= 0) {
+                        cp_async_wait<kLag>();
+                        fence_proxy_async_smem();
+                        mbar_arrive(&full_a[j % kWsStages]);
+                    }
+                } else {
                     fence_proxy_async_smem();
-                    mbar_arrive(&full_a[j % kWsStages]);
+                    mbar_arrive(&full_a[s % kWsStages]);
                 }
-            } else {
-                fence_proxy_async_smem();
-                mbar_arrive(&full_a[s % kWsStages]);
             }
         }
         cp_async_wait<0>();
@@ -389,11 +488,19 @@ gemm_ws_kernel(const __grid_constant__ CUtensorMap xmap, Geom L, const uint8_t *
             const float sc = (row < L.out && scales) ? __half2float(__ushort_as_half(scales[row])) : 1.f;
             const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16);
 #pragma unroll 1
-            for (int c0 = 0; c0 < kWsBN; c0 += 16) {
+            for (int c0 = 0; c0 < BN; c0 += 16) {
                 float v[16];
                 tmem_ld16(tbase + c0, v);
                 const int gn = n0 + c0;
-                if (row < L.out && gn < T) {
+                if (sp.partials) {
+                    // one of several splits: fp32 partial sums, T % 8 == 0 here
+                    if (row < L.out && gn < T) {
+                        float4 *dst = reinterpret_cast<float4 *>(sp.partials + ((size_t)blockIdx.z * L.out + row) * T + gn);
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4)
+                            if (gn + 4 * q4 < T) dst[q4] = make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
+                    }
+                } else if (row < L.out && gn < T) {
                     uint16_t *dst = y + (size_t)row * T + gn;
                     if (gn + 16 <= T) {
                         const uint4 o0 = make_uint4(f2h2(sc * v[0], sc * v[1]), f2h2(sc * v[2], sc * v[3]),
@@ -422,7 +529,10 @@ gemm_ws_kernel(const __grid_constant__ CUtensorMap xmap, Geom L, const uint8_t *
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, kWsBN);
+    if (warp == 0) tmem_dealloc(tmem, BN);
+    // arrive even after a timeout so the counters stay consistent (the
+    // status word already tells the caller the output is incomplete)
+    if (sp.partials) gemm_split_finish(L, sp, m0, n0, BN, T, scales, y);
 }
 
 // ---- self-test of the bounded wait -----------------------------------------
@@ -445,7 +555,44 @@ __global__ void selftest_wait_kernel(void *ws, int spin_limit)
 namespace aqh {
 using namespace aqk;
 
-size_t gemm_workspace_bytes(const Geom &, int) { return kWsHeader; }
+// Launch plan of the TMA path (T % 8 == 0): token tile, split-K, workspace.
+struct GemmPlan {
+    bool tma;         // warp-specialised kernel (X by TMA)
+    int bn;           // tokens per CTA: 512 above 256 tokens, else 256
+    int mtiles, ntiles;
+    int ks;           // splits of the input features (blockIdx.z)
+    int per_split;    // 64-feature stages per split
+    size_t ws_bytes;  // status word + tile counters + fp32 partials
+};
+
+static GemmPlan plan_gemm(const Geom &g, int T)
+{
+    GemmPlan p{};
+    p.tma = (T % 8) == 0;
+    p.ws_bytes = kWsHeader;
+    if (!p.tma) return p;
+    p.mtiles = (g.out + kBM - 1) / kBM;
+    // 512-token tiles halve the decode work per MMA; when they would leave
+    // more than half the SMs without a tile (and so need a deep split of
+    // the input features, whose partial sums cost a pass through L2),
+    // 256-token tiles with fewer splits are faster (measured on Llama-2-7B
+    // shapes at 512 tokens)
+    p.bn = (T > 256 && (long)p.mtiles * ((T + 511) / 512) * 2 >= kNumSMs) ? 512 : 256;
+    p.ntiles = (T + p.bn - 1) / p.bn;
+    const int nst = (g.in + kBK - 1) / kBK;
+    const long tiles = (long)p.mtiles * p.ntiles;
+    // the decode is the bound: split the input features until about one CTA
+    // per SM works, keeping at least 8 stages per split
+    int ks = tiles < kNumSMs ? (int)(kNumSMs / tiles) : 1;
+    ks = std::max(1, std::min(ks, nst / 8));
+    p.per_split = (nst + ks - 1) / ks;
+    p.ks = (nst + p.per_split - 1) / p.per_split;
+    p.ws_bytes = kWsHeader + align16(sizeof(unsigned) * (size_t)tiles);
+    if (p.ks > 1) p.ws_bytes += (size_t)p.ks * g.out * T * sizeof(float);
+    return p;
+}
+
+size_t gemm_workspace_bytes(const Geom &g, int T) { return plan_gemm(g, T).ws_bytes; }
 
 template <class S>
 static constexpr int gemm_smem_bytes()
@@ -467,10 +614,11 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
     return fn;
 }
 
-template <class S>
+template <class S, int BN>
 static constexpr int gemm_ws_smem_bytes()
 {
-    return 1024 + kWsStagesOf<S> * (kTileABytes + kWsTileB) + S::kSmemBookBytes + (3 * kWsStagesOf<S> + 1) * 8 + 16;
+    return 1024 + kWsStagesOf<S, BN> * (kTileABytes + kBK * BN * 2) + S::kSmemBookBytes +
+           (3 * kWsStagesOf<S, BN> + 1) * 8 + 16;
 }
 
 cudaError_t launch_gemm(const Geom &g, const void *packed, const uint16_t *cb,
@@ -479,7 +627,8 @@ cudaError_t launch_gemm(const Geom &g, const void *packed, const uint16_t *cb,
 {
     const uint8_t *pk = reinterpret_cast<const uint8_t *>(packed);
     const uint4 *c = reinterpret_cast<const uint4 *>(cb);
-    PFN_cuTensorMapEncodeTiled_v12000 encode = (T % 8 == 0) ? tensor_map_encoder() : nullptr;
+    const GemmPlan p = plan_gemm(g, T);
+    PFN_cuTensorMapEncodeTiled_v12000 encode = p.tma ? tensor_map_encoder() : nullptr;
     if (encode) {
         // X [in][T] binary16: innermost dimension tokens, box 64 tokens x 64 features
         CUtensorMap map;
@@ -491,15 +640,25 @@ cudaError_t launch_gemm(const Geom &g, const void *packed, const uint16_t *cb,
                             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                             CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
-        const dim3 grid((g.out + kBM - 1) / kBM, (T + kWsBN - 1) / kWsBN);
-        return with_scheme(g, [&](auto sch) {
+        const dim3 grid(p.mtiles, p.ntiles, p.ks);
+        GemmSplit sp{nullptr, reinterpret_cast<unsigned *>(reinterpret_cast<char *>(ws) + kWsHeader)};
+        if (p.ks > 1)
+            sp.partials = reinterpret_cast<float *>(reinterpret_cast<char *>(ws) + kWsHeader +
+                                                    align16(sizeof(unsigned) * (size_t)p.mtiles * p.ntiles));
+        auto launch = [&](auto sch, auto bn) {
             using S = decltype(sch);
-            constexpr int smem = gemm_ws_smem_bytes<S>();
+            constexpr int BN = decltype(bn)::value;
+            constexpr int smem = gemm_ws_smem_bytes<S, BN>();
             static_assert(smem <= 227 * 1024, "shared memory of the warp-specialised GEMM");
-            cudaError_t e = cudaFuncSetAttribute(gemm_ws_kernel<S>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+            cudaError_t e = cudaFuncSetAttribute(gemm_ws_kernel<S, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 smem);
             if (e != cudaSuccess) return e;
-            gemm_ws_kernel<S><<<grid, kWsThreads, smem, s>>>(map, g, pk, c, scales, T, y, ws);
+            gemm_ws_kernel<S, BN><<<grid, kWsThreads, smem, s>>>(map, g, pk, c, scales, T, y, ws, sp, p.per_split);
             return cudaGetLastError();
+        };
+        return with_scheme(g, [&](auto sch) {
+            return p.bn == 512 ? launch(sch, std::integral_constant<int, 512>{})
+                               : launch(sch, std::integral_constant<int, 256>{});
         });
     }
     // T not a multiple of 8: rows of X are not 16-byte aligned for TMA; the

@@ -553,7 +553,6 @@ struct GemvPlan {
     size_t ws_bytes;
 };
 
-inline size_t align16(size_t v) { return (v + 15) / 16 * 16; }
 
 // Depends on the shape and batch only, so the workspace size can be
 // computed on a host without a GPU.

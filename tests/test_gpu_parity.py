@@ -178,7 +178,7 @@ def test_gemv_rejects_small_workspace_without_writing():
 
 @pytest.mark.parametrize("K,B", SCHEMES)
 @pytest.mark.parametrize("out,inp", [(128, 64), (256, 512), (129, 136), (1000, 1032), (8, 8)])
-@pytest.mark.parametrize("T", [1, 5, 8, 64, 136, 300])
+@pytest.mark.parametrize("T", [1, 5, 8, 64, 136, 300, 520, 1032])
 def test_gemm_matches_oracle(K, B, out, inp, T):
     layer = _layer(out, inp, K, B, out + inp * 5 + T)
     x = make_activations(inp, T, T)
@@ -291,3 +291,23 @@ def test_other_schemes_llama_shape_sampled(K, B):
     assert np.array_equal(got.view(np.uint16), want.view(np.uint16))
     del dl
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("K,B", [(1, 16), (2, 8)])
+@pytest.mark.parametrize("T", [256, 512, 2048])
+def test_gemm_split_k_deterministic_and_reusable(K, B, T):
+    """Layers small enough that the input features are split across CTAs:
+    the split partial sums are added in split order, so repeated calls give
+    identical bits, and the tile counters are back at zero after each call
+    (the workspace is reused)."""
+    layer = _layer(256, 4096, K, B, T + K)
+    dl = DevLayer(layer)
+    desc = dl.desc
+    ws = workspace(aq.aq_gemm_workspace_bytes(desc, T))
+    x = make_activations(4096, T, (T, 1))
+    y1 = run_gemm(dl, x, ws)
+    y2 = run_gemm(dl, x, ws)
+    assert np.array_equal(y1, y2)
+    rows = np.arange(0, 256, 17)
+    ref, bound = oracle.matmul(layer.codes, layer.codebooks, layer.scales, x, rows=rows, threads=8)
+    assert_close(y1[rows], ref, bound, f"split-K {K}x{B} T{T}")
