@@ -18,6 +18,9 @@ Quantization" (AQLM wiki entry, "Niveau intermédiaire"; devtrends.ru summary,
 * ``backward``: gradients of sum(gy * y) with respect to the row scales and
   the codebook entries (the decode's rounding taken as the identity), with
   magnitude bounds;
+* ``encode`` / ``objective``: one-pass beam search of the codes for fixed
+  codebooks under e^T H e (the quantisation objective of the wiki entry),
+  and that objective for given codes;
 * ``pack`` / ``unpack``: the library's documented packed code layout;
 * ``bits_per_weight`` and ``layer_bytes``: the bit-rate closed form and the
   storage it implies.
@@ -82,6 +85,10 @@ def _load():
             lib.aqo_backward.argtypes = [_c_i64, _c_i64, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp,
                                          _c_i64, _vp, _vp, _vp, _vp]
             lib.aqo_backward.restype = _c_int
+            lib.aqo_encode.argtypes = [_c_i64, _c_i64, _c_int, _c_int, _vp, _vp, _vp, _vp, _c_int, _vp, _vp]
+            lib.aqo_encode.restype = _c_int
+            lib.aqo_objective.argtypes = [_c_i64, _c_i64, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp]
+            lib.aqo_objective.restype = _c_int
             lib.aqo_packed_bytes.argtypes = [_c_i64, _c_i64, _c_int, _c_int]
             lib.aqo_packed_bytes.restype = _c_i64
             lib.aqo_pack.argtypes = [_c_i64, _c_i64, _c_int, _c_int, _vp, _vp]
@@ -207,6 +214,44 @@ def backward(codes, codebooks, scales, x, gy):
     if rc:
         raise RuntimeError(f"aqo_backward failed ({rc})")
     return gs, gsb, gc, gcb
+
+
+def _enc_args(w, h, codebooks):
+    wb = _bits(w)
+    out, inp = wb.shape
+    hf = np.ascontiguousarray(h, dtype=np.float32)
+    if hf.shape != (inp, inp):
+        raise ValueError("h must be [in][in]")
+    cb = _bits(codebooks)
+    K, ncw, _ = cb.shape
+    B = int(ncw).bit_length() - 1
+    return wb, hf, cb, out, inp, K, B
+
+
+def encode(w, h, codebooks, codes_init, beam: int):
+    """Beam search of the codes of every row of ``w`` ([out][in] binary16)
+    for fixed codebooks under the objective e^T H e, e = w - sum_k C_k[i_k]
+    (``h`` [in][in] float32).  One pass over the slots (group, codebook)
+    from ``codes_init``; returns ``(codes [out][in/8][K], objective [out])``."""
+    wb, hf, cb, out, inp, K, B = _enc_args(w, h, codebooks)
+    ci = np.ascontiguousarray(np.asarray(codes_init).reshape(out, inp // 8, K), dtype=np.uint32)
+    co = np.empty_like(ci)
+    obj = np.empty(out, dtype=np.float64)
+    rc = _load().aqo_encode(out, inp, K, B, _ptr(wb), _ptr(hf), _ptr(cb), _ptr(ci), int(beam), _ptr(co), _ptr(obj))
+    if rc:
+        raise RuntimeError(f"aqo_encode failed ({rc})")
+    return co.astype(np.uint8 if B <= 8 else np.uint16), obj
+
+
+def objective(w, h, codebooks, codes):
+    """e^T H e per row for the given codes (exact codeword sums, double)."""
+    wb, hf, cb, out, inp, K, B = _enc_args(w, h, codebooks)
+    ci = np.ascontiguousarray(np.asarray(codes).reshape(out, inp // 8, K), dtype=np.uint32)
+    obj = np.empty(out, dtype=np.float64)
+    rc = _load().aqo_objective(out, inp, K, B, _ptr(wb), _ptr(hf), _ptr(cb), _ptr(ci), _ptr(obj))
+    if rc:
+        raise RuntimeError(f"aqo_objective failed ({rc})")
+    return obj
 
 
 def packed_bytes(out: int, inp: int, K: int, B: int) -> int:

@@ -306,6 +306,144 @@ int aqo_backward(int64_t out, int64_t in, int K, int B, const void *codes,
 }
 
 /* ------------------------------------------------------------------------ */
+/* Encoder: beam search of the codes for fixed codebooks.                   */
+/*                                                                          */
+/* The AQLM wiki entry ("Niveau tech avancé") states the objective          */
+/* sum over layers of || W - sum_k C_k[i_k] ||^2_H with H = 2 X^T X from     */
+/* calibration activations, and that the codes are assigned by beam search  */
+/* rather than greedily.  || (W - What) X^T ||^2 is a sum over output rows   */
+/* of e_o^T (X^T X) e_o, so every row is its own problem.  Reading taken:    */
+/*   - the reconstruction is the exact sum of the codewords (no rounding);   */
+/*   - one pass over the slots (group g ascending, codebook k ascending     */
+/*     within a group), starting from the given codes as the only beam;     */
+/*   - at each slot every beam proposes each of the 2^B codes for that slot */
+/*     (the other slots as in the beam); the `beam` proposals with the      */
+/*     smallest objective survive, ordered by (objective, parent beam,      */
+/*     code) so that ties resolve the same way every time; in one pass the   */
+/*     beams always differ in an already visited slot, so proposals never   */
+/*     repeat;                                                              */
+/*   - the result is the first surviving beam.                              */
+/* Every proposal is scored by the quadratic form written out, in double.   */
+/* ------------------------------------------------------------------------ */
+
+static double quad_form(const double *e, const double *h, int64_t in)
+{
+    double f = 0.0;
+    for (int64_t a = 0; a < in; ++a) {
+        double t = 0.0;
+        for (int64_t b = 0; b < in; ++b) t += h[a * in + b] * e[b];
+        f += e[a] * t;
+    }
+    return f;
+}
+
+/* Row error w - sum_k C_k[codes[g][k]] for one row's codes [G][K]. */
+static void row_error(int64_t in, int K, int B, const uint32_t *codes, const double *w,
+                      const uint16_t *codebooks, double *e)
+{
+    int64_t G = in / AQO_GROUP;
+    for (int64_t g = 0; g < G; ++g)
+        for (int j = 0; j < AQO_GROUP; ++j) {
+            double sum = 0.0;
+            for (int k = 0; k < K; ++k)
+                sum += aqo_half_to_double(codebooks[(((int64_t)k << B) + codes[g * K + k]) * AQO_GROUP + j]);
+            e[g * AQO_GROUP + j] = w[g * AQO_GROUP + j] - sum;
+        }
+}
+
+typedef struct { double f; int parent; uint32_t code; } aqo_prop;
+
+static int prop_less(const aqo_prop *a, const aqo_prop *b)
+{
+    if (a->f != b->f) return a->f < b->f;
+    if (a->parent != b->parent) return a->parent < b->parent;
+    return a->code < b->code;
+}
+
+/* codes_in / codes_out: [out][in/8][K] as uint32 (any B); w binary16
+ * [out][in]; h fp32 [in][in]; objective_out[out] (optional) the final
+ * objective of each row. */
+int aqo_encode(int64_t out, int64_t in, int K, int B, const uint16_t *w, const float *h,
+               const uint16_t *codebooks, const uint32_t *codes_in, int beam,
+               uint32_t *codes_out, double *objective_out)
+{
+    if (check_scheme(out, in, K, B) || beam < 1) return -1;
+    int64_t G = in / AQO_GROUP, S = G * K, ncw = (int64_t)1 << B;
+    double *hd = (double *)malloc(sizeof(double) * (size_t)(in * in > 0 ? in * in : 1));
+    double *wd = (double *)malloc(sizeof(double) * (size_t)(in > 0 ? in : 1));
+    double *e = (double *)malloc(sizeof(double) * (size_t)(in > 0 ? in : 1));
+    uint32_t *cur = (uint32_t *)malloc(sizeof(uint32_t) * (size_t)(beam * S > 0 ? beam * S : 1));
+    uint32_t *nxt = (uint32_t *)malloc(sizeof(uint32_t) * (size_t)(beam * S > 0 ? beam * S : 1));
+    double *fcur = (double *)malloc(sizeof(double) * (size_t)beam);
+    aqo_prop *props = (aqo_prop *)malloc(sizeof(aqo_prop) * (size_t)(beam * ncw));
+    uint32_t *trial = (uint32_t *)malloc(sizeof(uint32_t) * (size_t)(S > 0 ? S : 1));
+    if (!hd || !wd || !e || !cur || !nxt || !fcur || !props || !trial) {
+        free(hd); free(wd); free(e); free(cur); free(nxt); free(fcur); free(props); free(trial);
+        return -2;
+    }
+    for (int64_t t = 0; t < in * in; ++t) hd[t] = (double)h[t];
+    for (int64_t o = 0; o < out; ++o) {
+        for (int64_t i = 0; i < in; ++i) wd[i] = aqo_half_to_double(w[o * in + i]);
+        int nb = 1;
+        for (int64_t t = 0; t < S; ++t) cur[t] = codes_in[o * S + t];
+        row_error(in, K, B, cur, wd, codebooks, e);
+        fcur[0] = quad_form(e, hd, in);
+        for (int64_t sl = 0; sl < S; ++sl) {
+            int np = 0;
+            for (int b = 0; b < nb; ++b)
+                for (int64_t c = 0; c < ncw; ++c) {
+                    for (int64_t t = 0; t < S; ++t) trial[t] = cur[b * S + t];
+                    trial[sl] = (uint32_t)c;
+                    row_error(in, K, B, trial, wd, codebooks, e);
+                    props[np].f = quad_form(e, hd, in);
+                    props[np].parent = b;
+                    props[np].code = (uint32_t)c;
+                    ++np;
+                }
+            /* keep the `beam` smallest: selection by repeated minimum */
+            int keep = np < beam ? np : beam;
+            for (int r = 0; r < keep; ++r) {
+                int best = r;
+                for (int q = r + 1; q < np; ++q)
+                    if (prop_less(&props[q], &props[best])) best = q;
+                aqo_prop tmp = props[r]; props[r] = props[best]; props[best] = tmp;
+            }
+            for (int r = 0; r < keep; ++r) {
+                for (int64_t t = 0; t < S; ++t) nxt[r * S + t] = cur[props[r].parent * S + t];
+                nxt[r * S + sl] = props[r].code;
+                fcur[r] = props[r].f;
+            }
+            nb = keep;
+            uint32_t *sw = cur; cur = nxt; nxt = sw;
+        }
+        for (int64_t t = 0; t < S; ++t) codes_out[o * S + t] = cur[t];
+        if (objective_out) objective_out[o] = fcur[0];
+    }
+    free(hd); free(wd); free(e); free(cur); free(nxt); free(fcur); free(props); free(trial);
+    return 0;
+}
+
+/* Objective of given codes per row (same definition), for checks. */
+int aqo_objective(int64_t out, int64_t in, int K, int B, const uint16_t *w, const float *h,
+                  const uint16_t *codebooks, const uint32_t *codes, double *objective)
+{
+    if (check_scheme(out, in, K, B)) return -1;
+    int64_t S = (in / AQO_GROUP) * K;
+    double *hd = (double *)malloc(sizeof(double) * (size_t)(in * in > 0 ? in * in : 1));
+    double *wd = (double *)malloc(sizeof(double) * (size_t)(in > 0 ? in : 1));
+    double *e = (double *)malloc(sizeof(double) * (size_t)(in > 0 ? in : 1));
+    if (!hd || !wd || !e) { free(hd); free(wd); free(e); return -2; }
+    for (int64_t t = 0; t < in * in; ++t) hd[t] = (double)h[t];
+    for (int64_t o = 0; o < out; ++o) {
+        for (int64_t i = 0; i < in; ++i) wd[i] = aqo_half_to_double(w[o * in + i]);
+        row_error(in, K, B, codes + o * S, wd, codebooks, e);
+        objective[o] = quad_form(e, hd, in);
+    }
+    free(hd); free(wd); free(e);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
 /* Packed code layout (the library's documented interface).                 */
 /*                                                                          */
 /* Each group (o, g) has one word of W = K*B/8 bytes holding its K codes,   */

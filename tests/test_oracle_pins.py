@@ -470,3 +470,80 @@ def test_backward_bounds_dominate():
     gs, gsb, gc, gcb = oracle.backward(layer.codes, layer.codebooks, layer.scales, x, gy)
     assert np.all(np.abs(gs) <= gsb) and np.all(np.abs(gc) <= gcb)
     assert np.all(gcb >= 0) and gsb.min() > 0
+
+
+# ---------------------------------------------------------------------------
+# Encoder: beam search of the codes for fixed codebooks
+# ---------------------------------------------------------------------------
+
+def _int_problem(out, inp, K, B, seed):
+    """Small-integer weights, codebooks and a positive definite H: every
+    objective is an exact integer in fp32 and fp64."""
+    rng = np.random.default_rng(seed)
+    w = rng.integers(-4, 5, size=(out, inp)).astype(np.float16)
+    a = rng.integers(-1, 2, size=(inp, inp)).astype(np.float32)
+    h = (a.T @ a + np.eye(inp, dtype=np.float32)).astype(np.float32)
+    cb = rng.integers(-2, 3, size=(K, 1 << B, 8)).astype(np.float16)
+    c0 = rng.integers(0, 1 << B, size=(out, inp // 8, K)).astype(np.uint8 if B <= 8 else np.uint16)
+    return w, h, cb, c0
+
+
+def _np_objective(w, h, cb, codes):
+    out, inp = w.shape
+    K = cb.shape[0]
+    res = []
+    for o in range(out):
+        what = np.concatenate([sum(cb[k, codes[o, g, k]].astype(np.float64) for k in range(K))
+                               for g in range(inp // 8)])
+        e = w[o].astype(np.float64) - what
+        res.append(float(e @ h.astype(np.float64) @ e))
+    return np.array(res)
+
+
+def test_encode_one_group_full_beam_is_exhaustive():
+    """One group, beam = 2^B: the first slot keeps every code, the second
+    tries every pair, so the result is the brute-force optimum (any H)."""
+    w, h, cb, c0 = _int_problem(5, 8, 2, 3, 1)
+    codes, obj = oracle.encode(w, h, cb, c0, beam=8)
+    for o in range(5):
+        best = min(_np_objective(w[o:o + 1], h, cb, np.array([[[a, b]]], dtype=np.uint8))[0]
+                   for a in range(8) for b in range(8))
+        assert obj[o] == best
+
+
+def test_encode_identity_h_single_codebook_is_nearest_codeword():
+    w, _, cb, c0 = _int_problem(4, 32, 1, 4, 2)
+    h = np.eye(32, dtype=np.float32)
+    codes, _ = oracle.encode(w, h, cb, c0, beam=1)
+    for o in range(4):
+        for g in range(4):
+            d = ((cb[0].astype(np.float64) - w[o, 8 * g:8 * g + 8].astype(np.float64)) ** 2).sum(axis=1)
+            assert d[codes[o, g, 0]] == d.min()
+            assert codes[o, g, 0] == int(np.flatnonzero(d == d.min())[0])  # ties: smallest code
+
+
+def test_encode_beam_one_is_greedy_coordinate_pass():
+    w, h, cb, c0 = _int_problem(3, 24, 2, 2, 3)
+    codes, obj = oracle.encode(w, h, cb, c0, beam=1)
+    for o in range(3):
+        cur = c0[o:o + 1].copy()
+        for g in range(3):
+            for k in range(2):
+                scores = []
+                for c in range(4):
+                    t = cur.copy()
+                    t[0, g, k] = c
+                    scores.append(_np_objective(w[o:o + 1], h, cb, t)[0])
+                cur[0, g, k] = int(np.argmin(scores))  # first minimum: smallest code
+        assert np.array_equal(codes[o], cur[0])
+        assert obj[o] == _np_objective(w[o:o + 1], h, cb, cur)[0]
+
+
+@pytest.mark.parametrize("K,B,beam", [(1, 4, 1), (2, 3, 4), (2, 4, 8), (8, 2, 3)])
+def test_encode_never_worse_than_start_and_objective_consistent(K, B, beam):
+    w, h, cb, c0 = _int_problem(6, 32, K, B, K * 10 + B + beam)
+    codes, obj = oracle.encode(w, h, cb, c0, beam=beam)
+    start = _np_objective(w, h, cb, c0)
+    assert np.all(obj <= start)
+    assert np.array_equal(obj, _np_objective(w, h, cb, codes))
+    assert np.array_equal(oracle.objective(w, h, cb, codes), obj)
