@@ -18,9 +18,9 @@ Quantization" (AQLM wiki entry, "Niveau intermédiaire"; devtrends.ru summary,
 * ``backward``: gradients of sum(gy * y) with respect to the row scales and
   the codebook entries (the decode's rounding taken as the identity), with
   magnitude bounds;
-* ``encode`` / ``objective``: one-pass beam search of the codes for fixed
+* ``encode`` / ``objective``: beam search of each group's codes for fixed
   codebooks under e^T H e (the quantisation objective of the wiki entry),
-  and that objective for given codes;
+  group after group, and that objective for given codes;
 * ``pack`` / ``unpack``: the library's documented packed code layout;
 * ``bits_per_weight`` and ``layer_bytes``: the bit-rate closed form and the
   storage it implies.
@@ -231,8 +231,9 @@ def _enc_args(w, h, codebooks):
 def encode(w, h, codebooks, codes_init, beam: int):
     """Beam search of the codes of every row of ``w`` ([out][in] binary16)
     for fixed codebooks under the objective e^T H e, e = w - sum_k C_k[i_k]
-    (``h`` [in][in] float32).  One pass over the slots (group, codebook)
-    from ``codes_init``; returns ``(codes [out][in/8][K], objective [out])``."""
+    (``h`` [in][in] float32): group by group from ``codes_init``, a beam over
+    the group's K codes (codebook by codebook), the best beam kept before the
+    next group.  Returns ``(codes [out][in/8][K], objective [out])``."""
     wb, hf, cb, out, inp, K, B = _enc_args(w, h, codebooks)
     ci = np.ascontiguousarray(np.asarray(codes_init).reshape(out, inp // 8, K), dtype=np.uint32)
     co = np.empty_like(ci)

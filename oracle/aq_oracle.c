@@ -314,15 +314,16 @@ int aqo_backward(int64_t out, int64_t in, int K, int B, const void *codes,
 /* rather than greedily.  || (W - What) X^T ||^2 is a sum over output rows   */
 /* of e_o^T (X^T X) e_o, so every row is its own problem.  Reading taken:    */
 /*   - the reconstruction is the exact sum of the codewords (no rounding);   */
-/*   - one pass over the slots (group g ascending, codebook k ascending     */
-/*     within a group), starting from the given codes as the only beam;     */
-/*   - at each slot every beam proposes each of the 2^B codes for that slot */
-/*     (the other slots as in the beam); the `beam` proposals with the      */
+/*   - the beam search runs over the K codes of one group (the "index       */
+/*     combination" of that group), the other groups fixed: groups in       */
+/*     ascending order, starting from the given codes; for group g the      */
+/*     codebooks are visited k = 0..K-1; at each, every beam proposes each   */
+/*     of the 2^B codes for slot (g, k); the `beam` proposals with the      */
 /*     smallest objective survive, ordered by (objective, parent beam,      */
-/*     code) so that ties resolve the same way every time; in one pass the   */
-/*     beams always differ in an already visited slot, so proposals never   */
-/*     repeat;                                                              */
-/*   - the result is the first surviving beam.                              */
+/*     code) so that ties resolve the same way every time (beams differ in  */
+/*     an already visited code of the group, so proposals never repeat);    */
+/*   - after the group's last codebook the first surviving beam is kept     */
+/*     and the next group starts from it as the only beam.                  */
 /* Every proposal is scored by the quadratic form written out, in double.   */
 /* ------------------------------------------------------------------------ */
 
@@ -389,6 +390,7 @@ int aqo_encode(int64_t out, int64_t in, int K, int B, const uint16_t *w, const f
         row_error(in, K, B, cur, wd, codebooks, e);
         fcur[0] = quad_form(e, hd, in);
         for (int64_t sl = 0; sl < S; ++sl) {
+            if (sl % K == 0) nb = 1;  /* a new group starts from the best beam */
             int np = 0;
             for (int b = 0; b < nb; ++b)
                 for (int64_t c = 0; c < ncw; ++c) {

@@ -547,3 +547,24 @@ def test_encode_never_worse_than_start_and_objective_consistent(K, B, beam):
     assert np.all(obj <= start)
     assert np.array_equal(obj, _np_objective(w, h, cb, codes))
     assert np.array_equal(oracle.objective(w, h, cb, codes), obj)
+
+
+def test_encode_full_beam_is_sequential_exhaustive_per_group():
+    """beam = 2^B: each group's code pair is the brute-force optimum given
+    the groups before it (already chosen) and after it (still initial)."""
+    w, h, cb, c0 = _int_problem(3, 24, 2, 2, 7)
+    codes, obj = oracle.encode(w, h, cb, c0, beam=4)
+    for o in range(3):
+        cur = c0[o:o + 1].copy()
+        for g in range(3):
+            best = None
+            for a in range(4):
+                for b in range(4):
+                    t = cur.copy()
+                    t[0, g] = (a, b)
+                    f = _np_objective(w[o:o + 1], h, cb, t)[0]
+                    if best is None or f < best[0]:
+                        best = (f, a, b)
+            cur[0, g] = best[1:]
+        assert np.array_equal(codes[o], cur[0]), o
+        assert obj[o] == _np_objective(w[o:o + 1], h, cb, cur)[0]
