@@ -21,7 +21,7 @@ __all__ = [
     "aq_packed_codes_bytes", "aq_gemv_workspace_bytes", "aq_gemm_workspace_bytes",
     "aq_workspace_status", "aq_selftest_bounded_wait", "aq_pack_codes", "aq_unpack_codes",
     "aq_dequant", "aq_gemv", "aq_gemv_noalloc", "aq_gemm", "aq_param_grad_workspace_bytes",
-    "aq_param_grad", "EXPORTED_SYMBOLS",
+    "aq_param_grad", "aq_encode_workspace_bytes", "aq_encode", "EXPORTED_SYMBOLS",
     "GEMV_NOALLOC_SCRATCH_BYTES",
 ]
 
@@ -38,7 +38,7 @@ EXPORTED_SYMBOLS = (
     "aq_status_string", "aq_version", "aq_packed_codes_bytes", "aq_gemv_workspace_bytes",
     "aq_gemm_workspace_bytes", "aq_workspace_status", "aq_selftest_bounded_wait",
     "aq_pack_codes", "aq_unpack_codes", "aq_dequant", "aq_gemv", "aq_gemv_noalloc", "aq_gemm",
-    "aq_param_grad_workspace_bytes", "aq_param_grad",
+    "aq_param_grad_workspace_bytes", "aq_param_grad", "aq_encode_workspace_bytes", "aq_encode",
 )
 
 # AQ_GEMV_NOALLOC_SCRATCH_BYTES of include/aq.h: the fixed scratch behind
@@ -90,6 +90,8 @@ def _load() -> ctypes.CDLL:
         "aq_gemv_noalloc": ([dp, vp, vp, vp, vp, i32, vp, vp], i32),
         "aq_param_grad_workspace_bytes": ([dp, i32], sz),
         "aq_param_grad": ([dp, vp, vp, vp, vp, vp, i32, vp, vp, vp, sz, vp], i32),
+        "aq_encode_workspace_bytes": ([dp], sz),
+        "aq_encode": ([dp, vp, vp, vp, vp, i32, vp, vp, sz, vp], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -207,3 +209,17 @@ def aq_param_grad(desc: LayerDesc, packed, codebooks, scales, x, gy, T: int, gra
     _check("aq_param_grad", lib.aq_param_grad(ctypes.byref(desc), _ptr(packed), _ptr(codebooks), _ptr(scales),
                                               _ptr(x), _ptr(gy), T, _ptr(grad_scales), _ptr(grad_codebooks),
                                               _ptr(workspace), workspace_bytes, _stream(stream)))
+
+
+def aq_encode_workspace_bytes(desc: LayerDesc) -> int:
+    return lib.aq_encode_workspace_bytes(ctypes.byref(desc))
+
+
+def aq_encode(desc: LayerDesc, w, h, codebooks, codes_in, beam: int, codes_out, workspace,
+              workspace_bytes: int | None = None, stream=None) -> None:
+    """Beam search of the codes (8-bit codebooks) minimising e^T H e per row;
+    w [out][in] binary16, h [in][in] fp32, codes [out][in/8][K] uint8."""
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    _check("aq_encode", lib.aq_encode(ctypes.byref(desc), _ptr(w), _ptr(h), _ptr(codebooks), _ptr(codes_in), beam,
+                                      _ptr(codes_out), _ptr(workspace), workspace_bytes, _stream(stream)))

@@ -185,6 +185,30 @@ aq_status aq_gemm(const aq_layer_desc *desc, const void *packed, const uint16_t 
                                       reinterpret_cast<cudaStream_t>(stream)));
 }
 
+size_t aq_encode_workspace_bytes(const aq_layer_desc *desc)
+{
+    if (check_desc(desc) != AQ_OK || desc->nbits != 8 || desc->in_features > 16384) return 0;
+    return aqh::encode_workspace_bytes(aqk::make_geom(*desc));
+}
+
+aq_status aq_encode(const aq_layer_desc *desc, const uint16_t *w, const float *h, const uint16_t *codebooks,
+                    const void *codes_in, int beam, void *codes_out, void *workspace, size_t workspace_bytes,
+                    aq_stream_t stream)
+{
+    aq_status st = check_desc(desc);
+    if (st != AQ_OK) return st;
+    if (desc->nbits != 8) return AQ_ERR_UNSUPPORTED;
+    if (desc->in_features > 16384 || beam < 1 || beam > 16) return AQ_ERR_INVALID_ARG;
+    if (!w || !h || !codebooks || !codes_in || !codes_out || codes_in == codes_out) return AQ_ERR_INVALID_ARG;
+    if (!aligned16(w) || !aligned16(h) || !aligned16(codebooks)) return AQ_ERR_MISALIGNED;
+    const Geom g = aqk::make_geom(*desc);
+    const size_t need = aqh::encode_workspace_bytes(g);
+    if (!workspace || workspace_bytes < need) return AQ_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return AQ_ERR_MISALIGNED;
+    return from_cuda(aqh::launch_encode(g, w, h, codebooks, codes_in, codes_out, beam, workspace,
+                                        reinterpret_cast<cudaStream_t>(stream)));
+}
+
 size_t aq_param_grad_workspace_bytes(const aq_layer_desc *desc, int T)
 {
     if (check_desc(desc) != AQ_OK || T < 8 || T > (1 << 22) || T % 8) return 0;

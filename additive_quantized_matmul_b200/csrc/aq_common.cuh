@@ -246,5 +246,8 @@ size_t param_grad_workspace_bytes(const aqk::Geom &g, int T);
 cudaError_t launch_param_grad(const aqk::Geom &g, const void *packed, const uint16_t *cb, const uint16_t *scales,
                               const uint16_t *x, const uint16_t *gy, int T, float *grad_s, float *grad_cb,
                               void *ws, cudaStream_t s);
+size_t encode_workspace_bytes(const aqk::Geom &g);
+cudaError_t launch_encode(const aqk::Geom &g, const uint16_t *w, const float *h, const uint16_t *cb,
+                          const void *codes_in, void *codes_out, int beam, void *ws, cudaStream_t s);
 cudaError_t launch_selftest_wait(void *ws, int spin_limit, cudaStream_t s);
 }  // namespace aqh

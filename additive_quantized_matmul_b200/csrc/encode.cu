@@ -1,0 +1,271 @@
+// Encoder: beam search of the codes of a layer for fixed 8-bit codebooks
+// (1x8, 2x8, 8x8) under the quantisation objective of "Extreme Compression
+// of Large Language Models via Additive Quantization" (AQLM wiki entry,
+// "Niveau tech avancé"): || W - sum_k C_k[i_k] ||^2_H with H = 2 X^T X, the
+// codes assigned by beam search.  The objective is a sum over output rows of
+// e^T H e (e = w - reconstruction), so rows are independent: one CTA per row.
+//
+// Per row, groups in order, the others fixed: for group g the beam runs over
+// the group's K codes, codebook by codebook; every beam proposes each of the
+// 256 codes for slot (g, k); the `beam` proposals with the smallest
+// objective survive, ordered by (objective, parent beam, code); the best
+// beam is committed before group g + 1.  With the group's reconstruction
+// changed by D (8 values), the objective changes by
+//     delta = -2 D^T v + D^T H_gg D,   v = (H e)_g, H_gg the diagonal block,
+// and for a proposal D = a_b + C_k[c] (a_b = the beam's change so far minus
+// the slot's starting codeword) this is
+//     delta = const_b + q_gk(c) + 2 C_k[c] . w_b,
+//     const_b = a_b^T H_gg a_b - 2 a_b^T v,  w_b = H_gg a_b - v,
+//     q_gk(c) = C_k[c]^T H_gg C_k[c]           (a per-layer table).
+// The group's objective before the change is common to all its proposals,
+// so ranking by delta ranks by the objective.  fp32 throughout (exact for
+// integer-valued inputs of moderate size, which the tests use).
+#include <cuda_fp16.h>
+
+#include <type_traits>
+
+#include "scheme.cuh"
+
+namespace aqk {
+
+constexpr int kEncThreads = 256;   // one per code of an 8-bit codebook
+constexpr int kEncMaxBeam = 16;
+
+// q[(g * K + k) * 256 + c] = C_k[c]^T H_gg C_k[c]
+template <int K>
+__global__ void __launch_bounds__(256) encode_q_kernel(int in, const float *__restrict__ h,
+                                                       const uint4 *__restrict__ cb, float *__restrict__ q)
+{
+    __shared__ float hgg[64];
+    const int g = blockIdx.x, c = threadIdx.x;
+    if (c < 64) hgg[c] = h[(size_t)(8 * g + c / 8) * in + 8 * g + c % 8];
+    __syncthreads();
+#pragma unroll 1
+    for (int k = 0; k < K; ++k) {
+        const uint4 w = cb[k * 256 + c];
+        const float2 a = h2f2(w.x), b = h2f2(w.y), d = h2f2(w.z), e = h2f2(w.w);
+        const float x[8] = {a.x, a.y, b.x, b.y, d.x, d.y, e.x, e.y};
+        float acc = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            float t = 0.f;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) t = fmaf(hgg[i * 8 + j], x[j], t);
+            acc = fmaf(x[i], t, acc);
+        }
+        q[((size_t)g * K + k) * 256 + c] = acc;
+    }
+}
+
+__device__ __forceinline__ uint64_t enc_key(float s, int beam, int code)
+{
+    s = s + 0.f;  // -0 -> +0: equal objectives compare equal
+    uint32_t u = __float_as_uint(s);
+    u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);  // order-preserving
+    return ((uint64_t)u << 32) | ((uint32_t)beam << 8) | (uint32_t)code;
+}
+
+__device__ __forceinline__ float key_score(uint64_t key)
+{
+    uint32_t u = (uint32_t)(key >> 32);
+    u = (u & 0x80000000u) ? (u & 0x7fffffffu) : ~u;
+    return __uint_as_float(u);
+}
+
+__device__ __forceinline__ uint64_t warp_min_u64(uint64_t v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const uint64_t t = __shfl_xor_sync(0xffffffffu, v, o);
+        v = t < v ? t : v;
+    }
+    return v;
+}
+
+__device__ __forceinline__ void load_f8(const uint4 w, float x[8])
+{
+    const float2 a = h2f2(w.x), b = h2f2(w.y), d = h2f2(w.z), e = h2f2(w.w);
+    x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y; x[4] = d.x; x[5] = d.y; x[6] = e.x; x[7] = e.y;
+}
+
+// Sorting network: the 16 keys of a thread in ascending order.
+__device__ __forceinline__ void sort16(uint64_t (&k)[kEncMaxBeam])
+{
+#pragma unroll
+    for (int pass = 0; pass < kEncMaxBeam; ++pass)
+#pragma unroll
+        for (int i = pass & 1; i + 1 < kEncMaxBeam; i += 2) {
+            const uint64_t a = k[i], b = k[i + 1];
+            k[i] = a < b ? a : b;
+            k[i + 1] = a < b ? b : a;
+        }
+}
+
+__device__ __forceinline__ void pop16(uint64_t (&k)[kEncMaxBeam])
+{
+#pragma unroll
+    for (int i = 0; i + 1 < kEncMaxBeam; ++i) k[i] = k[i + 1];
+    k[kEncMaxBeam - 1] = ~0ull;
+}
+
+template <int K>
+__global__ void __launch_bounds__(kEncThreads) encode_kernel(Geom L, const uint16_t *__restrict__ w,
+                                                             const float *__restrict__ h, const uint4 *__restrict__ cb,
+                                                             const float *__restrict__ qtab,
+                                                             const uint8_t *__restrict__ codes_in,
+                                                             uint8_t *__restrict__ codes_out, int beam)
+{
+    extern __shared__ float e[];                   // [in] residual w - reconstruction of this row
+    __shared__ uint4 scb[K * 256];                 // the codebooks
+    __shared__ float hgg[64], v[8];                // H_gg and (H e)_g of the current group
+    __shared__ float bD[2][kEncMaxBeam][8];        // each beam's change of the group's reconstruction
+    __shared__ uint8_t bcode[2][kEncMaxBeam][K];   // each beam's codes for the group
+    __shared__ float bconst[kEncMaxBeam], bw[kEncMaxBeam][8];
+    __shared__ uint64_t wtop[kEncThreads / 32][kEncMaxBeam];
+    __shared__ uint64_t sel[kEncMaxBeam];
+    const int o = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int in = L.in, G = L.G;
+    const uint8_t *ci = codes_in + (size_t)o * G * K;
+    const __half *cbh = reinterpret_cast<const __half *>(scb);
+
+    for (int i = tid; i < K * 256; i += kEncThreads) scb[i] = cb[i];
+    __syncthreads();
+    for (int i = tid; i < in; i += kEncThreads) {
+        const int g = i >> 3, j = i & 7;
+        float r = 0.f;
+#pragma unroll
+        for (int k = 0; k < K; ++k) r += __half2float(cbh[(k * 256 + ci[g * K + k]) * 8 + j]);
+        e[i] = __half2float(__ushort_as_half(w[(size_t)o * in + i])) - r;
+    }
+    int cur = 0;
+#pragma unroll 1
+    for (int g = 0; g < G; ++g) {
+        __syncthreads();  // e holds every committed group
+        {
+            // v_j = sum_t H[8g + j][t] e[t], one warp per j (H rows coalesced)
+            const float *hr = h + (size_t)(8 * g + warp) * in;
+            float acc = 0.f;
+            for (int t = lane; t < in; t += 32) acc = fmaf(hr[t], e[t], acc);
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+            if (lane == 0) v[warp] = acc;
+        }
+        if (tid < 64) hgg[tid] = h[(size_t)(8 * g + tid / 8) * in + 8 * g + tid % 8];
+        if (tid < 8) bD[cur][0][tid] = 0.f;
+        if (tid < K) bcode[cur][0][tid] = ci[g * K + tid];
+        int nb = 1;
+        __syncthreads();
+#pragma unroll 1
+        for (int k = 0; k < K; ++k) {
+            const uint32_t c0 = ci[g * K + k];  // the slot's starting code, common to all beams
+            if (tid < nb) {
+                float a[8], c0v[8], ha[8];
+                load_f8(scb[k * 256 + c0], c0v);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) a[j] = bD[cur][tid][j] - c0v[j];
+                float cst = 0.f;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    float t = 0.f;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) t = fmaf(hgg[i * 8 + j], a[j], t);
+                    ha[i] = t;
+                    cst = fmaf(a[i], t - 2.f * v[i], cst);
+                    bw[tid][i] = t - v[i];
+                }
+                bconst[tid] = cst;
+            }
+            __syncthreads();
+            // scores of code c = tid for every beam
+            uint64_t kk[kEncMaxBeam];
+            {
+                float x[8];
+                load_f8(scb[k * 256 + tid], x);
+                const float qc = qtab[((size_t)g * K + k) * 256 + tid];
+#pragma unroll
+                for (int b = 0; b < kEncMaxBeam; ++b) {
+                    kk[b] = ~0ull;
+                    if (b < nb) {
+                        float d = 0.f;
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) d = fmaf(x[i], bw[b][i], d);
+                        kk[b] = enc_key(bconst[b] + qc + 2.f * d, b, tid);
+                    }
+                }
+            }
+            sort16(kk);
+            // the warp's `beam` smallest keys (keys are unique)
+            for (int r = 0; r < beam; ++r) {
+                const uint64_t m = warp_min_u64(kk[0]);
+                if (kk[0] == m) pop16(kk);
+                if (lane == 0) wtop[warp][r] = m;
+            }
+            __syncthreads();
+            if (warp == 0) {
+                uint64_t hl[kEncMaxBeam];
+#pragma unroll
+                for (int i = 0; i < kEncMaxBeam; ++i)
+                    hl[i] = (lane < kEncThreads / 32 && i < beam) ? wtop[lane][i] : ~0ull;
+                for (int r = 0; r < beam; ++r) {
+                    const uint64_t m = warp_min_u64(hl[0]);
+                    if (hl[0] == m) pop16(hl);
+                    if (lane == 0) sel[r] = m;
+                }
+            }
+            __syncthreads();
+            const int nxt = cur ^ 1;
+            if (tid < beam) {
+                const uint64_t key = sel[tid];
+                const int pb = (int)((key >> 8) & 0xff), c = (int)(key & 0xff);
+                float cv[8], c0v[8];
+                load_f8(scb[k * 256 + c], cv);
+                load_f8(scb[k * 256 + c0], c0v);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) bD[nxt][tid][j] = bD[cur][pb][j] + cv[j] - c0v[j];
+#pragma unroll
+                for (int q = 0; q < K; ++q) bcode[nxt][tid][q] = bcode[cur][pb][q];
+                bcode[nxt][tid][k] = (uint8_t)c;
+            }
+            nb = beam;
+            cur = nxt;
+            __syncthreads();
+        }
+        // commit the best beam of the group
+        if (tid < 8) e[8 * g + tid] -= bD[cur][0][tid];
+        if (tid < K) codes_out[((size_t)o * G + g) * K + tid] = bcode[cur][0][tid];
+    }
+}
+
+
+}  // namespace aqk
+
+namespace aqh {
+using namespace aqk;
+
+size_t encode_workspace_bytes(const Geom &g) { return kWsHeader + align16((size_t)g.G * g.K * 256 * sizeof(float)); }
+
+cudaError_t launch_encode(const Geom &g, const uint16_t *w, const float *h, const uint16_t *cb,
+                          const void *codes_in, void *codes_out, int beam, void *ws, cudaStream_t s)
+{
+    float *q = reinterpret_cast<float *>(reinterpret_cast<char *>(ws) + kWsHeader);
+    const uint4 *c = reinterpret_cast<const uint4 *>(cb);
+    const int smem = g.in * (int)sizeof(float);
+    auto run = [&](auto kk) {
+        constexpr int K = decltype(kk)::value;
+        encode_q_kernel<K><<<g.G, 256, 0, s>>>(g.in, h, c, q);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(encode_kernel<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        encode_kernel<K><<<g.out, kEncThreads, smem, s>>>(g, w, h, c, q, reinterpret_cast<const uint8_t *>(codes_in),
+                                                          reinterpret_cast<uint8_t *>(codes_out), beam);
+        return cudaGetLastError();
+    };
+    if (g.B != 8) return cudaErrorInvalidValue;
+    if (g.K == 1) return run(std::integral_constant<int, 1>{});
+    if (g.K == 2) return run(std::integral_constant<int, 2>{});
+    if (g.K == 8) return run(std::integral_constant<int, 8>{});
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace aqh

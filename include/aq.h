@@ -243,6 +243,34 @@ aq_status aq_gemm(const aq_layer_desc *desc, const void *packed, const uint16_t 
  * The sums are accumulated with fp32 atomic adds: their order, and so the
  * last bits of the result, may change from run to run.
  */
+/*
+ * Encoder: beam search of the codes for fixed codebooks under the
+ * quantisation objective of the AQLM wiki entry ("Niveau tech avancé"),
+ * || W - sum_k C_k[i_k] ||^2_H with H = 2 X^T X.  The objective is a sum
+ * over output rows of e^T H e (e = w - reconstruction), so rows are
+ * independent.  Per row, groups in order with the others fixed, a beam of
+ * width `beam` runs over the group's K codes, codebook by codebook: every
+ * beam proposes each code for the slot, the `beam` proposals with the
+ * smallest objective survive (ties: parent beam, then code), and the best
+ * beam is kept before the next group.  The reconstruction is the exact
+ * codeword sum; arithmetic is fp32.
+ *   w          [out][in] binary16 (the weights to approximate),
+ *   h          [in][in] fp32, symmetric (e.g. 2 X^T X of calibration
+ *              activations),
+ *   codes_in   [out][in/8][K] uint8: the starting codes,
+ *   codes_out  [out][in/8][K] uint8, written (may not alias codes_in),
+ *   beam       1..16,
+ *   workspace  >= aq_encode_workspace_bytes(desc) bytes (a per-layer table
+ *              of C_k[c]^T H_gg C_k[c]).
+ * Codebooks of 8-bit codes only (1x8, 2x8, 8x8; AQ_ERR_UNSUPPORTED for
+ * B = 16, whose 65536-way search per group this library does not run);
+ * in <= 16384.
+ */
+size_t aq_encode_workspace_bytes(const aq_layer_desc *desc);
+aq_status aq_encode(const aq_layer_desc *desc, const uint16_t *w, const float *h, const uint16_t *codebooks,
+                    const void *codes_in, int beam, void *codes_out, void *workspace, size_t workspace_bytes,
+                    aq_stream_t stream);
+
 size_t aq_param_grad_workspace_bytes(const aq_layer_desc *desc, int T);
 aq_status aq_param_grad(const aq_layer_desc *desc, const void *packed, const uint16_t *codebooks,
                         const uint16_t *scales, const uint16_t *x, const uint16_t *gy, int T,

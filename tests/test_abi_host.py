@@ -190,3 +190,21 @@ def test_param_grad_argument_errors():
     assert call(ws=None) == 4 and call(wsb=4) == 4
     bad = aq.LayerDesc.make(64, 256, 4, 8)
     assert f(ctypes.byref(bad), FAKE, FAKE, FAKE, FAKE, FAKE, 64, FAKE, FAKE, FAKE, 1 << 20, None) == 2
+
+
+def test_encode_argument_errors():
+    d = aq.LayerDesc.make(64, 256, 2, 8)
+    f = aq.lib.aq_encode
+
+    def call(desc=d, w=FAKE, h=FAKE, cb=FAKE, ci=FAKE, beam=4, co=FAKE + 64, ws=FAKE, wsb=1 << 20):
+        return f(ctypes.byref(desc), w, h, cb, ci, beam, co, ws, wsb, None)
+
+    assert aq.aq_encode_workspace_bytes(d) >= 16 + 32 * 2 * 256 * 4
+    assert call(beam=0) == 1 and call(beam=17) == 1
+    assert call(w=None) == 1 and call(h=None) == 1 and call(ci=None) == 1 and call(co=None) == 1
+    assert call(co=FAKE) == 1  # codes_out aliases codes_in
+    assert call(w=FAKE + 2) == 3 and call(h=FAKE + 4) == 3 and call(cb=FAKE + 8) == 3
+    assert call(ws=None) == 4 and call(wsb=16) == 4
+    assert call(desc=aq.LayerDesc.make(64, 256, 1, 16)) == 2   # 16-bit codes: not run
+    assert aq.aq_encode_workspace_bytes(aq.LayerDesc.make(64, 256, 1, 16)) == 0
+    assert call(desc=aq.LayerDesc.make(64, 16392, 2, 8)) == 1   # in > 16384
