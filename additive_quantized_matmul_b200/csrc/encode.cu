@@ -143,9 +143,20 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(Geom L, const uint1
         __syncthreads();  // e holds every committed group
         {
             // v_j = sum_t H[8g + j][t] e[t], one warp per j (H rows coalesced)
+            // eight independent loads in flight per lane (an L2 round trip
+            // per step otherwise)
             const float *hr = h + (size_t)(8 * g + warp) * in;
-            float acc = 0.f;
-            for (int t = lane; t < in; t += 32) acc = fmaf(hr[t], e[t], acc);
+            float a8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            int t = lane;
+            for (; t + 7 * 32 < in; t += 8 * 32) {
+                float hv[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) hv[u] = __ldg(hr + t + 32 * u);
+#pragma unroll
+                for (int u = 0; u < 8; ++u) a8[u] = fmaf(hv[u], e[t + 32 * u], a8[u]);
+            }
+            for (; t < in; t += 32) a8[0] = fmaf(__ldg(hr + t), e[t], a8[0]);
+            float acc = ((a8[0] + a8[1]) + (a8[2] + a8[3])) + ((a8[4] + a8[5]) + (a8[6] + a8[7]));
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
             if (lane == 0) v[warp] = acc;
@@ -183,17 +194,17 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(Geom L, const uint1
                 load_f8(scb[k * 256 + tid], x);
                 const float qc = qtab[((size_t)g * K + k) * 256 + tid];
 #pragma unroll
-                for (int b = 0; b < kEncMaxBeam; ++b) {
-                    kk[b] = ~0ull;
-                    if (b < nb) {
-                        float d = 0.f;
+                for (int b = 0; b < kEncMaxBeam; ++b) kk[b] = ~0ull;
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) d = fmaf(x[i], bw[b][i], d);
-                        kk[b] = enc_key(bconst[b] + qc + 2.f * d, b, tid);
-                    }
+                for (int b = 0; b < kEncMaxBeam; ++b) {
+                    if (b >= nb) break;
+                    float d = 0.f;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) d = fmaf(x[i], bw[b][i], d);
+                    kk[b] = enc_key(bconst[b] + qc + 2.f * d, b, tid);
                 }
             }
-            sort16(kk);
+            if (nb > 1) sort16(kk);  // one live beam: kk[0] is the only key
             // the warp's `beam` smallest keys (keys are unique)
             for (int r = 0; r < beam; ++r) {
                 const uint64_t m = warp_min_u64(kk[0]);

@@ -147,6 +147,10 @@ def workload(name: str) -> dict:
         layers = [(f"{tag}-{K}x{B}", LayerSpec(o, i, K, B)) for K, B in ((1, 16), (2, 8))
                   for tag, (o, i) in (("q", LLAMA2_7B_BLOCK["q"]), ("gate", LLAMA2_7B_BLOCK["gate"]))]
         return {"layers": layers, "n": [2048], "seed": 1007}
+    if name == "llama2-7b-encode":
+        # code assignment (beam 8) for a 2x8 q projection and MLP up shape
+        layers = [("q-2x8", LayerSpec(4096, 4096, 2, 8)), ("gate-2x8", LayerSpec(11008, 4096, 2, 8))]
+        return {"layers": layers, "n": [8], "seed": 1008}
     if name == "llama2-7b-schemes":
         # the other schemes the pages name, at the Llama-2-7B MLP up shape
         layers = [(f"11008x4096-{K}x{B}", LayerSpec(11008, 4096, K, B)) for K, B in ((1, 8), (2, 16), (8, 8))]
@@ -167,4 +171,5 @@ def workload(name: str) -> dict:
 
 
 WORKLOADS = ("tiny-2x8", "llama2-7b-1x16", "llama2-7b-mlp-2x8",
-             "llama2-70b-1x16", "llama2-7b-prefill", "llama2-7b-block", "llama2-7b-schemes", "llama2-7b-grad")
+             "llama2-70b-1x16", "llama2-7b-prefill", "llama2-7b-block", "llama2-7b-schemes", "llama2-7b-grad",
+             "llama2-7b-encode")

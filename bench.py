@@ -268,6 +268,29 @@ def recorded_traffic(workload_name: str, batch: int):
     return rec["per_launch_bytes"].get(str(batch))
 
 
+def encode_flops(spec: LayerSpec, beam: int) -> int:
+    """Arithmetic of one aq_encode call: (H e)_g for every row and group
+    (2 out in^2) plus scoring every code for every beam of every slot
+    (about 18 flops per score)."""
+    G = spec.in_features // 8
+    return (2 * spec.out_features * spec.in_features ** 2
+            + spec.out_features * G * spec.num_codebooks * beam * (1 << spec.nbits) * 18)
+
+
+def encode_inputs(spec: LayerSpec, beam: int, seed) -> dict:
+    """Synthetic encoder inputs on the device: weights, H = 2 X^T X / n from
+    random activations, starting codes; the codes buffer it writes."""
+    import torch
+    rng = np.random.default_rng(seed)
+    w = rng.normal(0, 0.02, size=(spec.out_features, spec.in_features)).astype(np.float16)
+    x = torch.from_numpy(rng.normal(0, 1, size=(512, spec.in_features)).astype(np.float32)).cuda()
+    h = (2.0 / 512) * (x.T @ x)
+    c0 = rng.integers(0, 1 << spec.nbits, size=(spec.out_features, spec.in_features // 8, spec.num_codebooks))
+    codes = torch.from_numpy(c0.astype(np.uint8)).cuda()
+    return {"w": torch.from_numpy(w.view(np.int16)).cuda(), "h": h.contiguous(), "codes_in": codes,
+            "codes_out": torch.empty_like(codes)}
+
+
 def flops(spec: LayerSpec, n: int) -> int:
     return 2 * spec.out_features * spec.in_features * n
 
@@ -283,8 +306,9 @@ def run_gpu(args) -> None:
     dist = init_dist(world, "nccl")
     dev = torch.device("cuda", local)
     wl = workload(args.workload)
-    op = {"llama2-7b-prefill": "gemm", "llama2-7b-grad": "grad"}.get(args.workload, "gemv")
+    op = {"llama2-7b-prefill": "gemm", "llama2-7b-grad": "grad", "llama2-7b-encode": "encode"}.get(args.workload, "gemv")
     tensor_op = op in ("gemm", "grad")  # reported in TFLOP/s against the tensor peak
+    alu_op = op == "encode"             # fp32 CUDA-core work, reported against the derived fp32 FMA peak
     peaks = measured_peaks()
 
     # ---- units: one (layer shape, batch) product kind each, over a rotation
@@ -303,16 +327,18 @@ def run_gpu(args) -> None:
     for si, (tag, spec) in enumerate(wl["layers"]):
         desc, packed0, cb0, sc0 = device_layer(spec, (wl["seed"], rank, si))  # seeded per rank and shape
         lb = alg_bytes(spec, 0)
-        ncopies = args.layers or (3 if tensor_op else max(4, int(3 * L2_BYTES / lb) + 1))
+        ncopies = args.layers or (1 if alu_op else 3 if tensor_op else max(4, int(3 * L2_BYTES / lb) + 1))
         copies = [(packed0.clone(), cb0.clone(), sc0.clone()) for _ in range(ncopies)]
         del packed0, cb0, sc0
         for n in wl["n"]:
             x = torch.from_numpy(make_activations(spec.in_features, n, (wl["seed"], rank, si, n)).view(np.int16)).to(dev)
             nbytes = {"gemm": aq.aq_gemm_workspace_bytes, "grad": aq.aq_param_grad_workspace_bytes,
-                      "gemv": aq.aq_gemv_workspace_bytes}[op](desc, n)
+                      "gemv": aq.aq_gemv_workspace_bytes,
+                      "encode": lambda d, n: aq.aq_encode_workspace_bytes(d)}[op](desc, n)
             units.append({
                 "tag": tag, "spec": spec, "n": n, "desc": desc, "copies": copies, "x": x,
-                "bytes": alg_bytes(spec, n), "flops": flops(spec, n),
+                "bytes": alg_bytes(spec, n), "flops": encode_flops(spec, n) if op == "encode" else flops(spec, n),
+                **(encode_inputs(spec, n, (wl["seed"], rank, si)) if op == "encode" else {}),
                 **({"gy": torch.from_numpy(make_activations(spec.out_features, n, (wl["seed"], rank, si, n, 1))
                                            .view(np.int16)).to(dev),
                     "grad_s": torch.empty(spec.out_features, dtype=torch.float32, device=dev),
@@ -359,6 +385,9 @@ def run_gpu(args) -> None:
                 aq.aq_gemv(desc, packed, cb, sc, inp, 1, out, u["ws"], stream=s)
             return
         packed, cb, sc = u["copies"][i]
+        if op == "encode":
+            aq.aq_encode(u["desc"], u["w"], u["h"], cb, u["codes_in"], u["n"], u["codes_out"], u["ws"], stream=s)
+            return
         if op == "grad":
             aq.aq_param_grad(u["desc"], packed, cb, sc, x_in, u["gy"], u["n"], u["grad_s"], u["grad_cb"], u["ws"],
                              stream=s)
@@ -436,7 +465,15 @@ def run_gpu(args) -> None:
         k["frac_tensor"] = round(k["tflops"] / peaks["bf16_tflops_sustained"], 4)
         kernels.append(k)
     dom = max(kernels, key=lambda k: k["total_us"])
-    if tensor_op:
+    if alu_op:
+        value = world * step_flops * args.steps / (elapsed_ms * 1e-3) / 1e12
+        unit = "TFLOP/s"
+        fp32_peak = 148 * 128 * 2 * 1.965e9 / 1e12  # SMs x fp32 FMA lanes x 2 flops x max SM clock
+        roofline = {"bound": "alu", "achieved": dom["tflops"], "peak": round(fp32_peak, 1), "unit": "TFLOP/s",
+                    "frac": round(dom["tflops"] / fp32_peak, 4), "traffic": None,
+                    "kernel": f"aq_encode {dom['layer']} beam={dom['n']}",
+                    "peak_source": "derived: 148 SMs x 128 fp32 FMA/clk x 2 x 1965 MHz"}
+    elif tensor_op:
         value = world * step_flops * args.steps / (elapsed_ms * 1e-3) / 1e12
         unit = "TFLOP/s"
         roofline = {"bound": "tensor", "achieved": dom["tflops"], "peak": peaks["bf16_tflops_sustained"],
@@ -455,7 +492,7 @@ def run_gpu(args) -> None:
 
     # ---- end-to-end through the public API with host buffers ----------------
     e2e = None
-    if not args.skip_e2e and op != "grad":  # the gradient's outputs are parameters, not a per-step result
+    if not args.skip_e2e and op not in ("grad", "encode"):  # the gradient's outputs are parameters, not a per-step result
         hx = [torch.empty((len(u["copies"]), u["x"].numel()), dtype=torch.int16).pin_memory() for u in units]
         hy = [torch.empty((len(u["copies"]), out_buf(u, 0).numel()), dtype=torch.int16).pin_memory() for u in units]
         dx = [torch.empty(h.shape, dtype=torch.int16, device=dev) for h in hx]
@@ -536,7 +573,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=WORKLOAD,
                     help="llama2-7b-1x16 (default), llama2-7b-mlp-2x8, llama2-70b-1x16, "
-                         "llama2-7b-prefill, llama2-7b-block, llama2-7b-schemes, llama2-7b-grad, tiny-2x8")
+                         "llama2-7b-prefill, llama2-7b-block, llama2-7b-schemes, llama2-7b-grad, "
+                         "llama2-7b-encode, tiny-2x8")
     ap.add_argument("--layers", type=int, default=0, help="copies per shape (0: > 3x L2)")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--skip-e2e", action="store_true")
