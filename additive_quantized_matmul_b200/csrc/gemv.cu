@@ -21,6 +21,7 @@
 //    clock), not HBM.
 // Split-K partial sums go to the workspace and the last CTA to arrive for a
 // row range adds them in split order (no float atomics: bit-reproducible).
+#include <algorithm>
 #include <mutex>
 
 #include "scheme.cuh"
@@ -303,7 +304,13 @@ constexpr int kTcN = 16;
 // registers, so only the x copies are asynchronous.
 template <class S> struct TcRing {
     static constexpr bool kAsyncWeights = (S::K == 1 && S::B == 16);
-    static constexpr int depth = kAsyncWeights ? 5 : 3, lag = kAsyncWeights ? 3 : 1;
+    // 8-bit codebooks of one or two books are held as 8 replicas, replica r
+    // of codeword c at 16-byte slot 8c + r: decoder lane gi reads replica
+    // gi, so the 8 lanes of a 16-byte load phase (gi = 0..7) hit 8 distinct
+    // bank quads whatever their codes (random codes would conflict ~2.5x).
+    // Their 64 KiB leave room for a 2-stage ring at two CTAs per SM.
+    static constexpr int kReplicas = (S::kBooksInSmem && S::K <= 2) ? 8 : 1;
+    static constexpr int depth = kAsyncWeights ? 5 : (kReplicas > 1 ? 2 : 3), lag = kAsyncWeights ? 3 : 1;
 };
 constexpr int kTcTileA = kTcBM * 64 * 2;  // 16 KiB
 constexpr int kTcTileB = 64 * 32;         // 2 KiB: 64 rows x 16 columns
@@ -325,7 +332,8 @@ gemv_tc_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restri
     uint8_t *tileB = tileA + R * kTcTileA;    // [R][2 KiB]
     uint8_t *xring = tileB + R * kTcTileB;    // [R][2 KiB] raw x rows
     uint4 *scb = reinterpret_cast<uint4 *>(xring + R * kTcXSlot);  // B = 8 codebooks
-    uint64_t *full = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(scb) + S::kSmemBookBytes);
+    constexpr int NR = TcRing<S>::kReplicas;
+    uint64_t *full = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(scb) + S::kSmemBookBytes * NR);
     uint64_t *empty = full + R;
     uint64_t *acc_full = empty + R;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 1);
@@ -341,7 +349,7 @@ gemv_tc_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restri
 
     if (S::B == 16 && tid == 0) prefetch_table_share(cb, (uint32_t)S::K * 65536u * 16u);
     if constexpr (S::kBooksInSmem)
-        for (int i = tid; i < S::K * 256; i += kTcThreads) scb[i] = cb[i];
+        for (int i = tid; i < S::K * 256 * NR; i += kTcThreads) scb[i] = cb[i / NR];
     if (tid == 0) {
         for (int s = 0; s < R; ++s) {
             mbar_init(&full[s], kTcDecoders);
@@ -410,7 +418,14 @@ gemv_tc_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restri
                         // next row's reads and serialise the eight rows
                         uint4 t[8][S::K];
 #pragma unroll
-                        for (int r = 0; r < 8; ++r) gather_terms<S>(code, r, scb, cb, t[r]);
+                        for (int r = 0; r < 8; ++r) {
+                            if constexpr (NR > 1) {
+#pragma unroll
+                                for (int k = 0; k < S::K; ++k) t[r][k] = scb[(k * 256 + code.code(r, k)) * NR + gi];
+                            } else {
+                                gather_terms<S>(code, r, scb, cb, t[r]);
+                            }
+                        }
 #pragma unroll
                         for (int r = 0; r < 8; ++r)
                             *reinterpret_cast<uint4 *>(A + sw128(rt_l * 8 + r, gi)) =
@@ -556,6 +571,21 @@ struct GemvPlan {
 
 // Depends on the shape and batch only, so the workspace size can be
 // computed on a host without a GPU.
+template <class S>
+constexpr int tc_smem_bytes();
+
+// CTAs of gemv_tc_kernel that fit on one SM (228 KiB of shared memory, 1 KiB
+// reserved per CTA; 160 threads each, far below the thread limit).
+int tc_resident_ctas(const Geom &g)
+{
+    int smem = 0;
+    with_scheme(g, [&](auto sch) {
+        smem = tc_smem_bytes<decltype(sch)>();
+        return cudaSuccess;
+    });
+    return smem > 0 ? std::max(1, (228 * 1024) / (smem + 1024)) : 1;
+}
+
 GemvPlan plan_gemv(const Geom &g, int batch)
 {
     GemvPlan p{};
@@ -572,13 +602,26 @@ GemvPlan plan_gemv(const Geom &g, int batch)
         p.path = kTensor;
         const int mtiles = (g.out + kTcBM - 1) / kTcBM;
         const int nst = (g.G + 7) / 8;
-        // ~1024 CTAs at batch 1 (short tail, many gathers in flight), ~4 per
-        // SM above it: the decoders of one CTA wait on shared-memory and L2
-        // latency, so several CTAs per SM keep the pipes busy
-        const int target = batch == 1 ? 1024 : 4 * kNumSMs;
-        int ks = (target + mtiles - 1) / mtiles;
-        ks = max(1, min(ks, (nst + 7) / 8));  // at least 8 stages per CTA: the ring fills
-        p.per_split = (nst + ks - 1) / ks;
+        // Split count by a wave model: CTAs of this kernel fit `res` per SM
+        // (shared memory), a CTA costs its stages plus about three stages of
+        // fixed latency (prologue, pipeline fill and drain, split-K finish),
+        // and a partial last wave costs a whole CTA.  At least 8 stages per
+        // split: shorter splits lose more to fill and drain, and their
+        // partial sums grow with the batch (measured on Llama-2 70B shapes).
+        const int slots = tc_resident_ctas(g) * kNumSMs;
+        const int min_stages = 8;
+        int best_ks = 1;
+        long best_cost = -1;
+        for (int ks = 1; ks <= std::max(1, nst / min_stages); ++ks) {
+            const long ctas = (long)mtiles * ks;
+            const long waves = (ctas + slots - 1) / slots;
+            const long cost = waves * ((nst + ks - 1) / ks + 3);
+            if (best_cost < 0 || cost < best_cost) {
+                best_cost = cost;
+                best_ks = ks;
+            }
+        }
+        p.per_split = (nst + best_ks - 1) / best_ks;
         p.ks = (nst + p.per_split - 1) / p.per_split;
         p.grid_x = mtiles;
         p.rt_per_cta = kTcBM / 8;
@@ -592,7 +635,7 @@ GemvPlan plan_gemv(const Geom &g, int batch)
 template <class S>
 constexpr int tc_smem_bytes()
 {
-    return 1024 + TcRing<S>::depth * (kTcTileA + kTcTileB + kTcXSlot) + S::kSmemBookBytes +
+    return 1024 + TcRing<S>::depth * (kTcTileA + kTcTileB + kTcXSlot) + S::kSmemBookBytes * TcRing<S>::kReplicas +
            (2 * TcRing<S>::depth + 1) * 8 + 16;
 }
 
