@@ -215,6 +215,12 @@ gemm_tc_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restri
 // for BN = 512.
 template <class S, int BN>
 constexpr int kWsStagesOf = (BN == 512) ? 2 : (S::kSmemBookBytes > 8192) ? 3 : 4;
+// The W (decoded) tiles have a ring of their own, 5 deep (4 with the 32 KiB
+// of 8x8 codebooks): with 512-token X tiles taking 64 KiB a stage, a shared
+// ring would be 2 deep and leave the 1x16 gathers a copy lag of 1 (about
+// 2000 codewords in flight per CTA); lag 3 here, 4000 in flight.
+template <class S, int BN>
+constexpr int kWsAStagesOf = (BN == 512) ? ((S::kSmemBookBytes > 8192) ? 4 : 5) : kWsStagesOf<S, BN>;
 constexpr int kWsThreads = 192;               // 6 warps
 constexpr int kWsLag = 2;                     // cp.async stages in flight per decoder (< ring depth)
 
@@ -296,19 +302,21 @@ gemm_ws_kernel(const __grid_constant__ CUtensorMap xmap, Geom L, const uint8_t *
                const uint4 *__restrict__ cb, const uint16_t *__restrict__ scales, int T,
                uint16_t *__restrict__ y, void *ws, GemmSplit sp, int stages_per_split)
 {
-    constexpr int kWsStages = kWsStagesOf<S, BN>;
+    constexpr int kWsStages = kWsStagesOf<S, BN>;    // X ring
+    constexpr int kWsAStages = kWsAStagesOf<S, BN>;  // W ring
     constexpr int kWsTileB = kBK * BN * 2;   // 32 or 64 KiB
     constexpr int kN = BN < 256 ? BN : 256;  // N of one MMA instruction
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t *smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
     uint8_t *tileA = smem;                                   // [stages][16 KiB]
-    uint8_t *tileB = smem + kWsStages * kTileABytes;         // [stages][32 KiB]
+    uint8_t *tileB = smem + kWsAStages * kTileABytes;        // [X stages][32 or 64 KiB]
     uint4 *scb = reinterpret_cast<uint4 *>(tileB + kWsStages * kWsTileB);
     uint64_t *full_a = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(scb) + S::kSmemBookBytes);
-    uint64_t *full_b = full_a + kWsStages;
-    uint64_t *empty = full_b + kWsStages;
-    uint64_t *acc_full = empty + kWsStages;
+    uint64_t *full_b = full_a + kWsAStages;
+    uint64_t *empty = full_b + kWsStages;       // X buffers free
+    uint64_t *empty_a = empty + kWsStages;      // W buffers free
+    uint64_t *acc_full = empty_a + kWsAStages;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 1);
     uint32_t *abort_flag = tmem_slot + 1;
 
@@ -327,8 +335,11 @@ gemm_ws_kernel(const __grid_constant__ CUtensorMap xmap, Geom L, const uint8_t *
     if constexpr (S::kBooksInSmem)
         for (int i = tid; i < S::K * 256; i += kWsThreads) scb[i] = cb[i];
     if (tid == 0) {
-        for (int s = 0; s < kWsStages; ++s) {
+        for (int s = 0; s < kWsAStages; ++s) {
             mbar_init(&full_a[s], 128);
+            mbar_init(&empty_a[s], 1);
+        }
+        for (int s = 0; s < kWsStages; ++s) {
             mbar_init(&full_b[s], 1);
             mbar_init(&empty[s], 1);
         }
@@ -366,15 +377,15 @@ gemm_ws_kernel(const __grid_constant__ CUtensorMap xmap, Geom L, const uint8_t *
             const uint32_t idesc = make_idesc(kBM, kN, true);
             int s = 0;
             for (; s < nk; ++s) {
-                const int buf = s % kWsStages;
-                const uint32_t par = (s / kWsStages) & 1;
-                if (!mbar_wait_ns(&full_a[buf], par, kWaitNs) || !mbar_wait_ns(&full_b[buf], par, kWaitNs)) {
+                const int buf = s % kWsStages, abuf = s % kWsAStages;
+                if (!mbar_wait_ns(&full_a[abuf], (s / kWsAStages) & 1, kWaitNs) ||
+                    !mbar_wait_ns(&full_b[buf], (s / kWsStages) & 1, kWaitNs)) {
                     *abort_v = 1;
                     break;
                 }
                 if (*abort_v) break;
                 tc_fence_after();
-                const uint32_t a0 = smem_u32(tileA + buf * kTileABytes);
+                const uint32_t a0 = smem_u32(tileA + abuf * kTileABytes);
                 const uint32_t b0 = smem_u32(tileB + buf * kWsTileB);
 #pragma unroll
                 for (int ks = 0; ks < kBK / 16; ++ks) {
@@ -386,7 +397,8 @@ gemm_ws_kernel(const __grid_constant__ CUtensorMap xmap, Geom L, const uint8_t *
                         mma_f16_ss(tmem + h * kN, ad, bd, idesc, (s > 0 || ks > 0) ? 1u : 0u);
                     }
                 }
-                mma_commit(&empty[buf]);
+                mma_commit(&empty[buf]);     // X buffer free once these MMAs complete
+                mma_commit(&empty_a[abuf]);  // and the W buffer
             }
             mma_commit(acc_full);  // completes when every MMA issued above has
         }
@@ -407,8 +419,8 @@ gemm_ws_kernel(const __grid_constant__ CUtensorMap xmap, Geom L, const uint8_t *
         // copies of kLag stages stay in flight; a stage is published kLag
         // iterations after it is issued, so kLag must stay below the ring
         // depth (the decoder waits for the MMAs of stage s - depth first)
-        constexpr int kLag = kAsyncWeights ? (kWsLag < kWsStages - 1 ? kWsLag : kWsStages - 1) : 0;
-        static_assert(kLag < kWsStages, "copy lag must be below the ring depth");
+        constexpr int kLag = !kAsyncWeights ? 0 : (BN == 512 ? 3 : (kWsLag < kWsAStages - 1 ? kWsLag : kWsAStages - 1));
+        static_assert(kLag < kWsAStages - 1 || !kAsyncWeights, "copy lag must leave the MMAs a stage of slack");
         bool ok = true;
         // unrolled by the ring depth so every ring index is static
         for (int s0i = 0; ok && s0i < nk + kLag; s0i += kCodeAhead) {
@@ -417,8 +429,8 @@ gemm_ws_kernel(const __grid_constant__ CUtensorMap xmap, Geom L, const uint8_t *
                 const int s = s0i + u;
                 if (s >= nk + kLag) break;
                 if (s < nk) {
-                    const int buf = s % kWsStages;
-                    if (s >= kWsStages && !mbar_wait_ns(&empty[buf], ((s / kWsStages) - 1) & 1, kWaitNs)) {
+                    const int buf = s % kWsAStages;
+                    if (s >= kWsAStages && !mbar_wait_ns(&empty_a[buf], ((s / kWsAStages) - 1) & 1, kWaitNs)) {
                         *abort_v = 1;
                     }
                     if (*abort_v) {
@@ -465,11 +477,11 @@ gemm_ws_kernel(const __grid_constant__ CUtensorMap xmap, Geom L, const uint8_t *
                     if (j >= 0) {
                         cp_async_wait<kLag>();
                         fence_proxy_async_smem();
-                        mbar_arrive(&full_a[j % kWsStages]);
+                        mbar_arrive(&full_a[j % kWsAStages]);
                     }
                 } else {
                     fence_proxy_async_smem();
-                    mbar_arrive(&full_a[s % kWsStages]);
+                    mbar_arrive(&full_a[s % kWsAStages]);
                 }
             }
         }
@@ -617,8 +629,8 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
 template <class S, int BN>
 static constexpr int gemm_ws_smem_bytes()
 {
-    return 1024 + kWsStagesOf<S, BN> * (kTileABytes + kBK * BN * 2) + S::kSmemBookBytes +
-           (3 * kWsStagesOf<S, BN> + 1) * 8 + 16;
+    return 1024 + kWsAStagesOf<S, BN> * kTileABytes + kWsStagesOf<S, BN> * (kBK * BN * 2) + S::kSmemBookBytes +
+           (2 * kWsAStagesOf<S, BN> + 2 * kWsStagesOf<S, BN> + 1) * 8 + 16;
 }
 
 cudaError_t launch_gemm(const Geom &g, const void *packed, const uint16_t *cb,
