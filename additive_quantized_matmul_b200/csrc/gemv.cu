@@ -311,6 +311,15 @@ template <class S> struct TcRing {
     // Their 64 KiB leave room for a 2-stage ring at two CTAs per SM.
     static constexpr int kReplicas = (S::kBooksInSmem && S::K <= 2) ? 8 : 1;
     static constexpr int depth = kAsyncWeights ? 5 : (kReplicas > 1 ? 2 : 3), lag = kAsyncWeights ? 3 : 1;
+    // 1x16: the decoders only gather weights and start before the previous
+    // launch ends; the MMA warp waits for it and loads the activations (B
+    // tiles, raw x slots) into a ring of their own, xpre stages ahead into
+    // slots last used xring - xpre stages earlier.  Other schemes: the
+    // decoders wait, then load each stage's x into the slot of their A
+    // buffer (their stage period is set by decode, and a shallow x ring on
+    // the MMA warp would put the x latency on its path).
+    static constexpr bool kXByMma = kAsyncWeights;
+    static constexpr int xring = kXByMma ? 4 : depth, xpre = 2;
 };
 constexpr int kTcTileA = kTcBM * 64 * 2;  // 16 KiB
 constexpr int kTcTileB = 64 * 32;         // 2 KiB: 64 rows x 16 columns
@@ -329,13 +338,15 @@ gemv_tc_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restri
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t *smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
     uint8_t *tileA = smem;                    // [R][16 KiB]
-    uint8_t *tileB = tileA + R * kTcTileA;    // [R][2 KiB]
-    uint8_t *xring = tileB + R * kTcTileB;    // [R][2 KiB] raw x rows
-    uint4 *scb = reinterpret_cast<uint4 *>(xring + R * kTcXSlot);  // B = 8 codebooks
+    constexpr int RX = TcRing<S>::xring, PRE = TcRing<S>::xpre;
+    uint8_t *tileB = tileA + R * kTcTileA;    // [RX][2 KiB]
+    uint8_t *xring = tileB + RX * kTcTileB;   // [RX][2 KiB] raw x rows
+    uint4 *scb = reinterpret_cast<uint4 *>(xring + RX * kTcXSlot);  // B = 8 codebooks
     constexpr int NR = TcRing<S>::kReplicas;
     uint64_t *full = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(scb) + S::kSmemBookBytes * NR);
     uint64_t *empty = full + R;
-    uint64_t *acc_full = empty + R;
+    uint64_t *emptyx = empty + R;          // [RX] activation slot free
+    uint64_t *acc_full = emptyx + RX;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 1);
     uint32_t *abort_flag = tmem_slot + 1;
 
@@ -355,6 +366,9 @@ gemv_tc_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restri
             mbar_init(&full[s], kTcDecoders);
             mbar_init(&empty[s], 1);
         }
+        for (int s = 0; s < RX; ++s) {
+            mbar_init(&emptyx[s], 1);
+        }
         mbar_init(acc_full, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -371,17 +385,20 @@ gemv_tc_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restri
         const int rt_l = tid >> 3, gi = tid & 7;  // A role: row tile, group
         const int rt = (m0 >> 3) + rt_l;
         const bool rows_live = rt < L.rtiles;
-        const int kr = tid >> 1, hb = tid & 1;    // B role: feature row, 8-column half
         Chunk<S> code_ring[kCodeAhead];
 #pragma unroll
         for (int q = 0; q < kCodeAhead; ++q) {
             const int g = (s0 + q) * 8 + gi;
             code_ring[q] = load_chunk<S>(packed, (size_t)rt * L.gp + g, q < nloc && rows_live && g < L.G);
         }
-        // everything above touched weights only; x, y and the workspace may
-        // be written by the previous launch on the stream
-        grid_dependency_wait();
+        // 1x16 decoders touch weights only (codes, codebook): they do not
+        // wait for the previous launch on the stream, so their gathers may
+        // overlap its end (the MMA warp waits before it loads x, and every
+        // store of partial sums or y follows the MMAs).  Other decoders also
+        // load x, so they wait first.
+        if constexpr (!TcRing<S>::kXByMma) grid_dependency_wait();
         grid_launch_dependents();
+        const int kr = tid >> 1, hb = tid & 1;  // x role (other schemes): feature row, 8-column half
         bool ok = true;
         // stage loop unrolled by the code-ring depth so every ring index is static
         for (int i0 = 0; ok && i0 < nloc + LAG; i0 += kCodeAhead) {
@@ -439,19 +456,22 @@ gemv_tc_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restri
                                 live ? sum_round_fast_h8<S::K>(t) : make_uint4(0, 0, 0, 0);
                         }
                     }
-                    // x rows of this stage: straight into the B tile when a row is
-                    // 16 or 32 bytes, else the raw rows into the stage's x slot
-                    if (x_direct) {
-                        const int k = s * 64 + kr, n0 = hb * 8;
-                        const bool in = k < L.in && n0 < batch;
-                        cp_async16(smem_u32(tileB + buf * kTcTileB) + sw32(kr, hb),
-                                   in ? (const void *)(x + (size_t)k * batch + n0) : (const void *)x, in ? 16u : 0u);
-                    } else if (tid < 8 * batch) {
-                        const int valid = max(0, min(64, L.in - s * 64)) * batch * 2;
-                        const int nb = max(0, min(16, valid - tid * 16));
-                        const uint8_t *src = reinterpret_cast<const uint8_t *>(x + (size_t)s * 64 * batch) + tid * 16;
-                        cp_async16(smem_u32(xring + buf * kTcXSlot) + tid * 16, nb > 0 ? (const void *)src : (const void *)x,
-                                   (uint32_t)nb);
+                    if constexpr (!TcRing<S>::kXByMma) {
+                        // x rows of this stage into the slot of this A buffer:
+                        // straight into the B tile when a row is 16 or 32
+                        // bytes, else the raw rows into the x slot
+                        if (x_direct) {
+                            const int k = s * 64 + kr, n0 = hb * 8;
+                            const bool in = k < L.in && n0 < batch;
+                            cp_async16(smem_u32(tileB + buf * kTcTileB) + sw32(kr, hb),
+                                       in ? (const void *)(x + (size_t)k * batch + n0) : (const void *)x, in ? 16u : 0u);
+                        } else if (tid < 8 * batch) {
+                            const int valid = max(0, min(64, L.in - s * 64)) * batch * 2;
+                            const int nb = max(0, min(16, valid - tid * 16));
+                            const uint8_t *src = reinterpret_cast<const uint8_t *>(x + (size_t)s * 64 * batch) + tid * 16;
+                            cp_async16(smem_u32(xring + buf * kTcXSlot) + tid * 16,
+                                       nb > 0 ? (const void *)src : (const void *)x, (uint32_t)nb);
+                        }
                     }
                 }
                 cp_async_commit();  // one group per iteration (empty in the drain)
@@ -495,9 +515,59 @@ gemv_tc_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restri
         }
     } else {
         // ------------------------------ MMA warp ------------------------------
+        // x, y and the workspace follow the previous launch on the stream:
+        // this warp waits for it, then loads x PRE stages ahead (x rows go
+        // straight into the B tile when a row is 16 or 32 bytes, else as raw
+        // rows into the slot's x buffer)
+        constexpr bool kX = TcRing<S>::kXByMma;
+        if constexpr (kX) grid_dependency_wait();
         const uint32_t idesc = make_idesc(kTcBM, kTcN, true);
+        auto load_x = [&](int q) {
+            const int sx = s0 + q, xb = q % RX;
+            if (x_direct) {
+#pragma unroll
+                for (int c = lane; c < 128; c += 32) {
+                    const int kr = c >> 1, n0 = (c & 1) * 8;
+                    const int k = sx * 64 + kr;
+                    const bool in = k < L.in && n0 < batch;
+                    cp_async16(smem_u32(tileB + xb * kTcTileB) + sw32(kr, c & 1),
+                               in ? (const void *)(x + (size_t)k * batch + n0) : (const void *)x, in ? 16u : 0u);
+                }
+            } else {
+                const int valid = max(0, min(64, L.in - sx * 64)) * batch * 2;
+                for (int t = lane; t < 8 * batch; t += 32) {
+                    const int nb = max(0, min(16, valid - t * 16));
+                    const uint8_t *src = reinterpret_cast<const uint8_t *>(x + (size_t)sx * 64 * batch) + t * 16;
+                    cp_async16(smem_u32(xring + xb * kTcXSlot) + t * 16, nb > 0 ? (const void *)src : (const void *)x,
+                               (uint32_t)nb);
+                }
+            }
+        };
+        if constexpr (kX) {
+#pragma unroll
+            for (int q = 0; q < PRE; ++q) {
+                if (q < nloc) load_x(q);
+                cp_async_commit();  // one group per stage, empty ones included
+            }
+        }
         for (int j = 0; j < nloc; ++j) {
-            const int buf = j % R;
+            const int buf = j % R, xb = kX ? j % RX : buf;
+            if constexpr (kX) {
+                // x of stage j + PRE, into a slot whose last MMAs (stage
+                // j + PRE - RX) were committed RX - PRE iterations ago
+                const int q = j + PRE;
+                bool fr = true;
+                if (q < nloc && q >= RX) fr = mbar_wait_ns(&emptyx[q % RX], ((q / RX) - 1) & 1, kWaitNs);
+                if (!__all_sync(0xffffffffu, fr)) {
+                    *abort_v = 1;
+                    break;
+                }
+                if (q < nloc) load_x(q);
+                cp_async_commit();
+                cp_async_wait<PRE>();  // this lane's copies of stage j have landed
+                __syncwarp();           // and every lane's
+                fence_proxy_async_smem();
+            }
             const bool got = mbar_wait_ns(&full[buf], (j / R) & 1, kWaitNs);
             if (!__all_sync(0xffffffffu, got)) {
                 *abort_v = 1;
@@ -506,14 +576,14 @@ gemv_tc_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restri
             if (__any_sync(0xffffffffu, *abort_v != 0)) break;
             if (!x_direct) {
                 // B tile rows from the stage's raw x slot: 64 rows x 2 halves
-                const uint16_t *xs = reinterpret_cast<const uint16_t *>(xring + buf * kTcXSlot);
+                const uint16_t *xs = reinterpret_cast<const uint16_t *>(xring + xb * kTcXSlot);
 #pragma unroll
                 for (int c = lane; c < 128; c += 32) {
                     const int krow = c >> 1, n0 = (c & 1) * 8;
                     uint16_t h[8];
 #pragma unroll
                     for (int q = 0; q < 8; ++q) h[q] = (n0 + q < batch) ? xs[krow * batch + n0 + q] : (uint16_t)0;
-                    *reinterpret_cast<uint4 *>(tileB + buf * kTcTileB + sw32(krow, c & 1)) =
+                    *reinterpret_cast<uint4 *>(tileB + xb * kTcTileB + sw32(krow, c & 1)) =
                         make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16), h[4] | (h[5] << 16), h[6] | (h[7] << 16));
                 }
                 fence_proxy_async_smem();
@@ -522,17 +592,19 @@ gemv_tc_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restri
             if (lane == 0) {
                 tc_fence_after();
                 const uint32_t a0 = smem_u32(tileA + buf * kTcTileA);
-                const uint32_t b0 = smem_u32(tileB + buf * kTcTileB);
+                const uint32_t b0 = smem_u32(tileB + xb * kTcTileB);
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks) {
                     const uint64_t ad = smem_desc_sw128(a0 + ks * 32, 16, 1024);
                     const uint64_t bd = smem_desc(b0 + ks * 512, kTcTileB, 256, kSwizzle32B);
                     mma_f16_ss(tmem, ad, bd, idesc, (j > 0 || ks > 0) ? 1u : 0u);
                 }
-                mma_commit(&empty[buf]);
+                mma_commit(&empty[buf]);                // A buffer free once these MMAs complete
+                if constexpr (kX) mma_commit(&emptyx[xb]);  // and the activation slot
             }
             __syncwarp();
         }
+        cp_async_wait<0>();  // no copy of x may still be landing when the CTA ends
         if (lane == 0) mma_commit(acc_full);  // completes when every MMA issued above has
     }
     __syncthreads();
@@ -635,8 +707,8 @@ GemvPlan plan_gemv(const Geom &g, int batch)
 template <class S>
 constexpr int tc_smem_bytes()
 {
-    return 1024 + TcRing<S>::depth * (kTcTileA + kTcTileB + kTcXSlot) + S::kSmemBookBytes * TcRing<S>::kReplicas +
-           (2 * TcRing<S>::depth + 1) * 8 + 16;
+    return 1024 + TcRing<S>::depth * kTcTileA + TcRing<S>::xring * (kTcTileB + kTcXSlot) +
+           S::kSmemBookBytes * TcRing<S>::kReplicas + (2 * TcRing<S>::depth + TcRing<S>::xring + 1) * 8 + 16;
 }
 
 template <class Kern>
