@@ -31,6 +31,13 @@
  *    state between calls (thread-safe; calls on one stream are ordered);
  *  - work is enqueued on `stream` (NULL = legacy default stream) and the
  *    call returns after the launch; the caller synchronises;
+ *  - the GEMV kernels use programmatic dependent launch: a GEMV may start
+ *    reading its weights (packed codes, codebooks) while the GEMV launched
+ *    just before it on the stream is still running; it reads x and writes
+ *    y and the workspace only after that launch has completed.  GEMVs write
+ *    no weights, and other kernels (this library's or the caller's) let the
+ *    next launch start only when they complete, so stream order holds for
+ *    every value a caller can observe;
  *  - all arguments are validated on the host before anything is launched;
  *    on any error status nothing is launched and no output byte is written;
  *  - array pointers must be 16-byte aligned (AQ_ERR_MISALIGNED otherwise);
