@@ -158,7 +158,6 @@ aq_status aq_gemv_noalloc(const aq_layer_desc *desc, const void *packed, const u
         return AQ_ERR_MISALIGNED;
     if (scales && (reinterpret_cast<uintptr_t>(scales) & 1u)) return AQ_ERR_MISALIGNED;
     const Geom g = aqk::make_geom(*desc);
-    if (aqh::gemv_workspace_bytes(g, batch) > AQ_GEMV_NOALLOC_SCRATCH_BYTES) return AQ_ERR_WORKSPACE;
     bool too_large = false;
     const cudaError_t e = aqh::launch_gemv_noalloc(g, packed, codebooks, scales, x, batch, y,
                                                    reinterpret_cast<cudaStream_t>(stream), &too_large);

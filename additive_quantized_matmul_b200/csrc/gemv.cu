@@ -30,19 +30,24 @@
 namespace aqk {
 
 struct SplitK {
-    float *partials;      // [ks][rows8][batch]
-    unsigned *counters;   // [grid.x]
+    float *partials;      // [slots][rows8][batch]
+    unsigned *counters;   // one per row range
 };
 
 // Called by every thread of a CTA after it stored its partial sums for rows
-// [row0, row0 + nrows), columns [0, batch) of split blockIdx.y (nrows is a
-// multiple of 8, so the block is a whole number of float4).  The last CTA of
-// the row range to arrive reduces the splits in split order, writes y and
-// resets the counter for the next call.  All loads of a float4 are issued
-// before the (ordered) sum, so the finish costs about one L2 round trip.
-__device__ __forceinline__ void splitk_finish(const Geom &L, SplitK sk, int row0, int nrows,
-                                              int batch, const uint16_t *__restrict__ scales,
-                                              uint16_t *__restrict__ y)
+// [row0, row0 + nrows), columns [0, batch), into its slot of that row range
+// (nrows is a multiple of 8 and row0 + nrows <= rows8, so the block is a
+// whole number of float4 inside every slot).  The row range has `ks` slots
+// and arrival counter `counter`; the last CTA to arrive reduces the slots in
+// slot order, writes y and resets the counter for the next call.  With
+// `stage` (shared memory the CTA no longer needs, `stage_bytes` of it) the
+// partial sums are staged there: every (slot, float4) of a pass is requested
+// at once with cp.async, so a pass costs about one L2 round trip whatever
+// ks.  Without it (or with fewer than 16 ks bytes) they are summed straight
+// from L2, eight slots in flight per float4.
+__device__ __forceinline__ void splitk_finish(const Geom &L, SplitK sk, int counter, int ks, int row0,
+                                              int nrows, int batch, const uint16_t *__restrict__ scales,
+                                              uint16_t *__restrict__ y, float4 *stage, int stage_bytes)
 {
     __shared__ unsigned s_last;
     __syncthreads();
@@ -51,42 +56,73 @@ __device__ __forceinline__ void splitk_finish(const Geom &L, SplitK sk, int row0
         // release fence, which publishes them with the counter increment;
         // the last CTA's acquire fence orders its reads after all of them
         fence_acq_rel_gpu();
-        const unsigned prev = atomicAdd(&sk.counters[blockIdx.x], 1u);
-        s_last = (prev == gridDim.y - 1) ? 1u : 0u;
+        const unsigned prev = atomicAdd(&sk.counters[counter], 1u);
+        s_last = (prev == (unsigned)ks - 1u) ? 1u : 0u;
         if (s_last) fence_acq_rel_gpu();
     }
     __syncthreads();
     if (!s_last) return;
-    const int ks = gridDim.y;
     const size_t vstride = (size_t)L.rows8 * batch / 4;
     const float4 *base = reinterpret_cast<const float4 *>(sk.partials + (size_t)row0 * batch);
     const int nvec = nrows * batch / 4;
-    for (int e = threadIdx.x; e < nvec; e += blockDim.x) {
-        float4 acc = __ldcg(base + e);
-        for (int s0 = 1; s0 < ks; s0 += 8) {
-            float4 t[8];
+    const int chunk = min(nvec, stage_bytes / (16 * ks));  // float4 elements per pass
+    if (chunk == 0) {
+        // no staging area, or more slots than it holds
+        for (int e = threadIdx.x; e < nvec; e += blockDim.x) {
+            float4 acc = __ldcg(base + e);
+            for (int s0 = 1; s0 < ks; s0 += 8) {
+                float4 t[8];
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-                if (s0 + j < ks) t[j] = __ldcg(base + (size_t)(s0 + j) * vstride + e);
+                for (int j = 0; j < 8; ++j)
+                    if (s0 + j < ks) t[j] = __ldcg(base + (size_t)(s0 + j) * vstride + e);
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-                if (s0 + j < ks) {
-                    acc.x += t[j].x; acc.y += t[j].y; acc.z += t[j].z; acc.w += t[j].w;
+                for (int j = 0; j < 8; ++j)
+                    if (s0 + j < ks) {
+                        acc.x += t[j].x; acc.y += t[j].y; acc.z += t[j].z; acc.w += t[j].w;
+                    }
+            }
+            const float v[4] = {acc.x, acc.y, acc.z, acc.w};
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const int idx = e * 4 + c;
+                const int row = row0 + idx / batch;
+                if (row < L.out) {
+                    const float sc = scales ? __half2float(__ushort_as_half(scales[row])) : 1.f;
+                    y[(size_t)row * batch + idx % batch] = __half_as_ushort(__float2half_rn(sc * v[c]));
                 }
-        }
-        const float v[4] = {acc.x, acc.y, acc.z, acc.w};
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            const int idx = e * 4 + c;
-            const int row = row0 + idx / batch;
-            const int b = idx % batch;
-            if (row < L.out) {
-                const float sc = scales ? __half2float(__ushort_as_half(scales[row])) : 1.f;
-                y[(size_t)row * batch + b] = __half_as_ushort(__float2half_rn(sc * v[c]));
             }
         }
     }
-    if (threadIdx.x == 0) sk.counters[blockIdx.x] = 0u;
+    for (int c0 = 0; chunk > 0 && c0 < nvec; c0 += chunk) {
+        const int n = min(chunk, nvec - c0);
+        for (int q = threadIdx.x; q < ks * n; q += blockDim.x) {
+            const int sl = q / n, e = q - sl * n;
+            cp_async16(smem_u32(stage + q), base + (size_t)sl * vstride + c0 + e, 16u);
+        }
+        cp_async_commit();
+        cp_async_wait<0>();
+        __syncthreads();
+        for (int e = threadIdx.x; e < n; e += blockDim.x) {
+            float4 acc = stage[e];
+            for (int sl = 1; sl < ks; ++sl) {
+                const float4 t = stage[sl * n + e];
+                acc.x += t.x; acc.y += t.y; acc.z += t.z; acc.w += t.w;
+            }
+            const float v[4] = {acc.x, acc.y, acc.z, acc.w};
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const int idx = (c0 + e) * 4 + c;
+                const int row = row0 + idx / batch;
+                const int b = idx % batch;
+                if (row < L.out) {
+                    const float sc = scales ? __half2float(__ushort_as_half(scales[row])) : 1.f;
+                    y[(size_t)row * batch + b] = __half_as_ushort(__float2half_rn(sc * v[c]));
+                }
+            }
+        }
+        __syncthreads();  // the next pass reuses the staging area
+    }
+    if (threadIdx.x == 0) sk.counters[counter] = 0u;
 }
 
 // ---------------------------------------------------------------------------
@@ -267,14 +303,28 @@ gemv_lut_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restr
         }
     }
     if (gridDim.y == 1) return;
-    splitk_finish(L, sk, rt0 * 8, (rt1 - rt0) * 8, 1, scales, y);
+    // one float4 per thread: summed straight from L2 (measured faster here
+    // than staging the slots in the tables' shared memory)
+    splitk_finish(L, sk, blockIdx.x, gridDim.y, rt0 * 8, (rt1 - rt0) * 8, 1, scales, y, nullptr, 0);
 }
 
 // ---------------------------------------------------------------------------
 // Small-batch product on the tensor cores (any batch for 1x16, batch 2..16
 // for 2x8), warp-specialised.
 //
-// CTA = 128 rows x one split of the K range; 4 decoder warps + 1 MMA warp.
+// Work split, one of two (a template flag): the units of work are (row
+// tile m of 128 rows, stage s of 64 input features).
+//  * per row tile (kSK false): CTA (m, q) takes stages [q len, (q + 1) len)
+//    of row tile m; grid (row tiles, splits).
+//  * stream-K (kSK true): units m-major, CTA c takes the `len` units from
+//    c len on, so every CTA does the same number of stages whatever the
+//    shape; len <= stages per row tile, so a CTA covers the end of one row
+//    tile and at most the start of the next: one fp32 TMEM accumulator of 16
+//    columns per row tile (segment).  It balances shapes whose row tiles
+//    split badly over the SMs (28672 x 8192: 224 tiles of 128 stages).
+// A row tile covered by several CTAs is finished by the last to arrive,
+// which adds the partial sums in split (CTA) order.
+// 4 decoder warps + 1 MMA warp.
 // Per stage of 64 input features (8 groups), decoder thread t owns code chunk
 // (row tile t/8, group t%8) of the 128 x 64 A tile (128-byte swizzle,
 // K-major):
@@ -297,8 +347,6 @@ constexpr int kTcDecoders = 128;
 constexpr int kTcThreads = kTcDecoders + 32;
 constexpr int kTcBM = 128;
 constexpr int kTcN = 16;
-// ring depth and copy-to-signal lag: deep for the asynchronous 1x16 gathers,
-// short for the synchronous 2x8 decode
 // Ring depth and copy lag: 1x16 codewords arrive by cp.async from L2 (deep
 // ring, copies of three stages in flight); the other schemes decode in
 // registers, so only the x copies are asynchronous.
@@ -324,14 +372,22 @@ template <class S> struct TcRing {
 constexpr int kTcTileA = kTcBM * 64 * 2;  // 16 KiB
 constexpr int kTcTileB = 64 * 32;         // 2 KiB: 64 rows x 16 columns
 constexpr int kTcXSlot = 64 * 16 * 2;     // raw x rows of one stage, batch <= 16
-constexpr int kTcTmemCols = 32;
+constexpr int kTcTmemCols = 32;  // two accumulators of 16 columns (row tiles ma, ma + 1)
+
+// Stream-K bookkeeping shared by the kernel and the host plan: row tile m
+// owns units [m nst, (m + 1) nst); CTA c owns [c len, (c + 1) len).
+struct TcSplit {
+    int nst, len;
+    __host__ __device__ int first_cta(int m) const { return (m * nst) / len; }
+    __host__ __device__ int segments(int m) const { return ((m + 1) * nst - 1) / len - first_cta(m) + 1; }
+};
 constexpr int kCodeAhead = 4;             // code chunks requested this many stages ahead
 
-template <class S>
+template <class S, bool kSK>
 __global__ void __launch_bounds__(kTcThreads)
 gemv_tc_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restrict__ cb,
                const uint16_t *__restrict__ scales, const uint16_t *__restrict__ x, int batch,
-               uint16_t *__restrict__ y, SplitK sk, void *ws, int stages_per_split)
+               uint16_t *__restrict__ y, SplitK sk, void *ws, int len)
 {
     constexpr int R = TcRing<S>::depth, LAG = TcRing<S>::lag;
     extern __shared__ uint8_t smem_raw[];
@@ -351,11 +407,29 @@ gemv_tc_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restri
     uint32_t *abort_flag = tmem_slot + 1;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int m0 = blockIdx.x * kTcBM;
-    const int nst = (L.G + 7) / 8;  // 64-feature stages
-    const int s0 = blockIdx.y * stages_per_split;
-    const int s1 = min(nst, s0 + stages_per_split);
-    const int nloc = max(0, s1 - s0);
+    const int nst = (L.G + 7) / 8;  // 64-feature stages per row tile
+    const TcSplit split{nst, len};
+    const int mtiles = (L.out + kTcBM - 1) / kTcBM;
+    int ma, sa, nloc, brk;  // first row tile, its first stage, stages, local stage of row tile ma + 1
+    if constexpr (kSK) {
+        const int u0 = blockIdx.x * len;
+        nloc = min(len, mtiles * nst - u0);  // >= 1: the grid ends at the last unit
+        ma = u0 / nst;
+        sa = u0 - ma * nst;
+        brk = nst - sa;
+    } else {
+        ma = blockIdx.x;
+        sa = blockIdx.y * len;
+        nloc = min(len, nst - sa);  // >= 1: the grid ends at the last split
+        brk = nloc;
+    }
+    const int nseg = (kSK && brk < nloc) ? 2 : 1;
+    // row tile and stage of local stage i
+    auto tile_of = [&](int i) { return (kSK && i >= brk) ? ma + 1 : ma; };
+    auto stage_of = [&](int i) { return (kSK && i >= brk) ? i - brk : sa + i; };
+    // partial-sum slots of row tile m, and this CTA's slot
+    auto segments = [&](int m) { return kSK ? split.segments(m) : (int)gridDim.y; };
+    auto slot_of = [&](int m) { return kSK ? (int)blockIdx.x - split.first_cta(m) : (int)blockIdx.y; };
     const bool x_direct = (batch == 16 || batch == 8);
 
     if (S::B == 16 && tid == 0) prefetch_table_share(cb, (uint32_t)S::K * 65536u * 16u);
@@ -382,15 +456,15 @@ gemv_tc_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restri
 
     if (warp < kTcDecoders / 32) {
         // ------------------------------ decoders ------------------------------
-        const int rt_l = tid >> 3, gi = tid & 7;  // A role: row tile, group
-        const int rt = (m0 >> 3) + rt_l;
-        const bool rows_live = rt < L.rtiles;
+        const int rt_l = tid >> 3, gi = tid & 7;  // A role: 8-row tile within the 128 rows, group
+        // code chunk of local stage q for this thread, zero past the end
+        auto fetch = [&](int q) {
+            const int rt = tile_of(q) * (kTcBM / 8) + rt_l, g = stage_of(q) * 8 + gi;
+            return load_chunk<S>(packed, (size_t)rt * L.gp + g, q < nloc && rt < L.rtiles && g < L.G);
+        };
         Chunk<S> code_ring[kCodeAhead];
 #pragma unroll
-        for (int q = 0; q < kCodeAhead; ++q) {
-            const int g = (s0 + q) * 8 + gi;
-            code_ring[q] = load_chunk<S>(packed, (size_t)rt * L.gp + g, q < nloc && rows_live && g < L.G);
-        }
+        for (int q = 0; q < kCodeAhead; ++q) code_ring[q] = fetch(q);
         // 1x16 decoders touch weights only (codes, codebook): they do not
         // wait for the previous launch on the stream, so their gathers may
         // overlap its end (the MMA warp waits before it loads x, and every
@@ -400,6 +474,7 @@ gemv_tc_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restri
         grid_launch_dependents();
         const int kr = tid >> 1, hb = tid & 1;  // x role (other schemes): feature row, 8-column half
         bool ok = true;
+        int published = 0;  // this thread has arrived on full[] for stages below this
         // stage loop unrolled by the code-ring depth so every ring index is static
         for (int i0 = 0; ok && i0 < nloc + LAG; i0 += kCodeAhead) {
 #pragma unroll
@@ -407,20 +482,28 @@ gemv_tc_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restri
                 const int i = i0 + u;
                 if (i >= nloc + LAG) break;
                 if (i < nloc) {
-                    const int s = s0 + i, buf = i % R;
-                    // the buffer is free once the MMAs of stage i - R completed
-                    if (i >= R && !mbar_wait_ns(&empty[buf], ((i / R) - 1) & 1, kWaitNs)) *abort_v = 1;
+                    const int s = stage_of(i), buf = i % R;
+                    // the buffer is free once the MMAs of stage i - R completed.
+                    // If they have not, the MMA warp is behind (at the start,
+                    // it waits for the previous launch): publish every stage
+                    // issued so far before blocking, so that it can run them
+                    // back to back once it starts.
+                    if (i >= R) {
+                        const uint32_t par = ((i / R) - 1) & 1;
+                        if (!mbar_test_wait(&empty[buf], par)) {
+                            cp_async_wait<0>();
+                            fence_proxy_async_smem();
+                            for (; published < i; ++published) mbar_arrive(&full[published % R]);
+                            if (!mbar_wait_ns(&empty[buf], par, kWaitNs)) *abort_v = 1;
+                        }
+                    }
                     if (*abort_v) {
                         ok = false;
                         break;
                     }
                     const Chunk<S> code = code_ring[u];
-                    {
-                        const int g = (s + kCodeAhead) * 8 + gi;
-                        code_ring[u] = load_chunk<S>(packed, (size_t)rt * L.gp + g,
-                                                     i + kCodeAhead < nloc && rows_live && g < L.G);
-                    }
-                    const bool live = rows_live && s * 8 + gi < L.G;
+                    code_ring[u] = fetch(i + kCodeAhead);
+                    const bool live = tile_of(i) * (kTcBM / 8) + rt_l < L.rtiles && s * 8 + gi < L.G;
                     uint8_t *A = tileA + buf * kTcTileA;
                     if constexpr (TcRing<S>::kAsyncWeights) {
                         const uint32_t a0 = smem_u32(A);
@@ -476,11 +559,12 @@ gemv_tc_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restri
                 }
                 cp_async_commit();  // one group per iteration (empty in the drain)
                 const int j = i - LAG;
-                if (j >= 0) {
+                if (j >= published) {
                     // this thread's copies of stage j have landed: publish them
                     cp_async_wait<LAG>();
                     fence_proxy_async_smem();
                     mbar_arrive(&full[j % R]);
+                    published = j + 1;
                 }
             }
         }
@@ -490,26 +574,24 @@ gemv_tc_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restri
         if (!got) *abort_v = 1;
         tc_fence_after();
         if (__all_sync(0xffffffffu, got)) {
-            const int row = m0 + warp * 32 + lane;  // TMEM lane quarter = warp
-            float v[16];
-            if (nloc > 0) {
-                tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16), v);
-            } else {
+            for (int e = 0; e < nseg; ++e) {
+                const int m = ma + e;
+                const int row = m * kTcBM + warp * 32 + lane;  // TMEM lane quarter = warp
+                float v[16];
+                tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + 16u * e, v);
+                if (row < L.out) {
+                    if (segments(m) == 1) {
+                        const float sc = scales ? __half2float(__ushort_as_half(scales[row])) : 1.f;
 #pragma unroll
-                for (int n = 0; n < 16; ++n) v[n] = 0.f;
-            }
-            if (row < L.out) {
-                if (gridDim.y == 1) {
-                    const float sc = scales ? __half2float(__ushort_as_half(scales[row])) : 1.f;
+                        for (int n = 0; n < 16; ++n)
+                            if (n < batch)
+                                y[(size_t)row * batch + n] = __half_as_ushort(__float2half_rn(sc * v[n]));
+                    } else {
+                        float *p = sk.partials + ((size_t)slot_of(m) * L.rows8 + row) * batch;
 #pragma unroll
-                    for (int n = 0; n < 16; ++n)
-                        if (n < batch)
-                            y[(size_t)row * batch + n] = __half_as_ushort(__float2half_rn(sc * v[n]));
-                } else {
-                    float *p = sk.partials + (size_t)blockIdx.y * L.rows8 * batch + (size_t)row * batch;
-#pragma unroll
-                    for (int n = 0; n < 16; ++n)
-                        if (n < batch) p[n] = v[n];
+                        for (int n = 0; n < 16; ++n)
+                            if (n < batch) p[n] = v[n];
+                    }
                 }
             }
         }
@@ -523,7 +605,7 @@ gemv_tc_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restri
         if constexpr (kX) grid_dependency_wait();
         const uint32_t idesc = make_idesc(kTcBM, kTcN, true);
         auto load_x = [&](int q) {
-            const int sx = s0 + q, xb = q % RX;
+            const int sx = stage_of(q), xb = q % RX;
             if (x_direct) {
 #pragma unroll
                 for (int c = lane; c < 128; c += 32) {
@@ -593,11 +675,14 @@ gemv_tc_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restri
                 tc_fence_after();
                 const uint32_t a0 = smem_u32(tileA + buf * kTcTileA);
                 const uint32_t b0 = smem_u32(tileB + xb * kTcTileB);
+                // the first stage of each row tile starts its accumulator
+                const uint32_t acc = tmem + ((kSK && j >= brk) ? 16u : 0u);
+                const bool first = (j == 0 || (kSK && j == brk));
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks) {
                     const uint64_t ad = smem_desc_sw128(a0 + ks * 32, 16, 1024);
                     const uint64_t bd = smem_desc(b0 + ks * 512, kTcTileB, 256, kSwizzle32B);
-                    mma_f16_ss(tmem, ad, bd, idesc, (j > 0 || ks > 0) ? 1u : 0u);
+                    mma_f16_ss(acc, ad, bd, idesc, (!first || ks > 0) ? 1u : 0u);
                 }
                 mma_commit(&empty[buf]);                // A buffer free once these MMAs complete
                 if constexpr (kX) mma_commit(&emptyx[xb]);  // and the activation slot
@@ -619,7 +704,12 @@ gemv_tc_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restri
     if (warp == 0) tmem_dealloc(tmem, kTcTmemCols);
     // arrive even after a timeout so the counters stay consistent (the
     // status word already tells the caller the output is incomplete)
-    if (gridDim.y > 1) splitk_finish(L, sk, m0, kTcBM, batch, scales, y);
+    for (int e = 0; e < nseg; ++e) {
+        const int m = ma + e, ns = segments(m);
+        if (ns > 1)
+            splitk_finish(L, sk, m, ns, m * kTcBM, min(kTcBM, L.rows8 - m * kTcBM), batch, scales, y,
+                          reinterpret_cast<float4 *>(tileA), R * kTcTileA);
+    }
 }
 
 }  // namespace aqk
@@ -633,10 +723,13 @@ enum Path { kLut = 1, kTensor = 2 };
 
 struct GemvPlan {
     Path path;
-    int ks;          // splits of the group sum (grid.y)
-    int per_split;   // group blocks (LUT: 1) or 64-feature stages (tensor) per split
+    int ks;          // splits of the group sum (grid.y; 1 for stream-K)
+    int len;         // tensor: stages per CTA
+    bool stream_k;   // tensor: stream-K split (else per row tile)
     int rt_per_cta;  // row tiles per CTA (LUT path)
     int grid_x;
+    int counters;    // arrival counters: LUT row ranges, tensor row tiles
+    int slots;       // partial-sum slots per row range (0: no split-K)
     size_t ws_bytes;
 };
 
@@ -658,7 +751,36 @@ int tc_resident_ctas(const Geom &g)
     return smem > 0 ? std::max(1, (228 * 1024) / (smem + 1024)) : 1;
 }
 
-GemvPlan plan_gemv(const Geom &g, int batch)
+// Shortest stream-K share: below 4 stages a CTA's fixed costs (prologue,
+// pipeline fill and drain, split-K finish) dominate.
+constexpr int kTcMinLen = 4;
+
+// Cost of `ctas` CTAs of `len` stages each, `res` of them resident per SM,
+// in tenths of the time in which an SM running two CTAs advances both by one
+// stage; a model fitted to Llama-2 7B/70B shapes at batch 1..16:
+//  * k >= 2 CTAs on an SM share its codeword-read throughput (k len / 2
+//    periods); a CTA alone on its SM has half the reads in flight and runs
+//    about 1.5x slower per stage;
+//  * every wave of CTAs pays about three stages of prologue, pipeline fill
+//    and drain and split-K finish;
+//  * where the decoders start before the previous launch ends (1x16), fewer
+//    than 32 free CTA slots keep the next launch from starting early in
+//    them, which exposes the fill and drain (about 1.4 + 0.2 batch stages).
+long tc_cost(long ctas, int len, int res, int batch, bool early)
+{
+    const long per_sm = (ctas + kNumSMs - 1) / kNumSMs;
+    const long waves = (per_sm + res - 1) / res;
+    const long k_last = per_sm - (waves - 1) * res;
+    long cost = (waves - 1) * (5L * res * len + 30) + (k_last == 1 ? 15 : 5 * k_last) * (long)len + 30;
+    const long last_wave = ctas - (waves - 1) * res * kNumSMs;
+    if (early && (long)res * kNumSMs - last_wave < 32) cost += 14 + 2 * batch;
+    return cost;
+}
+
+// `cap`: largest workspace the caller can offer (the no-allocation entry
+// point's scratch); the plan lengthens the CTAs' shares until its partial
+// sums fit, down to one row tile per CTA (no partials).
+GemvPlan plan_gemv(const Geom &g, int batch, size_t cap = ~(size_t)0)
 {
     GemvPlan p{};
     if (batch == 1 && g.B == 8 && g.K <= 2) {
@@ -669,37 +791,69 @@ GemvPlan plan_gemv(const Geom &g, int batch)
         const int ranges = max(1, min(g.rtiles, 2 * kNumSMs / g.gblocks));
         p.rt_per_cta = ((g.rtiles + ranges - 1) / ranges + 3) & ~3;  // whole quads of tiles
         p.grid_x = (g.rtiles + p.rt_per_cta - 1) / p.rt_per_cta;
-        p.per_split = 1;
+        p.counters = p.grid_x;
+        p.slots = p.ks > 1 ? p.ks : 0;
     } else {
         p.path = kTensor;
         const int mtiles = (g.out + kTcBM - 1) / kTcBM;
         const int nst = (g.G + 7) / 8;
-        // Split count by a wave model: CTAs of this kernel fit `res` per SM
-        // (shared memory), a CTA costs its stages plus about three stages of
-        // fixed latency (prologue, pipeline fill and drain, split-K finish),
-        // and a partial last wave costs a whole CTA.  At least 8 stages per
-        // split: shorter splits lose more to fill and drain, and their
-        // partial sums grow with the batch (measured on Llama-2 70B shapes).
-        const int slots = tc_resident_ctas(g) * kNumSMs;
-        const int min_stages = 8;
-        int best_ks = 1;
-        long best_cost = -1;
-        for (int ks = 1; ks <= std::max(1, nst / min_stages); ++ks) {
-            const long ctas = (long)mtiles * ks;
-            const long waves = (ctas + slots - 1) / slots;
-            const long cost = waves * ((nst + ks - 1) / ks + 3);
-            if (best_cost < 0 || cost < best_cost) {
-                best_cost = cost;
-                best_ks = ks;
+        const long units = (long)mtiles * nst;
+        const int res = tc_resident_ctas(g);
+        const long slots = (long)res * kNumSMs;
+        const bool early = (g.K == 1 && g.B == 16);  // decoders that do not wait for the previous launch
+        auto ws_of = [&](int nslots) {
+            return kWsHeader + align16(sizeof(unsigned) * (size_t)mtiles) + (size_t)nslots * g.rows8 * batch * sizeof(float);
+        };
+        // per row tile: ks splits of `per` stages (the last may be shorter)
+        long best_pt = -1;
+        p.stream_k = false;
+        p.len = nst;
+        p.ks = 1;
+        for (int ks = 1; ks <= std::max(1, nst / kTcMinLen); ++ks) {
+            const int per = (nst + ks - 1) / ks, kk = (nst + per - 1) / per;
+            if (kk < ks) continue;  // same split as a smaller ks
+            if (kk > 1 && ws_of(kk) > cap) break;
+            const long c = tc_cost((long)mtiles * kk, per, res, batch, early);
+            if (best_pt < 0 || c < best_pt) {
+                best_pt = c;
+                p.len = per;
+                p.ks = kk;
             }
         }
-        p.per_split = (nst + best_ks - 1) / best_ks;
-        p.ks = (nst + p.per_split - 1) / p.per_split;
-        p.grid_x = mtiles;
+        // stream-K: from the share that fills every resident CTA slot in one
+        // wave up to one CTA per SM; a row tile meets at most
+        // ceil((nst - 1) / len) + 1 shares
+        const int lmin = (int)std::min<long>(nst, std::max<long>(kTcMinLen, (units + slots - 1) / slots));
+        const int lmax = (int)std::min<long>(nst, std::max<long>(lmin, (units + kNumSMs - 1) / kNumSMs));
+        auto sk_slots = [&](int len) { return len >= nst ? 0 : (nst - 1 + len - 1) / len + 1; };
+        long best_sk = -1;
+        int sk_len = nst;
+        for (int len = lmin; len <= lmax; ++len) {
+            if (ws_of(sk_slots(len)) > cap) continue;
+            const long c = tc_cost((units + len - 1) / len, len, res, batch, early);
+            if (best_sk < 0 || c < best_sk) {
+                best_sk = c;
+                sk_len = len;
+            }
+        }
+        // stream-K only on a clear predicted gain (the model favours it by
+        // a few percent where the per-tile split measures faster: crossing
+        // row tiles costs what the model does not see)
+        if (best_sk >= 0 && (best_pt < 0 || best_sk * 100 < best_pt * (early ? 95 : 85))) {
+            p.stream_k = true;
+            p.len = sk_len;
+            p.ks = 1;
+            p.slots = sk_slots(sk_len);
+            p.grid_x = (int)((units + sk_len - 1) / sk_len);
+        } else {
+            p.slots = p.ks > 1 ? p.ks : 0;
+            p.grid_x = mtiles;
+        }
+        p.counters = mtiles;
         p.rt_per_cta = kTcBM / 8;
     }
-    p.ws_bytes = kWsHeader + align16(sizeof(unsigned) * (size_t)p.grid_x);
-    if (p.ks > 1) p.ws_bytes += (size_t)p.ks * g.rows8 * batch * sizeof(float);
+    p.ws_bytes = kWsHeader + align16(sizeof(unsigned) * (size_t)p.counters) +
+                 (size_t)p.slots * g.rows8 * batch * sizeof(float);
     return p;
 }
 
@@ -741,16 +895,17 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, int smem, 
 
 size_t gemv_workspace_bytes(const Geom &g, int batch) { return plan_gemv(g, batch).ws_bytes; }
 
-cudaError_t launch_gemv(const Geom &g, const void *packed, const uint16_t *cb,
-                        const uint16_t *scales, const uint16_t *x, int batch, uint16_t *y,
-                        void *ws, cudaStream_t s)
+namespace {
+
+cudaError_t launch_plan(const Geom &g, const GemvPlan &p, const void *packed, const uint16_t *cb,
+                        const uint16_t *scales, const uint16_t *x, int batch, uint16_t *y, void *ws,
+                        cudaStream_t s)
 {
-    const GemvPlan p = plan_gemv(g, batch);
     SplitK sk;
     char *base = reinterpret_cast<char *>(ws);
     sk.counters = reinterpret_cast<unsigned *>(base + kWsHeader);
     sk.partials = reinterpret_cast<float *>(base + kWsHeader +
-                                            align16(sizeof(unsigned) * (size_t)p.grid_x));
+                                            align16(sizeof(unsigned) * (size_t)p.counters));
     const uint8_t *pk = reinterpret_cast<const uint8_t *>(packed);
     const uint4 *c = reinterpret_cast<const uint4 *>(cb);
     const dim3 grid(p.grid_x, p.ks);
@@ -773,14 +928,29 @@ cudaError_t launch_gemv(const Geom &g, const void *packed, const uint16_t *cb,
         e = with_scheme(g, [&](auto sch) {
             using S = decltype(sch);
             const int smem = tc_smem_bytes<S>();
-            cudaError_t r = set_smem(gemv_tc_kernel<S>, smem);
+            if (p.stream_k) {
+                cudaError_t r = set_smem(gemv_tc_kernel<S, true>, smem);
+                if (r != cudaSuccess) return r;
+                return launch_pdl(gemv_tc_kernel<S, true>, dim3(p.grid_x), dim3(kTcThreads), smem, s, g, pk, c,
+                                  scales, x, batch, y, sk, ws, p.len);
+            }
+            cudaError_t r = set_smem(gemv_tc_kernel<S, false>, smem);
             if (r != cudaSuccess) return r;
-            return launch_pdl(gemv_tc_kernel<S>, grid, dim3(kTcThreads), smem, s, g, pk, c, scales, x, batch, y, sk,
-                              ws, p.per_split);
+            return launch_pdl(gemv_tc_kernel<S, false>, dim3(p.grid_x, p.ks), dim3(kTcThreads), smem, s, g, pk, c,
+                              scales, x, batch, y, sk, ws, p.len);
         });
     }
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gemv(const Geom &g, const void *packed, const uint16_t *cb,
+                        const uint16_t *scales, const uint16_t *x, int batch, uint16_t *y,
+                        void *ws, cudaStream_t s)
+{
+    return launch_plan(g, plan_gemv(g, batch), packed, cb, scales, x, batch, y, ws, s);
 }
 
 // ---------------------------------------------------------------------------
@@ -826,7 +996,7 @@ cudaError_t launch_gemv_noalloc(const Geom &g, const void *packed, const uint16_
                                 const uint16_t *scales, const uint16_t *x, int batch, uint16_t *y,
                                 cudaStream_t s, bool *too_large)
 {
-    const GemvPlan p = plan_gemv(g, batch);
+    const GemvPlan p = plan_gemv(g, batch, AQ_GEMV_NOALLOC_SCRATCH_BYTES);
     *too_large = p.ws_bytes > AQ_GEMV_NOALLOC_SCRATCH_BYTES;
     if (*too_large) return cudaSuccess;
     void *scratch = nullptr;
@@ -834,10 +1004,10 @@ cudaError_t launch_gemv_noalloc(const Geom &g, const void *packed, const uint16_
     if (e != cudaSuccess) return e;
     // status word and arrival counters must start at zero; the partials are
     // fully written before they are read
-    const size_t clear = kWsHeader + align16(sizeof(unsigned) * (size_t)p.grid_x);
+    const size_t clear = kWsHeader + align16(sizeof(unsigned) * (size_t)p.counters);
     e = cudaMemsetAsync(scratch, 0, clear, s);
     if (e != cudaSuccess) return e;
-    return launch_gemv(g, packed, cb, scales, x, batch, y, scratch, s);
+    return launch_plan(g, p, packed, cb, scales, x, batch, y, scratch, s);
 }
 
 }  // namespace aqh

@@ -186,8 +186,12 @@ aq_status aq_gemv(const aq_layer_desc *desc, const void *packed, const uint16_t 
  * plugins handed only input and output buffers.  The paper has no
  * counterpart; this is an interface convenience.
  *
- * Same arguments, results and bits as aq_gemv, minus the workspace.  The
- * split-K scratch is a fixed device array inside the library of
+ * Same arguments and results as aq_gemv, minus the workspace.  Where
+ * aq_gemv's split-K partial sums would not fit the scratch, this call splits
+ * the sum more coarsely (on the tensor-core path, down to one CTA per 128
+ * rows), so its y agrees with aq_gemv's within rounding rather than bit for
+ * bit; it is deterministic run to run.  The split-K scratch is a fixed
+ * device array inside the library of
  * AQ_GEMV_NOALLOC_SCRATCH_BYTES bytes, which every GPU that loads the
  * library holds until the process exits.  The call allocates nothing (no
  * cudaMalloc/cudaFree, no allocating library routine); it clears the part
@@ -200,8 +204,10 @@ aq_status aq_gemv(const aq_layer_desc *desc, const void *packed, const uint16_t 
  *    give wrong results.  Serialise them, or use aq_gemv with a workspace
  *    per stream.
  *  - AQ_ERR_WORKSPACE if the layer and batch need more scratch than the
- *    array holds (aq_gemv_workspace_bytes(desc, batch) greater than
- *    AQ_GEMV_NOALLOC_SCRATCH_BYTES); nothing is launched then.
+ *    array holds even at the coarsest split; nothing is launched then.
+ *    Only the batch-1 table path of 8-bit codebooks (one partial sum per
+ *    row and 32-group block) can need that much: it is refused when
+ *    aq_gemv_workspace_bytes(desc, 1) exceeds AQ_GEMV_NOALLOC_SCRATCH_BYTES.
  *  - A bounded wait that gives up inside the kernel cannot be reported (the
  *    status word is internal): use aq_gemv when that report is needed.
  */

@@ -125,6 +125,27 @@ def test_gemv_every_batch(K, B, batch):
     assert_close(y, ref, bound, f"gemv {K}x{B} b{batch}")
 
 
+@pytest.mark.parametrize("batch", [1, 5, 16])
+def test_gemv_stream_k_rows_checked_in_full(batch):
+    """20000 x 1032, 1x16: 157 row tiles of only 17 stages balance badly over
+    the SMs, so the work is split stream-K (shares of 11 stages that run
+    across row-tile boundaries, two TMEM accumulators per CTA); the last row
+    tile is ragged (32 rows) and so is the last stage (one group).  Every
+    output is checked against the oracle."""
+    out, inp = 20000, 1032
+    layer = _layer(out, inp, 1, 16, 4321)
+    desc = aq.LayerDesc.make(out, inp, 1, 16)
+    # a per-tile split would need no partial sums at all for this shape:
+    # partial-sum slots in the workspace mean the stream-K split is in use
+    header_and_counters = 16 + ((4 * ((out + 127) // 128) + 15) // 16) * 16
+    assert aq.aq_gemv_workspace_bytes(desc, batch) > header_and_counters
+    x = make_activations(inp, batch, 313 + batch)
+    dl = DevLayer(layer)
+    y = run_gemv(dl, x)
+    ref, bound = oracle.matmul(layer.codes, layer.codebooks, layer.scales, x, threads=8)
+    assert_close(y, ref, bound, f"stream-K 1x16 {out}x{inp} b{batch}")
+
+
 @pytest.mark.parametrize("K,B", SCHEMES)
 def test_gemv_deterministic_and_workspace_reusable(K, B):
     """Same inputs give the same bits; a workspace reused across calls with
