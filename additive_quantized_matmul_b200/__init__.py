@@ -21,7 +21,8 @@ __all__ = [
     "aq_packed_codes_bytes", "aq_gemv_workspace_bytes", "aq_gemm_workspace_bytes",
     "aq_workspace_status", "aq_selftest_bounded_wait", "aq_pack_codes", "aq_unpack_codes",
     "aq_dequant", "aq_gemv", "aq_gemv_noalloc", "aq_gemm", "aq_param_grad_workspace_bytes",
-    "aq_param_grad", "aq_encode_workspace_bytes", "aq_encode", "EXPORTED_SYMBOLS",
+    "aq_param_grad", "aq_encode_workspace_bytes", "aq_encode", "aq_gather_probe_sink_bytes",
+    "aq_gather_probe", "EXPORTED_SYMBOLS",
     "GEMV_NOALLOC_SCRATCH_BYTES",
 ]
 
@@ -39,6 +40,7 @@ EXPORTED_SYMBOLS = (
     "aq_gemm_workspace_bytes", "aq_workspace_status", "aq_selftest_bounded_wait",
     "aq_pack_codes", "aq_unpack_codes", "aq_dequant", "aq_gemv", "aq_gemv_noalloc", "aq_gemm",
     "aq_param_grad_workspace_bytes", "aq_param_grad", "aq_encode_workspace_bytes", "aq_encode",
+    "aq_gather_probe_sink_bytes", "aq_gather_probe",
 )
 
 # AQ_GEMV_NOALLOC_SCRATCH_BYTES of include/aq.h: the fixed scratch behind
@@ -92,6 +94,8 @@ def _load() -> ctypes.CDLL:
         "aq_param_grad": ([dp, vp, vp, vp, vp, vp, i32, vp, vp, vp, sz, vp], i32),
         "aq_encode_workspace_bytes": ([dp], sz),
         "aq_encode": ([dp, vp, vp, vp, vp, i32, vp, vp, sz, vp], i32),
+        "aq_gather_probe_sink_bytes": ([i32], sz),
+        "aq_gather_probe": ([vp, vp, sz, i32, vp, vp], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -223,3 +227,15 @@ def aq_encode(desc: LayerDesc, w, h, codebooks, codes_in, beam: int, codes_out, 
         workspace_bytes = workspace.numel() * workspace.element_size()
     _check("aq_encode", lib.aq_encode(ctypes.byref(desc), _ptr(w), _ptr(h), _ptr(codebooks), _ptr(codes_in), beam,
                                       _ptr(codes_out), _ptr(workspace), workspace_bytes, _stream(stream)))
+
+
+def aq_gather_probe_sink_bytes(mode: int) -> int:
+    return lib.aq_gather_probe_sink_bytes(mode)
+
+
+def aq_gather_probe(codebook, codes, n: int, mode: int, sink, stream=None) -> None:
+    """Measurement aid: read codebook[codes[i]] for each of the n 16-bit codes
+    (mode 0: from L2 into shared memory as the 1x16 GEMV does; mode 1: from
+    the codebook split over 8-CTA clusters' shared memory); per-thread XOR
+    checksums go to ``sink``."""
+    _check("aq_gather_probe", lib.aq_gather_probe(_ptr(codebook), _ptr(codes), n, mode, _ptr(sink), _stream(stream)))

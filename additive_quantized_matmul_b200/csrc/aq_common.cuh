@@ -264,4 +264,7 @@ size_t encode_workspace_bytes(const aqk::Geom &g);
 cudaError_t launch_encode(const aqk::Geom &g, const uint16_t *w, const float *h, const uint16_t *cb,
                           const void *codes_in, void *codes_out, int beam, void *ws, cudaStream_t s);
 cudaError_t launch_selftest_wait(void *ws, int spin_limit, cudaStream_t s);
+size_t gather_probe_sink_bytes(int mode);
+cudaError_t launch_gather_probe(const uint16_t *codebook, const uint16_t *codes, size_t n, int mode, void *sink,
+                                cudaStream_t s);
 }  // namespace aqh

@@ -1,0 +1,223 @@
+// Codeword-read ceiling of the 1x16 decode-time product (a measurement aid,
+// not part of the product path).
+//
+// The 1x16 GEMV is bound by random 16-byte reads from the 1 MiB codebook
+// (65536 codewords of 8 binary16 weights), one read per code.  These kernels
+// issue the same reads and nothing else, so their time is the ceiling the
+// GEMV is measured against:
+//  * mode 0 (L2, the route of the GEMV's decoders): two CTAs of 128 threads
+//    per SM; per stage each thread takes one 16-byte chunk of 8 codes and
+//    copies their codewords with cp.async into its slots of a 5-stage
+//    shared-memory ring, three stages in flight, then folds the landed
+//    stage into a checksum;
+//  * mode 1 (distributed shared memory): clusters of 8 CTAs, each holding
+//    one eighth of the codebook (128 KiB) in shared memory, loaded once per
+//    launch; every codeword is read from its owner's shared memory with
+//    ld.shared::cluster, a chunk's 8 reads in flight.
+// Each thread XORs every 32-bit word it reads into a 16-byte checksum
+// written to `sink` (so the reads cannot be elided, and a test can compare
+// the XOR of all checksums with the XOR of the codewords the codes select).
+#include "aq_common.cuh"
+#include "tc_common.cuh"
+
+namespace aqk {
+
+constexpr int kProbeThreads = 128;
+constexpr int kProbeRing = 5;   // stages of the shared-memory ring (mode 0)
+constexpr int kProbeLag = 3;    // stages in flight (mode 0)
+constexpr int kClusterCtas = 8;  // mode 1
+constexpr int kSliceWords = 65536 / kClusterCtas;
+
+__device__ __forceinline__ void xor_into(uint4 &a, uint4 v)
+{
+    a.x ^= v.x;
+    a.y ^= v.y;
+    a.z ^= v.z;
+    a.w ^= v.w;
+}
+
+__device__ __forceinline__ uint32_t code_of(uint4 w, int j)
+{
+    const uint32_t u = (j < 2) ? w.x : (j < 4) ? w.y : (j < 6) ? w.z : w.w;
+    return (u >> (16 * (j & 1))) & 0xffffu;
+}
+
+// Chunk q of the n / 8 chunks for thread (CTA c, thread t) at step k:
+// (k * gridDim + c) * blockDim + t, so a warp reads 512 consecutive bytes.
+__global__ void __launch_bounds__(kProbeThreads)
+probe_l2_kernel(const uint4 *__restrict__ cb, const uint4 *__restrict__ chunks, long nchunks, uint4 *sink)
+{
+    extern __shared__ uint4 ring[];  // [kProbeRing][8][kProbeThreads]
+    const int t = threadIdx.x;
+    const long stride = (long)gridDim.x * kProbeThreads;
+    const long first = (long)blockIdx.x * kProbeThreads + t;
+    const int steps = first < nchunks ? (int)((nchunks - 1 - first) / stride + 1) : 0;
+    grid_launch_dependents();
+    uint4 acc = make_uint4(0u, 0u, 0u, 0u);
+    auto slot = [&](int i, int j) { return smem_u32(ring + (((i % kProbeRing) * 8 + j) * kProbeThreads + t)); };
+    for (int i = 0; i < steps + kProbeLag; ++i) {
+        if (i < steps) {
+            const uint4 w = ldg_stream_v4(chunks + first + (long)i * stride);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) cp_async16(slot(i, j), cb + code_of(w, j), 16u);
+        }
+        cp_async_commit();
+        const int d = i - kProbeLag;  // its copies have landed once kProbeLag newer groups are pending
+        if (d >= 0) {
+            cp_async_wait<kProbeLag>();
+            if (d < steps) {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    uint4 v;
+                    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                                 : "r"(slot(d, j)));
+                    xor_into(acc, v);
+                }
+            }
+        }
+    }
+    cp_async_wait<0>();
+    grid_dependency_wait();  // the previous launch on the stream may still write the sink
+    sink[first] = acc;
+}
+
+__device__ __forceinline__ uint32_t cluster_ctarank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_sync_all()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ uint4 ld_peer_shared(uint32_t local_addr, uint32_t rank)
+{
+    uint32_t a;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(local_addr), "r"(rank));
+    uint4 v;
+    asm volatile("ld.shared::cluster.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(a)
+                 : "memory");
+    return v;
+}
+
+__global__ void __launch_bounds__(kProbeThreads)
+probe_dsmem_kernel(const uint4 *__restrict__ cb, const uint4 *__restrict__ chunks, long nchunks, uint4 *sink)
+{
+    extern __shared__ uint4 slice[];  // codewords [rank * kSliceWords, (rank + 1) * kSliceWords)
+    const int t = threadIdx.x;
+    const uint32_t rank = cluster_ctarank();
+    for (int i = t; i < kSliceWords; i += kProbeThreads)
+        cp_async16(smem_u32(slice + i), cb + (size_t)rank * kSliceWords + i, 16u);
+    cp_async_commit();
+    cp_async_wait<0>();
+    cluster_sync_all();  // every slice of the cluster is loaded
+    grid_launch_dependents();
+    const uint32_t base = smem_u32(slice);
+    const long stride = (long)gridDim.x * kProbeThreads;
+    const long first = (long)blockIdx.x * kProbeThreads + t;
+    uint4 acc = make_uint4(0u, 0u, 0u, 0u);
+    for (long q = first; q < nchunks; q += stride) {
+        const uint4 w = ldg_stream_v4(chunks + q);
+        uint4 v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const uint32_t c = code_of(w, j);
+            v[j] = ld_peer_shared(base + (c % kSliceWords) * 16u, c / kSliceWords);
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) xor_into(acc, v[j]);
+    }
+    cluster_sync_all();  // no CTA leaves while another still reads its slice
+    grid_dependency_wait();
+    sink[first] = acc;
+}
+
+}  // namespace aqk
+
+namespace aqh {
+using namespace aqk;
+
+namespace {
+
+int probe_l2_ctas() { return 2 * kNumSMs; }
+
+cudaError_t probe_dsmem_ctas(int *ctas)
+{
+    const int smem = kSliceWords * 16;
+    cudaError_t e = cudaFuncSetAttribute(probe_dsmem_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kClusterCtas;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(kClusterCtas);
+    cfg.blockDim = dim3(kProbeThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int clusters = 0;
+    e = cudaOccupancyMaxActiveClusters(&clusters, (void *)probe_dsmem_kernel, &cfg);
+    if (e != cudaSuccess) return e;
+    *ctas = std::max(1, clusters) * kClusterCtas;
+    return cudaSuccess;
+}
+
+}  // namespace
+
+size_t gather_probe_sink_bytes(int mode)
+{
+    // mode 1 runs at most one CTA per SM (128 KiB of shared memory each)
+    const int ctas = mode == 0 ? probe_l2_ctas() : kNumSMs;
+    return (size_t)ctas * kProbeThreads * sizeof(uint4);
+}
+
+cudaError_t launch_gather_probe(const uint16_t *codebook, const uint16_t *codes, size_t n, int mode, void *sink,
+                                cudaStream_t s)
+{
+    const uint4 *cb = reinterpret_cast<const uint4 *>(codebook);
+    const uint4 *chunks = reinterpret_cast<const uint4 *>(codes);
+    const long nchunks = (long)(n / 8);
+    uint4 *out = reinterpret_cast<uint4 *>(sink);
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.blockDim = dim3(kProbeThreads);
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cudaError_t e;
+    if (mode == 0) {
+        const int smem = kProbeRing * 8 * kProbeThreads * (int)sizeof(uint4);
+        e = cudaFuncSetAttribute(probe_l2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        cfg.gridDim = dim3(probe_l2_ctas());
+        cfg.dynamicSmemBytes = smem;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, probe_l2_kernel, cb, chunks, nchunks, out);
+    } else {
+        int ctas = 0;
+        e = probe_dsmem_ctas(&ctas);
+        if (e != cudaSuccess) return e;
+        ctas = std::min(ctas, kNumSMs / kClusterCtas * kClusterCtas);  // the sink holds one CTA per SM
+        attr[1].id = cudaLaunchAttributeClusterDimension;
+        attr[1].val.clusterDim.x = kClusterCtas;
+        attr[1].val.clusterDim.y = 1;
+        attr[1].val.clusterDim.z = 1;
+        cfg.gridDim = dim3(ctas);
+        cfg.dynamicSmemBytes = kSliceWords * 16;
+        cfg.numAttrs = 2;
+        e = cudaLaunchKernelEx(&cfg, probe_dsmem_kernel, cb, chunks, nchunks, out);
+    }
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+}  // namespace aqh

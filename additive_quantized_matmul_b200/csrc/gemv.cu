@@ -347,9 +347,12 @@ constexpr int kTcDecoders = 128;
 constexpr int kTcThreads = kTcDecoders + 32;
 constexpr int kTcBM = 128;
 constexpr int kTcN = 16;
-// Ring depth and copy lag: 1x16 codewords arrive by cp.async from L2 (deep
-// ring, copies of three stages in flight); the other schemes decode in
-// registers, so only the x copies are asynchronous.
+// Ring depth and copy lag: 1x16 codewords arrive by cp.async from L2 (a
+// 6-stage ring, copies of four stages in flight, which still fits two CTAs
+// per SM beside a 3-slot activation ring: the second CTA is what lets
+// consecutive launches overlap on an SM, worth more than a deeper ring in a
+// lone CTA); the other schemes decode in registers, so only the x copies
+// are asynchronous.
 template <class S> struct TcRing {
     static constexpr bool kAsyncWeights = (S::K == 1 && S::B == 16);
     // 8-bit codebooks of one or two books are held as 8 replicas, replica r
@@ -358,7 +361,7 @@ template <class S> struct TcRing {
     // bank quads whatever their codes (random codes would conflict ~2.5x).
     // Their 64 KiB leave room for a 2-stage ring at two CTAs per SM.
     static constexpr int kReplicas = (S::kBooksInSmem && S::K <= 2) ? 8 : 1;
-    static constexpr int depth = kAsyncWeights ? 5 : (kReplicas > 1 ? 2 : 3), lag = kAsyncWeights ? 3 : 1;
+    static constexpr int depth = kAsyncWeights ? 6 : (kReplicas > 1 ? 2 : 3), lag = kAsyncWeights ? 4 : 1;
     // 1x16: the decoders only gather weights and start before the previous
     // launch ends; the MMA warp waits for it and loads the activations (B
     // tiles, raw x slots) into a ring of their own, xpre stages ahead into
@@ -367,7 +370,7 @@ template <class S> struct TcRing {
     // buffer (their stage period is set by decode, and a shallow x ring on
     // the MMA warp would put the x latency on its path).
     static constexpr bool kXByMma = kAsyncWeights;
-    static constexpr int xring = kXByMma ? 4 : depth, xpre = 2;
+    static constexpr int xring = kXByMma ? 3 : depth, xpre = 2;
 };
 constexpr int kTcTileA = kTcBM * 64 * 2;  // 16 KiB
 constexpr int kTcTileB = 64 * 32;         // 2 KiB: 64 rows x 16 columns

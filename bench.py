@@ -295,6 +295,56 @@ def flops(spec: LayerSpec, n: int) -> int:
     return 2 * spec.out_features * spec.in_features * n
 
 
+def gather_ceiling(aq, units, kernels, stream, reps: int = 5):
+    """Codeword-read ceiling of each 1x16 shape: aq_gather_probe (the same
+    random 16-byte codeword reads as the GEMV, one per code, nothing else)
+    over the same rotated layer copies, captured in a CUDA graph and timed
+    with CUDA events like the GEMV; mode 0 reads from L2 into shared memory
+    as the GEMV's decoders do, mode 1 from the codebook split over 8-CTA
+    clusters' shared memory."""
+    import torch
+    rows, seen = [], set()
+    for u in units:
+        spec = u.get("spec")
+        if spec is None or (spec.num_codebooks, spec.nbits) != (1, 16) or u["tag"] in seen:
+            continue
+        seen.add(u["tag"])
+        n = spec.out_features * spec.in_features // 64 * 8  # the layer's codes, a multiple of 8
+        row = {"layer": u["tag"], "codes": n}
+        for mode, key in ((0, "l2_cp_async"), (1, "dsmem_cluster8")):
+            sink = torch.zeros(aq.aq_gather_probe_sink_bytes(mode) // 4, dtype=torch.int32, device=stream.device)
+
+            def once():
+                for packed, cb, _ in u["copies"]:
+                    aq.aq_gather_probe(cb, packed, n, mode, sink, stream=stream)
+
+            with torch.cuda.stream(stream):
+                once()
+            torch.cuda.synchronize()
+            graph = torch.cuda.CUDAGraph(keep_graph=True)
+            with torch.cuda.graph(graph, stream=stream):
+                once()
+            graph.instantiate()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                graph.replay()
+                e0.record(stream)
+                for _ in range(reps):
+                    graph.replay()
+                e1.record(stream)
+            torch.cuda.synchronize()
+            us = 1e3 * e0.elapsed_time(e1) / (reps * len(u["copies"]))
+            row[f"{key}_us_per_layer"] = round(us, 3)
+            row[f"{key}_gathers_per_s"] = round(n / (us * 1e-6), -6)
+            del graph
+        for k in kernels:
+            if k["layer"] == u["tag"] and "us_per_layer" in k:
+                row[f"gemv_n{k['n']}_us"] = k["us_per_layer"]
+                row[f"gemv_n{k['n']}_frac_of_ceiling"] = round(row["l2_cp_async_us_per_layer"] / k["us_per_layer"], 3)
+        rows.append(row)
+    return rows or None
+
+
 def run_gpu(args) -> None:
     import torch
 
@@ -490,6 +540,12 @@ def run_gpu(args) -> None:
     for k in kernels:
         del k["total_us"]
 
+    # ---- codeword-read ceiling of the 1x16 shapes (secondary bound) ----------
+    if op == "gemv" and not args.skip_ceiling:
+        ceiling = gather_ceiling(aq, units, kernels, stream)
+        if ceiling:
+            roofline["gather_ceiling"] = ceiling
+
     # ---- end-to-end through the public API with host buffers ----------------
     e2e = None
     if not args.skip_e2e and op not in ("grad", "encode"):  # the gradient's outputs are parameters, not a per-step result
@@ -570,6 +626,8 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--skip-ceiling", action="store_true",
+                    help="do not time the 1x16 codeword-read ceiling (aq_gather_probe)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=WORKLOAD,
                     help="llama2-7b-1x16 (default), llama2-7b-mlp-2x8, llama2-70b-1x16, "

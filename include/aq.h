@@ -290,6 +290,36 @@ aq_status aq_param_grad(const aq_layer_desc *desc, const void *packed, const uin
                         float *grad_scales, float *grad_codebooks, void *workspace,
                         size_t workspace_bytes, aq_stream_t stream);
 
+/*
+ * Measurement aid, not part of the product path: the codeword-read ceiling
+ * of the 1x16 decode-time product.  A 1x16 layer decodes each code by
+ * reading its 16-byte codeword from the 1 MiB codebook (the paper's 1x16
+ * scheme: one codebook of 2^16 vectors of 8 weights); at decode batch
+ * sizes these random reads, not HBM, bound aq_gemv.  aq_gather_probe
+ * issues the same reads and nothing else, one per code:
+ *   mode 0  from L2 into shared memory with cp.async, as aq_gemv's
+ *           decoders do (two CTAs per SM, three stages in flight);
+ *   mode 1  from the codebook split over the shared memory of 8-CTA
+ *           thread-block clusters (128 KiB per CTA, loaded once per call)
+ *           with distributed shared-memory loads.
+ *   codebook  [65536][8] binary16, device, 16-byte aligned,
+ *   codes     n 16-bit codes, device, 16-byte aligned, n a multiple of 8
+ *             (a 1x16 layer's packed codes are such an array),
+ *   sink      device, >= aq_gather_probe_sink_bytes(mode) bytes, 16-byte
+ *             aligned: receives 16-byte checksums, one per thread (the XOR
+ *             of every 32-bit word it read); the XOR of all of them equals
+ *             the XOR of codebook[codes[i]] over every i, if the sink was
+ *             zero-filled first (threads without codes write zeros).
+ * Asynchronous on `stream`, launched with programmatic stream
+ * serialisation like aq_gemv, so back-to-back calls overlap the same way.
+ * AQ_ERR_INVALID_ARG for another mode, null pointers, n = 0 or n not a
+ * multiple of 8 (aq_gather_probe_sink_bytes returns 0 for another mode);
+ * AQ_ERR_MISALIGNED for a pointer off a 16-byte boundary.
+ */
+size_t aq_gather_probe_sink_bytes(int mode);
+aq_status aq_gather_probe(const uint16_t *codebook, const uint16_t *codes, size_t n, int mode, void *sink,
+                          aq_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -208,3 +208,17 @@ def test_encode_argument_errors():
     assert call(desc=aq.LayerDesc.make(64, 256, 1, 16)) == 2   # 16-bit codes: not run
     assert aq.aq_encode_workspace_bytes(aq.LayerDesc.make(64, 256, 1, 16)) == 0
     assert call(desc=aq.LayerDesc.make(64, 16392, 2, 8)) == 1   # in > 16384
+
+
+def test_gather_probe_argument_errors():
+    f = aq.lib.aq_gather_probe
+    assert aq.aq_gather_probe_sink_bytes(0) > 0 and aq.aq_gather_probe_sink_bytes(1) > 0
+    assert aq.aq_gather_probe_sink_bytes(2) == 0
+    assert f(FAKE, FAKE, 64, 2, FAKE, None) == 1       # unknown mode
+    assert f(FAKE, FAKE, 0, 0, FAKE, None) == 1        # no codes
+    assert f(FAKE, FAKE, 12, 0, FAKE, None) == 1       # n not a multiple of 8
+    assert f(None, FAKE, 64, 0, FAKE, None) == 1
+    assert f(FAKE, None, 64, 1, FAKE, None) == 1
+    assert f(FAKE, FAKE, 64, 0, None, None) == 1
+    assert f(FAKE + 8, FAKE, 64, 0, FAKE, None) == 3   # misaligned codebook
+    assert f(FAKE, FAKE + 2, 64, 1, FAKE, None) == 3   # misaligned codes
