@@ -129,10 +129,12 @@ __device__ __forceinline__ void splitk_finish(const Geom &L, SplitK sk, int coun
 // 2x8, batch 1: per-group codebook x activation lookup tables.
 //
 // For one block of 32 groups the CTA tabulates L_k[g][c] = <C_k[c], x_g> for
-// both codebooks (2 x 256 x 32 fp32 = 64 KiB of shared memory), laid out
-// lane-private: entry (k, c, g) at word (k*256 + c)*32 + g, so lane l
-// (group 32*gb + l) always reads bank l and random codes never conflict.
-// A row's contribution from the block is then two table reads per group.
+// both codebooks (256 x 64 fp32 words = 64 KiB of shared memory), laid out
+// lane-private: entry (k, c, g) at word c*64 + k*32 + g, so lane l (group
+// 32*gb + l) always reads bank l and random codes never conflict.  A row's
+// contribution from the block is then two table reads per group; the byte
+// offset of a read, c*256 + l*4, is one byte permute of the code byte and
+// l*4 (the k*128 goes into the load's immediate).
 //
 // The tables are one small matrix product, T[g][k*256 + c] =
 // sum_j x_g[j] C_k[c][j] (32 x 512, inner size 8), computed with
@@ -150,6 +152,20 @@ __device__ __forceinline__ void splitk_finish(const Geom &L, SplitK sk, int coun
 // CTA waits on the previous launch.
 // ---------------------------------------------------------------------------
 constexpr int kLutWarps = 8;
+constexpr int kLutBytes = 256 * 64 * 4;  // the tables: 256 codes x 64 words
+
+// Byte offset c*256 + lane4 of the table entry of code (r, k) of a chunk (8-bit
+// codes: code (r, k) is byte r*K + k of the chunk) by one byte permute: the
+// code byte goes to byte 1, lane4 (the lane's word offset, < 256) to byte 0.
+template <class S>
+__device__ __forceinline__ uint32_t lut_offset(const Chunk<S> &c, int r, int k, uint32_t lane4)
+{
+    const int bi = r * S::K + k;
+    const uint32_t sel = 0x5504u | ((uint32_t)(bi & 3) << 4);
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(c.w[bi >> 2]), "r"(lane4), "r"(sel));
+    return d;
+}
 constexpr int kLutRing = 2;  // quads of code chunks (4 row tiles) in flight per warp
 
 // Reduce-scatter of 32 values per lane over the warp: lane l returns the
@@ -195,7 +211,7 @@ gemv_lut_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restr
 {
     static_assert(S::B == 8 && S::K <= 2, "tables for one or two 8-bit codebooks");
     constexpr int K = S::K;
-    extern __shared__ float lut[];       // [K][256][32] tables
+    extern __shared__ float lut[];       // [256][64] tables: word c*64 + k*32 + g
     __shared__ uint4 scb[K * 256];       // the codebooks, binary16, row k*256 + c
     __shared__ uint4 xs[32];             // activations of the block's 32 groups
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -239,8 +255,8 @@ gemv_lut_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restr
             a[m][0] = xw[(16 * m + gid) * 4 + t4];
             a[m][1] = xw[(16 * m + gid + 8) * 4 + t4];
         }
-        const int kc0 = warp * 32 * K;
-        float *dst = lut + (kc0 + 2 * t4) * 32 + gid;
+        const int kc0 = warp * 32 * K;  // codeword k*256 + c: this warp's all share one k
+        float *dst = lut + ((kc0 & 255) + 2 * t4) * 64 + (kc0 >> 8) * 32 + gid;
         int off[4];
 #pragma unroll
         for (int s = 0; s < 4; ++s) off[s] = 8 * ((t4 + s) & 3);
@@ -261,12 +277,13 @@ gemv_lut_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restr
                 for (int s = 0; s < 4; ++s) w[s] = (t4 & 2) ? r[(s + 2) & 3] : r[s];
                 // w[s] = v[(t4 + s) & 3]: slot s writes group gid + off[s]
 #pragma unroll
-                for (int s = 0; s < 4; ++s) dst[n * 256 + b * 32 + off[s]] = w[s];
+                for (int s = 0; s < 4; ++s) dst[n * 512 + b * 64 + off[s]] = w[s];
             }
         }
     }
     __syncthreads();
-    const float *lutl = lut + lane;  // table k at lutl + k * 256 * 32
+    const char *lutb = reinterpret_cast<const char *>(lut);
+    const uint32_t lane4 = lane * 4;
     float *part = sk.partials + (size_t)gb * L.rows8;
     for (int j0 = 0; j0 < nq; j0 += kLutRing) {
 #pragma unroll
@@ -278,9 +295,10 @@ gemv_lut_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restr
             for (int t = 0; t < 4; ++t)
 #pragma unroll
                 for (int r = 0; r < 8; ++r) {
-                    float a = lutl[ring[i][t].code(r, 0) * 32];
+                    float a = *reinterpret_cast<const float *>(lutb + lut_offset<S>(ring[i][t], r, 0, lane4));
 #pragma unroll
-                    for (int k = 1; k < K; ++k) a += lutl[(k * 256 + ring[i][t].code(r, k)) * 32];
+                    for (int k = 1; k < K; ++k)
+                        a += *reinterpret_cast<const float *>(lutb + lut_offset<S>(ring[i][t], r, k, lane4) + k * 128);
                     acc[8 * t + r] = a;
                 }
             const int jn = j + kLutRing;
@@ -914,7 +932,7 @@ cudaError_t launch_plan(const Geom &g, const GemvPlan &p, const void *packed, co
     const dim3 grid(p.grid_x, p.ks);
     cudaError_t e = cudaSuccess;
     if (p.path == kLut) {
-        const int smem = g.K * 256 * 32 * (int)sizeof(float);  // the tables
+        const int smem = kLutBytes;  // the tables
         auto lut = [&](auto sch) {
             using S = decltype(sch);
             if constexpr (S::B == 8 && S::K <= 2) {
