@@ -214,14 +214,26 @@ gemm_tc_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restri
 // 32 KiB of 8x8 codebooks share the shared memory; 2 stages of (16 + 64 KiB)
 // for BN = 512.
 template <class S, int BN>
-constexpr int kWsStagesOf = (BN == 512) ? 2 : (S::kSmemBookBytes > 8192) ? 3 : 4;
+constexpr int kWsStagesOf = (BN == 512) ? 2 : (S::kSmemBookBytes > 8192 || (S::K == 1 && S::B == 16)) ? 3 : 4;
 // The W (decoded) tiles have a ring of their own, 5 deep (4 with the 32 KiB
 // of 8x8 codebooks): with 512-token X tiles taking 64 KiB a stage, a shared
-// ring would be 2 deep and leave the 1x16 gathers a copy lag of 1 (about
-// 2000 codewords in flight per CTA); lag 3 here, 4000 in flight.
+// ring would be 2 deep.  The 1x16 decoders (two groups of 128 threads, two
+// of each group's stages in flight: about 4000 codeword reads per CTA) need
+// the depth; at 256-token tiles 1x16 trades an X stage for two W stages
+// (6 W, 3 X).
 template <class S, int BN>
-constexpr int kWsAStagesOf = (BN == 512) ? ((S::kSmemBookBytes > 8192) ? 4 : 5) : kWsStagesOf<S, BN>;
-constexpr int kWsThreads = 192;               // 6 warps
+constexpr int kWsAStagesOf = (BN == 512) ? ((S::kSmemBookBytes > 8192) ? 4 : 5)
+                                         : ((S::K == 1 && S::B == 16) ? 6 : kWsStagesOf<S, BN>);
+// Decoder groups of 4 warps taking alternate stages: one CTA per SM (the X
+// tiles fill its shared memory), so the decode rate per SM is that of its
+// decoders; with one or two codebooks two groups run (twice the 1x16
+// codeword reads in flight; twice the shared-memory decode of 8-bit codes:
+// at 512 tokens 20 % faster for both), eight 8-bit codebooks keep one (their
+// registers).
+template <class S>
+constexpr int kWsGroupsOf = (S::K <= 2) ? 2 : 1;
+template <class S>
+constexpr int kWsThreadsOf = 64 + 128 * kWsGroupsOf<S>;  // X producer, MMA issuer, decoders
 constexpr int kWsLag = 2;                     // cp.async stages in flight per decoder (< ring depth)
 
 struct GemmSplit {
@@ -297,7 +309,7 @@ __device__ __forceinline__ void gemm_split_finish(const Geom &L, GemmSplit sp, i
 }
 
 template <class S, int BN>
-__global__ void __launch_bounds__(kWsThreads, 1)
+__global__ void __launch_bounds__(kWsThreadsOf<S>, 1)
 gemm_ws_kernel(const __grid_constant__ CUtensorMap xmap, Geom L, const uint8_t *__restrict__ packed,
                const uint4 *__restrict__ cb, const uint16_t *__restrict__ scales, int T,
                uint16_t *__restrict__ y, void *ws, GemmSplit sp, int stages_per_split)
@@ -333,7 +345,7 @@ gemm_ws_kernel(const __grid_constant__ CUtensorMap xmap, Geom L, const uint8_t *
     constexpr bool kAsyncWeights = (S::K == 1 && S::B == 16);
     if (S::B == 16 && tid == 0) prefetch_table_share(cb, (uint32_t)S::K * 65536u * 16u);
     if constexpr (S::kBooksInSmem)
-        for (int i = tid; i < S::K * 256; i += kWsThreads) scb[i] = cb[i];
+        for (int i = tid; i < S::K * 256; i += kWsThreadsOf<S>) scb[i] = cb[i];
     if (tid == 0) {
         for (int s = 0; s < kWsAStages; ++s) {
             mbar_init(&full_a[s], 128);
@@ -404,7 +416,12 @@ gemm_ws_kernel(const __grid_constant__ CUtensorMap xmap, Geom L, const uint8_t *
         }
     } else {
         // ---------------- decoders ----------------
-        const int t = tid - 64;  // 0..127
+        // group dg takes stages dg, dg + NG, dg + 2 NG, ... (its own stage k
+        // is stage dg + NG k); group 0 also runs the epilogue
+        constexpr int NG = kWsGroupsOf<S>;
+        const int dg = (tid - 64) / 128;
+        const int t = (tid - 64) % 128;
+        const int nown = (nk - dg + NG - 1) / NG;
         const int rt_l = t >> 3, gi = t & 7;
         const int rt = (m0 >> 3) + rt_l;
         const bool rows_live = rt < L.rtiles;
@@ -413,25 +430,41 @@ gemm_ws_kernel(const __grid_constant__ CUtensorMap xmap, Geom L, const uint8_t *
         constexpr int kCodeAhead = 4;
         Chunk<S> code_ring[kCodeAhead];
 #pragma unroll
-        for (int q = 0; q < kCodeAhead; ++q)
-            code_ring[q] = load_chunk<S>(packed, (size_t)rt * L.gp + g0 + q * 8 + gi,
-                                         q < nk && rows_live && g0 + q * 8 + gi < L.G);
+        for (int q = 0; q < kCodeAhead; ++q) {
+            const int sq = dg + NG * q;
+            code_ring[q] = load_chunk<S>(packed, (size_t)rt * L.gp + g0 + sq * 8 + gi,
+                                         sq < nk && rows_live && g0 + sq * 8 + gi < L.G);
+        }
         // copies of kLag stages stay in flight; a stage is published kLag
         // iterations after it is issued, so kLag must stay below the ring
         // depth (the decoder waits for the MMAs of stage s - depth first)
-        constexpr int kLag = !kAsyncWeights ? 0 : (BN == 512 ? 3 : (kWsLag < kWsAStages - 1 ? kWsLag : kWsAStages - 1));
-        static_assert(kLag < kWsAStages - 1 || !kAsyncWeights, "copy lag must leave the MMAs a stage of slack");
+        // (with NG groups a lag of kLag own stages spans NG kLag stages of the ring)
+        constexpr int kLag = !kAsyncWeights ? 0 : kWsLag;
+        static_assert(NG * kLag < kWsAStages || !kAsyncWeights, "copy lag must leave the MMAs a stage of slack");
         bool ok = true;
+        int published = 0;  // own stages below this have been arrived on full_a[]
         // unrolled by the ring depth so every ring index is static
-        for (int s0i = 0; ok && s0i < nk + kLag; s0i += kCodeAhead) {
+        for (int k0 = 0; ok && k0 < nown + kLag; k0 += kCodeAhead) {
 #pragma unroll
             for (int u = 0; u < kCodeAhead; ++u) {
-                const int s = s0i + u;
-                if (s >= nk + kLag) break;
-                if (s < nk) {
+                const int k = k0 + u, s = dg + NG * k;  // own stage, stage
+                if (k >= nown + kLag) break;
+                if (k < nown) {
                     const int buf = s % kWsAStages;
-                    if (s >= kWsAStages && !mbar_wait_ns(&empty_a[buf], ((s / kWsAStages) - 1) & 1, kWaitNs)) {
-                        *abort_v = 1;
+                    // the buffer is free once the MMAs of stage s - depth
+                    // completed; before blocking on it, publish every stage
+                    // this thread has issued (the MMAs may need them first)
+                    if (s >= kWsAStages) {
+                        const uint32_t par = ((s / kWsAStages) - 1) & 1;
+                        if (!mbar_test_wait(&empty_a[buf], par)) {
+                            if constexpr (kAsyncWeights) {
+                                cp_async_wait<0>();
+                                fence_proxy_async_smem();
+                                for (; published < k; ++published)
+                                    mbar_arrive(&full_a[(dg + NG * published) % kWsAStages]);
+                            }
+                            if (!mbar_wait_ns(&empty_a[buf], par, kWaitNs)) *abort_v = 1;
+                        }
                     }
                     if (*abort_v) {
                         ok = false;
@@ -440,9 +473,9 @@ gemm_ws_kernel(const __grid_constant__ CUtensorMap xmap, Geom L, const uint8_t *
                     const Chunk<S> code = code_ring[u];
                     const bool live = rows_live && g0 + s * 8 + gi < L.G;
                     {
-                        const int g = g0 + (s + kCodeAhead) * 8 + gi;
-                        code_ring[u] = load_chunk<S>(packed, (size_t)rt * L.gp + g,
-                                                     s + kCodeAhead < nk && rows_live && g < L.G);
+                        const int sn = s + NG * kCodeAhead;
+                        const int g = g0 + sn * 8 + gi;
+                        code_ring[u] = load_chunk<S>(packed, (size_t)rt * L.gp + g, sn < nk && rows_live && g < L.G);
                     }
                     uint8_t *A = tileA + buf * kTileABytes;
                     if constexpr (kAsyncWeights) {
@@ -473,11 +506,12 @@ gemm_ws_kernel(const __grid_constant__ CUtensorMap xmap, Geom L, const uint8_t *
                 }
                 if constexpr (kAsyncWeights) {
                     cp_async_commit();
-                    const int j = s - kLag;
-                    if (j >= 0) {
+                    const int j = k - kLag;  // own stage whose copies have landed
+                    if (j >= published) {
                         cp_async_wait<kLag>();
                         fence_proxy_async_smem();
-                        mbar_arrive(&full_a[j % kWsAStages]);
+                        mbar_arrive(&full_a[(dg + NG * j) % kWsAStages]);
+                        published = j + 1;
                     }
                 } else {
                     fence_proxy_async_smem();
@@ -494,7 +528,7 @@ gemm_ws_kernel(const __grid_constant__ CUtensorMap xmap, Geom L, const uint8_t *
         // this point by a role that gave up, or just above by a lane whose
         // wait failed (then its warp-mates see it through the ballot)
         const bool warp_ok = __all_sync(0xffffffffu, got);
-        if (warp_ok) {
+        if (warp_ok && dg == 0) {
             const int q = warp & 3;  // TMEM lane quarter of this warp
             const int row = m0 + q * 32 + lane;
             const float sc = (row < L.out && scales) ? __half2float(__ushort_as_half(scales[row])) : 1.f;
@@ -665,7 +699,7 @@ cudaError_t launch_gemm(const Geom &g, const void *packed, const uint16_t *cb,
             cudaError_t e = cudaFuncSetAttribute(gemm_ws_kernel<S, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                  smem);
             if (e != cudaSuccess) return e;
-            gemm_ws_kernel<S, BN><<<grid, kWsThreads, smem, s>>>(map, g, pk, c, scales, T, y, ws, sp, p.per_split);
+            gemm_ws_kernel<S, BN><<<grid, kWsThreadsOf<S>, smem, s>>>(map, g, pk, c, scales, T, y, ws, sp, p.per_split);
             return cudaGetLastError();
         };
         return with_scheme(g, [&](auto sch) {
