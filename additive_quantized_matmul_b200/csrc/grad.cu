@@ -200,19 +200,32 @@ param_grad_kernel(const __grid_constant__ CUtensorMap gymap, const __grid_consta
         int lt = 0;
         for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++lt) {
             const int ab = lt & 1;
+            const int m0 = (t / ntn) * kGradBM, n0 = (t % ntn) * kGradBN;
+            const int o = m0 + qd * 32 + lane;
+            const bool row_ok = o < L.out;
+            // 8-bit codebooks with private accumulators: this row's codes of
+            // the tile's 16 groups are requested before the accumulator is
+            // waited for (they do not depend on it), so the scatter rounds of
+            // the slices below do not each wait on an L2 round trip; the
+            // other schemes read them slice by slice (measured faster there)
+            constexpr bool kPrefetch = kGradPrivateAcc<S>;
+            uint64_t words[kGradBN / 8];
+            if constexpr (kPrefetch) {
+#pragma unroll
+                for (int q = 0; q < kGradBN / 8; ++q) {
+                    const int g = n0 / 8 + q;
+                    words[q] = (row_ok && g < L.G) ? load_word<S>(L, packed, o, g) : 0ull;
+                }
+            }
             const bool got = (*abort_v == 0) && mbar_wait_ns(&acc_full[ab], (lt >> 1) & 1, kWaitNs);
             if (!got) *abort_v = 1;
             // tcgen05.ld is warp-collective: a failed wait in any lane ends the warp
             if (!__all_sync(0xffffffffu, got)) break;
             tc_fence_after();
-            const int m0 = (t / ntn) * kGradBM, n0 = (t % ntn) * kGradBN;
-            const int o = m0 + qd * 32 + lane;
-            const bool row_ok = o < L.out;
             const float so = (row_ok && scales) ? __half2float(__ushort_as_half(scales[o])) : 1.f;
             const uint32_t tbase = tmem + (uint32_t)(ab * kGradBN) + ((uint32_t)(qd * 32) << 16);
             float gs = 0.f;
-#pragma unroll 1
-            for (int c0 = 0; c0 < kGradBN; c0 += 16) {
+            auto slice = [&](int c0) {
                 float v[16];
                 tmem_ld16(tbase + c0, v);  // M[o][n0 + c0 .. + 15]: two groups
 #pragma unroll
@@ -220,14 +233,11 @@ param_grad_kernel(const __grid_constant__ CUtensorMap gymap, const __grid_consta
                     const int g = (n0 + c0) / 8 + h;
                     if (g >= L.G) continue;  // the same for the whole warp
                     uint32_t code[S::K];
-                    if (row_ok) {
-                        const uint64_t word = load_word<S>(L, packed, o, g);
+                    uint64_t word = 0;
+                    if constexpr (kPrefetch) word = words[c0 / 8 + h];
+                    else if (row_ok) word = load_word<S>(L, packed, o, g);
 #pragma unroll
-                        for (int k = 0; k < S::K; ++k) code[k] = (uint32_t)(word >> (k * S::B)) & S::kMask;
-                    } else {
-#pragma unroll
-                        for (int k = 0; k < S::K; ++k) code[k] = 0u;
-                    }
+                    for (int k = 0; k < S::K; ++k) code[k] = (uint32_t)(word >> (k * S::B)) & S::kMask;
                     const float *m = v + 8 * h;
                     if (grad_s && row_ok) {
                         uint4 t[S::K];
@@ -282,6 +292,13 @@ param_grad_kernel(const __grid_constant__ CUtensorMap gymap, const __grid_consta
                         }
                     }
                 }
+            };
+            if constexpr (kPrefetch) {
+#pragma unroll
+                for (int c0 = 0; c0 < kGradBN; c0 += 16) slice(c0);
+            } else {
+#pragma unroll 1
+                for (int c0 = 0; c0 < kGradBN; c0 += 16) slice(c0);
             }
             if (row_ok && grad_s) atomicAdd(grad_s + o, gs);
             tc_fence_before();
