@@ -184,17 +184,33 @@ def oracle_sample(rows: int, threads: int, repeats: int = 1):
     return dt, nbytes
 
 
-def cpu_baseline(budget_s: float = 10.0) -> dict:
+def cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def cpu_baseline(budget_s: float = 10.0, single_budget_s: float = 3.0) -> dict:
     import oracle
     threads = os.cpu_count() or 1
     # calibrate on a small sample, then size the measured sample to the budget
     dt, _ = oracle_sample(64, threads)
     rows = int(min(SPEC.out_features, max(64, 64 * budget_s / max(dt, 1e-3))))
     dt, nbytes = oracle_sample(rows, threads)
+    # the same at one thread, on a smaller sample
+    dt1, _ = oracle_sample(8, 1)
+    rows1 = int(min(SPEC.out_features, max(8, 8 * single_budget_s / max(dt1, 1e-3))))
+    dt1, nbytes1 = oracle_sample(rows1, 1)
     return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": min(threads, oracle.max_threads()),
             "kind": "oracle",
             "sample": f"{rows} of {SPEC.out_features} rows of one 4096x4096 1x16 layer at batch "
-                      f"1, 4, 16 (fp64 C oracle, OpenMP over rows), scaled to the layer's bytes"}
+                      f"1, 4, 16 (fp64 C oracle, OpenMP over rows), scaled to the layer's bytes",
+            "single_thread": {"value": nbytes1 / dt1 / 1e9, "sample_rows": rows1},
+            "nproc": threads, "cpu_model": cpu_model()}
 
 
 def run_reference(args) -> None:
