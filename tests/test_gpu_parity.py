@@ -127,16 +127,17 @@ def test_gemv_every_batch(K, B, batch):
 
 @pytest.mark.parametrize("batch", [1, 5, 16])
 def test_gemv_stream_k_rows_checked_in_full(batch):
-    """20000 x 1032, 1x16: 157 row tiles of only 17 stages balance badly over
-    the SMs, so the work is split stream-K (shares of 11 stages that run
-    across row-tile boundaries, two TMEM accumulators per CTA); the last row
-    tile is ragged (32 rows) and so is the last stage (one group).  Every
-    output is checked against the oracle."""
+    """20000 x 1032, 1x16: at batch 5 and 16, 157 row tiles of only 17
+    stages balance badly over the SMs, so the tensor-core path splits the
+    work stream-K (shares that run across row-tile boundaries, two TMEM
+    accumulators per CTA); at batch 1 the CUDA-core path splits the groups
+    five ways.  The last row tile is ragged (32 rows) and so is the last
+    stage (one group).  Every output is checked against the oracle."""
     out, inp = 20000, 1032
     layer = _layer(out, inp, 1, 16, 4321)
     desc = aq.LayerDesc.make(out, inp, 1, 16)
     # a per-tile split would need no partial sums at all for this shape:
-    # partial-sum slots in the workspace mean the stream-K split is in use
+    # partial-sum slots in the workspace mean a split of the sum is in use
     header_and_counters = 16 + ((4 * ((out + 127) // 128) + 15) // 16) * 16
     assert aq.aq_gemv_workspace_bytes(desc, batch) > header_and_counters
     x = make_activations(inp, batch, 313 + batch)
@@ -144,6 +145,22 @@ def test_gemv_stream_k_rows_checked_in_full(batch):
     y = run_gemv(dl, x)
     ref, bound = oracle.matmul(layer.codes, layer.codebooks, layer.scales, x, threads=8)
     assert_close(y, ref, bound, f"stream-K 1x16 {out}x{inp} b{batch}")
+
+
+def test_gemv_cuda_core_path_deterministic_and_reusable():
+    """1x16 at batch 1 on the CUDA cores (4096 x 2048: 16 row ranges, 27
+    group splits finished by the last CTA of each range): same bits twice,
+    correct results with one workspace reused across activations."""
+    layer = _layer(4096, 2048, 1, 16, 17)
+    dl = DevLayer(layer)
+    ws = workspace(aq.aq_gemv_workspace_bytes(dl.desc, 1))
+    x = make_activations(2048, 1, 5)
+    y1 = run_gemv(dl, x, ws)
+    assert np.array_equal(y1, run_gemv(dl, x, ws))
+    for rep in range(3):
+        x2 = make_activations(2048, 1, (rep, 23))
+        ref, bound = oracle.matmul(layer.codes, layer.codebooks, layer.scales, x2, threads=8)
+        assert_close(run_gemv(dl, x2, ws), ref, bound, f"cuda-core 1x16 reuse {rep}")
 
 
 @pytest.mark.parametrize("K,B", SCHEMES)
