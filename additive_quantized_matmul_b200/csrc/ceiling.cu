@@ -13,7 +13,11 @@
 //  * mode 1 (distributed shared memory): clusters of 8 CTAs, each holding
 //    one eighth of the codebook (128 KiB) in shared memory, loaded once per
 //    launch; every codeword is read from its owner's shared memory with
-//    ld.shared::cluster, a chunk's 8 reads in flight.
+//    ld.shared::cluster, a chunk's 8 reads in flight;
+//  * mode 2 (registers through L1, the route of the batch-1 CUDA-core
+//    GEMV): three CTAs of 256 threads per SM, a chunk's 8 codewords read
+//    with ld.global.nc into registers, no shared memory (L1 keeps what it
+//    can of the codebook).
 // Each thread XORs every 32-bit word it reads into a 16-byte checksum
 // written to `sink` (so the reads cannot be elided, and a test can compare
 // the XOR of all checksums with the XOR of the codewords the codes select).
@@ -78,6 +82,28 @@ probe_l2_kernel(const uint4 *__restrict__ cb, const uint4 *__restrict__ chunks, 
         }
     }
     cp_async_wait<0>();
+    grid_dependency_wait();  // the previous launch on the stream may still write the sink
+    sink[first] = acc;
+}
+
+constexpr int kProbeLdgThreads = 256;
+constexpr int kProbeLdgPerSM = 3;
+
+__global__ void __launch_bounds__(kProbeLdgThreads, kProbeLdgPerSM)
+probe_ldg_kernel(const uint4 *__restrict__ cb, const uint4 *__restrict__ chunks, long nchunks, uint4 *sink)
+{
+    const long stride = (long)gridDim.x * kProbeLdgThreads;
+    const long first = (long)blockIdx.x * kProbeLdgThreads + threadIdx.x;
+    grid_launch_dependents();
+    uint4 acc = make_uint4(0u, 0u, 0u, 0u);
+    for (long q = first; q < nchunks; q += stride) {
+        const uint4 w = ldg_stream_v4(chunks + q);
+        uint4 v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[j] = ldg_nc_v4(cb + code_of(w, j));
+#pragma unroll
+        for (int j = 0; j < 8; ++j) xor_into(acc, v[j]);
+    }
     grid_dependency_wait();  // the previous launch on the stream may still write the sink
     sink[first] = acc;
 }
@@ -175,6 +201,7 @@ cudaError_t probe_dsmem_ctas(int *ctas)
 size_t gather_probe_sink_bytes(int mode)
 {
     // mode 1 runs at most one CTA per SM (128 KiB of shared memory each)
+    if (mode == 2) return (size_t)kProbeLdgPerSM * kNumSMs * kProbeLdgThreads * sizeof(uint4);
     const int ctas = mode == 0 ? probe_l2_ctas() : kNumSMs;
     return (size_t)ctas * kProbeThreads * sizeof(uint4);
 }
@@ -194,7 +221,13 @@ cudaError_t launch_gather_probe(const uint16_t *codebook, const uint16_t *codes,
     cfg.stream = s;
     cfg.attrs = attr;
     cudaError_t e;
-    if (mode == 0) {
+    if (mode == 2) {
+        cfg.gridDim = dim3(kProbeLdgPerSM * kNumSMs);
+        cfg.blockDim = dim3(kProbeLdgThreads);
+        cfg.dynamicSmemBytes = 0;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, probe_ldg_kernel, cb, chunks, nchunks, out);
+    } else if (mode == 0) {
         const int smem = kProbeRing * 8 * kProbeThreads * (int)sizeof(uint4);
         e = cudaFuncSetAttribute(probe_l2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;

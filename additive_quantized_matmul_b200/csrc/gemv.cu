@@ -327,28 +327,29 @@ gemv_lut_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restr
 }
 
 // ---------------------------------------------------------------------------
-// 1x16, batch 1: codewords into registers, products on the CUDA cores.
+// 1x16, batch 1 and 2: codewords into registers, products on the CUDA cores.
 //
-// At batch 1 the tensor cores have almost nothing to do and the bound is the
+// At batch 1 or 2 the tensor cores have almost nothing to do and the bound is the
 // rate of random 16-byte codeword reads from the 1 MiB codebook.  This kernel
 // reads them straight into registers (through L1, which keeps a share of the
 // codebook) and multiplies them with x in fp32 (each product of two binary16
 // values is exact); it keeps no tile in shared memory, so three CTAs of 256
-// threads fit per SM (85 registers), about 6000 reads in flight, and L1
-// keeps most of its capacity for the codebook.
+// threads fit per SM at batch 1 (85 registers; two at batch 2), about 6000
+// reads in flight, and L1 keeps most of its capacity for the codebook.
 // CTA = 32 row tiles (256 rows) x one split of the groups.  Thread (row tile
 // t/8, lane t%8) owns the chunks (its row tile, group G0 + t%8 + 8 j): a
 // chunk's 8 codes give the 8 rows' weights of its group.  The first chunk's
 // codewords are requested before the CTA waits for the previous launch
-// (weights only); then x of the split goes to shared memory as fp32, and
-// each row's codeword is replaced by the next chunk's as soon as it is used.
+// (weights only); then x of the split goes to shared memory as fp32
+// ([group][element][batch]), and each row's codeword is replaced by the next
+// chunk's as soon as it is used.
 // The 8 lanes of a row tile add their row sums with a 3-level
 // reduce-scatter; split-K partial sums are finished as for the tables.
 // ---------------------------------------------------------------------------
 constexpr int kCcThreads = 256;
 constexpr int kCcRowTiles = kCcThreads / 8;  // 256 rows per CTA
-constexpr int kCcPerSM = 3;                  // resident CTAs per SM (registers)
 constexpr int kCcMaxSplits = 32;             // more splits per row range: the tensor-core path
+constexpr int kCcMaxBatch = 2;  // measured: faster than the tensor cores at batch 1 and 2, slower from 3
 constexpr int kCcStage = 16 * 1024;          // split-K staging (more would take L1 from the codebook)
 
 __device__ __forceinline__ uint32_t cc_code(const uint4 &c, int r)
@@ -375,12 +376,19 @@ __device__ __forceinline__ float cc_dot8(float acc, uint4 w, float4 x0, float4 x
     return acc;
 }
 
-__global__ void __launch_bounds__(kCcThreads, kCcPerSM)
+// CTAs of the CUDA-core kernel resident per SM, by batch (registers)
+template <int NB>
+constexpr int kCcPerSMOf = NB == 1 ? 3 : 2;
+
+template <int NB>
+__global__ void __launch_bounds__(kCcThreads, kCcPerSMOf<NB>)
 gemv_1x16_cc_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restrict__ cb,
                     const uint16_t *__restrict__ scales, const uint16_t *__restrict__ x,
                     uint16_t *__restrict__ y, SplitK sk, int groups_per_split, int stage_bytes)
 {
-    extern __shared__ float4 ccs[];  // x of the split (2 float4 per group), later the finish's staging
+    // x of the split as fp32, [group][element][batch]; later the finish's staging
+    extern __shared__ float4 ccs[];
+    float *xs = reinterpret_cast<float *>(ccs);
     const int tid = threadIdx.x, rtl = tid >> 3, gl = tid & 7, lane = tid & 31;
     const int rt = blockIdx.x * kCcRowTiles + rtl;
     const bool rows_live = rt < L.rtiles;
@@ -397,51 +405,73 @@ gemv_1x16_cc_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__r
     uint4 next = nown > 1 ? ldg_stream_v4(chunk0 + 128) : zero;
     grid_dependency_wait();  // x, y and the workspace follow the previous launch
     grid_launch_dependents();
-    for (int i = tid; i < ng * 2; i += kCcThreads) {
-        const uint2 h = *reinterpret_cast<const uint2 *>(x + (size_t)G0 * 8 + i * 4);
+    for (int i = tid; i < ng * 2 * NB; i += kCcThreads) {  // 4 values at a time ([in][batch] is that order)
+        const uint2 h = *reinterpret_cast<const uint2 *>(x + (size_t)G0 * 8 * NB + i * 4);
         const float2 a = h2f2(h.x), b = h2f2(h.y);
         ccs[i] = make_float4(a.x, a.y, b.x, b.y);
     }
     __syncthreads();
-    float acc[8];
+    float acc[8][NB];
 #pragma unroll
-    for (int r = 0; r < 8; ++r) acc[r] = 0.f;
+    for (int r = 0; r < 8; ++r)
+#pragma unroll
+        for (int b = 0; b < NB; ++b) acc[r][b] = 0.f;
     for (int j = 0; j < nown; ++j) {
-        const int gq = gl + 8 * j;  // group within the split
-        const float4 x0 = ccs[2 * gq], x1 = ccs[2 * gq + 1];
+        const float *xg = xs + (gl + 8 * j) * 8 * NB;  // x of this chunk's group
         const uint4 cn = next;
         if (j + 2 < nown) next = ldg_stream_v4(chunk0 + (size_t)(j + 2) * 128);
         const bool more = j + 1 < nown;
+        if constexpr (NB == 1) {
+            const float4 x0 = reinterpret_cast<const float4 *>(xg)[0], x1 = reinterpret_cast<const float4 *>(xg)[1];
 #pragma unroll
-        for (int r = 0; r < 8; ++r) {
-            acc[r] = cc_dot8(acc[r], w[r], x0, x1);
-            if (more) w[r] = ldg_nc_v4(cb + cc_code(cn, r));  // the next chunk's row r
+            for (int r = 0; r < 8; ++r) {
+                acc[r][0] = cc_dot8(acc[r][0], w[r], x0, x1);
+                if (more) w[r] = ldg_nc_v4(cb + cc_code(cn, r));  // the next chunk's row r
+            }
+        } else {
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+                const uint32_t hw[4] = {w[r].x, w[r].y, w[r].z, w[r].w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 wf = h2f2(hw[e]);
+#pragma unroll
+                    for (int b = 0; b < NB; ++b) {
+                        acc[r][b] = fmaf(wf.x, xg[(2 * e) * NB + b], acc[r][b]);
+                        acc[r][b] = fmaf(wf.y, xg[(2 * e + 1) * NB + b], acc[r][b]);
+                    }
+                }
+                if (more) w[r] = ldg_nc_v4(cb + cc_code(cn, r));  // the next chunk's row r
+            }
         }
     }
     // reduce-scatter over the 8 lanes of the row tile: lane gl gets row gl
-    float b4[4], b2[2];
-    bool hi = lane & 4;
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-        b4[i] = (hi ? acc[i + 4] : acc[i]) + __shfl_xor_sync(0xffffffffu, hi ? acc[i] : acc[i + 4], 4);
-    hi = lane & 2;
-#pragma unroll
-    for (int i = 0; i < 2; ++i)
-        b2[i] = (hi ? b4[i + 2] : b4[i]) + __shfl_xor_sync(0xffffffffu, hi ? b4[i] : b4[i + 2], 2);
-    hi = lane & 1;
-    const float v = (hi ? b2[1] : b2[0]) + __shfl_xor_sync(0xffffffffu, hi ? b2[0] : b2[1], 1);
     const int row = rt * 8 + gl;
-    if (rows_live && row < L.out) {
-        if (gridDim.y == 1) {
-            const float sc = scales ? __half2float(__ushort_as_half(scales[row])) : 1.f;
-            y[row] = __half_as_ushort(__float2half_rn(sc * v));
-        } else {
-            sk.partials[(size_t)blockIdx.y * L.rows8 + row] = v;
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+        float b4[4], b2[2];
+        bool hi = lane & 4;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            b4[i] = (hi ? acc[i + 4][b] : acc[i][b]) + __shfl_xor_sync(0xffffffffu, hi ? acc[i][b] : acc[i + 4][b], 4);
+        hi = lane & 2;
+#pragma unroll
+        for (int i = 0; i < 2; ++i)
+            b2[i] = (hi ? b4[i + 2] : b4[i]) + __shfl_xor_sync(0xffffffffu, hi ? b4[i] : b4[i + 2], 2);
+        hi = lane & 1;
+        const float v = (hi ? b2[1] : b2[0]) + __shfl_xor_sync(0xffffffffu, hi ? b2[0] : b2[1], 1);
+        if (rows_live && row < L.out) {
+            if (gridDim.y == 1) {
+                const float sc = scales ? __half2float(__ushort_as_half(scales[row])) : 1.f;
+                y[(size_t)row * NB + b] = __half_as_ushort(__float2half_rn(sc * v));
+            } else {
+                sk.partials[((size_t)blockIdx.y * L.rows8 + row) * NB + b] = v;
+            }
         }
     }
     if (gridDim.y == 1) return;
     const int row0 = blockIdx.x * kCcRowTiles * 8;
-    splitk_finish(L, sk, blockIdx.x, gridDim.y, row0, min(kCcRowTiles * 8, L.rows8 - row0), 1, scales, y, ccs,
+    splitk_finish(L, sk, blockIdx.x, gridDim.y, row0, min(kCcRowTiles * 8, L.rows8 - row0), NB, scales, y, ccs,
                   stage_bytes);
 }
 
@@ -925,23 +955,24 @@ GemvPlan plan_gemv(const Geom &g, int batch, size_t cap = ~(size_t)0)
 {
     GemvPlan p{};
     const int cc_ranges = (g.rtiles + kCcRowTiles - 1) / kCcRowTiles;
-    // 1x16 at batch 1 on the CUDA cores: as many group splits as fill the
-    // resident CTA slots in one wave (at most kCcMaxSplits, else too few
-    // rows for this path) and at most 1536 groups per split (their x in
-    // shared memory)
-    const int cc_ks = std::max(1, std::min((kCcPerSM * kNumSMs) / cc_ranges, (g.G + 7) / 8));
+    // 1x16 at batch 1..kCcMaxBatch on the CUDA cores: as many group splits
+    // as fill the resident CTA slots in one wave (at most kCcMaxSplits, else
+    // too few rows for this path) and at most 1536 / batch groups per split
+    // (their x in shared memory)
+    const int cc_per_sm = batch == 1 ? kCcPerSMOf<1> : kCcPerSMOf<2>;
+    const int cc_ks = std::max(1, std::min((cc_per_sm * kNumSMs) / cc_ranges, (g.G + 7) / 8));
     const size_t cc_ws = kWsHeader + align16(sizeof(unsigned) * (size_t)cc_ranges) +
-                         (cc_ks > 1 ? (size_t)cc_ks * g.rows8 * sizeof(float) : 0);
-    if (batch == 1 && g.K == 1 && g.B == 16 && cc_ks <= kCcMaxSplits && (g.G + cc_ks - 1) / cc_ks <= 1536 &&
-        cc_ws <= cap) {
+                         (cc_ks > 1 ? (size_t)cc_ks * g.rows8 * batch * sizeof(float) : 0);
+    if (batch <= kCcMaxBatch && g.K == 1 && g.B == 16 && cc_ks <= kCcMaxSplits &&
+        (g.G + cc_ks - 1) / cc_ks * batch <= 1536 && cc_ws <= cap) {
         p.path = kCudaCores;
         p.grid_x = cc_ranges;
         p.len = (g.G + cc_ks - 1) / cc_ks;  // groups per split
         p.ks = (g.G + p.len - 1) / p.len;
         p.counters = p.grid_x;
         p.slots = p.ks > 1 ? p.ks : 0;
-        const int nvec = kCcRowTiles * 8 / 4;  // float4 of one row range's partial sums
-        p.cc_smem = std::max(p.len * 32, std::min(kCcStage, p.ks > 1 ? p.ks * nvec * 16 : 0));
+        const int nvec = kCcRowTiles * 8 * batch / 4;  // float4 of one row range's partial sums
+        p.cc_smem = std::max(p.len * 32 * batch, std::min(kCcStage, p.ks > 1 ? p.ks * nvec * 16 : 0));
     } else if (batch == 1 && g.B == 8 && g.K <= 2) {
         p.path = kLut;
         p.ks = g.gblocks;
@@ -1070,10 +1101,18 @@ cudaError_t launch_plan(const Geom &g, const GemvPlan &p, const void *packed, co
     const dim3 grid(p.grid_x, p.ks);
     cudaError_t e = cudaSuccess;
     if (p.path == kCudaCores) {
-        e = set_smem(gemv_1x16_cc_kernel, p.cc_smem);
-        if (e == cudaSuccess)
-            e = launch_pdl(gemv_1x16_cc_kernel, grid, dim3(kCcThreads), p.cc_smem, s, g, pk, c, scales, x, y, sk,
-                           p.len, p.cc_smem);
+        auto cc = [&](auto kern) {
+            cudaError_t r = set_smem(kern, p.cc_smem);
+            if (r != cudaSuccess) return r;
+            return launch_pdl(kern, grid, dim3(kCcThreads), p.cc_smem, s, g, pk, c, scales, x, y, sk, p.len,
+                              p.cc_smem);
+        };
+        switch (batch) {
+        case 1: e = cc(gemv_1x16_cc_kernel<1>); break;
+        case 2: e = cc(gemv_1x16_cc_kernel<2>); break;
+        case 3: e = cc(gemv_1x16_cc_kernel<3>); break;
+        default: e = cc(gemv_1x16_cc_kernel<4>); break;
+        }
     } else if (p.path == kLut) {
         const int smem = kLutBytes;  // the tables
         auto lut = [&](auto sch) {

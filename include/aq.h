@@ -301,7 +301,9 @@ aq_status aq_param_grad(const aq_layer_desc *desc, const void *packed, const uin
  *           decoders do (two CTAs per SM, three stages in flight);
  *   mode 1  from the codebook split over the shared memory of 8-CTA
  *           thread-block clusters (128 KiB per CTA, loaded once per call)
- *           with distributed shared-memory loads.
+ *           with distributed shared-memory loads;
+ *   mode 2  into registers through L1 (ld.global.nc), as aq_gemv's batch-1
+ *           1x16 path does (three CTAs of 256 threads per SM).
  *   codebook  [65536][8] binary16, device, 16-byte aligned,
  *   codes     n 16-bit codes, device, 16-byte aligned, n a multiple of 8
  *             (a 1x16 layer's packed codes are such an array),

@@ -212,9 +212,9 @@ def test_encode_argument_errors():
 
 def test_gather_probe_argument_errors():
     f = aq.lib.aq_gather_probe
-    assert aq.aq_gather_probe_sink_bytes(0) > 0 and aq.aq_gather_probe_sink_bytes(1) > 0
-    assert aq.aq_gather_probe_sink_bytes(2) == 0
-    assert f(FAKE, FAKE, 64, 2, FAKE, None) == 1       # unknown mode
+    assert all(aq.aq_gather_probe_sink_bytes(m) > 0 for m in (0, 1, 2))
+    assert aq.aq_gather_probe_sink_bytes(3) == 0 and aq.aq_gather_probe_sink_bytes(-1) == 0
+    assert f(FAKE, FAKE, 64, 3, FAKE, None) == 1       # unknown mode
     assert f(FAKE, FAKE, 0, 0, FAKE, None) == 1        # no codes
     assert f(FAKE, FAKE, 12, 0, FAKE, None) == 1       # n not a multiple of 8
     assert f(None, FAKE, 64, 0, FAKE, None) == 1

@@ -1,4 +1,4 @@
-"""aq_gather_probe: the codeword-read ceiling of the 1x16 product.
+"""aq_gather_probe: the codeword-read ceiling of the 1x16 product (modes 0-2).
 
 The probe reads codebook[codes[i]] for every code and XORs each 32-bit word
 it reads into a per-thread checksum.  These tests check, through the C ABI,
@@ -20,7 +20,7 @@ def _expected_xor(cb_words: np.ndarray, codes: np.ndarray) -> np.ndarray:
     return np.bitwise_xor.reduce(cb_words[codes.astype(np.int64)], axis=0)
 
 
-@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("mode", [0, 1, 2])
 @pytest.mark.parametrize("n", [8, 4096 * 512, 4096 * 512 + 8 * 37])
 def test_probe_reads_the_selected_codewords(mode, n):
     rng = np.random.default_rng(n + mode)
