@@ -500,8 +500,13 @@ def run_gpu(args) -> None:
     t_stop = torch.cuda.Event(enable_timing=True)
     cvd = os.environ.get("CUDA_VISIBLE_DEVICES", "")
     gpu_index = int(cvd.split(",")[local]) if cvd.replace(",", "").isdigit() else local
-    os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
-    sampler = ClockSampler(gpu_index, os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv"))
+    # the raw clock samples go to the CSV named by AQ_CLOCK_LOG ({rank} is
+    # replaced by the rank), if set; the JSON line carries their summary
+    log = os.environ.get("AQ_CLOCK_LOG")
+    if log:
+        log = log.replace("{rank}", str(rank))
+        os.makedirs(os.path.dirname(os.path.abspath(log)), exist_ok=True)
+    sampler = ClockSampler(gpu_index, log)
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()

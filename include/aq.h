@@ -75,7 +75,7 @@ typedef struct CUstream_st *aq_stream_t;
 typedef enum {
     AQ_OK = 0,
     AQ_ERR_INVALID_ARG = 1, /* null pointer, bad size, in % 8 != 0, ...     */
-    AQ_ERR_UNSUPPORTED = 2, /* (K, B) or group size this build cannot run  */
+    AQ_ERR_UNSUPPORTED = 2, /* (K, B) or group size the library cannot run */
     AQ_ERR_MISALIGNED = 3,  /* an array pointer not 16-byte aligned         */
     AQ_ERR_WORKSPACE = 4,   /* workspace missing or smaller than required   */
     AQ_ERR_CUDA = 5,        /* the CUDA runtime reported an error           */
