@@ -333,10 +333,11 @@ gemv_lut_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restr
 // rate of random 16-byte codeword reads from the 1 MiB codebook.  This kernel
 // reads them straight into registers (through L1, which keeps a share of the
 // codebook) and multiplies them with x in fp32 (each product of two binary16
-// values is exact); it keeps no tile in shared memory, so three CTAs of 256
-// threads fit per SM at batch 1 (85 registers; two at batch 2), about 6000
+// values is exact); it keeps no tile in shared memory, so six CTAs of 128
+// threads fit per SM at batch 1 (85 registers; four at batch 2), about 6000
 // reads in flight, and L1 keeps most of its capacity for the codebook.
-// CTA = 32 row tiles (256 rows) x one split of the groups.  Thread (row tile
+// CTA = 16 row tiles (128 rows) x one split of the groups (128 rows rather
+// than 256: half the splits per row range, a shorter split-K finish).  Thread (row tile
 // t/8, lane t%8) owns the chunks (its row tile, group G0 + t%8 + 8 j): a
 // chunk's 8 codes give the 8 rows' weights of its group.  The first chunk's
 // codewords are requested before the CTA waits for the previous launch
@@ -346,8 +347,8 @@ gemv_lut_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restr
 // The 8 lanes of a row tile add their row sums with a 3-level
 // reduce-scatter; split-K partial sums are finished as for the tables.
 // ---------------------------------------------------------------------------
-constexpr int kCcThreads = 256;
-constexpr int kCcRowTiles = kCcThreads / 8;  // 256 rows per CTA
+constexpr int kCcThreads = 128;
+constexpr int kCcRowTiles = kCcThreads / 8;  // 128 rows per CTA
 constexpr int kCcMaxSplits = 32;             // more splits per row range: the tensor-core path
 constexpr int kCcMaxBatch = 2;  // measured: faster than the tensor cores at batch 1 and 2, slower from 3
 constexpr int kCcStage = 16 * 1024;          // split-K staging (more would take L1 from the codebook)
@@ -378,7 +379,7 @@ __device__ __forceinline__ float cc_dot8(float acc, uint4 w, float4 x0, float4 x
 
 // CTAs of the CUDA-core kernel resident per SM, by batch (registers)
 template <int NB>
-constexpr int kCcPerSMOf = NB == 1 ? 3 : 2;
+constexpr int kCcPerSMOf = NB == 1 ? 6 : 4;
 
 template <int NB>
 __global__ void __launch_bounds__(kCcThreads, kCcPerSMOf<NB>)
@@ -1107,12 +1108,8 @@ cudaError_t launch_plan(const Geom &g, const GemvPlan &p, const void *packed, co
             return launch_pdl(kern, grid, dim3(kCcThreads), p.cc_smem, s, g, pk, c, scales, x, y, sk, p.len,
                               p.cc_smem);
         };
-        switch (batch) {
-        case 1: e = cc(gemv_1x16_cc_kernel<1>); break;
-        case 2: e = cc(gemv_1x16_cc_kernel<2>); break;
-        case 3: e = cc(gemv_1x16_cc_kernel<3>); break;
-        default: e = cc(gemv_1x16_cc_kernel<4>); break;
-        }
+        static_assert(kCcMaxBatch == 2, "one instantiation per batch on this path");
+        e = batch == 1 ? cc(gemv_1x16_cc_kernel<1>) : cc(gemv_1x16_cc_kernel<2>);
     } else if (p.path == kLut) {
         const int smem = kLutBytes;  // the tables
         auto lut = [&](auto sch) {

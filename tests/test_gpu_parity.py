@@ -148,7 +148,7 @@ def test_gemv_stream_k_rows_checked_in_full(batch):
 
 
 def test_gemv_cuda_core_path_deterministic_and_reusable():
-    """1x16 at batch 1 on the CUDA cores (4096 x 2048: 16 row ranges, 27
+    """1x16 at batch 1 on the CUDA cores (4096 x 2048: 32 row ranges, 27
     group splits finished by the last CTA of each range): same bits twice,
     correct results with one workspace reused across activations."""
     layer = _layer(4096, 2048, 1, 16, 17)
