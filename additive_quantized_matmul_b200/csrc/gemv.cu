@@ -6,19 +6,22 @@
 // 8) and multiplied with the matching 8 activations, the product the
 // paper's abstract names for token generation.
 //
-// Two kernels, chosen by scheme and batch:
+// Three kernels, chosen by scheme, batch and shape:
 //  * 8-bit codes with one or two codebooks (1x8, 2x8), batch 1 --
 //    `gemv_lut_kernel`: per-group codebook x activation tables in shared
 //    memory, lane-private so random codes never conflict; K 4-byte table
 //    reads per group.
-//  * every other case (1x16, 2x16, 8x8 at any batch; 1x8, 2x8 at batch
-//    2..16) -- `gemv_tc_kernel`: codes are decoded into a 128x64 binary16
-//    tile in shared memory (128-byte-swizzled, K-major) and multiplied by the
-//    activations on the tensor cores (tcgen05.mma, M = 128, N = 16, fp32
-//    accumulator in tensor memory), so the cost per group does not grow with
-//    the batch.  For 1x16 the bound is the rate of random 16-byte codeword
-//    reads from the L2-resident 1 MiB codebook (about one request per SM
-//    clock), not HBM.
+//  * 1x16 at batch 1 and 2 (unless the layer has too few rows to fill the
+//    SMs without more than 32 splits per row range) -- `gemv_1x16_cc_kernel`:
+//    codewords read into registers through L1 and multiplied with x on the
+//    CUDA cores, no tile in shared memory.
+//  * every other case -- `gemv_tc_kernel`: codes are decoded into a 128x64
+//    binary16 tile in shared memory (128-byte-swizzled, K-major) and
+//    multiplied by the activations on the tensor cores (tcgen05.mma,
+//    M = 128, N = 16, fp32 accumulator in tensor memory), so the cost per
+//    group does not grow with the batch.
+// For 1x16 the bound is the rate of random 16-byte codeword reads from the
+// 1 MiB codebook (through L2, partly L1), not HBM.
 // Split-K partial sums go to the workspace and the last CTA to arrive for a
 // row range adds them in split order (no float atomics: bit-reproducible).
 #include <algorithm>
