@@ -1,0 +1,67 @@
+"""Host-side parts of bench.py that need no GPU: the algorithmic-bytes
+formula the bench reports against, the committed traffic record's source
+check, the oracle baseline's fields and the clock-sample summary."""
+import json
+import os
+
+import bench
+from aq_inputs import LayerSpec
+from conftest import ROOT
+
+
+def test_algorithmic_bytes_of_the_default_layer():
+    # codes 4096*512*2 + codebook 65536*16 + scales 2*4096 + x 2*4096 + y 2*4096
+    assert bench.alg_bytes(LayerSpec(4096, 4096, 1, 16), 1) == 4194304 + 1048576 + 8192 + 8192 + 8192
+    # batch grows x and y only
+    assert (bench.alg_bytes(LayerSpec(4096, 4096, 1, 16), 16) - bench.alg_bytes(LayerSpec(4096, 4096, 1, 16), 1)
+            == 15 * (2 * 4096 + 2 * 4096))
+    # 2x8: two 8-bit codes per group, two 256-entry codebooks
+    # (codes 11008*512*2, codebooks 2*256*16, scales and y 2*11008 each, x 2*4096)
+    assert bench.alg_bytes(LayerSpec(11008, 4096, 2, 8), 1) == 11008 * 512 * 2 + 2 * 256 * 16 + 4 * 11008 + 2 * 4096
+
+
+def test_traffic_record_only_while_the_sources_match(tmp_path, monkeypatch):
+    rec = json.load(open(os.path.join(ROOT, "profiles", "traffic_gemv_tc.json")))
+    assert set(rec["per_launch_bytes"]) == {"1", "4", "16"}
+    for b in (1, 4, 16):
+        assert bench.recorded_traffic(bench.WORKLOAD, b) == rec["per_launch_bytes"][str(b)]
+    assert bench.recorded_traffic("llama2-70b-1x16", 1) is None
+    # a copy of the repository whose kernel source differs gives no traffic
+    fake = tmp_path / "repo"
+    (fake / "profiles").mkdir(parents=True)
+    (fake / "profiles" / "traffic_gemv_tc.json").write_text(json.dumps(rec))
+    for f in rec["sources"]:
+        dst = fake / f
+        dst.parent.mkdir(parents=True, exist_ok=True)
+        dst.write_bytes(open(os.path.join(ROOT, f), "rb").read() + (b"\n// changed\n" if f.endswith("gemv.cu") else b""))
+    monkeypatch.setattr(bench, "ROOT", str(fake))
+    assert bench.recorded_traffic(bench.WORKLOAD, 1) is None
+
+
+def test_cpu_baseline_fields():
+    r = bench.cpu_baseline(budget_s=0.05, single_budget_s=0.02)
+    for k in ("value", "unit", "cores", "kind", "sample", "single_thread", "nproc", "cpu_model"):
+        assert k in r
+    assert r["kind"] == "oracle" and r["unit"] == "GB/s"
+    assert r["value"] > 0 and r["single_thread"]["value"] > 0
+    assert 1 <= r["cores"] <= r["nproc"]
+
+
+def test_clock_summary_flags_throttle_reasons():
+    s = bench.ClockSampler(0)
+    s.lines = [
+        "0, 1965, 1965, 700.1, 0x0, Not Active, Not Active, Not Active, Not Active",
+        "0, 1900, 1965, 999.0, 0x4, Not Active, Not Active, Not Active, Active",
+        "0, 1965, 1965, 800.0, 0x0, Not Active, Not Active, Not Active, Not Active",
+    ]
+    out = s.summary()
+    assert out["sm_mhz"] == 1965.0 and out["sm_max_mhz"] == 1965.0
+    assert out["reasons"] == ["sw_power_cap"]
+    assert out["samples"] == 3
+
+
+def test_clock_summary_without_samples():
+    s = bench.ClockSampler(0)
+    s.lines = []
+    out = s.summary()
+    assert out["sm_mhz"] is None and out["samples"] == 0
