@@ -549,6 +549,29 @@ def test_encode_never_worse_than_start_and_objective_consistent(K, B, beam):
     assert np.array_equal(oracle.objective(w, h, cb, codes), obj)
 
 
+def test_encode_ties_resolved_by_parent_beam_then_code():
+    """Hand-worked tie (one group, K = 3, B = 2, beam 2, H = I, lane 0 only).
+    Target 3; codebook 0 holds 2 (code 1) and 0 (code 2), codebook 1 holds 0
+    (code 0) and -2 (code 1), codebook 2 holds 0 (code 0) and 3 (code 1);
+    every other codeword is 100.  Codebook 0 keeps beams [code 1 (error 1),
+    code 2 (error 9)].  Codebook 1: the best is (beam 0, code 0) with error
+    1, then (beam 0, code 1) and (beam 1, code 0) tie at 9 -- the lower
+    parent beam goes first, so the second beam is (1, 1).  Codebook 2: that
+    beam plus code 1 reaches the target exactly, giving codes (1, 1, 1);
+    ordering ties by code alone would give (2, 0, 1) at the same objective."""
+    cb = np.full((3, 4, 8), 0.0, dtype=np.float16)
+    cb[:, :, 0] = 100.0
+    cb[0, 1, 0], cb[0, 2, 0] = 2.0, 0.0
+    cb[1, 0, 0], cb[1, 1, 0] = 0.0, -2.0
+    cb[2, 0, 0], cb[2, 1, 0] = 0.0, 3.0
+    w = np.zeros((1, 8), dtype=np.float16)
+    w[0, 0] = 3.0
+    c0 = np.zeros((1, 1, 3), dtype=np.uint8)
+    codes, obj = oracle.encode(w, np.eye(8, dtype=np.float32), cb, c0, beam=2)
+    assert codes[0, 0].tolist() == [1, 1, 1]
+    assert obj[0] == 0.0
+
+
 def test_encode_full_beam_is_sequential_exhaustive_per_group():
     """beam = 2^B: each group's code pair is the brute-force optimum given
     the groups before it (already chosen) and after it (still initial)."""
