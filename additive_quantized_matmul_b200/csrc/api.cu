@@ -11,6 +11,7 @@ namespace {
 using aqk::Geom;
 
 constexpr int kVersion = 10000;  // 1.0.0
+constexpr int32_t kMaxInFeatures = 65535 * 256;
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -24,8 +25,10 @@ aq_status check_desc(const aq_layer_desc *d)
     // keep every byte offset and element count within 64-bit range and the
     // per-row chunk count within 32-bit kernel indices
     if ((int64_t)d->out_features * d->in_features > (int64_t)1 << 40) return AQ_ERR_INVALID_ARG;
-    // grid.y of the split-K launches is bounded by 65535 group blocks
-    if (d->in_features > (1 << 24) || d->out_features > (1 << 28)) return AQ_ERR_INVALID_ARG;
+    // grid.y of the split-K launches is at most 65535: the batch-1 table
+    // path takes one split per block of 32 groups (in / 256 splits) and the
+    // tensor path at most one per 4 stages of 8 groups (in / 256 again)
+    if (d->in_features > kMaxInFeatures || d->out_features > (1 << 28)) return AQ_ERR_INVALID_ARG;
     return AQ_OK;
 }
 

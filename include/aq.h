@@ -85,7 +85,7 @@ typedef enum {
 /* One quantised linear layer: y[out] = diag(s) W[out][in] x[in]. */
 typedef struct {
     int32_t out_features;  /* rows of W, 1 .. 2^28                         */
-    int32_t in_features;   /* columns of W, 8 .. 2^24, multiple of 8       */
+    int32_t in_features;   /* columns of W, 8 .. 65535*256, multiple of 8  */
     int32_t group_size;    /* weights per code group; must be 8            */
     int32_t num_codebooks; /* K: 1x16, 2x8, 1x8, 2x16 or 8x8 with nbits    */
     int32_t nbits;         /* B: bits per code, codebook has 2^B entries   */

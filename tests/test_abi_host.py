@@ -73,6 +73,10 @@ def test_packed_bytes_matches_oracle(out, inp, K, B):
     ((16, 64, 4, 1, 16), "group size"), ((16, 64, 8, 4, 8), "4x8"), ((16, 64, 8, 2, 4), "2x4"),
     ((16, 64, 8, 1, 12), "1x12"), ((16, 64, 8, 3, 8), "3x8"), ((16, 64, 8, 8, 16), "8x16"),
     ((-1, 64, 8, 1, 16), "negative"),
+    ((8, 1 << 24, 8, 2, 8), "in = 2^24 (65536 blocks of 32 groups: one grid row too many)"),
+    ((8, 65535 * 256 + 8, 8, 1, 16), "in above 65535 * 256"),
+    ((1 << 20, 1 << 21, 8, 2, 8), "out * in above 2^40"),
+    ((1 << 28 + 1, 8, 8, 2, 8), "out above 2^28"),
 ])
 def test_invalid_descriptors(desc, why):
     d = aq.LayerDesc(*desc)
@@ -85,6 +89,16 @@ def test_invalid_descriptors(desc, why):
     assert st == want, why
     st = aq.lib.aq_dequant(ctypes.byref(d), FAKE, FAKE, None, FAKE, None)
     assert st == want, why
+
+
+def test_largest_input_width_is_accepted():
+    """in = 65535 * 256 is the widest layer: its 65535 blocks of 32 groups
+    are the most split-K grid rows a launch can have."""
+    for K, B in SCHEMES:
+        d = aq.LayerDesc.make(8, 65535 * 256, K, B)
+        assert aq.aq_packed_codes_bytes(d) == oracle.packed_bytes(8, 65535 * 256, K, B)
+        for b in (1, 2, 16):
+            assert aq.aq_gemv_workspace_bytes(d, b) >= 16
 
 
 def test_workspace_sizes_host_only():
