@@ -28,7 +28,9 @@
  *  - binary16 values are passed as uint16_t bit patterns (IEEE 754 half);
  *  - every array pointer is a DEVICE pointer on the current CUDA device,
  *    owned by the caller; the library allocates no memory and keeps no
- *    state between calls (thread-safe; calls on one stream are ordered);
+ *    state between calls (thread-safe; calls on one stream are ordered),
+ *    except aq_gemv_noalloc, which uses one fixed device array of the
+ *    library (described at that function);
  *  - work is enqueued on `stream` (NULL = legacy default stream) and the
  *    call returns after the launch; the caller synchronises;
  *  - the GEMV kernels use programmatic dependent launch: a GEMV may start
