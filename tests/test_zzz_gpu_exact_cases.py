@@ -11,13 +11,21 @@ are exact too.  So the decode-time product (table, CUDA-core and
 tensor-core paths, any split) and the prefill product must equal the dense
 product exactly, not just within the tolerance.  The same holds for a 1x16
 layer whose codes all select one codeword (every gather hits one address).
+
+The parameter gradient has the same property on these layers: with gy in
+{-1, 0, 1} as well, M = gy x^T holds integers of magnitude at most T, and
+dL/ds and dL/dC are sums of integers and half-integers far below 2^24, so
+the order of the kernel's atomics and shared-memory scatter cannot change
+them: they must equal the oracle's fp64 values exactly.
 """
 import numpy as np
 import pytest
+import torch
 
+import additive_quantized_matmul_b200 as aq
 import oracle
 from aq_inputs import Layer, LayerSpec
-from aqtest import DevLayer, run_gemm, run_gemv
+from aqtest import DevLayer, dev, run_gemm, run_gemv, workspace
 
 pytestmark = pytest.mark.gpu
 
@@ -97,3 +105,27 @@ def test_gemv_every_code_the_same_codeword(code, batch):
     want = _expected(layer, x)
     got = run_gemv(DevLayer(layer), x)
     assert np.array_equal(got, want)
+
+
+@pytest.mark.parametrize("K,B,inp", CASES)
+@pytest.mark.parametrize("T", [64, 136])
+def test_param_grad_one_hot_codebooks_exact(K, B, inp, T):
+    layer = _one_hot_layer(1000, inp, K, B, 13 * K + B + T)
+    x = _int_activations(inp, T, T)
+    gy = _int_activations(1000, T, T + 1)
+    dl = DevLayer(layer)
+    gs = torch.full((1000,), float("nan"), dtype=torch.float32, device="cuda")
+    gc = torch.full(((K << B) * 8,), float("nan"), dtype=torch.float32, device="cuda")
+    ws = workspace(aq.aq_param_grad_workspace_bytes(dl.desc, T))
+    aq.aq_param_grad(dl.desc, dl.packed, dl.codebooks, dl.scales, dev(x.view(np.uint16)),
+                     dev(gy.view(np.uint16)), T, gs, gc, ws)
+    torch.cuda.synchronize()
+    assert aq.aq_workspace_status(ws) == 0
+    rs, _, rc, _ = oracle.backward(layer.codes, layer.codebooks, layer.scales, x, gy)
+    assert np.abs(rc).max() < 2 ** 22 and np.abs(rs).max() < 2 ** 22
+    got_s = gs.cpu().numpy().astype(np.float64)
+    got_c = gc.cpu().numpy().astype(np.float64)
+    bad_s = np.flatnonzero(got_s != rs)
+    bad_c = np.flatnonzero(got_c != rc.ravel())
+    assert bad_s.size == 0, f"{K}x{B} T{T} grad_s: {bad_s.size} differ"
+    assert bad_c.size == 0, f"{K}x{B} T{T} grad_C: {bad_c.size} differ"
