@@ -236,3 +236,22 @@ def test_gather_probe_argument_errors():
     assert f(FAKE, FAKE, 64, 0, None, None) == 1
     assert f(FAKE + 8, FAKE, 64, 0, FAKE, None) == 3   # misaligned codebook
     assert f(FAKE, FAKE + 2, 64, 1, FAKE, None) == 3   # misaligned codes
+
+
+def test_binding_fails_loudly_without_the_library(tmp_path):
+    """A copy of the package without libaq_b200.so must refuse to import
+    (there is no CPU path to fall back to)."""
+    import shutil
+    import subprocess
+    import sys
+    pkg = tmp_path / "additive_quantized_matmul_b200"
+    pkg.mkdir()
+    shutil.copy(os.path.join(ROOT, "additive_quantized_matmul_b200", "__init__.py"), pkg / "__init__.py")
+    code = ("import sys; sys.path.insert(0, sys.argv[1])\n"
+            "try:\n    import additive_quantized_matmul_b200\n"
+            "except ImportError as e:\n    print('ImportError:', e); sys.exit(3)\n"
+            "sys.exit(0)\n")
+    r = subprocess.run([sys.executable, "-c", code, str(tmp_path)], capture_output=True, text=True, timeout=120,
+                       cwd=str(tmp_path))
+    assert r.returncode == 3, r.stdout + r.stderr
+    assert "libaq_b200.so is missing" in r.stdout and "build.py" in r.stdout
