@@ -86,6 +86,19 @@ MUTANTS = [
      "word |= (uint64_t)code_at(codes, B, (o * G + g) * K + k) << (k * B);",
      "word |= (uint64_t)code_at(codes, B, (o * G + g) * K + k) << ((K - 1 - k) * B);"),
     ("pack: groups not padded", "int64_t gp = (in / AQO_GROUP + 31) / 32 * 32;", "int64_t gp = in / AQO_GROUP;"),
+    ("pack: rows not padded", "int64_t rows = (out + 7) / 8 * 8;", "int64_t rows = out;"),
+    # (a 16-bit mask for 8-bit codes is no mistake: the uint8_t store masks)
+    ("unpack: codes shifted by bytes", "uint64_t c = (word >> (k * B)) & mask;", "uint64_t c = (word >> (k * 8)) & mask;"),
+    # more of the gradient and the encoder
+    ("backward: scale bound without abs", "gsb += fabs(row[i]) * mabs[i];", "gsb += row[i] * mabs[i];"),
+    ("encode: beam width ignored", "int keep = np < beam ? np : beam;", "int keep = 1;"),
+    ("encode: every survivor from beam 0", "nxt[r * S + t] = cur[props[r].parent * S + t];", "nxt[r * S + t] = cur[t];"),
+    ("encode: H taken as its diagonal", "for (int64_t b = 0; b < in; ++b) t += h[a * in + b] * e[b];",
+     "t += h[a * in + a] * e[a];"),
+    ("objective: first row's codes for every row", "row_error(in, K, B, codes + o * S, wd, codebooks, e);",
+     "row_error(in, K, B, codes, wd, codebooks, e);"),
+    ("storage: weights counted as groups", "double code_bits = (double)out * (double)(in / AQO_GROUP) * K * B;",
+     "double code_bits = (double)out * (double)in * K * B;"),
 ]
 
 # Runs the pins against the oracle built from the mutated source.
