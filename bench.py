@@ -54,6 +54,13 @@ def alg_bytes(spec: LayerSpec, n: int) -> int:
     return codes + cbs + 2 * spec.out_features + 2 * spec.in_features * n + 2 * spec.out_features * n
 
 
+def bits_per_weight(spec: LayerSpec) -> dict:
+    """Stored bits per weight of one layer: the closed form K*B/8 (codes
+    only) and with the codebooks and row scales counted."""
+    return {"codes": spec.num_codebooks * spec.nbits / 8,
+            "stored": round(8 * alg_bytes(spec, 0) / (spec.out_features * spec.in_features), 3)}
+
+
 def measured_peaks() -> dict:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -537,6 +544,8 @@ def run_gpu(args) -> None:
         if "chain" in u:  # one call is a whole block of layers
             k["layers_per_call"] = len(u["chain"])
             k["us_per_block"] = k.pop("us_per_layer")
+        if op == "gemv" and "spec" in u:
+            k["bits_per_weight"] = bits_per_weight(u["spec"])
         k["frac_hbm"] = round(k["gbs"] / peaks["hbm_gbs"], 4)
         k["frac_tensor"] = round(k["tflops"] / peaks["bf16_tflops_sustained"], 4)
         kernels.append(k)

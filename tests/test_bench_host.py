@@ -65,3 +65,13 @@ def test_clock_summary_without_samples():
     s.lines = []
     out = s.summary()
     assert out["sm_mhz"] is None and out["samples"] == 0
+
+
+def test_stored_bits_per_weight():
+    # closed form 2.0 for 1x16 and 2x8; with codebooks and scales counted
+    # the 1 MiB 1x16 codebook weighs on small layers
+    for (o, i, K, B), stored in [((4096, 4096, 1, 16), 2.504), ((28672, 8192, 1, 16), 2.038),
+                                 ((1024, 8192, 1, 16), 3.002), ((11008, 4096, 2, 8), 2.005)]:
+        b = bench.bits_per_weight(LayerSpec(o, i, K, B))
+        assert b["codes"] == 2.0 and b["stored"] == stored, (o, i, K, B, b)
+    assert bench.bits_per_weight(LayerSpec(11008, 4096, 2, 16))["codes"] == 4.0
