@@ -235,7 +235,8 @@ def aq_gather_probe_sink_bytes(mode: int) -> int:
 
 def aq_gather_probe(codebook, codes, n: int, mode: int, sink, stream=None) -> None:
     """Measurement aid: read codebook[codes[i]] for each of the n 16-bit codes
-    (mode 0: from L2 into shared memory as the 1x16 GEMV does; mode 1: from
-    the codebook split over 8-CTA clusters' shared memory); per-thread XOR
-    checksums go to ``sink``."""
+    (mode 0: from L2 into shared memory with cp.async, as the tensor-core
+    GEMV's decoders do; mode 1: from the codebook split over 8-CTA
+    clusters' shared memory; mode 2: through L1 into registers, as the
+    batch-1 CUDA-core GEMV does); per-thread XOR checksums go to ``sink``."""
     _check("aq_gather_probe", lib.aq_gather_probe(_ptr(codebook), _ptr(codes), n, mode, _ptr(sink), _stream(stream)))
