@@ -36,7 +36,8 @@
  * exhaustive single-group decode, one-hot codebooks, additivity, permutation
  * invariance, integer-exact products, pure-Python brute force on tiny inputs,
  * the pages' bit-rate examples and model sizes, pack round trip and
- * hand-worked layout offsets.
+ * hand-worked layout offsets.  tests/test_oracle_mutants.py checks the pins
+ * themselves: copies of this file with one planted slip each must fail them.
  */
 #include <math.h>
 #include <stdint.h>
