@@ -20,7 +20,7 @@ __all__ = [
     "AQError", "LayerDesc", "lib", "library_path", "aq_version", "aq_status_string",
     "aq_packed_codes_bytes", "aq_gemv_workspace_bytes", "aq_gemm_workspace_bytes",
     "aq_workspace_status", "aq_selftest_bounded_wait", "aq_pack_codes", "aq_unpack_codes",
-    "aq_dequant", "aq_gemv", "aq_gemv_noalloc", "aq_gemm", "aq_param_grad_workspace_bytes",
+    "aq_dequant", "aq_gemv", "aq_gemv_ordered", "aq_gemv_noalloc", "aq_gemm", "aq_param_grad_workspace_bytes",
     "aq_param_grad", "aq_encode_workspace_bytes", "aq_encode", "aq_gather_probe_sink_bytes",
     "aq_gather_probe", "EXPORTED_SYMBOLS",
     "GEMV_NOALLOC_SCRATCH_BYTES",
@@ -38,7 +38,7 @@ STATUS_NAMES = {0: "AQ_OK", 1: "AQ_ERR_INVALID_ARG", 2: "AQ_ERR_UNSUPPORTED",
 EXPORTED_SYMBOLS = (
     "aq_status_string", "aq_version", "aq_packed_codes_bytes", "aq_gemv_workspace_bytes",
     "aq_gemm_workspace_bytes", "aq_workspace_status", "aq_selftest_bounded_wait",
-    "aq_pack_codes", "aq_unpack_codes", "aq_dequant", "aq_gemv", "aq_gemv_noalloc", "aq_gemm",
+    "aq_pack_codes", "aq_unpack_codes", "aq_dequant", "aq_gemv", "aq_gemv_ordered", "aq_gemv_noalloc", "aq_gemm",
     "aq_param_grad_workspace_bytes", "aq_param_grad", "aq_encode_workspace_bytes", "aq_encode",
     "aq_gather_probe_sink_bytes", "aq_gather_probe",
 )
@@ -88,6 +88,7 @@ def _load() -> ctypes.CDLL:
         "aq_unpack_codes": ([dp, vp, vp, vp], i32),
         "aq_dequant": ([dp, vp, vp, vp, vp, vp], i32),
         "aq_gemv": ([dp, vp, vp, vp, vp, i32, vp, vp, sz, vp], i32),
+        "aq_gemv_ordered": ([dp, vp, vp, vp, vp, i32, vp, vp, sz, vp], i32),
         "aq_gemm": ([dp, vp, vp, vp, vp, i32, vp, vp, sz, vp], i32),
         "aq_gemv_noalloc": ([dp, vp, vp, vp, vp, i32, vp, vp], i32),
         "aq_param_grad_workspace_bytes": ([dp, i32], sz),
@@ -183,6 +184,17 @@ def aq_gemv(desc: LayerDesc, packed, codebooks, scales, x, batch: int, y, worksp
                                   _stream(stream)))
 
 
+def aq_gemv_ordered(desc: LayerDesc, packed, codebooks, scales, x, batch: int, y, workspace,
+                    workspace_bytes: int | None = None, stream=None) -> None:
+    """aq_gemv launched without programmatic dependent launch: no weight is
+    read before the previous work on the stream has completed."""
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    _check("aq_gemv_ordered", lib.aq_gemv_ordered(ctypes.byref(desc), _ptr(packed), _ptr(codebooks), _ptr(scales),
+                                                  _ptr(x), batch, _ptr(y), _ptr(workspace), workspace_bytes,
+                                                  _stream(stream)))
+
+
 def aq_gemv_noalloc(desc: LayerDesc, packed, codebooks, scales, x, batch: int, y, stream=None) -> None:
     """aq_gemv for callers that cannot allocate device memory: the split-K
     scratch is a fixed array inside the library (see include/aq.h); calls
@@ -238,5 +250,7 @@ def aq_gather_probe(codebook, codes, n: int, mode: int, sink, stream=None) -> No
     (mode 0: from L2 into shared memory with cp.async, as the tensor-core
     GEMV's decoders do; mode 1: from the codebook split over 8-CTA
     clusters' shared memory; mode 2: through L1 into registers, as the
-    batch-1 CUDA-core GEMV does); per-thread XOR checksums go to ``sink``."""
+    batch-1 CUDA-core GEMV does; mode 3: no codeword, ``codes`` itself read
+    once as a stream, the read-only HBM bandwidth; ``codebook`` may then be
+    None); per-thread XOR checksums go to ``sink``."""
     _check("aq_gather_probe", lib.aq_gather_probe(_ptr(codebook), _ptr(codes), n, mode, _ptr(sink), _stream(stream)))

@@ -130,9 +130,11 @@ aq_status aq_dequant(const aq_layer_desc *desc, const void *packed, const uint16
                                          reinterpret_cast<cudaStream_t>(stream)));
 }
 
-aq_status aq_gemv(const aq_layer_desc *desc, const void *packed, const uint16_t *codebooks,
-                  const uint16_t *scales, const uint16_t *x, int batch, uint16_t *y,
-                  void *workspace, size_t workspace_bytes, aq_stream_t stream)
+namespace {
+
+aq_status gemv_entry(const aq_layer_desc *desc, const void *packed, const uint16_t *codebooks,
+                     const uint16_t *scales, const uint16_t *x, int batch, uint16_t *y,
+                     void *workspace, size_t workspace_bytes, aq_stream_t stream, bool pdl)
 {
     aq_status st = check_desc(desc);
     if (st != AQ_OK) return st;
@@ -146,7 +148,23 @@ aq_status aq_gemv(const aq_layer_desc *desc, const void *packed, const uint16_t 
     if (!workspace || workspace_bytes < need) return AQ_ERR_WORKSPACE;
     if (!aligned16(workspace)) return AQ_ERR_MISALIGNED;
     return from_cuda(aqh::launch_gemv(g, packed, codebooks, scales, x, batch, y, workspace,
-                                      reinterpret_cast<cudaStream_t>(stream)));
+                                      reinterpret_cast<cudaStream_t>(stream), pdl));
+}
+
+}  // namespace
+
+aq_status aq_gemv(const aq_layer_desc *desc, const void *packed, const uint16_t *codebooks,
+                  const uint16_t *scales, const uint16_t *x, int batch, uint16_t *y,
+                  void *workspace, size_t workspace_bytes, aq_stream_t stream)
+{
+    return gemv_entry(desc, packed, codebooks, scales, x, batch, y, workspace, workspace_bytes, stream, true);
+}
+
+aq_status aq_gemv_ordered(const aq_layer_desc *desc, const void *packed, const uint16_t *codebooks,
+                          const uint16_t *scales, const uint16_t *x, int batch, uint16_t *y,
+                          void *workspace, size_t workspace_bytes, aq_stream_t stream)
+{
+    return gemv_entry(desc, packed, codebooks, scales, x, batch, y, workspace, workspace_bytes, stream, false);
 }
 
 aq_status aq_gemv_noalloc(const aq_layer_desc *desc, const void *packed, const uint16_t *codebooks,
@@ -240,16 +258,17 @@ aq_status aq_param_grad(const aq_layer_desc *desc, const void *packed, const uin
 
 size_t aq_gather_probe_sink_bytes(int mode)
 {
-    if (mode < 0 || mode > 2) return 0;
+    if (mode < 0 || mode > 3) return 0;
     return aqh::gather_probe_sink_bytes(mode);
 }
 
 aq_status aq_gather_probe(const uint16_t *codebook, const uint16_t *codes, size_t n, int mode, void *sink,
                           aq_stream_t stream)
 {
-    if (mode < 0 || mode > 2) return AQ_ERR_INVALID_ARG;
-    if (!codebook || !codes || !sink || n == 0 || n % 8 || n > ((size_t)1 << 36)) return AQ_ERR_INVALID_ARG;
-    if (!aligned16(codebook) || !aligned16(codes) || !aligned16(sink)) return AQ_ERR_MISALIGNED;
+    if (mode < 0 || mode > 3) return AQ_ERR_INVALID_ARG;
+    if ((mode != 3 && !codebook) || !codes || !sink || n == 0 || n % 8 || n > ((size_t)1 << 36))
+        return AQ_ERR_INVALID_ARG;
+    if ((codebook && !aligned16(codebook)) || !aligned16(codes) || !aligned16(sink)) return AQ_ERR_MISALIGNED;
     return from_cuda(
         aqh::launch_gather_probe(codebook, codes, n, mode, sink, reinterpret_cast<cudaStream_t>(stream)));
 }

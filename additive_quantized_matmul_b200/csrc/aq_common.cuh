@@ -248,7 +248,7 @@ cudaError_t launch_dequant(const aqk::Geom &g, const void *packed, const uint16_
 size_t gemv_workspace_bytes(const aqk::Geom &g, int batch);
 cudaError_t launch_gemv(const aqk::Geom &g, const void *packed, const uint16_t *cb,
                         const uint16_t *scales, const uint16_t *x, int batch, uint16_t *y,
-                        void *ws, cudaStream_t s);
+                        void *ws, cudaStream_t s, bool pdl = true);
 cudaError_t launch_gemv_noalloc(const aqk::Geom &g, const void *packed, const uint16_t *cb,
                                 const uint16_t *scales, const uint16_t *x, int batch, uint16_t *y,
                                 cudaStream_t s, bool *too_large);

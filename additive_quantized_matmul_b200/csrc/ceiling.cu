@@ -18,6 +18,11 @@
 //    GEMV): three CTAs of 256 threads per SM, a chunk's 8 codewords read
 //    with ld.global.nc into registers, no shared memory (L1 keeps what it
 //    can of the codebook).
+//  * mode 3 (read-only HBM stream, the cross-check of the copy bandwidth
+//    the HBM roofline uses): the `codes` array itself is read once, 16
+//    bytes per load, eight loads in flight per thread, four CTAs of 256
+//    threads per SM, L1 bypassed; no codebook read.  Over an array much
+//    larger than L2 its time is the read bandwidth of HBM.
 // Each thread XORs every 32-bit word it reads into a 16-byte checksum
 // written to `sink` (so the reads cannot be elided, and a test can compare
 // the XOR of all checksums with the XOR of the codewords the codes select).
@@ -103,6 +108,37 @@ probe_ldg_kernel(const uint4 *__restrict__ cb, const uint4 *__restrict__ chunks,
         for (int j = 0; j < 8; ++j) v[j] = ldg_nc_v4(cb + code_of(w, j));
 #pragma unroll
         for (int j = 0; j < 8; ++j) xor_into(acc, v[j]);
+    }
+    grid_dependency_wait();  // the previous launch on the stream may still write the sink
+    sink[first] = acc;
+}
+
+constexpr int kProbeStreamThreads = 256;
+constexpr int kProbeStreamPerSM = 4;
+constexpr int kProbeStreamUnroll = 8;
+
+// Thread (CTA c, thread t) reads chunks q = base + u * stride for u < 8,
+// base = (k * gridDim + c) * 8 * blockDim + t at step k: every load
+// instruction of a warp reads 512 consecutive bytes.
+__global__ void __launch_bounds__(kProbeStreamThreads, kProbeStreamPerSM)
+probe_stream_kernel(const uint4 *__restrict__ chunks, long nchunks, uint4 *sink)
+{
+    const long per_step = (long)gridDim.x * kProbeStreamThreads * kProbeStreamUnroll;
+    const long first = (long)blockIdx.x * kProbeStreamThreads + threadIdx.x;
+    const long cta0 = (long)blockIdx.x * kProbeStreamThreads * kProbeStreamUnroll + threadIdx.x;
+    grid_launch_dependents();
+    uint4 acc = make_uint4(0u, 0u, 0u, 0u);
+    long q0 = cta0;
+    for (; q0 + (long)(kProbeStreamUnroll - 1) * kProbeStreamThreads < nchunks; q0 += per_step) {
+        uint4 v[kProbeStreamUnroll];
+#pragma unroll
+        for (int u = 0; u < kProbeStreamUnroll; ++u) v[u] = ldg_stream_v4(chunks + q0 + (long)u * kProbeStreamThreads);
+#pragma unroll
+        for (int u = 0; u < kProbeStreamUnroll; ++u) xor_into(acc, v[u]);
+    }
+    for (int u = 0; u < kProbeStreamUnroll; ++u) {  // the ragged last step
+        const long q = q0 + (long)u * kProbeStreamThreads;
+        if (q < nchunks) xor_into(acc, ldg_stream_v4(chunks + q));
     }
     grid_dependency_wait();  // the previous launch on the stream may still write the sink
     sink[first] = acc;
@@ -202,6 +238,7 @@ size_t gather_probe_sink_bytes(int mode)
 {
     // mode 1 runs at most one CTA per SM (128 KiB of shared memory each)
     if (mode == 2) return (size_t)kProbeLdgPerSM * kNumSMs * kProbeLdgThreads * sizeof(uint4);
+    if (mode == 3) return (size_t)kProbeStreamPerSM * kNumSMs * kProbeStreamThreads * sizeof(uint4);
     const int ctas = mode == 0 ? probe_l2_ctas() : kNumSMs;
     return (size_t)ctas * kProbeThreads * sizeof(uint4);
 }
@@ -221,7 +258,13 @@ cudaError_t launch_gather_probe(const uint16_t *codebook, const uint16_t *codes,
     cfg.stream = s;
     cfg.attrs = attr;
     cudaError_t e;
-    if (mode == 2) {
+    if (mode == 3) {
+        cfg.gridDim = dim3(kProbeStreamPerSM * kNumSMs);
+        cfg.blockDim = dim3(kProbeStreamThreads);
+        cfg.dynamicSmemBytes = 0;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, probe_stream_kernel, chunks, nchunks, out);
+    } else if (mode == 2) {
         cfg.gridDim = dim3(kProbeLdgPerSM * kNumSMs);
         cfg.blockDim = dim3(kProbeLdgThreads);
         cfg.dynamicSmemBytes = 0;

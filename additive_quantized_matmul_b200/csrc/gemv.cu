@@ -27,6 +27,8 @@
 #include <algorithm>
 #include <mutex>
 
+#include <cuda.h>  // driver types only; the calls are fetched at run time
+
 #include "scheme.cuh"
 #include "tc_common.cuh"
 
@@ -952,6 +954,23 @@ long tc_cost(long ctas, int len, int res, int batch, bool early)
     return cost;
 }
 
+// Row tiles per CTA of the table path (whole quads of four tiles): as many
+// row ranges as put about two CTAs per SM in one wave.
+int lut_rt_per_cta(const Geom &g)
+{
+    const int ranges = std::max(1, std::min(g.rtiles, 2 * kNumSMs / g.gblocks));
+    return ((g.rtiles + ranges - 1) / ranges + 3) & ~3;
+}
+
+// Workspace of the table path: status word, one arrival counter per row
+// range, one partial sum per row and 32-group block.
+size_t lut_ws(const Geom &g)
+{
+    const int ranges = (g.rtiles + lut_rt_per_cta(g) - 1) / lut_rt_per_cta(g);
+    return kWsHeader + align16(sizeof(unsigned) * (size_t)ranges) +
+           (g.gblocks > 1 ? (size_t)g.gblocks * g.rows8 * sizeof(float) : 0);
+}
+
 // `cap`: largest workspace the caller can offer (the no-allocation entry
 // point's scratch); the plan lengthens the CTAs' shares until its partial
 // sums fit, down to one row tile per CTA (no partials).
@@ -977,17 +996,18 @@ GemvPlan plan_gemv(const Geom &g, int batch, size_t cap = ~(size_t)0)
         p.slots = p.ks > 1 ? p.ks : 0;
         const int nvec = kCcRowTiles * 8 * batch / 4;  // float4 of one row range's partial sums
         p.cc_smem = std::max(p.len * 32 * batch, std::min(kCcStage, p.ks > 1 ? p.ks * nvec * 16 : 0));
-    } else if (batch == 1 && g.B == 8 && g.K <= 2) {
+    } else if (batch == 1 && g.B == 8 && g.K <= 2 && lut_ws(g) <= cap) {
         p.path = kLut;
         p.ks = g.gblocks;
         // two CTAs per SM in one wave: every CTA builds its tables once, and
         // a third CTA per SM fits, so the next launch can start early
-        const int ranges = max(1, min(g.rtiles, 2 * kNumSMs / g.gblocks));
-        p.rt_per_cta = ((g.rtiles + ranges - 1) / ranges + 3) & ~3;  // whole quads of tiles
+        p.rt_per_cta = lut_rt_per_cta(g);
         p.grid_x = (g.rtiles + p.rt_per_cta - 1) / p.rt_per_cta;
         p.counters = p.grid_x;
         p.slots = p.ks > 1 ? p.ks : 0;
     } else {
+        // the tensor-core path, also for 8-bit codebooks at batch 1 when the
+        // table path's partial sums would not fit `cap`
         p.path = kTensor;
         const int mtiles = (g.out + kTcBM - 1) / kTcBM;
         const int nst = (g.G + 7) / 8;
@@ -1069,8 +1089,12 @@ cudaError_t set_smem(Kern k, int bytes)
 // prologue may overlap the tail of the previous kernel on the stream; the
 // kernel itself waits (griddepcontrol.wait) before touching x, y or the
 // workspace.
+// With `pdl` false the launch is an ordinary one: the kernel starts only
+// after the previous work on the stream has completed (griddepcontrol.wait
+// then returns at once).
 template <class... KArgs, class... Args>
-cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, int smem, cudaStream_t s, Args... args)
+cudaError_t launch_pdl(bool pdl, void (*kern)(KArgs...), dim3 grid, dim3 block, int smem, cudaStream_t s,
+                       Args... args)
 {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
@@ -1081,7 +1105,7 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, int smem, 
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = pdl ? 1 : 0;
     return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
 }
 
@@ -1093,7 +1117,7 @@ namespace {
 
 cudaError_t launch_plan(const Geom &g, const GemvPlan &p, const void *packed, const uint16_t *cb,
                         const uint16_t *scales, const uint16_t *x, int batch, uint16_t *y, void *ws,
-                        cudaStream_t s)
+                        cudaStream_t s, bool pdl)
 {
     SplitK sk;
     char *base = reinterpret_cast<char *>(ws);
@@ -1108,7 +1132,7 @@ cudaError_t launch_plan(const Geom &g, const GemvPlan &p, const void *packed, co
         auto cc = [&](auto kern) {
             cudaError_t r = set_smem(kern, p.cc_smem);
             if (r != cudaSuccess) return r;
-            return launch_pdl(kern, grid, dim3(kCcThreads), p.cc_smem, s, g, pk, c, scales, x, y, sk, p.len,
+            return launch_pdl(pdl, kern, grid, dim3(kCcThreads), p.cc_smem, s, g, pk, c, scales, x, y, sk, p.len,
                               p.cc_smem);
         };
         static_assert(kCcMaxBatch == 2, "one instantiation per batch on this path");
@@ -1120,7 +1144,7 @@ cudaError_t launch_plan(const Geom &g, const GemvPlan &p, const void *packed, co
             if constexpr (S::B == 8 && S::K <= 2) {
                 cudaError_t r = set_smem(gemv_lut_kernel<S>, smem);
                 if (r != cudaSuccess) return r;
-                return launch_pdl(gemv_lut_kernel<S>, grid, dim3(kLutWarps * 32), smem, s, g, pk, c, scales, x, y,
+                return launch_pdl(pdl, gemv_lut_kernel<S>, grid, dim3(kLutWarps * 32), smem, s, g, pk, c, scales, x, y,
                                   sk, p.rt_per_cta);
             } else {
                 return cudaErrorInvalidValue;
@@ -1134,12 +1158,12 @@ cudaError_t launch_plan(const Geom &g, const GemvPlan &p, const void *packed, co
             if (p.stream_k) {
                 cudaError_t r = set_smem(gemv_tc_kernel<S, true>, smem);
                 if (r != cudaSuccess) return r;
-                return launch_pdl(gemv_tc_kernel<S, true>, dim3(p.grid_x), dim3(kTcThreads), smem, s, g, pk, c,
+                return launch_pdl(pdl, gemv_tc_kernel<S, true>, dim3(p.grid_x), dim3(kTcThreads), smem, s, g, pk, c,
                                   scales, x, batch, y, sk, ws, p.len);
             }
             cudaError_t r = set_smem(gemv_tc_kernel<S, false>, smem);
             if (r != cudaSuccess) return r;
-            return launch_pdl(gemv_tc_kernel<S, false>, dim3(p.grid_x, p.ks), dim3(kTcThreads), smem, s, g, pk, c,
+            return launch_pdl(pdl, gemv_tc_kernel<S, false>, dim3(p.grid_x, p.ks), dim3(kTcThreads), smem, s, g, pk, c,
                               scales, x, batch, y, sk, ws, p.len);
         });
     }
@@ -1151,9 +1175,9 @@ cudaError_t launch_plan(const Geom &g, const GemvPlan &p, const void *packed, co
 
 cudaError_t launch_gemv(const Geom &g, const void *packed, const uint16_t *cb,
                         const uint16_t *scales, const uint16_t *x, int batch, uint16_t *y,
-                        void *ws, cudaStream_t s)
+                        void *ws, cudaStream_t s, bool pdl)
 {
-    return launch_plan(g, plan_gemv(g, batch), packed, cb, scales, x, batch, y, ws, s);
+    return launch_plan(g, plan_gemv(g, batch), packed, cb, scales, x, batch, y, ws, s, pdl);
 }
 
 // ---------------------------------------------------------------------------
@@ -1162,8 +1186,8 @@ cudaError_t launch_gemv(const Geom &g, const void *packed, const uint16_t *cb,
 // The split-K partial sums, arrival counters and status word live in one
 // file-scope device array (every GPU that loads this library holds it until
 // the process exits).  Host code must not hand the array's name to a kernel:
-// on the host it is only a stand-in, so its device address is looked up once
-// per device, with that device current, through cudaGetSymbolAddress.  All
+// on the host it is only a stand-in, so its device address is looked up
+// with cudaGetSymbolAddress, the device current, once per device and context.  All
 // calls share the array, so calls that overlap on the GPU race; each call
 // clears the status word and counters (cudaMemsetAsync on its stream) before
 // its kernel starts.
@@ -1172,24 +1196,71 @@ static __device__ __align__(256) unsigned char g_gemv_scratch[AQ_GEMV_NOALLOC_SC
 
 namespace {
 
-constexpr int kMaxDevices = 64;
-std::mutex g_scratch_mutex;
-void *g_scratch_ptr[kMaxDevices] = {};
+// The array's device address belongs to one CUDA context.  It is looked up
+// once per context (the runtime's primary context of a device, or another
+// context the caller made current) and kept with the context's id, which
+// the driver never reuses within a process: after cudaDeviceReset, or under
+// a different current context, the next call looks the address up again
+// instead of using a stale one.  The driver calls are fetched at run time,
+// so the library does not link the driver library itself.
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long *);
 
-cudaError_t scratch_for_current_device(void **out)
+// Id of the calling thread's current context, or 0 if there is none (or the
+// driver lacks the calls).
+unsigned long long current_context_id()
+{
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &f, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<CtxGetCurrentFn>(f);
+        f = nullptr;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &f, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<CtxGetIdFn>(f);
+        cudaGetLastError();  // a failed query leaves no sticky error behind
+    });
+    if (!get_current || !get_id) return 0;
+    CUcontext ctx = nullptr;
+    if (get_current(&ctx) != CUDA_SUCCESS || !ctx) return 0;
+    unsigned long long id = 0;
+    return get_id(ctx, &id) == CUDA_SUCCESS ? id : 0;
+}
+
+constexpr int kMaxDevices = 64;
+struct ScratchAddr {
+    unsigned long long ctx_id;  // 0: not looked up
+    void *ptr;
+};
+std::mutex g_scratch_mutex;
+ScratchAddr g_scratch_addr[kMaxDevices] = {};
+
+cudaError_t scratch_for_current_context(void **out)
 {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    const unsigned long long id = current_context_id();
     std::lock_guard<std::mutex> lock(g_scratch_mutex);
-    if (!g_scratch_ptr[dev]) {
-        void *p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_gemv_scratch);
-        if (e != cudaSuccess) return e;
-        g_scratch_ptr[dev] = p;
+    ScratchAddr &a = g_scratch_addr[dev];
+    if (id != 0 && a.ctx_id == id) {
+        *out = a.ptr;
+        return cudaSuccess;
     }
-    *out = g_scratch_ptr[dev];
+    // with this device current: the array's address in the current context
+    // (this also makes the device's primary context current if none was)
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_gemv_scratch);
+    if (e != cudaSuccess) return e;
+    a.ctx_id = id != 0 ? id : current_context_id();
+    a.ptr = p;
+    *out = p;
     return cudaSuccess;
 }
 
@@ -1203,14 +1274,14 @@ cudaError_t launch_gemv_noalloc(const Geom &g, const void *packed, const uint16_
     *too_large = p.ws_bytes > AQ_GEMV_NOALLOC_SCRATCH_BYTES;
     if (*too_large) return cudaSuccess;
     void *scratch = nullptr;
-    cudaError_t e = scratch_for_current_device(&scratch);
+    cudaError_t e = scratch_for_current_context(&scratch);
     if (e != cudaSuccess) return e;
     // status word and arrival counters must start at zero; the partials are
     // fully written before they are read
     const size_t clear = kWsHeader + align16(sizeof(unsigned) * (size_t)p.counters);
     e = cudaMemsetAsync(scratch, 0, clear, s);
     if (e != cudaSuccess) return e;
-    return launch_plan(g, p, packed, cb, scales, x, batch, y, scratch, s);
+    return launch_plan(g, p, packed, cb, scales, x, batch, y, scratch, s, true);
 }
 
 }  // namespace aqh

@@ -126,6 +126,12 @@ def workload(name: str) -> dict:
     if name == "llama2-7b-1x16":
         sp = LayerSpec(4096, 4096, 1, 16)
         return {"layers": [("4096x4096", sp)], "n": [1, 4, 16], "seed": 1001}
+    if name == "llama2-7b-decode":
+        # the decode-time products the headline metric covers: the 1x16
+        # 4096 x 4096 layer at batch 1, 4, 16 and the 2x8 MLP layers
+        # (uniform and Zipf codes) at batch 1 and 8, each part keeping its
+        # own batches and seed
+        return {"parts": ["llama2-7b-1x16", "llama2-7b-mlp-2x8"]}
     if name == "llama2-7b-mlp-2x8":
         layers = []
         for dist in ("uniform", "zipf"):
@@ -170,6 +176,15 @@ def workload(name: str) -> dict:
     raise KeyError(name)
 
 
-WORKLOADS = ("tiny-2x8", "llama2-7b-1x16", "llama2-7b-mlp-2x8",
+def workload_units(name: str) -> list:
+    """Flatten a workload into ``[(tag, spec, batches, seed), ...]`` (a
+    composite workload lists the parts it is made of)."""
+    wl = workload(name)
+    if "parts" in wl:
+        return [u for part in wl["parts"] for u in workload_units(part)]
+    return [(tag, spec, tuple(wl["n"]), wl["seed"]) for tag, spec in wl["layers"]]
+
+
+WORKLOADS = ("tiny-2x8", "llama2-7b-decode", "llama2-7b-1x16", "llama2-7b-mlp-2x8",
              "llama2-70b-1x16", "llama2-7b-prefill", "llama2-7b-block", "llama2-7b-schemes", "llama2-7b-grad",
              "llama2-7b-encode")

@@ -1,18 +1,25 @@
 """Benchmark of the additive-quantised decode-time product on B200.
 
-Workload: Llama-2-7B-shaped 1x16 layers (out = in = 4096, g = 8, K = 1,
-B = 16; 2 bits per weight), decode-time products at batch 1, 4 and 16.
+Default workload (``llama2-7b-decode``): the decode-time products the metric
+names, 1x16 and 2x8 at Llama-2-7B shapes --
+* 4096 x 4096 layers in 1x16 (K = 1, B = 16, g = 8; 2 bits per weight) at
+  batch 1, 4 and 16;
+* the MLP layers 11008 x 4096 and 4096 x 11008 in 2x8 (K = 2, B = 8), with
+  uniform and with Zipf(1.1)-skewed codes, at batch 1 and 8.
 One step = the product at each batch for every layer of a rotation set of
-distinct layers whose bytes exceed three times the L2 cache (codes and
-codebooks come from HBM, not L2), ordered batch-major so that a layer is
-re-read only after every other layer.  The timed region replays a CUDA graph
-of one step K times, bracketed by a barrier and device synchronisation;
-time comes from CUDA events on the launching stream, max over ranks.
+distinct copies per shape (about 4 GB of layer bytes per shape, 30x the L2
+cache, so codes and codebooks come from HBM, not L2), ordered batch-major
+so that a layer is re-read only after every other layer.  The timed region
+replays a CUDA graph of one step K times, bracketed by a barrier and device
+synchronisation; time comes from CUDA events on the launching stream, max
+over ranks.  Per-kernel times are the median over further replays of the
+same graph.
 
 Metric: achieved throughput of algorithmic bytes (codes + codebooks +
 scales + x + y per product; the dense matrix is never counted) in GB/s,
-plus microseconds per layer for each batch.  The roofline object reports
-the dominant kernel against the measured HBM copy bandwidth.
+plus microseconds per layer for each shape and batch.  The roofline object
+reports the dominant kernel against the measured HBM copy bandwidth, with
+the read-only HBM stream and the 1x16 codeword-read ceiling beside it.
 
 ``--impl reference`` times the CPU oracle (the plain fp64 C implementation
 the tests compare against) on a bounded sample of the same workload.
@@ -37,14 +44,12 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-from aq_inputs import LayerSpec, make_activations, make_layer  # noqa: E402
+from aq_inputs import LayerSpec, make_activations, make_layer, workload_units  # noqa: E402
 
 METRIC = "AQ-GEMV µs/layer & achieved HBM GB/s vs roofline (1x16, 2x8; batch 1–16)"
-WORKLOAD = "llama2-7b-1x16"
-SPEC = LayerSpec(4096, 4096, 1, 16)
-BATCHES = (1, 4, 16)
-SEED = 1001
+WORKLOAD = "llama2-7b-decode"
 L2_BYTES = 126 * 1024 * 1024
+ROTATION_BYTES = 4e9  # layer bytes per shape in the rotation set of a decode step
 
 
 def alg_bytes(spec: LayerSpec, n: int) -> int:
@@ -120,7 +125,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
@@ -171,24 +176,49 @@ class ClockSampler:
 _SAMPLE_INPUTS = {}
 
 
-def oracle_sample(rows: int, threads: int, repeats: int = 1):
-    """Time the oracle on ``rows`` rows of one layer at every batch.
+def _sample_layer(tag, spec, seed):
+    key = (tag, seed)
+    if key not in _SAMPLE_INPUTS:
+        _SAMPLE_INPUTS[key] = make_layer(spec, (seed, 0))
+    return _SAMPLE_INPUTS[key]
+
+
+def oracle_sample(units, frac: float, threads: int):
+    """Time the oracle on the first ``frac`` of the rows (at least 8) of one
+    layer of each unit, at each of the unit's batches.
 
     Returns (seconds, algorithmic bytes the sample stands for)."""
     import oracle
-    if not _SAMPLE_INPUTS:
-        _SAMPLE_INPUTS["layer"] = make_layer(SPEC, (SEED, 0, 0))
-        _SAMPLE_INPUTS["xs"] = {b: make_activations(SPEC.in_features, b, (SEED, 0, b)) for b in BATCHES}
-    layer, xs = _SAMPLE_INPUTS["layer"], _SAMPLE_INPUTS["xs"]
-    sel = np.arange(rows, dtype=np.int64)
-    frac = rows / SPEC.out_features
-    t0 = time.perf_counter()
-    for _ in range(repeats):
-        for b in BATCHES:
-            oracle.matmul(layer.codes, layer.codebooks, layer.scales, xs[b], rows=sel, threads=threads)
-    dt = time.perf_counter() - t0
-    nbytes = repeats * sum(alg_bytes(SPEC, b) for b in BATCHES) * frac
+    dt = nbytes = 0.0
+    for tag, spec, batches, seed in units:
+        layer = _sample_layer(tag, spec, seed)
+        rows = int(min(spec.out_features, max(8, round(frac * spec.out_features))))
+        sel = np.arange(rows, dtype=np.int64)
+        for b in batches:
+            x = make_activations(spec.in_features, b, (seed, 0, b))
+            t0 = time.perf_counter()
+            oracle.matmul(layer.codes, layer.codebooks, layer.scales, x, rows=sel, threads=threads)
+            dt += time.perf_counter() - t0
+            nbytes += alg_bytes(spec, b) * rows / spec.out_features
     return dt, nbytes
+
+
+def _sized_sample(units, threads: int, budget_s: float):
+    """Row fraction whose oracle sample takes about ``budget_s`` seconds."""
+    f = 1.0 / 512
+    for _ in range(3):  # small samples carry a fixed cost: re-measure nearer the target
+        dt, _ = oracle_sample(units, f, threads)
+        target = min(1.0, f * budget_s / max(dt, 1e-4))
+        if target <= 4 * f:
+            return float(target)
+        f = target / 4
+    return float(target)
+
+
+def _describe(units, frac: float) -> str:
+    parts = [f"{tag} {spec.scheme} b{'/'.join(map(str, n))}" for tag, spec, n, _ in units]
+    return (f"first {frac:.2%} of the rows (at least 8) of one layer of each shape: " + "; ".join(parts)
+            + " (fp64 C oracle, OpenMP over rows), scaled to the layers' algorithmic bytes")
 
 
 def cpu_model() -> str:
@@ -201,22 +231,16 @@ def cpu_model() -> str:
     return "unknown"
 
 
-def cpu_baseline(budget_s: float = 10.0, single_budget_s: float = 3.0) -> dict:
+def cpu_baseline(units, budget_s: float = 10.0, single_budget_s: float = 3.0) -> dict:
     import oracle
     threads = os.cpu_count() or 1
-    # calibrate on a small sample, then size the measured sample to the budget
-    dt, _ = oracle_sample(64, threads)
-    rows = int(min(SPEC.out_features, max(64, 64 * budget_s / max(dt, 1e-3))))
-    dt, nbytes = oracle_sample(rows, threads)
-    # the same at one thread, on a smaller sample
-    dt1, _ = oracle_sample(8, 1)
-    rows1 = int(min(SPEC.out_features, max(8, 8 * single_budget_s / max(dt1, 1e-3))))
-    dt1, nbytes1 = oracle_sample(rows1, 1)
+    frac = _sized_sample(units, threads, budget_s)
+    dt, nbytes = oracle_sample(units, frac, threads)
+    frac1 = _sized_sample(units, 1, single_budget_s)
+    dt1, nbytes1 = oracle_sample(units, frac1, 1)
     return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": min(threads, oracle.max_threads()),
-            "kind": "oracle",
-            "sample": f"{rows} of {SPEC.out_features} rows of one 4096x4096 1x16 layer at batch "
-                      f"1, 4, 16 (fp64 C oracle, OpenMP over rows), scaled to the layer's bytes",
-            "single_thread": {"value": nbytes1 / dt1 / 1e9, "sample_rows": rows1},
+            "kind": "oracle", "sample": _describe(units, frac),
+            "single_thread": {"value": nbytes1 / dt1 / 1e9, "row_fraction": round(frac1, 5)},
             "nproc": threads, "cpu_model": cpu_model()}
 
 
@@ -226,13 +250,13 @@ def run_reference(args) -> None:
         return
     import oracle
     threads = os.cpu_count() or 1
-    dt, _ = oracle_sample(32, threads)
-    rows = int(min(SPEC.out_features, max(16, 32 * 2.0 / max(dt, 1e-3))))  # ~2 s per step
+    units = workload_units(args.workload)
+    frac = _sized_sample(units, threads, 2.0)  # ~2 s of oracle work per step
     for _ in range(args.warmup):
-        oracle_sample(rows, threads)
+        oracle_sample(units, frac, threads)
     total_t, total_b = 0.0, 0.0
     for _ in range(args.steps):
-        dt, nb = oracle_sample(rows, threads)
+        dt, nb = oracle_sample(units, frac, threads)
         total_t += dt
         total_b += nb
     value = total_b / total_t / 1e9
@@ -242,10 +266,12 @@ def run_reference(args) -> None:
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * total_t / max(args.steps, 1), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "layer": "4096x4096 1x16 g8", "batches": list(BATCHES),
-                   "sample_rows_per_step": rows},
+        "config": {"workload": args.workload,
+                   "layers": [f"{tag} {spec.scheme} g8" for tag, spec, _, _ in units],
+                   "batches": {tag: list(n) for tag, _, n, _ in units},
+                   "row_fraction_per_step": round(frac, 5)},
         "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
-                         "sample": f"{rows} rows of one 4096x4096 1x16 layer at batch 1, 4, 16 per step"},
+                         "sample": _describe(units, frac) + ", per step"},
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -275,14 +301,17 @@ def count_graph_kernels(graph) -> int:
     return count
 
 
-def recorded_traffic(workload_name: str, batch: int):
-    """DRAM bytes per launch from the committed ncu record, or None when the
-    kernel sources changed since the counters were taken."""
+def recorded_traffic(layer: str, batch: int):
+    """DRAM bytes per launch of the product on ``layer`` at ``batch`` from
+    the committed ncu record, or None when there is none or the kernel
+    sources changed since the counters were taken."""
     import hashlib
     p = os.path.join(ROOT, "profiles", "traffic_gemv_tc.json")
-    if workload_name != WORKLOAD or not os.path.exists(p):
+    if not os.path.exists(p):
         return None
     rec = json.load(open(p))
+    if layer != rec.get("layer"):
+        return None
     h = hashlib.sha256()
     for f in rec["sources"]:
         h.update(open(os.path.join(ROOT, f), "rb").read())
@@ -373,6 +402,31 @@ def gather_ceiling(aq, units, kernels, stream, reps: int = 5):
     return rows or None
 
 
+def hbm_read_probe(aq, dev, stream, copy_gbs: float, nbytes: int = 4 << 30, reps: int = 7) -> dict:
+    """Read-only HBM bandwidth: aq_gather_probe mode 3 streams one array of
+    ``nbytes`` (32x the L2 cache) once per call; median of ``reps`` calls
+    timed with CUDA events on the launching stream."""
+    import torch
+    buf = torch.empty(nbytes, dtype=torch.uint8, device=dev)  # contents do not matter
+    sink = torch.zeros(aq.aq_gather_probe_sink_bytes(3) // 4, dtype=torch.int32, device=dev)
+    n = nbytes // 2
+    times = []
+    with torch.cuda.stream(stream):
+        aq.aq_gather_probe(None, buf, n, 3, sink, stream=stream)
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            aq.aq_gather_probe(None, buf, n, 3, sink, stream=stream)
+            e1.record(stream)
+            e1.synchronize()
+            times.append(e0.elapsed_time(e1) * 1e-3)
+    del buf
+    gbs = nbytes / statistics.median(times) / 1e9
+    return {"gbs": round(gbs, 1), "bytes": nbytes, "reps": reps, "vs_copy_peak": round(gbs / copy_gbs, 4),
+            "how": "aq_gather_probe mode 3: one 4 GiB array read once per call with 16-byte loads, "
+                   "median of CUDA-event times"}
+
+
 def run_gpu(args) -> None:
     import torch
 
@@ -384,6 +438,7 @@ def run_gpu(args) -> None:
     dist = init_dist(world, "nccl")
     dev = torch.device("cuda", local)
     wl = workload(args.workload)
+    layer_units = workload_units(args.workload)
     op = {"llama2-7b-prefill": "gemm", "llama2-7b-grad": "grad", "llama2-7b-encode": "encode"}.get(args.workload, "gemv")
     tensor_op = op in ("gemm", "grad")  # reported in TFLOP/s against the tensor peak
     alu_op = op == "encode"             # fp32 CUDA-core work, reported against the derived fp32 FMA peak
@@ -402,22 +457,23 @@ def run_gpu(args) -> None:
         return desc, packed, cb, sc
 
     units = []
-    for si, (tag, spec) in enumerate(wl["layers"]):
-        desc, packed0, cb0, sc0 = device_layer(spec, (wl["seed"], rank, si))  # seeded per rank and shape
+    rotation = max(3 * L2_BYTES, args.rotation_gb * 1e9)
+    for si, (tag, spec, batches, seed) in enumerate(layer_units):
+        desc, packed0, cb0, sc0 = device_layer(spec, (seed, rank, si))  # seeded per rank and shape
         lb = alg_bytes(spec, 0)
-        ncopies = args.layers or (1 if alu_op else 3 if tensor_op else max(4, int(3 * L2_BYTES / lb) + 1))
+        ncopies = args.layers or (1 if alu_op else 3 if tensor_op else max(4, int(rotation / lb) + 1))
         copies = [(packed0.clone(), cb0.clone(), sc0.clone()) for _ in range(ncopies)]
         del packed0, cb0, sc0
-        for n in wl["n"]:
-            x = torch.from_numpy(make_activations(spec.in_features, n, (wl["seed"], rank, si, n)).view(np.int16)).to(dev)
+        for n in batches:
+            x = torch.from_numpy(make_activations(spec.in_features, n, (seed, rank, si, n)).view(np.int16)).to(dev)
             nbytes = {"gemm": aq.aq_gemm_workspace_bytes, "grad": aq.aq_param_grad_workspace_bytes,
                       "gemv": aq.aq_gemv_workspace_bytes,
                       "encode": lambda d, n: aq.aq_encode_workspace_bytes(d)}[op](desc, n)
             units.append({
                 "tag": tag, "spec": spec, "n": n, "desc": desc, "copies": copies, "x": x,
                 "bytes": alg_bytes(spec, n), "flops": encode_flops(spec, n) if op == "encode" else flops(spec, n),
-                **(encode_inputs(spec, n, (wl["seed"], rank, si)) if op == "encode" else {}),
-                **({"gy": torch.from_numpy(make_activations(spec.out_features, n, (wl["seed"], rank, si, n, 1))
+                **(encode_inputs(spec, n, (seed, rank, si)) if op == "encode" else {}),
+                **({"gy": torch.from_numpy(make_activations(spec.out_features, n, (seed, rank, si, n, 1))
                                            .view(np.int16)).to(dev),
                     "grad_s": torch.empty(spec.out_features, dtype=torch.float32, device=dev),
                     "grad_cb": torch.empty((spec.num_codebooks << spec.nbits) * 8, dtype=torch.float32, device=dev)}
@@ -527,20 +583,30 @@ def run_gpu(args) -> None:
     if dist is not None:
         dist.barrier()
     elapsed_ms = max_over_ranks(t_start.elapsed_time(t_stop), dist, dev)
+
+    # per-kernel times: average duration per launch of each group of
+    # same-shape launches (events on the launching stream), median over
+    # further replays of the same graph
+    per_unit = [[] for _ in units]
+    with torch.cuda.stream(stream):
+        for _ in range(max(1, args.median_replays)):
+            graph.replay()
+            torch.cuda.synchronize()
+            for ui, u in enumerate(units):
+                per_unit[ui].append(1e3 * u["evs"][0].elapsed_time(u["evs"][1]) / len(u["copies"]))
     status_ok = all(aq.aq_workspace_status(u["ws"]) == 0 for u in units)
 
-    # average duration per launch of each group, from the last replay inside
-    # the timed region (events on the launching stream)
     kernels = []
     step_bytes = step_flops = 0
-    for u in units:
-        us = 1e3 * u["evs"][0].elapsed_time(u["evs"][1]) / len(u["copies"])
+    for u, times in zip(units, per_unit):
+        us = statistics.median(times)
         nb, nf = u["bytes"], u["flops"]
         step_bytes += nb * len(u["copies"])
         step_flops += nf * len(u["copies"])
         k = {"layer": u["tag"], "n": u["n"], "us_per_layer": round(us, 3),
              "gbs": round(nb / (us * 1e-6) / 1e9, 1), "tflops": round(nf / (us * 1e-6) / 1e12, 2),
-             "bytes_per_call": nb, "copies": len(u["copies"]), "total_us": us * len(u["copies"])}
+             "bytes_per_call": nb, "copies": len(u["copies"]), "total_us": us * len(u["copies"]),
+             "us_range": [round(min(times), 3), round(max(times), 3)]}
         if "chain" in u:  # one call is a whole block of layers
             k["layers_per_call"] = len(u["chain"])
             k["us_per_block"] = k.pop("us_per_layer")
@@ -569,11 +635,15 @@ def run_gpu(args) -> None:
         value = world * step_bytes * args.steps / (elapsed_ms * 1e-3) / 1e9
         unit = "GB/s"
         roofline = {"bound": "hbm", "achieved": dom["gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                    "frac": dom["frac_hbm"], "traffic": recorded_traffic(args.workload, dom["n"]),
+                    "frac": dom["frac_hbm"], "traffic": recorded_traffic(dom["layer"], dom["n"]),
                     "kernel": f"aq_gemv {dom['layer']} batch {dom['n']}",
                     "peak_source": f"{peaks['source']} hbm_gbs (STREAM-style copy)"}
     for k in kernels:
         del k["total_us"]
+
+    # ---- read-only HBM stream beside the copy figure of the peak -------------
+    if op == "gemv" and not args.skip_hbm_probe:
+        roofline["hbm_read_probe"] = hbm_read_probe(aq, dev, stream, peaks["hbm_gbs"])
 
     # ---- codeword-read ceiling of the 1x16 shapes (secondary bound) ----------
     if op == "gemv" and not args.skip_ceiling:
@@ -621,11 +691,11 @@ def run_gpu(args) -> None:
                "api": "additive_quantized_matmul_b200 (C ABI via ctypes), eager, pinned host buffers"}
 
     cpu = None
-    if rank == 0 and world == 1 and not args.skip_cpu and args.workload == WORKLOAD:
-        cpu = cpu_baseline()
+    if rank == 0 and world == 1 and not args.skip_cpu and op == "gemv" and layer_units:
+        cpu = cpu_baseline(layer_units)
 
     if rank == 0:
-        shapes = [f"{t} {sp.scheme} g8" for t, sp in wl["layers"]]
+        shapes = [f"{t} {sp.scheme} g8" for t, sp, _, _ in layer_units]
         shapes += [f"{t}: " + ", ".join(f"{lt} {sp.out_features}x{sp.in_features} {sp.scheme}" for lt, sp, _ in ch)
                    for t, ch in wl.get("chains", [])]
         line = {
@@ -636,20 +706,22 @@ def run_gpu(args) -> None:
             "data": "synthetic",
             "config": {"workload": args.workload,
                        "layers": shapes,
-                       "n": list(wl["n"]),
-                       "copies_per_shape": [len(u["copies"]) for u in units[::len(wl["n"])]],
+                       "n": {t: list(n) for t, _, n, _ in layer_units} if layer_units else [1],
+                       "copies_per_shape": {u["tag"]: len(u["copies"]) for u in units},
                        **({"chain": "per block: q, k, v read the block input; o reads v; gate and up "
                                     "read o; down reads up (one stream, each launch waits on the previous)"}
                           if wl.get("chains") else {}),
                        "l2": "inputs larger than L2: per shape, copies at distinct addresses whose "
-                             "bytes exceed 3x the 126 MB L2, visited in turn before any is re-read",
+                             "bytes exceed 3x the 126 MB L2 (about 4 GB per decode-time shape), visited in "
+                             "turn before any is re-read",
+                       "kernel_times": f"median over {max(1, args.median_replays)} replays of the step's graph",
                        "parallelism": f"replicas x{world} (independent layers per rank)"},
             "kernels": kernels, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "clocks": sampler.summary(), "status_ok": status_ok,
             "gpu_launches": launches_per_step * args.steps,
         }
-        if op == "gemv" and args.workload == WORKLOAD:
-            line["us_per_layer"] = {str(k["n"]): k["us_per_layer"] for k in kernels}
+        if op == "gemv" and layer_units:
+            line["us_per_layer"] = {f"{k['layer']} b{k['n']}": k["us_per_layer"] for k in kernels}
         print(json.dumps(line), flush=True)
     del graph
     if dist is not None:
@@ -665,10 +737,15 @@ def main():
                     help="do not time the 1x16 codeword-read ceiling (aq_gather_probe)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=WORKLOAD,
-                    help="llama2-7b-1x16 (default), llama2-7b-mlp-2x8, llama2-70b-1x16, "
+                    help="llama2-7b-decode (default), llama2-7b-1x16, llama2-7b-mlp-2x8, llama2-70b-1x16, "
                          "llama2-7b-prefill, llama2-7b-block, llama2-7b-schemes, llama2-7b-grad, "
                          "llama2-7b-encode, tiny-2x8")
-    ap.add_argument("--layers", type=int, default=0, help="copies per shape (0: > 3x L2)")
+    ap.add_argument("--layers", type=int, default=0, help="copies per shape (0: --rotation-gb of layer bytes)")
+    ap.add_argument("--rotation-gb", type=float, default=ROTATION_BYTES / 1e9,
+                    help="layer bytes per shape in the rotation set of a decode step (at least 3x L2)")
+    ap.add_argument("--median-replays", type=int, default=10,
+                    help="replays of the step's graph after the timed region for per-kernel medians")
+    ap.add_argument("--skip-hbm-probe", action="store_true", help="do not time the read-only HBM stream")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--skip-cpu", action="store_true")

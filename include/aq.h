@@ -176,10 +176,31 @@ aq_status aq_dequant(const aq_layer_desc *desc, const void *packed, const uint16
  *   workspace >= aq_gemv_workspace_bytes(desc, batch) bytes (see above)
  * Results are deterministic: the same inputs give the same bits.
  * AQ_ERR_INVALID_ARG for batch outside 1..16.
+ * Early weight reads: this kernel is launched with programmatic dependent
+ * launch and may read `packed` and `codebooks` before the kernel launched
+ * just before it on `stream` has finished (x, scales, y and the workspace
+ * only after).  That is safe whenever the previous kernel does not write
+ * this layer's packed codes or codebooks, or does not let its dependents
+ * start early (griddepcontrol.launch_dependents / cudaTriggerProgrammatic-
+ * LaunchCompletion) -- every kernel of this library and every kernel that
+ * does not use programmatic launch qualifies.  A caller whose own kernel
+ * triggers its dependents early and then rewrites these weights (a
+ * fine-tuning step, for instance) must write them before the trigger, or
+ * call aq_gemv_ordered instead.
  */
 aq_status aq_gemv(const aq_layer_desc *desc, const void *packed, const uint16_t *codebooks,
                   const uint16_t *scales, const uint16_t *x, int batch, uint16_t *y,
                   void *workspace, size_t workspace_bytes, aq_stream_t stream);
+
+/*
+ * aq_gemv with an ordinary launch: the kernel starts only after all work
+ * queued before it on `stream` has completed, so it reads no weight early.
+ * Same arguments, plan and results (bit for bit) as aq_gemv; it gives up
+ * the overlap of a launch with the end of the previous one.
+ */
+aq_status aq_gemv_ordered(const aq_layer_desc *desc, const void *packed, const uint16_t *codebooks,
+                          const uint16_t *scales, const uint16_t *x, int batch, uint16_t *y,
+                          void *workspace, size_t workspace_bytes, aq_stream_t stream);
 
 /*
  * aq_gemv without a workspace argument, for callers that cannot allocate
@@ -188,28 +209,31 @@ aq_status aq_gemv(const aq_layer_desc *desc, const void *packed, const uint16_t 
  * plugins handed only input and output buffers.  The paper has no
  * counterpart; this is an interface convenience.
  *
- * Same arguments and results as aq_gemv, minus the workspace.  Where
+ * Same arguments and results as aq_gemv, minus the workspace (including
+ * aq_gemv's rule on early weight reads).  Where
  * aq_gemv's split-K partial sums would not fit the scratch, this call splits
  * the sum more coarsely (on the tensor-core path, down to one CTA per 128
- * rows), so its y agrees with aq_gemv's within rounding rather than bit for
- * bit; it is deterministic run to run.  The split-K scratch is a fixed
- * device array inside the library of
+ * rows, which needs no partial sums; 8-bit codebooks at batch 1 then leave
+ * the table path for the tensor-core path), so its y agrees with aq_gemv's
+ * within rounding rather than bit for bit; it is deterministic run to run.
+ * The split-K scratch is a fixed device array inside the library of
  * AQ_GEMV_NOALLOC_SCRATCH_BYTES bytes, which every GPU that loads the
  * library holds until the process exits.  The call allocates nothing (no
  * cudaMalloc/cudaFree, no allocating library routine); it clears the part
  * of the array that must start at zero with cudaMemsetAsync on `stream`.
- *  - The first call on each device looks up the array's device address
- *    (cudaGetSymbolAddress, with that device current); make that first call
- *    before any stream capture on that device.
+ *  - The first call in each CUDA context of a device (the device's primary
+ *    context, or a context the caller made current) looks up the array's
+ *    device address (cudaGetSymbolAddress, with that device current) and
+ *    keeps it with the context's id; make that first call before any stream
+ *    capture on that device.  After cudaDeviceReset or under another
+ *    context the next call looks the address up again.
  *  - Every call shares the one array and it keeps the last call's contents:
  *    calls whose kernels may overlap on the GPU (different streams) race and
  *    give wrong results.  Serialise them, or use aq_gemv with a workspace
  *    per stream.
- *  - AQ_ERR_WORKSPACE if the layer and batch need more scratch than the
- *    array holds even at the coarsest split; nothing is launched then.
- *    Only the batch-1 table path of 8-bit codebooks (one partial sum per
- *    row and 32-group block) can need that much: it is refused when
- *    aq_gemv_workspace_bytes(desc, 1) exceeds AQ_GEMV_NOALLOC_SCRATCH_BYTES.
+ *  - AQ_ERR_WORKSPACE if the layer needs more scratch than the array holds
+ *    even at the coarsest split (one arrival counter per 128 rows: more
+ *    than about 134 million rows); nothing is launched then.
  *  - A bounded wait that gives up inside the kernel cannot be reported (the
  *    status word is internal): use aq_gemv when that report is needed.
  */
@@ -305,8 +329,14 @@ aq_status aq_param_grad(const aq_layer_desc *desc, const void *packed, const uin
  *           thread-block clusters (128 KiB per CTA, loaded once per call)
  *           with distributed shared-memory loads;
  *   mode 2  into registers through L1 (ld.global.nc), as aq_gemv's batch-1
- *           1x16 path does (three CTAs of 256 threads per SM).
- *   codebook  [65536][8] binary16, device, 16-byte aligned,
+ *           1x16 path does (three CTAs of 256 threads per SM);
+ *   mode 3  no codeword at all: `codes` itself is read once as a stream of
+ *           16-byte loads (L1 bypassed, four CTAs of 256 threads per SM),
+ *           the read-only HBM bandwidth when the array is much larger
+ *           than L2 (a cross-check of the copy bandwidth the HBM roofline
+ *           uses).  `codebook` is not read and may be NULL; the checksum
+ *           XOR is then that of the codes' 32-bit words.
+ *   codebook  [65536][8] binary16, device, 16-byte aligned (modes 0-2),
  *   codes     n 16-bit codes, device, 16-byte aligned, n a multiple of 8
  *             (a 1x16 layer's packed codes are such an array),
  *   sink      device, >= aq_gather_probe_sink_bytes(mode) bytes, 16-byte

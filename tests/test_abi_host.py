@@ -111,31 +111,32 @@ def test_workspace_sizes_host_only():
     assert aq.aq_gemm_workspace_bytes(d, 0) == 0
 
 
-def _gemv(d, packed=FAKE, cb=FAKE, s=FAKE, x=FAKE, batch=1, y=FAKE, ws=FAKE, wsb=1 << 30):
-    return aq.lib.aq_gemv(ctypes.byref(d), packed, cb, s, x, batch, y, ws, wsb, None)
+def _gemv(d, packed=FAKE, cb=FAKE, s=FAKE, x=FAKE, batch=1, y=FAKE, ws=FAKE, wsb=1 << 30, fn="aq_gemv"):
+    return getattr(aq.lib, fn)(ctypes.byref(d), packed, cb, s, x, batch, y, ws, wsb, None)
 
 
 def _gemm(d, packed=FAKE, cb=FAKE, s=FAKE, x=FAKE, T=64, y=FAKE, ws=FAKE, wsb=1 << 30):
     return aq.lib.aq_gemm(ctypes.byref(d), packed, cb, s, x, T, y, ws, wsb, None)
 
 
-def test_gemv_argument_errors():
+@pytest.mark.parametrize("fn", ["aq_gemv", "aq_gemv_ordered"])
+def test_gemv_argument_errors(fn):
     d = aq.LayerDesc.make(64, 256, 2, 8)
-    assert _gemv(None if False else d, batch=0) == 1
-    assert _gemv(d, batch=17) == 1
-    assert _gemv(d, packed=None) == 1
-    assert _gemv(d, cb=None) == 1
-    assert _gemv(d, x=None) == 1
-    assert _gemv(d, y=None) == 1
-    assert _gemv(d, packed=FAKE + 8) == 3
-    assert _gemv(d, x=FAKE + 2) == 3
-    assert _gemv(d, y=FAKE + 4) == 3
-    assert _gemv(d, cb=FAKE + 1) == 3
-    assert _gemv(d, s=FAKE + 1) == 3
-    assert _gemv(d, ws=None) == 4
-    assert _gemv(d, wsb=8) == 4
-    assert _gemv(d, ws=FAKE + 8) == 3
-    assert aq.lib.aq_gemv(None, FAKE, FAKE, FAKE, FAKE, 1, FAKE, FAKE, 1 << 20, None) == 1
+    assert _gemv(d, batch=0, fn=fn) == 1
+    assert _gemv(d, batch=17, fn=fn) == 1
+    assert _gemv(d, packed=None, fn=fn) == 1
+    assert _gemv(d, cb=None, fn=fn) == 1
+    assert _gemv(d, x=None, fn=fn) == 1
+    assert _gemv(d, y=None, fn=fn) == 1
+    assert _gemv(d, packed=FAKE + 8, fn=fn) == 3
+    assert _gemv(d, x=FAKE + 2, fn=fn) == 3
+    assert _gemv(d, y=FAKE + 4, fn=fn) == 3
+    assert _gemv(d, cb=FAKE + 1, fn=fn) == 3
+    assert _gemv(d, s=FAKE + 1, fn=fn) == 3
+    assert _gemv(d, ws=None, fn=fn) == 4
+    assert _gemv(d, wsb=8, fn=fn) == 4
+    assert _gemv(d, ws=FAKE + 8, fn=fn) == 3
+    assert getattr(aq.lib, fn)(None, FAKE, FAKE, FAKE, FAKE, 1, FAKE, FAKE, 1 << 20, None) == 1
 
 
 def test_gemm_argument_errors():
@@ -177,7 +178,9 @@ def test_gemv_noalloc_argument_errors():
     assert f(ctypes.byref(d), None, FAKE, FAKE, FAKE, 1, FAKE, None) == 1
     assert f(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE + 8, 1, FAKE, None) == 3
     assert f(None, FAKE, FAKE, FAKE, FAKE, 1, FAKE, None) == 1
-    big = aq.LayerDesc.make(32768, 65536, 2, 8)  # needs more scratch than the fixed array
+    # even one CTA per 128 rows needs an arrival counter per 128 rows: 2^28
+    # rows need more scratch than the fixed array (refused before any launch)
+    big = aq.LayerDesc.make(1 << 28, 8, 1, 16)
     assert aq.aq_gemv_workspace_bytes(big, 1) > aq.GEMV_NOALLOC_SCRATCH_BYTES
     assert f(ctypes.byref(big), FAKE, FAKE, FAKE, FAKE, 1, FAKE, None) == 4
 
@@ -226,9 +229,12 @@ def test_encode_argument_errors():
 
 def test_gather_probe_argument_errors():
     f = aq.lib.aq_gather_probe
-    assert all(aq.aq_gather_probe_sink_bytes(m) > 0 for m in (0, 1, 2))
-    assert aq.aq_gather_probe_sink_bytes(3) == 0 and aq.aq_gather_probe_sink_bytes(-1) == 0
-    assert f(FAKE, FAKE, 64, 3, FAKE, None) == 1       # unknown mode
+    assert all(aq.aq_gather_probe_sink_bytes(m) > 0 for m in (0, 1, 2, 3))
+    assert aq.aq_gather_probe_sink_bytes(4) == 0 and aq.aq_gather_probe_sink_bytes(-1) == 0
+    assert f(FAKE, FAKE, 64, 4, FAKE, None) == 1       # unknown mode
+    assert f(None, None, 64, 3, FAKE, None) == 1       # the stream mode still needs codes
+    assert f(None, FAKE, 64, 3, None, None) == 1       # and a sink
+    assert f(None, FAKE + 8, 64, 3, FAKE, None) == 3   # misaligned codes (no codebook needed)
     assert f(FAKE, FAKE, 0, 0, FAKE, None) == 1        # no codes
     assert f(FAKE, FAKE, 12, 0, FAKE, None) == 1       # n not a multiple of 8
     assert f(None, FAKE, 64, 0, FAKE, None) == 1

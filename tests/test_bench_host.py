@@ -21,25 +21,33 @@ def test_algorithmic_bytes_of_the_default_layer():
 
 
 def test_traffic_record_only_while_the_sources_match(tmp_path, monkeypatch):
+    import hashlib
     rec = json.load(open(os.path.join(ROOT, "profiles", "traffic_gemv_tc.json")))
-    assert set(rec["per_launch_bytes"]) == {"1", "4", "16"}
-    for b in (1, 4, 16):
-        assert bench.recorded_traffic(bench.WORKLOAD, b) == rec["per_launch_bytes"][str(b)]
-    assert bench.recorded_traffic("llama2-70b-1x16", 1) is None
-    # a copy of the repository whose kernel source differs gives no traffic
+    assert set(rec["per_launch_bytes"]) == {"1", "4", "16"} and rec["layer"] == "4096x4096"
+    # a copy of the repository whose record was taken on its current sources
     fake = tmp_path / "repo"
     (fake / "profiles").mkdir(parents=True)
-    (fake / "profiles" / "traffic_gemv_tc.json").write_text(json.dumps(rec))
+    h = hashlib.sha256()
     for f in rec["sources"]:
         dst = fake / f
         dst.parent.mkdir(parents=True, exist_ok=True)
-        dst.write_bytes(open(os.path.join(ROOT, f), "rb").read() + (b"\n// changed\n" if f.endswith("gemv.cu") else b""))
+        data = open(os.path.join(ROOT, f), "rb").read()
+        dst.write_bytes(data)
+        h.update(data)
+    rec = dict(rec, sources_sha256=h.hexdigest())
+    (fake / "profiles" / "traffic_gemv_tc.json").write_text(json.dumps(rec))
     monkeypatch.setattr(bench, "ROOT", str(fake))
-    assert bench.recorded_traffic(bench.WORKLOAD, 1) is None
+    for b in (1, 4, 16):
+        assert bench.recorded_traffic("4096x4096", b) == rec["per_launch_bytes"][str(b)]
+    assert bench.recorded_traffic("8192x8192", 1) is None  # another layer
+    # once a kernel source changes, the record no longer counts
+    gemv = next(f for f in rec["sources"] if f.endswith("gemv.cu"))
+    (fake / gemv).write_bytes(open(os.path.join(ROOT, gemv), "rb").read() + b"\n// changed\n")
+    assert bench.recorded_traffic("4096x4096", 1) is None
 
 
 def test_cpu_baseline_fields():
-    r = bench.cpu_baseline(budget_s=0.05, single_budget_s=0.02)
+    r = bench.cpu_baseline(bench.workload_units(bench.WORKLOAD), budget_s=0.05, single_budget_s=0.02)
     for k in ("value", "unit", "cores", "kind", "sample", "single_thread", "nproc", "cpu_model"):
         assert k in r
     assert r["kind"] == "oracle" and r["unit"] == "GB/s"

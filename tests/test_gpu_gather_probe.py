@@ -1,10 +1,13 @@
-"""aq_gather_probe: the codeword-read ceiling of the 1x16 product (modes 0-2).
+"""aq_gather_probe: the codeword-read ceiling of the 1x16 product (modes 0-2)
+and the read-only HBM stream (mode 3).
 
-The probe reads codebook[codes[i]] for every code and XORs each 32-bit word
-it reads into a per-thread checksum.  These tests check, through the C ABI,
-that both modes read exactly the codewords the codes select: the XOR of all
+Modes 0-2 read codebook[codes[i]] for every code and XOR each 32-bit word
+they read into a per-thread checksum.  These tests check, through the C ABI,
+that each mode reads exactly the codewords the codes select: the XOR of all
 checksums must equal the XOR of those codewords, computed here with numpy
-from the same inputs (a property of the data, not of the method).
+from the same inputs (a property of the data, not of the method).  Mode 3
+reads the code array itself once: its checksums XOR to the XOR of the
+array's 32-bit words.
 """
 import numpy as np
 import pytest
@@ -50,3 +53,17 @@ def test_probe_back_to_back_calls_keep_the_checksum():
     torch.cuda.synchronize()
     got = np.bitwise_xor.reduce(sink.cpu().numpy().view(np.uint32).reshape(-1, 4), axis=0)
     assert np.array_equal(got, _expected_xor(cb_words, codes))
+
+
+@pytest.mark.parametrize("n", [8, 8 * 592 * 256 * 8, 8 * 592 * 256 * 8 * 3 + 8 * 4099, (1 << 26) + 8 * 5])
+def test_stream_probe_reads_every_word_once(n):
+    rng = np.random.default_rng(n)
+    codes = rng.integers(0, 65536, size=n, dtype=np.int64).astype(np.uint16)
+    cd = torch.from_numpy(codes.view(np.int16)).cuda()
+    sink = torch.zeros(aq.aq_gather_probe_sink_bytes(3) // 4, dtype=torch.int32, device="cuda")
+    aq.aq_gather_probe(None, cd, n, 3, sink)
+    aq.aq_gather_probe(None, cd, n, 3, sink)  # a second call rewrites the same checksums
+    torch.cuda.synchronize()
+    got = np.bitwise_xor.reduce(sink.cpu().numpy().view(np.uint32).reshape(-1, 4), axis=0)
+    want = np.bitwise_xor.reduce(codes.view(np.uint32).reshape(-1, 4), axis=0)
+    assert np.array_equal(got, want)

@@ -5,7 +5,7 @@ named workloads carry the Llama-2 layer shapes."""
 import numpy as np
 import pytest
 
-from aq_inputs import WORKLOADS, LayerSpec, make_activations, make_layer, workload
+from aq_inputs import WORKLOADS, LayerSpec, make_activations, make_layer, workload, workload_units
 
 
 def test_same_seed_same_bytes_other_seed_other_bytes():
@@ -78,12 +78,19 @@ def test_named_workloads_have_llama2_shapes():
     dims = {4096, 11008, 8192, 28672, 1024, 256, 512}
     for name in WORKLOADS:
         wl = workload(name)
-        specs = [sp for _, sp in wl["layers"]] + [sp for _, chain in wl.get("chains", []) for _, sp, _ in chain]
+        specs = [sp for _, sp, _, _ in workload_units(name)] + [
+            sp for _, chain in wl.get("chains", []) for _, sp, _ in chain]
         assert specs, name
         for sp in specs:
             assert sp.out_features in dims and sp.in_features in dims, (name, sp)
             assert (sp.num_codebooks, sp.nbits) in {(1, 16), (2, 8), (1, 8), (2, 16), (8, 8)}
     assert workload("llama2-7b-1x16")["layers"][0][1] == LayerSpec(4096, 4096, 1, 16)
     assert workload("llama2-7b-1x16")["n"] == [1, 4, 16]
+    # the decode workload is the 1x16 layer and the 2x8 MLP layers, each with its own batches
+    units = workload_units("llama2-7b-decode")
+    assert [(t, sp.scheme, n) for t, sp, n, _ in units] == [
+        ("4096x4096", "1x16", (1, 4, 16)),
+        ("11008x4096-uniform", "2x8", (1, 8)), ("4096x11008-uniform", "2x8", (1, 8)),
+        ("11008x4096-zipf", "2x8", (1, 8)), ("4096x11008-zipf", "2x8", (1, 8))]
     with pytest.raises(KeyError):
         workload("no-such-workload")

@@ -3,10 +3,17 @@
 Some callers cannot call cudaMalloc (the host framework owns every device
 allocation, or allocation is forbidden after start-up), so they cannot hand
 aq_gemv a workspace.  aq_gemv_noalloc keeps its split-K scratch in a fixed
-array inside the library instead.  These tests check, through the C ABI,
-that two calls in a row give the same results as aq_gemv with a workspace
-(within the tolerance the other tests use), and that a layer needing more
-scratch than the array holds is refused without writing anything.
+array inside the library instead.  These tests check, through the C ABI:
+
+* two calls in a row, on layers whose usual workspace fits the array, give
+  results within the tolerance of the oracle, as aq_gemv's do;
+* layers whose usual workspace does not fit (a Llama-2-70B 1x16 layer at
+  batch 16, which must split its sum more coarsely; a wide 2x8 layer at
+  batch 1, whose table path's partial sums do not fit and which runs on the
+  tensor cores instead) stay within the tolerance on sampled rows, and two
+  calls on the same activations return the same bytes;
+* a layer needing more scratch than the array holds even at the coarsest
+  split is refused without writing anything.
 
 This file is collected last, so that a run stopping at the first failure
 has already run every other test; it also passes on its own in a fresh
@@ -27,6 +34,8 @@ CASES = [
     ((4096, 4096, 1, 16), 1), ((4096, 4096, 1, 16), 16),
     ((1000, 1032, 2, 8), 1), ((1000, 1032, 2, 8), 5), ((256, 512, 2, 8), 4),
 ]
+# usual workspace larger than the fixed array
+OVER_CAP = [((28672, 8192, 1, 16), 16), ((20000, 16384, 2, 8), 1)]
 
 
 def _noalloc(dl, x):
@@ -48,7 +57,7 @@ def _with_workspace(dl, x):
 
 
 @pytest.mark.parametrize("shape,batch", CASES)
-def test_noalloc_matches_workspace_entry_point(shape, batch):
+def test_noalloc_matches_oracle_like_workspace_entry_point(shape, batch):
     out, inp, K, B = shape
     spec = LayerSpec(out, inp, K, B, codebook_sigma=0.05)
     assert aq.aq_gemv_workspace_bytes(aq.LayerDesc.make(out, inp, K, B), batch) <= aq.GEMV_NOALLOC_SCRATCH_BYTES
@@ -56,16 +65,42 @@ def test_noalloc_matches_workspace_entry_point(shape, batch):
     dl = DevLayer(layer)
     for call in range(2):  # two calls in a row share the scratch array
         x = make_activations(inp, batch, (out, batch, call))
-        y_na = _noalloc(dl, x)
-        y_ws = _with_workspace(dl, x)
-        _, bound = oracle.matmul(layer.codes, layer.codebooks, layer.scales, x)
-        assert_close(y_na, y_ws, bound, f"noalloc vs workspace, call {call}")
+        ref, bound = oracle.matmul(layer.codes, layer.codebooks, layer.scales, x, threads=8)
+        assert_close(_noalloc(dl, x), ref, bound, f"noalloc vs oracle, call {call}")
+        assert_close(_with_workspace(dl, x), ref, bound, f"workspace entry point vs oracle, call {call}")
+
+
+def _sample_rows(out, n=64, seed=0):
+    rng = np.random.default_rng(seed)
+    rows = set(rng.choice(out, size=n, replace=False).tolist())
+    rows.update({0, 127, 128, out - 1})
+    return np.array(sorted(rows))
+
+
+@pytest.mark.parametrize("shape,batch", OVER_CAP)
+def test_noalloc_coarser_split_when_the_usual_one_does_not_fit(shape, batch):
+    out, inp, K, B = shape
+    assert aq.aq_gemv_workspace_bytes(aq.LayerDesc.make(out, inp, K, B), batch) > aq.GEMV_NOALLOC_SCRATCH_BYTES
+    layer = make_layer(LayerSpec(out, inp, K, B), (out, inp, batch))
+    dl = DevLayer(layer)
+    rows = _sample_rows(out, seed=out)
+    x = make_activations(inp, batch, (out, batch))
+    y1 = _noalloc(dl, x)
+    y2 = _noalloc(dl, x)
+    assert np.array_equal(y1.view(np.uint64), y2.view(np.uint64)), "two calls on the same x differ"
+    ref, bound = oracle.matmul(layer.codes, layer.codebooks, layer.scales, x, rows=rows, threads=8)
+    assert_close(y1[rows], ref, bound, f"noalloc {out}x{inp} {K}x{B} b{batch}")
+    x2 = make_activations(inp, batch, (out, batch, 2))
+    ref2, bound2 = oracle.matmul(layer.codes, layer.codebooks, layer.scales, x2, rows=rows, threads=8)
+    assert_close(_noalloc(dl, x2)[rows], ref2, bound2, f"noalloc {out}x{inp} {K}x{B} b{batch}, second x")
+    del dl
+    torch.cuda.empty_cache()
 
 
 def test_noalloc_refuses_layers_beyond_the_scratch():
-    # 2x8 at batch 1 keeps one partial per row and 32-group block:
-    # 32768 rows x 256 blocks x 4 bytes = 32 MiB > the fixed scratch
-    desc = aq.LayerDesc.make(32768, 65536, 2, 8)
+    # even one CTA per 128 rows needs an arrival counter per 128 rows:
+    # 2^28 rows need 8 MiB of counters > the fixed array
+    desc = aq.LayerDesc.make(1 << 28, 8, 1, 16)
     assert aq.aq_gemv_workspace_bytes(desc, 1) > aq.GEMV_NOALLOC_SCRATCH_BYTES
     small = torch.zeros(64, dtype=torch.int16, device="cuda")  # never read: refused first
     full, y = guarded(64)
