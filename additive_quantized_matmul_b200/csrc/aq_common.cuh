@@ -50,9 +50,16 @@ inline Geom make_geom(const aq_layer_desc &d)
 
 inline size_t align16(size_t v) { return (v + 15) / 16 * 16; }
 
-// Workspace header: status word at byte 0 (AQ_ERR_TIMEOUT when a bounded
-// wait gave up), arrival counters from byte 16.
+// Workspace layout, the same for every entry point, so that one workspace
+// serves any sequence of calls on a stream: status word at byte 0
+// (AQ_ERR_TIMEOUT when a bounded wait gave up); split-K arrival counters in
+// a fixed area of kWsMaxCounters words from byte 16, which only counters
+// ever use and every call leaves at zero; the entry point's own data
+// (split-K partial sums, tables) from kWsData on.  A plan splits a sum
+// over CTAs only when its counters fit the area.
 constexpr size_t kWsHeader = 16;
+constexpr int kWsMaxCounters = 1024;
+constexpr size_t kWsData = kWsHeader + sizeof(unsigned) * kWsMaxCounters;
 
 __device__ __forceinline__ void record_status(void *ws, uint32_t status)
 {

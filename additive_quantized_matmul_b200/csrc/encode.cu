@@ -253,12 +253,12 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(Geom L, const uint1
 namespace aqh {
 using namespace aqk;
 
-size_t encode_workspace_bytes(const Geom &g) { return kWsHeader + align16((size_t)g.G * g.K * 256 * sizeof(float)); }
+size_t encode_workspace_bytes(const Geom &g) { return kWsData + align16((size_t)g.G * g.K * 256 * sizeof(float)); }
 
 cudaError_t launch_encode(const Geom &g, const uint16_t *w, const float *h, const uint16_t *cb,
                           const void *codes_in, void *codes_out, int beam, void *ws, cudaStream_t s)
 {
-    float *q = reinterpret_cast<float *>(reinterpret_cast<char *>(ws) + kWsHeader);
+    float *q = reinterpret_cast<float *>(reinterpret_cast<char *>(ws) + kWsData);
     const uint4 *c = reinterpret_cast<const uint4 *>(cb);
     const int smem = g.in * (int)sizeof(float);
     auto run = [&](auto kk) {

@@ -633,8 +633,9 @@ static GemmPlan plan_gemm(const Geom &g, int T)
     ks = std::max(1, std::min(ks, nst / 8));
     p.per_split = (nst + ks - 1) / ks;
     p.ks = (nst + p.per_split - 1) / p.per_split;
-    p.ws_bytes = kWsHeader + align16(sizeof(unsigned) * (size_t)tiles);
-    if (p.ks > 1) p.ws_bytes += (size_t)p.ks * g.out * T * sizeof(float);
+    // split only while the tiles' arrival counters fit the fixed area
+    if (tiles > kWsMaxCounters) p.ks = 1, p.per_split = nst;
+    if (p.ks > 1) p.ws_bytes = kWsData + (size_t)p.ks * g.out * T * sizeof(float);
     return p;
 }
 
@@ -688,9 +689,7 @@ cudaError_t launch_gemm(const Geom &g, const void *packed, const uint16_t *cb,
         if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
         const dim3 grid(p.mtiles, p.ntiles, p.ks);
         GemmSplit sp{nullptr, reinterpret_cast<unsigned *>(reinterpret_cast<char *>(ws) + kWsHeader)};
-        if (p.ks > 1)
-            sp.partials = reinterpret_cast<float *>(reinterpret_cast<char *>(ws) + kWsHeader +
-                                                    align16(sizeof(unsigned) * (size_t)p.mtiles * p.ntiles));
+        if (p.ks > 1) sp.partials = reinterpret_cast<float *>(reinterpret_cast<char *>(ws) + kWsData);
         auto launch = [&](auto sch, auto bn) {
             using S = decltype(sch);
             constexpr int BN = decltype(bn)::value;

@@ -131,74 +131,45 @@ __device__ __forceinline__ void splitk_finish(const Geom &L, SplitK sk, int coun
 }
 
 // ---------------------------------------------------------------------------
-// 2x8, batch 1: per-group codebook x activation lookup tables.
+// 8-bit codes with one or two codebooks (2x8, 1x8), batch 1: per-group
+// codebook x activation tables in binary16.
 //
-// For one block of 32 groups the CTA tabulates L_k[g][c] = <C_k[c], x_g> for
-// both codebooks (256 x 64 fp32 words = 64 KiB of shared memory), laid out
-// lane-private: entry (k, c, g) at word c*64 + k*32 + g, so lane l (group
-// 32*gb + l) always reads bank l and random codes never conflict.  A row's
-// contribution from the block is then two table reads per group; the byte
-// offset of a read, c*256 + l*4, is one byte permute of the code byte and
-// l*4 (the k*128 goes into the load's immediate).
+// A CTA covers a range of rows and kLutGroups(K) groups: 64 for 2x8, 128
+// for 1x8.  For those groups it tabulates L_k[g][c] = <C_k[c], x_g> (each
+// product of two binary16 values is exact in fp32; the 8-term sum is
+// rounded once to fp32, then once to binary16) in 64 KiB of shared memory:
+// word (c, q, l) at c*64 + q*32 + l holds the entries of local groups
+// g0 + l (low half) and g0 + 32 + l (high half), where q is the codebook
+// (2x8, g0 = 0) or the half of the group range (1x8, g0 = 64 q).  Lane l
+// handles exactly the groups whose entries sit in bank l, so random codes
+// never conflict; a lookup's byte offset c*256 + l*4 is one byte permute of
+// the code byte and l*4, and q*128 + half*2 go into the load's immediate.
+// Each row and lane takes four lookups (two groups x two codebooks, or four
+// groups), summed in binary16 and added to the row's fp32 sum by a 16-row
+// warp reduce-scatter.
 //
-// The tables are one small matrix product, T[g][k*256 + c] =
-// sum_j x_g[j] C_k[c][j] (32 x 512, inner size 8), computed with
-// mma.sync m16n8k8 (binary16 operands, fp32 accumulation; each product of
-// two binary16 values is exact in fp32).  For each codeword it holds, the
-// accumulator fragment gives a lane groups gid, gid+8, gid+16, gid+24 (gid =
-// lane / 4), while the four lanes of a quad hold four different codewords.
-// Lanes rotate their four group slots by their index within the quad before
-// storing, so every store instruction covers 32 distinct groups, i.e. 32
-// distinct banks.  (A 16-byte store of a lane's four groups cannot be made
-// conflict-free: the eight lanes of a store phase would write eight groups
-// four times over, in four rows.)
-// grid = (row ranges, group blocks); each CTA is one split of the K sum.
-// Code chunks stream through a per-warp register ring, issued before the
-// CTA waits on the previous launch.
+// The tables are one small matrix product T = X C^T (groups x codewords,
+// inner size 8) on mma.sync m16n8k8, binary16 operands, fp32 accumulators:
+// groups on M, codewords on N, so a lane's fragment holds groups gid, gid+8
+// of two tiles 32 groups apart (one word each); lanes rotate their four
+// word slots by their index within the quad so that every store covers 32
+// distinct banks.  An entry that is finite in fp32 but beyond the binary16
+// range would become infinite: a CTA that sees one drops its tables and
+// decodes each weight group exactly (sum of the codewords rounded once, as
+// the dequantised matrix has it) and multiplies it in fp32 instead.
+// Rows come in pairs of 8-row tiles per warp step (one 16 B or 8 B code
+// chunk per row tile and group slot in registers, kLutRing steps in
+// flight); the codebooks, the first kLutRing steps of codes and an L2
+// prefetch of the rest are issued before the CTA waits for the previous
+// launch.  grid = (row ranges, group splits), about one CTA per SM; each
+// CTA is one split of the sum, finished by the last CTA of the row range.
 // ---------------------------------------------------------------------------
 constexpr int kLutWarps = 8;
+constexpr int kLutThreads = kLutWarps * 32;
 constexpr int kLutBytes = 256 * 64 * 4;  // the tables: 256 codes x 64 words
-
-// Byte offset c*256 + lane4 of the table entry of code (r, k) of a chunk (8-bit
-// codes: code (r, k) is byte r*K + k of the chunk) by one byte permute: the
-// code byte goes to byte 1, lane4 (the lane's word offset, < 256) to byte 0.
-template <class S>
-__device__ __forceinline__ uint32_t lut_offset(const Chunk<S> &c, int r, int k, uint32_t lane4)
-{
-    const int bi = r * S::K + k;
-    const uint32_t sel = 0x5504u | ((uint32_t)(bi & 3) << 4);
-    uint32_t d;
-    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(c.w[bi >> 2]), "r"(lane4), "r"(sel));
-    return d;
-}
-constexpr int kLutRing = 2;  // quads of code chunks (4 row tiles) in flight per warp
-
-// Reduce-scatter of 32 values per lane over the warp: lane l returns the
-// sum over all lanes of a[l].  Five butterfly levels; at each, a lane keeps
-// the half of its values selected by its own lane bit and adds the partner's
-// copy of that half.  16 + 8 + 4 + 2 + 1 shuffles, all of a level independent.
-__device__ __forceinline__ float warp_reduce32(float a[32], int lane)
-{
-    float b[16], c[8], d[4], e[2];
-    bool h = lane & 16;
-#pragma unroll
-    for (int i = 0; i < 16; ++i)
-        b[i] = (h ? a[i + 16] : a[i]) + __shfl_xor_sync(0xffffffffu, h ? a[i] : a[i + 16], 16);
-    h = lane & 8;
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-        c[i] = (h ? b[i + 8] : b[i]) + __shfl_xor_sync(0xffffffffu, h ? b[i] : b[i + 8], 8);
-    h = lane & 4;
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-        d[i] = (h ? c[i + 4] : c[i]) + __shfl_xor_sync(0xffffffffu, h ? c[i] : c[i + 4], 4);
-    h = lane & 2;
-#pragma unroll
-    for (int i = 0; i < 2; ++i)
-        e[i] = (h ? d[i + 2] : d[i]) + __shfl_xor_sync(0xffffffffu, h ? d[i] : d[i + 2], 2);
-    h = lane & 1;
-    return (h ? e[1] : e[0]) + __shfl_xor_sync(0xffffffffu, h ? e[0] : e[1], 1);
-}
+constexpr int kLutRing = 3;              // warp steps (row-tile pairs) of code chunks in flight
+template <int K>
+constexpr int kLutGroups = 128 / K;      // groups per CTA: 64 (2x8) or 128 (1x8)
 
 // D = A(16x8, row) * B(8x8, col), binary16 in, fp32 out (no addend).
 __device__ __forceinline__ void mma_m16n8k8(float d[4], uint32_t a0, uint32_t a1, uint32_t b0)
@@ -208,126 +179,222 @@ __device__ __forceinline__ void mma_m16n8k8(float d[4], uint32_t a0, uint32_t a1
         : "r"(a0), "r"(a1), "r"(b0), "f"(0.f));
 }
 
+// Byte offset c*256 + lane4 of the table row of code (r, k) of a chunk
+// (8-bit codes: code (r, k) is byte r*K + k of the chunk) by one byte
+// permute: the code byte goes to byte 1, lane4 (< 256) to byte 0.
 template <class S>
-__global__ void __launch_bounds__(kLutWarps * 32, 2)
+__device__ __forceinline__ uint32_t lut_offset(const Chunk<S> &c, int r, int k, uint32_t lane4)
+{
+    const int bi = r * S::K + k;
+    const uint32_t sel = 0x5504u | ((uint32_t)(bi & 3) << 4);
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(c.w[bi >> 2]), "r"(lane4), "r"(sel));
+    return d;
+}
+
+__device__ __forceinline__ __half lut_entry(const char *lutb, uint32_t off)
+{
+    return *reinterpret_cast<const __half *>(lutb + off);
+}
+
+// Reduce-scatter of 16 values per lane over the warp: lanes 2m and 2m+1
+// return the sum over all lanes of a[m].  Four halving levels (8 + 4 + 2 + 1
+// shuffles), then one shuffle with the neighbour lane.
+__device__ __forceinline__ float warp_reduce16(const float a[16], int lane)
+{
+    float b[8], c[4], d[2];
+    bool h = lane & 16;
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+        b[i] = (h ? a[i + 8] : a[i]) + __shfl_xor_sync(0xffffffffu, h ? a[i] : a[i + 8], 16);
+    h = lane & 8;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        c[i] = (h ? b[i + 4] : b[i]) + __shfl_xor_sync(0xffffffffu, h ? b[i] : b[i + 4], 8);
+    h = lane & 4;
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+        d[i] = (h ? c[i + 2] : c[i]) + __shfl_xor_sync(0xffffffffu, h ? c[i] : c[i + 2], 4);
+    h = lane & 2;
+    const float e = (h ? d[1] : d[0]) + __shfl_xor_sync(0xffffffffu, h ? d[0] : d[1], 2);
+    return e + __shfl_xor_sync(0xffffffffu, e, 1);
+}
+
+template <class S>
+__global__ void __launch_bounds__(kLutThreads, 2)
 gemv_lut_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restrict__ cb,
                 const uint16_t *__restrict__ scales, const uint16_t *__restrict__ x,
                 uint16_t *__restrict__ y, SplitK sk, int rt_per_cta)
 {
     static_assert(S::B == 8 && S::K <= 2, "tables for one or two 8-bit codebooks");
     constexpr int K = S::K;
-    extern __shared__ float lut[];       // [256][64] tables: word c*64 + k*32 + g
-    __shared__ uint4 scb[K * 256];       // the codebooks, binary16, row k*256 + c
-    __shared__ uint4 xs[32];             // activations of the block's 32 groups
+    constexpr int NG = kLutGroups<K>;  // groups of the CTA
+    constexpr int NSLOT = NG / 32;     // group slots per lane: 2 (2x8) or 4 (1x8)
+    extern __shared__ uint32_t lut[];  // [256][64] words, see above
+    __shared__ uint4 scb[K * 256];     // the codebooks, row k*256 + c
+    __shared__ uint4 xs[NG];           // activations of the CTA's groups
+    __shared__ int s_overflow;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int gb = blockIdx.y;
+    const int G0 = blockIdx.y * NG;
     const int rt0 = blockIdx.x * rt_per_cta;
     const int rt1 = min(L.rtiles, rt0 + rt_per_cta);
-    // this warp's row quads (4 row tiles, 32 rows) start at row tile
-    // rt0 + 4 (warp + kLutWarps j), j < nq; tiles at or past rt1 read as zero
-    const int nq = ((rt1 - rt0 + 3) / 4 - warp + kLutWarps - 1) / kLutWarps;
-    const size_t src = (size_t)(rt0 + 4 * warp) * L.gp + gb * 32 + lane;  // chunk index of tile 0
-    const size_t qstep = (size_t)4 * kLutWarps * L.gp;
-    const int tile_lim = rt1 - rt0 - 4 * warp;  // tile 4 kLutWarps j + t exists iff below this
-    // codebooks first: the table build needs them, the lookups come later
+    const int npairs = (rt1 - rt0 + 1) / 2;
+    // this warp's steps: row-tile pairs warp + kLutWarps j, j < nst
+    const int nst = (npairs - warp + kLutWarps - 1) / kLutWarps;
+
+    // code chunk (row tile rt0 + 2p + t, group G0 + 32 j + lane); zero past the layer
+    auto fetch = [&](int p, int t, int j) {
+        const int rt = rt0 + 2 * p + t, g = G0 + 32 * j + lane;
+        return load_chunk<S>(packed, (size_t)rt * L.gp + g, p < npairs && rt < rt1 && g < L.G);
+    };
+    // weights before the dependency wait: codebooks, the first steps' codes,
+    // and the rest of the CTA's codes into L2
     uint4 cw[K];
 #pragma unroll
     for (int k = 0; k < K; ++k) cw[k] = ldg_stream_v4(cb + k * 256 + threadIdx.x);
-    Chunk<S> ring[kLutRing][4];
+    Chunk<S> ring[kLutRing][2][NSLOT];
 #pragma unroll
     for (int i = 0; i < kLutRing; ++i)
 #pragma unroll
-        for (int t = 0; t < 4; ++t)
-            ring[i][t] = load_chunk<S>(packed, src + i * qstep + (size_t)t * L.gp,
-                                       i < nq && 4 * kLutWarps * i + t < tile_lim);
+        for (int t = 0; t < 2; ++t)
+#pragma unroll
+            for (int j = 0; j < NSLOT; ++j) ring[i][t][j] = fetch(i < nst ? warp + kLutWarps * i : npairs, t, j);
+    {
+        const int first = rt0 + 2 * kLutWarps * kLutRing;  // row tiles below this are in the rings
+        const int ngl = min(NG, L.gp - G0);                // groups of this split in the padded layout
+        for (int rt = first + (int)threadIdx.x; rt < rt1; rt += kLutThreads)
+            prefetch_l2_bulk(packed + ((size_t)rt * L.gp + G0) * S::kChunkBytes, (uint32_t)(ngl * S::kChunkBytes));
+    }
     grid_dependency_wait();  // x, y and the workspace follow the previous launch
     grid_launch_dependents();
-    if (threadIdx.x < 32) {
-        const int g = gb * 32 + threadIdx.x;
+    if (threadIdx.x < NG) {
+        const int g = G0 + threadIdx.x;
         xs[threadIdx.x] = (g < L.G) ? ldg_nc_v4(x + (size_t)g * 8) : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
     for (int k = 0; k < K; ++k) scb[k * 256 + threadIdx.x] = cw[k];
+    if (threadIdx.x == 0) s_overflow = 0;
     __syncthreads();
     {
-        // warp w fills codewords kc in [32 K w, 32 K (w + 1)) for all 32 groups
+        // warp w fills the codeword octets n = w + kLutWarps i (codeword kc =
+        // 8 n + 0..7, kc = k*256 + c) for every group of the CTA
         const int gid = lane >> 2, t4 = lane & 3;
         const uint32_t *xw = reinterpret_cast<const uint32_t *>(xs);
         const uint32_t *cbw = reinterpret_cast<const uint32_t *>(scb);
-        uint32_t a[2][2];
+        constexpr int MT = NG / 16;  // group tiles
+        uint32_t a[MT][2];
 #pragma unroll
-        for (int m = 0; m < 2; ++m) {
+        for (int m = 0; m < MT; ++m) {
             a[m][0] = xw[(16 * m + gid) * 4 + t4];
             a[m][1] = xw[(16 * m + gid + 8) * 4 + t4];
         }
-        const int kc0 = warp * 32 * K;  // codeword k*256 + c: this warp's all share one k
-        float *dst = lut + ((kc0 & 255) + 2 * t4) * 64 + (kc0 >> 8) * 32 + gid;
-        int off[4];
+        int off[4];  // slot s of a store writes word l = gid + off[s]
 #pragma unroll
-        for (int s = 0; s < 4; ++s) off[s] = 8 * ((t4 + s) & 3);
+        for (int s2 = 0; s2 < 4; ++s2) off[s2] = 8 * ((t4 + s2) & 3);
+        bool ovf = false;
+        constexpr int NOCT = K * 256 / 8;
+#pragma unroll 2
+        for (int n = warp; n < NOCT; n += kLutWarps) {
+            const uint32_t b0 = cbw[(8 * n + gid) * 4 + t4];
 #pragma unroll
-        for (int n = 0; n < 4 * K; ++n) {
-            const uint32_t b0 = cbw[(kc0 + 8 * n + gid) * 4 + t4];
-            float d0[4], d1[4];
-            mma_m16n8k8(d0, a[0][0], a[0][1], b0);  // groups gid, gid + 8
-            mma_m16n8k8(d1, a[1][0], a[1][1], b0);  // groups gid + 16, gid + 24
+            for (int qq = 0; qq < MT / 4; ++qq) {
+                // tiles 4 qq + {0, 1} hold groups 64 qq + gid + {0, 8, 16, 24};
+                // tiles 4 qq + {2, 3} the same groups + 32
+                float lo0[4], lo1[4], hi0[4], hi1[4];
+                mma_m16n8k8(lo0, a[4 * qq + 0][0], a[4 * qq + 0][1], b0);
+                mma_m16n8k8(lo1, a[4 * qq + 1][0], a[4 * qq + 1][1], b0);
+                mma_m16n8k8(hi0, a[4 * qq + 2][0], a[4 * qq + 2][1], b0);
+                mma_m16n8k8(hi1, a[4 * qq + 3][0], a[4 * qq + 3][1], b0);
 #pragma unroll
-            for (int b = 0; b < 2; ++b) {
-                // v[q] belongs to group gid + 8q, codeword kc0 + 8n + 2 t4 + b
-                const float v[4] = {d0[b], d0[2 + b], d1[b], d1[2 + b]};
-                float r[4], w[4];
+                for (int e = 0; e < 4; ++e) {
+                    ovf |= (fabsf(lo0[e]) >= 65520.f && fabsf(lo0[e]) < INFINITY) ||
+                           (fabsf(lo1[e]) >= 65520.f && fabsf(lo1[e]) < INFINITY) ||
+                           (fabsf(hi0[e]) >= 65520.f && fabsf(hi0[e]) < INFINITY) ||
+                           (fabsf(hi1[e]) >= 65520.f && fabsf(hi1[e]) < INFINITY);
+                }
+                const int kc = 8 * n + 2 * t4;  // this lane's codewords kc, kc + 1
+                // word (c, q, l): c = kc & 255, q = the codebook (2x8) or qq (1x8)
+                const int q = (K == 2) ? (kc >> 8) : qq;
 #pragma unroll
-                for (int s = 0; s < 4; ++s) r[s] = (t4 & 1) ? v[(s + 1) & 3] : v[s];
+                for (int b = 0; b < 2; ++b) {
+                    // v[s] is word l = gid + 8 s: groups (gid + 8 s, + 32) of codeword kc + b
+                    const uint32_t v[4] = {f2h2(lo0[b], hi0[b]), f2h2(lo0[2 + b], hi0[2 + b]),
+                                           f2h2(lo1[b], hi1[b]), f2h2(lo1[2 + b], hi1[2 + b])};
+                    uint32_t r[4], w[4];
 #pragma unroll
-                for (int s = 0; s < 4; ++s) w[s] = (t4 & 2) ? r[(s + 2) & 3] : r[s];
-                // w[s] = v[(t4 + s) & 3]: slot s writes group gid + off[s]
+                    for (int s2 = 0; s2 < 4; ++s2) r[s2] = (t4 & 1) ? v[(s2 + 1) & 3] : v[s2];
 #pragma unroll
-                for (int s = 0; s < 4; ++s) dst[n * 512 + b * 64 + off[s]] = w[s];
+                    for (int s2 = 0; s2 < 4; ++s2) w[s2] = (t4 & 2) ? r[(s2 + 2) & 3] : r[s2];
+                    // w[s2] = v[(t4 + s2) & 3], the word of l = gid + off[s2]
+                    uint32_t *dst = lut + ((kc + b) & 255) * 64 + q * 32 + gid;
+#pragma unroll
+                    for (int s2 = 0; s2 < 4; ++s2) dst[off[s2]] = w[s2];
+                }
             }
         }
+        if (ovf) s_overflow = 1;
     }
     __syncthreads();
+    const bool exact = s_overflow != 0;  // some entry is beyond binary16: decode each group instead
     const char *lutb = reinterpret_cast<const char *>(lut);
     const uint32_t lane4 = lane * 4;
-    float *part = sk.partials + (size_t)gb * L.rows8;
-    for (int j0 = 0; j0 < nq; j0 += kLutRing) {
+    float *part = sk.partials + (size_t)blockIdx.y * L.rows8;
+
+    // sum over this lane's groups of row r of chunk tile t
+    auto row_value = [&](const Chunk<S> (&ch)[2][NSLOT], int t, int r) -> float {
+        if (!exact) {
+            __half h[4];
+#pragma unroll
+            for (int j = 0; j < NSLOT; ++j)
+#pragma unroll
+                for (int k = 0; k < K; ++k) {
+                    const int q = (K == 2) ? k : (j >> 1), half = (K == 2) ? j : (j & 1);
+                    h[j * K + k] = lut_entry(lutb, lut_offset<S>(ch[t][j], r, k, lane4) + q * 128 + half * 2);
+                }
+            return __half2float(__hadd(__hadd(h[0], h[1]), __hadd(h[2], h[3])));
+        }
+        float acc = 0.f;
+#pragma unroll
+        for (int j = 0; j < NSLOT; ++j) {
+            uint4 tm[K];
+#pragma unroll
+            for (int k = 0; k < K; ++k) tm[k] = scb[k * 256 + ch[t][j].code(r, k)];
+            acc = dot8(sum_round_fast_h8<K>(tm), xs[32 * j + lane], acc);
+        }
+        return acc;
+    };
+
+    for (int j0 = 0; j0 < nst; j0 += kLutRing) {
 #pragma unroll
         for (int i = 0; i < kLutRing; ++i) {
-            const int j = j0 + i;
-            if (j >= nq) break;
-            float acc[32];  // acc[8 t + r]: row r of tile t of the quad, this lane's group
+            const int jj = j0 + i;
+            if (jj >= nst) break;
+            float acc[16];  // acc[8 t + r]: row r of tile t of the pair
 #pragma unroll
-            for (int t = 0; t < 4; ++t)
+            for (int t = 0; t < 2; ++t)
 #pragma unroll
-                for (int r = 0; r < 8; ++r) {
-                    float a = *reinterpret_cast<const float *>(lutb + lut_offset<S>(ring[i][t], r, 0, lane4));
+                for (int r = 0; r < 8; ++r) acc[8 * t + r] = row_value(ring[i], t, r);
+            const int jn = jj + kLutRing;  // the step this ring slot takes next
+            const int pn = jn < nst ? warp + kLutWarps * jn : npairs;
 #pragma unroll
-                    for (int k = 1; k < K; ++k)
-                        a += *reinterpret_cast<const float *>(lutb + lut_offset<S>(ring[i][t], r, k, lane4) + k * 128);
-                    acc[8 * t + r] = a;
-                }
-            const int jn = j + kLutRing;
+            for (int t = 0; t < 2; ++t)
 #pragma unroll
-            for (int t = 0; t < 4; ++t)
-                ring[i][t] = load_chunk<S>(packed, src + jn * qstep + (size_t)t * L.gp,
-                                           jn < nq && 4 * kLutWarps * jn + t < tile_lim);
-            const float r = warp_reduce32(acc, lane);
-            const int row = (rt0 + 4 * (warp + kLutWarps * j)) * 8 + lane;
-            if (row < rt1 * 8) {
+                for (int j = 0; j < NSLOT; ++j) ring[i][t][j] = fetch(pn, t, j);
+            const float v = warp_reduce16(acc, lane);
+            const int row = (rt0 + 2 * (warp + kLutWarps * jj)) * 8 + (lane >> 1);
+            if ((lane & 1) == 0 && row < rt1 * 8) {
                 if (gridDim.y == 1) {
                     if (row < L.out) {
                         const float sc = scales ? __half2float(__ushort_as_half(scales[row])) : 1.f;
-                        y[row] = __half_as_ushort(__float2half_rn(sc * r));
+                        y[row] = __half_as_ushort(__float2half_rn(sc * v));
                     }
                 } else {
-                    part[row] = r;
+                    part[row] = v;
                 }
             }
         }
     }
     if (gridDim.y == 1) return;
-    // one float4 per thread: summed straight from L2 (measured faster here
-    // than staging the slots in the tables' shared memory)
     splitk_finish(L, sk, blockIdx.x, gridDim.y, rt0 * 8, (rt1 - rt0) * 8, 1, scales, y, nullptr, 0);
 }
 
@@ -954,21 +1021,26 @@ long tc_cost(long ctas, int len, int res, int batch, bool early)
     return cost;
 }
 
-// Row tiles per CTA of the table path (whole quads of four tiles): as many
-// row ranges as put about two CTAs per SM in one wave.
-int lut_rt_per_cta(const Geom &g)
+// Group splits of the table path: one per kLutGroups groups.
+int lut_splits(const Geom &g)
 {
-    const int ranges = std::max(1, std::min(g.rtiles, 2 * kNumSMs / g.gblocks));
-    return ((g.rtiles + ranges - 1) / ranges + 3) & ~3;
+    const int ng = g.K == 1 ? kLutGroups<1> : kLutGroups<2>;
+    return (g.G + ng - 1) / ng;
 }
 
-// Workspace of the table path: status word, one arrival counter per row
-// range, one partial sum per row and 32-group block.
+// Row tiles per CTA of the table path (whole pairs of tiles): as many row
+// ranges as put one CTA on each SM in one wave.
+int lut_rt_per_cta(const Geom &g)
+{
+    const int ranges = std::max(1, std::min((g.rtiles + 1) / 2, kNumSMs / lut_splits(g)));
+    return ((g.rtiles + ranges - 1) / ranges + 1) & ~1;
+}
+
+// Workspace of the table path: one partial sum per row and group split.
 size_t lut_ws(const Geom &g)
 {
-    const int ranges = (g.rtiles + lut_rt_per_cta(g) - 1) / lut_rt_per_cta(g);
-    return kWsHeader + align16(sizeof(unsigned) * (size_t)ranges) +
-           (g.gblocks > 1 ? (size_t)g.gblocks * g.rows8 * sizeof(float) : 0);
+    const int ks = lut_splits(g);
+    return ks > 1 ? kWsData + (size_t)ks * g.rows8 * sizeof(float) : kWsHeader;
 }
 
 // `cap`: largest workspace the caller can offer (the no-allocation entry
@@ -984,10 +1056,10 @@ GemvPlan plan_gemv(const Geom &g, int batch, size_t cap = ~(size_t)0)
     // (their x in shared memory)
     const int cc_per_sm = batch == 1 ? kCcPerSMOf<1> : kCcPerSMOf<2>;
     const int cc_ks = std::max(1, std::min((cc_per_sm * kNumSMs) / cc_ranges, (g.G + 7) / 8));
-    const size_t cc_ws = kWsHeader + align16(sizeof(unsigned) * (size_t)cc_ranges) +
-                         (cc_ks > 1 ? (size_t)cc_ks * g.rows8 * batch * sizeof(float) : 0);
+    const size_t cc_ws = cc_ks > 1 ? kWsData + (size_t)cc_ks * g.rows8 * batch * sizeof(float) : kWsHeader;
     if (batch <= kCcMaxBatch && g.K == 1 && g.B == 16 && cc_ks <= kCcMaxSplits &&
-        (g.G + cc_ks - 1) / cc_ks * batch <= 1536 && cc_ws <= cap) {
+        (g.G + cc_ks - 1) / cc_ks * batch <= 1536 && cc_ws <= cap &&
+        (cc_ks == 1 || cc_ranges <= kWsMaxCounters)) {
         p.path = kCudaCores;
         p.grid_x = cc_ranges;
         p.len = (g.G + cc_ks - 1) / cc_ks;  // groups per split
@@ -998,9 +1070,9 @@ GemvPlan plan_gemv(const Geom &g, int batch, size_t cap = ~(size_t)0)
         p.cc_smem = std::max(p.len * 32 * batch, std::min(kCcStage, p.ks > 1 ? p.ks * nvec * 16 : 0));
     } else if (batch == 1 && g.B == 8 && g.K <= 2 && lut_ws(g) <= cap) {
         p.path = kLut;
-        p.ks = g.gblocks;
-        // two CTAs per SM in one wave: every CTA builds its tables once, and
-        // a third CTA per SM fits, so the next launch can start early
+        p.ks = lut_splits(g);
+        // one CTA per SM in one wave: every CTA builds its tables once, and
+        // a CTA of the next launch fits beside it, so that it can start early
         p.rt_per_cta = lut_rt_per_cta(g);
         p.grid_x = (g.rtiles + p.rt_per_cta - 1) / p.rt_per_cta;
         p.counters = p.grid_x;
@@ -1016,8 +1088,10 @@ GemvPlan plan_gemv(const Geom &g, int batch, size_t cap = ~(size_t)0)
         const long slots = (long)res * kNumSMs;
         const bool early = (g.K == 1 && g.B == 16);  // decoders that do not wait for the previous launch
         auto ws_of = [&](int nslots) {
-            return kWsHeader + align16(sizeof(unsigned) * (size_t)mtiles) + (size_t)nslots * g.rows8 * batch * sizeof(float);
+            return nslots > 0 ? kWsData + (size_t)nslots * g.rows8 * batch * sizeof(float) : kWsHeader;
         };
+        // a split needs one arrival counter per row tile in the fixed area
+        const bool may_split = mtiles <= kWsMaxCounters;
         // per row tile: ks splits of `per` stages (the last may be shorter)
         long best_pt = -1;
         p.stream_k = false;
@@ -1026,7 +1100,7 @@ GemvPlan plan_gemv(const Geom &g, int batch, size_t cap = ~(size_t)0)
         for (int ks = 1; ks <= std::max(1, nst / kTcMinLen); ++ks) {
             const int per = (nst + ks - 1) / ks, kk = (nst + per - 1) / per;
             if (kk < ks) continue;  // same split as a smaller ks
-            if (kk > 1 && ws_of(kk) > cap) break;
+            if (kk > 1 && (!may_split || ws_of(kk) > cap)) break;
             const long c = tc_cost((long)mtiles * kk, per, res, batch, early);
             if (best_pt < 0 || c < best_pt) {
                 best_pt = c;
@@ -1042,7 +1116,7 @@ GemvPlan plan_gemv(const Geom &g, int batch, size_t cap = ~(size_t)0)
         auto sk_slots = [&](int len) { return len >= nst ? 0 : (nst - 1 + len - 1) / len + 1; };
         long best_sk = -1;
         int sk_len = nst;
-        for (int len = lmin; len <= lmax; ++len) {
+        for (int len = lmin; len <= lmax && may_split; ++len) {
             if (ws_of(sk_slots(len)) > cap) continue;
             const long c = tc_cost((units + len - 1) / len, len, res, batch, early);
             if (best_sk < 0 || c < best_sk) {
@@ -1066,8 +1140,7 @@ GemvPlan plan_gemv(const Geom &g, int batch, size_t cap = ~(size_t)0)
         p.counters = mtiles;
         p.rt_per_cta = kTcBM / 8;
     }
-    p.ws_bytes = kWsHeader + align16(sizeof(unsigned) * (size_t)p.counters) +
-                 (size_t)p.slots * g.rows8 * batch * sizeof(float);
+    p.ws_bytes = p.slots > 0 ? kWsData + (size_t)p.slots * g.rows8 * batch * sizeof(float) : kWsHeader;
     return p;
 }
 
@@ -1122,8 +1195,7 @@ cudaError_t launch_plan(const Geom &g, const GemvPlan &p, const void *packed, co
     SplitK sk;
     char *base = reinterpret_cast<char *>(ws);
     sk.counters = reinterpret_cast<unsigned *>(base + kWsHeader);
-    sk.partials = reinterpret_cast<float *>(base + kWsHeader +
-                                            align16(sizeof(unsigned) * (size_t)p.counters));
+    sk.partials = reinterpret_cast<float *>(base + kWsData);
     const uint8_t *pk = reinterpret_cast<const uint8_t *>(packed);
     const uint4 *c = reinterpret_cast<const uint4 *>(cb);
     const dim3 grid(p.grid_x, p.ks);
@@ -1144,7 +1216,7 @@ cudaError_t launch_plan(const Geom &g, const GemvPlan &p, const void *packed, co
             if constexpr (S::B == 8 && S::K <= 2) {
                 cudaError_t r = set_smem(gemv_lut_kernel<S>, smem);
                 if (r != cudaSuccess) return r;
-                return launch_pdl(pdl, gemv_lut_kernel<S>, grid, dim3(kLutWarps * 32), smem, s, g, pk, c, scales, x, y,
+                return launch_pdl(pdl, gemv_lut_kernel<S>, grid, dim3(kLutThreads), smem, s, g, pk, c, scales, x, y,
                                   sk, p.rt_per_cta);
             } else {
                 return cudaErrorInvalidValue;
@@ -1278,7 +1350,7 @@ cudaError_t launch_gemv_noalloc(const Geom &g, const void *packed, const uint16_
     if (e != cudaSuccess) return e;
     // status word and arrival counters must start at zero; the partials are
     // fully written before they are read
-    const size_t clear = kWsHeader + align16(sizeof(unsigned) * (size_t)p.counters);
+    const size_t clear = p.slots > 0 ? kWsData : kWsHeader;
     e = cudaMemsetAsync(scratch, 0, clear, s);
     if (e != cudaSuccess) return e;
     return launch_plan(g, p, packed, cb, scales, x, batch, y, scratch, s, true);

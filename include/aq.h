@@ -107,13 +107,17 @@ int aq_version(void);
 size_t aq_packed_codes_bytes(const aq_layer_desc *desc);
 
 /*
- * Workspace.  aq_gemv and aq_gemm take a caller-owned device workspace.  Its
- * first 16 bytes hold a status word that a kernel sets when a bounded wait
- * gives up (read it with aq_workspace_status); the rest holds split-K
- * partial sums and arrival counters.  A workspace must be zero-filled once
- * before its first use; every completed call leaves it ready for the next
- * (counters back at zero).  Calls that may overlap in time (different
- * streams) must not share a workspace.
+ * Workspace.  aq_gemv, aq_gemm, aq_param_grad and aq_encode take a
+ * caller-owned device workspace.  Its first 16 bytes hold a status word that
+ * a kernel sets when a bounded wait gives up (read it with
+ * aq_workspace_status); then come split-K arrival counters in a fixed area
+ * of 4 KiB, then the call's own data (split-K partial sums, tables).  A
+ * workspace must be zero-filled once before its first use; every completed
+ * call leaves it ready for the next (counters back at zero), whatever the
+ * layer or entry point, so one workspace as large as the largest size any
+ * of the calls needs serves a whole sequence of calls on one stream (all
+ * the linears of a model, for instance).  Calls that may overlap in time
+ * (different streams) must not share a workspace.
  *
  * The sizes below are host-only (no GPU needed) and depend on the
  * descriptor and batch / token count alone.  They return 0 for invalid
@@ -231,9 +235,11 @@ aq_status aq_gemv_ordered(const aq_layer_desc *desc, const void *packed, const u
  *    calls whose kernels may overlap on the GPU (different streams) race and
  *    give wrong results.  Serialise them, or use aq_gemv with a workspace
  *    per stream.
- *  - AQ_ERR_WORKSPACE if the layer needs more scratch than the array holds
- *    even at the coarsest split (one arrival counter per 128 rows: more
- *    than about 134 million rows); nothing is launched then.
+ *  - AQ_ERR_WORKSPACE if the layer would need more scratch than the array
+ *    holds even at the coarsest split; nothing is launched then.  The
+ *    coarsest split (one CTA per 128 rows) needs no partial sums and no
+ *    counters, so no layer the descriptor limits allow reaches this today;
+ *    the status stays as the contract for plans that might.
  *  - A bounded wait that gives up inside the kernel cannot be reported (the
  *    status word is internal): use aq_gemv when that report is needed.
  */

@@ -178,11 +178,30 @@ def test_gemv_noalloc_argument_errors():
     assert f(ctypes.byref(d), None, FAKE, FAKE, FAKE, 1, FAKE, None) == 1
     assert f(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE + 8, 1, FAKE, None) == 3
     assert f(None, FAKE, FAKE, FAKE, FAKE, 1, FAKE, None) == 1
-    # even one CTA per 128 rows needs an arrival counter per 128 rows: 2^28
-    # rows need more scratch than the fixed array (refused before any launch)
-    big = aq.LayerDesc.make(1 << 28, 8, 1, 16)
-    assert aq.aq_gemv_workspace_bytes(big, 1) > aq.GEMV_NOALLOC_SCRATCH_BYTES
-    assert f(ctypes.byref(big), FAKE, FAKE, FAKE, FAKE, 1, FAKE, None) == 4
+
+
+
+def test_workspace_layout_is_shared_by_every_call():
+    """Counters live in a fixed area after the 16-byte status word, and
+    partial sums or tables only after it: a plan that splits needs the
+    4112-byte prefix, one that does not needs the status word alone."""
+    prefix = 16 + 4 * 1024
+    for (o, i, K, B), b in [((4096, 4096, 1, 16), 1), ((4096, 4096, 1, 16), 16), ((11008, 4096, 2, 8), 1),
+                            ((4096, 11008, 2, 8), 8)]:
+        d = aq.LayerDesc.make(o, i, K, B)
+        assert aq.aq_gemv_workspace_bytes(d, b) > prefix  # these split
+        assert (aq.aq_gemv_workspace_bytes(d, b) - prefix) % (4 * ((o + 7) // 8 * 8) * b) == 0
+    # 64 groups: one CTA's tables cover every group, no split
+    assert aq.aq_gemv_workspace_bytes(aq.LayerDesc.make(256, 512, 2, 8), 1) == 16
+    # 2^20 rows: 8192 row tiles fill the GPU without a split, and would need
+    # more counters than the fixed area holds
+    huge = aq.LayerDesc.make(1 << 20, 64, 1, 16)
+    assert aq.aq_gemv_workspace_bytes(huge, 4) == 16
+    assert aq.aq_gemm_workspace_bytes(huge, 64) == 16
+    assert aq.aq_gemm_workspace_bytes(aq.LayerDesc.make(256, 4096, 2, 8), 512) > prefix
+    assert aq.aq_encode_workspace_bytes(aq.LayerDesc.make(64, 256, 2, 8)) == prefix + 32 * 2 * 256 * 4
+    # the coarsest split of the no-allocation entry point always fits its array
+    assert aq.aq_gemv_workspace_bytes(aq.LayerDesc.make(1 << 28, 8, 1, 16), 1) <= aq.GEMV_NOALLOC_SCRATCH_BYTES
 
 
 def test_noalloc_scratch_size_matches_header():

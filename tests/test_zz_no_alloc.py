@@ -12,8 +12,8 @@ array inside the library instead.  These tests check, through the C ABI:
   batch 1, whose table path's partial sums do not fit and which runs on the
   tensor cores instead) stay within the tolerance on sampled rows, and two
   calls on the same activations return the same bytes;
-* a layer needing more scratch than the array holds even at the coarsest
-  split is refused without writing anything.
+* a layer of 2^20 rows, whose plan needs no split (and so no scratch
+  beyond the status word), runs through the same entry point.
 
 This file is collected last, so that a run stopping at the first failure
 has already run every other test; it also passes on its own in a fresh
@@ -97,15 +97,13 @@ def test_noalloc_coarser_split_when_the_usual_one_does_not_fit(shape, batch):
     torch.cuda.empty_cache()
 
 
-def test_noalloc_refuses_layers_beyond_the_scratch():
-    # even one CTA per 128 rows needs an arrival counter per 128 rows:
-    # 2^28 rows need 8 MiB of counters > the fixed array
-    desc = aq.LayerDesc.make(1 << 28, 8, 1, 16)
-    assert aq.aq_gemv_workspace_bytes(desc, 1) > aq.GEMV_NOALLOC_SCRATCH_BYTES
-    small = torch.zeros(64, dtype=torch.int16, device="cuda")  # never read: refused first
-    full, y = guarded(64)
-    with pytest.raises(aq.AQError) as e:
-        aq.aq_gemv_noalloc(desc, small, small, small, small, 1, y)
-    assert e.value.name == "AQ_ERR_WORKSPACE"
-    torch.cuda.synchronize()
-    assert guards_intact(full) and bool((y == 0x7E5A).all())
+def test_noalloc_layer_without_split():
+    out, inp = 1 << 20, 64
+    assert aq.aq_gemv_workspace_bytes(aq.LayerDesc.make(out, inp, 1, 16), 4) == 16
+    layer = make_layer(LayerSpec(out, inp, 1, 16), 11)
+    dl = DevLayer(layer)
+    x = make_activations(inp, 4, 12)
+    y = _noalloc(dl, x)
+    rows = _sample_rows(out, seed=3)
+    ref, bound = oracle.matmul(layer.codes, layer.codebooks, layer.scales, x, rows=rows, threads=8)
+    assert_close(y[rows], ref, bound, "noalloc 2^20 x 64")
