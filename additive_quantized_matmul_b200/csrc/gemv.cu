@@ -26,6 +26,7 @@
 // row range adds them in split order (no float atomics: bit-reproducible).
 #include <algorithm>
 #include <mutex>
+#include <type_traits>
 
 #include <cuda.h>  // driver types only; the calls are fetched at run time
 
@@ -50,6 +51,7 @@ struct SplitK {
 // at once with cp.async, so a pass costs about one L2 round trip whatever
 // ks.  Without it (or with fewer than 16 ks bytes) they are summed straight
 // from L2, eight slots in flight per float4.
+template <int kInFlight = 8>
 __device__ __forceinline__ void splitk_finish(const Geom &L, SplitK sk, int counter, int ks, int row0,
                                               int nrows, int batch, const uint16_t *__restrict__ scales,
                                               uint16_t *__restrict__ y, float4 *stage, int stage_bytes)
@@ -75,13 +77,13 @@ __device__ __forceinline__ void splitk_finish(const Geom &L, SplitK sk, int coun
         // no staging area, or more slots than it holds
         for (int e = threadIdx.x; e < nvec; e += blockDim.x) {
             float4 acc = __ldcg(base + e);
-            for (int s0 = 1; s0 < ks; s0 += 8) {
-                float4 t[8];
+            for (int s0 = 1; s0 < ks; s0 += kInFlight) {
+                float4 t[kInFlight];
 #pragma unroll
-                for (int j = 0; j < 8; ++j)
+                for (int j = 0; j < kInFlight; ++j)
                     if (s0 + j < ks) t[j] = __ldcg(base + (size_t)(s0 + j) * vstride + e);
 #pragma unroll
-                for (int j = 0; j < 8; ++j)
+                for (int j = 0; j < kInFlight; ++j)
                     if (s0 + j < ks) {
                         acc.x += t[j].x; acc.y += t[j].y; acc.z += t[j].z; acc.w += t[j].w;
                     }
@@ -134,9 +136,9 @@ __device__ __forceinline__ void splitk_finish(const Geom &L, SplitK sk, int coun
 // 8-bit codes with one or two codebooks (2x8, 1x8), batch 1: per-group
 // codebook x activation tables in binary16.
 //
-// A CTA covers a range of rows and kLutGroups(K) groups: 64 for 2x8, 128
-// for 1x8.  For those groups it tabulates L_k[g][c] = <C_k[c], x_g> (each
-// product of two binary16 values is exact in fp32; the 8-term sum is
+// A CTA covers a range of 8-row tiles and kLutGroups(K) groups: 64 for
+// 2x8, 128 for 1x8.  For those groups it tabulates L_k[g][c] = <C_k[c], x_g>
+// (each product of two binary16 values is exact in fp32; the 8-term sum is
 // rounded once to fp32, then once to binary16) in 64 KiB of shared memory:
 // word (c, q, l) at c*64 + q*32 + l holds the entries of local groups
 // g0 + l (low half) and g0 + 32 + l (high half), where q is the codebook
@@ -145,29 +147,35 @@ __device__ __forceinline__ void splitk_finish(const Geom &L, SplitK sk, int coun
 // never conflict; a lookup's byte offset c*256 + l*4 is one byte permute of
 // the code byte and l*4, and q*128 + half*2 go into the load's immediate.
 // Each row and lane takes four lookups (two groups x two codebooks, or four
-// groups), summed in binary16 and added to the row's fp32 sum by a 16-row
-// warp reduce-scatter.
+// groups), summed in binary16, and a warp reduction adds the lanes in fp32.
 //
 // The tables are one small matrix product T = X C^T (groups x codewords,
 // inner size 8) on mma.sync m16n8k8, binary16 operands, fp32 accumulators:
 // groups on M, codewords on N, so a lane's fragment holds groups gid, gid+8
 // of two tiles 32 groups apart (one word each); lanes rotate their four
 // word slots by their index within the quad so that every store covers 32
-// distinct banks.  An entry that is finite in fp32 but beyond the binary16
-// range would become infinite: a CTA that sees one drops its tables and
-// decodes each weight group exactly (sum of the codewords rounded once, as
-// the dequantised matrix has it) and multiplies it in fp32 instead.
-// Rows come in pairs of 8-row tiles per warp step (one 16 B or 8 B code
-// chunk per row tile and group slot in registers, kLutRing steps in
-// flight); the codebooks, the first kLutRing steps of codes and an L2
-// prefetch of the rest are issued before the CTA waits for the previous
-// launch.  grid = (row ranges, group splits), about one CTA per SM; each
-// CTA is one split of the sum, finished by the last CTA of the row range.
+// distinct banks.  Binary16 entries need |L| < 65504: the CTA bounds them
+// by 8 max|x| max|C| over its groups and codebooks, and when the bound
+// fails (or an input is not finite) it skips the tables and decodes each
+// weight group exactly (sum of the codewords rounded once, as the
+// dequantised matrix has it) and multiplies it in fp32 instead.
+//
+// 16 warps; warp w takes the CTA's row tiles w, w + 16, ...  A tile's codes
+// for the CTA's groups are one contiguous kilobyte of the packed layout;
+// each warp copies its tiles into a ring of its own in shared memory with
+// cp.async, kLutRing tiles ahead.  The codebooks, the first tiles of codes
+// and an L2 prefetch of the rest are requested before the CTA waits for the
+// previous launch.  grid = (row ranges, group splits), about one CTA per
+// SM, small enough (registers, shared memory) for a CTA of the next launch
+// to start beside it; each CTA is one split of the sum, finished by the
+// last CTA of the row range.
 // ---------------------------------------------------------------------------
-constexpr int kLutWarps = 8;
+constexpr int kLutWarps = 16;
 constexpr int kLutThreads = kLutWarps * 32;
 constexpr int kLutBytes = 256 * 64 * 4;  // the tables: 256 codes x 64 words
-constexpr int kLutRing = 3;              // warp steps (row-tile pairs) of code chunks in flight
+constexpr int kLutRing = 2;              // row tiles of codes in flight per warp
+constexpr int kLutTileBytes = 1024;      // codes of one row tile for the CTA's groups
+constexpr int kLutSmem = kLutBytes + kLutWarps * kLutRing * kLutTileBytes;  // dynamic shared memory
 template <int K>
 constexpr int kLutGroups = 128 / K;      // groups per CTA: 64 (2x8) or 128 (1x8)
 
@@ -192,34 +200,20 @@ __device__ __forceinline__ uint32_t lut_offset(const Chunk<S> &c, int r, int k, 
     return d;
 }
 
-__device__ __forceinline__ __half lut_entry(const char *lutb, uint32_t off)
+// Largest |v| over eight binary16 values, as the bits of a non-negative
+// binary16 (NaN orders above infinity).
+__device__ __forceinline__ uint32_t absmax_h8_bits(uint4 v)
 {
-    return *reinterpret_cast<const __half *>(lutb + off);
+    uint32_t m = 0;
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) m = max(m, max(w[i] & 0x7fffu, (w[i] >> 16) & 0x7fffu));
+    return m;
 }
 
-// Reduce-scatter of 16 values per lane over the warp: lanes 2m and 2m+1
-// return the sum over all lanes of a[m].  Four halving levels (8 + 4 + 2 + 1
-// shuffles), then one shuffle with the neighbour lane.
-__device__ __forceinline__ float warp_reduce16(const float a[16], int lane)
-{
-    float b[8], c[4], d[2];
-    bool h = lane & 16;
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-        b[i] = (h ? a[i + 8] : a[i]) + __shfl_xor_sync(0xffffffffu, h ? a[i] : a[i + 8], 16);
-    h = lane & 8;
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-        c[i] = (h ? b[i + 4] : b[i]) + __shfl_xor_sync(0xffffffffu, h ? b[i] : b[i + 4], 8);
-    h = lane & 4;
-#pragma unroll
-    for (int i = 0; i < 2; ++i)
-        d[i] = (h ? c[i + 2] : c[i]) + __shfl_xor_sync(0xffffffffu, h ? c[i] : c[i + 2], 4);
-    h = lane & 2;
-    const float e = (h ? d[1] : d[0]) + __shfl_xor_sync(0xffffffffu, h ? d[0] : d[1], 2);
-    return e + __shfl_xor_sync(0xffffffffu, e, 1);
-}
-
+// The table path's fallback: each row's weight groups decoded exactly
+// (codewords from the codebooks in shared memory, summed with one binary16
+// rounding) and multiplied with the activations in fp32.
 template <class S>
 __global__ void __launch_bounds__(kLutThreads, 2)
 gemv_lut_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restrict__ cb,
@@ -230,54 +224,74 @@ gemv_lut_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restr
     constexpr int K = S::K;
     constexpr int NG = kLutGroups<K>;  // groups of the CTA
     constexpr int NSLOT = NG / 32;     // group slots per lane: 2 (2x8) or 4 (1x8)
-    extern __shared__ uint32_t lut[];  // [256][64] words, see above
+    static_assert(NG * S::kChunkBytes == kLutTileBytes, "one kilobyte of codes per row tile");
+    extern __shared__ __align__(16) uint8_t lut_smem[];
+    uint32_t *lut = reinterpret_cast<uint32_t *>(lut_smem);  // [256][64] words, see above
     __shared__ uint4 scb[K * 256];     // the codebooks, row k*256 + c
     __shared__ uint4 xs[NG];           // activations of the CTA's groups
-    __shared__ int s_overflow;
+    __shared__ uint32_t s_max[2];      // largest |C|, |x| (binary16 bits)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G0 = blockIdx.y * NG;
     const int rt0 = blockIdx.x * rt_per_cta;
     const int rt1 = min(L.rtiles, rt0 + rt_per_cta);
-    const int npairs = (rt1 - rt0 + 1) / 2;
-    // this warp's steps: row-tile pairs warp + kLutWarps j, j < nst
-    const int nst = (npairs - warp + kLutWarps - 1) / kLutWarps;
+    const int ntw = (rt1 - rt0 - warp + kLutWarps - 1) / kLutWarps;  // this warp's tiles warp + 16 i
+    uint8_t *ring = lut_smem + kLutBytes + warp * (kLutRing * kLutTileBytes);
 
-    // code chunk (row tile rt0 + 2p + t, group G0 + 32 j + lane); zero past the layer
-    auto fetch = [&](int p, int t, int j) {
-        const int rt = rt0 + 2 * p + t, g = G0 + 32 * j + lane;
-        return load_chunk<S>(packed, (size_t)rt * L.gp + g, p < npairs && rt < rt1 && g < L.G);
+    // codes of this warp's tile i into ring slot i % kLutRing: the tile's
+    // kilobyte for the CTA's groups, zero past the padded groups or rows
+    auto copy_tile = [&](int i) {
+        const int rt = rt0 + warp + kLutWarps * i;
+        const bool tile_live = i < ntw && rt < rt1;
+        const uint8_t *src = packed + ((size_t)rt * L.gp + G0) * S::kChunkBytes;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int off = h * 512 + lane * 16;
+            const bool live = tile_live && G0 + off / S::kChunkBytes < L.gp;
+            cp_async16(smem_u32(ring + (i % kLutRing) * kLutTileBytes + off), live ? src + off : packed,
+                       live ? 16u : 0u);
+        }
     };
-    // weights before the dependency wait: codebooks, the first steps' codes,
+    // weights before the dependency wait: codebooks, the first tiles' codes,
     // and the rest of the CTA's codes into L2
-    uint4 cw[K];
+    uint4 cw = make_uint4(0u, 0u, 0u, 0u);
+    if (threadIdx.x < K * 256) cw = ldg_stream_v4(cb + threadIdx.x);
 #pragma unroll
-    for (int k = 0; k < K; ++k) cw[k] = ldg_stream_v4(cb + k * 256 + threadIdx.x);
-    Chunk<S> ring[kLutRing][2][NSLOT];
-#pragma unroll
-    for (int i = 0; i < kLutRing; ++i)
-#pragma unroll
-        for (int t = 0; t < 2; ++t)
-#pragma unroll
-            for (int j = 0; j < NSLOT; ++j) ring[i][t][j] = fetch(i < nst ? warp + kLutWarps * i : npairs, t, j);
+    for (int i = 0; i < kLutRing; ++i) {
+        copy_tile(i);
+        cp_async_commit();
+    }
     {
-        const int first = rt0 + 2 * kLutWarps * kLutRing;  // row tiles below this are in the rings
-        const int ngl = min(NG, L.gp - G0);                // groups of this split in the padded layout
-        for (int rt = first + (int)threadIdx.x; rt < rt1; rt += kLutThreads)
+        const int ngl = min(NG, L.gp - G0);  // groups of this split in the padded layout
+        for (int rt = rt0 + kLutWarps * kLutRing + (int)threadIdx.x; rt < rt1; rt += kLutThreads)
             prefetch_l2_bulk(packed + ((size_t)rt * L.gp + G0) * S::kChunkBytes, (uint32_t)(ngl * S::kChunkBytes));
     }
+    if (threadIdx.x < 2) s_max[threadIdx.x] = 0;
     grid_dependency_wait();  // x, y and the workspace follow the previous launch
     grid_launch_dependents();
+    uint4 xv = make_uint4(0u, 0u, 0u, 0u);
     if (threadIdx.x < NG) {
         const int g = G0 + threadIdx.x;
-        xs[threadIdx.x] = (g < L.G) ? ldg_nc_v4(x + (size_t)g * 8) : make_uint4(0, 0, 0, 0);
+        if (g < L.G) xv = ldg_nc_v4(x + (size_t)g * 8);
+        xs[threadIdx.x] = xv;
     }
-#pragma unroll
-    for (int k = 0; k < K; ++k) scb[k * 256 + threadIdx.x] = cw[k];
-    if (threadIdx.x == 0) s_overflow = 0;
-    __syncthreads();
+    if (threadIdx.x < K * 256) scb[threadIdx.x] = cw;
     {
-        // warp w fills the codeword octets n = w + kLutWarps i (codeword kc =
-        // 8 n + 0..7, kc = k*256 + c) for every group of the CTA
+        const uint32_t mc = __reduce_max_sync(0xffffffffu, absmax_h8_bits(cw));
+        const uint32_t mx = __reduce_max_sync(0xffffffffu, absmax_h8_bits(xv));
+        __syncthreads();  // s_max cleared by threads 0, 1 before anyone updates it
+        if (lane == 0) {
+            atomicMax(&s_max[0], mc);
+            atomicMax(&s_max[1], mx);
+        }
+    }
+    __syncthreads();
+    // entries are bounded by 8 max|x| max|C|; NaN or infinity fails the test
+    const float bound = 8.f * __half2float(__ushort_as_half((unsigned short)s_max[0])) *
+                        __half2float(__ushort_as_half((unsigned short)s_max[1]));
+    const bool exact = !(bound < 65504.f);
+    if (!exact) {
+        // warp w fills the codeword octets n = w + 16 i (codeword kc = 8 n +
+        // 0..7, kc = k*256 + c) for every group of the CTA
         const int gid = lane >> 2, t4 = lane & 3;
         const uint32_t *xw = reinterpret_cast<const uint32_t *>(xs);
         const uint32_t *cbw = reinterpret_cast<const uint32_t *>(scb);
@@ -291,9 +305,7 @@ gemv_lut_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restr
         int off[4];  // slot s of a store writes word l = gid + off[s]
 #pragma unroll
         for (int s2 = 0; s2 < 4; ++s2) off[s2] = 8 * ((t4 + s2) & 3);
-        bool ovf = false;
         constexpr int NOCT = K * 256 / 8;
-#pragma unroll 2
         for (int n = warp; n < NOCT; n += kLutWarps) {
             const uint32_t b0 = cbw[(8 * n + gid) * 4 + t4];
 #pragma unroll
@@ -305,13 +317,6 @@ gemv_lut_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restr
                 mma_m16n8k8(lo1, a[4 * qq + 1][0], a[4 * qq + 1][1], b0);
                 mma_m16n8k8(hi0, a[4 * qq + 2][0], a[4 * qq + 2][1], b0);
                 mma_m16n8k8(hi1, a[4 * qq + 3][0], a[4 * qq + 3][1], b0);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    ovf |= (fabsf(lo0[e]) >= 65520.f && fabsf(lo0[e]) < INFINITY) ||
-                           (fabsf(lo1[e]) >= 65520.f && fabsf(lo1[e]) < INFINITY) ||
-                           (fabsf(hi0[e]) >= 65520.f && fabsf(hi0[e]) < INFINITY) ||
-                           (fabsf(hi1[e]) >= 65520.f && fabsf(hi1[e]) < INFINITY);
-                }
                 const int kc = 8 * n + 2 * t4;  // this lane's codewords kc, kc + 1
                 // word (c, q, l): c = kc & 255, q = the codebook (2x8) or qq (1x8)
                 const int q = (K == 2) ? (kc >> 8) : qq;
@@ -332,57 +337,65 @@ gemv_lut_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restr
                 }
             }
         }
-        if (ovf) s_overflow = 1;
     }
     __syncthreads();
-    const bool exact = s_overflow != 0;  // some entry is beyond binary16: decode each group instead
     const char *lutb = reinterpret_cast<const char *>(lut);
     const uint32_t lane4 = lane * 4;
     float *part = sk.partials + (size_t)blockIdx.y * L.rows8;
 
-    // sum over this lane's groups of row r of chunk tile t
-    auto row_value = [&](const Chunk<S> (&ch)[2][NSLOT], int t, int r) -> float {
-        if (!exact) {
-            __half h[4];
+    // the tile loop, with the rows' sums from the tables or, when they were
+    // skipped, from the exact decode (two copies of the loop, one per case)
+    auto tiles = [&](auto exact_tag) {
+        constexpr bool kExact = decltype(exact_tag)::value;
+        for (int i = 0; i < ntw; ++i) {
+            cp_async_wait<kLutRing - 1>();  // tile i has landed (this lane's copies, then every lane's)
+            __syncwarp();
+            Chunk<S> ch[NSLOT];
+            const uint8_t *slot = ring + (i % kLutRing) * kLutTileBytes;
 #pragma unroll
-            for (int j = 0; j < NSLOT; ++j)
-#pragma unroll
-                for (int k = 0; k < K; ++k) {
-                    const int q = (K == 2) ? k : (j >> 1), half = (K == 2) ? j : (j & 1);
-                    h[j * K + k] = lut_entry(lutb, lut_offset<S>(ch[t][j], r, k, lane4) + q * 128 + half * 2);
+            for (int j = 0; j < NSLOT; ++j) {
+                const uint8_t *cp = slot + (32 * j + lane) * S::kChunkBytes;
+                if constexpr (S::kChunkBytes == 16) {
+                    const uint4 v = *reinterpret_cast<const uint4 *>(cp);
+                    ch[j].w[0] = v.x, ch[j].w[1] = v.y, ch[j].w[2] = v.z, ch[j].w[3] = v.w;
+                } else {
+                    const uint2 v = *reinterpret_cast<const uint2 *>(cp);
+                    ch[j].w[0] = v.x, ch[j].w[1] = v.y;
                 }
-            return __half2float(__hadd(__hadd(h[0], h[1]), __hadd(h[2], h[3])));
-        }
-        float acc = 0.f;
+            }
+            __syncwarp();  // every lane has read the slot
+            copy_tile(i + kLutRing);
+            cp_async_commit();
+            float acc[8];
 #pragma unroll
-        for (int j = 0; j < NSLOT; ++j) {
-            uint4 tm[K];
+            for (int r = 0; r < 8; ++r) {
+                if constexpr (!kExact) {
+                    __half h[4];
 #pragma unroll
-            for (int k = 0; k < K; ++k) tm[k] = scb[k * 256 + ch[t][j].code(r, k)];
-            acc = dot8(sum_round_fast_h8<K>(tm), xs[32 * j + lane], acc);
-        }
-        return acc;
-    };
-
-    for (int j0 = 0; j0 < nst; j0 += kLutRing) {
+                    for (int j = 0; j < NSLOT; ++j)
 #pragma unroll
-        for (int i = 0; i < kLutRing; ++i) {
-            const int jj = j0 + i;
-            if (jj >= nst) break;
-            float acc[16];  // acc[8 t + r]: row r of tile t of the pair
+                        for (int k = 0; k < K; ++k) {
+                            const int q = (K == 2) ? k : (j >> 1), half = (K == 2) ? j : (j & 1);
+                            h[j * K + k] = *reinterpret_cast<const __half *>(
+                                lutb + lut_offset<S>(ch[j], r, k, lane4) + q * 128 + half * 2);
+                        }
+                    acc[r] = __half2float(__hadd(__hadd(h[0], h[1]), __hadd(h[2], h[3])));
+                } else {
+                    float a = 0.f;
 #pragma unroll
-            for (int t = 0; t < 2; ++t)
+                    for (int j = 0; j < NSLOT; ++j) {
+                        if (G0 + 32 * j + lane >= L.G) continue;  // a padding group weighs nothing
+                        uint4 tm[K];
 #pragma unroll
-                for (int r = 0; r < 8; ++r) acc[8 * t + r] = row_value(ring[i], t, r);
-            const int jn = jj + kLutRing;  // the step this ring slot takes next
-            const int pn = jn < nst ? warp + kLutWarps * jn : npairs;
-#pragma unroll
-            for (int t = 0; t < 2; ++t)
-#pragma unroll
-                for (int j = 0; j < NSLOT; ++j) ring[i][t][j] = fetch(pn, t, j);
-            const float v = warp_reduce16(acc, lane);
-            const int row = (rt0 + 2 * (warp + kLutWarps * jj)) * 8 + (lane >> 1);
-            if ((lane & 1) == 0 && row < rt1 * 8) {
+                        for (int k = 0; k < K; ++k) tm[k] = scb[k * 256 + ch[j].code(r, k)];
+                        a = dot8(sum_round_fast_h8<K>(tm), xs[32 * j + lane], a);
+                    }
+                    acc[r] = a;
+                }
+            }
+            const float v = warp_reduce8(acc, lane);
+            const int row = (rt0 + warp + kLutWarps * i) * 8 + reduced_row_of_lane(lane);
+            if ((lane & 3) == 0) {
                 if (gridDim.y == 1) {
                     if (row < L.out) {
                         const float sc = scales ? __half2float(__ushort_as_half(scales[row])) : 1.f;
@@ -393,9 +406,14 @@ gemv_lut_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restr
                 }
             }
         }
-    }
+    };
+    if (exact)
+        tiles(std::true_type{});
+    else
+        tiles(std::false_type{});
+    cp_async_wait<0>();
     if (gridDim.y == 1) return;
-    splitk_finish(L, sk, blockIdx.x, gridDim.y, rt0 * 8, (rt1 - rt0) * 8, 1, scales, y, nullptr, 0);
+    splitk_finish<4>(L, sk, blockIdx.x, gridDim.y, rt0 * 8, (rt1 - rt0) * 8, 1, scales, y, nullptr, 0);
 }
 
 // ---------------------------------------------------------------------------
@@ -546,6 +564,246 @@ gemv_1x16_cc_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__r
     const int row0 = blockIdx.x * kCcRowTiles * 8;
     splitk_finish(L, sk, blockIdx.x, gridDim.y, row0, min(kCcRowTiles * 8, L.rows8 - row0), NB, scales, y, ccs,
                   stage_bytes);
+}
+
+// ---------------------------------------------------------------------------
+// 1x16 and 2x8 at decode batches: weights decoded straight into mma.sync
+// register fragments.
+//
+// At batch 2..16 the tensor work of a decode-time product is tiny; what
+// costs is producing the weights.  This kernel never stores a decoded tile:
+// each warp decodes its weights in registers, in the layout of the A
+// operand of mma.sync m16n8k16 (binary16 in, fp32 accumulators), and
+// multiplies them there.  The contraction index is permuted so that the
+// four k-slots a lane holds in each half of the A fragment are four
+// consecutive weights of one group: lane (gid, t4) holds rows gid and
+// gid + 8 (two 8-row tiles), group t4 of a set of four groups, weights
+// 4h..4h+3 in half h.  So one 16-byte codeword per row and group feeds both
+// halves, and the B fragments (the activations) follow the same
+// permutation, prebuilt once per CTA in shared memory.
+//  * 1x16: the codeword is read straight into registers through L1
+//    (ld.global.nc), kRfAhead sets ahead, as the batch-1 CUDA-core path
+//    does; the bound is the rate of these random reads.
+//  * 2x8: the two codewords come from 8 replicas of the codebooks in
+//    shared memory (lane l reads replica l % 8, so the eight lanes of a
+//    16-byte access phase never conflict) and are added with one binary16
+//    rounding (the exact decode).
+// Codes: each warp copies quads of four sets (2 row tiles x 16 groups, one
+// 16-byte chunk per lane) into a ring of its own in shared memory with
+// cp.async, kRfRing quads in flight, and reads each lane's code from there.
+// CTA = 8 warps x 16 rows = 128 rows x `gc` groups; grid = (row blocks,
+// group splits); splits are finished by the last CTA of the row block.
+// Codes, codebooks and (1x16) the first codewords are requested before the
+// CTA waits for the previous launch; activations, outputs and the workspace
+// after it.
+// ---------------------------------------------------------------------------
+constexpr int kRfWarps = 8;
+constexpr int kRfThreads = kRfWarps * 32;
+constexpr int kRfRows = 16 * kRfWarps;  // rows per CTA
+constexpr int kRfRing = 3;              // quads of code chunks per warp ring
+constexpr int kRfAhead = 4;             // 1x16: sets whose codewords are requested ahead
+constexpr int kRfMaxGroups = 256;       // groups per CTA (activation fragments in shared memory)
+
+template <class S>
+struct RfTraits {
+    static constexpr bool kReplicas = (S::K == 2 && S::B == 8);  // 8 replicas of both codebooks
+    static constexpr int kBookBytes = kReplicas ? 8 * S::K * 256 * 16 : 0;
+};
+
+// bytes of dynamic shared memory: codebook replicas, per-warp code rings,
+// activation fragments of the CTA's groups
+template <class S, int NT>
+__host__ __device__ constexpr int rf_smem_bytes(int gc)
+{
+    return RfTraits<S>::kBookBytes + kRfWarps * kRfRing * 512 + gc * 128 * NT;
+}
+
+// D += A(16x16, row) * B(16x8, col), binary16 in, fp32 accumulate.
+__device__ __forceinline__ void mma_m16n8k16(float d[4], const uint32_t a[4], uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint16_t lds_u16(uint32_t addr)
+{
+    uint16_t v;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
+    return v;
+}
+
+template <class S, int NT>
+__global__ void __launch_bounds__(kRfThreads, 2)
+gemv_rf_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restrict__ cb,
+               const uint16_t *__restrict__ scales, const uint16_t *__restrict__ x, int batch,
+               uint16_t *__restrict__ y, SplitK sk, int gc)
+{
+    static_assert(S::kChunkBytes == 16, "16-bit packed words (1x16, 2x8)");
+    constexpr bool kRep = RfTraits<S>::kReplicas;
+    extern __shared__ __align__(16) uint8_t rf_smem[];
+    uint4 *rep = reinterpret_cast<uint4 *>(rf_smem);                        // [K*256][8] replicas
+    uint4 *rings = reinterpret_cast<uint4 *>(rf_smem + RfTraits<S>::kBookBytes);  // [warp][kRfRing][32]
+    uint2 *xfrag = reinterpret_cast<uint2 *>(rf_smem + RfTraits<S>::kBookBytes + kRfWarps * kRfRing * 512);
+    // xfrag: [set][half][NT][32] B fragments
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int gid = lane >> 2, t4 = lane & 3;
+    const int ta = blockIdx.x * (kRfRows / 8) + 2 * warp;  // this warp's row tiles ta, ta + 1
+    const int G0 = blockIdx.y * gc;
+    const int ng = min(gc, L.G - G0);
+    const int nquads = (ng + 15) / 16;
+    const int nsets = 4 * nquads;
+
+    // code quad q of this warp into ring slot q % kRfRing: lane l copies chunk
+    // (row tile ta + l / 16, group G0 + 16 q + l % 16); zeros past the layer
+    uint4 *ring = rings + warp * (kRfRing * 32);
+    auto copy_quad = [&](int q) {
+        const int rt = ta + (lane >> 4), g = G0 + 16 * q + (lane & 15);
+        const bool live = q < nquads && rt < L.rtiles && g < L.G;
+        const uint8_t *src = live ? packed + ((size_t)rt * L.gp + g) * 16 : packed;
+        cp_async16(smem_u32(ring + (q % kRfRing) * 32 + lane), src, live ? 16u : 0u);
+    };
+    // this lane's 16-bit code words of set s (rows gid of tiles ta, ta + 1)
+    const uint32_t ring_base = smem_u32(ring);
+    auto codes_of = [&](int s, uint32_t &wa, uint32_t &wb) {
+        const int q = s >> 2, sl = s & 3;
+        const uint32_t a = ring_base + (q % kRfRing) * 512 + (4 * sl + t4) * 16 + gid * 2;
+        wa = lds_u16(a);
+        wb = lds_u16(a + 16 * 16);
+    };
+
+#pragma unroll
+    for (int q = 0; q < kRfRing; ++q) {
+        copy_quad(q);
+        cp_async_commit();
+    }
+    if constexpr (kRep) {
+        // 8 replicas of both codebooks: replica r of codeword kc at slot
+        // 8 kc + r; consecutive threads fill consecutive slots, so the stores
+        // never conflict (the 8 reads of one codeword hit L1)
+        for (int i = threadIdx.x; i < S::K * 256 * 8; i += kRfThreads) rep[i] = ldg_nc_v4(cb + (i >> 3));
+    }
+    // quads 0 and 1 landed (this lane's copies, then every lane's)
+    cp_async_wait<kRfRing - 2>();
+    __syncwarp();
+    uint4 gw[kRfAhead][2];  // 1x16: codewords of sets s .. s + kRfAhead - 1 (rows gid of ta, ta + 1)
+    if constexpr (!kRep) {
+#pragma unroll
+        for (int i = 0; i < kRfAhead; ++i) {
+            uint32_t wa, wb;
+            codes_of(i, wa, wb);
+            gw[i][0] = ldg_nc_v4(cb + wa);
+            gw[i][1] = ldg_nc_v4(cb + wb);
+        }
+    }
+    grid_dependency_wait();  // x, y and the workspace follow the previous launch
+    grid_launch_dependents();
+    {
+        // B fragments straight from x: entry (s, h, nt, lane (gid, t4)) holds
+        // x rows 8 (G0 + 4 s + t4) + 4 h + {0, 1} and {2, 3} of column
+        // nt * 8 + gid (zero past the batch or the layer), every load of a
+        // thread in flight at once
+        const int nent = nsets * 2 * NT * 32;
+        for (int e = threadIdx.x; e < nent; e += kRfThreads) {
+            const int ln = e & 31, nt = (e >> 5) % NT, h = (e >> 5) / NT % 2, st = (e >> 5) / NT / 2;
+            const int n = nt * 8 + (ln >> 2), g = G0 + 4 * st + (ln & 3);
+            const bool live = n < batch && g < L.G;
+            const uint16_t *xp = x + ((size_t)8 * g + 4 * h) * batch + n;
+            uint32_t v[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) v[j] = live ? (uint32_t)__ldg(xp + j * batch) : 0u;
+            xfrag[e] = make_uint2(v[0] | (v[1] << 16), v[2] | (v[3] << 16));
+        }
+        __syncthreads();  // also publishes the codebook replicas
+    }
+
+    float d[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) d[nt][j] = 0.f;
+    const uint32_t xfrag_base = smem_u32(xfrag);
+    for (int q = 0; q < nquads; ++q) {
+        // quads q and q + 1 of this warp have landed
+        cp_async_wait<kRfRing - 2>();
+        __syncwarp();
+#pragma unroll
+        for (int sl = 0; sl < 4; ++sl) {
+            const int s = 4 * q + sl;
+            uint4 wrow[2];  // decoded weights of rows gid (tile ta) and gid (tile ta + 1), group t4 of set s
+            const bool glive = G0 + 4 * s + t4 < L.G;  // groups past the layer weigh nothing
+            if constexpr (kRep) {
+                uint32_t wa, wb;
+                codes_of(s, wa, wb);
+                const uint32_t c[2] = {wa, wb};
+#pragma unroll
+                for (int t = 0; t < 2; ++t) {
+                    const uint4 t0 = rep[8 * (c[t] & 0xffu) + (lane & 7)];
+                    const uint4 t1 = rep[8 * (256u + (c[t] >> 8)) + (lane & 7)];
+                    wrow[t] = add_round_h8(t0, t1);
+                }
+            } else {
+                wrow[0] = gw[sl % kRfAhead][0];
+                wrow[1] = gw[sl % kRfAhead][1];
+                const int sn = s + kRfAhead;  // its codewords are requested now (codes are in quads q, q + 1)
+                if (sn < nsets) {
+                    uint32_t wa, wb;
+                    codes_of(sn, wa, wb);
+                    gw[sl % kRfAhead][0] = ldg_nc_v4(cb + wa);
+                    gw[sl % kRfAhead][1] = ldg_nc_v4(cb + wb);
+                }
+            }
+            if (!glive) wrow[0] = wrow[1] = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const uint32_t a[4] = {u4_at(wrow[0], 2 * h), u4_at(wrow[1], 2 * h), u4_at(wrow[0], 2 * h + 1),
+                                       u4_at(wrow[1], 2 * h + 1)};
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    uint32_t b0, b1;
+                    asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];"
+                                 : "=r"(b0), "=r"(b1)
+                                 : "r"(xfrag_base + (uint32_t)((((s * 2 + h) * NT + nt) * 32 + lane) * 8)));
+                    mma_m16n8k16(d[nt], a, b0, b1);
+                }
+            }
+        }
+        __syncwarp();  // every lane is done with slot q % kRfRing
+        copy_quad(q + kRfRing);
+        cp_async_commit();
+    }
+    cp_async_wait<0>();
+
+    // rows gid of tiles ta, ta + 1; columns nt * 8 + 2 t4 + {0, 1}
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+        const int rt = ta + t, row = rt * 8 + gid;
+        if (rt >= L.rtiles) continue;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int col = nt * 8 + 2 * t4 + j;
+                if (col >= batch) continue;
+                const float v = d[nt][2 * t + j];
+                if (gridDim.y == 1) {
+                    if (row < L.out) {
+                        const float sc = scales ? __half2float(__ushort_as_half(scales[row])) : 1.f;
+                        y[(size_t)row * batch + col] = __half_as_ushort(__float2half_rn(sc * v));
+                    }
+                } else {
+                    sk.partials[((size_t)blockIdx.y * L.rows8 + row) * batch + col] = v;
+                }
+            }
+    }
+    if (gridDim.y == 1) return;
+    const int row0 = blockIdx.x * kRfRows;
+    const int stage_bytes = rf_smem_bytes<S, NT>(gc) - RfTraits<S>::kBookBytes;
+    splitk_finish(L, sk, blockIdx.x, gridDim.y, row0, min(kRfRows, L.rows8 - row0), batch, scales, y,
+                  reinterpret_cast<float4 *>(rings), stage_bytes);
 }
 
 // ---------------------------------------------------------------------------
@@ -962,7 +1220,7 @@ using namespace aqk;
 
 namespace {
 
-enum Path { kLut = 1, kTensor = 2, kCudaCores = 3 };
+enum Path { kLut = 1, kTensor = 2, kCudaCores = 3, kRegFrag = 4 };
 
 struct GemvPlan {
     Path path;
@@ -1028,12 +1286,12 @@ int lut_splits(const Geom &g)
     return (g.G + ng - 1) / ng;
 }
 
-// Row tiles per CTA of the table path (whole pairs of tiles): as many row
-// ranges as put one CTA on each SM in one wave.
+// Row tiles per CTA of the table path: as many row ranges as put one CTA
+// on each SM in one wave.
 int lut_rt_per_cta(const Geom &g)
 {
-    const int ranges = std::max(1, std::min((g.rtiles + 1) / 2, kNumSMs / lut_splits(g)));
-    return ((g.rtiles + ranges - 1) / ranges + 1) & ~1;
+    const int ranges = std::max(1, std::min(g.rtiles, kNumSMs / lut_splits(g)));
+    return (g.rtiles + ranges - 1) / ranges;
 }
 
 // Workspace of the table path: one partial sum per row and group split.
@@ -1041,6 +1299,46 @@ size_t lut_ws(const Geom &g)
 {
     const int ks = lut_splits(g);
     return ks > 1 ? kWsData + (size_t)ks * g.rows8 * sizeof(float) : kWsHeader;
+}
+
+// Register-fragment path (1x16 from batch 3, 2x8 from batch 2): groups per
+// CTA and group splits.  At most kRfMaxGroups groups per CTA, and few
+// enough that two CTAs fit on an SM; about two CTAs per SM in all.
+// Returns false when the layer's scheme does not take this path, or when
+// the split's partial sums would not fit `cap`.
+bool plan_rf(const Geom &g, int batch, size_t cap, GemvPlan &p)
+{
+    const bool k2 = (g.K == 2 && g.B == 8);
+    if (!(k2 || (g.K == 1 && g.B == 16))) return false;
+    if (batch < (k2 ? 2 : 3)) return false;
+    const int nt = batch <= 8 ? 1 : 2;
+    auto smem = [&](int gc) {
+        return k2 ? (nt == 1 ? rf_smem_bytes<Scheme<2, 8>, 1>(gc) : rf_smem_bytes<Scheme<2, 8>, 2>(gc))
+                  : (nt == 1 ? rf_smem_bytes<Scheme<1, 16>, 1>(gc) : rf_smem_bytes<Scheme<1, 16>, 2>(gc));
+    };
+    int gc_max = kRfMaxGroups;
+    while (gc_max > 16 && smem(gc_max) > 113 * 1024) gc_max -= 16;
+    const int nrb = (g.rtiles + kRfRows / 8 - 1) / (kRfRows / 8);
+    // as many splits as fill the two CTA slots of every SM in one wave; a
+    // second, partial wave would double the time of the SMs it lands on
+    const int s_target = std::max(1, 2 * kNumSMs / nrb);
+    int gc = std::min(gc_max, std::max(16, ((g.G + s_target - 1) / s_target + 15) / 16 * 16));
+    auto ws_of = [&](int gcv) {
+        const int ks = (g.G + gcv - 1) / gcv;
+        return ks > 1 ? kWsData + (size_t)ks * g.rows8 * batch * sizeof(float) : kWsHeader;
+    };
+    // fewer, longer splits while the partial sums do not fit
+    while (ws_of(gc) > cap && gc < ((g.G + 15) / 16) * 16 && gc < gc_max) gc += 16;
+    const int ks = (g.G + gc - 1) / gc;
+    if (ws_of(gc) > cap || (ks > 1 && nrb > kWsMaxCounters)) return false;
+    p.path = kRegFrag;
+    p.len = gc;
+    p.ks = ks;
+    p.grid_x = nrb;
+    p.counters = nrb;
+    p.slots = ks > 1 ? ks : 0;
+    p.cc_smem = smem(gc);
+    return true;
 }
 
 // `cap`: largest workspace the caller can offer (the no-allocation entry
@@ -1068,6 +1366,8 @@ GemvPlan plan_gemv(const Geom &g, int batch, size_t cap = ~(size_t)0)
         p.slots = p.ks > 1 ? p.ks : 0;
         const int nvec = kCcRowTiles * 8 * batch / 4;  // float4 of one row range's partial sums
         p.cc_smem = std::max(p.len * 32 * batch, std::min(kCcStage, p.ks > 1 ? p.ks * nvec * 16 : 0));
+    } else if (plan_rf(g, batch, cap, p)) {
+        // p is filled in
     } else if (batch == 1 && g.B == 8 && g.K <= 2 && lut_ws(g) <= cap) {
         p.path = kLut;
         p.ks = lut_splits(g);
@@ -1209,8 +1509,23 @@ cudaError_t launch_plan(const Geom &g, const GemvPlan &p, const void *packed, co
         };
         static_assert(kCcMaxBatch == 2, "one instantiation per batch on this path");
         e = batch == 1 ? cc(gemv_1x16_cc_kernel<1>) : cc(gemv_1x16_cc_kernel<2>);
+    } else if (p.path == kRegFrag) {
+        auto rf = [&](auto sch, auto ntc) {
+            using S = decltype(sch);
+            constexpr int NT = decltype(ntc)::value;
+            cudaError_t r = set_smem(gemv_rf_kernel<S, NT>, p.cc_smem);
+            if (r != cudaSuccess) return r;
+            return launch_pdl(pdl, gemv_rf_kernel<S, NT>, grid, dim3(kRfThreads), p.cc_smem, s, g, pk, c, scales, x,
+                              batch, y, sk, p.len);
+        };
+        using One = std::integral_constant<int, 1>;
+        using Two = std::integral_constant<int, 2>;
+        if (g.K == 2)
+            e = batch <= 8 ? rf(Scheme<2, 8>{}, One{}) : rf(Scheme<2, 8>{}, Two{});
+        else
+            e = batch <= 8 ? rf(Scheme<1, 16>{}, One{}) : rf(Scheme<1, 16>{}, Two{});
     } else if (p.path == kLut) {
-        const int smem = kLutBytes;  // the tables
+        const int smem = kLutSmem;  // the tables and the code rings
         auto lut = [&](auto sch) {
             using S = decltype(sch);
             if constexpr (S::B == 8 && S::K <= 2) {

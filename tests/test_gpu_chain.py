@@ -46,7 +46,8 @@ def _block_layers(K, B, seed, unit_gain=False):
         # gain ~1: the decoded weight's spread (K codebook terms) times
         # sqrt(in) times the RMS row scale (~1.04) is about one
         sigma = 1.0 / (np.sqrt(K * inp) * 1.04) if unit_gain else 0.02
-        layers[tag] = make_layer(LayerSpec(out, inp, K, B, codebook_sigma=sigma), (seed, li))
+        base = seed if isinstance(seed, tuple) else (seed,)
+        layers[tag] = make_layer(LayerSpec(out, inp, K, B, codebook_sigma=sigma), (*base, li))
     return layers
 
 

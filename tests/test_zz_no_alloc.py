@@ -35,7 +35,7 @@ CASES = [
     ((1000, 1032, 2, 8), 1), ((1000, 1032, 2, 8), 5), ((256, 512, 2, 8), 4),
 ]
 # usual workspace larger than the fixed array
-OVER_CAP = [((28672, 8192, 1, 16), 16), ((20000, 16384, 2, 8), 1)]
+OVER_CAP = [((28672, 8192, 1, 16), 16), ((32768, 16384, 2, 8), 1)]
 
 
 def _noalloc(dl, x):
