@@ -413,6 +413,8 @@ gemv_lut_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restr
         tiles(std::false_type{});
     cp_async_wait<0>();
     if (gridDim.y == 1) return;
+    // summed straight from L2, four slots in flight per float4 (measured
+    // faster here than staging the slots in the free code rings)
     splitk_finish<4>(L, sk, blockIdx.x, gridDim.y, rt0 * 8, (rt1 - rt0) * 8, 1, scales, y, nullptr, 0);
 }
 
@@ -611,11 +613,12 @@ struct RfTraits {
 };
 
 // bytes of dynamic shared memory: codebook replicas, per-warp code rings,
-// activation fragments of the CTA's groups
+// activation fragments of the CTA's groups (the kernel works in quads of
+// 16 groups, so a split of gc groups has fragments for gc rounded up to 16)
 template <class S, int NT>
 __host__ __device__ constexpr int rf_smem_bytes(int gc)
 {
-    return RfTraits<S>::kBookBytes + kRfWarps * kRfRing * 512 + gc * 128 * NT;
+    return RfTraits<S>::kBookBytes + kRfWarps * kRfRing * 512 + (gc + 15) / 16 * 16 * 128 * NT;
 }
 
 // D += A(16x16, row) * B(16x8, col), binary16 in, fp32 accumulate.
@@ -653,7 +656,8 @@ gemv_rf_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restri
     const int gid = lane >> 2, t4 = lane & 3;
     const int ta = blockIdx.x * (kRfRows / 8) + 2 * warp;  // this warp's row tiles ta, ta + 1
     const int G0 = blockIdx.y * gc;
-    const int ng = min(gc, L.G - G0);
+    const int ng = min(gc, L.G - G0);   // groups of this split (gc is a multiple of 4)
+    const int G1 = G0 + ng;              // groups at or past this one belong to the next split
     const int nquads = (ng + 15) / 16;
     const int nsets = 4 * nquads;
 
@@ -662,7 +666,7 @@ gemv_rf_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restri
     uint4 *ring = rings + warp * (kRfRing * 32);
     auto copy_quad = [&](int q) {
         const int rt = ta + (lane >> 4), g = G0 + 16 * q + (lane & 15);
-        const bool live = q < nquads && rt < L.rtiles && g < L.G;
+        const bool live = q < nquads && rt < L.rtiles && g < G1;
         const uint8_t *src = live ? packed + ((size_t)rt * L.gp + g) * 16 : packed;
         cp_async16(smem_u32(ring + (q % kRfRing) * 32 + lane), src, live ? 16u : 0u);
     };
@@ -686,11 +690,11 @@ gemv_rf_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restri
         // never conflict (the 8 reads of one codeword hit L1)
         for (int i = threadIdx.x; i < S::K * 256 * 8; i += kRfThreads) rep[i] = ldg_nc_v4(cb + (i >> 3));
     }
-    // quads 0 and 1 landed (this lane's copies, then every lane's)
-    cp_async_wait<kRfRing - 2>();
-    __syncwarp();
     uint4 gw[kRfAhead][2];  // 1x16: codewords of sets s .. s + kRfAhead - 1 (rows gid of ta, ta + 1)
     if constexpr (!kRep) {
+        // quads 0 and 1 landed (this lane's copies, then every lane's)
+        cp_async_wait<kRfRing - 2>();
+        __syncwarp();
 #pragma unroll
         for (int i = 0; i < kRfAhead; ++i) {
             uint32_t wa, wb;
@@ -706,16 +710,40 @@ gemv_rf_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restri
         // x rows 8 (G0 + 4 s + t4) + 4 h + {0, 1} and {2, 3} of column
         // nt * 8 + gid (zero past the batch or the layer), every load of a
         // thread in flight at once
-        const int nent = nsets * 2 * NT * 32;
-        for (int e = threadIdx.x; e < nent; e += kRfThreads) {
-            const int ln = e & 31, nt = (e >> 5) % NT, h = (e >> 5) / NT % 2, st = (e >> 5) / NT / 2;
-            const int n = nt * 8 + (ln >> 2), g = G0 + 4 * st + (ln & 3);
-            const bool live = n < batch && g < L.G;
-            const uint16_t *xp = x + ((size_t)8 * g + 4 * h) * batch + n;
-            uint32_t v[4];
+        if (batch % 8 == 0) {
+            // the four x rows of an entry's column block are 16-byte loads:
+            // item (s, h, nt, t4) reads rows 8 g + 4 h + j, j < 4, columns
+            // nt * 8 .. + 7, and writes the entries of its eight lanes gid
+            const int nitem = nsets * 2 * NT * 4;
+            for (int it = threadIdx.x; it < nitem; it += kRfThreads) {
+                const int t4i = it & 3, nt = (it >> 2) % NT, h = (it >> 2) / NT % 2, st = (it >> 2) / NT / 2;
+                const int g = G0 + 4 * st + t4i;
+                uint4 r[4];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) v[j] = live ? (uint32_t)__ldg(xp + j * batch) : 0u;
-            xfrag[e] = make_uint2(v[0] | (v[1] << 16), v[2] | (v[3] << 16));
+                for (int j = 0; j < 4; ++j)
+                    r[j] = g < G1 ? ldg_nc_v4(x + ((size_t)8 * g + 4 * h + j) * batch + nt * 8)
+                                   : make_uint4(0u, 0u, 0u, 0u);
+                uint2 *dst = xfrag + ((st * 2 + h) * NT + nt) * 32 + t4i;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    uint32_t v[4];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) v[j] = (u4_at(r[j], c >> 1) >> (16 * (c & 1))) & 0xffffu;
+                    dst[4 * c] = make_uint2(v[0] | (v[1] << 16), v[2] | (v[3] << 16));
+                }
+            }
+        } else {
+            const int nent = nsets * 2 * NT * 32;
+            for (int e = threadIdx.x; e < nent; e += kRfThreads) {
+                const int ln = e & 31, nt = (e >> 5) % NT, h = (e >> 5) / NT % 2, st = (e >> 5) / NT / 2;
+                const int n = nt * 8 + (ln >> 2), g = G0 + 4 * st + (ln & 3);
+                const bool live = n < batch && g < G1;
+                const uint16_t *xp = x + ((size_t)8 * g + 4 * h) * batch + n;
+                uint32_t v[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) v[j] = live ? (uint32_t)__ldg(xp + j * batch) : 0u;
+                xfrag[e] = make_uint2(v[0] | (v[1] << 16), v[2] | (v[3] << 16));
+            }
         }
         __syncthreads();  // also publishes the codebook replicas
     }
@@ -734,7 +762,7 @@ gemv_rf_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restri
         for (int sl = 0; sl < 4; ++sl) {
             const int s = 4 * q + sl;
             uint4 wrow[2];  // decoded weights of rows gid (tile ta) and gid (tile ta + 1), group t4 of set s
-            const bool glive = G0 + 4 * s + t4 < L.G;  // groups past the layer weigh nothing
+            const bool glive = G0 + 4 * s + t4 < G1;  // groups past the split weigh nothing here
             if constexpr (kRep) {
                 uint32_t wa, wb;
                 codes_of(s, wa, wb);
@@ -1319,16 +1347,30 @@ bool plan_rf(const Geom &g, int batch, size_t cap, GemvPlan &p)
     int gc_max = kRfMaxGroups;
     while (gc_max > 16 && smem(gc_max) > 113 * 1024) gc_max -= 16;
     const int nrb = (g.rtiles + kRfRows / 8 - 1) / (kRfRows / 8);
-    // as many splits as fill the two CTA slots of every SM in one wave; a
-    // second, partial wave would double the time of the SMs it lands on
-    const int s_target = std::max(1, 2 * kNumSMs / nrb);
-    int gc = std::min(gc_max, std::max(16, ((g.G + s_target - 1) / s_target + 15) / 16 * 16));
     auto ws_of = [&](int gcv) {
         const int ks = (g.G + gcv - 1) / gcv;
         return ks > 1 ? kWsData + (size_t)ks * g.rows8 * batch * sizeof(float) : kWsHeader;
     };
-    // fewer, longer splits while the partial sums do not fit
-    while (ws_of(gc) > cap && gc < ((g.G + 15) / 16) * 16 && gc < gc_max) gc += 16;
+    // the split (groups per CTA, a multiple of 4) whose busiest SM has the
+    // least work: CTAs beyond the two slots of every SM form a second wave,
+    // and an SM that runs two CTAs takes about twice as long as one with one
+    int gc = std::min(gc_max, (g.G + 3) / 4 * 4);
+    double best = 0;
+    for (int ks = 1; ks <= (g.G + 3) / 4; ++ks) {
+        const int gcv = (g.G + ks - 1) / ks;
+        const int gc4 = (gcv + 3) / 4 * 4;
+        if (gc4 > gc_max || (g.G + gc4 - 1) / gc4 != ks) continue;
+        if (gc4 < std::min(32, (g.G + 3) / 4 * 4)) break;  // at least 8 sets per CTA: fixed costs dominate below
+        if (ws_of(gc4) > cap || (ks > 1 && nrb > kWsMaxCounters)) continue;
+        const long ctas = (long)nrb * ks;
+        const long per_sm = (ctas + kNumSMs - 1) / kNumSMs;  // CTAs on the busiest SM
+        const double load = (double)per_sm * gc4 + (per_sm > 2 ? 1e9 : 0);  // groups it works through
+        if (best == 0 || load < best) {
+            best = load;
+            gc = gc4;
+        }
+        if (ctas > 2L * kNumSMs) break;
+    }
     const int ks = (g.G + gc - 1) / gc;
     if (ws_of(gc) > cap || (ks > 1 && nrb > kWsMaxCounters)) return false;
     p.path = kRegFrag;
