@@ -252,5 +252,7 @@ def aq_gather_probe(codebook, codes, n: int, mode: int, sink, stream=None) -> No
     clusters' shared memory; mode 2: through L1 into registers, as the
     batch-1 CUDA-core GEMV does; mode 3: no codeword, ``codes`` itself read
     once as a stream, the read-only HBM bandwidth; ``codebook`` may then be
-    None); per-thread XOR checksums go to ``sink``."""
+    None; mode 4: the codebook sliced over 8-CTA clusters' shared memory,
+    each code handled by the CTA holding its slice); per-thread XOR
+    checksums go to ``sink``."""
     _check("aq_gather_probe", lib.aq_gather_probe(_ptr(codebook), _ptr(codes), n, mode, _ptr(sink), _stream(stream)))

@@ -258,14 +258,14 @@ aq_status aq_param_grad(const aq_layer_desc *desc, const void *packed, const uin
 
 size_t aq_gather_probe_sink_bytes(int mode)
 {
-    if (mode < 0 || mode > 3) return 0;
+    if (mode < 0 || mode > 4) return 0;
     return aqh::gather_probe_sink_bytes(mode);
 }
 
 aq_status aq_gather_probe(const uint16_t *codebook, const uint16_t *codes, size_t n, int mode, void *sink,
                           aq_stream_t stream)
 {
-    if (mode < 0 || mode > 3) return AQ_ERR_INVALID_ARG;
+    if (mode < 0 || mode > 4) return AQ_ERR_INVALID_ARG;
     if ((mode != 3 && !codebook) || !codes || !sink || n == 0 || n % 8 || n > ((size_t)1 << 36))
         return AQ_ERR_INVALID_ARG;
     if ((codebook && !aligned16(codebook)) || !aligned16(codes) || !aligned16(sink)) return AQ_ERR_MISALIGNED;

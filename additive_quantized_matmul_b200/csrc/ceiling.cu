@@ -18,6 +18,14 @@
 //    GEMV): three CTAs of 256 threads per SM, a chunk's 8 codewords read
 //    with ld.global.nc into registers, no shared memory (L1 keeps what it
 //    can of the codebook).
+//  * mode 4 (codebook slices, work moved to the slice): clusters of 8 CTAs
+//    of 512 threads, each holding one eighth of the codebook (128 KiB) in
+//    its own shared memory; every CTA of a cluster reads the cluster's code
+//    chunks (from L2: each chunk is read by the cluster's 8 CTAs) and
+//    handles only the codes whose top 3 bits name its slice, with local
+//    shared-memory reads.  The route a 1x16 product would take if it kept
+//    the codebook on chip and reduced the 8 CTAs' partial sums through
+//    distributed shared memory once per row tile.
 //  * mode 3 (read-only HBM stream, the cross-check of the copy bandwidth
 //    the HBM roofline uses): the `codes` array itself is read once, 16
 //    bytes per load, eight loads in flight per thread, four CTAs of 256
@@ -168,6 +176,36 @@ __device__ __forceinline__ uint4 ld_peer_shared(uint32_t local_addr, uint32_t ra
     return v;
 }
 
+constexpr int kProbeSliceThreads = 512;
+
+__global__ void __launch_bounds__(kProbeSliceThreads, 1)
+probe_slice_kernel(const uint4 *__restrict__ cb, const uint4 *__restrict__ chunks, long nchunks, uint4 *sink)
+{
+    extern __shared__ uint4 slice_words[];  // codewords [rank * kSliceWords, (rank + 1) * kSliceWords)
+    const int t = threadIdx.x;
+    const uint32_t rank = cluster_ctarank();
+    const long cluster = blockIdx.x / kClusterCtas, nclusters = gridDim.x / kClusterCtas;
+    for (int i = t; i < kSliceWords; i += kProbeSliceThreads)
+        cp_async16(smem_u32(slice_words + i), cb + (size_t)rank * kSliceWords + i, 16u);
+    cp_async_commit();
+    cp_async_wait<0>();
+    __syncthreads();
+    grid_launch_dependents();
+    // chunk q of the cluster's share, the same sequence in its 8 CTAs
+    const long stride = nclusters * kProbeSliceThreads;
+    uint4 acc = make_uint4(0u, 0u, 0u, 0u);
+    for (long q = cluster * kProbeSliceThreads + t; q < nchunks; q += stride) {
+        const uint4 w = ldg_stream_v4(chunks + q);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const uint32_t c = code_of(w, j);
+            if ((c >> 13) == rank) xor_into(acc, slice_words[c & (kSliceWords - 1)]);
+        }
+    }
+    grid_dependency_wait();  // the previous launch on the stream may still write the sink
+    sink[(long)blockIdx.x * kProbeSliceThreads + t] = acc;
+}
+
 __global__ void __launch_bounds__(kProbeThreads)
 probe_dsmem_kernel(const uint4 *__restrict__ cb, const uint4 *__restrict__ chunks, long nchunks, uint4 *sink)
 {
@@ -209,10 +247,13 @@ namespace {
 
 int probe_l2_ctas() { return 2 * kNumSMs; }
 
-cudaError_t probe_dsmem_ctas(int *ctas)
+// CTAs of whole 8-CTA clusters that run at once (mode 1: 128 threads,
+// mode 4: 512), at most one per SM
+cudaError_t probe_cluster_ctas(int mode, int *ctas)
 {
     const int smem = kSliceWords * 16;
-    cudaError_t e = cudaFuncSetAttribute(probe_dsmem_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    const void *kern = mode == 4 ? (const void *)probe_slice_kernel : (const void *)probe_dsmem_kernel;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
@@ -221,14 +262,14 @@ cudaError_t probe_dsmem_ctas(int *ctas)
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.gridDim = dim3(kClusterCtas);
-    cfg.blockDim = dim3(kProbeThreads);
+    cfg.blockDim = dim3(mode == 4 ? kProbeSliceThreads : kProbeThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int clusters = 0;
-    e = cudaOccupancyMaxActiveClusters(&clusters, (void *)probe_dsmem_kernel, &cfg);
+    e = cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg);
     if (e != cudaSuccess) return e;
-    *ctas = std::max(1, clusters) * kClusterCtas;
+    *ctas = std::min(std::max(1, clusters) * kClusterCtas, kNumSMs / kClusterCtas * kClusterCtas);
     return cudaSuccess;
 }
 
@@ -239,6 +280,7 @@ size_t gather_probe_sink_bytes(int mode)
     // mode 1 runs at most one CTA per SM (128 KiB of shared memory each)
     if (mode == 2) return (size_t)kProbeLdgPerSM * kNumSMs * kProbeLdgThreads * sizeof(uint4);
     if (mode == 3) return (size_t)kProbeStreamPerSM * kNumSMs * kProbeStreamThreads * sizeof(uint4);
+    if (mode == 4) return (size_t)kNumSMs * kProbeSliceThreads * sizeof(uint4);
     const int ctas = mode == 0 ? probe_l2_ctas() : kNumSMs;
     return (size_t)ctas * kProbeThreads * sizeof(uint4);
 }
@@ -279,10 +321,11 @@ cudaError_t launch_gather_probe(const uint16_t *codebook, const uint16_t *codes,
         cfg.numAttrs = 1;
         e = cudaLaunchKernelEx(&cfg, probe_l2_kernel, cb, chunks, nchunks, out);
     } else {
+        // modes 1 and 4: whole 8-CTA clusters, at most one CTA per SM (the
+        // sink holds one CTA per SM)
         int ctas = 0;
-        e = probe_dsmem_ctas(&ctas);
+        e = probe_cluster_ctas(mode, &ctas);
         if (e != cudaSuccess) return e;
-        ctas = std::min(ctas, kNumSMs / kClusterCtas * kClusterCtas);  // the sink holds one CTA per SM
         attr[1].id = cudaLaunchAttributeClusterDimension;
         attr[1].val.clusterDim.x = kClusterCtas;
         attr[1].val.clusterDim.y = 1;
@@ -290,7 +333,12 @@ cudaError_t launch_gather_probe(const uint16_t *codebook, const uint16_t *codes,
         cfg.gridDim = dim3(ctas);
         cfg.dynamicSmemBytes = kSliceWords * 16;
         cfg.numAttrs = 2;
-        e = cudaLaunchKernelEx(&cfg, probe_dsmem_kernel, cb, chunks, nchunks, out);
+        if (mode == 4) {
+            cfg.blockDim = dim3(kProbeSliceThreads);
+            e = cudaLaunchKernelEx(&cfg, probe_slice_kernel, cb, chunks, nchunks, out);
+        } else {
+            e = cudaLaunchKernelEx(&cfg, probe_dsmem_kernel, cb, chunks, nchunks, out);
+        }
     }
     if (e != cudaSuccess) return e;
     return cudaGetLastError();

@@ -599,17 +599,20 @@ gemv_1x16_cc_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__r
 // CTA waits for the previous launch; activations, outputs and the workspace
 // after it.
 // ---------------------------------------------------------------------------
-constexpr int kRfWarps = 8;
-constexpr int kRfThreads = kRfWarps * 32;
-constexpr int kRfRows = 16 * kRfWarps;  // rows per CTA
 constexpr int kRfRing = 3;              // quads of code chunks per warp ring
 constexpr int kRfAhead = 4;             // 1x16: sets whose codewords are requested ahead
 constexpr int kRfMaxGroups = 256;       // groups per CTA (activation fragments in shared memory)
 
+// 2x8: one CTA of 16 warps per SM, so that the 64 KiB of codebook
+// replicas are built once per SM; 1x16: two CTAs of 8 warps per SM.
 template <class S>
 struct RfTraits {
     static constexpr bool kReplicas = (S::K == 2 && S::B == 8);  // 8 replicas of both codebooks
     static constexpr int kBookBytes = kReplicas ? 8 * S::K * 256 * 16 : 0;
+    static constexpr int kWarps = kReplicas ? 16 : 8;
+    static constexpr int kThreads = kWarps * 32;
+    static constexpr int kRows = 16 * kWarps;  // rows per CTA
+    static constexpr int kPerSM = kReplicas ? 1 : 2;
 };
 
 // bytes of dynamic shared memory: codebook replicas, per-warp code rings,
@@ -618,7 +621,7 @@ struct RfTraits {
 template <class S, int NT>
 __host__ __device__ constexpr int rf_smem_bytes(int gc)
 {
-    return RfTraits<S>::kBookBytes + kRfWarps * kRfRing * 512 + (gc + 15) / 16 * 16 * 128 * NT;
+    return RfTraits<S>::kBookBytes + RfTraits<S>::kWarps * kRfRing * 512 + (gc + 15) / 16 * 16 * 128 * NT;
 }
 
 // D += A(16x16, row) * B(16x8, col), binary16 in, fp32 accumulate.
@@ -639,7 +642,7 @@ __device__ __forceinline__ uint16_t lds_u16(uint32_t addr)
 }
 
 template <class S, int NT>
-__global__ void __launch_bounds__(kRfThreads, 2)
+__global__ void __launch_bounds__(RfTraits<S>::kThreads, RfTraits<S>::kPerSM)
 gemv_rf_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restrict__ cb,
                const uint16_t *__restrict__ scales, const uint16_t *__restrict__ x, int batch,
                uint16_t *__restrict__ y, SplitK sk, int gc)
@@ -649,7 +652,8 @@ gemv_rf_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restri
     extern __shared__ __align__(16) uint8_t rf_smem[];
     uint4 *rep = reinterpret_cast<uint4 *>(rf_smem);                        // [K*256][8] replicas
     uint4 *rings = reinterpret_cast<uint4 *>(rf_smem + RfTraits<S>::kBookBytes);  // [warp][kRfRing][32]
-    uint2 *xfrag = reinterpret_cast<uint2 *>(rf_smem + RfTraits<S>::kBookBytes + kRfWarps * kRfRing * 512);
+    constexpr int kRfThreads = RfTraits<S>::kThreads, kRfRows = RfTraits<S>::kRows;
+    uint2 *xfrag = reinterpret_cast<uint2 *>(rf_smem + RfTraits<S>::kBookBytes + RfTraits<S>::kWarps * kRfRing * 512);
     // xfrag: [set][half][NT][32] B fragments
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -1344,9 +1348,11 @@ bool plan_rf(const Geom &g, int batch, size_t cap, GemvPlan &p)
         return k2 ? (nt == 1 ? rf_smem_bytes<Scheme<2, 8>, 1>(gc) : rf_smem_bytes<Scheme<2, 8>, 2>(gc))
                   : (nt == 1 ? rf_smem_bytes<Scheme<1, 16>, 1>(gc) : rf_smem_bytes<Scheme<1, 16>, 2>(gc));
     };
-    int gc_max = kRfMaxGroups;
-    while (gc_max > 16 && smem(gc_max) > 113 * 1024) gc_max -= 16;
-    const int nrb = (g.rtiles + kRfRows / 8 - 1) / (kRfRows / 8);
+    const int rows = k2 ? RfTraits<Scheme<2, 8>>::kRows : RfTraits<Scheme<1, 16>>::kRows;
+    const int per_sm_slots = k2 ? RfTraits<Scheme<2, 8>>::kPerSM : RfTraits<Scheme<1, 16>>::kPerSM;
+    int gc_max = kRfMaxGroups;  // as many groups as fit the CTAs an SM holds
+    while (gc_max > 16 && smem(gc_max) > (per_sm_slots == 1 ? 220 : 113) * 1024) gc_max -= 16;
+    const int nrb = (g.rtiles + rows / 8 - 1) / (rows / 8);
     auto ws_of = [&](int gcv) {
         const int ks = (g.G + gcv - 1) / gcv;
         return ks > 1 ? kWsData + (size_t)ks * g.rows8 * batch * sizeof(float) : kWsHeader;
@@ -1364,12 +1370,12 @@ bool plan_rf(const Geom &g, int batch, size_t cap, GemvPlan &p)
         if (ws_of(gc4) > cap || (ks > 1 && nrb > kWsMaxCounters)) continue;
         const long ctas = (long)nrb * ks;
         const long per_sm = (ctas + kNumSMs - 1) / kNumSMs;  // CTAs on the busiest SM
-        const double load = (double)per_sm * gc4 + (per_sm > 2 ? 1e9 : 0);  // groups it works through
+        const double load = (double)per_sm * gc4 + (per_sm > per_sm_slots ? 1e9 : 0);  // groups it works through
         if (best == 0 || load < best) {
             best = load;
             gc = gc4;
         }
-        if (ctas > 2L * kNumSMs) break;
+        if (ctas > (long)per_sm_slots * kNumSMs) break;
     }
     const int ks = (g.G + gc - 1) / gc;
     if (ws_of(gc) > cap || (ks > 1 && nrb > kWsMaxCounters)) return false;
@@ -1557,7 +1563,7 @@ cudaError_t launch_plan(const Geom &g, const GemvPlan &p, const void *packed, co
             constexpr int NT = decltype(ntc)::value;
             cudaError_t r = set_smem(gemv_rf_kernel<S, NT>, p.cc_smem);
             if (r != cudaSuccess) return r;
-            return launch_pdl(pdl, gemv_rf_kernel<S, NT>, grid, dim3(kRfThreads), p.cc_smem, s, g, pk, c, scales, x,
+            return launch_pdl(pdl, gemv_rf_kernel<S, NT>, grid, dim3(RfTraits<S>::kThreads), p.cc_smem, s, g, pk, c, scales, x,
                               batch, y, sk, p.len);
         };
         using One = std::integral_constant<int, 1>;

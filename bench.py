@@ -354,7 +354,8 @@ def gather_ceiling(aq, units, kernels, stream, reps: int = 5):
     with CUDA events like the GEMV; mode 0 reads from L2 into shared memory
     as the tensor-core GEMV's decoders do, mode 1 from the codebook split
     over 8-CTA clusters' shared memory, mode 2 through L1 into registers as
-    the batch-1 CUDA-core GEMV does."""
+    the batch-1 CUDA-core GEMV does, mode 4 from the codebook sliced over
+    8-CTA clusters with each code handled by the CTA holding its slice."""
     import torch
     rows, seen = [], set()
     for u in units:
@@ -364,7 +365,7 @@ def gather_ceiling(aq, units, kernels, stream, reps: int = 5):
         seen.add(u["tag"])
         n = spec.out_features * spec.in_features // 64 * 8  # the layer's codes, a multiple of 8
         row = {"layer": u["tag"], "codes": n}
-        for mode, key in ((0, "l2_cp_async"), (1, "dsmem_cluster8"), (2, "l1_ldg")):
+        for mode, key in ((0, "l2_cp_async"), (1, "dsmem_cluster8"), (2, "l1_ldg"), (4, "slice_cluster8")):
             sink = torch.zeros(aq.aq_gather_probe_sink_bytes(mode) // 4, dtype=torch.int32, device=stream.device)
 
             def once():
@@ -390,10 +391,12 @@ def gather_ceiling(aq, units, kernels, stream, reps: int = 5):
             row[f"{key}_us_per_layer"] = round(us, 3)
             row[f"{key}_gathers_per_s"] = round(n / (us * 1e-6), -6)
             del graph
-        # the ceiling is the faster route: through L1 into registers (the
-        # batch-1 CUDA-core path) or from L2 into shared memory (the
-        # tensor-core path)
+        # the ceiling is the fastest route the products take: through L1
+        # into registers (CUDA-core and register-fragment kernels) or from L2
+        # into shared memory; the codebook-slice route (mode 4) is reported
+        # beside it as the route a kernel could take instead
         row["ceiling_us_per_layer"] = min(row["l2_cp_async_us_per_layer"], row["l1_ldg_us_per_layer"])
+        row["slice_vs_l1"] = round(row["l1_ldg_us_per_layer"] / row["slice_cluster8_us_per_layer"], 3)
         for k in kernels:
             if k["layer"] == u["tag"] and "us_per_layer" in k:
                 row[f"gemv_n{k['n']}_us"] = k["us_per_layer"]

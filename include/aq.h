@@ -336,13 +336,18 @@ aq_status aq_param_grad(const aq_layer_desc *desc, const void *packed, const uin
  *           with distributed shared-memory loads;
  *   mode 2  into registers through L1 (ld.global.nc), as aq_gemv's batch-1
  *           1x16 path does (three CTAs of 256 threads per SM);
+ *   mode 4  the codebook sliced over the shared memory of 8-CTA clusters
+ *           (128 KiB per CTA, loaded once per call), the work moved to the
+ *           slice: every CTA of a cluster reads the cluster's codes and
+ *           reads, from its own shared memory, the codewords of the codes
+ *           whose top 3 bits name its slice;
  *   mode 3  no codeword at all: `codes` itself is read once as a stream of
  *           16-byte loads (L1 bypassed, four CTAs of 256 threads per SM),
  *           the read-only HBM bandwidth when the array is much larger
  *           than L2 (a cross-check of the copy bandwidth the HBM roofline
  *           uses).  `codebook` is not read and may be NULL; the checksum
  *           XOR is then that of the codes' 32-bit words.
- *   codebook  [65536][8] binary16, device, 16-byte aligned (modes 0-2),
+ *   codebook  [65536][8] binary16, device, 16-byte aligned (modes 0-2, 4),
  *   codes     n 16-bit codes, device, 16-byte aligned, n a multiple of 8
  *             (a 1x16 layer's packed codes are such an array),
  *   sink      device, >= aq_gather_probe_sink_bytes(mode) bytes, 16-byte

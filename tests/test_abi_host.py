@@ -248,9 +248,10 @@ def test_encode_argument_errors():
 
 def test_gather_probe_argument_errors():
     f = aq.lib.aq_gather_probe
-    assert all(aq.aq_gather_probe_sink_bytes(m) > 0 for m in (0, 1, 2, 3))
-    assert aq.aq_gather_probe_sink_bytes(4) == 0 and aq.aq_gather_probe_sink_bytes(-1) == 0
-    assert f(FAKE, FAKE, 64, 4, FAKE, None) == 1       # unknown mode
+    assert all(aq.aq_gather_probe_sink_bytes(m) > 0 for m in (0, 1, 2, 3, 4))
+    assert aq.aq_gather_probe_sink_bytes(5) == 0 and aq.aq_gather_probe_sink_bytes(-1) == 0
+    assert f(FAKE, FAKE, 64, 5, FAKE, None) == 1       # unknown mode
+    assert f(None, FAKE, 64, 4, FAKE, None) == 1       # the slice mode reads the codebook
     assert f(None, None, 64, 3, FAKE, None) == 1       # the stream mode still needs codes
     assert f(None, FAKE, 64, 3, None, None) == 1       # and a sink
     assert f(None, FAKE + 8, 64, 3, FAKE, None) == 3   # misaligned codes (no codebook needed)

@@ -1,7 +1,7 @@
-"""aq_gather_probe: the codeword-read ceiling of the 1x16 product (modes 0-2)
+"""aq_gather_probe: the codeword-read ceiling of the 1x16 product (modes 0-2, 4)
 and the read-only HBM stream (mode 3).
 
-Modes 0-2 read codebook[codes[i]] for every code and XOR each 32-bit word
+Modes 0-2 and 4 read codebook[codes[i]] for every code and XOR each 32-bit word
 they read into a per-thread checksum.  These tests check, through the C ABI,
 that each mode reads exactly the codewords the codes select: the XOR of all
 checksums must equal the XOR of those codewords, computed here with numpy
@@ -23,7 +23,7 @@ def _expected_xor(cb_words: np.ndarray, codes: np.ndarray) -> np.ndarray:
     return np.bitwise_xor.reduce(cb_words[codes.astype(np.int64)], axis=0)
 
 
-@pytest.mark.parametrize("mode", [0, 1, 2])
+@pytest.mark.parametrize("mode", [0, 1, 2, 4])
 @pytest.mark.parametrize("n", [8, 4096 * 512, 4096 * 512 + 8 * 37])
 def test_probe_reads_the_selected_codewords(mode, n):
     rng = np.random.default_rng(n + mode)
