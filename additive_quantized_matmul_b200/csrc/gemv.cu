@@ -645,7 +645,7 @@ template <class S, int NT>
 __global__ void __launch_bounds__(RfTraits<S>::kThreads, RfTraits<S>::kPerSM)
 gemv_rf_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restrict__ cb,
                const uint16_t *__restrict__ scales, const uint16_t *__restrict__ x, int batch,
-               uint16_t *__restrict__ y, SplitK sk, int gc)
+               uint16_t *__restrict__ y, SplitK sk, int gc, int smem_bytes)
 {
     static_assert(S::kChunkBytes == 16, "16-bit packed words (1x16, 2x8)");
     constexpr bool kRep = RfTraits<S>::kReplicas;
@@ -833,7 +833,9 @@ gemv_rf_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restri
     }
     if (gridDim.y == 1) return;
     const int row0 = blockIdx.x * kRfRows;
-    const int stage_bytes = rf_smem_bytes<S, NT>(gc) - RfTraits<S>::kBookBytes;
+    // everything past the replicas stages the finish (the launch sizes the
+    // shared memory so that a row block's partial sums fit in one pass)
+    const int stage_bytes = smem_bytes - RfTraits<S>::kBookBytes;
     splitk_finish(L, sk, blockIdx.x, gridDim.y, row0, min(kRfRows, L.rows8 - row0), batch, scales, y,
                   reinterpret_cast<float4 *>(rings), stage_bytes);
 }
@@ -1385,7 +1387,12 @@ bool plan_rf(const Geom &g, int batch, size_t cap, GemvPlan &p)
     p.grid_x = nrb;
     p.counters = nrb;
     p.slots = ks > 1 ? ks : 0;
-    p.cc_smem = smem(gc);
+    // shared memory: the kernel's own, or more, so that the last CTA of a
+    // row block stages all its splits' partial sums in one pass (one L2
+    // round trip), while the CTAs an SM holds still fit
+    const size_t stage = (size_t)ks * rows * batch * sizeof(float) + (k2 ? RfTraits<Scheme<2, 8>>::kBookBytes : 0);
+    const int cap_smem = (per_sm_slots == 1 ? 220 : 113) * 1024;
+    p.cc_smem = std::max(smem(gc), (int)std::min<size_t>(stage, (size_t)cap_smem));
     return true;
 }
 
@@ -1564,7 +1571,7 @@ cudaError_t launch_plan(const Geom &g, const GemvPlan &p, const void *packed, co
             cudaError_t r = set_smem(gemv_rf_kernel<S, NT>, p.cc_smem);
             if (r != cudaSuccess) return r;
             return launch_pdl(pdl, gemv_rf_kernel<S, NT>, grid, dim3(RfTraits<S>::kThreads), p.cc_smem, s, g, pk, c, scales, x,
-                              batch, y, sk, p.len);
+                              batch, y, sk, p.len, p.cc_smem);
         };
         using One = std::integral_constant<int, 1>;
         using Two = std::integral_constant<int, 2>;

@@ -349,3 +349,25 @@ def test_gemm_split_k_deterministic_and_reusable(K, B, T):
     rows = np.arange(0, 256, 17)
     ref, bound = oracle.matmul(layer.codes, layer.codebooks, layer.scales, x, rows=rows, threads=8)
     assert_close(y1[rows], ref, bound, f"split-K {K}x{B} T{T}")
+
+
+@pytest.mark.parametrize("K", [2, 1])
+def test_gemv_tables_fall_back_to_exact_decode_beyond_binary16(K):
+    """The batch-1 table path keeps its tables in binary16 and bounds their
+    entries by 8 max|x| max|C| per CTA.  Here one codebook entry of 30 and
+    activations of 300 in the first group make that bound 72000, beyond
+    binary16, for the CTAs holding the first group: they decode each group
+    exactly and multiply in fp32 instead, while the other group split keeps
+    its tables.  Both must agree with the oracle."""
+    layer = _layer(512, 1024, K, 8, 77)
+    cb = layer.codebooks.copy()
+    cb[0, 5, 0] = 30.0
+    layer.codebooks = cb
+    layer.codes[:64, 0, 0] = 5  # rows whose first group uses the large codeword
+    x = make_activations(1024, 1, 78)
+    x[:8, 0] = 300.0
+    dl = DevLayer(layer)
+    y = run_gemv(dl, x)
+    ref, bound = oracle.matmul(layer.codes, layer.codebooks, layer.scales, x)
+    assert np.abs(ref[:64]).max() > 1000  # the large terms are in the result
+    assert_close(y, ref, bound, f"{K}x8 tables beyond binary16")
