@@ -152,30 +152,6 @@ probe_stream_kernel(const uint4 *__restrict__ chunks, long nchunks, uint4 *sink)
     sink[first] = acc;
 }
 
-__device__ __forceinline__ uint32_t cluster_ctarank()
-{
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-
-__device__ __forceinline__ void cluster_sync_all()
-{
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
-__device__ __forceinline__ uint4 ld_peer_shared(uint32_t local_addr, uint32_t rank)
-{
-    uint32_t a;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(local_addr), "r"(rank));
-    uint4 v;
-    asm volatile("ld.shared::cluster.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "r"(a)
-                 : "memory");
-    return v;
-}
-
 constexpr int kProbeSliceThreads = 512;
 
 __global__ void __launch_bounds__(kProbeSliceThreads, 1)

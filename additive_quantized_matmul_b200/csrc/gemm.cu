@@ -308,11 +308,104 @@ __device__ __forceinline__ void gemm_split_finish(const Geom &L, GemmSplit sp, i
     if (threadIdx.x == 0) sp.counters[tile] = 0u;
 }
 
+// Split-K finish of a split launched as one thread-block cluster of `ks`
+// CTAs along blockIdx.z (ks = 2, 4 or 8; the split index is the CTA's rank).
+// The cluster guarantees that the splits of a tile run at the same time, so
+// the finish is spread over all of them instead of left to the last one:
+// CTA z owns the tile's columns [z BN / ks, (z + 1) BN / ks).  Each CTA
+// writes the fp32 sums of the columns it does not own from tensor memory
+// to its slice of the split scratch (L2), the cluster barrier publishes
+// them, and each CTA adds, for its own columns, every split's sums in split
+// order (its own straight from tensor memory), scales, rounds and writes y.
+// The scratch holds whole tiles in the order tensor memory hands them out:
+// float4 j of column block cb of tile row r at ((cb 4 + j) 128 + r), so a
+// warp's 32 rows are 512 contiguous bytes for the writer and the reader
+// alike (the owner's thread of a row is the writer's thread of that row).
+// `fw` numbers the finishing warps 0 .. NW - 1 (warp & 3 is the TMEM lane
+// quarter; NW = 8 splits the columns between two warps per quarter), -1
+// for the others.  Every thread of the CTA calls it (the cluster barrier
+// needs them all), also after a timeout: then no tensor memory is read and
+// the output is incomplete, which the status word reports.
+template <int BN, int NW>
+__device__ void gemm_cluster_finish(const Geom &L, uint32_t tmem, float *__restrict__ partials, int m0, int n0,
+                                    int T, int ks, const uint16_t *__restrict__ scales, uint16_t *__restrict__ y,
+                                    int fw, bool ok)
+{
+    constexpr int kH = NW / 4;  // warps per TMEM lane quarter
+    const int lane = threadIdx.x & 31, q = (threadIdx.x >> 5) & 3;
+    const int z = (int)blockIdx.z;
+    const int cw = BN / ks;  // columns each split owns (a multiple of 16)
+    const int r = q * 32 + lane, row = m0 + r;
+    // this tile's slices: one per split, kBM x BN floats each
+    const size_t tile = (size_t)blockIdx.y * gridDim.x + blockIdx.x;
+    float4 *slices = reinterpret_cast<float4 *>(partials) + tile * ks * (kBM * BN / 4);
+    constexpr size_t kSlice = kBM * BN / 4;  // float4 per slice
+    const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16);
+    tc_fence_after();
+    if (fw >= 0 && ok) {
+        float4 *mine = slices + (size_t)z * kSlice;
+#pragma unroll 1
+        for (int c0 = 16 * (fw / 4); c0 < BN; c0 += 16 * kH) {
+            if (c0 / cw == z || n0 + c0 >= T) continue;  // warp-uniform
+            float v[16];
+            tmem_ld16(tq + (uint32_t)c0, v);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                __stcg(mine + ((c0 / 16) * 4 + j) * kBM + r, make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]));
+        }
+        fence_acq_rel_gpu();
+    }
+    cluster_sync_all();  // every split's sums are in L2
+    if (fw < 0 || !ok) return;
+    const bool live_row = row < L.out;
+    const float sc = (live_row && scales) ? __half2float(__ushort_as_half(scales[row])) : 1.f;
+#pragma unroll 1
+    for (int c0 = z * cw + 16 * (fw / 4); c0 < (z + 1) * cw; c0 += 16 * kH) {
+        const int gn = n0 + c0;
+        if (gn >= T) break;  // warp-uniform
+        float v[16];
+        tmem_ld16(tq + (uint32_t)c0, v);
+        const float4 *src = slices + ((c0 / 16) * 4) * kBM + r;
+        float acc[16];
+        // four splits' loads in flight at a time, added in split order
+        for (int z0 = 0; z0 < ks; z0 += 4) {
+            float4 t[4][4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    if (z0 + i < ks && z0 + i != z) t[i][j] = __ldcg(src + (size_t)(z0 + i) * kSlice + j * kBM);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                if (z0 + i >= ks) break;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float4 u = (z0 + i == z) ? make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3])
+                                                   : t[i][j];
+                    if (z0 + i == 0) {
+                        acc[4 * j] = u.x, acc[4 * j + 1] = u.y, acc[4 * j + 2] = u.z, acc[4 * j + 3] = u.w;
+                    } else {
+                        acc[4 * j] += u.x, acc[4 * j + 1] += u.y, acc[4 * j + 2] += u.z, acc[4 * j + 3] += u.w;
+                    }
+                }
+            }
+        }
+        if (!live_row) continue;
+        uint16_t *dst = y + (size_t)row * T + gn;
+        const uint4 o0 = make_uint4(f2h2(sc * acc[0], sc * acc[1]), f2h2(sc * acc[2], sc * acc[3]),
+                                    f2h2(sc * acc[4], sc * acc[5]), f2h2(sc * acc[6], sc * acc[7]));
+        const uint4 o1 = make_uint4(f2h2(sc * acc[8], sc * acc[9]), f2h2(sc * acc[10], sc * acc[11]),
+                                    f2h2(sc * acc[12], sc * acc[13]), f2h2(sc * acc[14], sc * acc[15]));
+        reinterpret_cast<uint4 *>(dst)[0] = o0;  // T % 8 == 0: gn + 8 <= T
+        if (gn + 16 <= T) reinterpret_cast<uint4 *>(dst)[1] = o1;
+    }
+}
+
 template <class S, int BN>
 __global__ void __launch_bounds__(kWsThreadsOf<S>, 1)
 gemm_ws_kernel(const __grid_constant__ CUtensorMap xmap, Geom L, const uint8_t *__restrict__ packed,
                const uint4 *__restrict__ cb, const uint16_t *__restrict__ scales, int T,
-               uint16_t *__restrict__ y, void *ws, GemmSplit sp, int stages_per_split)
+               uint16_t *__restrict__ y, void *ws, GemmSplit sp, int stages_per_split, int cluster_ks)
 {
     constexpr int kWsStages = kWsStagesOf<S, BN>;    // X ring
     constexpr int kWsAStages = kWsAStagesOf<S, BN>;  // W ring
@@ -528,7 +621,7 @@ gemm_ws_kernel(const __grid_constant__ CUtensorMap xmap, Geom L, const uint8_t *
         // this point by a role that gave up, or just above by a lane whose
         // wait failed (then its warp-mates see it through the ballot)
         const bool warp_ok = __all_sync(0xffffffffu, got);
-        if (warp_ok && dg == 0) {
+        if (warp_ok && dg == 0 && cluster_ks == 0) {
             const int q = warp & 3;  // TMEM lane quarter of this warp
             const int row = m0 + q * 32 + lane;
             const float sc = (row < L.out && scales) ? __half2float(__ushort_as_half(scales[row])) : 1.f;
@@ -573,12 +666,18 @@ gemm_ws_kernel(const __grid_constant__ CUtensorMap xmap, Geom L, const uint8_t *
             for (int s = max(0, nk - kWsStages); s < nk; ++s)
                 mbar_wait_ns(&full_b[s % kWsStages], (s / kWsStages) & 1, kWaitNs);
     }
+    if (cluster_ks > 1) {
+        // the decoder warps finish: warp & 3 is their TMEM lane quarter
+        constexpr int NW = 4 * kWsGroupsOf<S>;
+        gemm_cluster_finish<BN, NW>(L, tmem, sp.partials, m0, n0, T, cluster_ks, scales, y,
+                                    warp >= 2 ? warp - 2 : -1, *abort_v == 0);
+    }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, BN);
     // arrive even after a timeout so the counters stay consistent (the
     // status word already tells the caller the output is incomplete)
-    if (sp.partials) gemm_split_finish(L, sp, m0, n0, BN, T, scales, y);
+    if (sp.partials && cluster_ks == 0) gemm_split_finish(L, sp, m0, n0, BN, T, scales, y);
 }
 
 // ---- self-test of the bounded wait -----------------------------------------
@@ -608,6 +707,7 @@ struct GemmPlan {
     int mtiles, ntiles;
     int ks;           // splits of the input features (blockIdx.z)
     int per_split;    // 64-feature stages per split
+    bool cluster;     // the splits form one cluster and finish on chip
     size_t ws_bytes;  // status word + tile counters + fp32 partials
 };
 
@@ -623,7 +723,10 @@ static GemmPlan plan_gemm(const Geom &g, int T)
     // the input features, whose partial sums cost a pass through L2),
     // 256-token tiles with fewer splits are faster (measured on Llama-2-7B
     // shapes at 512 tokens)
-    p.bn = (T > 256 && (long)p.mtiles * ((T + 511) / 512) * 2 >= kNumSMs) ? 512 : 256;
+    // 512-token tiles halve the decode work per MMA; with few row tiles
+    // (a 4096-row layer at 512 tokens) they need a split of the input
+    // features, which the cluster finish makes cheap
+    p.bn = T >= 384 || (T > 256 && (long)p.mtiles * ((T + 511) / 512) * 2 >= kNumSMs) ? 512 : 256;
     p.ntiles = (T + p.bn - 1) / p.bn;
     const int nst = (g.in + kBK - 1) / kBK;
     const long tiles = (long)p.mtiles * p.ntiles;
@@ -631,11 +734,26 @@ static GemmPlan plan_gemm(const Geom &g, int T)
     // per SM works, keeping at least 8 stages per split
     int ks = tiles < kNumSMs ? (int)(kNumSMs / tiles) : 1;
     ks = std::max(1, std::min(ks, nst / 8));
+    // a split of 2, 4 or 8 runs as one thread-block cluster along z whose
+    // CTAs share the finish (no arrival counters)
+    bool cluster = false;
+    if (ks >= 2) {
+        int kc = 2;
+        while (kc * 2 <= std::min(ks, 8)) kc *= 2;
+        const int per = (nst + kc - 1) / kc;
+        if ((nst + per - 1) / per == kc) {  // no empty split
+            ks = kc;
+            cluster = true;
+        }
+    }
     p.per_split = (nst + ks - 1) / ks;
     p.ks = (nst + p.per_split - 1) / p.per_split;
-    // split only while the tiles' arrival counters fit the fixed area
-    if (tiles > kWsMaxCounters) p.ks = 1, p.per_split = nst;
-    if (p.ks > 1) p.ws_bytes = kWsData + (size_t)p.ks * g.out * T * sizeof(float);
+    p.cluster = cluster;
+    // without a cluster, split only while the tiles' arrival counters fit
+    // the fixed area
+    if (!cluster && tiles > kWsMaxCounters) p.ks = 1, p.per_split = nst;
+    if (p.ks > 1)
+        p.ws_bytes = kWsData + (cluster ? (size_t)p.ks * tiles * kBM * p.bn : (size_t)p.ks * g.out * T) * sizeof(float);
     return p;
 }
 
@@ -698,7 +816,21 @@ cudaError_t launch_gemm(const Geom &g, const void *packed, const uint16_t *cb,
             cudaError_t e = cudaFuncSetAttribute(gemm_ws_kernel<S, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                  smem);
             if (e != cudaSuccess) return e;
-            gemm_ws_kernel<S, BN><<<grid, kWsThreadsOf<S>, smem, s>>>(map, g, pk, c, scales, T, y, ws, sp, p.per_split);
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = grid;
+            cfg.blockDim = dim3(kWsThreadsOf<S>);
+            cfg.dynamicSmemBytes = smem;
+            cfg.stream = s;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = 1;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = p.ks;
+            cfg.attrs = attr;
+            cfg.numAttrs = p.cluster ? 1 : 0;
+            e = cudaLaunchKernelEx(&cfg, gemm_ws_kernel<S, BN>, map, g, pk, c, scales, T, y, ws, sp, p.per_split,
+                                   p.cluster ? p.ks : 0);
+            if (e != cudaSuccess) return e;
             return cudaGetLastError();
         };
         return with_scheme(g, [&](auto sch) {

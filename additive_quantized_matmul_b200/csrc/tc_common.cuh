@@ -174,6 +174,36 @@ __device__ __forceinline__ void prefetch_table_share(const void *table, uint32_t
     if (off < bytes) prefetch_l2_bulk(reinterpret_cast<const uint8_t *>(table) + off, min(share, bytes - off));
 }
 
+// ---- thread-block clusters ----------------------------------------------------
+
+__device__ __forceinline__ uint32_t cluster_ctarank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// Every thread of every CTA of the cluster arrives (release) and waits
+// (acquire): shared-memory writes before it are visible to the cluster's
+// reads after it.
+__device__ __forceinline__ void cluster_sync_all()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// 16 bytes at `local_addr` in the shared memory of cluster CTA `rank`.
+__device__ __forceinline__ uint4 ld_peer_shared(uint32_t local_addr, uint32_t rank)
+{
+    uint32_t a;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(local_addr), "r"(rank));
+    uint4 v;
+    asm volatile("ld.shared::cluster.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(a)
+                 : "memory");
+    return v;
+}
+
 // 2-D tiled TMA load (no multicast) of box {c0.., c1..} into shared memory,
 // completing `bytes` on the mbarrier.  c0 is the innermost coordinate.
 __device__ __forceinline__ void tma_load_2d(uint32_t dst_smem, const void *tmap, int c0, int c1, uint64_t *bar)

@@ -306,7 +306,7 @@ def recorded_traffic(layer: str, batch: int):
     the committed ncu record, or None when there is none or the kernel
     sources changed since the counters were taken."""
     import hashlib
-    p = os.path.join(ROOT, "profiles", "traffic_gemv_tc.json")
+    p = os.path.join(ROOT, "profiles", "traffic_gemv_llama2-7b-1x16.json")
     if not os.path.exists(p):
         return None
     rec = json.load(open(p))

@@ -198,7 +198,9 @@ def test_workspace_layout_is_shared_by_every_call():
     huge = aq.LayerDesc.make(1 << 20, 64, 1, 16)
     assert aq.aq_gemv_workspace_bytes(huge, 4) == 16
     assert aq.aq_gemm_workspace_bytes(huge, 64) == 16
-    assert aq.aq_gemm_workspace_bytes(aq.LayerDesc.make(256, 4096, 2, 8), 512) > prefix
+    # a prefill split over the input features (here 8 splits, one cluster)
+    # keeps its fp32 partial sums after the counters area
+    assert aq.aq_gemm_workspace_bytes(aq.LayerDesc.make(256, 4096, 2, 8), 512) == prefix + 8 * 256 * 512 * 4
     assert aq.aq_encode_workspace_bytes(aq.LayerDesc.make(64, 256, 2, 8)) == prefix + 32 * 2 * 256 * 4
     # the coarsest split of the no-allocation entry point always fits its array
     assert aq.aq_gemv_workspace_bytes(aq.LayerDesc.make(1 << 28, 8, 1, 16), 1) <= aq.GEMV_NOALLOC_SCRATCH_BYTES

@@ -22,7 +22,7 @@ def test_algorithmic_bytes_of_the_default_layer():
 
 def test_traffic_record_only_while_the_sources_match(tmp_path, monkeypatch):
     import hashlib
-    rec = json.load(open(os.path.join(ROOT, "profiles", "traffic_gemv_tc.json")))
+    rec = json.load(open(os.path.join(ROOT, "profiles", "traffic_gemv_llama2-7b-1x16.json")))
     assert set(rec["per_launch_bytes"]) == {"1", "4", "16"} and rec["layer"] == "4096x4096"
     # a copy of the repository whose record was taken on its current sources
     fake = tmp_path / "repo"
@@ -35,7 +35,7 @@ def test_traffic_record_only_while_the_sources_match(tmp_path, monkeypatch):
         dst.write_bytes(data)
         h.update(data)
     rec = dict(rec, sources_sha256=h.hexdigest())
-    (fake / "profiles" / "traffic_gemv_tc.json").write_text(json.dumps(rec))
+    (fake / "profiles" / "traffic_gemv_llama2-7b-1x16.json").write_text(json.dumps(rec))
     monkeypatch.setattr(bench, "ROOT", str(fake))
     for b in (1, 4, 16):
         assert bench.recorded_traffic("4096x4096", b) == rec["per_launch_bytes"][str(b)]
