@@ -61,6 +61,15 @@ constexpr size_t kWsHeader = 16;
 constexpr int kWsMaxCounters = 1024;
 constexpr size_t kWsData = kWsHeader + sizeof(unsigned) * kWsMaxCounters;
 
+// Atomic add with release and acquire semantics at GPU scope; returns the
+// old value.
+__device__ __forceinline__ unsigned atom_add_acq_rel_gpu(unsigned *p, unsigned v)
+{
+    unsigned old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+
 __device__ __forceinline__ void record_status(void *ws, uint32_t status)
 {
     if (ws) atomicMax(reinterpret_cast<unsigned int *>(ws), status);

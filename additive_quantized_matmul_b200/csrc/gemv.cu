@@ -40,16 +40,73 @@ struct SplitK {
     unsigned *counters;   // one per row range
 };
 
+// Scales the float4 of outputs starting at element idx of a row block
+// ([rows][batch], rows from row0), rounds once to binary16 and stores it.
+// s_sc: the block's scales in shared memory (or null: read them here).
+// Batch a multiple of 4: one row, one 8-byte store; batch 1: four rows,
+// one 8-byte scale read and one 8-byte store.
+__device__ __forceinline__ void finish_store4(const Geom &L, int row0, int idx, int batch, float4 acc,
+                                              const uint16_t *__restrict__ scales, const float *s_sc,
+                                              uint16_t *__restrict__ y)
+{
+    if ((batch & 3) == 0) {
+        const int r = idx / batch, row = row0 + r;
+        if (row >= L.out) return;
+        const float sc = s_sc ? s_sc[r] : (scales ? __half2float(__ushort_as_half(scales[row])) : 1.f);
+        *reinterpret_cast<uint2 *>(y + (size_t)row * batch + idx % batch) =
+            make_uint2(f2h2(sc * acc.x, sc * acc.y), f2h2(sc * acc.z, sc * acc.w));
+        return;
+    }
+    const float v[4] = {acc.x, acc.y, acc.z, acc.w};
+    if (batch == 1 && row0 + idx + 3 < L.out) {
+        float sc[4] = {1.f, 1.f, 1.f, 1.f};
+        if (s_sc) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) sc[c] = s_sc[idx + c];
+        } else if (scales) {
+            const uint2 w = *reinterpret_cast<const uint2 *>(scales + row0 + idx);  // row0 + idx: a multiple of 4
+            const float2 lo = h2f2(w.x), hi = h2f2(w.y);
+            sc[0] = lo.x, sc[1] = lo.y, sc[2] = hi.x, sc[3] = hi.y;
+        }
+        *reinterpret_cast<uint2 *>(y + row0 + idx) =
+            make_uint2(f2h2(sc[0] * v[0], sc[1] * v[1]), f2h2(sc[2] * v[2], sc[3] * v[3]));
+        return;
+    }
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        const int r = (idx + c) / batch, row = row0 + r;
+        if (row < L.out) {
+            const float sc = s_sc ? s_sc[r] : (scales ? __half2float(__ushort_as_half(scales[row])) : 1.f);
+            y[(size_t)row * batch + (idx + c) % batch] = __half_as_ushort(__float2half_rn(sc * v[c]));
+        }
+    }
+}
+
+// Rows whose scales the split-K finish keeps in shared memory.
+constexpr int kFinishScaleRows = 256;
+
+// The split-K finish of rows [row0, row0 + nrows) reads their scales at the
+// end of the launch; one CTA of the row range brings them into L2 at its
+// start (a prefetch returns nothing, so it may precede the dependency wait).
+__device__ __forceinline__ void prefetch_range_scales(const Geom &L, const uint16_t *scales, int row0, int nrows)
+{
+    if (threadIdx.x != 0 || blockIdx.y != 0 || gridDim.y == 1 || !scales) return;
+    const int n = (min(row0 + nrows, L.out) - row0) & ~7;  // whole 16-byte pieces inside the array
+    if (n > 0) prefetch_l2_bulk(scales + row0, (uint32_t)n * 2u);
+}
+
 // Called by every thread of a CTA after it stored its partial sums for rows
 // [row0, row0 + nrows), columns [0, batch), into its slot of that row range
 // (nrows is a multiple of 8 and row0 + nrows <= rows8, so the block is a
 // whole number of float4 inside every slot).  The row range has `ks` slots
 // and arrival counter `counter`; the last CTA to arrive reduces the slots in
 // slot order, writes y and resets the counter for the next call.  With
-// `stage` (shared memory the CTA no longer needs, `stage_bytes` of it) the
-// partial sums are staged there: every (slot, float4) of a pass is requested
-// at once with cp.async, so a pass costs about one L2 round trip whatever
-// ks.  Without it (or with fewer than 16 ks bytes) they are summed straight
+// `stage` (shared memory the CTA no longer needs, `stage_bytes` of it, 16-byte
+// aligned) the partial sums are staged there: a pass takes the same float4
+// range of every slot, one contiguous run per slot, by one bulk copy each
+// (TMA engine), and the range's scales are read into shared memory
+// meanwhile.
+// Without it (or with fewer than 16 ks bytes) they are summed straight
 // from L2, eight slots in flight per float4.
 template <int kInFlight = 8>
 __device__ __forceinline__ void splitk_finish(const Geom &L, SplitK sk, int counter, int ks, int row0,
@@ -57,15 +114,15 @@ __device__ __forceinline__ void splitk_finish(const Geom &L, SplitK sk, int coun
                                               uint16_t *__restrict__ y, float4 *stage, int stage_bytes)
 {
     __shared__ unsigned s_last;
+    __shared__ float s_scale[kFinishScaleRows];
+    __shared__ uint64_t s_staged;  // the bulk copies of a pass have landed
     __syncthreads();
     if (threadIdx.x == 0) {
         // the barrier orders the CTA's partial stores before this thread's
-        // release fence, which publishes them with the counter increment;
-        // the last CTA's acquire fence orders its reads after all of them
-        fence_acq_rel_gpu();
-        const unsigned prev = atomicAdd(&sk.counters[counter], 1u);
+        // increment, whose release publishes them; its acquire orders the
+        // last CTA's reads after every slot's
+        const unsigned prev = atom_add_acq_rel_gpu(&sk.counters[counter], 1u);
         s_last = (prev == (unsigned)ks - 1u) ? 1u : 0u;
-        if (s_last) fence_acq_rel_gpu();
     }
     __syncthreads();
     if (!s_last) return;
@@ -88,44 +145,37 @@ __device__ __forceinline__ void splitk_finish(const Geom &L, SplitK sk, int coun
                         acc.x += t[j].x; acc.y += t[j].y; acc.z += t[j].z; acc.w += t[j].w;
                     }
             }
-            const float v[4] = {acc.x, acc.y, acc.z, acc.w};
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const int idx = e * 4 + c;
-                const int row = row0 + idx / batch;
-                if (row < L.out) {
-                    const float sc = scales ? __half2float(__ushort_as_half(scales[row])) : 1.f;
-                    y[(size_t)row * batch + idx % batch] = __half_as_ushort(__float2half_rn(sc * v[c]));
-                }
-            }
+            finish_store4(L, row0, e * 4, batch, acc, scales, nullptr, y);
         }
     }
-    for (int c0 = 0; chunk > 0 && c0 < nvec; c0 += chunk) {
+    const bool pre = scales && nrows <= kFinishScaleRows;  // scales staged too
+    for (int c0 = 0, pass = 0; chunk > 0 && c0 < nvec; c0 += chunk, ++pass) {
         const int n = min(chunk, nvec - c0);
-        for (int q = threadIdx.x; q < ks * n; q += blockDim.x) {
-            const int sl = q / n, e = q - sl * n;
-            cp_async16(smem_u32(stage + q), base + (size_t)sl * vstride + c0 + e, 16u);
+        if (threadIdx.x == 0) {
+            if (pass == 0) {
+                mbar_init(&s_staged, 1);
+                fence_mbar_init();
+            }
+            fence_proxy_async_global();  // the slots' stores, acquired above, before the bulk reads
+            fence_proxy_async_smem();    // the CTA's earlier use of the staging area before the bulk writes
+            mbar_arrive_expect_tx(&s_staged, (uint32_t)(ks * n * 16));
+            for (int sl = 0; sl < ks; ++sl)
+                bulk_load(smem_u32(stage + (size_t)sl * n), base + (size_t)sl * vstride + c0, (uint32_t)(n * 16),
+                          &s_staged);
         }
-        cp_async_commit();
-        cp_async_wait<0>();
-        __syncthreads();
+        if (pre && c0 == 0)  // while the copies are in flight
+            for (int i = threadIdx.x; i < nrows; i += blockDim.x)
+                s_scale[i] = row0 + i < L.out ? __half2float(__ushort_as_half(scales[row0 + i])) : 0.f;
+        __syncthreads();  // the barrier's initialisation and the scales
+        if (!mbar_wait_ns(&s_staged, pass & 1, kWaitNs) && threadIdx.x == 0)
+            record_status(reinterpret_cast<char *>(sk.counters) - kWsHeader, AQ_ERR_TIMEOUT);
         for (int e = threadIdx.x; e < n; e += blockDim.x) {
             float4 acc = stage[e];
             for (int sl = 1; sl < ks; ++sl) {
                 const float4 t = stage[sl * n + e];
                 acc.x += t.x; acc.y += t.y; acc.z += t.z; acc.w += t.w;
             }
-            const float v[4] = {acc.x, acc.y, acc.z, acc.w};
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const int idx = (c0 + e) * 4 + c;
-                const int row = row0 + idx / batch;
-                const int b = idx % batch;
-                if (row < L.out) {
-                    const float sc = scales ? __half2float(__ushort_as_half(scales[row])) : 1.f;
-                    y[(size_t)row * batch + b] = __half_as_ushort(__float2half_rn(sc * v[c]));
-                }
-            }
+            finish_store4(L, row0, (c0 + e) * 4, batch, acc, scales, pre ? s_scale : nullptr, y);
         }
         __syncthreads();  // the next pass reuses the staging area
     }
@@ -266,6 +316,7 @@ gemv_lut_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restr
             prefetch_l2_bulk(packed + ((size_t)rt * L.gp + G0) * S::kChunkBytes, (uint32_t)(ngl * S::kChunkBytes));
     }
     if (threadIdx.x < 2) s_max[threadIdx.x] = 0;
+    prefetch_range_scales(L, scales, rt0 * 8, (rt1 - rt0) * 8);
     grid_dependency_wait();  // x, y and the workspace follow the previous launch
     grid_launch_dependents();
     uint4 xv = make_uint4(0u, 0u, 0u, 0u);
@@ -496,6 +547,7 @@ gemv_1x16_cc_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__r
 #pragma unroll
     for (int r = 0; r < 8; ++r) w[r] = ldg_nc_v4(cb + cc_code(code, r));
     uint4 next = nown > 1 ? ldg_stream_v4(chunk0 + 128) : zero;
+    prefetch_range_scales(L, scales, blockIdx.x * kCcRowTiles * 8, kCcRowTiles * 8);
     grid_dependency_wait();  // x, y and the workspace follow the previous launch
     grid_launch_dependents();
     for (int i = tid; i < ng * 2 * NB; i += kCcThreads) {  // 4 values at a time ([in][batch] is that order)
@@ -707,6 +759,7 @@ gemv_rf_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restri
             gw[i][1] = ldg_nc_v4(cb + wb);
         }
     }
+    prefetch_range_scales(L, scales, blockIdx.x * kRfRows, kRfRows);
     grid_dependency_wait();  // x, y and the workspace follow the previous launch
     grid_launch_dependents();
     {

@@ -204,6 +204,20 @@ __device__ __forceinline__ uint4 ld_peer_shared(uint32_t local_addr, uint32_t ra
     return v;
 }
 
+// Orders this thread's generic-proxy view of global memory with its later
+// async-proxy (bulk copy) accesses.
+__device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
+
+// Bulk copy (TMA engine, no multicast) of `bytes` from global memory into
+// this CTA's shared memory, completing the bytes on the mbarrier.  Both
+// addresses 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_load(uint32_t dst_smem, const void *src, uint32_t bytes, uint64_t *bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(dst_smem), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+
 // 2-D tiled TMA load (no multicast) of box {c0.., c1..} into shared memory,
 // completing `bytes` on the mbarrier.  c0 is the innermost coordinate.
 __device__ __forceinline__ void tma_load_2d(uint32_t dst_smem, const void *tmap, int c0, int c1, uint64_t *bar)
