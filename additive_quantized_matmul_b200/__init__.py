@@ -233,8 +233,9 @@ def aq_encode_workspace_bytes(desc: LayerDesc) -> int:
 
 def aq_encode(desc: LayerDesc, w, h, codebooks, codes_in, beam: int, codes_out, workspace,
               workspace_bytes: int | None = None, stream=None) -> None:
-    """Beam search of the codes (8-bit codebooks) minimising e^T H e per row;
-    w [out][in] binary16, h [in][in] fp32, codes [out][in/8][K] uint8."""
+    """Beam search of the codes minimising e^T H e per row; w [out][in]
+    binary16, h [in][in] fp32, codes [out][in/8][K] uint8 (8-bit codebooks)
+    or uint16 (16-bit)."""
     if workspace_bytes is None:
         workspace_bytes = workspace.numel() * workspace.element_size()
     _check("aq_encode", lib.aq_encode(ctypes.byref(desc), _ptr(w), _ptr(h), _ptr(codebooks), _ptr(codes_in), beam,

@@ -207,7 +207,7 @@ aq_status aq_gemm(const aq_layer_desc *desc, const void *packed, const uint16_t 
 
 size_t aq_encode_workspace_bytes(const aq_layer_desc *desc)
 {
-    if (check_desc(desc) != AQ_OK || desc->nbits != 8 || desc->in_features > 16384) return 0;
+    if (check_desc(desc) != AQ_OK || desc->in_features > 16384) return 0;
     return aqh::encode_workspace_bytes(aqk::make_geom(*desc));
 }
 
@@ -217,7 +217,6 @@ aq_status aq_encode(const aq_layer_desc *desc, const uint16_t *w, const float *h
 {
     aq_status st = check_desc(desc);
     if (st != AQ_OK) return st;
-    if (desc->nbits != 8) return AQ_ERR_UNSUPPORTED;
     if (desc->in_features > 16384 || beam < 1 || beam > 16) return AQ_ERR_INVALID_ARG;
     if (!w || !h || !codebooks || !codes_in || !codes_out || codes_in == codes_out) return AQ_ERR_INVALID_ARG;
     if (!aligned16(w) || !aligned16(h) || !aligned16(codebooks)) return AQ_ERR_MISALIGNED;

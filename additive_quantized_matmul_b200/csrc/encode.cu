@@ -248,12 +248,264 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(Geom L, const uint1
 }
 
 
+// ---- 16-bit codebooks (1x16, 2x16) -----------------------------------------
+// The same search over 65536 codes per slot.  One CTA per tile of kE16Rows
+// rows (the codebook then streams through shared memory once per tile and
+// slot instead of once per row); each row's codes are split over kE16Slices
+// threads, each keeping its `nsel` best keys, merged per row at the slot's
+// end.  The residual e lives in the workspace ([out][in] fp32), the table
+// q[(g K + k) 65536 + c] = C_k[c]^T H_gg C_k[c] too.  Keys are (objective
+// change, parent beam, code), as above, with 16-bit codes.  With K = 1 the
+// one slot's best proposal is the group's (the beam keeps nothing past it);
+// with K = 2 the first slot keeps `beam` proposals and the second its best.
+constexpr int kE16Rows = 16;                     // rows per CTA
+constexpr int kE16Slices = kEncThreads / kE16Rows;  // threads per row
+constexpr int kE16Chunk = 512;                   // codes per shared-memory chunk
+constexpr int kE16Cols = 256;                    // residual columns per chunk of (H e)_g
+constexpr int encode16_smem_bytes()
+{
+    return kE16Rows * kE16Slices * kEncMaxBeam * 8 + kE16Chunk * 9 * 4 + kE16Rows * (kE16Cols + 1) * 4 +
+           8 * kE16Cols * 4 + 2 * kE16Rows * kEncMaxBeam * 8 * 4 + kE16Rows * kEncMaxBeam * 8 * 4;
+}
+
+template <int K>
+__global__ void __launch_bounds__(256) encode16_q_kernel(int in, const float *__restrict__ h,
+                                                         const uint4 *__restrict__ cb, float *__restrict__ q)
+{
+    __shared__ float hgg[64];
+    const int g = blockIdx.y;
+    if (threadIdx.x < 64) hgg[threadIdx.x] = h[(size_t)(8 * g + threadIdx.x / 8) * in + 8 * g + threadIdx.x % 8];
+    __syncthreads();
+    const int c = blockIdx.x * 256 + threadIdx.x;  // code 0 .. 65535
+#pragma unroll 1
+    for (int k = 0; k < K; ++k) {
+        float x[8];
+        load_f8(cb[(size_t)k * 65536 + c], x);
+        float acc = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            float t = 0.f;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) t = fmaf(hgg[i * 8 + j], x[j], t);
+            acc = fmaf(x[i], t, acc);
+        }
+        q[((size_t)g * K + k) * 65536 + c] = acc;
+    }
+}
+
+__device__ __forceinline__ uint64_t enc16_key(float s, int beam, int code)
+{
+    s = s + 0.f;  // -0 -> +0
+    uint32_t u = __float_as_uint(s);
+    u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    return ((uint64_t)u << 32) | ((uint32_t)beam << 16) | (uint32_t)code;
+}
+
+template <int K>
+__global__ void __launch_bounds__(kEncThreads) encode16_kernel(Geom L, const uint16_t *__restrict__ w,
+                                                               const float *__restrict__ h,
+                                                               const uint4 *__restrict__ cb,
+                                                               const float *__restrict__ qtab,
+                                                               const uint16_t *__restrict__ codes_in,
+                                                               uint16_t *__restrict__ codes_out,
+                                                               float *__restrict__ eg, int beam)
+{
+    constexpr int R = kE16Rows, S = kE16Slices;
+    // dynamic shared memory (encode16_smem_bytes), carved:
+    extern __shared__ __align__(16) uint8_t e16_smem[];
+    auto lists = reinterpret_cast<uint64_t(*)[S][kEncMaxBeam]>(e16_smem);         // [R]: per-slice best keys
+    auto sx = reinterpret_cast<float(*)[8]>(lists + R);                           // [kE16Chunk]: codebook chunk
+    float *sq = reinterpret_cast<float *>(sx + kE16Chunk);                        // [kE16Chunk]: its q
+    auto ec = reinterpret_cast<float(*)[kE16Cols + 1]>(sq + kE16Chunk);           // [R]: residual chunk
+    auto hc = reinterpret_cast<float(*)[kE16Cols]>(ec + R);                       // [8]: H rows 8g.. chunk
+    auto bD = reinterpret_cast<float(*)[R][kEncMaxBeam][8]>(hc + 8);              // [2]: beams' changes
+    auto bw = reinterpret_cast<float(*)[kEncMaxBeam][8]>(bD + 2);                 // [R]: proposals' w
+    __shared__ float hgg[64], v[R][8];
+    __shared__ uint16_t bcode[2][R][kEncMaxBeam][K];
+    __shared__ float bconst[R][kEncMaxBeam];
+    __shared__ uint64_t sel[R][kEncMaxBeam];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int my_r = tid / S, my_s = tid % S;
+    const int in = L.in, G = L.G, o0 = blockIdx.x * R;
+    const int nrows = min(R, L.out - o0);
+
+    // e = w - the starting codes' reconstruction
+    for (int i = tid; i < nrows * in; i += kEncThreads) {
+        const int r = i / in, c = i - r * in, g = c >> 3, j = c & 7;
+        const size_t o = (size_t)(o0 + r);
+        float rec = 0.f;
+#pragma unroll
+        for (int k = 0; k < K; ++k) {
+            float x[8];
+            load_f8(cb[(size_t)k * 65536 + codes_in[(o * G + g) * K + k]], x);
+            rec += x[j];
+        }
+        eg[o * in + c] = __half2float(__ushort_as_half(w[o * in + c])) - rec;
+    }
+    int cur = 0;
+#pragma unroll 1
+    for (int g = 0; g < G; ++g) {
+        __syncthreads();  // e holds every committed group (global writes of this CTA)
+        // v[r][j] = sum_t H[8g + j][t] e[r][t]: warp j, lane columns, 256-column chunks
+        float acc[R];
+#pragma unroll
+        for (int r = 0; r < R; ++r) acc[r] = 0.f;
+#pragma unroll 1
+        for (int c0 = 0; c0 < in; c0 += kE16Cols) {
+            const int nc = min(kE16Cols, in - c0);
+            for (int i = tid; i < R * kE16Cols; i += kEncThreads) {
+                const int r = i / kE16Cols, c = i % kE16Cols;
+                ec[r][c] = (r < nrows && c < nc) ? eg[(size_t)(o0 + r) * in + c0 + c] : 0.f;
+            }
+            for (int i = tid; i < 8 * kE16Cols; i += kEncThreads) {
+                const int j = i / kE16Cols, c = i % kE16Cols;
+                hc[j][c] = c < nc ? h[(size_t)(8 * g + j) * in + c0 + c] : 0.f;
+            }
+            __syncthreads();
+#pragma unroll
+            for (int m = 0; m < kE16Cols / 32; ++m) {
+                const float hv = hc[warp][lane + 32 * m];
+#pragma unroll
+                for (int r = 0; r < R; ++r) acc[r] = fmaf(hv, ec[r][lane + 32 * m], acc[r]);
+            }
+            __syncthreads();
+        }
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            float a = acc[r];
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) a += __shfl_xor_sync(0xffffffffu, a, off);
+            if (lane == 0) v[r][warp] = a;
+        }
+        if (tid < 64) hgg[tid] = h[(size_t)(8 * g + tid / 8) * in + 8 * g + tid % 8];
+        if (tid < R * 8) bD[cur][tid / 8][0][tid % 8] = 0.f;
+        if (tid < R * K && tid / K < nrows)
+            bcode[cur][tid / K][0][tid % K] = codes_in[((size_t)(o0 + tid / K) * G + g) * K + tid % K];
+        int nb = 1;
+        __syncthreads();
+#pragma unroll 1
+        for (int k = 0; k < K; ++k) {
+            const int nsel = (k == K - 1) ? 1 : beam;
+            // per row and live beam: a = D_b - C_k[c0], const and w of the proposals
+            for (int i = tid; i < R * nb; i += kEncThreads) {
+                const int r = i / nb, b = i % nb;
+                if (r >= nrows) continue;
+                const uint32_t c0 = codes_in[((size_t)(o0 + r) * G + g) * K + k];
+                float a[8], c0v[8];
+                load_f8(cb[(size_t)k * 65536 + c0], c0v);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) a[j] = bD[cur][r][b][j] - c0v[j];
+                float cst = 0.f;
+#pragma unroll
+                for (int ii = 0; ii < 8; ++ii) {
+                    float t = 0.f;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) t = fmaf(hgg[ii * 8 + j], a[j], t);
+                    cst = fmaf(a[ii], t - 2.f * v[r][ii], cst);
+                    bw[r][b][ii] = t - v[r][ii];
+                }
+                bconst[r][b] = cst;
+            }
+            uint64_t top[kEncMaxBeam];
+#pragma unroll
+            for (int i = 0; i < kEncMaxBeam; ++i) top[i] = ~0ull;
+            uint64_t worst = ~0ull;  // top[nsel - 1]
+            const float *qk = qtab + ((size_t)g * K + k) * 65536;
+#pragma unroll 1
+            for (int base = 0; base < 65536; base += kE16Chunk) {
+                __syncthreads();  // the previous chunk is consumed (and bw, bconst written)
+                for (int i = tid; i < kE16Chunk; i += kEncThreads) {
+                    float x[8];
+                    load_f8(cb[(size_t)k * 65536 + base + i], x);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) sx[i][j] = x[j];
+                    sq[i] = qk[base + i];
+                }
+                __syncthreads();
+                if (my_r >= nrows) continue;
+#pragma unroll 1
+                for (int c = my_s; c < kE16Chunk; c += S) {
+                    const float qc = sq[c];
+#pragma unroll 1
+                    for (int b = 0; b < nb; ++b) {
+                        float d = 0.f;
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) d = fmaf(sx[c][j], bw[my_r][b][j], d);
+                        const uint64_t key = enc16_key(bconst[my_r][b] + qc + 2.f * d, b, base + c);
+                        if (key < worst) {
+                            // insert, dropping the largest; keep the list sorted
+                            uint64_t x = key;
+#pragma unroll
+                            for (int i = 0; i < kEncMaxBeam; ++i)
+                                if (i < nsel) {
+                                    const uint64_t lo = top[i] < x ? top[i] : x, hi = top[i] < x ? x : top[i];
+                                    top[i] = lo;
+                                    x = hi;
+                                }
+#pragma unroll
+                            for (int i = 0; i < kEncMaxBeam; ++i)
+                                if (i == nsel - 1) worst = top[i];
+                        }
+                    }
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < kEncMaxBeam; ++i) lists[my_r][my_s][i] = top[i];
+            __syncthreads();
+            // per row, the nsel smallest of its S sorted lists: warp w takes
+            // rows w and w + 8, lane s < S holds list s's head
+            for (int r = warp; r < R; r += kEncThreads / 32) {
+                int head = 0;
+                for (int t = 0; t < nsel; ++t) {
+                    const uint64_t mine = (lane < S && head < kEncMaxBeam) ? lists[r][lane][head] : ~0ull;
+                    const uint64_t m = warp_min_u64(mine);
+                    if (lane < S && mine == m && m != ~0ull) ++head;
+                    if (lane == 0) sel[r][t] = m;
+                }
+            }
+            __syncthreads();
+            const int nxt = cur ^ 1;
+            for (int i = tid; i < R * nsel; i += kEncThreads) {
+                const int r = i / nsel, t = i % nsel;
+                if (r >= nrows) continue;
+                const uint64_t key = sel[r][t];
+                const int pb = (int)((key >> 16) & 0xff), c = (int)(key & 0xffff);
+                const uint32_t c0 = codes_in[((size_t)(o0 + r) * G + g) * K + k];
+                float cv[8], c0v[8];
+                load_f8(cb[(size_t)k * 65536 + c], cv);
+                load_f8(cb[(size_t)k * 65536 + c0], c0v);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) bD[nxt][r][t][j] = bD[cur][r][pb][j] + cv[j] - c0v[j];
+#pragma unroll
+                for (int qq = 0; qq < K; ++qq) bcode[nxt][r][t][qq] = bcode[cur][r][pb][qq];
+                bcode[nxt][r][t][k] = (uint16_t)c;
+            }
+            nb = nsel;
+            cur = nxt;
+            __syncthreads();
+        }
+        // commit each row's best beam
+        for (int i = tid; i < nrows * 8; i += kEncThreads) {
+            const int r = i / 8, j = i % 8;
+            eg[(size_t)(o0 + r) * in + 8 * g + j] -= bD[cur][r][0][j];
+        }
+        for (int i = tid; i < nrows * K; i += kEncThreads)
+            codes_out[((size_t)(o0 + i / K) * G + g) * K + i % K] = bcode[cur][i / K][0][i % K];
+    }
+}
+
+
 }  // namespace aqk
 
 namespace aqh {
 using namespace aqk;
 
-size_t encode_workspace_bytes(const Geom &g) { return kWsData + align16((size_t)g.G * g.K * 256 * sizeof(float)); }
+size_t encode_workspace_bytes(const Geom &g)
+{
+    if (g.B == 16)  // q table [G][K][65536] and the residual [out][in], fp32
+        return kWsData + align16((size_t)g.G * g.K * 65536 * sizeof(float)) + (size_t)g.out * g.in * sizeof(float);
+    return kWsData + align16((size_t)g.G * g.K * 256 * sizeof(float));
+}
 
 cudaError_t launch_encode(const Geom &g, const uint16_t *w, const float *h, const uint16_t *cb,
                           const void *codes_in, void *codes_out, int beam, void *ws, cudaStream_t s)
@@ -272,6 +524,26 @@ cudaError_t launch_encode(const Geom &g, const uint16_t *w, const float *h, cons
                                                           reinterpret_cast<uint8_t *>(codes_out), beam);
         return cudaGetLastError();
     };
+    if (g.B == 16) {
+        float *eg = reinterpret_cast<float *>(reinterpret_cast<char *>(ws) + kWsData +
+                                              align16((size_t)g.G * g.K * 65536 * sizeof(float)));
+        auto run16 = [&](auto kk) {
+            constexpr int K = decltype(kk)::value;
+            encode16_q_kernel<K><<<dim3(65536 / 256, g.G), 256, 0, s>>>(g.in, h, c, q);
+            cudaError_t e = cudaGetLastError();
+            if (e != cudaSuccess) return e;
+            constexpr int smem16 = encode16_smem_bytes();
+            e = cudaFuncSetAttribute(encode16_kernel<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem16);
+            if (e != cudaSuccess) return e;
+            encode16_kernel<K><<<(g.out + kE16Rows - 1) / kE16Rows, kEncThreads, smem16, s>>>(
+                g, w, h, c, q, reinterpret_cast<const uint16_t *>(codes_in), reinterpret_cast<uint16_t *>(codes_out),
+                eg, beam);
+            return cudaGetLastError();
+        };
+        if (g.K == 1) return run16(std::integral_constant<int, 1>{});
+        if (g.K == 2) return run16(std::integral_constant<int, 2>{});
+        return cudaErrorInvalidValue;
+    }
     if (g.B != 8) return cudaErrorInvalidValue;
     if (g.K == 1) return run(std::integral_constant<int, 1>{});
     if (g.K == 2) return run(std::integral_constant<int, 2>{});

@@ -302,14 +302,18 @@ aq_status aq_gemm(const aq_layer_desc *desc, const void *packed, const uint16_t 
  *   w          [out][in] binary16 (the weights to approximate),
  *   h          [in][in] fp32, symmetric (e.g. 2 X^T X of calibration
  *              activations),
- *   codes_in   [out][in/8][K] uint8: the starting codes,
- *   codes_out  [out][in/8][K] uint8, written (may not alias codes_in),
+ *   codes_in   [out][in/8][K] uint8 (B = 8) or uint16 (B = 16): the
+ *              starting codes,
+ *   codes_out  the same shape and type, written (may not alias codes_in),
  *   beam       1..16,
  *   workspace  >= aq_encode_workspace_bytes(desc) bytes (a per-layer table
- *              of C_k[c]^T H_gg C_k[c]).
- * Codebooks of 8-bit codes only (1x8, 2x8, 8x8; AQ_ERR_UNSUPPORTED for
- * B = 16, whose 65536-way search per group this library does not run);
- * in <= 16384.
+ *              of C_k[c]^T H_gg C_k[c]; for B = 16 also the rows' residual
+ *              w - reconstruction, [out][in] fp32).
+ * Every scheme (1x8, 2x8, 8x8, 1x16, 2x16); in <= 16384.  For B = 16 the
+ * search scores all 65536 codes of each slot (one CTA per 16 rows, the
+ * codebook streamed through shared memory): with one codebook the beam
+ * keeps nothing past the group's best proposal, so any beam gives the
+ * codes of beam 1; with two, the first slot keeps `beam` proposals.
  */
 size_t aq_encode_workspace_bytes(const aq_layer_desc *desc);
 aq_status aq_encode(const aq_layer_desc *desc, const uint16_t *w, const float *h, const uint16_t *codebooks,

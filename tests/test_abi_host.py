@@ -243,8 +243,10 @@ def test_encode_argument_errors():
     assert call(co=FAKE) == 1  # codes_out aliases codes_in
     assert call(w=FAKE + 2) == 3 and call(h=FAKE + 4) == 3 and call(cb=FAKE + 8) == 3
     assert call(ws=None) == 4 and call(wsb=16) == 4
-    assert call(desc=aq.LayerDesc.make(64, 256, 1, 16)) == 2   # 16-bit codes: not run
-    assert aq.aq_encode_workspace_bytes(aq.LayerDesc.make(64, 256, 1, 16)) == 0
+    # 16-bit codes: the q table [G][K][65536] and the residual [out][in], fp32
+    assert aq.aq_encode_workspace_bytes(aq.LayerDesc.make(64, 256, 1, 16)) == 4112 + 32 * 65536 * 4 + 64 * 256 * 4
+    assert aq.aq_encode_workspace_bytes(aq.LayerDesc.make(64, 256, 2, 16)) == 4112 + 32 * 2 * 65536 * 4 + 64 * 256 * 4
+    assert call(desc=aq.LayerDesc.make(64, 256, 1, 16), wsb=16) == 4
     assert call(desc=aq.LayerDesc.make(64, 16392, 2, 8)) == 1   # in > 16384
 
 

@@ -351,6 +351,27 @@ def test_gemm_split_k_deterministic_and_reusable(K, B, T):
     assert_close(y1[rows], ref, bound, f"split-K {K}x{B} T{T}")
 
 
+@pytest.mark.parametrize("K,B", [(1, 16), (2, 8)])
+@pytest.mark.parametrize("out,inp,T,ks", [(512, 2048, 392, 4), (256, 4096, 392, 8), (1000, 1032, 520, 2)])
+def test_gemm_cluster_split_ragged_tokens_every_element(K, B, out, inp, T, ks):
+    """Input-feature splits of 2, 4 and 8 that run as one thread-block
+    cluster: each split owns BN / ks of a tile's 512 columns and adds every
+    split's sums for them.  T leaves the last tile ragged (392 = 3 x 128 +
+    8: at 4 splits one owner has 8 live columns, at 8 splits one has 8 and
+    one none), and 1000 rows leave the last row tile ragged.  The workspace
+    size pins the plan (ks splits, tiles of 128 x 512, fp32 sums); every
+    element is checked against the oracle."""
+    desc = aq.LayerDesc.make(out, inp, K, B)
+    tiles = ((out + 127) // 128) * ((T + 511) // 512)
+    assert aq.aq_gemm_workspace_bytes(desc, T) == 4112 + ks * tiles * 128 * 512 * 4
+    layer = _layer(out, inp, K, B, out + inp + T + ks)
+    dl = DevLayer(layer)
+    x = make_activations(inp, T, (out, T, ks))
+    y = run_gemm(dl, x)
+    ref, bound = oracle.matmul(layer.codes, layer.codebooks, layer.scales, x, threads=8)
+    assert_close(y, ref, bound, f"cluster split {ks} {K}x{B} {out}x{inp} T{T}")
+
+
 @pytest.mark.parametrize("K", [2, 1])
 def test_gemv_tables_fall_back_to_exact_decode_beyond_binary16(K):
     """The batch-1 table path keeps its tables in binary16 and bounds their
