@@ -325,7 +325,10 @@ __global__ void __launch_bounds__(kEncThreads) encode16_kernel(Geom L, const uin
     __shared__ float bconst[R][kEncMaxBeam];
     __shared__ uint64_t sel[R][kEncMaxBeam];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int my_r = tid / S, my_s = tid % S;
+    // thread (row my_r, slice my_s): a warp's lanes are 16 rows x 2 slices,
+    // so a codeword read serves 16 rows (2 codewords per warp access)
+    static_assert(R == 16 && S == 16, "16 rows x 16 slices");
+    const int my_r = lane & 15, my_s = (warp << 1) | (lane >> 4);
     const int in = L.in, G = L.G, o0 = blockIdx.x * R;
     const int nrows = min(R, L.out - o0);
 
@@ -411,40 +414,77 @@ __global__ void __launch_bounds__(kEncThreads) encode16_kernel(Geom L, const uin
             for (int i = 0; i < kEncMaxBeam; ++i) top[i] = ~0ull;
             uint64_t worst = ~0ull;  // top[nsel - 1]
             const float *qk = qtab + ((size_t)g * K + k) * 65536;
+            const uint4 *cbk = cb + (size_t)k * 65536;
+            // each thread moves kPer codewords and q values of a chunk; the
+            // next chunk's are in flight (registers) while this one is scored
+            constexpr int kPer = kE16Chunk / kEncThreads;
+            uint4 nx[kPer];
+            float nq[kPer];
+#pragma unroll
+            for (int p = 0; p < kPer; ++p) {
+                nx[p] = cbk[tid + p * kEncThreads];
+                nq[p] = qk[tid + p * kEncThreads];
+            }
 #pragma unroll 1
             for (int base = 0; base < 65536; base += kE16Chunk) {
                 __syncthreads();  // the previous chunk is consumed (and bw, bconst written)
-                for (int i = tid; i < kE16Chunk; i += kEncThreads) {
+#pragma unroll
+                for (int p = 0; p < kPer; ++p) {
                     float x[8];
-                    load_f8(cb[(size_t)k * 65536 + base + i], x);
+                    load_f8(nx[p], x);
+                    const int i = tid + p * kEncThreads;
 #pragma unroll
                     for (int j = 0; j < 8; ++j) sx[i][j] = x[j];
-                    sq[i] = qk[base + i];
+                    sq[i] = nq[p];
                 }
+                if (base + kE16Chunk < 65536)
+#pragma unroll
+                    for (int p = 0; p < kPer; ++p) {
+                        nx[p] = cbk[base + kE16Chunk + tid + p * kEncThreads];
+                        nq[p] = qk[base + kE16Chunk + tid + p * kEncThreads];
+                    }
                 __syncthreads();
                 if (my_r >= nrows) continue;
-#pragma unroll 1
-                for (int c = my_s; c < kE16Chunk; c += S) {
-                    const float qc = sq[c];
-#pragma unroll 1
-                    for (int b = 0; b < nb; ++b) {
+                auto offer = [&](uint64_t key) {
+                    if (key < worst) {
+                        // insert, dropping the largest; keep the list sorted
+                        uint64_t x = key;
+#pragma unroll
+                        for (int i = 0; i < kEncMaxBeam; ++i)
+                            if (i < nsel) {
+                                const uint64_t lo = top[i] < x ? top[i] : x, hi = top[i] < x ? x : top[i];
+                                top[i] = lo;
+                                x = hi;
+                            }
+#pragma unroll
+                        for (int i = 0; i < kEncMaxBeam; ++i)
+                            if (i == nsel - 1) worst = top[i];
+                    }
+                };
+                if (nb == 1) {
+                    // one live beam (every slot of 1x16, the first of 2x16):
+                    // its w and constant stay in registers
+                    float wr[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) wr[j] = bw[my_r][0][j];
+                    const float cst = bconst[my_r][0];
+#pragma unroll 4
+                    for (int c = my_s; c < kE16Chunk; c += S) {
                         float d = 0.f;
 #pragma unroll
-                        for (int j = 0; j < 8; ++j) d = fmaf(sx[c][j], bw[my_r][b][j], d);
-                        const uint64_t key = enc16_key(bconst[my_r][b] + qc + 2.f * d, b, base + c);
-                        if (key < worst) {
-                            // insert, dropping the largest; keep the list sorted
-                            uint64_t x = key;
+                        for (int j = 0; j < 8; ++j) d = fmaf(sx[c][j], wr[j], d);
+                        offer(enc16_key(cst + sq[c] + 2.f * d, 0, base + c));
+                    }
+                } else {
+#pragma unroll 1
+                    for (int c = my_s; c < kE16Chunk; c += S) {
+                        const float qc = sq[c];
+#pragma unroll 1
+                        for (int b = 0; b < nb; ++b) {
+                            float d = 0.f;
 #pragma unroll
-                            for (int i = 0; i < kEncMaxBeam; ++i)
-                                if (i < nsel) {
-                                    const uint64_t lo = top[i] < x ? top[i] : x, hi = top[i] < x ? x : top[i];
-                                    top[i] = lo;
-                                    x = hi;
-                                }
-#pragma unroll
-                            for (int i = 0; i < kEncMaxBeam; ++i)
-                                if (i == nsel - 1) worst = top[i];
+                            for (int j = 0; j < 8; ++j) d = fmaf(sx[c][j], bw[my_r][b][j], d);
+                            offer(enc16_key(bconst[my_r][b] + qc + 2.f * d, b, base + c));
                         }
                     }
                 }

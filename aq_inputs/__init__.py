@@ -154,8 +154,10 @@ def workload(name: str) -> dict:
                   for tag, (o, i) in (("q", LLAMA2_7B_BLOCK["q"]), ("gate", LLAMA2_7B_BLOCK["gate"]))]
         return {"layers": layers, "n": [2048], "seed": 1007}
     if name == "llama2-7b-encode":
-        # code assignment (beam 8) for a 2x8 q projection and MLP up shape
-        layers = [("q-2x8", LayerSpec(4096, 4096, 2, 8)), ("gate-2x8", LayerSpec(11008, 4096, 2, 8))]
+        # code assignment (beam 8) for a 2x8 q projection and MLP up shape,
+        # and a 1x16 q projection (65536 codes scored per group)
+        layers = [("q-2x8", LayerSpec(4096, 4096, 2, 8)), ("gate-2x8", LayerSpec(11008, 4096, 2, 8)),
+                  ("q-1x16", LayerSpec(4096, 4096, 1, 16))]
         return {"layers": layers, "n": [8], "seed": 1008}
     if name == "llama2-7b-schemes":
         # the other schemes the pages name, at the Llama-2-7B MLP up shape

@@ -322,11 +322,13 @@ def recorded_traffic(layer: str, batch: int):
 
 def encode_flops(spec: LayerSpec, beam: int) -> int:
     """Arithmetic of one aq_encode call: (H e)_g for every row and group
-    (2 out in^2) plus scoring every code for every beam of every slot
-    (about 18 flops per score)."""
+    (2 out in^2) plus scoring every code of every slot for each live beam
+    (one at a group's first slot, `beam` after it; about 18 flops per
+    score)."""
     G = spec.in_features // 8
+    beams_per_group = 1 + (spec.num_codebooks - 1) * beam
     return (2 * spec.out_features * spec.in_features ** 2
-            + spec.out_features * G * spec.num_codebooks * beam * (1 << spec.nbits) * 18)
+            + spec.out_features * G * beams_per_group * (1 << spec.nbits) * 18)
 
 
 def encode_inputs(spec: LayerSpec, beam: int, seed) -> dict:
@@ -338,7 +340,7 @@ def encode_inputs(spec: LayerSpec, beam: int, seed) -> dict:
     x = torch.from_numpy(rng.normal(0, 1, size=(512, spec.in_features)).astype(np.float32)).cuda()
     h = (2.0 / 512) * (x.T @ x)
     c0 = rng.integers(0, 1 << spec.nbits, size=(spec.out_features, spec.in_features // 8, spec.num_codebooks))
-    codes = torch.from_numpy(c0.astype(np.uint8)).cuda()
+    codes = torch.from_numpy(c0.astype(np.uint8) if spec.nbits == 8 else c0.astype(np.uint16).view(np.int16)).cuda()
     return {"w": torch.from_numpy(w.view(np.int16)).cuda(), "h": h.contiguous(), "codes_in": codes,
             "codes_out": torch.empty_like(codes)}
 
