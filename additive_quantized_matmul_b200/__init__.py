@@ -20,7 +20,8 @@ __all__ = [
     "AQError", "LayerDesc", "lib", "library_path", "aq_version", "aq_status_string",
     "aq_packed_codes_bytes", "aq_gemv_workspace_bytes", "aq_gemm_workspace_bytes",
     "aq_workspace_status", "aq_selftest_bounded_wait", "aq_pack_codes", "aq_unpack_codes",
-    "aq_dequant", "aq_gemv", "aq_gemv_ordered", "aq_gemv_noalloc", "aq_gemm", "aq_param_grad_workspace_bytes",
+    "aq_dequant", "aq_gemv", "aq_gemv_ordered", "aq_gemv_noalloc", "aq_gemm", "aq_gemm_ordered",
+    "aq_param_grad_workspace_bytes",
     "aq_param_grad", "aq_encode_workspace_bytes", "aq_encode", "aq_gather_probe_sink_bytes",
     "aq_gather_probe", "EXPORTED_SYMBOLS",
     "GEMV_NOALLOC_SCRATCH_BYTES",
@@ -39,6 +40,7 @@ EXPORTED_SYMBOLS = (
     "aq_status_string", "aq_version", "aq_packed_codes_bytes", "aq_gemv_workspace_bytes",
     "aq_gemm_workspace_bytes", "aq_workspace_status", "aq_selftest_bounded_wait",
     "aq_pack_codes", "aq_unpack_codes", "aq_dequant", "aq_gemv", "aq_gemv_ordered", "aq_gemv_noalloc", "aq_gemm",
+    "aq_gemm_ordered",
     "aq_param_grad_workspace_bytes", "aq_param_grad", "aq_encode_workspace_bytes", "aq_encode",
     "aq_gather_probe_sink_bytes", "aq_gather_probe",
 )
@@ -90,6 +92,7 @@ def _load() -> ctypes.CDLL:
         "aq_gemv": ([dp, vp, vp, vp, vp, i32, vp, vp, sz, vp], i32),
         "aq_gemv_ordered": ([dp, vp, vp, vp, vp, i32, vp, vp, sz, vp], i32),
         "aq_gemm": ([dp, vp, vp, vp, vp, i32, vp, vp, sz, vp], i32),
+        "aq_gemm_ordered": ([dp, vp, vp, vp, vp, i32, vp, vp, sz, vp], i32),
         "aq_gemv_noalloc": ([dp, vp, vp, vp, vp, i32, vp, vp], i32),
         "aq_param_grad_workspace_bytes": ([dp, i32], sz),
         "aq_param_grad": ([dp, vp, vp, vp, vp, vp, i32, vp, vp, vp, sz, vp], i32),
@@ -210,6 +213,17 @@ def aq_gemm(desc: LayerDesc, packed, codebooks, scales, x, T: int, y, workspace,
     _check("aq_gemm", lib.aq_gemm(ctypes.byref(desc), _ptr(packed), _ptr(codebooks), _ptr(scales),
                                   _ptr(x), T, _ptr(y), _ptr(workspace), workspace_bytes,
                                   _stream(stream)))
+
+
+def aq_gemm_ordered(desc: LayerDesc, packed, codebooks, scales, x, T: int, y, workspace,
+                    workspace_bytes: int | None = None, stream=None) -> None:
+    """aq_gemm launched without programmatic dependent launch: no weight is
+    read before the previous work on the stream has completed."""
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    _check("aq_gemm_ordered", lib.aq_gemm_ordered(ctypes.byref(desc), _ptr(packed), _ptr(codebooks), _ptr(scales),
+                                                  _ptr(x), T, _ptr(y), _ptr(workspace), workspace_bytes,
+                                                  _stream(stream)))
 
 
 def aq_param_grad_workspace_bytes(desc: LayerDesc, T: int) -> int:

@@ -186,9 +186,9 @@ aq_status aq_gemv_noalloc(const aq_layer_desc *desc, const void *packed, const u
     return from_cuda(e);
 }
 
-aq_status aq_gemm(const aq_layer_desc *desc, const void *packed, const uint16_t *codebooks,
-                  const uint16_t *scales, const uint16_t *x, int T, uint16_t *y,
-                  void *workspace, size_t workspace_bytes, aq_stream_t stream)
+static aq_status gemm_entry(const aq_layer_desc *desc, const void *packed, const uint16_t *codebooks,
+                            const uint16_t *scales, const uint16_t *x, int T, uint16_t *y,
+                            void *workspace, size_t workspace_bytes, aq_stream_t stream, bool pdl)
 {
     aq_status st = check_desc(desc);
     if (st != AQ_OK) return st;
@@ -202,7 +202,21 @@ aq_status aq_gemm(const aq_layer_desc *desc, const void *packed, const uint16_t 
     if (!workspace || workspace_bytes < need) return AQ_ERR_WORKSPACE;
     if (!aligned16(workspace)) return AQ_ERR_MISALIGNED;
     return from_cuda(aqh::launch_gemm(g, packed, codebooks, scales, x, T, y, workspace,
-                                      reinterpret_cast<cudaStream_t>(stream)));
+                                      reinterpret_cast<cudaStream_t>(stream), pdl));
+}
+
+aq_status aq_gemm(const aq_layer_desc *desc, const void *packed, const uint16_t *codebooks,
+                  const uint16_t *scales, const uint16_t *x, int T, uint16_t *y,
+                  void *workspace, size_t workspace_bytes, aq_stream_t stream)
+{
+    return gemm_entry(desc, packed, codebooks, scales, x, T, y, workspace, workspace_bytes, stream, true);
+}
+
+aq_status aq_gemm_ordered(const aq_layer_desc *desc, const void *packed, const uint16_t *codebooks,
+                          const uint16_t *scales, const uint16_t *x, int T, uint16_t *y,
+                          void *workspace, size_t workspace_bytes, aq_stream_t stream)
+{
+    return gemm_entry(desc, packed, codebooks, scales, x, T, y, workspace, workspace_bytes, stream, false);
 }
 
 size_t aq_encode_workspace_bytes(const aq_layer_desc *desc)

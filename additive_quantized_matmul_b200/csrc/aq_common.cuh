@@ -271,7 +271,7 @@ cudaError_t launch_gemv_noalloc(const aqk::Geom &g, const void *packed, const ui
 size_t gemm_workspace_bytes(const aqk::Geom &g, int T);
 cudaError_t launch_gemm(const aqk::Geom &g, const void *packed, const uint16_t *cb,
                         const uint16_t *scales, const uint16_t *x, int T, uint16_t *y,
-                        void *ws, cudaStream_t s);
+                        void *ws, cudaStream_t s, bool pdl);
 size_t param_grad_workspace_bytes(const aqk::Geom &g, int T);
 cudaError_t launch_param_grad(const aqk::Geom &g, const void *packed, const uint16_t *cb, const uint16_t *scales,
                               const uint16_t *x, const uint16_t *gy, int T, float *grad_s, float *grad_cb,

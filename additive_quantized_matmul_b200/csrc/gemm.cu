@@ -458,10 +458,14 @@ gemm_ws_kernel(const __grid_constant__ CUtensorMap xmap, Geom L, const uint8_t *
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     volatile uint32_t *abort_v = abort_flag;
+    // programmatic dependent launch: before the wait a thread reads weights
+    // only (codes, codebooks); X, y, the scales and the workspace follow it
+    grid_launch_dependents();
 
     if (warp == 0) {
         // ---------------- X producer ----------------
         if (lane == 0) {
+            grid_dependency_wait();
             for (int s = 0; s < nk; ++s) {
                 const int buf = s % kWsStages;
                 if (s >= kWsStages && !mbar_wait_ns(&empty[buf], ((s / kWsStages) - 1) & 1, kWaitNs)) {
@@ -613,6 +617,7 @@ gemm_ws_kernel(const __grid_constant__ CUtensorMap xmap, Geom L, const uint8_t *
             }
         }
         cp_async_wait<0>();
+        grid_dependency_wait();  // y, the scales and the workspace
         // ---------------- epilogue ----------------
         const bool got = (*abort_v == 0) && mbar_wait_ns(acc_full, 0, kWaitNs);
         if (!got) *abort_v = 1;
@@ -657,6 +662,7 @@ gemm_ws_kernel(const __grid_constant__ CUtensorMap xmap, Geom L, const uint8_t *
             }
         }
     }
+    grid_dependency_wait();  // every thread, before the workspace and y
     __syncthreads();
     if (*abort_v) {
         // something gave up: record it and drain what was issued (bounded)
@@ -788,7 +794,7 @@ static constexpr int gemm_ws_smem_bytes()
 
 cudaError_t launch_gemm(const Geom &g, const void *packed, const uint16_t *cb,
                         const uint16_t *scales, const uint16_t *x, int T, uint16_t *y, void *ws,
-                        cudaStream_t s)
+                        cudaStream_t s, bool pdl)
 {
     const uint8_t *pk = reinterpret_cast<const uint8_t *>(packed);
     const uint4 *c = reinterpret_cast<const uint4 *>(cb);
@@ -821,13 +827,22 @@ cudaError_t launch_gemm(const Geom &g, const void *packed, const uint16_t *cb,
             cfg.blockDim = dim3(kWsThreadsOf<S>);
             cfg.dynamicSmemBytes = smem;
             cfg.stream = s;
-            cudaLaunchAttribute attr[1];
-            attr[0].id = cudaLaunchAttributeClusterDimension;
-            attr[0].val.clusterDim.x = 1;
-            attr[0].val.clusterDim.y = 1;
-            attr[0].val.clusterDim.z = p.ks;
+            cudaLaunchAttribute attr[2];
+            int na = 0;
+            if (p.cluster) {
+                attr[na].id = cudaLaunchAttributeClusterDimension;
+                attr[na].val.clusterDim.x = 1;
+                attr[na].val.clusterDim.y = 1;
+                attr[na].val.clusterDim.z = p.ks;
+                ++na;
+            }
+            if (pdl) {
+                attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+                attr[na].val.programmaticStreamSerializationAllowed = 1;
+                ++na;
+            }
             cfg.attrs = attr;
-            cfg.numAttrs = p.cluster ? 1 : 0;
+            cfg.numAttrs = na;
             e = cudaLaunchKernelEx(&cfg, gemm_ws_kernel<S, BN>, map, g, pk, c, scales, T, y, ws, sp, p.per_split,
                                    p.cluster ? p.ks : 0);
             if (e != cudaSuccess) return e;

@@ -258,10 +258,24 @@ aq_status aq_gemv_noalloc(const aq_layer_desc *desc, const void *packed, const u
  * records AQ_ERR_TIMEOUT in the workspace status word (see
  * aq_workspace_status), frees its tensor memory and returns; the output is
  * then incomplete but the context stays usable.
+ * Early weight reads: for T a multiple of 8 the kernel is launched with
+ * programmatic dependent launch, as aq_gemv is, and may read `packed` and
+ * `codebooks` before the kernel launched just before it on `stream` has
+ * finished (x, scales, y and the workspace only after); aq_gemv's rule on
+ * early weight reads applies, and aq_gemm_ordered is the ordinary launch.
  */
 aq_status aq_gemm(const aq_layer_desc *desc, const void *packed, const uint16_t *codebooks,
                   const uint16_t *scales, const uint16_t *x, int T, uint16_t *y,
                   void *workspace, size_t workspace_bytes, aq_stream_t stream);
+
+/*
+ * aq_gemm with an ordinary launch: the kernel starts only after all work
+ * queued before it on `stream` has completed, so it reads no weight early.
+ * Same arguments, plan and results (bit for bit) as aq_gemm.
+ */
+aq_status aq_gemm_ordered(const aq_layer_desc *desc, const void *packed, const uint16_t *codebooks,
+                          const uint16_t *scales, const uint16_t *x, int T, uint16_t *y,
+                          void *workspace, size_t workspace_bytes, aq_stream_t stream);
 
 /*
  * Parameter gradient of a quantised layer: for the loss L = sum(gy * y) with

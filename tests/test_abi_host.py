@@ -115,8 +115,8 @@ def _gemv(d, packed=FAKE, cb=FAKE, s=FAKE, x=FAKE, batch=1, y=FAKE, ws=FAKE, wsb
     return getattr(aq.lib, fn)(ctypes.byref(d), packed, cb, s, x, batch, y, ws, wsb, None)
 
 
-def _gemm(d, packed=FAKE, cb=FAKE, s=FAKE, x=FAKE, T=64, y=FAKE, ws=FAKE, wsb=1 << 30):
-    return aq.lib.aq_gemm(ctypes.byref(d), packed, cb, s, x, T, y, ws, wsb, None)
+def _gemm(d, packed=FAKE, cb=FAKE, s=FAKE, x=FAKE, T=64, y=FAKE, ws=FAKE, wsb=1 << 30, fn="aq_gemm"):
+    return getattr(aq.lib, fn)(ctypes.byref(d), packed, cb, s, x, T, y, ws, wsb, None)
 
 
 @pytest.mark.parametrize("fn", ["aq_gemv", "aq_gemv_ordered"])
@@ -139,14 +139,15 @@ def test_gemv_argument_errors(fn):
     assert getattr(aq.lib, fn)(None, FAKE, FAKE, FAKE, FAKE, 1, FAKE, FAKE, 1 << 20, None) == 1
 
 
-def test_gemm_argument_errors():
+@pytest.mark.parametrize("fn", ["aq_gemm", "aq_gemm_ordered"])
+def test_gemm_argument_errors(fn):
     d = aq.LayerDesc.make(64, 256, 1, 16)
-    assert _gemm(d, T=0) == 1
-    assert _gemm(d, T=-5) == 1
-    assert _gemm(d, x=None) == 1
-    assert _gemm(d, y=FAKE + 2) == 3
-    assert _gemm(d, ws=None) == 4
-    assert _gemm(d, wsb=0) == 4
+    assert _gemm(d, T=0, fn=fn) == 1
+    assert _gemm(d, T=-5, fn=fn) == 1
+    assert _gemm(d, x=None, fn=fn) == 1
+    assert _gemm(d, y=FAKE + 2, fn=fn) == 3
+    assert _gemm(d, ws=None, fn=fn) == 4
+    assert _gemm(d, wsb=0, fn=fn) == 4
 
 
 def test_pack_and_misc_argument_errors():

@@ -17,7 +17,9 @@ consumed, so every step is held to the tolerance on its own.
   block's down-projection output (16 dependent products deep);
 * the benchmark's rotation: 76 copies of a 4096 x 4096 1x16 layer at
   distinct addresses, batch 1, 4 and 16, in one CUDA graph, all copies of a
-  batch sharing one workspace.
+  batch sharing one workspace;
+* the block's seven prefill products (aq_gemm, also launched with
+  programmatic dependent launch) at 512 and 136 tokens.
 
 Weights of the multi-block chain are drawn with codebook spreads that keep
 the activations' magnitude about constant from layer to layer (gain ~1), so
@@ -207,3 +209,49 @@ def test_ordered_entry_point_same_bits_as_gemv(K, B, batch):
     for tag in BLOCK:
         assert torch.equal(ys_pdl[tag], ys_ord[tag]), f"{K}x{B} b{batch} {tag}: ordered launch differs"
     _check_block(layers, x, ys_ord, batch, f"ordered {K}x{B} b{batch}")
+
+
+@pytest.mark.parametrize("K,B", [(1, 16), (2, 8)])
+@pytest.mark.parametrize("T", [512, 136])
+def test_prefill_block_chain_under_programmatic_launch(K, B, T):
+    """The seven prefill products of a Llama-2-7B block on one stream, no
+    host synchronisation, one workspace: aq_gemm launches with programmatic
+    dependent launch (a kernel reads its weights while the previous product
+    may still run; x, y and the workspace only after it).  512 tokens: the
+    4096-row products split their input features 4 ways in clusters; 136
+    tokens: ragged 256-token tiles.  Each product is checked on sampled rows
+    against the oracle applied to the GPU input it consumed, and the same
+    chain through aq_gemm_ordered gives the same bits."""
+    layers = _block_layers(K, B, (T, K, 3), unit_gain=True)
+    dls = {tag: DevLayer(layers[tag]) for tag in BLOCK}
+    x_host = make_activations(LLAMA2_7B_BLOCK["q"][1], T, (T, K, 4))
+    x = dev(x_host.view(np.uint16))
+    ws = workspace(max(aq.aq_gemm_workspace_bytes(dls[tag].desc, T) for tag in BLOCK))
+    stream = torch.cuda.Stream()
+
+    def chain(fn):
+        ys = {tag: torch.empty(LLAMA2_7B_BLOCK[tag][0] * T, dtype=torch.int16, device="cuda") for tag in BLOCK}
+        for tag in BLOCK:
+            dl = dls[tag]
+            src = SOURCE[tag]
+            fn(dl.desc, dl.packed, dl.codebooks, dl.scales, x if src is None else ys[src], T, ys[tag], ws,
+               stream=stream)
+        torch.cuda.synchronize()
+        return ys
+
+    ys = chain(aq.aq_gemm)
+    assert aq.aq_workspace_status(ws, stream=stream) == 0, "a bounded wait gave up"
+    got = {tag: to_f16(ys[tag]).reshape(-1, T) for tag in BLOCK}
+    rng = np.random.default_rng(T + K)
+    for tag in BLOCK:
+        L = layers[tag]
+        src = SOURCE[tag]
+        xin = x_host if src is None else got[src]
+        assert np.isfinite(xin.astype(np.float64)).all()
+        out = LLAMA2_7B_BLOCK[tag][0]
+        rows = np.unique(np.concatenate([rng.choice(out, size=20, replace=False), [0, 127, 128, out - 1]]))
+        ref, bound = oracle.matmul(L.codes, L.codebooks, L.scales, xin, rows=rows, threads=8)
+        assert_close(got[tag][rows].astype(np.float64), ref, bound, f"prefill chain {K}x{B} T{T} {tag}")
+    ys2 = chain(aq.aq_gemm_ordered)
+    for tag in BLOCK:
+        assert torch.equal(ys[tag], ys2[tag]), f"ordered launch differs at {tag}"
