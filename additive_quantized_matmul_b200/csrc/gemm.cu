@@ -401,11 +401,109 @@ __device__ void gemm_cluster_finish(const Geom &L, uint32_t tmem, float *__restr
     }
 }
 
+// The tail of a tile grid larger than one wave: when the last wave would
+// hold few tiles, their input features are split over `ks` CTAs each (a 1-D
+// grid: whole tiles first, then the tail tiles' splits), so the last wave
+// fills the SMs.  Such a tile is finished by the last of its splits to
+// arrive: each writes its fp32 sums from tensor memory to its slice (the
+// order tensor memory hands them out, as gemm_cluster_finish), arrives on
+// the tile's counter (acq_rel), and the last adds every split's sums in
+// split order (its own from tensor memory; deterministic), scales, rounds,
+// writes y and resets the counter.  Every thread of the CTA calls it.
+template <int BN, int NW>
+__device__ void gemm_tail_finish(const Geom &L, uint32_t tmem, float *__restrict__ slices_base, unsigned *counter,
+                                 int m0, int n0, int T, int z, int ks, const uint16_t *__restrict__ scales,
+                                 uint16_t *__restrict__ y, int fw, bool ok)
+{
+    constexpr int kH = NW / 4;
+    constexpr size_t kSlice = kBM * BN / 4;  // float4 per slice
+    __shared__ unsigned s_last;
+    const int lane = threadIdx.x & 31, q = (threadIdx.x >> 5) & 3;
+    const int r = q * 32 + lane, row = m0 + r;
+    float4 *slices = reinterpret_cast<float4 *>(slices_base);
+    const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16);
+    tc_fence_after();
+    if (fw >= 0 && ok) {
+        float4 *mine = slices + (size_t)z * kSlice;
+#pragma unroll 1
+        for (int c0 = 16 * (fw / 4); c0 < BN; c0 += 16 * kH) {
+            if (n0 + c0 >= T) break;  // warp-uniform
+            float v[16];
+            tmem_ld16(tq + (uint32_t)c0, v);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                __stcg(mine + ((c0 / 16) * 4 + j) * kBM + r, make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]));
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        // the barrier orders the CTA's slice stores before this increment,
+        // whose release publishes them; its acquire orders the last CTA's
+        // reads after every split's
+        const unsigned prev = atom_add_acq_rel_gpu(counter, 1u);
+        s_last = (prev == (unsigned)ks - 1u) ? 1u : 0u;
+    }
+    __syncthreads();
+    if (!s_last) return;
+    if (fw >= 0 && ok) {
+        const bool live_row = row < L.out;
+        const float sc = (live_row && scales) ? __half2float(__ushort_as_half(scales[row])) : 1.f;
+#pragma unroll 1
+        for (int c0 = 16 * (fw / 4); c0 < BN; c0 += 16 * kH) {
+            const int gn = n0 + c0;
+            if (gn >= T) break;  // warp-uniform
+            float v[16];
+            tmem_ld16(tq + (uint32_t)c0, v);
+            const float4 *src = slices + ((c0 / 16) * 4) * kBM + r;
+            float acc[16];
+            for (int z0 = 0; z0 < ks; z0 += 4) {
+                float4 t[4][4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        if (z0 + i < ks && z0 + i != z) t[i][j] = __ldcg(src + (size_t)(z0 + i) * kSlice + j * kBM);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    if (z0 + i >= ks) break;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const float4 u = (z0 + i == z) ? make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3])
+                                                       : t[i][j];
+                        if (z0 + i == 0) {
+                            acc[4 * j] = u.x, acc[4 * j + 1] = u.y, acc[4 * j + 2] = u.z, acc[4 * j + 3] = u.w;
+                        } else {
+                            acc[4 * j] += u.x, acc[4 * j + 1] += u.y, acc[4 * j + 2] += u.z, acc[4 * j + 3] += u.w;
+                        }
+                    }
+                }
+            }
+            if (!live_row) continue;
+            uint16_t *dst = y + (size_t)row * T + gn;
+            const uint4 o0 = make_uint4(f2h2(sc * acc[0], sc * acc[1]), f2h2(sc * acc[2], sc * acc[3]),
+                                        f2h2(sc * acc[4], sc * acc[5]), f2h2(sc * acc[6], sc * acc[7]));
+            const uint4 o1 = make_uint4(f2h2(sc * acc[8], sc * acc[9]), f2h2(sc * acc[10], sc * acc[11]),
+                                        f2h2(sc * acc[12], sc * acc[13]), f2h2(sc * acc[14], sc * acc[15]));
+            reinterpret_cast<uint4 *>(dst)[0] = o0;  // T % 8 == 0: gn + 8 <= T
+            if (gn + 16 <= T) reinterpret_cast<uint4 *>(dst)[1] = o1;
+        }
+    }
+    if (threadIdx.x == 0) *counter = 0u;
+}
+
+// Grid of the tail mode: CTAs [0, full) take whole tiles (tile = index), the
+// others split the tiles from `full` on, `ks` CTAs of `per` stages each.
+struct TailMap {
+    int full;  // CTAs with a whole tile; 0: no tail mode (3-D grid)
+    int ks;    // splits per tail tile
+    int per;   // 64-feature stages per split
+};
+
 template <class S, int BN>
 __global__ void __launch_bounds__(kWsThreadsOf<S>, 1)
 gemm_ws_kernel(const __grid_constant__ CUtensorMap xmap, Geom L, const uint8_t *__restrict__ packed,
                const uint4 *__restrict__ cb, const uint16_t *__restrict__ scales, int T,
-               uint16_t *__restrict__ y, void *ws, GemmSplit sp, int stages_per_split, int cluster_ks)
+               uint16_t *__restrict__ y, void *ws, GemmSplit sp, int stages_per_split, int cluster_ks, TailMap tm)
 {
     constexpr int kWsStages = kWsStagesOf<S, BN>;    // X ring
     constexpr int kWsAStages = kWsAStagesOf<S, BN>;  // W ring
@@ -426,11 +524,29 @@ gemm_ws_kernel(const __grid_constant__ CUtensorMap xmap, Geom L, const uint8_t *
     uint32_t *abort_flag = tmem_slot + 1;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int m0 = blockIdx.x * kBM;
-    const int n0 = blockIdx.y * BN;
+    // the CTA's tile and split: a 3-D grid (row tile, token tile, split), or
+    // the tail mode's 1-D grid
+    int mt = blockIdx.x, nt = blockIdx.y, z = blockIdx.z, per = stages_per_split, tail_idx = -1;
+    if (tm.ks > 0) {
+        const int mtiles = (L.out + kBM - 1) / kBM;
+        int tile = blockIdx.x;
+        z = 0;
+        per = (L.in + kBK - 1) / kBK;
+        if (tile >= tm.full) {
+            const int rr = tile - tm.full;
+            tail_idx = rr / tm.ks;
+            z = rr % tm.ks;
+            tile = tm.full + tail_idx;
+            per = tm.per;
+        }
+        mt = tile % mtiles;
+        nt = tile / mtiles;
+    }
+    const int m0 = mt * kBM;
+    const int n0 = nt * BN;
     // this split's stages: global stages s0 .. s0 + nk - 1 (64 features each)
-    const int s0 = blockIdx.z * stages_per_split;
-    const int nk = max(0, min((L.in + kBK - 1) / kBK, s0 + stages_per_split) - s0);
+    const int s0 = z * per;
+    const int nk = max(0, min((L.in + kBK - 1) / kBK, s0 + per) - s0);
     const int g0 = s0 * 8;  // first code group of the split
 
     // 1x16: codewords go from L2 into the tile by cp.async, copies of kWsLag
@@ -626,7 +742,7 @@ gemm_ws_kernel(const __grid_constant__ CUtensorMap xmap, Geom L, const uint8_t *
         // this point by a role that gave up, or just above by a lane whose
         // wait failed (then its warp-mates see it through the ballot)
         const bool warp_ok = __all_sync(0xffffffffu, got);
-        if (warp_ok && dg == 0 && cluster_ks == 0) {
+        if (warp_ok && dg == 0 && cluster_ks == 0 && tail_idx < 0) {
             const int q = warp & 3;  // TMEM lane quarter of this warp
             const int row = m0 + q * 32 + lane;
             const float sc = (row < L.out && scales) ? __half2float(__ushort_as_half(scales[row])) : 1.f;
@@ -639,7 +755,7 @@ gemm_ws_kernel(const __grid_constant__ CUtensorMap xmap, Geom L, const uint8_t *
                 if (sp.partials) {
                     // one of several splits: fp32 partial sums, T % 8 == 0 here
                     if (row < L.out && gn < T) {
-                        float4 *dst = reinterpret_cast<float4 *>(sp.partials + ((size_t)blockIdx.z * L.out + row) * T + gn);
+                        float4 *dst = reinterpret_cast<float4 *>(sp.partials + ((size_t)z * L.out + row) * T + gn);
 #pragma unroll
                         for (int q4 = 0; q4 < 4; ++q4)
                             if (gn + 4 * q4 < T) dst[q4] = make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
@@ -678,12 +794,21 @@ gemm_ws_kernel(const __grid_constant__ CUtensorMap xmap, Geom L, const uint8_t *
         gemm_cluster_finish<BN, NW>(L, tmem, sp.partials, m0, n0, T, cluster_ks, scales, y,
                                     warp >= 2 ? warp - 2 : -1, *abort_v == 0);
     }
+    if (tail_idx >= 0) {
+        // a tail tile's split: the last of its splits finishes it
+        constexpr int NW = 4 * kWsGroupsOf<S>;
+        float *slices = reinterpret_cast<float *>(reinterpret_cast<char *>(ws) + kWsData) +
+                        (size_t)tail_idx * tm.ks * kBM * BN;
+        unsigned *counter = reinterpret_cast<unsigned *>(reinterpret_cast<char *>(ws) + kWsHeader) + tail_idx;
+        gemm_tail_finish<BN, NW>(L, tmem, slices, counter, m0, n0, T, z, tm.ks, scales, y,
+                                 warp >= 2 ? warp - 2 : -1, *abort_v == 0);
+    }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, BN);
     // arrive even after a timeout so the counters stay consistent (the
     // status word already tells the caller the output is incomplete)
-    if (sp.partials && cluster_ks == 0) gemm_split_finish(L, sp, m0, n0, BN, T, scales, y);
+    if (sp.partials && cluster_ks == 0 && tail_idx < 0) gemm_split_finish(L, sp, m0, n0, BN, T, scales, y);
 }
 
 // ---- self-test of the bounded wait -----------------------------------------
@@ -714,6 +839,7 @@ struct GemmPlan {
     int ks;           // splits of the input features (blockIdx.z)
     int per_split;    // 64-feature stages per split
     bool cluster;     // the splits form one cluster and finish on chip
+    TailMap tail;     // ks > 0: the tail mode's 1-D grid
     size_t ws_bytes;  // status word + tile counters + fp32 partials
 };
 
@@ -760,6 +886,21 @@ static GemmPlan plan_gemm(const Geom &g, int T)
     if (!cluster && tiles > kWsMaxCounters) p.ks = 1, p.per_split = nst;
     if (p.ks > 1)
         p.ws_bytes = kWsData + (cluster ? (size_t)p.ks * tiles * kBM * p.bn : (size_t)p.ks * g.out * T) * sizeof(float);
+    // more tiles than one wave, the last wave at most half full: its tiles'
+    // input features are split so that it fills the SMs (Llama-2-7B MLP
+    // rows at 2048 tokens: 344 tiles, 48 in the third wave, split 3 ways)
+    if (p.ks == 1 && tiles > kNumSMs) {
+        const long tail = tiles % kNumSMs;
+        if (tail > 0 && tail * 2 <= kNumSMs && tail <= kWsMaxCounters) {
+            int kt = std::min((int)(kNumSMs / tail), std::min(nst / 8, 8));
+            if (kt >= 2) {
+                const int per = (nst + kt - 1) / kt;
+                kt = (nst + per - 1) / per;  // no empty split
+                p.tail = TailMap{(int)(tiles - tail), kt, per};
+                p.ws_bytes = kWsData + (size_t)tail * kt * kBM * p.bn * sizeof(float);
+            }
+        }
+    }
     return p;
 }
 
@@ -811,7 +952,9 @@ cudaError_t launch_gemm(const Geom &g, const void *packed, const uint16_t *cb,
                             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                             CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
-        const dim3 grid(p.mtiles, p.ntiles, p.ks);
+        const long tiles = (long)p.mtiles * p.ntiles;
+        const dim3 grid = p.tail.ks > 0 ? dim3((unsigned)(p.tail.full + (tiles - p.tail.full) * p.tail.ks), 1, 1)
+                                        : dim3(p.mtiles, p.ntiles, p.ks);
         GemmSplit sp{nullptr, reinterpret_cast<unsigned *>(reinterpret_cast<char *>(ws) + kWsHeader)};
         if (p.ks > 1) sp.partials = reinterpret_cast<float *>(reinterpret_cast<char *>(ws) + kWsData);
         auto launch = [&](auto sch, auto bn) {
@@ -844,7 +987,7 @@ cudaError_t launch_gemm(const Geom &g, const void *packed, const uint16_t *cb,
             cfg.attrs = attr;
             cfg.numAttrs = na;
             e = cudaLaunchKernelEx(&cfg, gemm_ws_kernel<S, BN>, map, g, pk, c, scales, T, y, ws, sp, p.per_split,
-                                   p.cluster ? p.ks : 0);
+                                   p.cluster ? p.ks : 0, p.tail);
             if (e != cudaSuccess) return e;
             return cudaGetLastError();
         };

@@ -372,6 +372,28 @@ def test_gemm_cluster_split_ragged_tokens_every_element(K, B, out, inp, T, ks):
     assert_close(y, ref, bound, f"cluster split {ks} {K}x{B} {out}x{inp} T{T}")
 
 
+@pytest.mark.parametrize("K,B", [(1, 16), (2, 8)])
+@pytest.mark.parametrize("T", [2048, 2040])
+def test_gemm_wave_tail_split(K, B, T):
+    """A tile grid one wave and a bit: 38 row tiles x 4 token tiles = 152
+    tiles on 148 SMs.  The last 4 tiles (rows 4352..4863, tokens 1536..)
+    have their input features split 2 ways and are finished by the last of
+    their splits; the workspace size pins that plan.  Every row of the tail
+    tiles' row blocks and rows elsewhere are checked in full against the
+    oracle (T = 2040 leaves the tail's token tile ragged)."""
+    out, inp = 4864, 1024
+    desc = aq.LayerDesc.make(out, inp, K, B)
+    assert aq.aq_gemm_workspace_bytes(desc, T) == 4112 + 4 * 2 * 128 * 512 * 4
+    layer = _layer(out, inp, K, B, T + K)
+    dl = DevLayer(layer)
+    x = make_activations(inp, T, (T, K, 5))
+    y = run_gemm(dl, x)
+    rows = np.concatenate([np.arange(4352, 4864), np.arange(0, 4352, 97)])
+    ref, bound = oracle.matmul(layer.codes, layer.codebooks, layer.scales, x, rows=rows, threads=8)
+    assert_close(y[rows], ref, bound, f"wave tail {K}x{B} T{T}")
+    assert np.array_equal(run_gemm(dl, x)[rows], y[rows])  # deterministic
+
+
 @pytest.mark.parametrize("K", [2, 1])
 def test_gemv_tables_fall_back_to_exact_decode_beyond_binary16(K):
     """The batch-1 table path keeps its tables in binary16 and bounds their
