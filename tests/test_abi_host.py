@@ -286,3 +286,20 @@ def test_binding_fails_loudly_without_the_library(tmp_path):
                        cwd=str(tmp_path))
     assert r.returncode == 3, r.stdout + r.stderr
     assert "libaq_b200.so is missing" in r.stdout and "build.py" in r.stdout
+
+
+def test_prefill_plans_pinned_by_workspace_size():
+    """The prefill planner's choices for Llama-2-7B shapes, read back from
+    the workspace each needs (status word and counters, then fp32 sums):
+    a 4096-row layer at 512 tokens splits its input features 4 ways in one
+    cluster (32 tiles x 4 slices of 128 x 512); the 11008-row MLP layers at
+    2048 tokens split the 48 tiles of their third wave 3 ways; layers that
+    fill the SMs with whole tiles need no sums."""
+    prefix = 4112
+    slice_bytes = 128 * 512 * 4
+    for K, B in ((1, 16), (2, 8)):
+        assert aq.aq_gemm_workspace_bytes(aq.LayerDesc.make(4096, 4096, K, B), 512) == prefix + 32 * 4 * slice_bytes
+        assert aq.aq_gemm_workspace_bytes(aq.LayerDesc.make(4096, 11008, K, B), 512) == prefix + 32 * 4 * slice_bytes
+        assert aq.aq_gemm_workspace_bytes(aq.LayerDesc.make(11008, 4096, K, B), 2048) == prefix + 48 * 3 * slice_bytes
+        assert aq.aq_gemm_workspace_bytes(aq.LayerDesc.make(11008, 4096, K, B), 512) == 16
+        assert aq.aq_gemm_workspace_bytes(aq.LayerDesc.make(4096, 11008, K, B), 2048) == 16
