@@ -208,8 +208,8 @@ gemm_tc_kernel(Geom L, const uint8_t *__restrict__ packed, const uint4 *__restri
 //              Each thread fences its writes to the async proxy and arrives
 //              on full_a[stage] (128 arrivals).  The epilogue reads TMEM lanes
 //              32*(warp%4).. with tcgen05.ld, scales, rounds and stores (one
-//              split), or stores fp32 partial sums that the last CTA of the
-//              tile adds in split order (several splits).
+//              split); a split's CTAs finish together (gemm_cluster_finish,
+//              gemm_tail_finish).
 // Ring depth: 4 stages of (16 KiB A + 32 KiB B) for BN = 256, 3 when the
 // 32 KiB of 8x8 codebooks share the shared memory; 2 stages of (16 + 64 KiB)
 // for BN = 512.
@@ -237,76 +237,8 @@ constexpr int kWsThreadsOf = 64 + 128 * kWsGroupsOf<S>;  // X producer, MMA issu
 constexpr int kWsLag = 2;                     // cp.async stages in flight per decoder (< ring depth)
 
 struct GemmSplit {
-    float *partials;     // [splits][out][T] fp32, or null with one split
-    unsigned *counters;  // [grid.x * grid.y] arrivals per output tile
+    float *partials;  // a split cluster's scratch (gemm_cluster_finish's slices), or null with one split
 };
-
-// Called by every thread after the CTA stored its partial sums for output
-// tile (m0, n0) of split blockIdx.z.  The last CTA of the tile to arrive adds
-// the splits in split order (bit-reproducible), scales, rounds to binary16,
-// writes y and resets the tile's counter for the next call.
-__device__ __forceinline__ void gemm_split_finish(const Geom &L, GemmSplit sp, int m0, int n0, int bn, int T,
-                                                  const uint16_t *__restrict__ scales, uint16_t *__restrict__ y)
-{
-    __shared__ unsigned s_last;
-    __syncthreads();
-    const unsigned tile = blockIdx.y * gridDim.x + blockIdx.x;
-    if (threadIdx.x == 0) {
-        // the barrier orders the CTA's partial stores before this thread's
-        // release fence; the last CTA's acquire fence orders its reads
-        fence_acq_rel_gpu();
-        const unsigned prev = atomicAdd(&sp.counters[tile], 1u);
-        s_last = (prev == gridDim.z - 1) ? 1u : 0u;
-        if (s_last) fence_acq_rel_gpu();
-    }
-    __syncthreads();
-    if (!s_last) return;
-    const int cols4 = bn / 4;
-    const int ks = (int)gridDim.z;
-    const size_t zstride = (size_t)L.out * T / 4;  // float4 per split
-    // four float4 per thread per pass and four splits per batch of loads:
-    // sixteen independent L2 reads in flight; each element still adds its
-    // splits in split order
-    constexpr int kE = 4;
-    for (int e0 = threadIdx.x; e0 < kBM * cols4; e0 += kE * blockDim.x) {
-        const float4 *p[kE];
-        bool ok[kE];
-        float4 acc[kE];
-#pragma unroll
-        for (int i = 0; i < kE; ++i) {
-            const int e = e0 + i * blockDim.x;
-            const int row = m0 + e / cols4, gn = n0 + 4 * (e % cols4);
-            ok[i] = e < kBM * cols4 && row < L.out && gn < T;
-            p[i] = reinterpret_cast<const float4 *>(sp.partials + (size_t)(ok[i] ? row : 0) * T + (ok[i] ? gn : 0));
-            acc[i] = ok[i] ? __ldcg(p[i]) : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-        for (int z0 = 1; z0 < ks; z0 += 4) {
-            float4 t[4][kE];
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-#pragma unroll
-                for (int i = 0; i < kE; ++i)
-                    if (z0 + j < ks && ok[i]) t[j][i] = __ldcg(p[i] + (size_t)(z0 + j) * zstride);
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-#pragma unroll
-                for (int i = 0; i < kE; ++i)
-                    if (z0 + j < ks && ok[i]) {
-                        acc[i].x += t[j][i].x; acc[i].y += t[j][i].y; acc[i].z += t[j][i].z; acc[i].w += t[j][i].w;
-                    }
-        }
-#pragma unroll
-        for (int i = 0; i < kE; ++i) {
-            if (!ok[i]) continue;
-            const int e = e0 + i * blockDim.x;
-            const int row = m0 + e / cols4, gn = n0 + 4 * (e % cols4);
-            const float sc = scales ? __half2float(__ushort_as_half(scales[row])) : 1.f;
-            *reinterpret_cast<uint2 *>(y + (size_t)row * T + gn) =
-                make_uint2(f2h2(sc * acc[i].x, sc * acc[i].y), f2h2(sc * acc[i].z, sc * acc[i].w));
-        }
-    }
-    if (threadIdx.x == 0) sp.counters[tile] = 0u;
-}
 
 // Split-K finish of a split launched as one thread-block cluster of `ks`
 // CTAs along blockIdx.z (ks = 2, 4 or 8; the split index is the CTA's rank).
@@ -752,15 +684,7 @@ gemm_ws_kernel(const __grid_constant__ CUtensorMap xmap, Geom L, const uint8_t *
                 float v[16];
                 tmem_ld16(tbase + c0, v);
                 const int gn = n0 + c0;
-                if (sp.partials) {
-                    // one of several splits: fp32 partial sums, T % 8 == 0 here
-                    if (row < L.out && gn < T) {
-                        float4 *dst = reinterpret_cast<float4 *>(sp.partials + ((size_t)z * L.out + row) * T + gn);
-#pragma unroll
-                        for (int q4 = 0; q4 < 4; ++q4)
-                            if (gn + 4 * q4 < T) dst[q4] = make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
-                    }
-                } else if (row < L.out && gn < T) {
+                if (row < L.out && gn < T) {
                     uint16_t *dst = y + (size_t)row * T + gn;
                     if (gn + 16 <= T) {
                         const uint4 o0 = make_uint4(f2h2(sc * v[0], sc * v[1]), f2h2(sc * v[2], sc * v[3]),
@@ -806,9 +730,6 @@ gemm_ws_kernel(const __grid_constant__ CUtensorMap xmap, Geom L, const uint8_t *
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, BN);
-    // arrive even after a timeout so the counters stay consistent (the
-    // status word already tells the caller the output is incomplete)
-    if (sp.partials && cluster_ks == 0 && tail_idx < 0) gemm_split_finish(L, sp, m0, n0, BN, T, scales, y);
 }
 
 // ---- self-test of the bounded wait -----------------------------------------
@@ -866,26 +787,19 @@ static GemmPlan plan_gemm(const Geom &g, int T)
     // per SM works, keeping at least 8 stages per split
     int ks = tiles < kNumSMs ? (int)(kNumSMs / tiles) : 1;
     ks = std::max(1, std::min(ks, nst / 8));
-    // a split of 2, 4 or 8 runs as one thread-block cluster along z whose
-    // CTAs share the finish (no arrival counters)
-    bool cluster = false;
+    // the split runs as one thread-block cluster along z whose CTAs share
+    // the finish: 2, 4 or 8 CTAs (the largest power of two not above ks).
+    // With at least 8 stages per split (nst >= 8 kc) none of them is empty:
+    // per = ceil(nst / kc) gives exactly kc non-empty splits
     if (ks >= 2) {
         int kc = 2;
         while (kc * 2 <= std::min(ks, 8)) kc *= 2;
-        const int per = (nst + kc - 1) / kc;
-        if ((nst + per - 1) / per == kc) {  // no empty split
-            ks = kc;
-            cluster = true;
-        }
+        ks = kc;
     }
     p.per_split = (nst + ks - 1) / ks;
     p.ks = (nst + p.per_split - 1) / p.per_split;
-    p.cluster = cluster;
-    // without a cluster, split only while the tiles' arrival counters fit
-    // the fixed area
-    if (!cluster && tiles > kWsMaxCounters) p.ks = 1, p.per_split = nst;
-    if (p.ks > 1)
-        p.ws_bytes = kWsData + (cluster ? (size_t)p.ks * tiles * kBM * p.bn : (size_t)p.ks * g.out * T) * sizeof(float);
+    p.cluster = p.ks > 1;
+    if (p.ks > 1) p.ws_bytes = kWsData + (size_t)p.ks * tiles * kBM * p.bn * sizeof(float);
     // more tiles than one wave, the last wave at most half full: its tiles'
     // input features are split so that it fills the SMs (Llama-2-7B MLP
     // rows at 2048 tokens: 344 tiles, 48 in the third wave, split 3 ways)
@@ -955,7 +869,7 @@ cudaError_t launch_gemm(const Geom &g, const void *packed, const uint16_t *cb,
         const long tiles = (long)p.mtiles * p.ntiles;
         const dim3 grid = p.tail.ks > 0 ? dim3((unsigned)(p.tail.full + (tiles - p.tail.full) * p.tail.ks), 1, 1)
                                         : dim3(p.mtiles, p.ntiles, p.ks);
-        GemmSplit sp{nullptr, reinterpret_cast<unsigned *>(reinterpret_cast<char *>(ws) + kWsHeader)};
+        GemmSplit sp{nullptr};
         if (p.ks > 1) sp.partials = reinterpret_cast<float *>(reinterpret_cast<char *>(ws) + kWsData);
         auto launch = [&](auto sch, auto bn) {
             using S = decltype(sch);
